@@ -1,0 +1,488 @@
+/*
+ * bsa_oracle.c -- plain, slow CPU oracle for query-aware top-k block-sparse
+ * causal attention.
+ *
+ * TEST INFRASTRUCTURE.  Only the tests, the smoke check and the CPU-baseline
+ * leg of the benchmark may load or call this file's library.  The product
+ * path (the CUDA library and its Python binding) never does, and shares no
+ * code, header, table or helper with it.
+ *
+ * What it computes, step by step, in the order the source pages give:
+ *
+ *   1. pool   -- one mean vector per block of consecutive tokens ("粗粒度
+ *                Block 打分", 稀疏注意力 tutorial §4.6; block = consecutive
+ *                tokens, §4.5; "按块聚合 key" in the gated-sparse essay's
+ *                pseudo-code step 1; "块级池化的Token表示" in the Sparse
+ *                Frontier review §2.1).
+ *   2. score  -- selector score s = pooled-q . pooled-k / sqrt(d): the
+ *                "continuous score per context unit" of the SAS page
+ *                (核心模块 1).  For gists (SSA page, 推理时的关键模块 1) the
+ *                query is scored against every chunk's gist key.
+ *   3. select -- hard top-k of the history units per query unit, with the
+ *                current block always kept (SAS page, 核心洞察 / 核心模块 3,
+ *                推理 paragraph: "each query selects the k highest units";
+ *                essay pseudo-code step 2).  Ties go to the lowest index.
+ *   4. attend -- softmax(QK^T/sqrt(d) + M)V with the additive mask
+ *                M in {0, -inf} (稀疏注意力 tutorial §1 formula and §2 mask
+ *                formula): M = 0 exactly on keys of the selected blocks that
+ *                are not in the future of the query.
+ *   5. gate   -- (SAS page, 核心模块 2-3) the selector's continuous score
+ *                enters the logits in log space, normalised by a softmax over
+ *                the kept blocks (current block included):
+ *                logit += log g_j,  g_j = exp(s_j) / sum_{l kept} exp(s_l).
+ *   6. gist   -- (SSA page, 推理时的关键模块 1-3) expand the top-k chunks to
+ *                their tokens; every other chunk is represented by its gist
+ *                key/value; attend over the mixture.
+ *
+ * Precision: steps 1-2 run in fp32 in a fixed order (pooling over heads then
+ * tokens ascending; dot product over the channel index ascending; every
+ * product and sum rounded to fp32; no fused multiply-add -- this file is
+ * compiled with -ffp-contract=off).  Steps 4-6 run in fp64.  Inputs arrive as
+ * fp32 arrays (a bf16 input is upcast exactly before the call).
+ *
+ * Readings where the pages are silent (each is also listed in the design
+ * notes):
+ *   - under GQA the selection unit is the KV-head group: one score row per
+ *     group, from the query mean over the group's heads and the block's
+ *     tokens; the gate uses the same group score;
+ *   - the current block's score uses full-block means (block-coarse);
+ *   - fewer candidates than the budget: keep them all;
+ *   - decode: every cached token is history; the "last block" is block nb-1;
+ *   - gist decode keeps no forced chunk and drops the gists of expanded chunks;
+ *   - NaN scores rank below every number, -inf included.
+ *
+ * Parallelism: OpenMP over independent output units only (rows, blocks,
+ * selection rows); every unit's arithmetic is sequential, so results do not
+ * depend on the thread count.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ------------------------------------------------------------------------ */
+/* 1. Pooling (fixed-order fp32)                                            */
+/* ------------------------------------------------------------------------ */
+
+/* kbar[b,h,j,c] = (sum_{t in block j, ascending} k[b,h,t,c]) / bs */
+void oracle_pool_keys(const float* k, int64_t B, int64_t H, int64_t N, int64_t d,
+                      int64_t bs, float* kbar)
+{
+    const int64_t nb = N / bs;
+    const int64_t units = B * H * nb;
+#pragma omp parallel for schedule(static)
+    for (int64_t u = 0; u < units; ++u) {
+        const int64_t bh = u / nb, j = u % nb;
+        for (int64_t c = 0; c < d; ++c) {
+            float acc = 0.0f;
+            for (int64_t t = 0; t < bs; ++t)
+                acc = acc + k[(bh * N + j * bs + t) * d + c];
+            kbar[u * d + c] = acc / (float)bs;
+        }
+    }
+}
+
+/* qbar[b,g,i,c] = (sum_{h in group g asc} sum_{t in block i asc} q[b,h,t,c]) / (G*bs)
+ * Group g holds query heads g*G .. g*G+G-1 (G = Hq/Hkv). */
+void oracle_pool_queries_grouped(const float* q, int64_t B, int64_t Hq, int64_t Hkv,
+                                 int64_t N, int64_t d, int64_t bs, float* qbar)
+{
+    const int64_t nb = N / bs, G = Hq / Hkv;
+    const int64_t units = B * Hkv * nb;
+#pragma omp parallel for schedule(static)
+    for (int64_t u = 0; u < units; ++u) {
+        const int64_t b = u / (Hkv * nb), g = (u / nb) % Hkv, i = u % nb;
+        for (int64_t c = 0; c < d; ++c) {
+            float acc = 0.0f;
+            for (int64_t hh = 0; hh < G; ++hh) {
+                const int64_t h = g * G + hh;
+                for (int64_t t = 0; t < bs; ++t)
+                    acc = acc + q[((b * Hq + h) * N + i * bs + t) * d + c];
+            }
+            qbar[u * d + c] = acc / (float)(G * bs);
+        }
+    }
+}
+
+/* Decode: one query token per sequence, q [B,Hq,d].
+ * qbar[b,g,c] = (sum_{h in group g asc} q[b,h,c]) / G */
+void oracle_group_mean_query(const float* q, int64_t B, int64_t Hq, int64_t Hkv,
+                             int64_t d, float* qbar)
+{
+    const int64_t G = Hq / Hkv;
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t g = 0; g < Hkv; ++g)
+            for (int64_t c = 0; c < d; ++c) {
+                float acc = 0.0f;
+                for (int64_t hh = 0; hh < G; ++hh)
+                    acc = acc + q[(b * Hq + g * G + hh) * d + c];
+                qbar[(b * Hkv + g) * d + c] = acc / (float)G;
+            }
+}
+
+/* ------------------------------------------------------------------------ */
+/* 2. Selector scores (fixed-order fp32)                                    */
+/* ------------------------------------------------------------------------ */
+
+/* The scale 1/sqrt(d), rounded once to fp32. */
+static float score_scale(int64_t d) { return (float)(1.0 / sqrt((double)d)); }
+
+/* acc = sum_c a[c]*b[c], channel index ascending, each product and each sum
+ * rounded to fp32; then one fp32 multiply by the rounded scale. */
+static float score_dot(const float* a, const float* b, int64_t d, float scale)
+{
+    float acc = 0.0f;
+    for (int64_t c = 0; c < d; ++c) {
+        const float prod = a[c] * b[c];
+        acc = acc + prod;
+    }
+    return acc * scale;
+}
+
+/* Prefill: s[b,g,i,j] = qbar[b,g,i] . kbar[b,g,j] / sqrt(d) for j <= i,
+ * -inf for j > i (future blocks are never candidates). */
+void oracle_scores_prefill(const float* qbar, const float* kbar, int64_t B, int64_t Hkv,
+                           int64_t nb, int64_t d, float* s)
+{
+    const float scale = score_scale(d);
+    const int64_t rows = B * Hkv * nb;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        const int64_t bg = r / nb, i = r % nb;
+        for (int64_t j = 0; j < nb; ++j)
+            s[r * nb + j] = (j <= i) ? score_dot(qbar + r * d, kbar + (bg * nb + j) * d, d, scale)
+                                     : -INFINITY;
+    }
+}
+
+/* Decode: s[b,g,j] = qbar[b,g] . kbar[b,g,j] / sqrt(d) for every block j. */
+void oracle_scores_decode(const float* qbar, const float* kbar, int64_t B, int64_t Hkv,
+                          int64_t nb, int64_t d, float* s)
+{
+    const float scale = score_scale(d);
+    const int64_t rows = B * Hkv;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < nb; ++j)
+            s[r * nb + j] = score_dot(qbar + r * d, kbar + (r * nb + j) * d, d, scale);
+}
+
+/* Gist: s[b,h,c] = q[b,h] . gk[b,g(h),c] / sqrt(d), one row per query head
+ * (SSA page: under GQA each query head chooses its own chunks). */
+void oracle_scores_gist(const float* q, const float* gk, int64_t B, int64_t Hq, int64_t Hkv,
+                        int64_t nc, int64_t d, float* s)
+{
+    const float scale = score_scale(d);
+    const int64_t G = Hq / Hkv;
+    const int64_t rows = B * Hq;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        const int64_t b = r / Hq, h = r % Hq, g = h / G;
+        for (int64_t c = 0; c < nc; ++c)
+            s[r * nc + c] = score_dot(q + r * d, gk + ((b * Hkv + g) * nc + c) * d, d, scale);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* 3. Top-k selection                                                       */
+/* ------------------------------------------------------------------------ */
+
+typedef struct { float s; int32_t j; } cand_t;
+
+/* Order: larger score first; equal scores -> lower index first; a NaN ranks
+ * below every number (including -inf). */
+static int cand_cmp(const void* pa, const void* pb)
+{
+    const cand_t* a = (const cand_t*)pa;
+    const cand_t* b = (const cand_t*)pb;
+    const int an = isnan(a->s), bn = isnan(b->s);
+    if (an != bn) return an ? 1 : -1;
+    if (!an) {
+        if (a->s > b->s) return -1;
+        if (a->s < b->s) return 1;
+    }
+    return (a->j < b->j) ? -1 : (a->j > b->j) ? 1 : 0;
+}
+
+static int int_cmp(const void* pa, const void* pb)
+{
+    const int32_t a = *(const int32_t*)pa, b = *(const int32_t*)pb;
+    return (a < b) ? -1 : (a > b);
+}
+
+/* mode 0 (causal block, prefill): row r is query block i = r % ncols;
+ *        candidates are blocks j < i; block i is always kept.
+ * mode 1 (last block, decode): candidates are j < ncols-1; block ncols-1 is
+ *        always kept.
+ * mode 2 (plain, gist): candidates are all j < ncols; nothing is forced.
+ * Output per row: the kept indices ascending, then -1 up to idx_stride.
+ * count (optional) receives the number of kept indices per row. */
+void oracle_topk(const float* s, int64_t rows, int64_t ncols, int mode, int64_t kb,
+                 int32_t* idx, int64_t idx_stride, int32_t* count)
+{
+#pragma omp parallel for schedule(dynamic, 16)
+    for (int64_t r = 0; r < rows; ++r) {
+        int64_t ncand, forced;
+        if (mode == 0) { ncand = r % ncols; forced = r % ncols; }
+        else if (mode == 1) { ncand = ncols - 1; forced = ncols - 1; }
+        else { ncand = ncols; forced = -1; }
+        cand_t* c = (cand_t*)malloc(sizeof(cand_t) * (size_t)(ncand > 0 ? ncand : 1));
+        for (int64_t j = 0; j < ncand; ++j) { c[j].s = s[r * ncols + j]; c[j].j = (int32_t)j; }
+        qsort(c, (size_t)ncand, sizeof(cand_t), cand_cmp);
+        const int64_t take = (kb < ncand) ? kb : ncand;
+        int32_t* out = idx + r * idx_stride;
+        int64_t n = 0;
+        for (int64_t t = 0; t < take; ++t) out[n++] = c[t].j;
+        if (forced >= 0) out[n++] = (int32_t)forced;
+        qsort(out, (size_t)n, sizeof(int32_t), int_cmp);
+        for (int64_t t = n; t < idx_stride; ++t) out[t] = -1;
+        if (count) count[r] = (int32_t)n;
+        free(c);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* 4. The mask M of one query row                                           */
+/* ------------------------------------------------------------------------ */
+
+/* Mark the blocks listed in one index row (entries < 0 end the list). */
+static void mark_blocks(const int32_t* list, int64_t stride, int64_t nb, unsigned char* sel)
+{
+    memset(sel, 0, (size_t)nb);
+    for (int64_t t = 0; t < stride; ++t) {
+        const int32_t j = list[t];
+        if (j < 0) break;
+        if (j < nb) sel[j] = 1;
+    }
+}
+
+/* M_u = 0 iff key u lies in a selected block and is not in the query's
+ * future (u <= t); -inf otherwise. Returned as an "allowed" flag. */
+static int key_allowed(const unsigned char* sel, int64_t bs, int64_t t, int64_t u)
+{
+    return sel[u / bs] && (u <= t);
+}
+
+/* The full mask of one (batch, group) in prefill: mask[t*N + u] = 1 where
+ * M_{t,u} = 0.  idx holds one row per query block: [nb, idx_stride]. */
+void oracle_prefill_mask(int64_t N, int64_t bs, const int32_t* idx, int64_t idx_stride,
+                         unsigned char* mask)
+{
+    const int64_t nb = N / bs;
+    unsigned char* sel = (unsigned char*)malloc((size_t)nb);
+    for (int64_t t = 0; t < N; ++t) {
+        mark_blocks(idx + (t / bs) * idx_stride, idx_stride, nb, sel);
+        for (int64_t u = 0; u < N; ++u) mask[t * N + u] = (unsigned char)key_allowed(sel, bs, t, u);
+    }
+    free(sel);
+}
+
+/* ------------------------------------------------------------------------ */
+/* 5. Gate                                                                   */
+/* ------------------------------------------------------------------------ */
+
+/* logg[j] = log g_j for every kept block j of one row, g = softmax over the
+ * kept blocks' scores (fp64; the largest score is subtracted before exp,
+ * which leaves g unchanged). Blocks not kept get -inf. */
+static void gate_log_weights(const float* srow, const int32_t* list, int64_t stride,
+                             int64_t nb, double* logg)
+{
+    double smax = -INFINITY;
+    for (int64_t j = 0; j < nb; ++j) logg[j] = -INFINITY;
+    for (int64_t t = 0; t < stride && list[t] >= 0; ++t) {
+        const double sj = (double)srow[list[t]];
+        if (sj > smax) smax = sj;
+    }
+    double z = 0.0;
+    for (int64_t t = 0; t < stride && list[t] >= 0; ++t)
+        z += exp((double)srow[list[t]] - smax);
+    for (int64_t t = 0; t < stride && list[t] >= 0; ++t) {
+        const double g = exp((double)srow[list[t]] - smax) / z;
+        logg[list[t]] = log(g);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* 6. Attention rows (fp64)                                                 */
+/* ------------------------------------------------------------------------ */
+
+static double dot64(const float* a, const float* b, int64_t d)
+{
+    double acc = 0.0;
+    for (int64_t c = 0; c < d; ++c) acc += (double)a[c] * (double)b[c];
+    return acc;
+}
+
+/* softmax over the allowed keys; writes out[d] and the natural-log LSE.
+ * logits[n] are the finite logits of the n allowed keys, vals[n] their
+ * value rows. With no allowed key the row is 0 and LSE is -inf. */
+static void softmax_rows(const double* logits, const float* const* vals, int64_t n, int64_t d,
+                         double* out, double* lse)
+{
+    for (int64_t c = 0; c < d; ++c) out[c] = 0.0;
+    if (n == 0) { *lse = -INFINITY; return; }
+    double m = -INFINITY;
+    for (int64_t u = 0; u < n; ++u) if (logits[u] > m) m = logits[u];
+    double z = 0.0;
+    for (int64_t u = 0; u < n; ++u) {
+        const double p = exp(logits[u] - m);
+        z += p;
+        const float* vr = vals[u];
+        for (int64_t c = 0; c < d; ++c) out[c] += p * (double)vr[c];
+    }
+    for (int64_t c = 0; c < d; ++c) out[c] /= z;
+    *lse = m + log(z);
+}
+
+/* Prefill rows.  q [B,Hq,N,d], k/v [B,Hkv,N,d], idx [B,Hkv,nb,idx_stride],
+ * gate_scores (NULL = ungated) [B,Hkv,nb,nb] = the selector scores s_{i,j}.
+ * rows[n] = (b*Hq + h)*N + t selects the query rows to compute.
+ * out [nrows,d], lse [nrows] (natural log). */
+void oracle_attend_prefill_rows(const float* q, const float* k, const float* v,
+                                int64_t B, int64_t Hq, int64_t Hkv, int64_t N, int64_t d,
+                                int64_t bs, const int32_t* idx, int64_t idx_stride,
+                                const float* gate_scores, double scale,
+                                const int64_t* rows, int64_t nrows, double* out, double* lse)
+{
+    const int64_t nb = N / bs, G = Hq / Hkv;
+    (void)B;
+#pragma omp parallel
+    {
+        unsigned char* sel = (unsigned char*)malloc((size_t)nb);
+        double* logg = (double*)malloc(sizeof(double) * (size_t)nb);
+        double* logits = (double*)malloc(sizeof(double) * (size_t)N);
+        const float** vals = (const float**)malloc(sizeof(float*) * (size_t)N);
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t n = 0; n < nrows; ++n) {
+            const int64_t r = rows[n];
+            const int64_t b = r / (Hq * N), h = (r / N) % Hq, t = r % N;
+            const int64_t g = h / G, i = t / bs;
+            const int32_t* list = idx + ((b * Hkv + g) * nb + i) * idx_stride;
+            mark_blocks(list, idx_stride, nb, sel);
+            if (gate_scores)
+                gate_log_weights(gate_scores + ((b * Hkv + g) * nb + i) * nb, list, idx_stride, nb, logg);
+            const float* qr = q + r * d;
+            const float* kb = k + (b * Hkv + g) * N * d;
+            const float* vb = v + (b * Hkv + g) * N * d;
+            int64_t m = 0;
+            for (int64_t u = 0; u < N; ++u) {
+                if (!key_allowed(sel, bs, t, u)) continue;   /* M_u = -inf: weight exactly 0 */
+                double l = dot64(qr, kb + u * d, d) * scale;
+                if (gate_scores) {
+                    const double bias = logg[u / bs];
+                    if (bias == -INFINITY) continue;          /* g_j = 0 */
+                    l += bias;
+                }
+                logits[m] = l;
+                vals[m] = vb + u * d;
+                ++m;
+            }
+            softmax_rows(logits, vals, m, d, out + n * d, lse + n);
+        }
+        free(sel); free(logg); free(logits); free(vals);
+    }
+}
+
+/* Decode rows.  q [B,Hq,d] (one token per sequence), k/v [B,Hkv,Nk,d],
+ * idx [B,Hkv,idx_stride].  Every cached token is history of the query.
+ * rows[n] = b*Hq + h. */
+void oracle_attend_decode_rows(const float* q, const float* k, const float* v,
+                               int64_t B, int64_t Hq, int64_t Hkv, int64_t Nk, int64_t d,
+                               int64_t bs, const int32_t* idx, int64_t idx_stride, double scale,
+                               const int64_t* rows, int64_t nrows, double* out, double* lse)
+{
+    const int64_t nb = Nk / bs, G = Hq / Hkv;
+    (void)B;
+#pragma omp parallel
+    {
+        unsigned char* sel = (unsigned char*)malloc((size_t)nb);
+        double* logits = (double*)malloc(sizeof(double) * (size_t)Nk);
+        const float** vals = (const float**)malloc(sizeof(float*) * (size_t)Nk);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t n = 0; n < nrows; ++n) {
+            const int64_t r = rows[n];
+            const int64_t b = r / Hq, h = r % Hq, g = h / G;
+            mark_blocks(idx + (b * Hkv + g) * idx_stride, idx_stride, nb, sel);
+            const float* kb = k + (b * Hkv + g) * Nk * d;
+            const float* vb = v + (b * Hkv + g) * Nk * d;
+            int64_t m = 0;
+            for (int64_t u = 0; u < Nk; ++u) {
+                if (!sel[u / bs]) continue;
+                logits[m] = dot64(q + r * d, kb + u * d, d) * scale;
+                vals[m] = vb + u * d;
+                ++m;
+            }
+            softmax_rows(logits, vals, m, d, out + n * d, lse + n);
+        }
+        free(sel); free(logits); free(vals);
+    }
+}
+
+/* Gist rows.  q [B,Hq,d], token k/v [B,Hkv,Nk,d], gist gk/gv [B,Hkv,nc,d]
+ * with nc = Nk/chunk, idx [B,Hq,idx_stride] = the expanded chunks of each
+ * query head.  Keys: every token of an expanded chunk, and the gist of every
+ * chunk that is not expanded.  rows[n] = b*Hq + h. */
+void oracle_attend_gist_rows(const float* q, const float* k, const float* v,
+                             const float* gk, const float* gv,
+                             int64_t B, int64_t Hq, int64_t Hkv, int64_t Nk, int64_t d,
+                             int64_t chunk, const int32_t* idx, int64_t idx_stride, double scale,
+                             const int64_t* rows, int64_t nrows, double* out, double* lse)
+{
+    const int64_t nc = Nk / chunk, G = Hq / Hkv;
+    (void)B;
+#pragma omp parallel
+    {
+        unsigned char* sel = (unsigned char*)malloc((size_t)nc);
+        double* logits = (double*)malloc(sizeof(double) * (size_t)(Nk + nc));
+        const float** vals = (const float**)malloc(sizeof(float*) * (size_t)(Nk + nc));
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t n = 0; n < nrows; ++n) {
+            const int64_t r = rows[n];
+            const int64_t b = r / Hq, h = r % Hq, g = h / G;
+            mark_blocks(idx + r * idx_stride, idx_stride, nc, sel);
+            const float* kb = k + (b * Hkv + g) * Nk * d;
+            const float* vb = v + (b * Hkv + g) * Nk * d;
+            const float* gkb = gk + (b * Hkv + g) * nc * d;
+            const float* gvb = gv + (b * Hkv + g) * nc * d;
+            int64_t m = 0;
+            for (int64_t c = 0; c < nc; ++c) {
+                if (sel[c]) {
+                    for (int64_t u = c * chunk; u < (c + 1) * chunk; ++u) {
+                        logits[m] = dot64(q + r * d, kb + u * d, d) * scale;
+                        vals[m] = vb + u * d;
+                        ++m;
+                    }
+                } else {
+                    logits[m] = dot64(q + r * d, gkb + c * d, d) * scale;
+                    vals[m] = gvb + c * d;
+                    ++m;
+                }
+            }
+            softmax_rows(logits, vals, m, d, out + n * d, lse + n);
+        }
+        free(sel); free(logits); free(vals);
+    }
+}
+
+/* Threads the OpenMP runtime will use (for reporting the CPU baseline). */
+int oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void oracle_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}

@@ -1,0 +1,478 @@
+"""Pins for the CPU oracle: every check compares the oracle with something
+other than itself -- the pages' worked examples (tests/golden/), closed forms,
+invariants, a library routine the special case reduces to, or brute force.
+
+Runs on CPU only (no GPU marker).
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _read_golden_sets(name):
+    rows = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, vals = line.split(":")
+            rows[int(key)] = [int(x) for x in vals.split()]
+    return rows
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _sdpa64(q, k, v, mask=None, causal=False):
+    """Library attention in fp64 on CPU (the dense formula's own routine)."""
+    q = torch.as_tensor(q, dtype=torch.float64)
+    k = torch.as_tensor(k, dtype=torch.float64)
+    v = torch.as_tensor(v, dtype=torch.float64)
+    if mask is not None:
+        mask = torch.as_tensor(mask)
+    return F.scaled_dot_product_attention(q, k, v, attn_mask=mask, is_causal=causal).numpy()
+
+
+# ----------------------------------------------------------------------------
+# pooling: closed forms and the fixed summation order
+# ----------------------------------------------------------------------------
+
+def test_pool_keys_constant_input_is_exact():
+    k = np.full((2, 3, 128, 16), 0.375, np.float32)
+    kbar = oracle.pool_keys(k, 64)
+    assert kbar.shape == (2, 3, 2, 16)
+    assert np.all(kbar == np.float32(0.375))
+
+
+def test_pool_keys_integer_input_exact_mean():
+    r = _rng(1)
+    k = r.integers(-8, 9, size=(2, 2, 256, 8)).astype(np.float32)
+    kbar = oracle.pool_keys(k, 64)
+    exact = k.reshape(2, 2, 4, 64, 8).astype(np.int64).sum(axis=3) / 64.0
+    assert np.array_equal(kbar.astype(np.float64), exact)
+
+
+def test_pool_keys_sequential_fp32_order():
+    # np.add.accumulate is a strictly left-to-right fp32 running sum: the
+    # oracle's fixed order must reproduce its last element bit for bit.
+    r = _rng(2)
+    k = r.standard_normal((1, 2, 192, 8)).astype(np.float32)
+    kbar = oracle.pool_keys(k, 64)
+    blocks = k.reshape(1, 2, 3, 64, 8)
+    seq = np.add.accumulate(blocks, axis=3, dtype=np.float32)[:, :, :, -1, :]
+    assert np.array_equal(kbar, seq / np.float32(64))
+
+
+def test_pool_queries_grouped_heads_then_tokens():
+    r = _rng(3)
+    B, Hq, Hkv, N, d, bs = 1, 6, 2, 128, 8, 32
+    q = r.standard_normal((B, Hq, N, d)).astype(np.float32)
+    qbar = oracle.pool_queries_grouped(q, Hkv, bs)
+    G = Hq // Hkv
+    # group g, block i: the G*bs rows in (head asc, token asc) order
+    seqs = q.reshape(B, Hkv, G, N // bs, bs, d).transpose(0, 1, 3, 2, 4, 5)
+    seqs = seqs.reshape(B, Hkv, N // bs, G * bs, d)
+    ref = np.add.accumulate(seqs, axis=3, dtype=np.float32)[:, :, :, -1, :] / np.float32(G * bs)
+    assert np.array_equal(qbar, ref)
+
+
+def test_group_mean_query():
+    r = _rng(4)
+    q = r.integers(-4, 5, size=(3, 8, 16)).astype(np.float32)
+    qbar = oracle.group_mean_query(q, 2)
+    exact = q.reshape(3, 2, 4, 16).astype(np.int64).sum(axis=2) / 4.0
+    assert np.array_equal(qbar.astype(np.float64), exact)
+
+
+# ----------------------------------------------------------------------------
+# selector scores
+# ----------------------------------------------------------------------------
+
+def test_scores_prefill_integer_exact_and_causal():
+    r = _rng(5)
+    B, Hkv, nb, d = 1, 2, 6, 16
+    qbar = r.integers(-3, 4, size=(B, Hkv, nb, d)).astype(np.float32)
+    kbar = r.integers(-3, 4, size=(B, Hkv, nb, d)).astype(np.float32)
+    s = oracle.scores_prefill(qbar, kbar)
+    scale = np.float32(1.0 / math.sqrt(d))
+    dots = np.einsum("bgic,bgjc->bgij", qbar.astype(np.int64), kbar.astype(np.int64))
+    for i in range(nb):
+        for j in range(nb):
+            if j <= i:
+                assert np.array_equal(s[:, :, i, j], (dots[:, :, i, j].astype(np.float32) * scale))
+            else:
+                assert np.all(np.isneginf(s[:, :, i, j]))
+
+
+def test_scores_sequential_fp32_products():
+    r = _rng(6)
+    B, Hkv, nb, d = 1, 1, 5, 32
+    qbar = r.standard_normal((B, Hkv, nb, d)).astype(np.float32)
+    kbar = r.standard_normal((B, Hkv, nb, d)).astype(np.float32)
+    s = oracle.scores_prefill(qbar, kbar)
+    scale = np.float32(1.0 / math.sqrt(d))
+    for i in range(nb):
+        for j in range(i + 1):
+            prods = (qbar[0, 0, i] * kbar[0, 0, j]).astype(np.float32)
+            acc = np.add.accumulate(prods, dtype=np.float32)[-1]
+            assert s[0, 0, i, j] == np.float32(acc * scale)
+
+
+def test_group_score_is_mean_of_head_scores():
+    # Linearity: pooled-over-heads query . pooled key = mean of the per-head
+    # pooled scores, up to fp32 rounding.
+    r = _rng(7)
+    B, Hq, Hkv, N, d, bs = 1, 4, 1, 256, 64, 64
+    q = r.standard_normal((B, Hq, N, d)).astype(np.float32)
+    k = r.standard_normal((B, Hkv, N, d)).astype(np.float32)
+    s_group = oracle.scores_prefill(oracle.pool_queries_grouped(q, Hkv, bs), oracle.pool_keys(k, bs))
+    per_head = []
+    for h in range(Hq):
+        qh = q[:, h:h + 1]
+        per_head.append(oracle.scores_prefill(oracle.pool_queries_grouped(qh, 1, bs),
+                                              oracle.pool_keys(k, bs)))
+    mean = np.mean(np.stack(per_head), axis=0)
+    tri = np.tril(np.ones((N // bs, N // bs), bool))
+    assert np.allclose(s_group[0, 0][tri], mean[0, 0][tri], atol=1e-5)
+
+
+def test_scores_decode_and_gist_shapes_and_values():
+    r = _rng(8)
+    B, Hq, Hkv, nb, d = 2, 4, 2, 7, 16
+    q = r.integers(-2, 3, size=(B, Hq, d)).astype(np.float32)
+    kbar = r.integers(-2, 3, size=(B, Hkv, nb, d)).astype(np.float32)
+    scale = np.float32(1.0 / math.sqrt(d))
+    qbar = oracle.group_mean_query(q, Hkv)
+    s = oracle.scores_decode(qbar, kbar)
+    ref = np.einsum("bgc,bgjc->bgj", qbar.astype(np.float64), kbar.astype(np.float64))
+    assert np.array_equal(s, ref.astype(np.float32) * scale)
+    sg = oracle.scores_gist(q, kbar)
+    G = Hq // Hkv
+    refg = np.einsum("bhc,bhjc->bhj", q.astype(np.int64), np.repeat(kbar, G, axis=1).astype(np.int64))
+    assert np.array_equal(sg, refg.astype(np.float32) * scale)
+
+
+# ----------------------------------------------------------------------------
+# top-k selection: brute force over every subset
+# ----------------------------------------------------------------------------
+
+def _brute_topk(scores, cand, kb):
+    """Max-sum subset of size min(kb,|cand|); ties -> lexicographically smallest."""
+    take = min(kb, len(cand))
+    best, best_sum = None, None
+    for comb in itertools.combinations(sorted(cand), take):
+        ssum = sum(scores[j] for j in comb)
+        if best is None or ssum > best_sum or (ssum == best_sum and comb < best):
+            best, best_sum = comb, ssum
+    return list(best)
+
+
+@pytest.mark.parametrize("mode", [oracle.TOPK_CAUSAL_BLOCK, oracle.TOPK_LAST_BLOCK, oracle.TOPK_PLAIN])
+def test_topk_matches_bruteforce(mode):
+    r = _rng(10 + mode)
+    for trial in range(40):
+        nb = int(r.integers(1, 10))
+        kb = int(r.integers(0, nb + 2))
+        s = r.integers(-3, 4, size=(nb, nb)).astype(np.float32)   # many ties
+        idx, cnt = oracle.topk(s, mode, kb)
+        for row in range(nb):
+            if mode == oracle.TOPK_CAUSAL_BLOCK:
+                cand, forced = list(range(row)), [row]
+            elif mode == oracle.TOPK_LAST_BLOCK:
+                cand, forced = list(range(nb - 1)), [nb - 1]
+            else:
+                cand, forced = list(range(nb)), []
+            want = sorted(_brute_topk(s[row].tolist(), cand, kb) + forced)
+            got = [int(x) for x in idx[row] if x >= 0]
+            assert got == want, (trial, row, s[row], kb)
+            assert cnt[row] == len(want)
+            assert np.all(idx[row][len(want):] == -1)
+
+
+def test_topk_ties_go_to_lowest_index():
+    s = np.array([[1.0, 2.0, 2.0, 2.0, 0.5, 2.0]], np.float32)
+    idx, _ = oracle.topk(s, oracle.TOPK_PLAIN, 2)
+    assert idx.tolist() == [[1, 2]]
+
+
+def test_topk_nan_ranks_last():
+    s = np.array([[np.nan, -np.inf, 0.0, np.nan, -1.0]], np.float32)
+    idx, _ = oracle.topk(s, oracle.TOPK_PLAIN, 3)
+    assert idx.tolist() == [[1, 2, 4]]
+    idx, _ = oracle.topk(s, oracle.TOPK_PLAIN, 4)
+    assert idx.tolist() == [[0, 1, 2, 4]]
+
+
+# ----------------------------------------------------------------------------
+# the mask: the pages' two worked examples
+# ----------------------------------------------------------------------------
+
+def test_sliding_window_w3_pattern_from_tutorial():
+    """bs = 1 (one token per block), budget 2 history blocks, recency scores
+    s_{i,j} = j: selection + forced current block must give the page's w=3
+    causal window, and the mask must equal its printed 6x6 pattern."""
+    golden = _read_golden_sets("sliding_window_w3.txt")
+    N = 6
+    s = np.full((N, N), -np.inf, np.float32)
+    for i in range(N):
+        for j in range(i + 1):
+            s[i, j] = float(j)
+    idx, _ = oracle.topk(s, oracle.TOPK_CAUSAL_BLOCK, 2)
+    mask = oracle.prefill_mask(N, 1, idx)
+    for t in range(N):
+        seen = [u + 1 for u in range(N) if mask[t, u]]
+        assert seen == golden[t + 1], (t, seen)
+
+
+def test_block_sparse_4block_pattern_from_tutorial():
+    golden = _read_golden_sets("block_sparse_4blocks.txt")
+    idx = np.full((4, 3), -1, np.int32)
+    for qb, ks in golden.items():
+        idx[qb - 1, :len(ks)] = [x - 1 for x in ks]
+    mask = oracle.prefill_mask(4, 1, idx)
+    for t in range(4):
+        assert [u + 1 for u in range(4) if mask[t, u]] == golden[t + 1]
+    # At bs > 1 the same block pattern holds, with causality inside the
+    # diagonal block only.
+    bs = 3
+    mask3 = oracle.prefill_mask(4 * bs, bs, idx)
+    for t in range(4 * bs):
+        for u in range(4 * bs):
+            want = ((u // bs) + 1 in golden[t // bs + 1]) and u <= t
+            assert mask3[t, u] == want
+
+
+# ----------------------------------------------------------------------------
+# attention: special cases that reduce to the dense library routine
+# ----------------------------------------------------------------------------
+
+def _small_prefill(seed, B=1, Hq=4, Hkv=2, N=192, d=16):
+    r = _rng(seed)
+    q = r.standard_normal((B, Hq, N, d)).astype(np.float32)
+    k = r.standard_normal((B, Hkv, N, d)).astype(np.float32)
+    v = r.standard_normal((B, Hkv, N, d)).astype(np.float32)
+    return q, k, v
+
+
+def test_prefill_full_budget_equals_dense_causal():
+    q, k, v = _small_prefill(20)
+    bs = 32
+    Hkv = k.shape[1]
+    G = q.shape[1] // Hkv
+    _, _, _, idx, cnt = oracle.prefill_select(q, k, Hkv, bs, kb=64)
+    nb = q.shape[2] // bs
+    assert np.all(cnt == np.arange(nb)[None, None, :] + 1)
+    out, lse = oracle.attend_prefill(q, k, v, bs, idx)
+    ref = _sdpa64(q, np.repeat(k, G, 1), np.repeat(v, G, 1), causal=True)
+    assert np.allclose(out.reshape(ref.shape), ref, atol=1e-10, rtol=0)
+    # lse against the library logsumexp of the causal logits
+    qt = torch.as_tensor(q, dtype=torch.float64)
+    kt = torch.as_tensor(np.repeat(k, G, 1), dtype=torch.float64)
+    logits = qt @ kt.transpose(-1, -2) / math.sqrt(q.shape[-1])
+    causal = torch.ones(logits.shape[-2:], dtype=torch.bool).tril()
+    ref_lse = torch.logsumexp(logits.masked_fill(~causal, -math.inf), dim=-1).numpy()
+    assert np.allclose(lse.reshape(ref_lse.shape), ref_lse, atol=1e-10)
+
+
+def test_prefill_sparse_equals_masked_library_attention():
+    q, k, v = _small_prefill(21, B=2)
+    bs, kb = 32, 2
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    _, _, _, idx, _ = oracle.prefill_select(q, k, Hkv, bs, kb)
+    out, _ = oracle.attend_prefill(q, k, v, bs, idx)
+    mask = np.zeros((B, Hq, N, N), bool)
+    for b in range(B):
+        for h in range(Hq):
+            for t in range(N):
+                blocks = set(int(x) for x in idx[b, h // G, t // bs] if x >= 0)
+                for u in range(t + 1):
+                    mask[b, h, t, u] = (u // bs) in blocks
+    ref = _sdpa64(q, np.repeat(k, G, 1), np.repeat(v, G, 1), mask=mask)
+    assert np.allclose(out.reshape(ref.shape), ref, atol=1e-10, rtol=0)
+
+
+def test_prefill_selection_keeps_current_and_budget():
+    q, k, v = _small_prefill(22, N=512)
+    bs, kb = 32, 3
+    _, _, _, idx, cnt = oracle.prefill_select(q, k, k.shape[1], bs, kb)
+    nb = 512 // bs
+    for i in range(nb):
+        row = idx[0, 0, i]
+        kept = [int(x) for x in row if x >= 0]
+        assert kept[-1] == i                       # current block kept, list ascending
+        assert kept == sorted(kept)
+        assert len(kept) == min(kb, i) + 1
+
+
+# ----------------------------------------------------------------------------
+# the gate (SAS): invariants and the library routine with an additive bias
+# ----------------------------------------------------------------------------
+
+def test_gate_with_uniform_scores_equals_ungated():
+    q, k, v = _small_prefill(30)
+    bs, kb = 32, 2
+    _, _, s, idx, _ = oracle.prefill_select(q, k, k.shape[1], bs, kb)
+    ungated, lse_u = oracle.attend_prefill(q, k, v, bs, idx)
+    uniform = np.full_like(s, 0.7)
+    gated, _ = oracle.attend_prefill(q, k, v, bs, idx, gate_scores=uniform)
+    assert np.allclose(gated, ungated, atol=1e-12, rtol=0)
+
+
+def test_gate_is_shift_invariant():
+    q, k, v = _small_prefill(31)
+    bs, kb = 32, 2
+    _, _, s, idx, _ = oracle.prefill_select(q, k, k.shape[1], bs, kb)
+    # dyadic scores (multiples of 2^-10, |s| < 8) so that s + 3 is exact in fp32
+    s = (np.round(s * 1024) / 1024).astype(np.float32)
+    a, _ = oracle.attend_prefill(q, k, v, bs, idx, gate_scores=s)
+    b, _ = oracle.attend_prefill(q, k, v, bs, idx, gate_scores=s + np.float32(3.0))
+    assert np.allclose(a, b, atol=1e-12, rtol=0)
+
+
+def test_gate_equals_library_attention_with_log_softmax_bias():
+    q, k, v = _small_prefill(32)
+    bs, kb = 32, 2
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    _, _, s, idx, _ = oracle.prefill_select(q, k, Hkv, bs, kb)
+    s = s * np.float32(5.0)   # make the gate far from uniform
+    out, _ = oracle.attend_prefill(q, k, v, bs, idx, gate_scores=s)
+    bias = np.full((B, Hq, N, N), -np.inf)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // G
+            for i in range(N // bs):
+                kept = [int(x) for x in idx[b, g, i] if x >= 0]
+                logg = torch.log_softmax(torch.tensor([float(s[b, g, i, j]) for j in kept],
+                                                      dtype=torch.float64), 0).numpy()
+                for t in range(i * bs, (i + 1) * bs):
+                    for jj, j in enumerate(kept):
+                        for u in range(j * bs, (j + 1) * bs):
+                            if u <= t:
+                                bias[b, h, t, u] = logg[jj]
+    ref = _sdpa64(q, np.repeat(k, G, 1), np.repeat(v, G, 1), mask=bias)
+    assert np.allclose(out.reshape(ref.shape), ref, atol=1e-10, rtol=0)
+
+
+# ----------------------------------------------------------------------------
+# decode
+# ----------------------------------------------------------------------------
+
+def _small_decode(seed, B=2, Hq=8, Hkv=2, Nk=512, d=16):
+    r = _rng(seed)
+    q = r.standard_normal((B, Hq, d)).astype(np.float32)
+    k = r.standard_normal((B, Hkv, Nk, d)).astype(np.float32)
+    v = r.standard_normal((B, Hkv, Nk, d)).astype(np.float32)
+    return q, k, v
+
+
+def test_decode_full_budget_equals_dense():
+    q, k, v = _small_decode(40)
+    bs = 32
+    B, Hq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    G = Hq // Hkv
+    kbar = oracle.pool_keys(k, bs)
+    _, _, idx, cnt = oracle.decode_select(q, kbar, Hkv, kb=Nk // bs)
+    assert np.all(cnt == Nk // bs)
+    out, _ = oracle.attend_decode(q, k, v, bs, idx)
+    ref = _sdpa64(q[:, :, None, :], np.repeat(k, G, 1), np.repeat(v, G, 1))
+    assert np.allclose(out.reshape(B, Hq, d), ref[:, :, 0], atol=1e-10, rtol=0)
+
+
+def test_decode_sparse_keeps_last_block_and_matches_library():
+    q, k, v = _small_decode(41)
+    bs, kb = 32, 3
+    B, Hq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    G = Hq // Hkv
+    kbar = oracle.pool_keys(k, bs)
+    _, _, idx, cnt = oracle.decode_select(q, kbar, Hkv, kb)
+    assert np.all(idx[:, :, kb] == Nk // bs - 1)
+    out, _ = oracle.attend_decode(q, k, v, bs, idx)
+    mask = np.zeros((B, Hq, 1, Nk), bool)
+    for b in range(B):
+        for h in range(Hq):
+            for j in idx[b, h // G]:
+                mask[b, h, 0, j * bs:(j + 1) * bs] = True
+    ref = _sdpa64(q[:, :, None, :], np.repeat(k, G, 1), np.repeat(v, G, 1), mask=mask)
+    assert np.allclose(out.reshape(B, Hq, d), ref[:, :, 0], atol=1e-10, rtol=0)
+
+
+# ----------------------------------------------------------------------------
+# gist selective expansion (SSA)
+# ----------------------------------------------------------------------------
+
+def _small_gist(seed, B=2, Hq=4, Hkv=2, Nk=256, d=16, chunk=32):
+    r = _rng(seed)
+    q, k, v = _small_decode(seed, B, Hq, Hkv, Nk, d)
+    nc = Nk // chunk
+    gk = r.standard_normal((B, Hkv, nc, d)).astype(np.float32)
+    gv = r.standard_normal((B, Hkv, nc, d)).astype(np.float32)
+    return q, k, v, gk, gv
+
+
+def test_gist_all_chunks_expanded_equals_dense():
+    q, k, v, gk, gv = _small_gist(50)
+    chunk = 32
+    B, Hq, d = q.shape
+    G = Hq // k.shape[1]
+    _, idx, _ = oracle.gist_select(q, gk, kb=k.shape[2] // chunk)
+    out, _ = oracle.attend_gist(q, k, v, gk, gv, chunk, idx)
+    ref = _sdpa64(q[:, :, None, :], np.repeat(k, G, 1), np.repeat(v, G, 1))
+    assert np.allclose(out.reshape(B, Hq, d), ref[:, :, 0], atol=1e-10, rtol=0)
+
+
+def test_gist_nothing_expanded_equals_attention_over_gists():
+    q, k, v, gk, gv = _small_gist(51)
+    chunk = 32
+    B, Hq, d = q.shape
+    G = Hq // k.shape[1]
+    _, idx, cnt = oracle.gist_select(q, gk, kb=0)
+    assert np.all(cnt == 0)
+    out, _ = oracle.attend_gist(q, k, v, gk, gv, chunk, np.full((B, Hq, 1), -1, np.int32))
+    ref = _sdpa64(q[:, :, None, :], np.repeat(gk, G, 1), np.repeat(gv, G, 1))
+    assert np.allclose(out.reshape(B, Hq, d), ref[:, :, 0], atol=1e-10, rtol=0)
+
+
+def test_gist_mixture_matches_library_on_explicit_key_set():
+    q, k, v, gk, gv = _small_gist(52)
+    chunk, kb = 32, 3
+    B, Hq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    G = Hq // Hkv
+    nc = Nk // chunk
+    s, idx, _ = oracle.gist_select(q, gk, kb)
+    # per-head choices are independent: heads of one group may differ
+    out, _ = oracle.attend_gist(q, k, v, gk, gv, chunk, idx)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // G
+            chosen = set(int(x) for x in idx[b, h] if x >= 0)
+            assert len(chosen) == kb
+            top = np.argsort(-s[b, h], kind="stable")[:kb]
+            assert chosen == set(int(x) for x in top)
+            keys, vals = [], []
+            for c in range(nc):
+                if c in chosen:
+                    keys.append(k[b, g, c * chunk:(c + 1) * chunk]); vals.append(v[b, g, c * chunk:(c + 1) * chunk])
+                else:
+                    keys.append(gk[b, g, c:c + 1]); vals.append(gv[b, g, c:c + 1])
+            K = np.concatenate(keys)[None, None]
+            V = np.concatenate(vals)[None, None]
+            ref = _sdpa64(q[b, h][None, None, None, :], K, V)
+            assert np.allclose(out[b * Hq + h], ref[0, 0, 0], atol=1e-10, rtol=0)
