@@ -1,0 +1,430 @@
+#!/usr/bin/env python
+"""Benchmark of the query-aware top-k block-sparse attention hot path on B200.
+
+One step = the whole path over one batch of synthetic input: block pooling
+and scoring, top-k selection (current block kept), and sparse attention over
+the kept blocks, as consecutive library calls on one stream.  The headline
+workload is the GQA prefill (B=1, 32 query / 8 KV heads, d=128, 32768
+tokens, 64-token blocks, 16 history blocks + the current one).
+
+Prints ONE JSON line (rank 0).  `value` is selected query-key pairs per
+second over the whole step, aggregated over all ranks (each rank runs its own
+independent problem: weak scaling, no collective on the data path).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+`--impl reference` times the CPU oracle (the plain definition of the method)
+on the host cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "selected QK-pairs/s (prefill step: pool+score+top-k+sparse attention)"
+UNIT = "pairs/s"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="prefill_gqa_bf16")
+    ap.add_argument("--cpu-rows", type=int, default=8192, help="query rows in the oracle CPU-baseline sample")
+    ap.add_argument("--ref-rows", type=int, default=1024, help="query rows per reference-arm step")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-secondary", action="store_true", help="skip the decode secondary figures")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------
+# environment: ranks, peaks, clocks
+# ----------------------------------------------------------------------------
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """Samples SM clock, power and throttle reasons through NVML (read-only)
+    every `period` seconds in a background thread."""
+
+    REASONS = {
+        "hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+        "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+        "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+        "sw_power_cap": "nvmlClocksEventReasonSwPowerCap",
+        "hw_power_brake_slowdown": "nvmlClocksEventReasonHwPowerBrakeSlowdown",
+    }
+
+    def __init__(self, device_index: int, period: float = 0.02):
+        self.samples = []
+        self.period = period
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            self.max_mhz = None
+        self.t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                power = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                self.samples.append((time.time(), mhz, reasons, power))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self._ok:
+            self.t.start()
+        return self
+
+    def stop(self):
+        self._stop.set()
+        if self._ok:
+            self.t.join(timeout=2)
+
+    def summary(self, t0, t1):
+        if not self._ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"], "samples": 0}
+        win = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not win:   # region shorter than the sampling period: nearest samples
+            win = sorted(self.samples, key=lambda s: min(abs(s[0] - t0), abs(s[0] - t1)))[:3]
+        active = set()
+        for _, _, r, _ in win:
+            for name, const in self.REASONS.items():
+                if r & getattr(self.nv, const):
+                    active.add(name)
+        return {"sm_mhz": statistics.median([s[1] for s in win]) if win else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(active),
+                "power_w_max": max(s[3] for s in win) if win else None, "samples": len(win)}
+
+
+def profile_traffic(kernel_file: str, summary_name: str):
+    """Per-launch DRAM traffic of the kernel from a committed ncu summary, or
+    None when absent or taken on a different kernel source."""
+    path = os.path.join(ROOT, "profiles", summary_name)
+    if not os.path.exists(path):
+        return None, None
+    text = open(path).read()
+    m_t = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    m_h = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", text)
+    if not m_t or not m_h:
+        return None, None
+    return float(m_t.group(1)), m_h.group(1)
+
+
+def kernel_source_sha(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "top_block_sparse_bsa_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+# ----------------------------------------------------------------------------
+# oracle sample (CPU baseline and reference arm)
+# ----------------------------------------------------------------------------
+
+def oracle_prefill_sample(w, q, k, v, group: int, rows: int, seed: int):
+    """Times the oracle on one KV group: its selector (pool + score + top-k)
+    over the group's whole sequence, and attention for `rows` random query
+    rows of the group's heads.  Returns (pairs, seconds charged, detail)."""
+    import oracle
+    b, g = divmod(group, w.Hkv)
+    G = w.G
+    qs = q[b:b + 1, g * G:(g + 1) * G].float().cpu().numpy()
+    ks = k[b:b + 1, g:g + 1].float().cpu().numpy()
+    vs = v[b:b + 1, g:g + 1].float().cpu().numpy()
+    t0 = time.perf_counter()
+    _, _, s, idx, _ = oracle.prefill_select(qs, ks, 1, w.bs, w.kb)
+    t_sel = time.perf_counter() - t0
+    r = np.random.default_rng(seed)
+    flat = r.choice(G * w.N, size=min(rows, G * w.N), replace=False).astype(np.int64)
+    t1 = time.perf_counter()
+    oracle.attend_prefill(qs, ks, vs, w.bs, idx, gate_scores=s if w.kind == "gated" else None, rows=flat)
+    t_att = time.perf_counter() - t1
+    # exact pairs of the sampled rows
+    tpos = flat % w.N
+    pairs = 0
+    for t in tpos:
+        i = int(t) // w.bs
+        for j in idx[0, 0, i]:
+            if j < 0:
+                break
+            pairs += w.bs if j < i else (int(t) % w.bs) + 1
+    charged = t_att + t_sel * (len(flat) / (G * w.N))
+    return pairs, charged, {"t_select_s": t_sel, "t_attend_s": t_att, "rows": int(len(flat))}
+
+
+def run_reference(args, world, rank):
+    import bsa_workloads as W
+    import oracle
+    import torch
+    if rank != 0:
+        return 0
+    w = W.get(args.config)
+    inp = W.make_inputs(w, "cpu")
+    threads = oracle.max_threads()
+    pairs_total, secs_total = 0, 0.0
+    for s in range(args.warmup + args.steps):
+        group = s % (w.B * w.Hkv)
+        pairs, secs, _ = oracle_prefill_sample(w, inp["q"], inp["k"], inp["v"], group, args.ref_rows, seed=s)
+        if s >= args.warmup:
+            pairs_total += pairs
+            secs_total += secs
+    value = pairs_total / secs_total
+    sample = (f"per step: oracle selector (pool+score+top-k) on one KV group's full sequence, charged "
+              f"pro rata, plus fp64 attention for {args.ref_rows} random query rows of that group")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs_total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": w.name},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+
+def run_prefill(args, world, rank, local, peaks, peak_src):
+    import torch
+    import bsa_workloads as W
+    from top_block_sparse_bsa_b200 import accounting as acc
+    from top_block_sparse_bsa_b200 import pipeline
+
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    base = W.get(args.config)
+    w = base.scaled(seed=base.seed + 1000 * rank, name=base.name) if rank else base
+    inp = W.make_inputs(w, dev)
+    q, k, v = inp["q"], inp["k"], inp["v"]
+    step = pipeline.PrefillStep(q, k, v, w.bs, w.kb, gated=(w.kind == "gated"))
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        step.run(with_lse=False)
+    torch.cuda.synchronize()
+    idx = step.bufs["idx"].cpu().numpy()
+    pairs = acc.prefill_pairs(idx, w.bs, w.G)
+    flops = 4.0 * w.d * pairs
+    kv_bytes = acc.prefill_kv_bytes(idx, w.bs, w.d, 2 if w.dtype == "bf16" else 4)
+    full_pairs = acc.dense_pairs(w.N, causal=True) * w.B * w.Hq
+
+    sampler = ClockSampler(local).start()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ka = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    kb_ = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    ev0.record(stream)
+    for s in range(args.steps):
+        step.select()
+        ka[s].record(stream)
+        step.attend(with_lse=False)
+        kb_[s].record(stream)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    if dist:
+        dist.barrier()
+    sampler.stop()
+    step_ms = ev0.elapsed_time(ev1) / args.steps
+    attn_ms = statistics.mean(ka[s].elapsed_time(kb_[s]) for s in range(args.steps))
+    if dist:
+        t = torch.tensor([step_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        step_ms = float(t.item())
+    value = pairs * world / (step_ms / 1e3)
+
+    # roofline of the dominant kernel (sparse attention)
+    sustained = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    achieved_tflops = flops / (attn_ms / 1e3) / 1e12
+    hbm = peaks["hbm_gbs"]
+    t_flop = flops / (sustained * 1e12)
+    t_hbm = kv_bytes / (hbm * 1e9)
+    traffic, sha = profile_traffic("attn_prefill.cu", f"attn_prefill_{w.name}.md")
+    if sha is not None and sha != kernel_source_sha(["attn_prefill.cu", "common.cuh"]):
+        traffic = None
+    roofline = {
+        "bound": "tensor", "achieved": achieved_tflops, "peak": sustained, "unit": "TFLOP/s",
+        "frac": achieved_tflops / sustained, "traffic": traffic,
+        "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step loop)",
+        "frac_of_burst_peak": achieved_tflops / peaks["bf16_tflops"],
+        "kernel": "attn_prefill_kernel", "kernel_ms": attn_ms,
+        "algorithmic_flop_per_launch": flops, "selected_kv_bytes_per_launch": kv_bytes,
+        "roofline_time_ms": 1e3 * max(t_flop, t_hbm),
+        "frac_of_roofline_time": (1e3 * max(t_flop, t_hbm)) / attn_ms,
+        "hbm_gbs_on_selected_bytes": kv_bytes / (attn_ms / 1e3) / 1e9,
+    }
+    clocks = sampler.summary(t_wall0, t_wall1)
+
+    # end to end through the C ABI with host buffers
+    e2e = None
+    if args.e2e_steps > 0:
+        hq = q.cpu().pin_memory()
+        hk = k.cpu().pin_memory()
+        hv = v.cpu().pin_memory()
+        ho = torch.empty_like(hq).pin_memory()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        for it in range(args.e2e_steps + 1):
+            if it == 1:
+                e0.record(stream)
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            step.run(with_lse=False)
+            ho.copy_(step.bufs["o"], non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+        if dist:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        h2d = (hq.numel() + hk.numel() + hv.numel()) * hq.element_size()
+        e2e = {"value": pairs * world / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": ho.numel() * ho.element_size(), "ms_per_step": e2e_ms}
+
+    secondary = None
+    if not args.no_secondary and world == 1:
+        secondary = {"decode": run_decode_secondary(dev, peaks)}
+
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        pairs_s, secs, detail = oracle_prefill_sample(w, q, k, v, group=0, rows=args.cpu_rows, seed=0)
+        cpu_baseline = {"value": pairs_s / secs, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
+                        "sample": (f"oracle selector (pool+score+top-k) on KV group 0's full 32768-token "
+                                   f"sequence, charged pro rata, plus fp64 attention for {detail['rows']} "
+                                   f"random query rows of that group"),
+                        "detail": detail}
+
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "seq_len": w.N, "d": w.d,
+                   "block": w.bs, "budget": f"{w.kb}+current", "global_batch": w.B * world,
+                   "parallelism": f"independent problems x{world}",
+                   "l2": f"inputs larger than L2 ({(q.numel() + k.numel() + v.numel()) * 2 / 2**20:.0f} MiB > 126 MiB)",
+                   "sparsity": acc.sparsity(pairs, full_pairs)},
+        "roofline": roofline,
+        "cpu_baseline": cpu_baseline,
+        "e2e": e2e,
+        "clocks": clocks,
+        "gpu_launches": 5 * args.steps,
+        "secondary": secondary,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_decode_secondary(dev, peaks, iters: int = 20):
+    """µs per decode step and HBM GB/s over the selected bytes for the
+    131072-token decode workload, L2 flushed before every iteration."""
+    import torch
+    import bsa_workloads as W
+    from top_block_sparse_bsa_b200 import accounting as acc
+    from top_block_sparse_bsa_b200 import pipeline
+    w = W.get("decode_bf16")
+    inp = W.make_inputs(w, dev)
+    step = pipeline.DecodeStep(inp["q"], inp["k"], inp["v"], w.bs, w.kb)
+    step.pool_cache()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        step.run(with_lse=False)
+    torch.cuda.synchronize()
+    idx = step.bufs["idx"].cpu().numpy()
+    kv_bytes = acc.decode_kv_bytes(idx, w.bs, w.d, 2)
+    stream = torch.cuda.current_stream()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(iters)]
+    for it in range(iters):
+        flush.fill_(it & 0xFF)
+        ev[it][0].record(stream)
+        step.select()
+        ev[it][1].record(stream)
+        step.attend(with_lse=False)
+        ev[it][2].record(stream)
+    torch.cuda.synchronize()
+    step_us = statistics.median(1e3 * e[0].elapsed_time(e[2]) for e in ev)
+    attn_us = statistics.median(1e3 * e[1].elapsed_time(e[2]) for e in ev)
+    gbs = kv_bytes / (attn_us / 1e6) / 1e9
+    del inp, step, flush
+    torch.cuda.empty_cache()
+    return {"workload": w.name, "us_per_step": step_us, "attn_us": attn_us, "selected_kv_bytes": kv_bytes,
+            "hbm_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
+            "roofline_us": kv_bytes / (peaks["hbm_gbs"] * 1e9) * 1e6, "l2": "flushed (256 MiB write) per iteration"}
+
+
+def main():
+    args = parse_args()
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+    peaks, src = load_peaks()
+    return run_prefill(args, world, rank, local, peaks, src)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,223 @@
+/*
+ * bsa.h -- C ABI of libbsa: query-aware top-k block-sparse causal attention
+ * on NVIDIA B200 (sm_100a).
+ *
+ * The method, as the source pages state it:
+ *   - a cheap selector scores every KV block (or chunk gist) against the
+ *     query -- "粗粒度 Block 打分" (coarse block scoring), 稀疏注意力 tutorial
+ *     §4.6; SAS page, 核心模块 1; SSA page, 推理时的关键模块 1;
+ *   - the top-k blocks are kept per query block or decode token, per KV-head
+ *     group, with the current block always kept -- SAS page, 核心洞察 and
+ *     核心模块 3 ("始终保留的当前块"), and its 推理 paragraph;
+ *   - FlashAttention-style attention runs over the kept blocks only -- the
+ *     tutorial §2 (real speed-up needs the skipped region never computed) and
+ *     §7 (Block-Sparse FlashAttention);
+ *   - the gated variant adds log g_j to the logits of every token of block j,
+ *     g = softmax of the selector scores over the kept blocks -- SAS page,
+ *     核心模块 2-3.
+ *
+ * Conventions shared by every call
+ *   Layout     all tensors are dense and contiguous, head-major [B, H, N, d]
+ *              with d innermost; block j of a sequence is tokens
+ *              [j*block, (j+1)*block).  Query head h belongs to KV group
+ *              h / (Hq/Hkv) (GQA grouping).
+ *   Pointers   all data pointers are DEVICE pointers, 16-byte aligned, owned
+ *              by the caller.  The library never allocates, frees or
+ *              synchronises device memory on these paths; scratch space is
+ *              passed in by the caller (see bsa_workspace_bytes).
+ *   Streams    `stream` is a cudaStream_t (NULL = legacy default stream).
+ *              Every compute call only enqueues work on it and returns.
+ *   Errors     arguments are checked on the host before anything is launched:
+ *              malformed -> BSA_ERR_INVALID_ARG, legal but not built ->
+ *              BSA_ERR_UNSUPPORTED, a failed launch -> BSA_ERR_CUDA.  Nothing is
+ *              enqueued when a check fails.  Device-side problems (an index
+ *              out of range, a bounded wait that expired) never trap: the
+ *              kernel records a flag in the device status word, skips the bad
+ *              work and returns; read it with bsa_device_status().
+ *   Threads    calls are thread-safe; the only global state is the tensor-map
+ *              entry point and the device status word.
+ */
+#ifndef BSA_H_
+#define BSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BSA_OK = 0,
+  BSA_ERR_INVALID_ARG = 1,
+  BSA_ERR_UNSUPPORTED = 2,
+  BSA_ERR_CUDA = 3,
+  BSA_ERR_TIMEOUT = 4,      /* device status: a bounded wait expired */
+  BSA_ERR_DEVICE = 5        /* device status: bad index or shape seen by a kernel */
+} bsa_status_t;
+
+typedef enum { BSA_F32 = 0, BSA_BF16 = 1 } bsa_dtype_t;
+
+/* Problem shape.  Nq = query tokens (prefill: Nq == Nk; decode: Nq == 1),
+ * Nk = key/value tokens, block = KV block size (or gist chunk size). */
+typedef struct {
+  int B, Hq, Hkv, Nq, Nk, d, block;
+  bsa_dtype_t dtype;
+} bsa_shape_t;
+
+/* selector modes for bsa_score_blocks */
+enum { BSA_SCORE_PREFILL = 0, BSA_SCORE_DECODE = 1, BSA_SCORE_GIST = 2 };
+/* candidate rules for bsa_topk_select */
+enum { BSA_TOPK_CAUSAL_BLOCK = 0, BSA_TOPK_LAST_BLOCK = 1, BSA_TOPK_PLAIN = 2 };
+/* operations for bsa_workspace_bytes */
+enum { BSA_OP_DECODE = 0, BSA_OP_GIST_DECODE = 1 };
+
+/*
+ * bsa_score_blocks -- the cheap selector (block pooling + scoring).
+ * Cite: 稀疏注意力 tutorial §4.5 (a block = consecutive tokens) and §4.6
+ * (coarse block scoring instead of a full QK^T); SAS page 核心模块 1
+ * (continuous per-unit score); SSA page 推理时的关键模块 1 (score the query
+ * against every gist).  Score s = pooled-q . pooled-k / sqrt(d), in fp32 in
+ * a fixed order: pooling sums heads ascending then tokens ascending and
+ * divides once; the dot product runs over the channel ascending with every
+ * product and sum rounded to fp32; then one multiply by fp32(1/sqrt(d)).
+ *
+ * mode BSA_SCORE_PREFILL  (dtype BF16 or F32, Nq == Nk, Nk % block == 0)
+ *   q [B,Hq,Nq,d], k [B,Hkv,Nk,d]           (dtype)
+ *   pooled_q_out [B,Hkv,nb,d] fp32          (required) group query means
+ *   pooled_k_out [B,Hkv,nb,d] fp32          (required) block key means
+ *   pooled_k_in                              must be NULL
+ *   scores [B,Hkv,nb,nb] fp32: s[i][j] for j <= i, -inf for j > i.
+ * mode BSA_SCORE_DECODE   (one query token per sequence)
+ *   q [B,Hq,d]; pooled_k_in [B,Hkv,nb,d] fp32, the block-mean summary kept
+ *   next to the KV cache.  If pooled_k_in is NULL, k [B,Hkv,Nk,d] is pooled
+ *   into pooled_k_out (required then) first.
+ *   pooled_q_out [B,Hkv,d] fp32 (optional) receives the group query means.
+ *   scores [B,Hkv,nb] fp32.
+ * mode BSA_SCORE_GIST     (SSA: per query head, no pooling)
+ *   q [B,Hq,d]; k = gist keys [B,Hkv,nc,d] with nc = Nk/block;
+ *   scores [B,Hq,nc] fp32.  pooled_* must be NULL.
+ */
+bsa_status_t bsa_score_blocks(const bsa_shape_t* shape, int mode, const void* q, const void* k,
+                              const float* pooled_k_in, float* pooled_q_out, float* pooled_k_out,
+                              float* scores, void* stream);
+
+/*
+ * bsa_topk_select -- hard top-k selection of history blocks.
+ * Cite: SAS page, 推理 paragraph (each query keeps the k highest-scoring
+ * units) and 核心模块 3 (the current block is always kept); gated-sparse
+ * essay §四, pseudo-code step 2 (top-k blocks form the sparse index).
+ * scores [rows, ncols] fp32 (row-major).  Per row, candidates and the forced
+ * block depend on `mode`:
+ *   BSA_TOPK_CAUSAL_BLOCK  row r is query block i = r % ncols: candidates
+ *                          j < i, block i always kept (prefill);
+ *   BSA_TOPK_LAST_BLOCK    candidates j < ncols-1, block ncols-1 kept (decode);
+ *   BSA_TOPK_PLAIN         candidates j < ncols, nothing forced (gist).
+ * Order: larger score first, equal scores -> lower index first, NaN below
+ * every number.  min(kb, #candidates) are kept.
+ * idx_out [rows, idx_stride] int32: kept indices ascending, then -1;
+ *   idx_stride >= kb + (mode != PLAIN).  count_out [rows] int32 (optional).
+ * Limits: ncols <= 8192.
+ */
+bsa_status_t bsa_topk_select(const float* scores, int rows, int ncols, int mode, int kb,
+                             int* idx_out, int idx_stride, int* count_out, void* stream);
+
+/*
+ * bsa_sparse_attn_prefill -- block-sparse causal attention (prefill).
+ * Cite: 稀疏注意力 tutorial §1 (softmax(QK^T/sqrt(d))V), §2 (additive mask
+ * M in {0,-inf}; skip the masked region instead of computing it), §4.5
+ * (block-sparse pattern), §7 (Block-Sparse FlashAttention: online softmax).
+ * q [B,Hq,N,d], k/v [B,Hkv,N,d] (dtype), N = Nq = Nk, N % block == 0.
+ * idx [B,Hkv,nb,idx_stride] int32: for query block i of group g, the kept
+ *   blocks ascending, ended by -1 (or by idx_stride).  Entries must satisfy
+ *   0 <= j <= i; a kernel that finds another value skips it and sets
+ *   BSA_DEV_BAD_INDEX.  Inside block i, key u is masked for query t when u > t.
+ * softmax_scale: usually 1/sqrt(d).
+ * o [B,Hq,N,d] (dtype) output; lse [B,Hq,N] fp32 natural-log row LSE of the
+ *   scaled logits (optional, NULL to skip).
+ * Built: BF16 with d = 128 and block in {64,128} (tcgen05 + TMA kernel);
+ *   F32 with d in {64,128} and block in {64,128} (fp32 SIMT kernel).
+ */
+bsa_status_t bsa_sparse_attn_prefill(const bsa_shape_t* shape, const void* q, const void* k,
+                                     const void* v, const int* idx, int idx_stride,
+                                     float softmax_scale, void* o, float* lse, void* stream);
+
+/*
+ * bsa_gated_attn_fwd -- SAS gated sparse attention (inner log-gate).
+ * Cite: SAS page, 核心模块 2 (the selector's continuous score enters the
+ * softmax logits in log form) and 核心模块 3 (the gate is a normalised softmax
+ * over the kept history blocks and the always-kept current block).
+ * As bsa_sparse_attn_prefill, plus sel_scores [B,Hkv,nb,nb] fp32 (the prefill
+ * selector scores, as bsa_score_blocks writes them): for query block i the
+ * logit of every key of kept block j gains log g_j with
+ *   g_j = exp(s[i][j]) / sum_{l kept} exp(s[i][l]).
+ * All heads of a KV group share the group's gate.
+ */
+bsa_status_t bsa_gated_attn_fwd(const bsa_shape_t* shape, const void* q, const void* k,
+                                const void* v, const int* idx, int idx_stride,
+                                const float* sel_scores, float softmax_scale, void* o, float* lse,
+                                void* stream);
+
+/*
+ * bsa_sparse_attn_decode -- one query token per sequence over a retained KV
+ * cache, reading only the kept blocks.
+ * Cite: 稀疏注意力 tutorial §5 (decode: one new query against the history);
+ * Sparse Frontier review §2.4.2 (full cache retained, selective loading, as
+ * Quest does with query-aware pages).
+ * q [B,Hq,d] (dtype BF16), k_cache/v_cache [B,Hkv,Nk,d], Nk % block == 0,
+ * idx [B,Hkv,idx_stride] int32 kept blocks ascending, -1 ended; every cached
+ * token is history of the query (no causal mask).  All heads of a group
+ * share one gather of the kept blocks.
+ * workspace: device scratch of at least
+ *   bsa_workspace_bytes(BSA_OP_DECODE, shape, idx_stride) bytes, 256-byte
+ *   aligned; its contents on entry do not matter.
+ * o [B,Hq,d] (dtype); lse [B,Hq] fp32 (optional).
+ * Built: BF16, d = 128, block = 64.
+ */
+bsa_status_t bsa_sparse_attn_decode(const bsa_shape_t* shape, const void* q, const void* k_cache,
+                                    const void* v_cache, const int* idx, int idx_stride,
+                                    float softmax_scale, void* workspace, size_t workspace_bytes,
+                                    void* o, float* lse, void* stream);
+
+/*
+ * bsa_gist_expand_decode -- SSA gist scoring + selective expansion decode.
+ * Cite: SSA page, 推理时的关键模块: (1) score the query against every chunk's
+ * gist key, (2) expand the top-k chunks back to their tokens -- under GQA
+ * each query head chooses its own chunks, (3) attend over the expanded tokens
+ * together with the gists of the chunks that were not expanded.
+ * q [B,Hq,d], k_cache/v_cache [B,Hkv,Nk,d] (tokens), gist_k/gist_v
+ * [B,Hkv,nc,d] with nc = Nk/block (one gist per chunk), all BF16.
+ * topk: chunks expanded per query head (0 <= topk <= nc).
+ * idx_in [B,Hq,topk] int32 (optional): if given, these chunks are expanded
+ *   and no scoring/selection runs (the way to inject a known index set).
+ * idx_out [B,Hq,topk] int32 (optional): receives the chosen chunks ascending.
+ * workspace: bsa_workspace_bytes(BSA_OP_GIST_DECODE, shape, topk) bytes.
+ * o [B,Hq,d] (dtype); lse [B,Hq] fp32 (optional).
+ * Built: BF16, d = 128, block = 64.
+ */
+bsa_status_t bsa_gist_expand_decode(const bsa_shape_t* shape, const void* q, const void* k_cache,
+                                    const void* v_cache, const void* gist_k, const void* gist_v,
+                                    int topk, const int* idx_in, int* idx_out,
+                                    float softmax_scale, void* workspace, size_t workspace_bytes,
+                                    void* o, float* lse, void* stream);
+
+/* Scratch bytes a decode call needs (op = BSA_OP_*; budget = idx_stride for
+ * BSA_OP_DECODE, topk for BSA_OP_GIST_DECODE).  0 on a bad shape. */
+size_t bsa_workspace_bytes(int op, const bsa_shape_t* shape, int budget);
+
+/* Human-readable name of a status code (static string). */
+const char* bsa_status_string(bsa_status_t status);
+
+/* Reads (and, if reset != 0, clears) the current device's status word.
+ * Synchronises the device.  flags may be NULL.  Returns BSA_ERR_TIMEOUT or
+ * BSA_ERR_DEVICE when a flag is set, BSA_OK otherwise. */
+bsa_status_t bsa_device_status(unsigned int* flags, int reset);
+
+/* Library ABI version (major*100 + minor). */
+int bsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSA_H_ */

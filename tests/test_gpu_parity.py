@@ -1,0 +1,368 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs.
+
+Selection: the selector is computed in the same fixed fp32 order on both
+sides, so pooled means, scores and kept indices are compared bit for bit.
+Attention: both sides are fed the oracle's index set, and the outputs must
+be within max-abs 2e-2 / mean-abs 2e-3 (bf16 inputs) or max-abs 1e-4 (fp32
+inputs) of the oracle's fp64 result.
+
+Small cases span several tiles and odd (ragged) kept lists and are checked on
+every output row; the full workload sizes are checked on sampled rows.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import bsa_workloads as W
+import oracle
+
+pytestmark = pytest.mark.gpu
+
+TOL_BF16 = dict(max_abs=2e-2, mean_abs=2e-3)
+TOL_F32 = dict(max_abs=1e-4, mean_abs=1e-4)
+
+
+def _bsa():
+    import top_block_sparse_bsa_b200 as bsa
+    return bsa
+
+
+def _pipe():
+    from top_block_sparse_bsa_b200 import pipeline
+    return pipeline
+
+
+def _tol(dtype):
+    return TOL_F32 if dtype == "f32" else TOL_BF16
+
+
+def _assert_close(got, want, tol, what=""):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    assert got.shape == want.shape, (what, got.shape, want.shape)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    err = np.abs(got - want)
+    assert err.max() <= tol["max_abs"], f"{what}: max-abs {err.max():.3e} > {tol['max_abs']}"
+    assert err.mean() <= tol["mean_abs"], f"{what}: mean-abs {err.mean():.3e} > {tol['mean_abs']}"
+
+
+def _status_clean():
+    bsa = _bsa()
+    code, flags = bsa.bsa_device_status(reset=True)
+    assert code == 0 and flags == 0, f"device status {code} flags {flags:#x}"
+
+
+# ----------------------------------------------------------------------------
+# prefill (ungated and gated)
+# ----------------------------------------------------------------------------
+
+def _prefill_case(w: W.Workload, gated: bool, rows_sample=None):
+    pipe = _pipe()
+    inp = W.make_inputs(w, "cuda")
+    q, k, v = inp["q"], inp["k"], inp["v"]
+    step = pipe.PrefillStep(q, k, v, w.bs, w.kb, gated=gated)
+    step.select()
+    torch.cuda.synchronize()
+    qc, kc, vc = q.float().cpu(), k.float().cpu(), v.float().cpu()
+    qbar, kbar, s, idx, cnt = oracle.prefill_select(qc, kc, w.Hkv, w.bs, w.kb)
+    b = step.bufs
+    # selector: bit-exact
+    assert np.array_equal(b["kbar"].cpu().numpy(), kbar), "pooled keys differ"
+    assert np.array_equal(b["qbar"].cpu().numpy(), qbar), "pooled queries differ"
+    assert np.array_equal(b["scores"].cpu().numpy(), s), "scores differ"
+    assert np.array_equal(b["idx"].cpu().numpy(), idx), "kept indices differ"
+    assert np.array_equal(b["count"].cpu().numpy(), cnt)
+    # attention on the oracle's index set
+    idx_dev = torch.from_numpy(idx).cuda()
+    step.attend(idx=idx_dev)
+    torch.cuda.synchronize()
+    _status_clean()
+    total = w.B * w.Hq * w.N
+    rows = np.arange(total) if rows_sample is None else np.asarray(rows_sample, dtype=np.int64)
+    want, want_lse = oracle.attend_prefill(qc, kc, vc, w.bs, idx, gate_scores=s if gated else None, rows=rows)
+    got = b["o"].float().reshape(total, w.d)[torch.from_numpy(rows).cuda()].cpu().numpy()
+    got_lse = b["lse"].reshape(total)[torch.from_numpy(rows).cuda()].cpu().numpy()
+    _assert_close(got, want, _tol(w.dtype), f"{w.name} out")
+    _assert_close(got_lse, want_lse, dict(max_abs=2e-3, mean_abs=2e-4) if w.dtype == "bf16" else TOL_F32,
+                  f"{w.name} lse")
+
+
+@pytest.mark.parametrize("gated", [False, True])
+def test_tiny_prefill_f32_full_config(gated):
+    _prefill_case(W.get("tiny_prefill_f32"), gated)
+
+
+@pytest.mark.parametrize("kb", [4, 5])
+def test_prefill_gqa_bf16_small(kb):
+    # 32 blocks, kept lists of odd and even length, two 128-row tiles per CTA
+    w = W.get("prefill_gqa_bf16").scaled(Hq=8, Hkv=2, N=2048, kb=kb)
+    _prefill_case(w, gated=False)
+
+
+def test_gated_bf16_small_group_of_seven():
+    # G = 7 heads x 128 rows: four CTAs per unit, the last with one tile
+    w = W.get("gated_prefill_bf16").scaled(B=1, Hq=7, Hkv=1, N=2048, kb=3)
+    _prefill_case(w, gated=True)
+
+
+def test_gated_bf16_small_gqa():
+    w = W.get("gated_prefill_bf16").scaled(B=2, Hq=8, Hkv=2, N=1024, kb=2)
+    _prefill_case(w, gated=True)
+
+
+def test_prefill_bf16_block128_ungated():
+    w = W.get("gated_prefill_bf16").scaled(B=1, Hq=4, Hkv=2, N=2048, kb=4, kind="prefill")
+    _prefill_case(w, gated=False)
+
+
+def _sample_rows(w: W.Workload, n: int, seed: int):
+    r = np.random.default_rng(seed)
+    b = r.integers(0, w.B, n)
+    h = r.integers(0, w.Hq, n)
+    t = r.integers(0, w.N, n)
+    t[:4] = [0, w.bs - 1, w.N - 1, w.N - w.bs]   # first / last rows of the first and last blocks
+    return (b * w.Hq + h) * w.N + t
+
+
+def test_prefill_gqa_bf16_full_size_sampled():
+    w = W.get("prefill_gqa_bf16")
+    _prefill_case(w, gated=False, rows_sample=_sample_rows(w, 96, 1))
+
+
+def test_gated_bf16_full_size_sampled():
+    w = W.get("gated_prefill_bf16")
+    _prefill_case(w, gated=True, rows_sample=_sample_rows(w, 96, 3))
+
+
+def test_prefill_empty_and_bad_lists():
+    """A query block with an empty list gives zero rows and LSE -inf; an entry
+    in the future (> i) is skipped and flagged, never read."""
+    bsa = _bsa()
+    pipe = _pipe()
+    w = W.get("prefill_gqa_bf16").scaled(Hq=4, Hkv=1, N=512, kb=2)
+    inp = W.make_inputs(w, "cuda")
+    step = pipe.PrefillStep(inp["q"], inp["k"], inp["v"], w.bs, w.kb)
+    step.select()
+    idx = step.bufs["idx"].clone()
+    a = int(idx[0, 0, 5, 0].item())
+    idx[0, 0, 3, :] = -1                                                   # empty list
+    idx[0, 0, 5, :] = torch.tensor([a, 7, -1], dtype=torch.int32)          # 7 > 5: future block
+    good = idx.clone()
+    good[0, 0, 5, :] = torch.tensor([a, -1, -1], dtype=torch.int32)
+    bsa.bsa_device_status(reset=True)
+    step.attend(idx=idx)
+    code, flags = bsa.bsa_device_status(reset=True)
+    assert flags & 2, "bad index not flagged"
+    o_bad = step.bufs["o"].clone()
+    lse_bad = step.bufs["lse"].clone()
+    # block 3 rows are zero with LSE -inf
+    assert torch.all(o_bad[0, :, 3 * w.bs:4 * w.bs] == 0)
+    assert torch.all(torch.isneginf(lse_bad[0, :, 3 * w.bs:4 * w.bs]))
+    # block 5 equals the run without the bad entry
+    step.attend(idx=good)
+    torch.cuda.synchronize()
+    assert torch.equal(o_bad[0, :, 5 * w.bs:6 * w.bs], step.bufs["o"][0, :, 5 * w.bs:6 * w.bs])
+    _status_clean()
+
+
+# ----------------------------------------------------------------------------
+# top-k selection on crafted scores (ties, NaN, budgets)
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("mode", [0, 1, 2])
+def test_topk_ties_nan_and_budgets(mode):
+    bsa = _bsa()
+    r = np.random.default_rng(100 + mode)
+    for ncols in (1, 7, 33, 300, 2048):
+        for kb in (0, 1, 5, 64, ncols + 3):
+            rows = 9
+            s = r.integers(-4, 5, size=(rows, ncols)).astype(np.float32)
+            s[0, ::3] = np.nan
+            s[1, :] = 0.0
+            s[2, ::2] = -np.inf
+            s[3, 1::2] = -0.0
+            forced = 0 if mode == 2 else 1
+            stride = kb + forced + 2
+            want, cnt = oracle.topk(s, mode, kb, idx_stride=stride)
+            sd = torch.from_numpy(s).cuda()
+            idx = torch.empty((rows, stride), dtype=torch.int32, device="cuda")
+            count = torch.empty((rows,), dtype=torch.int32, device="cuda")
+            bsa.bsa_topk_select(sd, rows, ncols, mode, kb, idx, stride, count)
+            torch.cuda.synchronize()
+            assert np.array_equal(idx.cpu().numpy(), want), (ncols, kb)
+            assert np.array_equal(count.cpu().numpy(), cnt)
+
+
+# ----------------------------------------------------------------------------
+# decode
+# ----------------------------------------------------------------------------
+
+def _decode_case(w: W.Workload, groups=None):
+    """groups: list of (b, g) to check (default: all)."""
+    pipe = _pipe()
+    inp = W.make_inputs(w, "cuda")
+    q, kc, vc = inp["q"], inp["k"], inp["v"]
+    step = pipe.DecodeStep(q, kc, vc, w.bs, w.kb)
+    step.pool_cache()
+    step.select()
+    torch.cuda.synchronize()
+    b_ = step.bufs
+    G = w.G
+    if groups is None:
+        groups = [(b, g) for b in range(w.B) for g in range(w.Hkv)]
+    idx_all = b_["idx"].cpu().numpy()
+    oracle_idx = idx_all.copy()
+    for (b, g) in groups:
+        ks = kc[b:b + 1, g:g + 1].float().cpu()
+        qs = q[b:b + 1, g * G:(g + 1) * G].float().cpu()
+        kbar = oracle.pool_keys(ks, w.bs)
+        assert np.array_equal(b_["kbar"][b:b + 1, g:g + 1].cpu().numpy(), kbar), (b, g)
+        _, s, idx, cnt = oracle.decode_select(qs, kbar, 1, w.kb)
+        assert np.array_equal(b_["scores"][b, g].cpu().numpy(), s[0, 0]), (b, g)
+        assert np.array_equal(idx_all[b, g], idx[0, 0]), (b, g)
+        oracle_idx[b, g] = idx[0, 0]
+    step.attend(idx=torch.from_numpy(oracle_idx).cuda())
+    torch.cuda.synchronize()
+    _status_clean()
+    for (b, g) in groups:
+        ks = kc[b:b + 1, g:g + 1].float().cpu()
+        vs = vc[b:b + 1, g:g + 1].float().cpu()
+        qs = q[b:b + 1, g * G:(g + 1) * G].float().cpu()
+        want, want_lse = oracle.attend_decode(qs, ks, vs, w.bs, oracle_idx[b:b + 1, g:g + 1])
+        got = b_["o"][b, g * G:(g + 1) * G].float().cpu().numpy()
+        _assert_close(got, want, TOL_BF16, f"{w.name} decode ({b},{g})")
+        _assert_close(b_["lse"][b, g * G:(g + 1) * G].cpu().numpy(), want_lse,
+                      dict(max_abs=2e-3, mean_abs=2e-4), "decode lse")
+
+
+def test_decode_bf16_small():
+    w = W.get("decode_bf16").scaled(B=2, Hq=8, Hkv=2, N=8192, kb=12)
+    _decode_case(w)
+
+
+def test_decode_bf16_small_even_list_and_full_budget():
+    w = W.get("decode_bf16").scaled(B=1, Hq=4, Hkv=1, N=4096, kb=63)   # every block kept
+    _decode_case(w)
+
+
+def test_decode_bf16_full_size_sampled():
+    w = W.get("decode_bf16")
+    _decode_case(w, groups=[(0, 0), (5, 3), (15, 7), (9, 1)])
+
+
+def test_decode_split_count_invariance():
+    bsa = _bsa()
+    pipe = _pipe()
+    w = W.get("decode_bf16").scaled(B=2, Hq=8, Hkv=2, N=8192, kb=40)
+    inp = W.make_inputs(w, "cuda")
+    outs = []
+    for splits in ("1", "3", "7"):
+        os.environ["BSA_DECODE_SPLITS"] = splits
+        try:
+            step = pipe.DecodeStep(inp["q"], inp["k"], inp["v"], w.bs, w.kb)
+            step.pool_cache()
+            step.run()
+            torch.cuda.synchronize()
+            outs.append(step.bufs["o"].float().cpu())
+        finally:
+            del os.environ["BSA_DECODE_SPLITS"]
+    for o in outs[1:]:
+        assert (o - outs[0]).abs().max().item() <= 1e-2
+    _status_clean()
+
+
+# ----------------------------------------------------------------------------
+# gist selective expansion (SSA)
+# ----------------------------------------------------------------------------
+
+def _gist_case(w: W.Workload, groups=None, topk=None):
+    pipe = _pipe()
+    inp = W.make_inputs(w, "cuda")
+    topk = w.kb if topk is None else topk
+    G = w.G
+    nc = w.N // w.bs
+    step = pipe.GistStep(inp["q"], inp["k"], inp["v"], inp["gk"], inp["gv"], w.bs, topk)
+    step.run()
+    torch.cuda.synchronize()
+    _status_clean()
+    if groups is None:
+        groups = [(b, g) for b in range(w.B) for g in range(w.Hkv)]
+    for (b, g) in groups:
+        qs = inp["q"][b:b + 1, g * G:(g + 1) * G].float().cpu()
+        gks = inp["gk"][b:b + 1, g:g + 1].float().cpu()
+        gvs = inp["gv"][b:b + 1, g:g + 1].float().cpu()
+        ks = inp["k"][b:b + 1, g:g + 1].float().cpu()
+        vs = inp["v"][b:b + 1, g:g + 1].float().cpu()
+        s, idx, _ = oracle.gist_select(qs, gks, topk)
+        if topk > 0:
+            assert np.array_equal(step.bufs["idx"][b, g * G:(g + 1) * G, :topk].cpu().numpy(), idx[0]), (b, g)
+        else:
+            idx = np.full((1, G, 1), -1, np.int32)
+        want, want_lse = oracle.attend_gist(qs, ks, vs, gks, gvs, w.bs, idx)
+        got = step.bufs["o"][b, g * G:(g + 1) * G].float().cpu().numpy()
+        _assert_close(got, want, TOL_BF16, f"gist ({b},{g}) topk={topk}")
+        _assert_close(step.bufs["lse"][b, g * G:(g + 1) * G].cpu().numpy(), want_lse,
+                      dict(max_abs=2e-3, mean_abs=2e-4), "gist lse")
+
+
+def test_gist_bf16_small():
+    w = W.get("gist_decode_bf16").scaled(B=2, Hq=8, Hkv=2, N=8192, kb=8)
+    _gist_case(w)
+
+
+@pytest.mark.parametrize("topk", [0, 1, 128])
+def test_gist_bf16_edge_budgets(topk):
+    w = W.get("gist_decode_bf16").scaled(B=1, Hq=4, Hkv=1, N=8192, kb=topk)
+    _gist_case(w, topk=topk)
+
+
+def test_gist_bf16_full_size_sampled():
+    w = W.get("gist_decode_bf16")
+    _gist_case(w, groups=[(0, 0), (3, 5), (7, 7)])
+
+
+def test_gist_injected_index_set():
+    """idx_in bypasses scoring/selection: the given chunks are expanded."""
+    pipe = _pipe()
+    w = W.get("gist_decode_bf16").scaled(B=1, Hq=4, Hkv=1, N=8192, kb=3)
+    inp = W.make_inputs(w, "cuda")
+    idx = torch.tensor([[[0, 5, 127], [1, 2, 3], [7, 64, 100], [0, 1, 2]]], dtype=torch.int32, device="cuda")
+    step = pipe.GistStep(inp["q"], inp["k"], inp["v"], inp["gk"], inp["gv"], w.bs, 3)
+    step.run(idx_in=idx)
+    torch.cuda.synchronize()
+    want, _ = oracle.attend_gist(inp["q"].float().cpu(), inp["k"].float().cpu(), inp["v"].float().cpu(),
+                                 inp["gk"].float().cpu(), inp["gv"].float().cpu(), w.bs, idx.cpu().numpy())
+    _assert_close(step.bufs["o"][0].float().cpu().numpy(), want, TOL_BF16, "gist injected")
+    _status_clean()
+
+
+# ----------------------------------------------------------------------------
+# host-side argument checks (nothing is launched when they fail)
+# ----------------------------------------------------------------------------
+
+def test_invalid_arguments_rejected():
+    bsa = _bsa()
+    q = torch.zeros((1, 4, 256, 128), dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros((1, 1, 256, 128), dtype=torch.bfloat16, device="cuda")
+    o = torch.empty_like(q)
+    idx = torch.zeros((1, 1, 4, 3), dtype=torch.int32, device="cuda")
+    bad_g = bsa.make_shape(1, 4, 3, 256, 256, 128, 64, torch.bfloat16)   # Hq % Hkv != 0
+    with pytest.raises(bsa.BsaError) as e:
+        bsa.bsa_sparse_attn_prefill(bad_g, q, k, k, idx, 3, 0.1, o)
+    assert e.value.code == 1
+    bad_block = bsa.make_shape(1, 4, 1, 256, 256, 128, 32, torch.bfloat16)  # block 32 not built
+    with pytest.raises(bsa.BsaError) as e:
+        bsa.bsa_sparse_attn_prefill(bad_block, q, k, k, idx, 3, 0.1, o)
+    assert e.value.code == 2
+    good = bsa.make_shape(1, 4, 1, 256, 256, 128, 64, torch.bfloat16)
+    with pytest.raises(bsa.BsaError) as e:
+        bsa.bsa_sparse_attn_prefill(good, q, k, k, idx, 3, -1.0, o)   # bad scale
+    assert e.value.code == 1
+    with pytest.raises(bsa.BsaError) as e:
+        bsa.bsa_topk_select(torch.zeros((2, 8), device="cuda"), 2, 8, 0, 4, idx, 3)   # stride < kb+1
+    assert e.value.code == 1
+    _status_clean()

@@ -1,0 +1,419 @@
+// api.cu -- the C ABI of libbsa (see include/bsa.h): argument checks, TMA
+// tensor maps, workspace layout and kernel dispatch.  No call here allocates
+// or frees device memory; scratch comes from the caller.
+#include <math.h>
+#include <stdlib.h>
+
+#include <mutex>
+
+#include "../../include/bsa.h"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace bsa {
+
+// Device status word: kernels OR flags into it instead of trapping.
+__device__ uint32_t g_status_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+uint32_t* g_status_ptr[kMaxDevices] = {};
+int g_num_sms[kMaxDevices] = {};
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+bsa_status_t device_state(uint32_t** status, int* num_sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_status_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return BSA_ERR_CUDA;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return BSA_ERR_CUDA;
+    g_status_ptr[dev] = static_cast<uint32_t*>(p);
+    g_num_sms[dev] = sms;
+  }
+  if (g_encode == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+      return BSA_ERR_CUDA;
+    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  if (status) *status = g_status_ptr[dev];
+  if (num_sms) *num_sms = g_num_sms[dev];
+  return BSA_OK;
+}
+
+// 2-D bf16 view [rows, 128] with a box of 64 columns x box_rows rows and the
+// 128-byte swizzle the MMA descriptors expect.
+bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+  const cuuint64_t dims[2] = {128, rows};
+  const cuuint64_t strides[1] = {128 * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bsa_status_t check_shape(const bsa_shape_t* s) {
+  if (s == nullptr) return BSA_ERR_INVALID_ARG;
+  if (s->B <= 0 || s->Hq <= 0 || s->Hkv <= 0 || s->Nq <= 0 || s->Nk <= 0 || s->d <= 0 || s->block <= 0)
+    return BSA_ERR_INVALID_ARG;
+  if (s->Hq % s->Hkv != 0 || s->Nk % s->block != 0) return BSA_ERR_INVALID_ARG;
+  if (s->dtype != BSA_F32 && s->dtype != BSA_BF16) return BSA_ERR_INVALID_ARG;
+  const int64_t rows_q = static_cast<int64_t>(s->B) * s->Hq * s->Nq;
+  const int64_t rows_k = static_cast<int64_t>(s->B) * s->Hkv * s->Nk;
+  if (rows_q >= (1ll << 31) || rows_k >= (1ll << 31)) return BSA_ERR_UNSUPPORTED;
+  return BSA_OK;
+}
+
+bsa_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? BSA_OK : BSA_ERR_CUDA; }
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+float score_scale(int d) { return static_cast<float>(1.0 / sqrt(static_cast<double>(d))); }
+
+// split-K factor of the decode kernels: enough CTAs to cover every SM about
+// twice, each CTA keeping at least a few steps of two tiles.
+int decode_splits(int rows, int max_tiles, int num_sms) {
+  if (const char* env = getenv("BSA_DECODE_SPLITS")) {
+    const int v = atoi(env);
+    if (v > 0) return v;
+  }
+  int want = (2 * num_sms + rows - 1) / rows;
+  const int by_work = (max_tiles + 7) / 8;   // >= 4 steps (8 tiles) per split
+  if (want > by_work) want = by_work;
+  if (want < 1) want = 1;
+  // no CTA may own more than the kernel's tile-list capacity (1024)
+  const int min_for_cap = (max_tiles + 1023) / 1024;
+  if (want < min_for_cap) want = min_for_cap;
+  return want;
+}
+
+struct GistLayout {
+  size_t scores, idx, expanded, union_list, partial, total;
+  int union_stride, nsplit;
+};
+
+GistLayout gist_layout(const bsa_shape_t* s, int topk, int num_sms) {
+  GistLayout L{};
+  const int nc = s->Nk / s->block;
+  const int G = s->Hq / s->Hkv;
+  const int64_t rows = static_cast<int64_t>(s->B) * s->Hq;
+  L.union_stride = 1 + G * topk + nc / 64;
+  L.nsplit = decode_splits(s->B * s->Hkv, L.union_stride - 1, num_sms);
+  size_t off = 0;
+  L.scores = off;
+  off = align256(off + rows * nc * sizeof(float));
+  L.idx = off;
+  off = align256(off + rows * (topk > 0 ? topk : 1) * sizeof(int));
+  L.expanded = off;
+  off = align256(off + rows * (nc / 32) * sizeof(uint32_t));
+  L.union_list = off;
+  off = align256(off + static_cast<size_t>(s->B) * s->Hkv * L.union_stride * sizeof(int));
+  L.partial = off;
+  off = align256(off + rows * L.nsplit * (s->d + 4) * sizeof(float));
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+}  // namespace bsa
+
+using namespace bsa;
+
+extern "C" {
+
+int bsa_version(void) { return 100; }
+
+const char* bsa_status_string(bsa_status_t st) {
+  switch (st) {
+    case BSA_OK: return "BSA_OK";
+    case BSA_ERR_INVALID_ARG: return "BSA_ERR_INVALID_ARG";
+    case BSA_ERR_UNSUPPORTED: return "BSA_ERR_UNSUPPORTED";
+    case BSA_ERR_CUDA: return "BSA_ERR_CUDA";
+    case BSA_ERR_TIMEOUT: return "BSA_ERR_TIMEOUT";
+    case BSA_ERR_DEVICE: return "BSA_ERR_DEVICE";
+  }
+  return "BSA_ERR_UNKNOWN";
+}
+
+bsa_status_t bsa_device_status(unsigned int* flags, int reset) {
+  uint32_t* dev_ptr = nullptr;
+  bsa_status_t st = device_state(&dev_ptr, nullptr);
+  if (st != BSA_OK) return st;
+  if (cudaDeviceSynchronize() != cudaSuccess) return BSA_ERR_CUDA;
+  uint32_t v = 0;
+  if (cudaMemcpy(&v, dev_ptr, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return BSA_ERR_CUDA;
+  if (reset) {
+    const uint32_t zero = 0;
+    if (cudaMemcpy(dev_ptr, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return BSA_ERR_CUDA;
+  }
+  if (flags) *flags = v;
+  if (v & BSA_DEV_TIMEOUT) return BSA_ERR_TIMEOUT;
+  if (v) return BSA_ERR_DEVICE;
+  return BSA_OK;
+}
+
+size_t bsa_workspace_bytes(int op, const bsa_shape_t* s, int budget) {
+  if (check_shape(s) != BSA_OK || budget < 0) return 0;
+  int sms = 0;
+  if (device_state(nullptr, &sms) != BSA_OK) return 0;
+  if (op == BSA_OP_DECODE) {
+    const int nsplit = decode_splits(s->B * s->Hkv, budget, sms);
+    return align256(static_cast<size_t>(s->B) * s->Hq * nsplit * (s->d + 4) * sizeof(float));
+  }
+  if (op == BSA_OP_GIST_DECODE) return gist_layout(s, budget, sms).total;
+  return 0;
+}
+
+bsa_status_t bsa_score_blocks(const bsa_shape_t* s, int mode, const void* q, const void* k,
+                              const float* pooled_k_in, float* pooled_q_out, float* pooled_k_out, float* scores,
+                              void* stream) {
+  bsa_status_t st = check_shape(s);
+  if (st != BSA_OK) return st;
+  if (q == nullptr || scores == nullptr || !aligned16(q) || !aligned16(scores)) return BSA_ERR_INVALID_ARG;
+  if (s->d % 8 != 0 || s->d > 1024) return BSA_ERR_UNSUPPORTED;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const bool bf16 = s->dtype == BSA_BF16;
+  const int nb = s->Nk / s->block;
+  const int G = s->Hq / s->Hkv;
+  if ((st = device_state(nullptr, nullptr)) != BSA_OK) return st;
+  const float scale = score_scale(s->d);
+  if (mode == BSA_SCORE_PREFILL) {
+    if (s->Nq != s->Nk || k == nullptr || pooled_q_out == nullptr || pooled_k_out == nullptr ||
+        pooled_k_in != nullptr)
+      return BSA_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(pooled_q_out) || !aligned16(pooled_k_out)) return BSA_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(nb) * nb >= (1ll << 31)) return BSA_ERR_UNSUPPORTED;
+    cudaError_t e = launch_pool(k, bf16, s->B, s->Hkv, s->Hkv, 1, s->Nk, s->d, s->block, pooled_k_out, cs);
+    if (e == cudaSuccess)
+      e = launch_pool(q, bf16, s->B, s->Hq, s->Hkv, G, s->Nq, s->d, s->block, pooled_q_out, cs);
+    if (e == cudaSuccess) e = launch_score_prefill(pooled_q_out, pooled_k_out, s->B, s->Hkv, nb, s->d, scale, scores, cs);
+    return cuda_status(e);
+  }
+  if (mode == BSA_SCORE_DECODE) {
+    if (s->Nq != 1) return BSA_ERR_INVALID_ARG;
+    const float* kbar = pooled_k_in;
+    cudaError_t e = cudaSuccess;
+    if (kbar == nullptr) {
+      if (k == nullptr || pooled_k_out == nullptr || !aligned16(k) || !aligned16(pooled_k_out))
+        return BSA_ERR_INVALID_ARG;
+      e = launch_pool(k, bf16, s->B, s->Hkv, s->Hkv, 1, s->Nk, s->d, s->block, pooled_k_out, cs);
+      kbar = pooled_k_out;
+    } else if (!aligned16(kbar)) {
+      return BSA_ERR_INVALID_ARG;
+    }
+    if (e == cudaSuccess)
+      e = launch_score_decode(q, bf16, kbar, s->B, s->Hq, s->Hkv, nb, s->d, scale, scores, pooled_q_out, cs);
+    return cuda_status(e);
+  }
+  if (mode == BSA_SCORE_GIST) {
+    if (s->Nq != 1 || k == nullptr || !aligned16(k) || pooled_k_in || pooled_q_out || pooled_k_out)
+      return BSA_ERR_INVALID_ARG;
+    if (G > 16) return BSA_ERR_UNSUPPORTED;
+    return cuda_status(launch_score_gist(q, k, bf16, s->B, s->Hq, s->Hkv, nb, s->d, scale, scores, cs));
+  }
+  return BSA_ERR_INVALID_ARG;
+}
+
+bsa_status_t bsa_topk_select(const float* scores, int rows, int ncols, int mode, int kb, int* idx_out,
+                             int idx_stride, int* count_out, void* stream) {
+  if (scores == nullptr || idx_out == nullptr || rows < 0 || ncols < 1 || kb < 0) return BSA_ERR_INVALID_ARG;
+  if (mode != BSA_TOPK_CAUSAL_BLOCK && mode != BSA_TOPK_LAST_BLOCK && mode != BSA_TOPK_PLAIN)
+    return BSA_ERR_INVALID_ARG;
+  const int forced = (mode == BSA_TOPK_PLAIN) ? 0 : 1;
+  if (idx_stride < kb + forced || idx_stride < 1) return BSA_ERR_INVALID_ARG;
+  if (ncols > 8192) return BSA_ERR_UNSUPPORTED;
+  if (rows == 0) return BSA_OK;
+  bsa_status_t st = device_state(nullptr, nullptr);
+  if (st != BSA_OK) return st;
+  return cuda_status(launch_topk(scores, rows, ncols, mode, kb, idx_out, idx_stride, count_out,
+                                 static_cast<cudaStream_t>(stream)));
+}
+
+static bsa_status_t prefill_common(const bsa_shape_t* s, const void* q, const void* k, const void* v,
+                                   const int* idx, int idx_stride, const float* sel, float scale, void* o,
+                                   float* lse, void* stream) {
+  bsa_status_t st = check_shape(s);
+  if (st != BSA_OK) return st;
+  if (s->Nq != s->Nk) return BSA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !idx || !o) return BSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return BSA_ERR_INVALID_ARG;
+  if (idx_stride < 1 || !(scale > 0.0f) || !isfinite(scale)) return BSA_ERR_INVALID_ARG;
+  if (idx_stride > 256) return BSA_ERR_UNSUPPORTED;
+  if (s->block != 64 && s->block != 128) return BSA_ERR_UNSUPPORTED;
+  uint32_t* status = nullptr;
+  if ((st = device_state(&status, nullptr)) != BSA_OK) return st;
+  PrefillArgs a;
+  a.B = s->B;
+  a.Hq = s->Hq;
+  a.Hkv = s->Hkv;
+  a.N = s->Nk;
+  a.bs = s->block;
+  a.idx = idx;
+  a.idx_stride = idx_stride;
+  a.sel_scores = sel;
+  a.softmax_scale = scale;
+  a.o = o;
+  a.lse = lse;
+  a.status = status;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (s->dtype == BSA_BF16) {
+    if (s->d != 128) return BSA_ERR_UNSUPPORTED;
+    CUtensorMap mq, mk, mv;
+    if (!make_map_bf16(&mq, q, static_cast<uint64_t>(s->B) * s->Hq * s->Nq, 64) ||
+        !make_map_bf16(&mk, k, static_cast<uint64_t>(s->B) * s->Hkv * s->Nk, 64) ||
+        !make_map_bf16(&mv, v, static_cast<uint64_t>(s->B) * s->Hkv * s->Nk, 64))
+      return BSA_ERR_CUDA;
+    return cuda_status(launch_attn_prefill_bf16(&mq, &mk, &mv, a, cs));
+  }
+  if (s->d != 64 && s->d != 128) return BSA_ERR_UNSUPPORTED;
+  return cuda_status(launch_attn_prefill_f32(static_cast<const float*>(q), static_cast<const float*>(k),
+                                             static_cast<const float*>(v), a, s->d, cs));
+}
+
+bsa_status_t bsa_sparse_attn_prefill(const bsa_shape_t* s, const void* q, const void* k, const void* v,
+                                     const int* idx, int idx_stride, float softmax_scale, void* o, float* lse,
+                                     void* stream) {
+  return prefill_common(s, q, k, v, idx, idx_stride, nullptr, softmax_scale, o, lse, stream);
+}
+
+bsa_status_t bsa_gated_attn_fwd(const bsa_shape_t* s, const void* q, const void* k, const void* v,
+                                const int* idx, int idx_stride, const float* sel_scores, float softmax_scale,
+                                void* o, float* lse, void* stream) {
+  if (sel_scores == nullptr) return BSA_ERR_INVALID_ARG;
+  return prefill_common(s, q, k, v, idx, idx_stride, sel_scores, softmax_scale, o, lse, stream);
+}
+
+static bsa_status_t decode_checks(const bsa_shape_t* s, const void* q, const void* kc, const void* vc, void* o) {
+  bsa_status_t st = check_shape(s);
+  if (st != BSA_OK) return st;
+  if (s->Nq != 1 || !q || !kc || !vc || !o) return BSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kc) || !aligned16(vc) || !aligned16(o)) return BSA_ERR_INVALID_ARG;
+  if (s->dtype != BSA_BF16 || s->d != 128 || s->block != 64) return BSA_ERR_UNSUPPORTED;
+  if (s->Hq / s->Hkv > 32) return BSA_ERR_UNSUPPORTED;
+  return BSA_OK;
+}
+
+bsa_status_t bsa_sparse_attn_decode(const bsa_shape_t* s, const void* q, const void* k_cache, const void* v_cache,
+                                    const int* idx, int idx_stride, float softmax_scale, void* workspace,
+                                    size_t workspace_bytes, void* o, float* lse, void* stream) {
+  bsa_status_t st = decode_checks(s, q, k_cache, v_cache, o);
+  if (st != BSA_OK) return st;
+  if (!idx || idx_stride < 1 || !(softmax_scale > 0.0f) || !workspace) return BSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return BSA_ERR_INVALID_ARG;
+  uint32_t* status = nullptr;
+  int sms = 0;
+  if ((st = device_state(&status, &sms)) != BSA_OK) return st;
+  const int G = s->Hq / s->Hkv;
+  const int nsplit = decode_splits(s->B * s->Hkv, idx_stride, sms);
+  const size_t need = align256(static_cast<size_t>(s->B) * s->Hq * nsplit * (s->d + 4) * sizeof(float));
+  if (workspace_bytes < need) return BSA_ERR_INVALID_ARG;
+  CUtensorMap mq, mk, mv;
+  if (!make_map_bf16(&mq, q, static_cast<uint64_t>(s->B) * s->Hq, static_cast<uint32_t>(G)) ||
+      !make_map_bf16(&mk, k_cache, static_cast<uint64_t>(s->B) * s->Hkv * s->Nk, 64) ||
+      !make_map_bf16(&mv, v_cache, static_cast<uint64_t>(s->B) * s->Hkv * s->Nk, 64))
+    return BSA_ERR_CUDA;
+  DecodeArgs a;
+  a.B = s->B;
+  a.Hq = s->Hq;
+  a.Hkv = s->Hkv;
+  a.Nk = s->Nk;
+  a.bs = s->block;
+  a.list = idx;
+  a.list_stride = idx_stride;
+  a.list_has_count = 0;
+  a.expanded = nullptr;
+  a.nc = 0;
+  a.nsplit = nsplit;
+  a.softmax_scale = softmax_scale;
+  a.partial = static_cast<float*>(workspace);
+  a.status = status;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_attn_decode_bf16(&mq, &mk, &mv, nullptr, nullptr, a, cs);
+  if (e == cudaSuccess) e = launch_decode_combine(a.partial, s->B * s->Hq, nsplit, s->d, true, o, lse, cs);
+  return cuda_status(e);
+}
+
+bsa_status_t bsa_gist_expand_decode(const bsa_shape_t* s, const void* q, const void* k_cache, const void* v_cache,
+                                    const void* gist_k, const void* gist_v, int topk, const int* idx_in,
+                                    int* idx_out, float softmax_scale, void* workspace, size_t workspace_bytes,
+                                    void* o, float* lse, void* stream) {
+  bsa_status_t st = decode_checks(s, q, k_cache, v_cache, o);
+  if (st != BSA_OK) return st;
+  const int nc = s->Nk / s->block;
+  if (!gist_k || !gist_v || !aligned16(gist_k) || !aligned16(gist_v)) return BSA_ERR_INVALID_ARG;
+  if (topk < 0 || topk > nc || !(softmax_scale > 0.0f) || !workspace) return BSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return BSA_ERR_INVALID_ARG;
+  if (nc % 64 != 0 || nc > 8192) return BSA_ERR_UNSUPPORTED;
+  if (s->Hq / s->Hkv > 16) return BSA_ERR_UNSUPPORTED;
+  uint32_t* status = nullptr;
+  int sms = 0;
+  if ((st = device_state(&status, &sms)) != BSA_OK) return st;
+  const GistLayout L = gist_layout(s, topk, sms);
+  if (workspace_bytes < L.total) return BSA_ERR_INVALID_ARG;
+  char* ws = static_cast<char*>(workspace);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const int G = s->Hq / s->Hkv;
+  const int rows = s->B * s->Hq;
+  const int* idx = idx_in;
+  const int idx_stride = topk > 0 ? topk : 1;
+  cudaError_t e = cudaSuccess;
+  if (idx == nullptr) {
+    int* idx_dst = (idx_out && topk > 0) ? idx_out : reinterpret_cast<int*>(ws + L.idx);
+    if (topk > 0) {
+      float* sc = reinterpret_cast<float*>(ws + L.scores);
+      e = launch_score_gist(q, gist_k, true, s->B, s->Hq, s->Hkv, nc, s->d, score_scale(s->d), sc, cs);
+      if (e == cudaSuccess) e = launch_topk(sc, rows, nc, BSA_TOPK_PLAIN, topk, idx_dst, idx_stride, nullptr, cs);
+    } else {
+      e = cudaMemsetAsync(idx_dst, 0xff, static_cast<size_t>(rows) * sizeof(int), cs);
+    }
+    idx = idx_dst;
+  } else if (idx_out != nullptr && topk > 0) {
+    e = cudaMemcpyAsync(idx_out, idx_in, static_cast<size_t>(rows) * topk * sizeof(int), cudaMemcpyDeviceToDevice, cs);
+  }
+  uint32_t* expanded = reinterpret_cast<uint32_t*>(ws + L.expanded);
+  int* ulist = reinterpret_cast<int*>(ws + L.union_list);
+  if (e == cudaSuccess)
+    e = launch_gist_union(idx, s->B, s->Hq, s->Hkv, topk, idx_stride, nc, expanded, ulist, L.union_stride, status, cs);
+  CUtensorMap mq, mk, mv, mgk, mgv;
+  if (!make_map_bf16(&mq, q, static_cast<uint64_t>(rows), static_cast<uint32_t>(G)) ||
+      !make_map_bf16(&mk, k_cache, static_cast<uint64_t>(s->B) * s->Hkv * s->Nk, 64) ||
+      !make_map_bf16(&mv, v_cache, static_cast<uint64_t>(s->B) * s->Hkv * s->Nk, 64) ||
+      !make_map_bf16(&mgk, gist_k, static_cast<uint64_t>(s->B) * s->Hkv * nc, 64) ||
+      !make_map_bf16(&mgv, gist_v, static_cast<uint64_t>(s->B) * s->Hkv * nc, 64))
+    return BSA_ERR_CUDA;
+  DecodeArgs a;
+  a.B = s->B;
+  a.Hq = s->Hq;
+  a.Hkv = s->Hkv;
+  a.Nk = s->Nk;
+  a.bs = s->block;
+  a.list = ulist;
+  a.list_stride = L.union_stride;
+  a.list_has_count = 1;
+  a.expanded = expanded;
+  a.nc = nc;
+  a.nsplit = L.nsplit;
+  a.softmax_scale = softmax_scale;
+  a.partial = reinterpret_cast<float*>(ws + L.partial);
+  a.status = status;
+  if (e == cudaSuccess) e = launch_attn_decode_bf16(&mq, &mk, &mv, &mgk, &mgv, a, cs);
+  if (e == cudaSuccess) e = launch_decode_combine(a.partial, rows, L.nsplit, s->d, true, o, lse, cs);
+  return cuda_status(e);
+}
+
+}  // extern "C"

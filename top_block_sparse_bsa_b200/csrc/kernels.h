@@ -1,0 +1,64 @@
+// kernels.h -- internal launchers of libbsa (C++ linkage, not part of the ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace bsa {
+
+// selector.cu
+cudaError_t launch_pool(const void* src, bool bf16, int B, int Hsrc, int Hgroups, int heads_sum, int N,
+                        int d, int bs, float* out, cudaStream_t st);
+cudaError_t launch_score_prefill(const float* qbar, const float* kbar, int B, int Hkv, int nb, int d,
+                                 float scale, float* s, cudaStream_t st);
+cudaError_t launch_score_decode(const void* q, bool bf16, const float* kbar, int B, int Hq, int Hkv,
+                                int nb, int d, float scale, float* s, float* qbar_out, cudaStream_t st);
+cudaError_t launch_score_gist(const void* q, const void* gk, bool bf16, int B, int Hq, int Hkv, int nc,
+                              int d, float scale, float* s, cudaStream_t st);
+cudaError_t launch_topk(const float* scores, int rows, int ncols, int mode, int kb, int* idx_out,
+                        int idx_stride, int* count_out, cudaStream_t st);
+
+// attn_prefill.cu (bf16, d = 128, tcgen05)
+struct PrefillArgs {
+  int B, Hq, Hkv, N, bs;
+  const int* idx;
+  int idx_stride;
+  const float* sel_scores;   // non-null: gated (SAS log-gate)
+  float softmax_scale;
+  void* o;
+  float* lse;
+  uint32_t* status;
+};
+cudaError_t launch_attn_prefill_bf16(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
+                                     const PrefillArgs& a, cudaStream_t st);
+
+// attn_f32.cu (fp32 SIMT path)
+cudaError_t launch_attn_prefill_f32(const float* q, const float* k, const float* v, const PrefillArgs& a,
+                                    int d, cudaStream_t st);
+
+// attn_decode.cu (bf16, d = 128, tcgen05, split-K + combine)
+struct DecodeArgs {
+  int B, Hq, Hkv, Nk, bs;
+  // tile list: plain decode reads idx [B*Hkv][list_stride]; gist decode reads
+  // the union list built in the workspace (count at [bg][0], entries after).
+  const int* list;
+  int list_stride;
+  int list_has_count;        // 1: entry 0 is the count (gist union list)
+  const uint32_t* expanded;  // gist: [B*Hq][nc/32] bitmap of expanded chunks; null for plain decode
+  int nc;                    // gist: number of chunks
+  int nsplit;
+  float softmax_scale;
+  float* partial;            // [B*Hq][nsplit][d+2]
+  uint32_t* status;
+};
+cudaError_t launch_attn_decode_bf16(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
+                                    const CUtensorMap* tmGK, const CUtensorMap* tmGV, const DecodeArgs& a,
+                                    cudaStream_t st);
+cudaError_t launch_decode_combine(const float* partial, int rows, int nsplit, int d, bool out_bf16, void* o,
+                                  float* lse, cudaStream_t st);
+cudaError_t launch_gist_union(const int* idx, int B, int Hq, int Hkv, int topk, int idx_stride, int nc,
+                              uint32_t* expanded, int* union_list, int union_stride, uint32_t* status,
+                              cudaStream_t st);
+
+}  // namespace bsa

@@ -1,0 +1,380 @@
+// selector.cu -- the cheap selector of query-aware block-sparse attention:
+// block pooling, block / gist scoring and hard top-k selection.
+//
+// Sources: "稀疏注意力" tutorial §4.5 (a block is a run of consecutive tokens)
+// and §4.6 (coarse block scoring avoids the full QK^T); SAS page, 核心模块 1
+// (a continuous score per context unit) and 推理 paragraph (each query keeps
+// its k best units, the current block always kept); SSA page, 推理时的关键模块
+// 1-2 (score the query against every gist, expand the top-k chunks, each
+// query head choosing its own chunks under GQA).
+//
+// Arithmetic contract (kept identical on purpose to the plain definition, so
+// selected indices are reproducible bit for bit): pooled means are fp32 sums
+// in a fixed order (heads ascending, then tokens ascending) followed by one
+// IEEE division; a score is an fp32 dot product over the channel index
+// ascending with each product and each sum rounded separately (no FMA),
+// then one multiply by fp32(1/sqrt(d)).  These kernels are bandwidth-bound,
+// so the sequential order costs nothing that matters.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace bsa {
+
+// ------------------------------------------------------------------ pooling
+// One group of 8 channels per thread, 16-byte loads along d, every thread
+// summing its channels over the unit's rows in order.
+template <typename T>
+struct Vec8;
+template <>
+struct Vec8<__nv_bfloat16> {
+  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&x)[8]) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      x[2 * i] = __uint_as_float(w[i] << 16);
+      x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+};
+template <>
+struct Vec8<float> {
+  static __device__ __forceinline__ void load(const float* p, float (&x)[8]) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  }
+};
+
+// unit u = (b, g, j): rows base + hh*N + t for hh < heads_sum, t < bs,
+// base = ((b*Hsrc + g*heads_sum)*N + j*bs).  out[u][c] = sum / (heads_sum*bs).
+template <typename T>
+__global__ void pool_kernel(const T* __restrict__ src, int B, int Hsrc, int Hgroups, int heads_sum,
+                            int N, int d, int bs, float* __restrict__ out) {
+  const int lanes_per_unit = d / 8;
+  const int64_t gtid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t unit = gtid / lanes_per_unit;
+  const int cg = static_cast<int>(gtid % lanes_per_unit);
+  const int nb = N / bs;
+  const int64_t units = static_cast<int64_t>(B) * Hgroups * nb;
+  if (unit >= units) return;
+  const int64_t b = unit / (static_cast<int64_t>(Hgroups) * nb);
+  const int64_t g = (unit / nb) % Hgroups;
+  const int64_t j = unit % nb;
+  const int64_t base = ((b * Hsrc + g * heads_sum) * N + j * bs) * d + cg * 8;
+  float acc[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) acc[c] = 0.0f;
+  for (int hh = 0; hh < heads_sum; ++hh) {
+    const T* p = src + base + static_cast<int64_t>(hh) * N * d;
+#pragma unroll 8
+    for (int t = 0; t < bs; ++t) {
+      float x[8];
+      Vec8<T>::load(p + static_cast<int64_t>(t) * d, x);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[c] = __fadd_rn(acc[c], x[c]);
+    }
+  }
+  const float div = static_cast<float>(heads_sum * bs);
+  float* o = out + unit * d + cg * 8;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) o[c] = __fdiv_rn(acc[c], div);
+}
+
+template <typename T>
+static cudaError_t launch_pool_t(const void* src, int B, int Hsrc, int Hgroups, int heads_sum, int N,
+                                 int d, int bs, float* out, cudaStream_t st) {
+  const int64_t threads = static_cast<int64_t>(B) * Hgroups * (N / bs) * (d / 8);
+  const int tpb = 256;
+  const int64_t blocks = (threads + tpb - 1) / tpb;
+  pool_kernel<T><<<static_cast<unsigned>(blocks), tpb, 0, st>>>(
+      static_cast<const T*>(src), B, Hsrc, Hgroups, heads_sum, N, d, bs, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pool(const void* src, bool bf16, int B, int Hsrc, int Hgroups, int heads_sum, int N,
+                        int d, int bs, float* out, cudaStream_t st) {
+  return bf16 ? launch_pool_t<__nv_bfloat16>(src, B, Hsrc, Hgroups, heads_sum, N, d, bs, out, st)
+              : launch_pool_t<float>(src, B, Hsrc, Hgroups, heads_sum, N, d, bs, out, st);
+}
+
+// ------------------------------------------------------------------ scores
+__device__ __forceinline__ float dot_fixed_order(const float* a, const float* b, int d, int bstride) {
+  float acc = 0.0f;
+  for (int c = 0; c < d; ++c) acc = __fadd_rn(acc, __fmul_rn(a[c], b[c * bstride]));
+  return acc;
+}
+
+// Prefill: one 32x32 (i, j) tile per CTA; rows of qbar/kbar staged in shared
+// memory (row pitch d+1 floats: no bank conflicts along j).
+__global__ void score_prefill_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
+                                     int nb, int d, float scale, float* __restrict__ s) {
+  extern __shared__ float sm[];
+  const int pitch = d + 1;
+  float* qs = sm;
+  float* ks = sm + 32 * pitch;
+  const int ti = blockIdx.y, tj = blockIdx.x;
+  const int64_t bg = blockIdx.z;
+  const int tx = threadIdx.x, ty = threadIdx.y;   // 32 x 8
+  const int i0 = ti * 32, j0 = tj * 32;
+  float* srow = s + bg * nb * static_cast<int64_t>(nb);
+  if (j0 > i0 + 31) {   // tile entirely above the diagonal
+    for (int r = ty; r < 32; r += 8) {
+      const int i = i0 + r, j = j0 + tx;
+      if (i < nb && j < nb) srow[static_cast<int64_t>(i) * nb + j] = -INFINITY;
+    }
+    return;
+  }
+  for (int r = ty; r < 32; r += 8) {
+    for (int c = tx; c < d; c += 32) {
+      const int i = i0 + r, j = j0 + r;
+      qs[r * pitch + c] = (i < nb) ? qbar[(bg * nb + i) * d + c] : 0.0f;
+      ks[r * pitch + c] = (j < nb) ? kbar[(bg * nb + j) * d + c] : 0.0f;
+    }
+  }
+  __syncthreads();
+  for (int r = ty; r < 32; r += 8) {
+    const int i = i0 + r, j = j0 + tx;
+    if (i >= nb || j >= nb) continue;
+    float v = -INFINITY;
+    if (j <= i) v = __fmul_rn(dot_fixed_order(qs + r * pitch, ks + tx * pitch, d, 1), scale);
+    srow[static_cast<int64_t>(i) * nb + j] = v;
+  }
+}
+
+cudaError_t launch_score_prefill(const float* qbar, const float* kbar, int B, int Hkv, int nb, int d,
+                                 float scale, float* s, cudaStream_t st) {
+  dim3 grid((nb + 31) / 32, (nb + 31) / 32, B * Hkv);
+  dim3 block(32, 8);
+  const size_t smem = 2 * 32 * (d + 1) * sizeof(float);
+  score_prefill_kernel<<<grid, block, smem, st>>>(qbar, kbar, nb, d, scale, s);
+  return cudaGetLastError();
+}
+
+// Decode: grid (tiles of 64 blocks, B*Hkv).  The group query mean is formed
+// in fixed order (heads ascending) by every CTA.
+template <typename T>
+__global__ void score_decode_kernel(const T* __restrict__ q, const float* __restrict__ kbar, int Hq,
+                                    int Hkv, int nb, int d, float scale, float* __restrict__ s,
+                                    float* __restrict__ qbar_out) {
+  extern __shared__ float sm[];
+  const int pitch = d + 1;
+  float* qm = sm;              // [d]
+  float* ks = sm + d;          // [64][pitch]
+  const int64_t bg = blockIdx.y;
+  const int64_t b = bg / Hkv, g = bg % Hkv;
+  const int G = Hq / Hkv;
+  const int j0 = blockIdx.x * 64;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    float acc = 0.0f;
+    for (int hh = 0; hh < G; ++hh) {
+      const T* qp = q + ((b * Hq + g * G + hh) * d + c);
+      acc = __fadd_rn(acc, static_cast<float>(*qp));
+    }
+    const float m = __fdiv_rn(acc, static_cast<float>(G));
+    qm[c] = m;
+    if (qbar_out && blockIdx.x == 0) qbar_out[bg * d + c] = m;
+  }
+  const int rows = min(64, nb - j0);
+  for (int e = threadIdx.x; e < rows * d; e += blockDim.x) {
+    const int r = e / d, c = e % d;
+    ks[r * pitch + c] = kbar[(bg * nb + j0 + r) * d + c];
+  }
+  __syncthreads();
+  const int r = threadIdx.x;
+  if (r < rows) s[bg * nb + j0 + r] = __fmul_rn(dot_fixed_order(qm, ks + r * pitch, d, 1), scale);
+}
+
+cudaError_t launch_score_decode(const void* q, bool bf16, const float* kbar, int B, int Hq, int Hkv,
+                                int nb, int d, float scale, float* s, float* qbar_out,
+                                cudaStream_t st) {
+  dim3 grid((nb + 63) / 64, B * Hkv);
+  const size_t smem = (d + 64 * (d + 1)) * sizeof(float);
+  if (bf16)
+    score_decode_kernel<__nv_bfloat16><<<grid, 64, smem, st>>>(
+        static_cast<const __nv_bfloat16*>(q), kbar, Hq, Hkv, nb, d, scale, s, qbar_out);
+  else
+    score_decode_kernel<float><<<grid, 64, smem, st>>>(static_cast<const float*>(q), kbar, Hq, Hkv,
+                                                       nb, d, scale, s, qbar_out);
+  return cudaGetLastError();
+}
+
+// Gist: grid (tiles of 64 gists, B*Hkv); threads (64 gists) x G heads.
+template <typename T>
+__global__ void score_gist_kernel(const T* __restrict__ q, const T* __restrict__ gk, int Hq, int Hkv,
+                                  int nc, int d, float scale, float* __restrict__ s) {
+  extern __shared__ float sm[];
+  const int pitch = d + 1;
+  const int G = Hq / Hkv;
+  float* qs = sm;                 // [G][d]
+  float* ks = sm + G * d;         // [64][pitch]
+  const int64_t bg = blockIdx.y;
+  const int64_t b = bg / Hkv, g = bg % Hkv;
+  const int c0 = blockIdx.x * 64;
+  const int rows = min(64, nc - c0);
+  for (int e = threadIdx.x; e < G * d; e += blockDim.x)
+    qs[e] = static_cast<float>(q[(b * Hq + g * G) * d + e]);
+  for (int e = threadIdx.x; e < rows * d; e += blockDim.x) {
+    const int r = e / d, c = e % d;
+    ks[r * pitch + c] = static_cast<float>(gk[(bg * nc + c0 + r) * d + c]);
+  }
+  __syncthreads();
+  const int hh = threadIdx.x / 64, r = threadIdx.x % 64;
+  if (hh < G && r < rows)
+    s[((b * Hq + g * G + hh) * nc) + c0 + r] =
+        __fmul_rn(dot_fixed_order(qs + hh * d, ks + r * pitch, d, 1), scale);
+}
+
+cudaError_t launch_score_gist(const void* q, const void* gk, bool bf16, int B, int Hq, int Hkv, int nc,
+                              int d, float scale, float* s, cudaStream_t st) {
+  const int G = Hq / Hkv;
+  dim3 grid((nc + 63) / 64, B * Hkv);
+  const size_t smem = (G * d + 64 * (d + 1)) * sizeof(float);
+  if (bf16)
+    score_gist_kernel<__nv_bfloat16><<<grid, 64 * G, smem, st>>>(
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(gk), Hq, Hkv, nc, d,
+        scale, s);
+  else
+    score_gist_kernel<float><<<grid, 64 * G, smem, st>>>(static_cast<const float*>(q),
+                                                         static_cast<const float*>(gk), Hq, Hkv, nc,
+                                                         d, scale, s);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ top-k
+// Monotone unsigned key of an fp32 score: a larger score gives a larger key,
+// -0 and +0 share one key, and every NaN gets key 0 (below -inf).
+__device__ __forceinline__ uint32_t order_key(float f) {
+  if (f != f) return 0u;
+  uint32_t u = __float_as_uint(f);
+  if (f == 0.0f) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// One CTA per row.  Radix select (4 passes of 8 bits, most significant
+// first) finds the key T of the k-th best candidate and how many candidates
+// equal to T must be taken; warp 0 then walks the candidates in index order,
+// taking every key > T and the lowest-index ties, which writes the kept list
+// already ascending.  The forced block (current / last) is larger than every
+// candidate, so it is appended at the end.
+constexpr int kTopkThreads = 256;
+
+__global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restrict__ scores, int ncols,
+                                                            int mode, int kb, int* __restrict__ idx_out,
+                                                            int idx_stride, int* __restrict__ count_out) {
+  extern __shared__ uint32_t skeys[];
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t s_digit;
+  __shared__ int s_remaining;
+  const int64_t r = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int ncand, forced;
+  if (mode == 0) {
+    ncand = static_cast<int>(r % ncols);
+    forced = ncand;
+  } else if (mode == 1) {
+    ncand = ncols - 1;
+    forced = ncols - 1;
+  } else {
+    ncand = ncols;
+    forced = -1;
+  }
+  const float* srow = scores + r * ncols;
+  for (int j = tid; j < ncand; j += kTopkThreads) skeys[j] = order_key(srow[j]);
+  const int take = min(kb, ncand);
+  const bool take_all = (take == ncand);
+  uint32_t thresh = 0;
+  int remaining = take;
+  __syncthreads();
+  if (!take_all && take > 0) {
+    uint32_t prefix = 0, pmask = 0;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int i = tid; i < 256; i += kTopkThreads) hist[i] = 0;
+      __syncthreads();
+      for (int j = tid; j < ncand; j += kTopkThreads) {
+        const uint32_t k = skeys[j];
+        if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+      }
+      __syncthreads();
+      if (warp == 0) {
+        // lane l owns digits 255-8l down to 248-8l (descending)
+        uint32_t cnt[8];
+        uint32_t mine = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          cnt[e] = hist[255 - 8 * lane - e];
+          mine += cnt[e];
+        }
+        uint32_t incl = mine;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += v;
+        }
+        const uint32_t excl = incl - mine;
+        const unsigned hit = __ballot_sync(0xffffffffu, incl >= static_cast<uint32_t>(remaining));
+        const int first = __ffs(hit) - 1;   // always found: total >= remaining
+        if (lane == first) {
+          uint32_t cum = excl;
+          for (int e = 0; e < 8; ++e) {
+            if (cum + cnt[e] >= static_cast<uint32_t>(remaining)) {
+              s_digit = 255 - 8 * lane - e;
+              s_remaining = remaining - static_cast<int>(cum);
+              break;
+            }
+            cum += cnt[e];
+          }
+        }
+      }
+      __syncthreads();
+      remaining = s_remaining;
+      prefix |= s_digit << shift;
+      pmask |= 255u << shift;
+      __syncthreads();
+    }
+    thresh = prefix;
+  }
+  if (warp != 0) return;
+  int* out = idx_out + r * idx_stride;
+  int run_sel = 0, run_tie = 0;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int base = 0; base < ncand; base += 32) {
+    const int j = base + lane;
+    const bool valid = j < ncand;
+    const uint32_t k = valid ? skeys[j] : 0u;
+    bool gt, tie;
+    if (take_all) {
+      gt = valid;
+      tie = false;
+    } else if (take == 0) {
+      gt = false;
+      tie = false;
+    } else {
+      gt = valid && k > thresh;
+      tie = valid && k == thresh;
+    }
+    const unsigned tb = __ballot_sync(0xffffffffu, tie);
+    const int tie_rank = run_tie + __popc(tb & lt_mask);
+    const bool sel = gt || (tie && tie_rank < remaining);
+    const unsigned sb = __ballot_sync(0xffffffffu, sel);
+    if (sel) out[run_sel + __popc(sb & lt_mask)] = j;
+    run_sel += __popc(sb);
+    run_tie += __popc(tb);
+  }
+  if (forced >= 0) {
+    if (lane == 0) out[run_sel] = forced;
+    ++run_sel;
+  }
+  for (int t = run_sel + lane; t < idx_stride; t += 32) out[t] = -1;
+  if (count_out && lane == 0) count_out[r] = run_sel;
+}
+
+cudaError_t launch_topk(const float* scores, int rows, int ncols, int mode, int kb, int* idx_out,
+                        int idx_stride, int* count_out, cudaStream_t st) {
+  const size_t smem = static_cast<size_t>(ncols) * sizeof(uint32_t);
+  topk_kernel<<<rows, kTopkThreads, smem, st>>>(scores, ncols, mode, kb, idx_out, idx_stride, count_out);
+  return cudaGetLastError();
+}
+
+}  // namespace bsa

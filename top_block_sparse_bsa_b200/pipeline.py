@@ -1,0 +1,180 @@
+"""Whole steps of the hot path, composed from the C entry points.
+
+A step is the pages' sequence -- score the blocks, keep the top-k (with the
+current / last block), attend over the kept blocks -- issued as consecutive
+library calls on one stream.  Buffers are allocated once (torch is only the
+device-memory provider here) and reused, so a step launches kernels and
+nothing else.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+from typing import Dict, Optional
+
+import torch
+
+from . import (BSA_OP_DECODE, BSA_OP_GIST_DECODE, BSA_SCORE_DECODE, BSA_SCORE_PREFILL,
+               BSA_TOPK_CAUSAL_BLOCK, BSA_TOPK_LAST_BLOCK, bsa_gated_attn_fwd, bsa_gist_expand_decode,
+               bsa_score_blocks, bsa_sparse_attn_decode, bsa_sparse_attn_prefill, bsa_topk_select,
+               bsa_workspace_bytes, make_shape)
+
+
+def _dev(t: torch.Tensor):
+    return t.device
+
+
+@dataclass
+class PrefillStep:
+    """pool+score -> top-k -> sparse (or gated) attention for q [B,Hq,N,d], k/v [B,Hkv,N,d]."""
+    q: torch.Tensor
+    k: torch.Tensor
+    v: torch.Tensor
+    block: int
+    kb: int
+    gated: bool = False
+    softmax_scale: Optional[float] = None
+    bufs: Dict[str, torch.Tensor] = field(default_factory=dict)
+
+    def __post_init__(self):
+        B, Hq, N, d = self.q.shape
+        Hkv = self.k.shape[1]
+        nb = N // self.block
+        self.shape = make_shape(B, Hq, Hkv, N, N, d, self.block, self.q.dtype)
+        self.nb = nb
+        self.idx_stride = self.kb + 1
+        if self.softmax_scale is None:
+            self.softmax_scale = 1.0 / math.sqrt(d)
+        dev = _dev(self.q)
+        f32 = torch.float32
+        b = self.bufs
+        b.setdefault("qbar", torch.empty((B, Hkv, nb, d), dtype=f32, device=dev))
+        b.setdefault("kbar", torch.empty((B, Hkv, nb, d), dtype=f32, device=dev))
+        b.setdefault("scores", torch.empty((B, Hkv, nb, nb), dtype=f32, device=dev))
+        b.setdefault("idx", torch.empty((B, Hkv, nb, self.idx_stride), dtype=torch.int32, device=dev))
+        b.setdefault("count", torch.empty((B, Hkv, nb), dtype=torch.int32, device=dev))
+        b.setdefault("o", torch.empty_like(self.q))
+        b.setdefault("lse", torch.empty((B, Hq, N), dtype=f32, device=dev))
+
+    def select(self, stream=None):
+        b = self.bufs
+        bsa_score_blocks(self.shape, BSA_SCORE_PREFILL, self.q, self.k, None, b["qbar"], b["kbar"],
+                         b["scores"], stream=stream)
+        rows = self.shape.B * self.shape.Hkv * self.nb
+        bsa_topk_select(b["scores"], rows, self.nb, BSA_TOPK_CAUSAL_BLOCK, self.kb, b["idx"], self.idx_stride,
+                        b["count"], stream=stream)
+
+    def attend(self, idx: Optional[torch.Tensor] = None, stream=None, with_lse: bool = True):
+        b = self.bufs
+        idx = b["idx"] if idx is None else idx
+        lse = b["lse"] if with_lse else None
+        if self.gated:
+            bsa_gated_attn_fwd(self.shape, self.q, self.k, self.v, idx, idx.shape[-1], b["scores"],
+                               self.softmax_scale, b["o"], lse, stream=stream)
+        else:
+            bsa_sparse_attn_prefill(self.shape, self.q, self.k, self.v, idx, idx.shape[-1], self.softmax_scale,
+                                    b["o"], lse, stream=stream)
+
+    def run(self, stream=None, with_lse: bool = True):
+        self.select(stream)
+        self.attend(stream=stream, with_lse=with_lse)
+        return self.bufs
+
+
+@dataclass
+class DecodeStep:
+    """score (against the resident pooled-key summary) -> top-k -> split-K sparse decode.
+
+    q [B,Hq,d]; k_cache/v_cache [B,Hkv,Nk,d]; kbar [B,Hkv,nb,d] fp32 is the
+    block-mean summary kept next to the cache (built once by ``pool_cache``).
+    """
+    q: torch.Tensor
+    k_cache: torch.Tensor
+    v_cache: torch.Tensor
+    block: int
+    kb: int
+    softmax_scale: Optional[float] = None
+    bufs: Dict[str, torch.Tensor] = field(default_factory=dict)
+
+    def __post_init__(self):
+        B, Hq, d = self.q.shape
+        Hkv, Nk = self.k_cache.shape[1], self.k_cache.shape[2]
+        nb = Nk // self.block
+        self.nb = nb
+        self.shape = make_shape(B, Hq, Hkv, 1, Nk, d, self.block, self.q.dtype)
+        self.idx_stride = self.kb + 1
+        if self.softmax_scale is None:
+            self.softmax_scale = 1.0 / math.sqrt(d)
+        dev = _dev(self.q)
+        f32 = torch.float32
+        b = self.bufs
+        b.setdefault("kbar", torch.empty((B, Hkv, nb, d), dtype=f32, device=dev))
+        b.setdefault("qbar", torch.empty((B, Hkv, d), dtype=f32, device=dev))
+        b.setdefault("scores", torch.empty((B, Hkv, nb), dtype=f32, device=dev))
+        b.setdefault("idx", torch.empty((B, Hkv, self.idx_stride), dtype=torch.int32, device=dev))
+        b.setdefault("count", torch.empty((B, Hkv), dtype=torch.int32, device=dev))
+        ws = bsa_workspace_bytes(BSA_OP_DECODE, self.shape, self.idx_stride)
+        b.setdefault("workspace", torch.empty((max(ws, 256),), dtype=torch.uint8, device=dev))
+        b.setdefault("o", torch.empty_like(self.q))
+        b.setdefault("lse", torch.empty((B, Hq), dtype=f32, device=dev))
+
+    def pool_cache(self, stream=None):
+        """Build the pooled-key summary from the cache (off the per-step path)."""
+        b = self.bufs
+        bsa_score_blocks(self.shape, BSA_SCORE_DECODE, self.q, self.k_cache, None, b["qbar"], b["kbar"],
+                         b["scores"], stream=stream)
+
+    def select(self, stream=None):
+        b = self.bufs
+        bsa_score_blocks(self.shape, BSA_SCORE_DECODE, self.q, None, b["kbar"], b["qbar"], None, b["scores"],
+                         stream=stream)
+        rows = self.shape.B * self.shape.Hkv
+        bsa_topk_select(b["scores"], rows, self.nb, BSA_TOPK_LAST_BLOCK, self.kb, b["idx"], self.idx_stride,
+                        b["count"], stream=stream)
+
+    def attend(self, idx: Optional[torch.Tensor] = None, stream=None, with_lse: bool = True):
+        b = self.bufs
+        idx = b["idx"] if idx is None else idx
+        bsa_sparse_attn_decode(self.shape, self.q, self.k_cache, self.v_cache, idx, idx.shape[-1],
+                               self.softmax_scale, b["workspace"], b["o"], b["lse"] if with_lse else None,
+                               stream=stream)
+
+    def run(self, stream=None, with_lse: bool = True):
+        self.select(stream)
+        self.attend(stream=stream, with_lse=with_lse)
+        return self.bufs
+
+
+@dataclass
+class GistStep:
+    """SSA decode: gist scores -> per-head top-k chunks -> mixed attention (one C call)."""
+    q: torch.Tensor
+    k_cache: torch.Tensor
+    v_cache: torch.Tensor
+    gist_k: torch.Tensor
+    gist_v: torch.Tensor
+    chunk: int
+    topk: int
+    softmax_scale: Optional[float] = None
+    bufs: Dict[str, torch.Tensor] = field(default_factory=dict)
+
+    def __post_init__(self):
+        B, Hq, d = self.q.shape
+        Hkv, Nk = self.k_cache.shape[1], self.k_cache.shape[2]
+        self.shape = make_shape(B, Hq, Hkv, 1, Nk, d, self.chunk, self.q.dtype)
+        if self.softmax_scale is None:
+            self.softmax_scale = 1.0 / math.sqrt(d)
+        dev = _dev(self.q)
+        b = self.bufs
+        ws = bsa_workspace_bytes(BSA_OP_GIST_DECODE, self.shape, self.topk)
+        b.setdefault("workspace", torch.empty((max(ws, 256),), dtype=torch.uint8, device=dev))
+        b.setdefault("idx", torch.empty((B, Hq, max(self.topk, 1)), dtype=torch.int32, device=dev))
+        b.setdefault("o", torch.empty_like(self.q))
+        b.setdefault("lse", torch.empty((B, Hq), dtype=torch.float32, device=dev))
+
+    def run(self, idx_in: Optional[torch.Tensor] = None, stream=None, with_lse: bool = True):
+        b = self.bufs
+        bsa_gist_expand_decode(self.shape, self.q, self.k_cache, self.v_cache, self.gist_k, self.gist_v,
+                               self.topk, idx_in, b["idx"] if self.topk > 0 else None, self.softmax_scale,
+                               b["workspace"], b["o"], b["lse"] if with_lse else None, stream=stream)
+        return b
