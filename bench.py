@@ -47,11 +47,12 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="prefill_gqa_bf16")
-    ap.add_argument("--cpu-rows", type=int, default=8192, help="query rows in the oracle CPU-baseline sample")
+    ap.add_argument("--cpu-rows", type=int, default=65536, help="query rows in the oracle CPU-baseline sample")
     ap.add_argument("--ref-rows", type=int, default=1024, help="query rows per reference-arm step")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-secondary", action="store_true", help="skip the decode secondary figures")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=0, help="override the workload batch (small profiling cases)")
     return ap.parse_args()
 
 
@@ -247,6 +248,8 @@ def run_prefill(args, world, rank, local, peaks, peak_src):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     base = W.get(args.config)
+    if args.batch:
+        base = base.scaled(B=args.batch, name=base.name)
     w = base.scaled(seed=base.seed + 1000 * rank, name=base.name) if rank else base
     inp = W.make_inputs(w, dev)
     q, k, v = inp["q"], inp["k"], inp["v"]
@@ -417,12 +420,75 @@ def run_decode_secondary(dev, peaks, iters: int = 20):
             "roofline_us": kv_bytes / (peaks["hbm_gbs"] * 1e9) * 1e6, "l2": "flushed (256 MiB write) per iteration"}
 
 
+def run_decode_like(args, world, rank, local, peaks, peak_src):
+    """Decode or gist-decode workload: microseconds per step, HBM GB/s over
+    the bytes the attention must read, L2 flushed before every step."""
+    import torch
+    import bsa_workloads as W
+    from top_block_sparse_bsa_b200 import accounting as acc
+    from top_block_sparse_bsa_b200 import pipeline
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = W.get(args.config)
+    if args.batch:
+        w = w.scaled(B=args.batch, name=w.name)
+    inp = W.make_inputs(w, dev)
+    if w.kind == "decode":
+        step = pipeline.DecodeStep(inp["q"], inp["k"], inp["v"], w.bs, w.kb)
+        step.pool_cache()
+        run = lambda: step.run(with_lse=False)   # noqa: E731
+        launches = 5
+    else:
+        step = pipeline.GistStep(inp["q"], inp["k"], inp["v"], inp["gk"], inp["gv"], w.bs, w.kb)
+        run = lambda: step.run(with_lse=False)   # noqa: E731
+        launches = 5
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        run()
+    torch.cuda.synchronize()
+    idx = step.bufs["idx"].cpu().numpy()
+    if w.kind == "decode":
+        nbytes = acc.decode_kv_bytes(idx, w.bs, w.d, 2)
+    else:
+        nbytes = acc.gist_kv_bytes(idx, w.G, w.bs, w.N // w.bs, w.d, 2)
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler(local).start()
+    t0 = time.time()
+    for s in range(args.steps):
+        flush.fill_(s & 0xFF)
+        ev[s][0].record(stream)
+        run()
+        ev[s][1].record(stream)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    sampler.stop()
+    us = statistics.mean(1e3 * a.elapsed_time(b) for a, b in ev)
+    gbs = nbytes / (us / 1e6) / 1e9
+    line = {
+        "metric": "us per decode step", "value": us, "unit": "us", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": us / 1e3, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "ctx": w.N, "block": w.bs,
+                   "budget": w.kb, "l2": "flushed (256 MiB write) before every step, outside the events"},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm_gbs"], "traffic": None, "peak_source": peak_src,
+                     "bytes_per_step": nbytes, "note": "whole step (score + top-k + attention + combine)"},
+        "clocks": sampler.summary(t0, t1), "gpu_launches": launches * args.steps,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     world, rank, local = dist_setup(args)
     if args.impl == "reference":
         return run_reference(args, world, rank)
     peaks, src = load_peaks()
+    import bsa_workloads as W
+    if W.get(args.config).kind in ("decode", "gist"):
+        return run_decode_like(args, world, rank, local, peaks, src)
     return run_prefill(args, world, rank, local, peaks, src)
 
 
