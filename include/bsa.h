@@ -201,6 +201,28 @@ bsa_status_t bsa_gist_expand_decode(const bsa_shape_t* shape, const void* q, con
                                     float softmax_scale, void* workspace, size_t workspace_bytes,
                                     void* o, float* lse, void* stream);
 
+/*
+ * bsa_sparse_attn_decode_noalloc -- bsa_sparse_attn_decode for callers that
+ * cannot allocate device memory (no counterpart on the source pages; it is a
+ * deployment convenience).  Some callers have no way to provide the decode
+ * scratch buffer: a server that reserves all its device memory at start-up
+ * and allocates nothing afterwards, or a plugin whose host framework owns
+ * every device buffer.  This call takes no workspace; it uses a fixed
+ * 4 MiB array built into the library, held on every GPU that loads the
+ * library until the process exits.
+ * Arguments, layouts and results are those of bsa_sparse_attn_decode.
+ * Returns BSA_ERR_UNSUPPORTED, before launching anything, when the shape
+ * needs more than 4 MiB of scratch (bsa_workspace_bytes(BSA_OP_DECODE, ...)).
+ * The first call on a device looks up the array's device address; make that
+ * first call before any stream capture.  All calls on a device share the
+ * array: calls whose work may overlap on the GPU (unordered streams) race.
+ * Nothing in the array needs to start zeroed between calls.
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ */
+bsa_status_t bsa_sparse_attn_decode_noalloc(const bsa_shape_t* shape, const void* q, const void* k_cache,
+                                            const void* v_cache, const int* idx, int idx_stride,
+                                            float softmax_scale, void* o, float* lse, void* stream);
+
 /* Scratch bytes a decode call needs (op = BSA_OP_*; budget = idx_stride for
  * BSA_OP_DECODE, topk for BSA_OP_GIST_DECODE).  0 on a bad shape. */
 size_t bsa_workspace_bytes(int op, const bsa_shape_t* shape, int budget);

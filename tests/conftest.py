@@ -10,6 +10,14 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) GPU and the built CUDA library")
+    # (re)build libbsa.so and the oracle if their sources are newer; loaded by
+    # path because importing the package loads the library
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_bsa_build", os.path.join(ROOT, "top_block_sparse_bsa_b200", "_build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
 
 
 def pytest_collection_modifyitems(config, items):

@@ -19,9 +19,7 @@ def _declared():
 
 @pytest.fixture(scope="module")
 def bsa():
-    from top_block_sparse_bsa_b200 import _build
-    _build.build()
-    import top_block_sparse_bsa_b200 as m
+    import top_block_sparse_bsa_b200 as m   # conftest has built libbsa.so
     return m
 
 

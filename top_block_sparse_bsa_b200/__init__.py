@@ -5,7 +5,7 @@ Argument marshalling only: every function here forwards torch tensors'
 device pointers and the current CUDA stream to the C entry point of the same
 name declared in ``include/bsa.h``; all computation runs in the library's
 CUDA kernels.  There is no CPU fallback: importing the package fails if
-``libbsa.so`` has not been built (``python -m top_block_sparse_bsa_b200._build``).
+``libbsa.so`` has not been built (``python top_block_sparse_bsa_b200/_build.py``).
 """
 from __future__ import annotations
 
@@ -24,7 +24,7 @@ __all__ = [
     "make_shape", "bsa_score_blocks", "bsa_topk_select", "bsa_sparse_attn_prefill",
     "bsa_gated_attn_fwd", "bsa_sparse_attn_decode", "bsa_gist_expand_decode",
     "bsa_workspace_bytes", "bsa_status_string", "bsa_device_status", "bsa_version",
-    "EXPORTED_SYMBOLS",
+    "bsa_sparse_attn_decode_noalloc", "EXPORTED_SYMBOLS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libbsa.so")
@@ -39,7 +39,7 @@ BSA_OP_DECODE, BSA_OP_GIST_DECODE = 0, 1
 EXPORTED_SYMBOLS = (
     "bsa_score_blocks", "bsa_topk_select", "bsa_sparse_attn_prefill", "bsa_gated_attn_fwd",
     "bsa_sparse_attn_decode", "bsa_gist_expand_decode", "bsa_workspace_bytes",
-    "bsa_status_string", "bsa_device_status", "bsa_version",
+    "bsa_status_string", "bsa_device_status", "bsa_version", "bsa_sparse_attn_decode_noalloc",
 )
 
 
@@ -69,6 +69,8 @@ _SIGS = {
                                     ctypes.c_size_t, _p, _p, _p]),
     "bsa_gist_expand_decode": (_i, [ctypes.POINTER(BsaShape), _p, _p, _p, _p, _p, _i, _p, _p, ctypes.c_float,
                                     _p, ctypes.c_size_t, _p, _p, _p]),
+    "bsa_sparse_attn_decode_noalloc": (_i, [ctypes.POINTER(BsaShape), _p, _p, _p, _p, _i, ctypes.c_float, _p,
+                                            _p, _p]),
     "bsa_workspace_bytes": (ctypes.c_size_t, [_i, ctypes.POINTER(BsaShape), _i]),
     "bsa_status_string": (ctypes.c_char_p, [_i]),
     "bsa_device_status": (_i, [ctypes.POINTER(ctypes.c_uint), _i]),
@@ -79,7 +81,7 @@ _SIGS = {
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"libbsa.so is not built at {LIB_PATH}; build it with "
-                          "`python -m top_block_sparse_bsa_b200._build`")
+                          "`python top_block_sparse_bsa_b200/_build.py`")
     L = ctypes.CDLL(LIB_PATH)
     for name, (res, args) in _SIGS.items():
         f = getattr(L, name)
@@ -195,3 +197,11 @@ def bsa_gist_expand_decode(shape: BsaShape, q, k_cache, v_cache, gist_k, gist_v,
         _ptr(idx_in), _ptr(idx_out), ctypes.c_float(softmax_scale), _ptr(workspace),
         ctypes.c_size_t(workspace.numel() * workspace.element_size() if workspace is not None else 0),
         _ptr(o), _ptr(lse), _stream(stream)))
+
+
+def bsa_sparse_attn_decode_noalloc(shape: BsaShape, q, k_cache, v_cache, idx, idx_stride: int,
+                                   softmax_scale: float, o, lse=None, stream=None) -> None:
+    """Decode without a caller-provided workspace (scratch lives in the library)."""
+    _check("bsa_sparse_attn_decode_noalloc", lib.bsa_sparse_attn_decode_noalloc(
+        ctypes.byref(shape), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(idx), int(idx_stride),
+        ctypes.c_float(softmax_scale), _ptr(o), _ptr(lse), _stream(stream)))
