@@ -256,8 +256,10 @@ static bsa_status_t prefill_common(const bsa_shape_t* s, const void* q, const vo
   if (idx_stride > 256) return BSA_ERR_UNSUPPORTED;
   if (s->block != 64 && s->block != 128) return BSA_ERR_UNSUPPORTED;
   uint32_t* status = nullptr;
-  if ((st = device_state(&status, nullptr)) != BSA_OK) return st;
+  int sms = 0;
+  if ((st = device_state(&status, &sms)) != BSA_OK) return st;
   PrefillArgs a;
+  a.num_sms = sms;
   a.B = s->B;
   a.Hq = s->Hq;
   a.Hkv = s->Hkv;

@@ -29,6 +29,7 @@ struct PrefillArgs {
   void* o;
   float* lse;
   uint32_t* status;
+  int num_sms;
 };
 cudaError_t launch_attn_prefill_bf16(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
                                      const PrefillArgs& a, cudaStream_t st);

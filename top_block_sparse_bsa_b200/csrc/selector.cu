@@ -152,12 +152,48 @@ cudaError_t launch_score_prefill(const float* qbar, const float* kbar, int B, in
   return cudaGetLastError();
 }
 
-// Decode: grid (tiles of 64 blocks, B*Hkv).  The group query mean is formed
-// in fixed order (heads ascending) by every CTA.
+// Decode: grid (tiles of 128 blocks, B*Hkv); one thread per block.  Each
+// thread streams its own pooled-key row with independent 16-byte loads (all
+// in flight at once), then runs the fixed-order dot product from registers.
+// The group query mean is formed in fixed order (heads ascending) per CTA.
+template <typename T, int D>
+__global__ void __launch_bounds__(128) score_decode_kernel(const T* __restrict__ q, const float* __restrict__ kbar,
+                                                           int Hq, int Hkv, int nb, float scale,
+                                                           float* __restrict__ s, float* __restrict__ qbar_out) {
+  __shared__ float qm[D];
+  const int64_t bg = blockIdx.y;
+  const int64_t b = bg / Hkv, g = bg % Hkv;
+  const int G = Hq / Hkv;
+  for (int c = threadIdx.x; c < D; c += blockDim.x) {
+    float acc = 0.0f;
+    for (int hh = 0; hh < G; ++hh) acc = __fadd_rn(acc, static_cast<float>(q[(b * Hq + g * G + hh) * D + c]));
+    const float m = __fdiv_rn(acc, static_cast<float>(G));
+    qm[c] = m;
+    if (qbar_out && blockIdx.x == 0) qbar_out[bg * D + c] = m;
+  }
+  __syncthreads();
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= nb) return;
+  const float4* row = reinterpret_cast<const float4*>(kbar + (bg * nb + j) * D);
+  float4 kv[D / 4];
+#pragma unroll
+  for (int e = 0; e < D / 4; ++e) kv[e] = __ldg(row + e);
+  float acc = 0.0f;
+#pragma unroll
+  for (int e = 0; e < D / 4; ++e) {
+    acc = __fadd_rn(acc, __fmul_rn(qm[4 * e + 0], kv[e].x));
+    acc = __fadd_rn(acc, __fmul_rn(qm[4 * e + 1], kv[e].y));
+    acc = __fadd_rn(acc, __fmul_rn(qm[4 * e + 2], kv[e].z));
+    acc = __fadd_rn(acc, __fmul_rn(qm[4 * e + 3], kv[e].w));
+  }
+  s[bg * nb + j] = __fmul_rn(acc, scale);
+}
+
+// Generic-d fallback: rows staged through shared memory.
 template <typename T>
-__global__ void score_decode_kernel(const T* __restrict__ q, const float* __restrict__ kbar, int Hq,
-                                    int Hkv, int nb, int d, float scale, float* __restrict__ s,
-                                    float* __restrict__ qbar_out) {
+__global__ void score_decode_generic_kernel(const T* __restrict__ q, const float* __restrict__ kbar, int Hq,
+                                            int Hkv, int nb, int d, float scale, float* __restrict__ s,
+                                            float* __restrict__ qbar_out) {
   extern __shared__ float sm[];
   const int pitch = d + 1;
   float* qm = sm;              // [d]
@@ -168,10 +204,7 @@ __global__ void score_decode_kernel(const T* __restrict__ q, const float* __rest
   const int j0 = blockIdx.x * 64;
   for (int c = threadIdx.x; c < d; c += blockDim.x) {
     float acc = 0.0f;
-    for (int hh = 0; hh < G; ++hh) {
-      const T* qp = q + ((b * Hq + g * G + hh) * d + c);
-      acc = __fadd_rn(acc, static_cast<float>(*qp));
-    }
+    for (int hh = 0; hh < G; ++hh) acc = __fadd_rn(acc, static_cast<float>(q[(b * Hq + g * G + hh) * d + c]));
     const float m = __fdiv_rn(acc, static_cast<float>(G));
     qm[c] = m;
     if (qbar_out && blockIdx.x == 0) qbar_out[bg * d + c] = m;
@@ -189,14 +222,33 @@ __global__ void score_decode_kernel(const T* __restrict__ q, const float* __rest
 cudaError_t launch_score_decode(const void* q, bool bf16, const float* kbar, int B, int Hq, int Hkv,
                                 int nb, int d, float scale, float* s, float* qbar_out,
                                 cudaStream_t st) {
+  if (d == 128 || d == 64) {
+    dim3 grid((nb + 127) / 128, B * Hkv);
+    if (bf16) {
+      if (d == 128)
+        score_decode_kernel<__nv_bfloat16, 128><<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(q), kbar,
+                                                                      Hq, Hkv, nb, scale, s, qbar_out);
+      else
+        score_decode_kernel<__nv_bfloat16, 64><<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(q), kbar,
+                                                                     Hq, Hkv, nb, scale, s, qbar_out);
+    } else {
+      if (d == 128)
+        score_decode_kernel<float, 128><<<grid, 128, 0, st>>>(static_cast<const float*>(q), kbar, Hq, Hkv, nb,
+                                                              scale, s, qbar_out);
+      else
+        score_decode_kernel<float, 64><<<grid, 128, 0, st>>>(static_cast<const float*>(q), kbar, Hq, Hkv, nb,
+                                                             scale, s, qbar_out);
+    }
+    return cudaGetLastError();
+  }
   dim3 grid((nb + 63) / 64, B * Hkv);
   const size_t smem = (d + 64 * (d + 1)) * sizeof(float);
   if (bf16)
-    score_decode_kernel<__nv_bfloat16><<<grid, 64, smem, st>>>(
+    score_decode_generic_kernel<__nv_bfloat16><<<grid, 64, smem, st>>>(
         static_cast<const __nv_bfloat16*>(q), kbar, Hq, Hkv, nb, d, scale, s, qbar_out);
   else
-    score_decode_kernel<float><<<grid, 64, smem, st>>>(static_cast<const float*>(q), kbar, Hq, Hkv,
-                                                       nb, d, scale, s, qbar_out);
+    score_decode_generic_kernel<float><<<grid, 64, smem, st>>>(static_cast<const float*>(q), kbar, Hq, Hkv,
+                                                               nb, d, scale, s, qbar_out);
   return cudaGetLastError();
 }
 
