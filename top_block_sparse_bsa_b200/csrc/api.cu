@@ -85,26 +85,34 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 float score_scale(int d) { return static_cast<float>(1.0 / sqrt(static_cast<double>(d))); }
 
-// split-K factor of the decode kernels: enough CTAs to cover every SM about
-// twice, each CTA keeping at least a few steps of two tiles.
-int decode_splits(int rows, int max_tiles, int num_sms) {
+// Split-K plan of the decode kernels: the group rows' list positions are laid
+// end to end and cut into num_ctas equal ranges (one persistent CTA per SM by
+// default); no range may exceed the kernel's 128-tile item capacity.
+struct DecodePlan {
+  int num_ctas, max_slots, list_len;
+};
+
+DecodePlan decode_plan(int rows, int list_len, int num_sms) {
+  DecodePlan P;
+  P.list_len = list_len;
+  const int64_t total = static_cast<int64_t>(rows) * list_len;
+  int64_t c = num_sms;
   if (const char* env = getenv("BSA_DECODE_SPLITS")) {
     const int v = atoi(env);
-    if (v > 0) return v;
+    if (v > 0) c = v;
   }
-  int want = (2 * num_sms + rows - 1) / rows;
-  const int by_work = (max_tiles + 7) / 8;   // >= 4 steps (8 tiles) per split
-  if (want > by_work) want = by_work;
-  if (want < 1) want = 1;
-  // no CTA may own more than the kernel's tile-list capacity (1024)
-  const int min_for_cap = (max_tiles + 1023) / 1024;
-  if (want < min_for_cap) want = min_for_cap;
-  return want;
+  const int64_t need = (total + 127) / 128;   // ceil(total / c) <= 128
+  if (c < need) c = need;
+  if (c > total) c = total > 0 ? total : 1;
+  P.num_ctas = static_cast<int>(c);
+  P.max_slots = decode_slots_for(rows, list_len, P.num_ctas);
+  return P;
 }
 
 struct GistLayout {
   size_t scores, idx, expanded, union_list, partial, total;
-  int union_stride, nsplit;
+  int union_stride;
+  DecodePlan plan;
 };
 
 GistLayout gist_layout(const bsa_shape_t* s, int topk, int num_sms) {
@@ -113,7 +121,7 @@ GistLayout gist_layout(const bsa_shape_t* s, int topk, int num_sms) {
   const int G = s->Hq / s->Hkv;
   const int64_t rows = static_cast<int64_t>(s->B) * s->Hq;
   L.union_stride = 1 + G * topk + nc / 64;
-  L.nsplit = decode_splits(s->B * s->Hkv, L.union_stride - 1, num_sms);
+  L.plan = decode_plan(s->B * s->Hkv, L.union_stride - 1, num_sms);
   size_t off = 0;
   L.scores = off;
   off = align256(off + rows * nc * sizeof(float));
@@ -124,7 +132,7 @@ GistLayout gist_layout(const bsa_shape_t* s, int topk, int num_sms) {
   L.union_list = off;
   off = align256(off + static_cast<size_t>(s->B) * s->Hkv * L.union_stride * sizeof(int));
   L.partial = off;
-  off = align256(off + rows * L.nsplit * (s->d + 4) * sizeof(float));
+  off = align256(off + rows * L.plan.max_slots * (s->d + 4) * sizeof(float));
   L.total = off;
   return L;
 }
@@ -172,8 +180,9 @@ size_t bsa_workspace_bytes(int op, const bsa_shape_t* s, int budget) {
   int sms = 0;
   if (device_state(nullptr, &sms) != BSA_OK) return 0;
   if (op == BSA_OP_DECODE) {
-    const int nsplit = decode_splits(s->B * s->Hkv, budget, sms);
-    return align256(static_cast<size_t>(s->B) * s->Hq * nsplit * (s->d + 4) * sizeof(float));
+    if (budget < 1) return 0;
+    const DecodePlan P = decode_plan(s->B * s->Hkv, budget, sms);
+    return align256(static_cast<size_t>(s->B) * s->Hq * P.max_slots * (s->d + 4) * sizeof(float));
   }
   if (op == BSA_OP_GIST_DECODE) return gist_layout(s, budget, sms).total;
   return 0;
@@ -198,9 +207,8 @@ bsa_status_t bsa_score_blocks(const bsa_shape_t* s, int mode, const void* q, con
       return BSA_ERR_INVALID_ARG;
     if (!aligned16(k) || !aligned16(pooled_q_out) || !aligned16(pooled_k_out)) return BSA_ERR_INVALID_ARG;
     if (static_cast<int64_t>(nb) * nb >= (1ll << 31)) return BSA_ERR_UNSUPPORTED;
-    cudaError_t e = launch_pool(k, bf16, s->B, s->Hkv, s->Hkv, 1, s->Nk, s->d, s->block, pooled_k_out, cs);
-    if (e == cudaSuccess)
-      e = launch_pool(q, bf16, s->B, s->Hq, s->Hkv, G, s->Nq, s->d, s->block, pooled_q_out, cs);
+    cudaError_t e = launch_pool_prefill(q, k, bf16, s->B, s->Hq, s->Hkv, s->Nk, s->d, s->block, pooled_q_out,
+                                        pooled_k_out, cs);
     if (e == cudaSuccess) e = launch_score_prefill(pooled_q_out, pooled_k_out, s->B, s->Hkv, nb, s->d, scale, scores, cs);
     return cuda_status(e);
   }
@@ -321,8 +329,8 @@ bsa_status_t bsa_sparse_attn_decode(const bsa_shape_t* s, const void* q, const v
   int sms = 0;
   if ((st = device_state(&status, &sms)) != BSA_OK) return st;
   const int G = s->Hq / s->Hkv;
-  const int nsplit = decode_splits(s->B * s->Hkv, idx_stride, sms);
-  const size_t need = align256(static_cast<size_t>(s->B) * s->Hq * nsplit * (s->d + 4) * sizeof(float));
+  const DecodePlan P = decode_plan(s->B * s->Hkv, idx_stride, sms);
+  const size_t need = align256(static_cast<size_t>(s->B) * s->Hq * P.max_slots * (s->d + 4) * sizeof(float));
   if (workspace_bytes < need) return BSA_ERR_INVALID_ARG;
   CUtensorMap mq, mk, mv;
   if (!make_map_bf16(&mq, q, static_cast<uint64_t>(s->B) * s->Hq, static_cast<uint32_t>(G)) ||
@@ -340,13 +348,15 @@ bsa_status_t bsa_sparse_attn_decode(const bsa_shape_t* s, const void* q, const v
   a.list_has_count = 0;
   a.expanded = nullptr;
   a.nc = 0;
-  a.nsplit = nsplit;
+  a.list_len = P.list_len;
+  a.num_ctas = P.num_ctas;
+  a.max_slots = P.max_slots;
   a.softmax_scale = softmax_scale;
   a.partial = static_cast<float*>(workspace);
   a.status = status;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   cudaError_t e = launch_attn_decode_bf16(&mq, &mk, &mv, nullptr, nullptr, a, cs);
-  if (e == cudaSuccess) e = launch_decode_combine(a.partial, s->B * s->Hq, nsplit, s->d, true, o, lse, cs);
+  if (e == cudaSuccess) e = launch_decode_combine(a.partial, a, s->d, true, o, lse, cs);
   return cuda_status(e);
 }
 
@@ -409,12 +419,14 @@ bsa_status_t bsa_gist_expand_decode(const bsa_shape_t* s, const void* q, const v
   a.list_has_count = 1;
   a.expanded = expanded;
   a.nc = nc;
-  a.nsplit = L.nsplit;
+  a.list_len = L.plan.list_len;
+  a.num_ctas = L.plan.num_ctas;
+  a.max_slots = L.plan.max_slots;
   a.softmax_scale = softmax_scale;
   a.partial = reinterpret_cast<float*>(ws + L.partial);
   a.status = status;
   if (e == cudaSuccess) e = launch_attn_decode_bf16(&mq, &mk, &mv, &mgk, &mgv, a, cs);
-  if (e == cudaSuccess) e = launch_decode_combine(a.partial, rows, L.nsplit, s->d, true, o, lse, cs);
+  if (e == cudaSuccess) e = launch_decode_combine(a.partial, a, s->d, true, o, lse, cs);
   return cuda_status(e);
 }
 

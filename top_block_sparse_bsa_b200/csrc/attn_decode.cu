@@ -10,17 +10,23 @@
 // did not expand.
 //
 // Work decomposition.  All G query heads of a KV group read the same kept
-// blocks (decode) or the union of their expanded chunks (gist), so one CTA
-// gathers each 64-token tile once for the whole group: the G query rows form
-// the M dimension of the MMA (rows >= G are padding and never read back).
-// The tile list of a group is split across `nsplit` CTAs (split-K); each CTA
-// writes an unnormalised partial (running max m, sum l, O row) per head and a
-// second kernel merges them.
+// blocks (decode) or the union of their expanded chunks (gist), so each
+// 64-token tile is gathered once for the whole group.  The MMAs are "swapped":
+// the 128 keys of a step are the M dimension and the group's heads (padded to
+// 16) the N dimension, S^T = K Q^T and O^T += V^T P^T, so one softmax thread
+// owns one key and evaluates only G exponentials per step.  Split-K: the
+// groups' tile lists are laid end to end and cut into equal contiguous
+// ranges, one per persistent CTA (about one per SM), so every CTA streams the
+// same number of tiles through its TMA ring; a CTA's range covers one to a few
+// row segments, and each segment writes an unnormalised partial (running max
+// m, sum l, O) per head; a second kernel merges a row's segments.
 //
-// Roles (128 threads): warp 0 softmax (TMEM lanes 0-31 = query rows),
-// warp 1 TMA producer, warp 2 TMEM owner + MMA issuer, warp 3 list loader.
-// Tensor memory: S buffers A and B (128 columns each, double-buffered so the
-// next S = Q K^T runs while the softmax works) and O (128 columns).
+// Roles (256 threads): warps 0-3 softmax (TMEM lanes 0-127 = the step's keys)
+// and epilogue (lanes = channels of O^T), warp 4 TMA producer, warp 5 TMEM
+// owner + MMA issuer, warp 6 slice loader.  Tensor memory: two S^T buffers
+// (16 columns each) and O^T (16 columns).  The four softmax warps exchange
+// per-head maxima through shared memory with mbarrier hand-offs (bounded
+// waits, never bar.sync, so an abort cannot strand a warp).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -28,36 +34,55 @@ namespace bsa {
 namespace decode {
 
 constexpr int kD = 128;
-constexpr int kThreads = 128;
-constexpr int kStages = 2;
-constexpr int kMaxTiles = 1024;        // tiles one CTA may own
-constexpr uint32_t kHalfBytes = 128u * 128u;
-constexpr uint32_t kTileBytes = 2u * kHalfBytes;     // 128 rows x 128 bf16
-constexpr uint32_t kSmemQ = 0;
-constexpr uint32_t kSmemK = kTileBytes;
+constexpr int kNH = 16;                 // query heads of a group, padded (MMA N)
+constexpr int kThreads = 256;
+constexpr int kStages = 3;
+constexpr int kMaxItemTiles = 128;      // tiles one item may own
+constexpr uint32_t kHalfBytes = 128u * 128u;          // 128 rows x 64 bf16
+constexpr uint32_t kTileBytes = 2u * kHalfBytes;      // 128 rows x 128 bf16 (one step of K or V)
+constexpr uint32_t kSmallHalf = 16u * 128u;           // 16 rows x 64 bf16
+constexpr uint32_t kSmallBytes = 2u * kSmallHalf;     // Q^T or P^T buffer
+constexpr uint32_t kSmemK = 0;
 constexpr uint32_t kSmemV = kSmemK + kStages * kTileBytes;
-constexpr uint32_t kSmemBar = kSmemV + kStages * kTileBytes;
+constexpr uint32_t kSmemQ = kSmemV + kStages * kTileBytes;   // 2 buffers
+constexpr uint32_t kSmemP = kSmemQ + 2 * kSmallBytes;        // 2 buffers
+constexpr uint32_t kSmemBar = kSmemP + 2 * kSmallBytes;
 
 enum {
-  BAR_Q = 0,
-  BAR_KF = 1,
+  BAR_KF = 0,
   BAR_KE = BAR_KF + kStages,
   BAR_VF = BAR_KE + kStages,
   BAR_VE = BAR_VF + kStages,
-  BAR_SF = BAR_VE + kStages,   // two S buffers
-  BAR_PF = BAR_SF + 2,
-  BAR_OD = BAR_PF + 1,         // one completion per O += P V
-  BAR_OF = BAR_OD + 1,
-  BAR_AB = BAR_OF + 1,
-  NUM_BARS = BAR_AB + 1
+  BAR_QF = BAR_VE + kStages,   // per Q buffer
+  BAR_QE = BAR_QF + 2,
+  BAR_SF = BAR_QE + 2,         // per S buffer
+  BAR_SE = BAR_SF + 2,
+  BAR_PF = BAR_SE + 2,         // per P buffer
+  BAR_PE = BAR_PF + 2,
+  BAR_OD = BAR_PE + 2,         // one completion per O += V^T P^T
+  BAR_OF = BAR_OD + 1,         // per item: O complete
+  BAR_OE = BAR_OF + 1,         // per item: O read back
+  BAR_LF = BAR_OE + 1,         // per metadata slot
+  BAR_LE = BAR_LF + 2,
+  BAR_RX = BAR_LE + 2,         // cross-warp tile-maximum exchange, by step parity
+  BAR_LX = BAR_RX + 2,         // cross-warp row-sum exchange, by epilogue parity
+  BAR_AB = BAR_LX + 2,
+  NUM_BARS
+};
+constexpr uint32_t kListConsumers = 2 + 4;   // producer, MMA, one lane per softmax warp
+
+struct ItemInfo {
+  int n, b, g, bg, slot, pad0, pad1, pad2;
+  int tiles[kMaxItemTiles];
 };
 
 struct Misc {
   uint32_t tmem_base;
   int abort_flag;
-  int n_tiles;
-  int pad;
-  int tiles[kMaxTiles];
+  int pad[2];
+  float red[2][4][kNH];    // per-warp tile maxima, double-buffered by step parity
+  float lred[2][4][kNH];   // per-warp row sums at the end of an item, by epilogue parity
+  ItemInfo info[2];
 };
 constexpr uint32_t kSmemMisc = kSmemBar + NUM_BARS * 8;
 constexpr uint32_t kSmemBytes = kSmemMisc + sizeof(Misc) + 1024;
@@ -73,92 +98,212 @@ struct Params {
   int list_stride;
   int list_has_count;
   const uint32_t* expanded;
-  int nsplit;
+  int list_len;        // positions per group row (the split space is rows x list_len)
+  int64_t total;       // rows * list_len
+  int num_ctas;        // CTAs sharing the split space
+  int max_slots;       // partial records per head
   float scale_log2;
   float* partial;
   uint32_t* status;
 };
+
+// The split space is every group row's list positions laid end to end; CTA c
+// owns positions [c*total/C, (c+1)*total/C).  cta_of(x) is the CTA owning x.
+__host__ __device__ __forceinline__ int cta_of(int64_t x, int64_t total, int C) {
+  return static_cast<int>(((x + 1) * C + total - 1) / total) - 1;
+}
+
+// Number of row segments (work items) of this CTA, and its first row.
+__device__ __forceinline__ int cta_items(const Params& p, int c, int* r0) {
+  const int64_t lo = static_cast<int64_t>(c) * p.total / p.num_ctas;
+  const int64_t hi = static_cast<int64_t>(c + 1) * p.total / p.num_ctas;
+  if (lo >= hi) return 0;
+  *r0 = static_cast<int>(lo / p.list_len);
+  return static_cast<int>((hi - 1) / p.list_len) - *r0 + 1;
+}
 
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* ab, uint32_t* st) {
   bool ok = mbar_wait(bar, parity, ab, st);
   return __all_sync(0xffffffffu, ok);
 }
 
-// Key-column mask word of a 64-key tile for one head (bit e = key e allowed).
-__device__ __forceinline__ uint64_t tile_mask(int tile, const uint32_t* bits) {
-  if (bits == nullptr) return ~0ull;                       // plain decode: every key
-  if (tile >= 0) return ((bits[tile >> 5] >> (tile & 31)) & 1u) ? ~0ull : 0ull;   // expanded chunk
-  const int gb = -(tile + 1);                              // gist block: gists not expanded
-  const uint64_t w = static_cast<uint64_t>(bits[2 * gb]) | (static_cast<uint64_t>(bits[2 * gb + 1]) << 32);
-  return ~w;
+// Is key `kk` (0..127) of a step allowed for head slot h?  tile_a / tile_b
+// are the step's two tiles (tile_b < INT_MIN marks "no second tile").
+__device__ __forceinline__ bool key_allowed(int kk, int tile_a, int tile_b, bool has_b, const uint32_t* bits) {
+  const bool second = kk >= 64;
+  if (second && !has_b) return false;
+  const int tile = second ? tile_b : tile_a;
+  if (bits == nullptr) return true;                                  // plain decode
+  if (tile >= 0) return (bits[tile >> 5] >> (tile & 31)) & 1u;        // expanded chunk: its tokens
+  const int c = (-(tile + 1)) * 64 + (kk & 63);                      // gist of chunk c
+  return !((bits[c >> 5] >> (c & 31)) & 1u);                          // only if c is not expanded
 }
 
-template <int KEYS>
-__device__ __forceinline__ void softmax_step(uint32_t t_s, uint32_t t_o, float scale_log2, uint64_t mask0,
-                                             uint64_t mask1, int s, uint32_t bar_od, volatile int* ab,
-                                             uint32_t* st, float& m_run, float& l_run, bool& ok) {
-  float mx = -INFINITY;
+
+// Softmax role (warps 0-3), specialised on GH >= G query heads per group:
+// only GH columns of S^T and O^T are read, reduced and written.
+template <int GH>
+__device__ __forceinline__ void softmax_role(const Params& p, Misc* misc, uint8_t* smem, uint32_t sbase, uint32_t tmem,
+                                             volatile int* abortp, int warp, int lane, bool gist) {
+  auto bar = [&](int b) -> uint32_t { return sbase + kSmemBar + 8u * b; };
+    const int r = warp * 32 + lane;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    int s_read = 0, p_written = 0, od_seen = 0, items_done = 0, rx = 0;
+    bool ok = true;
+    int r0 = 0;
+    const int nitems = cta_items(p, blockIdx.x, &r0);
+    for (int k = 0; ok && k < nitems; ++k) {
+      const int buf = k & 1;
+      if (!(ok = warp_wait(bar(BAR_LF + buf), (k >> 1) & 1, abortp, p.status))) break;
+      const ItemInfo* inf = &misc->info[buf];
+      const int n = inf->n, G = p.G;
+      const int b = inf->b, g = inf->g;
+      float* part_base = p.partial + (static_cast<int64_t>(inf->bg) * G * p.max_slots + inf->slot) * kRec;
+      const int64_t head_stride = static_cast<int64_t>(p.max_slots) * kRec;
+      if (n == 0) {
+        // empty slice: m = -inf, l = 0, O = 0
+        for (int h = 0; h < G; ++h) {
+          float* part = part_base + h * head_stride;
+          if (r == 0) {
+            part[0] = -INFINITY;
+            part[1] = 0.0f;
+          }
+          part[4 + r] = 0.0f;
+        }
+      } else {
+        const uint32_t* bits_base =
+            gist ? p.expanded + (static_cast<int64_t>(b) * p.Hq + g * G) * (p.nc / 32) : nullptr;
+        float m_run[GH], l_part[GH];
 #pragma unroll
-  for (int ch = 0; ch < KEYS / 32; ++ch) {
-    uint32_t v[32];
-    tmem_ld32(t_s + ch * 32, v);
-    const uint64_t mk = (ch < 2) ? mask0 : mask1;
+        for (int h = 0; h < GH; ++h) {
+          m_run[h] = -INFINITY;
+          l_part[h] = 0.0f;
+        }
+        const int nsteps = (n + 1) / 2;
+        for (int s = 0; s < nsteps; ++s) {
+          const int sb = s_read & 1;
+          if (!(ok = warp_wait(bar(BAR_SF + sb), (s_read >> 1) & 1, abortp, p.status))) break;
+          tc_fence_after();
+          uint32_t sv[GH];
+          tmem_ldn<GH>(lane_addr + sb * 16, sv);
+          tc_fence_before();
+          mbar_arrive(bar(BAR_SE + sb));   // S buffer may be rewritten
+          ++s_read;
+          const int ta = inf->tiles[2 * s];
+          const bool has_b = 2 * s + 1 < n;
+          const int tbv = has_b ? inf->tiles[2 * s + 1] : 0;
+          float x[GH];
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const int bit = (ch & 1) * 32 + e;
-      float x = __uint_as_float(v[e]) * scale_log2;
-      if (!((mk >> bit) & 1ull)) x = -INFINITY;
-      mx = fmaxf(mx, x);
-    }
-  }
-  const float m_new = fmaxf(m_run, mx);
-  const bool need = m_new > m_run + kRescaleThreshold;
-  const float m_use = need ? m_new : m_run;
-  const float m_sub = (m_use == -INFINITY) ? 0.0f : m_use;
-  const float alpha = need ? fast_exp2(m_run - m_use) : 1.0f;
-  if (s > 0 && __any_sync(0xffffffffu, need)) {
-    // the previous O += P V must be complete before O is rescaled
-    if (!warp_wait(bar_od, (s - 1) & 1, ab, st)) {
-      ok = false;
-      return;
-    }
-    tc_fence_after();
-#pragma unroll 1
-    for (int ch = 0; ch < kD / 32; ++ch) {
-      uint32_t v[32];
-      tmem_ld32(t_o + ch * 32, v);
+          for (int h = 0; h < GH; ++h) {
+            bool allowed = h < G;
+            if (allowed) allowed = key_allowed(r, ta, tbv, has_b, gist ? bits_base + h * (p.nc / 32) : nullptr);
+            x[h] = allowed ? __uint_as_float(sv[h]) * p.scale_log2 : -INFINITY;
+          }
+          // tile maximum per head across the 128 keys
+          float tm[GH];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-      tmem_st32(t_o + ch * 32, v);
-    }
-  }
-  l_run *= alpha;
-  m_run = m_use;
-  float sum = 0.0f;
+          for (int h = 0; h < GH; ++h) {
+            float v = x[h];
+            if (h < G) {
 #pragma unroll
-  for (int ch = 0; ch < KEYS / 32; ++ch) {
-    uint32_t v[32];
-    tmem_ld32(t_s + ch * 32, v);
-    const uint64_t mk = (ch < 2) ? mask0 : mask1;
-    uint32_t pk[16];
+              for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+            }
+            tm[h] = v;
+          }
+          // exchange the four warps' maxima (bounded mbarrier wait, double-buffered)
+          const int xb = rx & 1;
+          if (lane == 0) {
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      float p2[2];
+            for (int h = 0; h < GH; ++h) misc->red[xb][warp][h] = tm[h];
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(BAR_RX + xb));
+          if (!(ok = warp_wait(bar(BAR_RX + xb), (rx >> 1) & 1, abortp, p.status))) break;
+          ++rx;
+          bool any_need = false;
+          float alpha[GH], msub[GH];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int bit = (ch & 1) * 32 + 2 * e + h;
-        float x = __uint_as_float(v[2 * e + h]) * scale_log2;
-        if (!((mk >> bit) & 1ull)) x = -INFINITY;
-        p2[h] = fast_exp2(x - m_sub);
-        sum += p2[h];
+          for (int h = 0; h < GH; ++h) {
+            float t = -INFINITY;
+            if (h < G) {
+#pragma unroll
+              for (int w2 = 0; w2 < 4; ++w2) t = fmaxf(t, misc->red[xb][w2][h]);
+            }
+            const float m_new = fmaxf(m_run[h], t);
+            const bool need = m_new > m_run[h] + kRescaleThreshold;
+            const float m_use = need ? m_new : m_run[h];
+            alpha[h] = need ? fast_exp2(m_run[h] - m_use) : 1.0f;
+            any_need |= need && s > 0;
+            m_run[h] = m_use;
+            msub[h] = (m_use == -INFINITY) ? 0.0f : m_use;
+            l_part[h] *= alpha[h];
+          }
+          if (any_need) {
+            // rescale O^T (this thread's lane = channel r): the previous PV must be done
+            if (!(ok = warp_wait(bar(BAR_OD), (od_seen + s - 1) & 1, abortp, p.status))) break;
+            tc_fence_after();
+            uint32_t ov[GH];
+            tmem_ldn<GH>(lane_addr + 32, ov);
+#pragma unroll
+            for (int h = 0; h < GH; ++h) ov[h] = __float_as_uint(__uint_as_float(ov[h]) * alpha[h]);
+            tmem_stn<GH>(lane_addr + 32, ov);
+            tmem_wait_st();
+          }
+          // P^T[h][key] = exp2(x - m), written into the swizzled B operand
+          const int pb = p_written & 1;
+          if (p_written >= 2 && !(ok = warp_wait(bar(BAR_PE + pb), ((p_written >> 1) - 1) & 1, abortp, p.status))) break;
+          uint8_t* pbase = smem + kSmemP + pb * kSmallBytes + (r >> 6) * kSmallHalf;
+          const int kr = r & 63;
+#pragma unroll
+          for (int h = 0; h < GH; ++h) {
+            const float pv = (h < G) ? fast_exp2(x[h] - msub[h]) : 0.0f;
+            l_part[h] += pv;
+            const uint32_t off = h * 128 + ((((kr >> 3) ^ (h & 7)) & 7) << 4) + (kr & 7) * 2;
+            *reinterpret_cast<__nv_bfloat16*>(pbase + off) = __float2bfloat16_rn(pv);
+          }
+          fence_proxy_async_smem();
+          tc_fence_before();
+          mbar_arrive(bar(BAR_PF + pb));
+          ++p_written;
+        }
+        if (!ok) break;
+        od_seen += nsteps;
+        // ---- epilogue: row sums across the 128 keys, then O^T row r = channel r
+        const int lb = items_done & 1;
+#pragma unroll
+        for (int h = 0; h < GH; ++h) {
+          float v = l_part[h];
+          if (h < G) {
+#pragma unroll
+            for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+          }
+          if (lane == 0) misc->lred[lb][warp][h] = v;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(BAR_LX + lb));
+        if (!(ok = warp_wait(bar(BAR_OF), items_done & 1, abortp, p.status))) break;
+        tc_fence_after();
+        uint32_t ov[GH];
+        tmem_ldn<GH>(lane_addr + 32, ov);
+        tc_fence_before();
+        mbar_arrive(bar(BAR_OE));
+        if (!(ok = warp_wait(bar(BAR_LX + lb), (items_done >> 1) & 1, abortp, p.status))) break;
+        ++items_done;
+#pragma unroll
+        for (int h = 0; h < GH; ++h) {
+          if (h >= G) continue;
+          float* part = part_base + h * head_stride;
+          part[4 + r] = __uint_as_float(ov[h]);
+          if (r == 0) {
+            part[0] = m_run[h];
+            part[1] = misc->lred[lb][0][h] + misc->lred[lb][1][h] + misc->lred[lb][2][h] + misc->lred[lb][3][h];
+          }
+        }
       }
-      pk[e] = pack_bf16x2(p2[0], p2[1]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BAR_LE + buf));
     }
-    tmem_st16(t_s + ch * 16, pk);
   }
-  l_run += sum;
-  tmem_wait_st();
-}
 
 __global__ void __launch_bounds__(kThreads, 1)
     attn_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -170,30 +315,36 @@ __global__ void __launch_bounds__(kThreads, 1)
   Misc* misc = reinterpret_cast<Misc*>(smem + kSmemMisc);
   auto bar = [&](int b) -> uint32_t { return sbase + kSmemBar + 8u * b; };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int split = blockIdx.x;
-  const int bg = blockIdx.y;
-  const int b = bg / p.Hkv, g = bg % p.Hkv;
   volatile int* abortp = &misc->abort_flag;
   const bool gist = p.expanded != nullptr;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(BAR_Q), 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(bar(BAR_KF + s), 1);
       mbar_init(bar(BAR_KE + s), 1);
       mbar_init(bar(BAR_VF + s), 1);
       mbar_init(bar(BAR_VE + s), 1);
     }
-    mbar_init(bar(BAR_SF + 0), 1);
-    mbar_init(bar(BAR_SF + 1), 1);
-    mbar_init(bar(BAR_PF), 32);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(BAR_QF + t), 1);
+      mbar_init(bar(BAR_QE + t), 1);
+      mbar_init(bar(BAR_SF + t), 1);
+      mbar_init(bar(BAR_SE + t), 128);
+      mbar_init(bar(BAR_PF + t), 128);
+      mbar_init(bar(BAR_PE + t), 1);
+      mbar_init(bar(BAR_LF + t), 1);
+      mbar_init(bar(BAR_LE + t), kListConsumers);
+      mbar_init(bar(BAR_RX + t), 4);
+      mbar_init(bar(BAR_LX + t), 4);
+    }
     mbar_init(bar(BAR_OD), 1);
     mbar_init(bar(BAR_OF), 1);
+    mbar_init(bar(BAR_OE), 128);
     mbar_init(bar(BAR_AB), 1);
     misc->abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 1 && lane == 0) {
+  if (warp == 4 && lane == 0) {
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
@@ -202,225 +353,265 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmGV);
     }
   }
-  if (warp == 2) {
-    tmem_alloc(sbase + kSmemMisc + offsetof(Misc, tmem_base), 512);
+  if (warp == 5) {
+    tmem_alloc(sbase + kSmemMisc + offsetof(Misc, tmem_base), 64);
     tmem_relinquish();
-  }
-  if (warp == 3) {
-    // this CTA's slice of the group's tile list
-    const int* src = p.list + static_cast<int64_t>(bg) * p.list_stride;
-    int total;
-    if (p.list_has_count) {
-      total = src[0];
-      src += 1;
-    } else {
-      total = 0;
-      for (int base = 0; base < p.list_stride; base += 32) {
-        const int t = base + lane;
-        const int v = (t < p.list_stride) ? src[t] : -1;
-        const unsigned neg = __ballot_sync(0xffffffffu, v < 0);
-        total += neg ? __ffs(neg) - 1 : 32;
-        if (neg) break;
-      }
-    }
-    const int per = (total + p.nsplit - 1) / p.nsplit;
-    const int t0 = min(total, split * per), t1 = min(total, t0 + per);
-    int cnt = t1 - t0;
-    if (cnt > kMaxTiles) {
-      if (lane == 0) atomicOr(p.status, BSA_DEV_BAD_SHAPE);
-      cnt = kMaxTiles;
-    }
-    const int nb_cache = p.Nk / 64;
-    const int ngist = p.nc / 64;
-    for (int t = lane; t < cnt; t += 32) {
-      int v = src[t0 + t];
-      const bool bad = gist ? (v >= nb_cache || v < -ngist) : (v < 0 || v >= nb_cache);
-      if (bad) {
-        atomicOr(p.status, BSA_DEV_BAD_INDEX);
-        v = 0x7fffffff;   // marks a skipped tile
-      }
-      misc->tiles[t] = v;
-    }
-    __syncwarp();
-    if (lane == 0) {
-      // drop skipped tiles, keeping order
-      int w = 0;
-      for (int t = 0; t < cnt; ++t)
-        if (misc->tiles[t] != 0x7fffffff) misc->tiles[w++] = misc->tiles[t];
-      misc->n_tiles = w;
-    }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  const uint32_t tmem = misc->tmem_base;   // S^T buffers at columns 0 / 16, O^T at 32
 
-  const uint32_t tmem = misc->tmem_base;
-  const int n = misc->n_tiles;
-  const int nsteps = (n + 1) / 2;
-
-  if (warp == 1) {
-    if (lane == 0 && n > 0) {
-      // ------------------------------------------------ TMA producer
-      mbar_arrive_expect_tx(bar(BAR_Q), static_cast<uint32_t>(p.G) * 256u);
-      for (int hf = 0; hf < 2; ++hf)
-        tma_load_2d(sbase + kSmemQ + hf * kHalfBytes, &tmQ, bar(BAR_Q), hf * 64, b * p.Hq + g * p.G);
-      int k_issued = 0, v_issued = 0;
-      for (int s = 0; s < nsteps; ++s) {
-        const int slot = s % kStages, use = s / kStages;
-        const int nt = (2 * s + 1 < n) ? 2 : 1;
-        const uint32_t bytes = static_cast<uint32_t>(nt) * 64u * 256u;
-        for (int kv = 0; kv < 2; ++kv) {
-          const int full = kv ? BAR_VF : BAR_KF, empty = kv ? BAR_VE : BAR_KE;
-          const uint32_t dst0 = sbase + (kv ? kSmemV : kSmemK) + slot * kTileBytes;
-          if (s >= kStages && !mbar_wait(bar(empty + slot), (use - 1) & 1, abortp, p.status)) break;
-          mbar_arrive_expect_tx(bar(full + slot), bytes);
-          for (int tt = 0; tt < nt; ++tt) {
-            const int tile = misc->tiles[2 * s + tt];
-            const CUtensorMap* map;
-            int y;
-            if (tile >= 0) {
-              map = kv ? &tmV : &tmK;
-              y = bg * p.Nk + tile * 64;
-            } else {
-              map = kv ? &tmGV : &tmGK;
-              y = bg * p.nc + (-(tile + 1)) * 64;
-            }
-            for (int hf = 0; hf < 2; ++hf)
-              tma_load_2d(dst0 + hf * kHalfBytes + tt * 8192u, map, bar(full + slot), hf * 64, y);
+  if (warp == 6) {
+    // ------------------------------------------------ item loader
+    const int nb_cache = p.Nk / 64, ngist = p.nc / 64;
+    int r0 = 0;
+    const int nitems = cta_items(p, blockIdx.x, &r0);
+    const int64_t lo = static_cast<int64_t>(blockIdx.x) * p.total / p.num_ctas;
+    const int64_t hi = static_cast<int64_t>(blockIdx.x + 1) * p.total / p.num_ctas;
+    const unsigned lt = (1u << lane) - 1u;
+    for (int k = 0; k < nitems; ++k) {
+      const int buf = k & 1;
+      if (k >= 2 && !warp_wait(bar(BAR_LE + buf), ((k >> 1) - 1) & 1, abortp, p.status)) break;
+      ItemInfo* inf = &misc->info[buf];
+      const int bg = r0 + k;
+      const int64_t row0 = static_cast<int64_t>(bg) * p.list_len;
+      const int a = static_cast<int>(max(lo, row0) - row0);
+      const int e = static_cast<int>(min(hi, row0 + p.list_len) - row0);
+      const int* src = p.list + static_cast<int64_t>(bg) * p.list_stride;
+      int count;
+      if (p.list_has_count) {
+        count = min(src[0], p.list_len);
+        src += 1;
+      } else {
+        count = e;   // the first negative entry ends the list
+        for (int base = 0; base < e; base += 32) {
+          const int t = base + lane;
+          const int v = (t < e) ? src[t] : 0;
+          const unsigned neg = __ballot_sync(0xffffffffu, v < 0);
+          if (neg) {
+            count = base + __ffs(neg) - 1;
+            break;
           }
-          if (kv) ++v_issued; else ++k_issued;
         }
-        if (*abortp) break;
+      }
+      const int stop = min(e, count);
+      int w = 0;
+      for (int base = a; base < stop; base += 32) {
+        const int t = base + lane;
+        const int v = (t < stop) ? src[t] : 0;
+        const bool bad = (t < stop) && (gist ? (v >= nb_cache || v < -ngist) : (v < 0 || v >= nb_cache));
+        if (bad) atomicOr(p.status, BSA_DEV_BAD_INDEX);
+        const bool keep = (t < stop) && !bad && (w + (t - base) < kMaxItemTiles);
+        const unsigned km = __ballot_sync(0xffffffffu, keep);
+        if (keep) inf->tiles[w + __popc(km & lt)] = v;
+        w += __popc(km);
+      }
+      if (lane == 0) {
+        if (stop - a > kMaxItemTiles) atomicOr(p.status, BSA_DEV_BAD_SHAPE);
+        inf->n = w;
+        inf->bg = bg;
+        inf->b = bg / p.Hkv;
+        inf->g = bg % p.Hkv;
+        inf->slot = static_cast<int>(blockIdx.x) - cta_of(row0, p.total, p.num_ctas);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BAR_LF + buf));
+    }
+  } else if (warp == 4) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      int gs = 0, qcount = 0, k_issued = 0, v_issued = 0;
+      bool ok = true;
+      int r0 = 0;
+      const int nitems = cta_items(p, blockIdx.x, &r0);
+      for (int k = 0; ok && k < nitems; ++k) {
+        const int buf = k & 1;
+        if (!(ok = mbar_wait(bar(BAR_LF + buf), (k >> 1) & 1, abortp, p.status))) break;
+        const ItemInfo* inf = &misc->info[buf];
+        const int n = inf->n;
+        if (n > 0) {
+          const int qb = qcount & 1;
+          if (qcount >= 2 && !(ok = mbar_wait(bar(BAR_QE + qb), ((qcount >> 1) - 1) & 1, abortp, p.status))) break;
+          mbar_arrive_expect_tx(bar(BAR_QF + qb), static_cast<uint32_t>(p.G) * 256u);
+          for (int hf = 0; hf < 2; ++hf)
+            tma_load_2d(sbase + kSmemQ + qb * kSmallBytes + hf * kSmallHalf, &tmQ, bar(BAR_QF + qb), hf * 64,
+                        inf->b * p.Hq + inf->g * p.G);
+          ++qcount;
+          const int nsteps = (n + 1) / 2;
+          for (int s = 0; s < nsteps; ++s, ++gs) {
+            const int slot = gs % kStages, use = gs / kStages;
+            const int nt = (2 * s + 1 < n) ? 2 : 1;
+            const uint32_t bytes = static_cast<uint32_t>(nt) * 64u * 256u;
+            for (int kv = 0; kv < 2; ++kv) {
+              const int full = kv ? BAR_VF : BAR_KF, empty = kv ? BAR_VE : BAR_KE;
+              const uint32_t dst0 = sbase + (kv ? kSmemV : kSmemK) + slot * kTileBytes;
+              if (gs >= kStages && !(ok = mbar_wait(bar(empty + slot), (use - 1) & 1, abortp, p.status))) break;
+              mbar_arrive_expect_tx(bar(full + slot), bytes);
+              for (int tt = 0; tt < nt; ++tt) {
+                const int tile = inf->tiles[2 * s + tt];
+                const CUtensorMap* map;
+                int y;
+                if (tile >= 0) {
+                  map = kv ? &tmV : &tmK;
+                  y = inf->bg * p.Nk + tile * 64;
+                } else {
+                  map = kv ? &tmGV : &tmGK;
+                  y = inf->bg * p.nc + (-(tile + 1)) * 64;
+                }
+                for (int hf = 0; hf < 2; ++hf)
+                  tma_load_2d(dst0 + hf * kHalfBytes + tt * 8192u, map, bar(full + slot), hf * 64, y);
+              }
+              if (kv) ++v_issued; else ++k_issued;
+            }
+            if (!ok) break;
+          }
+          if (!ok) break;
+        }
+        mbar_arrive(bar(BAR_LE + buf));
       }
       if (*abortp) {
-        mbar_drain(bar(BAR_Q), 0);
+        for (int q = max(0, qcount - 2); q < qcount; ++q) mbar_drain(bar(BAR_QF + (q & 1)), (q >> 1) & 1);
         for (int s = max(0, k_issued - kStages); s < k_issued; ++s) mbar_drain(bar(BAR_KF + s % kStages), (s / kStages) & 1);
         for (int s = max(0, v_issued - kStages); s < v_issued; ++s) mbar_drain(bar(BAR_VF + s % kStages), (s / kStages) & 1);
       }
     }
-  } else if (warp == 2) {
-    if (lane == 0 && n > 0) {
+  } else if (warp == 5) {
+    if (lane == 0) {
       // ------------------------------------------------ MMA issuer
-      const uint32_t id_s128 = idesc_bf16_f32(128, 128, 0, 0);
-      const uint32_t id_s64 = idesc_bf16_f32(128, 64, 0, 0);
-      const uint32_t id_pv = idesc_bf16_f32(128, 128, 0, 1);
-      auto keys_of = [&](int s) -> int { return (2 * s + 1 < n) ? 128 : 64; };
-      auto issue_s = [&](int s) {
-        const int slot = s % kStages;
+      const uint32_t id_s = idesc_bf16_f32(128, kNH, 0, 0);    // S^T = K Q^T, both K-major
+      const uint32_t id_pv = idesc_bf16_f32(128, kNH, 1, 0);   // O^T = V^T P^T, V^T MN-major
+      int gs = 0, qcount = 0, items_done = 0;
+      int s_issued = 0, p_used = 0;   // S buffers written / P buffers consumed (global counts)
+      bool ok = true;
+      auto issue_s = [&](int slot, int qb, int sbuf) {
         const uint32_t ka = sbase + kSmemK + slot * kTileBytes;
-        const uint32_t qa = sbase + kSmemQ;
-        const uint32_t id = keys_of(s) == 128 ? id_s128 : id_s64;
+        const uint32_t qa = sbase + kSmemQ + qb * kSmallBytes;
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-          mma_ss(tmem + (s & 1) * 128, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), id,
-                 kk > 0 ? 1u : 0u);
+          const uint32_t offk = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+          const uint32_t offq = (kk >> 2) * kSmallHalf + (kk & 3) * 32;
+          mma_ss(tmem + sbuf * 16, smem_desc_sw128(ka + offk, 16, 1024), smem_desc_sw128(qa + offq, 16, 1024),
+                 id_s, kk > 0 ? 1u : 0u);
         }
-        tc_commit(bar(BAR_SF + (s & 1)));
-        tc_commit(bar(BAR_KE + slot));
       };
-      bool ok = mbar_wait(bar(BAR_Q), 0, abortp, p.status) &&
-                mbar_wait(bar(BAR_KF + 0), 0, abortp, p.status);
-      tc_fence_after();
-      if (ok) issue_s(0);
-      for (int s = 0; ok && s < nsteps; ++s) {
-        if (s + 1 < nsteps) {
-          const int s1 = s + 1;
-          if (!(ok = mbar_wait(bar(BAR_KF + s1 % kStages), (s1 / kStages) & 1, abortp, p.status))) break;
+      int r0 = 0;
+      const int nitems = cta_items(p, blockIdx.x, &r0);
+      for (int k = 0; ok && k < nitems; ++k) {
+        const int buf = k & 1;
+        if (!(ok = mbar_wait(bar(BAR_LF + buf), (k >> 1) & 1, abortp, p.status))) break;
+        const int n = misc->info[buf].n;
+        if (n > 0) {
+          const int nsteps = (n + 1) / 2;
+          const int qb = qcount & 1;
+          if (!(ok = mbar_wait(bar(BAR_QF + qb), (qcount >> 1) & 1, abortp, p.status))) break;
+          ++qcount;
           tc_fence_after();
-          issue_s(s1);
+          const int gs0 = gs;
+          // S for the first step of the item
+          for (int s = 0; ok && s < nsteps; ++s) {
+            // issue S(s) (the softmax must have read the S buffer two steps back)
+            {
+              const int g_s = gs0 + s, slot = g_s % kStages, sb = s_issued & 1;
+              if (!(ok = mbar_wait(bar(BAR_KF + slot), (g_s / kStages) & 1, abortp, p.status))) break;
+              if (s_issued >= 2 && !(ok = mbar_wait(bar(BAR_SE + sb), ((s_issued >> 1) - 1) & 1, abortp, p.status)))
+                break;
+              tc_fence_after();
+              issue_s(slot, qb, sb);
+              tc_commit(bar(BAR_SF + sb));
+              tc_commit(bar(BAR_KE + slot));
+              ++s_issued;
+            }
+            // O^T += V^T P^T for step s-1 (one step behind, so S(s) overlaps the softmax of s-1)
+            if (s > 0) {
+              const int ps = s - 1, g_p = gs0 + ps, slot = g_p % kStages, pb = p_used & 1;
+              if (!(ok = mbar_wait(bar(BAR_PF + pb), (p_used >> 1) & 1, abortp, p.status))) break;
+              if (!(ok = mbar_wait(bar(BAR_VF + slot), (g_p / kStages) & 1, abortp, p.status))) break;
+              if (ps == 0 && items_done > 0 &&
+                  !(ok = mbar_wait(bar(BAR_OE), (items_done - 1) & 1, abortp, p.status)))
+                break;
+              tc_fence_after();
+              const int keys = (2 * ps + 1 < n) ? 128 : 64;
+              const uint32_t va = sbase + kSmemV + slot * kTileBytes;
+              const uint32_t pa = sbase + kSmemP + pb * kSmallBytes;
+              for (int kk = 0; kk < keys / 16; ++kk)
+                mma_ss(tmem + 32, smem_desc_sw128(va + kk * 2048, kHalfBytes, 1024),
+                       smem_desc_sw128(pa + (kk >> 2) * kSmallHalf + (kk & 3) * 32, 16, 1024), id_pv,
+                       (ps > 0 || kk > 0) ? 1u : 0u);
+              tc_commit(bar(BAR_OD));
+              tc_commit(bar(BAR_VE + slot));
+              tc_commit(bar(BAR_PE + pb));
+              ++p_used;
+            }
+          }
+          if (!ok) break;
+          tc_commit(bar(BAR_QE + qb));
+          {
+            const int ps = nsteps - 1, g_p = gs0 + ps, slot = g_p % kStages, pb = p_used & 1;
+            if (!(ok = mbar_wait(bar(BAR_PF + pb), (p_used >> 1) & 1, abortp, p.status))) break;
+            if (!(ok = mbar_wait(bar(BAR_VF + slot), (g_p / kStages) & 1, abortp, p.status))) break;
+            if (ps == 0 && items_done > 0 && !(ok = mbar_wait(bar(BAR_OE), (items_done - 1) & 1, abortp, p.status)))
+              break;
+            tc_fence_after();
+            const int keys = (2 * ps + 1 < n) ? 128 : 64;
+            const uint32_t va = sbase + kSmemV + slot * kTileBytes;
+            const uint32_t pa = sbase + kSmemP + pb * kSmallBytes;
+            for (int kk = 0; kk < keys / 16; ++kk)
+              mma_ss(tmem + 32, smem_desc_sw128(va + kk * 2048, kHalfBytes, 1024),
+                     smem_desc_sw128(pa + (kk >> 2) * kSmallHalf + (kk & 3) * 32, 16, 1024), id_pv,
+                     (ps > 0 || kk > 0) ? 1u : 0u);
+            tc_commit(bar(BAR_OD));
+            tc_commit(bar(BAR_VE + slot));
+            tc_commit(bar(BAR_PE + pb));
+            ++p_used;
+          }
+          tc_commit(bar(BAR_OF));
+          ++items_done;
+          gs += nsteps;
         }
-        const int slot = s % kStages;
-        if (!(ok = mbar_wait(bar(BAR_PF), s & 1, abortp, p.status))) break;
-        if (!(ok = mbar_wait(bar(BAR_VF + slot), (s / kStages) & 1, abortp, p.status))) break;
-        tc_fence_after();
-        const uint32_t va = sbase + kSmemV + slot * kTileBytes;
-        const int keys = keys_of(s);
-        for (int kk = 0; kk < keys / 16; ++kk)
-          mma_ts(tmem + 256, tmem + (s & 1) * 128 + kk * 8, smem_desc_sw128(va + kk * 2048, kHalfBytes, 1024), id_pv,
-                 (s > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(bar(BAR_OD));
-        tc_commit(bar(BAR_VE + slot));
+        mbar_arrive(bar(BAR_LE + buf));
       }
-      if (ok) tc_commit(bar(BAR_OF));
       if (!ok) {
         tc_commit(bar(BAR_AB));
         mbar_drain(bar(BAR_AB), 0);
       }
     }
-  } else if (warp == 0) {
-    // ------------------------------------------------ softmax + partial out
-    const int r = lane;                      // query row = head g*G + r
-    const bool valid = r < p.G;
-    const int h = g * p.G + (valid ? r : 0);
-    const uint32_t* bits = gist ? p.expanded + (static_cast<int64_t>(b) * p.Hq + h) * (p.nc / 32) : nullptr;
-    const uint32_t t_o = tmem + 256;
-    float m_run = -INFINITY, l_run = 0.0f;
-    bool ok = true;
-    for (int s = 0; s < nsteps; ++s) {
-      if (!(ok = warp_wait(bar(BAR_SF + (s & 1)), (s >> 1) & 1, abortp, p.status))) break;
-      tc_fence_after();
-      const int tA = misc->tiles[2 * s];
-      const uint64_t mA = tile_mask(tA, bits);
-      const uint32_t t_s = tmem + (s & 1) * 128;
-      if (2 * s + 1 < n) {
-        const uint64_t mB = tile_mask(misc->tiles[2 * s + 1], bits);
-        softmax_step<128>(t_s, t_o, p.scale_log2, mA, mB, s, bar(BAR_OD), abortp, p.status, m_run, l_run, ok);
-      } else {
-        softmax_step<64>(t_s, t_o, p.scale_log2, mA, 0ull, s, bar(BAR_OD), abortp, p.status, m_run, l_run, ok);
-      }
-      if (!ok) break;
-      tc_fence_before();
-      mbar_arrive(bar(BAR_PF));
-    }
-    float* part = p.partial + ((static_cast<int64_t>(bg) * p.G + r) * p.nsplit + split) * kRec;
-    if (n == 0) {
-      if (valid) {
-        part[0] = -INFINITY;
-        part[1] = 0.0f;
-        for (int c = 0; c < kD; ++c) part[4 + c] = 0.0f;
-      }
-    } else if (ok && warp_wait(bar(BAR_OF), 0, abortp, p.status)) {
-      tc_fence_after();
-#pragma unroll 1
-      for (int ch = 0; ch < kD / 32; ++ch) {
-        uint32_t v[32];
-        tmem_ld32(t_o + ch * 32, v);
-        if (valid) {
-          float4* dst = reinterpret_cast<float4*>(part + 4 + ch * 32);
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            dst[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
-                                 __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
-        }
-      }
-      if (valid) {
-        part[0] = m_run;
-        part[1] = l_run;
-      }
-    }
+  } else if (warp < 4) {
+    // ------------------------------------------------ softmax (thread = key) + epilogue (thread = d)
+    if (p.G <= 4)
+      softmax_role<4>(p, misc, smem, sbase, tmem, abortp, warp, lane, gist);
+    else if (p.G <= 8)
+      softmax_role<8>(p, misc, smem, sbase, tmem, abortp, warp, lane, gist);
+    else
+      softmax_role<16>(p, misc, smem, sbase, tmem, abortp, warp, lane, gist);
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 2) {
+  if (warp == 5) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, 64);
   }
 }
 
-// Merge the split partials of one row (one warp per row).
-__global__ void combine_kernel(const float* __restrict__ partial, int rows, int nsplit, int d, int out_bf16,
-                               void* __restrict__ o, float* __restrict__ lse) {
+// Merge the partial records of one output row (b, h) (one warp per row):
+// the row's group was cut into nseg segments, one record each.
+__global__ void combine_kernel(const float* __restrict__ partial, int rows, int G, int list_len, int64_t total,
+                               int num_ctas, int max_slots, int d, int out_bf16, void* __restrict__ o,
+                               float* __restrict__ lse) {
   const int row = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
+  const int64_t bg = row / G;
+  const int first = cta_of(bg * list_len, total, num_ctas);
+  const int last = cta_of((bg + 1) * list_len - 1, total, num_ctas);
+  const int nseg = min(max_slots, last - first + 1);
   const int rec = d + 4;
-  const float* pr = partial + static_cast<int64_t>(row) * nsplit * rec;
+  const float* pr = partial + static_cast<int64_t>(row) * max_slots * rec;
   float M = -INFINITY;
-  for (int s = 0; s < nsplit; ++s) M = fmaxf(M, pr[s * rec]);
+  for (int s = 0; s < nseg; ++s) M = fmaxf(M, pr[s * rec]);
   float L = 0.0f;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int s = 0; s < nsplit; ++s) {
+  for (int s = 0; s < nseg; ++s) {
     const float ms = pr[s * rec];
     if (ms == -INFINITY) continue;
     const float w = exp2f(ms - M);
@@ -504,13 +695,9 @@ __global__ void gist_union_kernel(const int* __restrict__ idx, int Hq, int Hkv, 
 cudaError_t launch_attn_decode_bf16(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
                                     const CUtensorMap* tmGK, const CUtensorMap* tmGV, const DecodeArgs& a,
                                     cudaStream_t st) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(decode::attn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(decode::kSmemBytes));
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  cudaError_t e = cudaFuncSetAttribute(decode::attn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(decode::kSmemBytes));
+  if (e != cudaSuccess) return e;
   decode::Params p;
   p.B = a.B;
   p.Hq = a.Hq;
@@ -522,22 +709,39 @@ cudaError_t launch_attn_decode_bf16(const CUtensorMap* tmQ, const CUtensorMap* t
   p.list_stride = a.list_stride;
   p.list_has_count = a.list_has_count;
   p.expanded = a.expanded;
-  p.nsplit = a.nsplit;
+  p.list_len = a.list_len;
+  p.total = static_cast<int64_t>(a.B) * a.Hkv * a.list_len;
+  p.num_ctas = a.num_ctas;
+  p.max_slots = a.max_slots;
   p.scale_log2 = a.softmax_scale * decode::kLog2e;
   p.partial = a.partial;
   p.status = a.status;
-  dim3 grid(a.nsplit, a.B * a.Hkv);
+  const int grid = a.num_ctas;
   decode::attn_decode_kernel<<<grid, decode::kThreads, decode::kSmemBytes, st>>>(
       *tmQ, *tmK, *tmV, tmGK ? *tmGK : *tmK, tmGV ? *tmGV : *tmV, p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_decode_combine(const float* partial, int rows, int nsplit, int d, bool out_bf16, void* o,
+cudaError_t launch_decode_combine(const float* partial, const DecodeArgs& a, int d, bool out_bf16, void* o,
                                   float* lse, cudaStream_t st) {
   const int warps = 8;
-  decode::combine_kernel<<<(rows + warps - 1) / warps, warps * 32, 0, st>>>(partial, rows, nsplit, d,
-                                                                             out_bf16 ? 1 : 0, o, lse);
+  const int rows = a.B * a.Hq;
+  const int64_t total = static_cast<int64_t>(a.B) * a.Hkv * a.list_len;
+  decode::combine_kernel<<<(rows + warps - 1) / warps, warps * 32, 0, st>>>(
+      partial, rows, a.Hq / a.Hkv, a.list_len, total, a.num_ctas, a.max_slots, d, out_bf16 ? 1 : 0, o, lse);
   return cudaGetLastError();
+}
+
+int decode_slots_for(int rows, int list_len, int num_ctas) {
+  // the largest number of CTAs that can share one row's positions
+  const int64_t total = static_cast<int64_t>(rows) * list_len;
+  int best = 1;
+  for (int r = 0; r < rows; ++r) {
+    const int first = decode::cta_of(static_cast<int64_t>(r) * list_len, total, num_ctas);
+    const int last = decode::cta_of(static_cast<int64_t>(r + 1) * list_len - 1, total, num_ctas);
+    if (last - first + 1 > best) best = last - first + 1;
+  }
+  return best;
 }
 
 cudaError_t launch_gist_union(const int* idx, int B, int Hq, int Hkv, int topk, int idx_stride, int nc,

@@ -10,6 +10,8 @@ namespace bsa {
 // selector.cu
 cudaError_t launch_pool(const void* src, bool bf16, int B, int Hsrc, int Hgroups, int heads_sum, int N,
                         int d, int bs, float* out, cudaStream_t st);
+cudaError_t launch_pool_prefill(const void* q, const void* k, bool bf16, int B, int Hq, int Hkv, int N, int d,
+                                int bs, float* qbar, float* kbar, cudaStream_t st);
 cudaError_t launch_score_prefill(const float* qbar, const float* kbar, int B, int Hkv, int nb, int d,
                                  float scale, float* s, cudaStream_t st);
 cudaError_t launch_score_decode(const void* q, bool bf16, const float* kbar, int B, int Hq, int Hkv,
@@ -48,16 +50,19 @@ struct DecodeArgs {
   int list_has_count;        // 1: entry 0 is the count (gist union list)
   const uint32_t* expanded;  // gist: [B*Hq][nc/32] bitmap of expanded chunks; null for plain decode
   int nc;                    // gist: number of chunks
-  int nsplit;
+  int list_len;              // list positions per group row (split space = rows x list_len)
+  int num_ctas;              // persistent CTAs sharing the split space
+  int max_slots;             // partial records per output row
   float softmax_scale;
-  float* partial;            // [B*Hq][nsplit][d+2]
+  float* partial;            // [B*Hq][max_slots][d+4]
   uint32_t* status;
 };
 cudaError_t launch_attn_decode_bf16(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
                                     const CUtensorMap* tmGK, const CUtensorMap* tmGV, const DecodeArgs& a,
                                     cudaStream_t st);
-cudaError_t launch_decode_combine(const float* partial, int rows, int nsplit, int d, bool out_bf16, void* o,
+cudaError_t launch_decode_combine(const float* partial, const DecodeArgs& a, int d, bool out_bf16, void* o,
                                   float* lse, cudaStream_t st);
+int decode_slots_for(int rows, int list_len, int num_ctas);
 cudaError_t launch_gist_union(const int* idx, int B, int Hq, int Hkv, int topk, int idx_stride, int nc,
                               uint32_t* expanded, int* union_list, int union_stride, uint32_t* status,
                               cudaStream_t st);

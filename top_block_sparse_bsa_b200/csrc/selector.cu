@@ -82,6 +82,57 @@ __global__ void pool_kernel(const T* __restrict__ src, int B, int Hsrc, int Hgro
   for (int c = 0; c < 8; ++c) o[c] = __fdiv_rn(acc[c], div);
 }
 
+// Staged variant for bf16 units of at most kPoolStageBytes: one CTA per unit
+// copies the unit's rows (heads_sum runs of bs contiguous rows) into shared
+// memory with every 16-byte load in flight at once, then thread c sums column
+// c over the rows in the fixed order (heads ascending, tokens ascending).
+// blockIdx.y selects the job (a launch may carry two).
+constexpr int kPoolThreads = 256;
+constexpr int kPoolStageBytes = 64 * 1024;
+
+struct PoolJob {
+  const __nv_bfloat16* src;
+  int Hsrc, heads_sum;
+  float* out;
+};
+
+__global__ void __launch_bounds__(kPoolThreads) pool_staged_kernel(PoolJob job0, PoolJob job1, int Hgroups, int N,
+                                                                   int d, int bs, int64_t units) {
+  extern __shared__ __align__(16) uint8_t pool_smem[];
+  const PoolJob job = blockIdx.y ? job1 : job0;
+  if (job.src == nullptr) return;
+  const int nb = N / bs;
+  for (int64_t unit = blockIdx.x; unit < units; unit += gridDim.x) {
+    const int64_t b = unit / (static_cast<int64_t>(Hgroups) * nb);
+    const int64_t g = (unit / nb) % Hgroups;
+    const int64_t j = unit % nb;
+    const int run = bs * d;                 // elements of one head's run
+    const int run16 = run / 8;              // 16-byte chunks of one run
+    const int chunks = run16 * job.heads_sum;
+    uint4* stage = reinterpret_cast<uint4*>(pool_smem);
+    __syncthreads();                        // previous unit fully consumed
+    for (int e = threadIdx.x; e < chunks; e += kPoolThreads) {
+      const int hh = e / run16, w = e % run16;
+      const __nv_bfloat16* p = job.src + ((b * job.Hsrc + g * job.heads_sum + hh) * static_cast<int64_t>(N) + j * bs) * d;
+      stage[e] = __ldg(reinterpret_cast<const uint4*>(p) + w);
+    }
+    __syncthreads();
+    const __nv_bfloat16* sv = reinterpret_cast<const __nv_bfloat16*>(pool_smem);
+    const int rows = job.heads_sum * bs;   // a multiple of 16 (bs is 64 or 128)
+    for (int c = threadIdx.x; c < d; c += kPoolThreads) {
+      float acc = 0.0f;
+      for (int r = 0; r < rows; r += 16) {
+        float x[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) x[u] = __bfloat162float(sv[(r + u) * d + c]);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) acc = __fadd_rn(acc, x[u]);
+      }
+      job.out[unit * d + c] = __fdiv_rn(acc, static_cast<float>(rows));
+    }
+  }
+}
+
 template <typename T>
 static cudaError_t launch_pool_t(const void* src, int B, int Hsrc, int Hgroups, int heads_sum, int N,
                                  int d, int bs, float* out, cudaStream_t st) {
@@ -99,6 +150,33 @@ cudaError_t launch_pool(const void* src, bool bf16, int B, int Hsrc, int Hgroups
               : launch_pool_t<float>(src, B, Hsrc, Hgroups, heads_sum, N, d, bs, out, st);
 }
 
+// Prefill: keys (heads_sum 1) and grouped queries (heads_sum G), staged when a
+// query unit fits the stage; otherwise the plain per-thread kernel.
+cudaError_t launch_pool_prefill(const void* q, const void* k, bool bf16, int B, int Hq, int Hkv, int N, int d,
+                                int bs, float* qbar, float* kbar, cudaStream_t st) {
+  const int G = Hq / Hkv;
+  const size_t stage = static_cast<size_t>(G) * bs * d * 2;
+  if (!bf16 || stage > kPoolStageBytes || d % 8 != 0) {
+    cudaError_t e = launch_pool(k, bf16, B, Hkv, Hkv, 1, N, d, bs, kbar, st);
+    if (e == cudaSuccess) e = launch_pool(q, bf16, B, Hq, Hkv, G, N, d, bs, qbar, st);
+    return e;
+  }
+  cudaError_t e = cudaFuncSetAttribute(pool_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(stage));
+  if (e != cudaSuccess) return e;
+  const int64_t units = static_cast<int64_t>(B) * Hkv * (N / bs);
+  PoolJob jk{static_cast<const __nv_bfloat16*>(k), Hkv, 1, kbar};
+  PoolJob jq{static_cast<const __nv_bfloat16*>(q), Hq, G, qbar};
+  const PoolJob none{nullptr, 0, 0, nullptr};
+  const unsigned gx = static_cast<unsigned>(units < 65535 ? units : 65535);
+  pool_staged_kernel<<<dim3(gx, 1), kPoolThreads, static_cast<size_t>(bs) * d * 2, st>>>(jk, none, Hkv, N, d, bs,
+                                                                                          units);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  pool_staged_kernel<<<dim3(gx, 1), kPoolThreads, stage, st>>>(jq, none, Hkv, N, d, bs, units);
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ scores
 __device__ __forceinline__ float dot_fixed_order(const float* a, const float* b, int d, int bstride) {
   float acc = 0.0f;
@@ -106,49 +184,77 @@ __device__ __forceinline__ float dot_fixed_order(const float* a, const float* b,
   return acc;
 }
 
-// Prefill: one 32x32 (i, j) tile per CTA; rows of qbar/kbar staged in shared
-// memory (row pitch d+1 floats: no bank conflicts along j).
-__global__ void score_prefill_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
-                                     int nb, int d, float scale, float* __restrict__ s) {
+// Prefill: one 64x64 (i, j) tile per CTA of 256 threads; each thread owns a
+// 4x4 micro-tile (rows ty + 16a, columns tx + 16b), i.e. 16 independent
+// fixed-order dot products advanced together over the channel index.  Rows
+// of qbar/kbar are staged in shared memory with a pitch of d+1 floats.
+constexpr int kScoreTile = 64;
+
+__global__ void __launch_bounds__(256) score_prefill_kernel(const float* __restrict__ qbar,
+                                                            const float* __restrict__ kbar, int nb, int d,
+                                                            float scale, float* __restrict__ s) {
   extern __shared__ float sm[];
   const int pitch = d + 1;
   float* qs = sm;
-  float* ks = sm + 32 * pitch;
+  float* ks = sm + kScoreTile * pitch;
   const int ti = blockIdx.y, tj = blockIdx.x;
   const int64_t bg = blockIdx.z;
-  const int tx = threadIdx.x, ty = threadIdx.y;   // 32 x 8
-  const int i0 = ti * 32, j0 = tj * 32;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;   // 16 x 16
+  const int i0 = ti * kScoreTile, j0 = tj * kScoreTile;
   float* srow = s + bg * nb * static_cast<int64_t>(nb);
-  if (j0 > i0 + 31) {   // tile entirely above the diagonal
-    for (int r = ty; r < 32; r += 8) {
-      const int i = i0 + r, j = j0 + tx;
+  if (j0 > i0 + kScoreTile - 1) {   // tile entirely above the diagonal
+    for (int e = threadIdx.x; e < kScoreTile * kScoreTile; e += blockDim.x) {
+      const int i = i0 + e / kScoreTile, j = j0 + e % kScoreTile;
       if (i < nb && j < nb) srow[static_cast<int64_t>(i) * nb + j] = -INFINITY;
     }
     return;
   }
-  for (int r = ty; r < 32; r += 8) {
-    for (int c = tx; c < d; c += 32) {
-      const int i = i0 + r, j = j0 + r;
-      qs[r * pitch + c] = (i < nb) ? qbar[(bg * nb + i) * d + c] : 0.0f;
-      ks[r * pitch + c] = (j < nb) ? kbar[(bg * nb + j) * d + c] : 0.0f;
-    }
+  for (int e = threadIdx.x; e < kScoreTile * d; e += blockDim.x) {
+    const int r = e / d, c = e % d;
+    const int i = i0 + r, j = j0 + r;
+    qs[r * pitch + c] = (i < nb) ? qbar[(bg * nb + i) * d + c] : 0.0f;
+    ks[r * pitch + c] = (j < nb) ? kbar[(bg * nb + j) * d + c] : 0.0f;
   }
   __syncthreads();
-  for (int r = ty; r < 32; r += 8) {
-    const int i = i0 + r, j = j0 + tx;
-    if (i >= nb || j >= nb) continue;
-    float v = -INFINITY;
-    if (j <= i) v = __fmul_rn(dot_fixed_order(qs + r * pitch, ks + tx * pitch, d, 1), scale);
-    srow[static_cast<int64_t>(i) * nb + j] = v;
+  float acc[4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
+  for (int c = 0; c < d; ++c) {
+    float qv[4], kv[4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) qv[a] = qs[(ty + 16 * a) * pitch + c];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) kv[b] = ks[(tx + 16 * b) * pitch + c];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) acc[a][b] = __fadd_rn(acc[a][b], __fmul_rn(qv[a], kv[b]));
+  }
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    const int i = i0 + ty + 16 * a;
+    if (i >= nb) continue;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int j = j0 + tx + 16 * b;
+      if (j >= nb) continue;
+      srow[static_cast<int64_t>(i) * nb + j] = (j <= i) ? __fmul_rn(acc[a][b], scale) : -INFINITY;
+    }
   }
 }
 
 cudaError_t launch_score_prefill(const float* qbar, const float* kbar, int B, int Hkv, int nb, int d,
                                  float scale, float* s, cudaStream_t st) {
-  dim3 grid((nb + 31) / 32, (nb + 31) / 32, B * Hkv);
-  dim3 block(32, 8);
-  const size_t smem = 2 * 32 * (d + 1) * sizeof(float);
-  score_prefill_kernel<<<grid, block, smem, st>>>(qbar, kbar, nb, d, scale, s);
+  dim3 grid((nb + kScoreTile - 1) / kScoreTile, (nb + kScoreTile - 1) / kScoreTile, B * Hkv);
+  const size_t smem = 2 * kScoreTile * (d + 1) * sizeof(float);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(score_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  score_prefill_kernel<<<grid, 256, smem, st>>>(qbar, kbar, nb, d, scale, s);
   return cudaGetLastError();
 }
 
@@ -422,10 +528,205 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restr
   if (count_out && lane == 0) count_out[r] = run_sel;
 }
 
+// Warp-per-row variant for rows of at most 32*KPL candidates: lane l holds
+// candidates e*32 + l (e < KPL) in registers, loaded with coalesced reads.
+// The key T of the k-th best candidate is found bit by bit from the most
+// significant end (the largest T with at least k keys >= T), counting with
+// warp reductions; then the warp walks e = 0, 1, ... (index order), taking
+// every key > T and the lowest-index keys equal to T, and writes them at
+// ballot prefix positions -- already ascending.
+template <int KPL>
+__global__ void __launch_bounds__(128) topk_warp_kernel(const float* __restrict__ scores, int rows, int ncols,
+                                                        int mode, int kb, int* __restrict__ idx_out, int idx_stride,
+                                                        int* __restrict__ count_out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  int ncand, forced;
+  if (mode == 0) {
+    ncand = static_cast<int>(r % ncols);
+    forced = ncand;
+  } else if (mode == 1) {
+    ncand = ncols - 1;
+    forced = ncols - 1;
+  } else {
+    ncand = ncols;
+    forced = -1;
+  }
+  const float* srow = scores + r * ncols;
+  uint32_t key[KPL];
+#pragma unroll
+  for (int e = 0; e < KPL; ++e) {
+    const int j = e * 32 + lane;
+    key[e] = (j < ncand) ? order_key(__ldg(srow + j)) : 0u;
+  }
+  const int take = min(kb, ncand);
+  const bool take_all = (take == ncand);
+  uint32_t thresh = 0u;
+  int remaining = take;     // how many keys equal to thresh are taken
+  if (!take_all && take > 0) {
+    uint32_t prefix = 0u;
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = prefix | (1u << bit);
+      int cnt = 0;
+#pragma unroll
+      for (int e = 0; e < KPL; ++e) cnt += (e * 32 + lane < ncand && key[e] >= cand) ? 1 : 0;
+      cnt = __reduce_add_sync(0xffffffffu, cnt);
+      if (cnt >= take) prefix = cand;
+    }
+    thresh = prefix;
+    int gt = 0;
+#pragma unroll
+    for (int e = 0; e < KPL; ++e) gt += (e * 32 + lane < ncand && key[e] > thresh) ? 1 : 0;
+    gt = __reduce_add_sync(0xffffffffu, gt);
+    remaining = take - gt;
+  }
+  int* out = idx_out + r * idx_stride;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  int run_sel = 0, run_tie = 0;
+#pragma unroll
+  for (int e = 0; e < KPL; ++e) {
+    const int j = e * 32 + lane;
+    const bool valid = j < ncand;
+    bool gt, tie;
+    if (take_all) {
+      gt = valid;
+      tie = false;
+    } else if (take == 0) {
+      gt = false;
+      tie = false;
+    } else {
+      gt = valid && key[e] > thresh;
+      tie = valid && key[e] == thresh;
+    }
+    const unsigned tb = __ballot_sync(0xffffffffu, tie);
+    const bool sel = gt || (tie && run_tie + __popc(tb & lt_mask) < remaining);
+    const unsigned sb = __ballot_sync(0xffffffffu, sel);
+    if (sel) out[run_sel + __popc(sb & lt_mask)] = j;
+    run_sel += __popc(sb);
+    run_tie += __popc(tb);
+  }
+  int n = run_sel;
+  if (forced >= 0) {
+    if (lane == 0) out[n] = forced;
+    ++n;
+  }
+  for (int t = n + lane; t < idx_stride; t += 32) out[t] = -1;
+  if (count_out && lane == 0) count_out[r] = n;
+}
+
+// CTA-per-row variant for long rows (up to 256*KPT candidates): the same
+// bitwise threshold search, each thread holding KPT candidates (coalesced,
+// j = e*256 + tid), the per-bit counts summed over the eight warps through a
+// double-buffered shared array; warp 0 then writes the kept list in index
+// order from the keys staged in shared memory.
+template <int KPT>
+__global__ void __launch_bounds__(256) topk_cta_kernel(const float* __restrict__ scores, int ncols, int mode, int kb,
+                                                       int* __restrict__ idx_out, int idx_stride,
+                                                       int* __restrict__ count_out) {
+  __shared__ uint32_t skeys[256 * KPT];
+  __shared__ int cnts[2][8];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t r = blockIdx.x;
+  int ncand, forced;
+  if (mode == 0) {
+    ncand = static_cast<int>(r % ncols);
+    forced = ncand;
+  } else if (mode == 1) {
+    ncand = ncols - 1;
+    forced = ncols - 1;
+  } else {
+    ncand = ncols;
+    forced = -1;
+  }
+  const float* srow = scores + r * ncols;
+  uint32_t key[KPT];
+#pragma unroll
+  for (int e = 0; e < KPT; ++e) {
+    const int j = e * 256 + tid;
+    key[e] = (j < ncand) ? order_key(__ldg(srow + j)) : 0u;
+    skeys[j] = key[e];
+  }
+  const int take = min(kb, ncand);
+  const bool take_all = (take == ncand);
+  uint32_t thresh = 0u;
+  int remaining = take;
+  __syncthreads();
+  if (!take_all && take > 0) {
+    uint32_t prefix = 0u;
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = prefix | (1u << bit);
+      int c = 0;
+#pragma unroll
+      for (int e = 0; e < KPT; ++e) c += (e * 256 + tid < ncand && key[e] >= cand) ? 1 : 0;
+      c = __reduce_add_sync(0xffffffffu, c);
+      if (lane == 0) cnts[bit & 1][warp] = c;
+      __syncthreads();
+      int total = 0;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) total += cnts[bit & 1][w];
+      if (total >= take) prefix = cand;
+    }
+    thresh = prefix;
+    int c = 0;
+#pragma unroll
+    for (int e = 0; e < KPT; ++e) c += (e * 256 + tid < ncand && key[e] > thresh) ? 1 : 0;
+    c = __reduce_add_sync(0xffffffffu, c);
+    __syncthreads();   // everyone is done reading cnts of the last bit
+    if (lane == 0) cnts[0][warp] = c;
+    __syncthreads();
+    int gt = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) gt += cnts[0][w];
+    remaining = take - gt;
+  }
+  if (warp != 0) return;
+  int* out = idx_out + r * idx_stride;
+  int run_sel = 0, run_tie = 0;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int base = 0; base < ncand; base += 32) {
+    const int j = base + lane;
+    const bool valid = j < ncand;
+    const uint32_t k = valid ? skeys[j] : 0u;
+    bool gt, tie;
+    if (take_all) {
+      gt = valid;
+      tie = false;
+    } else if (take == 0) {
+      gt = false;
+      tie = false;
+    } else {
+      gt = valid && k > thresh;
+      tie = valid && k == thresh;
+    }
+    const unsigned tb = __ballot_sync(0xffffffffu, tie);
+    const bool sel = gt || (tie && run_tie + __popc(tb & lt_mask) < remaining);
+    const unsigned sb = __ballot_sync(0xffffffffu, sel);
+    if (sel) out[run_sel + __popc(sb & lt_mask)] = j;
+    run_sel += __popc(sb);
+    run_tie += __popc(tb);
+  }
+  int n = run_sel;
+  if (forced >= 0) {
+    if (lane == 0) out[n] = forced;
+    ++n;
+  }
+  for (int t = n + lane; t < idx_stride; t += 32) out[t] = -1;
+  if (count_out && lane == 0) count_out[r] = n;
+}
+
 cudaError_t launch_topk(const float* scores, int rows, int ncols, int mode, int kb, int* idx_out,
                         int idx_stride, int* count_out, cudaStream_t st) {
-  const size_t smem = static_cast<size_t>(ncols) * sizeof(uint32_t);
-  topk_kernel<<<rows, kTopkThreads, smem, st>>>(scores, ncols, mode, kb, idx_out, idx_stride, count_out);
+  if (ncols <= 32 * 16) {
+    const int warps = 4;
+    const unsigned grid = static_cast<unsigned>((rows + warps - 1) / warps);
+    topk_warp_kernel<16><<<grid, 32 * warps, 0, st>>>(scores, rows, ncols, mode, kb, idx_out, idx_stride, count_out);
+  } else if (ncols <= 256 * 8) {
+    topk_cta_kernel<8><<<rows, 256, 0, st>>>(scores, ncols, mode, kb, idx_out, idx_stride, count_out);
+  } else {
+    const size_t smem = static_cast<size_t>(ncols) * sizeof(uint32_t);
+    topk_kernel<<<rows, kTopkThreads, smem, st>>>(scores, ncols, mode, kb, idx_out, idx_stride, count_out);
+  }
   return cudaGetLastError();
 }
 
