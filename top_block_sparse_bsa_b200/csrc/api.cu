@@ -207,8 +207,11 @@ bsa_status_t bsa_score_blocks(const bsa_shape_t* s, int mode, const void* q, con
       return BSA_ERR_INVALID_ARG;
     if (!aligned16(k) || !aligned16(pooled_q_out) || !aligned16(pooled_k_out)) return BSA_ERR_INVALID_ARG;
     if (static_cast<int64_t>(nb) * nb >= (1ll << 31)) return BSA_ERR_UNSUPPORTED;
+    uint32_t* status = nullptr;
+    int sms = 0;
+    if ((st = device_state(&status, &sms)) != BSA_OK) return st;
     cudaError_t e = launch_pool_prefill(q, k, bf16, s->B, s->Hq, s->Hkv, s->Nk, s->d, s->block, pooled_q_out,
-                                        pooled_k_out, cs);
+                                        pooled_k_out, sms, status, cs);
     if (e == cudaSuccess) e = launch_score_prefill(pooled_q_out, pooled_k_out, s->B, s->Hkv, nb, s->d, scale, scores, cs);
     return cuda_status(e);
   }

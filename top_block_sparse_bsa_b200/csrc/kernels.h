@@ -11,7 +11,7 @@ namespace bsa {
 cudaError_t launch_pool(const void* src, bool bf16, int B, int Hsrc, int Hgroups, int heads_sum, int N,
                         int d, int bs, float* out, cudaStream_t st);
 cudaError_t launch_pool_prefill(const void* q, const void* k, bool bf16, int B, int Hq, int Hkv, int N, int d,
-                                int bs, float* qbar, float* kbar, cudaStream_t st);
+                                int bs, float* qbar, float* kbar, int num_sms, uint32_t* status, cudaStream_t st);
 cudaError_t launch_score_prefill(const float* qbar, const float* kbar, int B, int Hkv, int nb, int d,
                                  float scale, float* s, cudaStream_t st);
 cudaError_t launch_score_decode(const void* q, bool bf16, const float* kbar, int B, int Hq, int Hkv,

@@ -49,9 +49,21 @@ struct Vec8<float> {
 
 // unit u = (b, g, j): rows base + hh*N + t for hh < heads_sum, t < bs,
 // base = ((b*Hsrc + g*heads_sum)*N + j*bs).  out[u][c] = sum / (heads_sum*bs).
-template <typename T>
-__global__ void pool_kernel(const T* __restrict__ src, int B, int Hsrc, int Hgroups, int heads_sum,
-                            int N, int d, int bs, float* __restrict__ out) {
+// One thread per (unit, 8-channel group).  Rows are read in batches of RB
+// rows whose loads are all issued before the batch is summed in order, so a
+// thread has RB 16-byte (bf16) loads in flight instead of one.
+struct PoolJob {
+  const void* src;
+  int Hsrc, heads_sum;
+  float* out;
+};
+
+template <typename T, int RB>
+__global__ void __launch_bounds__(256) pool_kernel(PoolJob job0, PoolJob job1, int B, int Hgroups, int N, int d,
+                                                   int bs) {
+  const PoolJob job = blockIdx.y ? job1 : job0;
+  if (job.src == nullptr) return;
+  const T* src = static_cast<const T*>(job.src);
   const int lanes_per_unit = d / 8;
   const int64_t gtid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t unit = gtid / lanes_per_unit;
@@ -62,118 +74,163 @@ __global__ void pool_kernel(const T* __restrict__ src, int B, int Hsrc, int Hgro
   const int64_t b = unit / (static_cast<int64_t>(Hgroups) * nb);
   const int64_t g = (unit / nb) % Hgroups;
   const int64_t j = unit % nb;
-  const int64_t base = ((b * Hsrc + g * heads_sum) * N + j * bs) * d + cg * 8;
+  const int64_t base = ((b * job.Hsrc + g * job.heads_sum) * N + j * bs) * d + cg * 8;
   float acc[8];
 #pragma unroll
   for (int c = 0; c < 8; ++c) acc[c] = 0.0f;
-  for (int hh = 0; hh < heads_sum; ++hh) {
+  for (int hh = 0; hh < job.heads_sum; ++hh) {
     const T* p = src + base + static_cast<int64_t>(hh) * N * d;
-#pragma unroll 8
-    for (int t = 0; t < bs; ++t) {
-      float x[8];
-      Vec8<T>::load(p + static_cast<int64_t>(t) * d, x);
+    for (int t0 = 0; t0 < bs; t0 += RB) {
+      float x[RB][8];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) acc[c] = __fadd_rn(acc[c], x[c]);
+      for (int t = 0; t < RB; ++t) Vec8<T>::load(p + static_cast<int64_t>(t0 + t) * d, x[t]);
+#pragma unroll
+      for (int t = 0; t < RB; ++t)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[c] = __fadd_rn(acc[c], x[t][c]);
     }
   }
-  const float div = static_cast<float>(heads_sum * bs);
-  float* o = out + unit * d + cg * 8;
+  const float div = static_cast<float>(job.heads_sum * bs);
+  float* o = job.out + unit * d + cg * 8;
 #pragma unroll
   for (int c = 0; c < 8; ++c) o[c] = __fdiv_rn(acc[c], div);
 }
 
-// Staged variant for bf16 units of at most kPoolStageBytes: one CTA per unit
-// copies the unit's rows (heads_sum runs of bs contiguous rows) into shared
-// memory with every 16-byte load in flight at once, then thread c sums column
-// c over the rows in the fixed order (heads ascending, tokens ascending).
-// blockIdx.y selects the job (a launch may carry two).
-constexpr int kPoolThreads = 256;
-constexpr int kPoolStageBytes = 64 * 1024;
-
-struct PoolJob {
-  const __nv_bfloat16* src;
-  int Hsrc, heads_sum;
-  float* out;
-};
-
-__global__ void __launch_bounds__(kPoolThreads) pool_staged_kernel(PoolJob job0, PoolJob job1, int Hgroups, int N,
-                                                                   int d, int bs, int64_t units) {
-  extern __shared__ __align__(16) uint8_t pool_smem[];
-  const PoolJob job = blockIdx.y ? job1 : job0;
-  if (job.src == nullptr) return;
-  const int nb = N / bs;
-  for (int64_t unit = blockIdx.x; unit < units; unit += gridDim.x) {
-    const int64_t b = unit / (static_cast<int64_t>(Hgroups) * nb);
-    const int64_t g = (unit / nb) % Hgroups;
-    const int64_t j = unit % nb;
-    const int run = bs * d;                 // elements of one head's run
-    const int run16 = run / 8;              // 16-byte chunks of one run
-    const int chunks = run16 * job.heads_sum;
-    uint4* stage = reinterpret_cast<uint4*>(pool_smem);
-    __syncthreads();                        // previous unit fully consumed
-    for (int e = threadIdx.x; e < chunks; e += kPoolThreads) {
-      const int hh = e / run16, w = e % run16;
-      const __nv_bfloat16* p = job.src + ((b * job.Hsrc + g * job.heads_sum + hh) * static_cast<int64_t>(N) + j * bs) * d;
-      stage[e] = __ldg(reinterpret_cast<const uint4*>(p) + w);
-    }
-    __syncthreads();
-    const __nv_bfloat16* sv = reinterpret_cast<const __nv_bfloat16*>(pool_smem);
-    const int rows = job.heads_sum * bs;   // a multiple of 16 (bs is 64 or 128)
-    for (int c = threadIdx.x; c < d; c += kPoolThreads) {
-      float acc = 0.0f;
-      for (int r = 0; r < rows; r += 16) {
-        float x[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u) x[u] = __bfloat162float(sv[(r + u) * d + c]);
-#pragma unroll
-        for (int u = 0; u < 16; ++u) acc = __fadd_rn(acc, x[u]);
-      }
-      job.out[unit * d + c] = __fdiv_rn(acc, static_cast<float>(rows));
-    }
-  }
-}
-
-template <typename T>
-static cudaError_t launch_pool_t(const void* src, int B, int Hsrc, int Hgroups, int heads_sum, int N,
-                                 int d, int bs, float* out, cudaStream_t st) {
+static cudaError_t launch_pool_jobs(const PoolJob& j0, const PoolJob& j1, bool bf16, int B, int Hgroups, int N, int d,
+                                    int bs, cudaStream_t st) {
   const int64_t threads = static_cast<int64_t>(B) * Hgroups * (N / bs) * (d / 8);
   const int tpb = 256;
-  const int64_t blocks = (threads + tpb - 1) / tpb;
-  pool_kernel<T><<<static_cast<unsigned>(blocks), tpb, 0, st>>>(
-      static_cast<const T*>(src), B, Hsrc, Hgroups, heads_sum, N, d, bs, out);
+  const dim3 grid(static_cast<unsigned>((threads + tpb - 1) / tpb), j1.src ? 2u : 1u);
+  if (bf16) {
+    if (bs % 32 == 0)
+      pool_kernel<__nv_bfloat16, 32><<<grid, tpb, 0, st>>>(j0, j1, B, Hgroups, N, d, bs);
+    else
+      pool_kernel<__nv_bfloat16, 1><<<grid, tpb, 0, st>>>(j0, j1, B, Hgroups, N, d, bs);
+  } else {
+    if (bs % 16 == 0)
+      pool_kernel<float, 16><<<grid, tpb, 0, st>>>(j0, j1, B, Hgroups, N, d, bs);
+    else
+      pool_kernel<float, 1><<<grid, tpb, 0, st>>>(j0, j1, B, Hgroups, N, d, bs);
+  }
   return cudaGetLastError();
+}
+
+// Streamed variant (persistent, one CTA per SM): a producer thread copies each
+// unit's rows (heads_sum runs of bs*d contiguous elements) into one of two
+// shared-memory buffers with bulk copies while 128 threads sum the previous
+// unit, column c by thread c, rows in the fixed order.  Units of the query
+// job come first, then those of the key job.
+constexpr int kPoolStreamBytes = 64 * 1024;
+
+template <typename T>
+__global__ void __launch_bounds__(160, 1) pool_stream_kernel(PoolJob jq, PoolJob jk, int B, int Hgroups, int N, int d,
+                                                             int bs, uint32_t* status) {
+  extern __shared__ uint8_t psmem_raw[];
+  uint8_t* psmem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(psmem_raw) + 127) & ~uintptr_t(127));
+  __shared__ __align__(8) uint64_t bars[4];   // full[2], empty[2]
+  __shared__ int abort_flag;
+  const uint32_t sb = smem_u32(psmem);
+  auto bar = [&](int i) -> uint32_t { return smem_u32(&bars[i]); };
+  const int nb = N / bs;
+  const int64_t units_per_job = static_cast<int64_t>(B) * Hgroups * nb;
+  const int64_t units = units_per_job * (jk.src ? 2 : 1);
+  if (threadIdx.x == 0) {
+    mbar_init(bar(0), 1);
+    mbar_init(bar(1), 1);
+    mbar_init(bar(2), 128);
+    mbar_init(bar(3), 128);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  volatile int* ab = &abort_flag;
+  const int warp = threadIdx.x >> 5;
+  if (warp == 4) {
+    if ((threadIdx.x & 31) == 0) {
+      int k = 0;
+      int issued = 0;
+      for (int64_t u = blockIdx.x; u < units; u += gridDim.x, ++k) {
+        const bool isk = u >= units_per_job;
+        const PoolJob& job = isk ? jk : jq;
+        const int64_t unit = isk ? u - units_per_job : u;
+        const int64_t b = unit / (static_cast<int64_t>(Hgroups) * nb);
+        const int64_t g = (unit / nb) % Hgroups;
+        const int64_t j = unit % nb;
+        const int buf = k & 1;
+        if (k >= 2 && !mbar_wait(bar(2 + buf), ((k >> 1) - 1) & 1, ab, status)) break;
+        const uint32_t run = static_cast<uint32_t>(bs) * d * sizeof(T);
+        mbar_arrive_expect_tx(bar(buf), run * job.heads_sum);
+        const T* src = static_cast<const T*>(job.src);
+        for (int hh = 0; hh < job.heads_sum; ++hh)
+          bulk_load(sb + buf * kPoolStreamBytes + hh * run,
+                    src + ((b * job.Hsrc + g * job.heads_sum + hh) * static_cast<int64_t>(N) + j * bs) * d, run,
+                    bar(buf));
+        ++issued;
+      }
+      if (*ab) {   // let the copies still in flight land before the CTA exits
+        for (int q = issued > 2 ? issued - 2 : 0; q < issued; ++q) mbar_drain(bar(q & 1), (q >> 1) & 1);
+      }
+    }
+  } else {
+    const int c = threadIdx.x;   // column
+    int k = 0;
+    for (int64_t u = blockIdx.x; u < units; u += gridDim.x, ++k) {
+      const bool isk = u >= units_per_job;
+      const PoolJob& job = isk ? jk : jq;
+      const int64_t unit = isk ? u - units_per_job : u;
+      const int buf = k & 1;
+      if (!mbar_wait(bar(buf), (k >> 1) & 1, ab, status)) break;
+      const T* sv = reinterpret_cast<const T*>(psmem + buf * kPoolStreamBytes);
+      const int rows = job.heads_sum * bs;   // a multiple of 16
+      if (c < d) {
+        float acc = 0.0f;
+        for (int r = 0; r < rows; r += 16) {
+          float x[16];
+#pragma unroll
+          for (int t = 0; t < 16; ++t) x[t] = static_cast<float>(sv[(r + t) * d + c]);
+#pragma unroll
+          for (int t = 0; t < 16; ++t) acc = __fadd_rn(acc, x[t]);
+        }
+        job.out[unit * d + c] = __fdiv_rn(acc, static_cast<float>(rows));
+      }
+      mbar_arrive(bar(2 + buf));
+    }
+  }
+  __syncthreads();
 }
 
 cudaError_t launch_pool(const void* src, bool bf16, int B, int Hsrc, int Hgroups, int heads_sum, int N,
                         int d, int bs, float* out, cudaStream_t st) {
-  return bf16 ? launch_pool_t<__nv_bfloat16>(src, B, Hsrc, Hgroups, heads_sum, N, d, bs, out, st)
-              : launch_pool_t<float>(src, B, Hsrc, Hgroups, heads_sum, N, d, bs, out, st);
+  const PoolJob j0{src, Hsrc, heads_sum, out};
+  const PoolJob none{nullptr, 0, 0, nullptr};
+  return launch_pool_jobs(j0, none, bf16, B, Hgroups, N, d, bs, st);
 }
 
-// Prefill: keys (heads_sum 1) and grouped queries (heads_sum G), staged when a
-// query unit fits the stage; otherwise the plain per-thread kernel.
+// Prefill: grouped queries (heads_sum G) and keys (heads_sum 1) in one launch
+// of the streamed kernel when a query unit fits a buffer and d <= 128.
 cudaError_t launch_pool_prefill(const void* q, const void* k, bool bf16, int B, int Hq, int Hkv, int N, int d,
-                                int bs, float* qbar, float* kbar, cudaStream_t st) {
-  const int G = Hq / Hkv;
-  const size_t stage = static_cast<size_t>(G) * bs * d * 2;
-  if (!bf16 || stage > kPoolStageBytes || d % 8 != 0) {
-    cudaError_t e = launch_pool(k, bf16, B, Hkv, Hkv, 1, N, d, bs, kbar, st);
-    if (e == cudaSuccess) e = launch_pool(q, bf16, B, Hq, Hkv, G, N, d, bs, qbar, st);
-    return e;
+                                int bs, float* qbar, float* kbar, int num_sms, uint32_t* status, cudaStream_t st) {
+  const PoolJob jq{q, Hq, Hq / Hkv, qbar};
+  const PoolJob jk{k, Hkv, 1, kbar};
+  const size_t esize = bf16 ? 2 : 4;
+  const size_t unit_bytes = static_cast<size_t>(Hq / Hkv) * bs * d * esize;
+  if (unit_bytes > kPoolStreamBytes || d > 128 || bs % 16 != 0 || (static_cast<size_t>(bs) * d * esize) % 16 != 0)
+    return launch_pool_jobs(jq, jk, bf16, B, Hkv, N, d, bs, st);
+  const size_t smem = 2 * kPoolStreamBytes + 128;
+  const int64_t units = 2ll * B * Hkv * (N / bs);
+  const unsigned grid = static_cast<unsigned>(units < num_sms ? units : num_sms);
+  cudaError_t e;
+  if (bf16) {
+    e = cudaFuncSetAttribute(pool_stream_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    pool_stream_kernel<__nv_bfloat16><<<grid, 160, smem, st>>>(jq, jk, B, Hkv, N, d, bs, status);
+  } else {
+    e = cudaFuncSetAttribute(pool_stream_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    pool_stream_kernel<float><<<grid, 160, smem, st>>>(jq, jk, B, Hkv, N, d, bs, status);
   }
-  cudaError_t e = cudaFuncSetAttribute(pool_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(stage));
-  if (e != cudaSuccess) return e;
-  const int64_t units = static_cast<int64_t>(B) * Hkv * (N / bs);
-  PoolJob jk{static_cast<const __nv_bfloat16*>(k), Hkv, 1, kbar};
-  PoolJob jq{static_cast<const __nv_bfloat16*>(q), Hq, G, qbar};
-  const PoolJob none{nullptr, 0, 0, nullptr};
-  const unsigned gx = static_cast<unsigned>(units < 65535 ? units : 65535);
-  pool_staged_kernel<<<dim3(gx, 1), kPoolThreads, static_cast<size_t>(bs) * d * 2, st>>>(jk, none, Hkv, N, d, bs,
-                                                                                          units);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  pool_staged_kernel<<<dim3(gx, 1), kPoolThreads, stage, st>>>(jq, none, Hkv, N, d, bs, units);
   return cudaGetLastError();
 }
 
@@ -187,14 +244,14 @@ __device__ __forceinline__ float dot_fixed_order(const float* a, const float* b,
 // Prefill: one 64x64 (i, j) tile per CTA of 256 threads; each thread owns a
 // 4x4 micro-tile (rows ty + 16a, columns tx + 16b), i.e. 16 independent
 // fixed-order dot products advanced together over the channel index.  Rows
-// of qbar/kbar are staged in shared memory with a pitch of d+1 floats.
+// of qbar/kbar are staged in shared memory with a pitch of d+4 floats.
 constexpr int kScoreTile = 64;
 
 __global__ void __launch_bounds__(256) score_prefill_kernel(const float* __restrict__ qbar,
                                                             const float* __restrict__ kbar, int nb, int d,
                                                             float scale, float* __restrict__ s) {
-  extern __shared__ float sm[];
-  const int pitch = d + 1;
+  extern __shared__ __align__(16) float sm[];
+  const int pitch = d + 4;   // 16-byte aligned rows for the asynchronous copies
   float* qs = sm;
   float* ks = sm + kScoreTile * pitch;
   const int ti = blockIdx.y, tj = blockIdx.x;
@@ -209,11 +266,20 @@ __global__ void __launch_bounds__(256) score_prefill_kernel(const float* __restr
     }
     return;
   }
-  for (int e = threadIdx.x; e < kScoreTile * d; e += blockDim.x) {
-    const int r = e / d, c = e % d;
-    const int i = i0 + r, j = j0 + r;
-    qs[r * pitch + c] = (i < nb) ? qbar[(bg * nb + i) * d + c] : 0.0f;
-    ks[r * pitch + c] = (j < nb) ? kbar[(bg * nb + j) * d + c] : 0.0f;
+  {
+    // 64 rows x d floats per matrix with 16-byte asynchronous copies (every
+    // copy of a thread in flight at once); rows past nb are zero-filled
+    const int q4 = d / 4;
+    for (int e = threadIdx.x; e < kScoreTile * q4; e += blockDim.x) {
+      const int r = e / q4, c4 = e % q4;
+      float* qd = qs + r * pitch + c4 * 4;
+      float* kd = ks + r * pitch + c4 * 4;
+      if (i0 + r < nb) cp_async16(smem_u32(qd), qbar + (bg * nb + i0 + r) * d + c4 * 4);
+      else *reinterpret_cast<float4*>(qd) = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (j0 + r < nb) cp_async16(smem_u32(kd), kbar + (bg * nb + j0 + r) * d + c4 * 4);
+      else *reinterpret_cast<float4*>(kd) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    cp_async_wait_all();
   }
   __syncthreads();
   float acc[4][4];
@@ -247,8 +313,9 @@ __global__ void __launch_bounds__(256) score_prefill_kernel(const float* __restr
 
 cudaError_t launch_score_prefill(const float* qbar, const float* kbar, int B, int Hkv, int nb, int d,
                                  float scale, float* s, cudaStream_t st) {
+  if (d % 4 != 0 || d > 128) return cudaErrorInvalidValue;
   dim3 grid((nb + kScoreTile - 1) / kScoreTile, (nb + kScoreTile - 1) / kScoreTile, B * Hkv);
-  const size_t smem = 2 * kScoreTile * (d + 1) * sizeof(float);
+  const size_t smem = 2 * kScoreTile * (d + 4) * sizeof(float);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(score_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
