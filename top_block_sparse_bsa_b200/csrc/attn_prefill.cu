@@ -63,8 +63,8 @@ constexpr uint32_t kSmemQ = 0;
 constexpr uint32_t kSmemK = kSmemQ + 2 * kTileBytes;
 constexpr uint32_t kSmemV = kSmemK + kStages * kTileBytes;
 constexpr uint32_t kSmemBar = kSmemV + kStages * kTileBytes;
-constexpr int kCtrlRegs = 64;       // warps 0-3 after setmaxnreg.dec
-constexpr int kMathRegs = 216;      // warps 4-11 after setmaxnreg.inc (128*64 + 256*216 <= 384*168)
+constexpr int kCtrlRegs = 96;       // warps 0-3 after setmaxnreg.dec
+constexpr int kMathRegs = 200;      // warps 4-11 after setmaxnreg.inc (128*96 + 256*200 <= 384*168)
 
 enum {
   BAR_QF = 0,
@@ -82,7 +82,7 @@ enum {
   BAR_AB = BAR_LE + 2,
   NUM_BARS
 };
-constexpr uint32_t kListConsumers = 2 + 8;   // producer, MMA, one lane per softmax warp
+constexpr uint32_t kListConsumers = 3 + 8;   // two producers, MMA, one lane per softmax warp
 
 struct ItemInfo {
   int n, ntiles, b, g, i, tile0, pad0, pad1;
@@ -153,11 +153,21 @@ __device__ __forceinline__ void softmax_step(uint32_t t_s, uint32_t t_o, bool fi
   // row maximum of the raw scores per block (the scale is positive and the
   // bias is constant over a block, so the maximum commutes with both)
   constexpr int H0 = (BS == 64 && KEYS == 128) ? 64 : KEYS;
-  float mx0 = -INFINITY, mx1 = -INFINITY;
+  // tree reductions: 8 independent chains, then a short combine
+  float m8[8];
 #pragma unroll
-  for (int c = 0; c < H0; ++c) mx0 = fmaxf(mx0, __uint_as_float(v[c]));
+  for (int a = 0; a < 8; ++a) m8[a] = -INFINITY;
 #pragma unroll
-  for (int c = H0; c < KEYS; ++c) mx1 = fmaxf(mx1, __uint_as_float(v[c]));
+  for (int c = 0; c < H0; ++c) m8[c & 7] = fmaxf(m8[c & 7], __uint_as_float(v[c]));
+  const float mx0 = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+  float mx1 = -INFINITY;
+  if constexpr (H0 < KEYS) {
+#pragma unroll
+    for (int a = 0; a < 8; ++a) m8[a] = -INFINITY;
+#pragma unroll
+    for (int c = H0; c < KEYS; ++c) m8[c & 7] = fmaxf(m8[c & 7], __uint_as_float(v[c]));
+    mx1 = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+  }
   float mx = fmaf(mx0, scale_log2, bias0);
   if (H0 < KEYS) mx = fmaxf(mx, fmaf(mx1, scale_log2, bias1));
   const float m_new = fmaxf(m_run, mx);
@@ -178,7 +188,7 @@ __device__ __forceinline__ void softmax_step(uint32_t t_s, uint32_t t_o, bool fi
   l_run *= alpha;
   m_run = m_use;
   const float off0 = bias0 - m_sub, off1 = bias1 - m_sub;
-  float sum = 0.0f;
+  float s4[4] = {0.0f, 0.0f, 0.0f, 0.0f};   // independent partial row sums
 #pragma unroll
   for (int half = 0; half < KEYS / 64; ++half) {
     uint32_t pk[32];
@@ -188,12 +198,12 @@ __device__ __forceinline__ void softmax_step(uint32_t t_s, uint32_t t_o, bool fi
       const float off = (c < H0) ? off0 : off1;
       const float p0 = fast_exp2(fmaf(__uint_as_float(v[c]), scale_log2, off));
       const float p1 = fast_exp2(fmaf(__uint_as_float(v[c + 1]), scale_log2, off));
-      sum += p0 + p1;
+      s4[e & 3] += p0 + p1;
       pk[e] = pack_bf16x2(p0, p1);
     }
     tmem_st32(t_s + half * 32, pk);
   }
-  l_run += sum;
+  l_run += (s4[0] + s4[1]) + (s4[2] + s4[3]);
   tmem_wait_st();
 }
 
@@ -321,10 +331,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(BAR_LF + buf));
     }
-  } else if (warp == 0) {
+  } else if (warp == 0 || warp == 3) {
     if (lane == 0) {
-      // ------------------------------------------------ TMA producer
-      int gs = 0, qcount = 0, k_issued = 0, v_issued = 0;
+      // ------------------------------------------------ TMA producers
+      // warp 0 loads Q and K, warp 3 loads V: the two rings drain at
+      // different points of the MMA order (K after S, V after O += P V), so
+      // separate threads keep a late V slot from holding back the next K.
+      const int kv = (warp == 3) ? 1 : 0;
+      const int full = kv ? BAR_VF : BAR_KF, empty = kv ? BAR_VE : BAR_KE;
+      const CUtensorMap* map = kv ? &tmV : &tmK;
+      const uint32_t ring = sbase + (kv ? kSmemV : kSmemK);
+      int gs = 0, qcount = 0;
       bool ok = true;
       for (int k = 0; ok; ++k) {
         const int item = blockIdx.x + k * gridDim.x;
@@ -335,23 +352,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n = inf->n;
         if (n > 0) {
           const int ntiles = inf->ntiles, tile0 = inf->tile0, b = inf->b, g = inf->g, i = inf->i;
-          if (qcount > 0 && !(ok = mbar_wait(bar(BAR_QE), (qcount - 1) & 1, abortp, p.status))) break;
-          uint32_t qbytes = 0;
-          for (int m = 0; m < ntiles; ++m)
-            for (int pc = 0; pc < 2; ++pc)
-              if ((tile0 + m) * 128 + pc * 64 < p.rows_per_unit) qbytes += 2 * 8192;
-          mbar_arrive_expect_tx(bar(BAR_QF), qbytes);
-          for (int m = 0; m < ntiles; ++m)
-            for (int pc = 0; pc < 2; ++pc) {
-              const int R0 = (tile0 + m) * 128 + pc * 64;
-              if (R0 >= p.rows_per_unit) continue;
-              const int h = g * p.G + R0 / BS;
-              const int y = (b * p.Hq + h) * p.N + i * BS + R0 % BS;
-              for (int hf = 0; hf < 2; ++hf)
-                tma_load_2d(sbase + kSmemQ + m * kTileBytes + hf * kHalfBytes + pc * 8192, &tmQ, bar(BAR_QF),
-                            hf * 64, y);
-            }
-          ++qcount;
+          if (kv == 0) {
+            if (qcount > 0 && !(ok = mbar_wait(bar(BAR_QE), (qcount - 1) & 1, abortp, p.status))) break;
+            uint32_t qbytes = 0;
+            for (int m = 0; m < ntiles; ++m)
+              for (int pc = 0; pc < 2; ++pc)
+                if ((tile0 + m) * 128 + pc * 64 < p.rows_per_unit) qbytes += 2 * 8192;
+            mbar_arrive_expect_tx(bar(BAR_QF), qbytes);
+            for (int m = 0; m < ntiles; ++m)
+              for (int pc = 0; pc < 2; ++pc) {
+                const int R0 = (tile0 + m) * 128 + pc * 64;
+                if (R0 >= p.rows_per_unit) continue;
+                const int h = g * p.G + R0 / BS;
+                const int y = (b * p.Hq + h) * p.N + i * BS + R0 % BS;
+                for (int hf = 0; hf < 2; ++hf)
+                  tma_load_2d(sbase + kSmemQ + m * kTileBytes + hf * kHalfBytes + pc * 8192, &tmQ, bar(BAR_QF),
+                              hf * 64, y);
+              }
+            ++qcount;
+          }
           const int kvrow0 = (b * p.Hkv + g) * p.N;
           const int nsteps = (BS == 64) ? (n + 1) / 2 : n;
           for (int s = 0; s < nsteps; ++s, ++gs) {
@@ -366,23 +385,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               jb[0] = inf->list[s];
               jb[1] = 0;
             }
-            const uint32_t bytes = static_cast<uint32_t>(nblk * BS) * 256u;
-            for (int kv = 0; kv < 2; ++kv) {
-              const int full = kv ? BAR_VF : BAR_KF, empty = kv ? BAR_VE : BAR_KE;
-              const uint32_t dst0 = sbase + (kv ? kSmemV : kSmemK) + slot * kTileBytes;
-              const CUtensorMap* map = kv ? &tmV : &tmK;
-              if (gs >= kStages && !(ok = mbar_wait(bar(empty + slot), (use - 1) & 1, abortp, p.status))) break;
-              mbar_arrive_expect_tx(bar(full + slot), bytes);
-              for (int bl = 0; bl < nblk; ++bl)
-                for (int r = 0; r < BS / 64; ++r) {
-                  const uint32_t rowoff = static_cast<uint32_t>(bl * BS + r * 64);
-                  const int y = kvrow0 + jb[bl] * BS + r * 64;
-                  for (int hf = 0; hf < 2; ++hf)
-                    tma_load_2d(dst0 + hf * kHalfBytes + rowoff * 128u, map, bar(full + slot), hf * 64, y);
-                }
-              if (kv) ++v_issued; else ++k_issued;
-            }
-            if (!ok) break;
+            if (gs >= kStages && !(ok = mbar_wait(bar(empty + slot), (use - 1) & 1, abortp, p.status))) break;
+            mbar_arrive_expect_tx(bar(full + slot), static_cast<uint32_t>(nblk * BS) * 256u);
+            const uint32_t dst0 = ring + slot * kTileBytes;
+            for (int bl = 0; bl < nblk; ++bl)
+              for (int r = 0; r < BS / 64; ++r) {
+                const uint32_t rowoff = static_cast<uint32_t>(bl * BS + r * 64);
+                const int y = kvrow0 + jb[bl] * BS + r * 64;
+                for (int hf = 0; hf < 2; ++hf)
+                  tma_load_2d(dst0 + hf * kHalfBytes + rowoff * 128u, map, bar(full + slot), hf * 64, y);
+              }
           }
           if (!ok) break;
         }
@@ -391,8 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (*abortp) {
         // let every copy this thread issued land before the CTA exits
         if (qcount > 0) mbar_drain(bar(BAR_QF), (qcount - 1) & 1);
-        for (int s = max(0, k_issued - kStages); s < k_issued; ++s) mbar_drain(bar(BAR_KF + s % kStages), (s / kStages) & 1);
-        for (int s = max(0, v_issued - kStages); s < v_issued; ++s) mbar_drain(bar(BAR_VF + s % kStages), (s / kStages) & 1);
+        for (int s = max(0, gs - kStages); s < gs; ++s) mbar_drain(bar(full + s % kStages), (s / kStages) & 1);
       }
     }
   } else if (warp == 1) {
@@ -401,22 +412,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t id_s128 = idesc_bf16_f32(128, 128, 0, 0);
       const uint32_t id_s64 = idesc_bf16_f32(128, 64, 0, 0);
       const uint32_t id_pv = idesc_bf16_f32(128, 128, 0, 1);
+      // Descriptors are built once; a k-step only adds its byte offset (>> 4)
+      // to the start-address field, so issuing an MMA is one add and the MMA.
+      const uint64_t q_desc0 = smem_desc_sw128(sbase + kSmemQ, 16, 1024);
+      const uint64_t k_desc0 = smem_desc_sw128(sbase + kSmemK, 16, 1024);
+      const uint64_t v_desc0 = smem_desc_sw128(sbase + kSmemV, kHalfBytes, 1024);
       auto issue_s = [&](int m, int slot, int keys) {
-        const uint32_t qa = sbase + kSmemQ + m * kTileBytes;
-        const uint32_t ka = sbase + kSmemK + slot * kTileBytes;
+        const uint64_t qd = q_desc0 + ((m * kTileBytes) >> 4);
+        const uint64_t kd = k_desc0 + ((slot * kTileBytes) >> 4);
         const uint32_t id = (keys == 128) ? id_s128 : id_s64;
+        const uint32_t d_tmem = tmem + m * 128;
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-          mma_ss(tmem + m * 128, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), id,
-                 kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+          mma_ss(d_tmem, qd + off, kd + off, id, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int m, int slot, int keys, bool acc) {
-        const uint32_t va = sbase + kSmemV + slot * kTileBytes;
-        for (int kk = 0; kk < keys / 16; ++kk)
-          mma_ts(tmem + 256 + m * 128, tmem + m * 128 + kk * 8, smem_desc_sw128(va + kk * 2048, kHalfBytes, 1024),
-                 id_pv, (acc || kk > 0) ? 1u : 0u);
+        const uint64_t vd = v_desc0 + ((slot * kTileBytes) >> 4);
+        const uint32_t d_tmem = tmem + 256 + m * 128;
+        const uint32_t a_tmem = tmem + m * 128;
+        if (keys == 128) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(d_tmem, a_tmem + kk * 8, vd + ((kk * 2048) >> 4), id_pv, (acc || kk > 0) ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ts(d_tmem, a_tmem + kk * 8, vd + ((kk * 2048) >> 4), id_pv, (acc || kk > 0) ? 1u : 0u);
+        }
       };
       int gs = 0, qcount = 0;
       int st[2] = {0, 0};        // completed S/P steps per tile
@@ -439,10 +463,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int s = 0; ok && s < nsteps; ++s, ++gs) {
             const int slot = gs % kStages, use = gs / kStages;
             const int pslot = (gs + kStages - 1) % kStages, puse = (gs - 1) / kStages;
-            if (!(ok = mbar_wait(bar(BAR_KF + slot), use & 1, abortp, p.status))) break;
-            tc_fence_after();
+            bool have_k = false;
             for (int m = 0; m < ntiles; ++m) {
               if (s > 0) {
+                // O += P V of the previous step first: it needs V and P, not K
                 if (m == 0 && !(ok = mbar_wait(bar(BAR_VF + pslot), puse & 1, abortp, p.status))) break;
                 if (!(ok = mbar_wait(bar(BAR_PF + m), (st[m] - 1) & 1, abortp, p.status))) break;
                 if (s == 1 && pv_items[m] > 0 &&
@@ -450,13 +474,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                   break;
                 tc_fence_after();
                 issue_pv(m, pslot, keys_of(s - 1), s - 1 > 0);
+                // the V slot is free as soon as the last tile's O += P V is done
+                if (m == ntiles - 1) tc_commit(bar(BAR_VE + pslot));
+              }
+              if (!have_k) {
+                if (!(ok = mbar_wait(bar(BAR_KF + slot), use & 1, abortp, p.status))) break;
+                tc_fence_after();
+                have_k = true;
               }
               issue_s(m, slot, keys_of(s));
               tc_commit(bar(BAR_SF + m));
               ++st[m];
             }
             if (!ok) break;
-            if (s > 0) tc_commit(bar(BAR_VE + pslot));
             tc_commit(bar(BAR_KE + slot));
           }
           if (!ok) break;
