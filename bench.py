@@ -142,6 +142,15 @@ class ClockSampler:
                 "power_w_max": max(s[3] for s in win) if win else None, "samples": len(win)}
 
 
+def wait_gpu(ev):
+    """Wait for a recorded event by polling with short sleeps, so that the
+    clock-sampling thread keeps the interpreter lock while the GPU works."""
+    import torch
+    while not ev.query():
+        time.sleep(0.0005)
+    torch.cuda.synchronize()
+
+
 def profile_traffic(kernel_file: str, summary_name: str):
     """Per-launch DRAM traffic of the kernel from a committed ncu summary, or
     None when absent or taken on a different kernel source."""
@@ -281,7 +290,7 @@ def run_prefill(args, world, rank, local, peaks, peak_src):
         step.attend(with_lse=False)
         kb_[s].record(stream)
     ev1.record(stream)
-    torch.cuda.synchronize()
+    wait_gpu(ev1)
     t_wall1 = time.time()
     if dist:
         dist.barrier()
@@ -460,7 +469,7 @@ def run_decode_like(args, world, rank, local, peaks, peak_src):
         ev[s][0].record(stream)
         run()
         ev[s][1].record(stream)
-    torch.cuda.synchronize()
+    wait_gpu(ev[-1][1])
     t1 = time.time()
     sampler.stop()
     us = statistics.mean(1e3 * a.elapsed_time(b) for a, b in ev)

@@ -151,25 +151,21 @@ __device__ __forceinline__ void softmax_step(uint32_t t_s, uint32_t t_o, bool fi
     }
   }
   // row maximum of the raw scores per block (the scale is positive and the
-  // bias is constant over a block, so the maximum commutes with both)
+  // bias is constant over a block, so the maximum commutes with both);
+  // three-input maxima in 8 independent chains
   constexpr int H0 = (BS == 64 && KEYS == 128) ? 64 : KEYS;
-  // tree reductions: 8 independent chains, then a short combine
-  float m8[8];
-#pragma unroll
-  for (int a = 0; a < 8; ++a) m8[a] = -INFINITY;
-#pragma unroll
-  for (int c = 0; c < H0; ++c) m8[c & 7] = fmaxf(m8[c & 7], __uint_as_float(v[c]));
-  const float mx0 = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-  float mx1 = -INFINITY;
-  if constexpr (H0 < KEYS) {
+  auto block_max = [&](int c0, int c1) {
+    float m8[8];
 #pragma unroll
     for (int a = 0; a < 8; ++a) m8[a] = -INFINITY;
 #pragma unroll
-    for (int c = H0; c < KEYS; ++c) m8[c & 7] = fmaxf(m8[c & 7], __uint_as_float(v[c]));
-    mx1 = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-  }
+    for (int c = c0; c < c1; c += 2)
+      m8[(c >> 1) & 7] = fmax3(m8[(c >> 1) & 7], __uint_as_float(v[c]), __uint_as_float(v[c + 1]));
+    return fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+  };
+  const float mx0 = block_max(0, H0);
   float mx = fmaf(mx0, scale_log2, bias0);
-  if (H0 < KEYS) mx = fmaxf(mx, fmaf(mx1, scale_log2, bias1));
+  if constexpr (H0 < KEYS) mx = fmaxf(mx, fmaf(block_max(H0, KEYS), scale_log2, bias1));
   const float m_new = fmaxf(m_run, mx);
   const bool need = m_new > m_run + kRescaleThreshold;
   const float m_use = need ? m_new : m_run;
@@ -187,23 +183,31 @@ __device__ __forceinline__ void softmax_step(uint32_t t_s, uint32_t t_o, bool fi
   }
   l_run *= alpha;
   m_run = m_use;
-  const float off0 = bias0 - m_sub, off1 = bias1 - m_sub;
-  float s4[4] = {0.0f, 0.0f, 0.0f, 0.0f};   // independent partial row sums
+  // p = 2^(s * scale*log2(e) + bias - m), two keys per packed FMA; packed
+  // partial row sums
+  const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
+  const uint64_t off0 = f2_pack(bias0 - m_sub, bias0 - m_sub), off1 = f2_pack(bias1 - m_sub, bias1 - m_sub);
+  uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};   // independent packed partial row sums (+0.0f pairs)
 #pragma unroll
   for (int half = 0; half < KEYS / 64; ++half) {
     uint32_t pk[32];
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
       const int c = half * 64 + 2 * e;
-      const float off = (c < H0) ? off0 : off1;
-      const float p0 = fast_exp2(fmaf(__uint_as_float(v[c]), scale_log2, off));
-      const float p1 = fast_exp2(fmaf(__uint_as_float(v[c + 1]), scale_log2, off));
-      s4[e & 3] += p0 + p1;
+      const uint64_t x = f2_fma(f2_pack(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), sc2,
+                                (c < H0) ? off0 : off1);
+      float x0, x1;
+      f2_unpack(x, x0, x1);
+      const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+      acc[e & 3] = f2_add(acc[e & 3], f2_pack(p0, p1));
       pk[e] = pack_bf16x2(p0, p1);
     }
     tmem_st32(t_s + half * 32, pk);
   }
-  l_run += (s4[0] + s4[1]) + (s4[2] + s4[3]);
+  float a0, a1, a2, a3;
+  f2_unpack(f2_add(acc[0], acc[1]), a0, a1);
+  f2_unpack(f2_add(acc[2], acc[3]), a2, a3);
+  l_run += (a0 + a1) + (a2 + a3);
   tmem_wait_st();
 }
 
@@ -247,9 +251,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar(BAR_SF + t), 1);
-      mbar_init(bar(BAR_PF + t), 128);
+      mbar_init(bar(BAR_PF + t), 4);    // one arrive per softmax warp
       mbar_init(bar(BAR_OF + t), 1);
-      mbar_init(bar(BAR_OE + t), 128);
+      mbar_init(bar(BAR_OE + t), 4);
       mbar_init(bar(BAR_LF + t), 1);
       mbar_init(bar(BAR_LE + t), kListConsumers);
     }
@@ -569,7 +573,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           softmax_dispatch<BS>(keys, j0 == i || j1 == i, t_s, t_o, s == 0, p.scale_log2, b0, b1, j0 == i, j1 == i,
                                tb, m_run, l_run);
           tc_fence_before();
-          mbar_arrive(bar(BAR_PF + t));
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(BAR_PF + t));
         }
         if (!ok) break;
         if (!(ok = warp_wait(bar(BAR_OF + t), oc & 1, abortp, p.status))) break;
@@ -587,7 +592,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             ob[ch * 16 + e] = pack_bf16x2(__uint_as_float(v[2 * e]) * inv, __uint_as_float(v[2 * e + 1]) * inv);
         }
         tc_fence_before();
-        mbar_arrive(bar(BAR_OE + t));   // O may be overwritten by the next item from here on
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(BAR_OE + t));   // O may be overwritten by the next item from here on
         if (valid) {
           uint4* dst = reinterpret_cast<uint4*>(p.o + orow_idx * kD);
 #pragma unroll
