@@ -325,18 +325,33 @@ cudaError_t launch_score_prefill(const float* qbar, const float* kbar, int B, in
   return cudaGetLastError();
 }
 
-// Decode: grid (tiles of 128 blocks, B*Hkv); one thread per block.  Each
-// thread streams its own pooled-key row with independent 16-byte loads (all
-// in flight at once), then runs the fixed-order dot product from registers.
-// The group query mean is formed in fixed order (heads ascending) per CTA.
+// Decode: grid (tiles of 128 blocks, B*Hkv); one thread per block.  The
+// CTA's 128 pooled-key rows are copied into shared memory with coalesced
+// 16-byte cp.async (a warp moves 512 contiguous bytes per instruction) into
+// rows padded to d+4 floats, so that the per-thread float4 reads of eight
+// consecutive rows fall into distinct banks; each thread then runs the
+// fixed-order dot product of its row.  The group query mean is formed in
+// fixed order (heads ascending) per CTA.
 template <typename T, int D>
 __global__ void __launch_bounds__(128) score_decode_kernel(const T* __restrict__ q, const float* __restrict__ kbar,
                                                            int Hq, int Hkv, int nb, float scale,
                                                            float* __restrict__ s, float* __restrict__ qbar_out) {
-  __shared__ float qm[D];
+  constexpr int kPitch = D + 4;
+  constexpr int kChunks = D / 4;   // 16-byte chunks per row
+  extern __shared__ __align__(16) float sm_dec[];
+  float* ks = sm_dec;                 // [128][kPitch]
+  float* qm = sm_dec + 128 * kPitch;  // [D]
   const int64_t bg = blockIdx.y;
   const int64_t b = bg / Hkv, g = bg % Hkv;
   const int G = Hq / Hkv;
+  const int j0 = blockIdx.x * 128;
+  const int rows = min(128, nb - j0);
+  const float* src = kbar + (bg * nb + j0) * D;
+  for (int e = threadIdx.x; e < rows * kChunks; e += 128) {
+    const int r = e / kChunks, c = e % kChunks;
+    cp_async16(smem_u32(ks + r * kPitch + 4 * c), src + static_cast<int64_t>(r) * D + 4 * c);
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
   for (int c = threadIdx.x; c < D; c += blockDim.x) {
     float acc = 0.0f;
     for (int hh = 0; hh < G; ++hh) acc = __fadd_rn(acc, static_cast<float>(q[(b * Hq + g * G + hh) * D + c]));
@@ -344,22 +359,21 @@ __global__ void __launch_bounds__(128) score_decode_kernel(const T* __restrict__
     qm[c] = m;
     if (qbar_out && blockIdx.x == 0) qbar_out[bg * D + c] = m;
   }
+  cp_async_wait_all();
   __syncthreads();
-  const int j = blockIdx.x * blockDim.x + threadIdx.x;
-  if (j >= nb) return;
-  const float4* row = reinterpret_cast<const float4*>(kbar + (bg * nb + j) * D);
-  float4 kv[D / 4];
-#pragma unroll
-  for (int e = 0; e < D / 4; ++e) kv[e] = __ldg(row + e);
+  const int r = threadIdx.x;
+  if (r >= rows) return;
+  const float4* row = reinterpret_cast<const float4*>(ks + r * kPitch);
   float acc = 0.0f;
 #pragma unroll
-  for (int e = 0; e < D / 4; ++e) {
-    acc = __fadd_rn(acc, __fmul_rn(qm[4 * e + 0], kv[e].x));
-    acc = __fadd_rn(acc, __fmul_rn(qm[4 * e + 1], kv[e].y));
-    acc = __fadd_rn(acc, __fmul_rn(qm[4 * e + 2], kv[e].z));
-    acc = __fadd_rn(acc, __fmul_rn(qm[4 * e + 3], kv[e].w));
+  for (int e = 0; e < kChunks; ++e) {
+    const float4 kv = row[e];
+    acc = __fadd_rn(acc, __fmul_rn(qm[4 * e + 0], kv.x));
+    acc = __fadd_rn(acc, __fmul_rn(qm[4 * e + 1], kv.y));
+    acc = __fadd_rn(acc, __fmul_rn(qm[4 * e + 2], kv.z));
+    acc = __fadd_rn(acc, __fmul_rn(qm[4 * e + 3], kv.w));
   }
-  s[bg * nb + j] = __fmul_rn(acc, scale);
+  s[bg * nb + j0 + r] = __fmul_rn(acc, scale);
 }
 
 // Generic-d fallback: rows staged through shared memory.
@@ -392,27 +406,27 @@ __global__ void score_decode_generic_kernel(const T* __restrict__ q, const float
   if (r < rows) s[bg * nb + j0 + r] = __fmul_rn(dot_fixed_order(qm, ks + r * pitch, d, 1), scale);
 }
 
+template <typename T, int D>
+static cudaError_t launch_score_decode_d(dim3 grid, const void* q, const float* kbar, int Hq, int Hkv, int nb,
+                                        float scale, float* s, float* qbar_out, cudaStream_t st) {
+  constexpr size_t smem = (128 * (D + 4) + D) * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(score_decode_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  score_decode_kernel<T, D><<<grid, 128, smem, st>>>(static_cast<const T*>(q), kbar, Hq, Hkv, nb, scale, s, qbar_out);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_score_decode(const void* q, bool bf16, const float* kbar, int B, int Hq, int Hkv,
                                 int nb, int d, float scale, float* s, float* qbar_out,
                                 cudaStream_t st) {
   if (d == 128 || d == 64) {
     dim3 grid((nb + 127) / 128, B * Hkv);
-    if (bf16) {
-      if (d == 128)
-        score_decode_kernel<__nv_bfloat16, 128><<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(q), kbar,
-                                                                      Hq, Hkv, nb, scale, s, qbar_out);
-      else
-        score_decode_kernel<__nv_bfloat16, 64><<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(q), kbar,
-                                                                     Hq, Hkv, nb, scale, s, qbar_out);
-    } else {
-      if (d == 128)
-        score_decode_kernel<float, 128><<<grid, 128, 0, st>>>(static_cast<const float*>(q), kbar, Hq, Hkv, nb,
-                                                              scale, s, qbar_out);
-      else
-        score_decode_kernel<float, 64><<<grid, 128, 0, st>>>(static_cast<const float*>(q), kbar, Hq, Hkv, nb,
-                                                             scale, s, qbar_out);
-    }
-    return cudaGetLastError();
+    if (bf16)
+      return d == 128 ? launch_score_decode_d<__nv_bfloat16, 128>(grid, q, kbar, Hq, Hkv, nb, scale, s, qbar_out, st)
+                      : launch_score_decode_d<__nv_bfloat16, 64>(grid, q, kbar, Hq, Hkv, nb, scale, s, qbar_out, st);
+    return d == 128 ? launch_score_decode_d<float, 128>(grid, q, kbar, Hq, Hkv, nb, scale, s, qbar_out, st)
+                    : launch_score_decode_d<float, 64>(grid, q, kbar, Hq, Hkv, nb, scale, s, qbar_out, st);
   }
   dim3 grid((nb + 63) / 64, B * Hkv);
   const size_t smem = (d + 64 * (d + 1)) * sizeof(float);
@@ -682,17 +696,23 @@ __global__ void __launch_bounds__(128) topk_warp_kernel(const float* __restrict_
   if (count_out && lane == 0) count_out[r] = n;
 }
 
-// CTA-per-row variant for long rows (up to 256*KPT candidates): the same
-// bitwise threshold search, each thread holding KPT candidates (coalesced,
-// j = e*256 + tid), the per-bit counts summed over the eight warps through a
-// double-buffered shared array; warp 0 then writes the kept list in index
-// order from the keys staged in shared memory.
+// CTA-per-row variant for rows of up to 256*KPT candidates.  Thread t holds
+// candidates j = t*KPT .. t*KPT+KPT-1 (index order within the CTA).  Radix
+// select in four 8-bit passes (most significant first): each pass builds a
+// 256-bin shared histogram of the digit among the candidates that match the
+// prefix found so far, and one warp's suffix scan over the bins picks the
+// digit that holds the k-th best key.  The result is the key T of the k-th
+// best candidate and the number of candidates equal to T still to be taken.
+// A block-wide exclusive scan of each thread's (> T, == T) counts then gives
+// every kept candidate its output slot directly: the number of kept
+// candidates of lower index, i.e. all keys > T plus the lowest-index ties.
 template <int KPT>
 __global__ void __launch_bounds__(256) topk_cta_kernel(const float* __restrict__ scores, int ncols, int mode, int kb,
                                                        int* __restrict__ idx_out, int idx_stride,
                                                        int* __restrict__ count_out) {
-  __shared__ uint32_t skeys[256 * KPT];
-  __shared__ int cnts[2][8];
+  __shared__ int hist[256];
+  __shared__ uint32_t wsum[8];
+  __shared__ int sel_digit, sel_above;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t r = blockIdx.x;
   int ncand, forced;
@@ -707,79 +727,114 @@ __global__ void __launch_bounds__(256) topk_cta_kernel(const float* __restrict__
     forced = -1;
   }
   const float* srow = scores + r * ncols;
+  const int j0 = tid * KPT;
   uint32_t key[KPT];
 #pragma unroll
-  for (int e = 0; e < KPT; ++e) {
-    const int j = e * 256 + tid;
-    key[e] = (j < ncand) ? order_key(__ldg(srow + j)) : 0u;
-    skeys[j] = key[e];
-  }
+  for (int e = 0; e < KPT; ++e) key[e] = (j0 + e < ncand) ? order_key(__ldg(srow + j0 + e)) : 0u;
   const int take = min(kb, ncand);
   const bool take_all = (take == ncand);
   uint32_t thresh = 0u;
-  int remaining = take;
-  __syncthreads();
+  int remaining = take;   // ties (== thresh) to keep
   if (!take_all && take > 0) {
-    uint32_t prefix = 0u;
-    for (int bit = 31; bit >= 0; --bit) {
-      const uint32_t cand = prefix | (1u << bit);
-      int c = 0;
-#pragma unroll
-      for (int e = 0; e < KPT; ++e) c += (e * 256 + tid < ncand && key[e] >= cand) ? 1 : 0;
-      c = __reduce_add_sync(0xffffffffu, c);
-      if (lane == 0) cnts[bit & 1][warp] = c;
+    uint32_t prefix = 0u, pmask = 0u;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      hist[tid] = 0;
       __syncthreads();
-      int total = 0;
 #pragma unroll
-      for (int w = 0; w < 8; ++w) total += cnts[bit & 1][w];
-      if (total >= take) prefix = cand;
+      for (int e = 0; e < KPT; ++e)
+        if (j0 + e < ncand && (key[e] & pmask) == prefix) atomicAdd(&hist[(key[e] >> shift) & 255u], 1);
+      __syncthreads();
+      if (warp == 0) {
+        // lane l owns bins 255-8l .. 248-8l (descending); suffix counts
+        int c[8];
+        int run = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          run += hist[255 - 8 * lane - i];
+          c[i] = run;
+        }
+        int incl = run;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        const int excl = incl - run;   // keys in higher bins than this lane's
+        // the digit is the first bin (from the top) whose suffix count reaches remaining
+        int found = -1, above = 0;
+#pragma unroll
+        for (int i = 7; i >= 0; --i) {
+          const int ge = excl + c[i];
+          const int gt = excl + (i ? c[i - 1] : 0);
+          if (ge >= remaining && gt < remaining) {
+            found = 255 - 8 * lane - i;
+            above = gt;
+          }
+        }
+        const unsigned who = __ballot_sync(0xffffffffu, found >= 0);
+        const int src = __ffs(who) - 1;
+        const int d = __shfl_sync(0xffffffffu, found, src);
+        const int ab = __shfl_sync(0xffffffffu, above, src);
+        if (lane == 0) {
+          sel_digit = d;
+          sel_above = ab;
+        }
+      }
+      __syncthreads();
+      prefix |= static_cast<uint32_t>(sel_digit) << shift;
+      pmask |= 255u << shift;
+      remaining -= sel_above;
+      __syncthreads();   // hist and sel_* are rewritten by the next pass
     }
     thresh = prefix;
-    int c = 0;
-#pragma unroll
-    for (int e = 0; e < KPT; ++e) c += (e * 256 + tid < ncand && key[e] > thresh) ? 1 : 0;
-    c = __reduce_add_sync(0xffffffffu, c);
-    __syncthreads();   // everyone is done reading cnts of the last bit
-    if (lane == 0) cnts[0][warp] = c;
-    __syncthreads();
-    int gt = 0;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) gt += cnts[0][w];
-    remaining = take - gt;
   }
-  if (warp != 0) return;
-  int* out = idx_out + r * idx_stride;
-  int run_sel = 0, run_tie = 0;
-  const unsigned lt_mask = (1u << lane) - 1u;
-  for (int base = 0; base < ncand; base += 32) {
-    const int j = base + lane;
-    const bool valid = j < ncand;
-    const uint32_t k = valid ? skeys[j] : 0u;
-    bool gt, tie;
+  // this thread's kept candidates: every key > thresh, ties counted separately
+  int ngt = 0, ntie = 0;
+#pragma unroll
+  for (int e = 0; e < KPT; ++e) {
+    const bool valid = j0 + e < ncand;
     if (take_all) {
-      gt = valid;
-      tie = false;
-    } else if (take == 0) {
-      gt = false;
-      tie = false;
-    } else {
-      gt = valid && k > thresh;
-      tie = valid && k == thresh;
+      ngt += valid ? 1 : 0;
+    } else if (take > 0) {
+      ngt += (valid && key[e] > thresh) ? 1 : 0;
+      ntie += (valid && key[e] == thresh) ? 1 : 0;
     }
-    const unsigned tb = __ballot_sync(0xffffffffu, tie);
-    const bool sel = gt || (tie && run_tie + __popc(tb & lt_mask) < remaining);
-    const unsigned sb = __ballot_sync(0xffffffffu, sel);
-    if (sel) out[run_sel + __popc(sb & lt_mask)] = j;
-    run_sel += __popc(sb);
-    run_tie += __popc(tb);
   }
-  int n = run_sel;
+  // block exclusive scan of the packed (gt, tie) counts (each < 2^16)
+  const uint32_t mine = static_cast<uint32_t>(ngt) | (static_cast<uint32_t>(ntie) << 16);
+  uint32_t incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  uint32_t base = 0u, total = 0u;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) {
+    if (w < warp) base += wsum[w];
+    total += wsum[w];
+  }
+  const uint32_t excl = base + incl - mine;
+  int gt_before = static_cast<int>(excl & 0xFFFFu), tie_before = static_cast<int>(excl >> 16);
+  int* out = idx_out + r * idx_stride;
+#pragma unroll
+  for (int e = 0; e < KPT; ++e) {
+    const bool valid = j0 + e < ncand;
+    const bool gt = take_all ? valid : (take > 0 && valid && key[e] > thresh);
+    const bool tie = !take_all && take > 0 && valid && key[e] == thresh;
+    if (gt || (tie && tie_before < remaining)) out[gt_before + min(tie_before, remaining)] = j0 + e;
+    gt_before += gt ? 1 : 0;
+    tie_before += tie ? 1 : 0;
+  }
+  int n = static_cast<int>(total & 0xFFFFu) + min(static_cast<int>(total >> 16), remaining);
   if (forced >= 0) {
-    if (lane == 0) out[n] = forced;
+    if (tid == 0) out[n] = forced;
     ++n;
   }
-  for (int t = n + lane; t < idx_stride; t += 32) out[t] = -1;
-  if (count_out && lane == 0) count_out[r] = n;
+  for (int t = n + tid; t < idx_stride; t += 256) out[t] = -1;
+  if (count_out && tid == 0) count_out[r] = n;
 }
 
 cudaError_t launch_topk(const float* scores, int rows, int ncols, int mode, int kb, int* idx_out,
