@@ -151,6 +151,18 @@ def wait_gpu(ev):
     torch.cuda.synchronize()
 
 
+def capture_graph(fn):
+    """A CUDA graph holding the launches of fn (the same C-ABI calls, captured
+    once after warm-up).  Decode steps are replayed this way, as a serving
+    loop issues them: the device-timed step then holds no host enqueue gaps."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="thread_local"):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
 def profile_traffic(kernel_file: str, summary_name: str):
     """Per-launch DRAM traffic of the kernel from a committed ncu summary, or
     None when absent or taken on a different kernel source."""
@@ -409,16 +421,19 @@ def run_decode_secondary(dev, peaks, iters: int = 20):
     torch.cuda.synchronize()
     idx = step.bufs["idx"].cpu().numpy()
     kv_bytes = acc.decode_kv_bytes(idx, w.bs, w.d, 2)
+    g_sel = capture_graph(step.select)
+    g_att = capture_graph(lambda: step.attend(with_lse=False))
     stream = torch.cuda.current_stream()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(iters)]
     for it in range(iters):
         flush.fill_(it & 0xFF)
         ev[it][0].record(stream)
-        step.select()
+        g_sel.replay()
         ev[it][1].record(stream)
-        step.attend(with_lse=False)
+        g_att.replay()
         ev[it][2].record(stream)
     torch.cuda.synchronize()
+    del g_sel, g_att
     step_us = statistics.median(1e3 * e[0].elapsed_time(e[2]) for e in ev)
     attn_us = statistics.median(1e3 * e[1].elapsed_time(e[2]) for e in ev)
     gbs = kv_bytes / (attn_us / 1e6) / 1e9
@@ -426,7 +441,8 @@ def run_decode_secondary(dev, peaks, iters: int = 20):
     torch.cuda.empty_cache()
     return {"workload": w.name, "us_per_step": step_us, "attn_us": attn_us, "selected_kv_bytes": kv_bytes,
             "hbm_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
-            "roofline_us": kv_bytes / (peaks["hbm_gbs"] * 1e9) * 1e6, "l2": "flushed (256 MiB write) per iteration"}
+            "roofline_us": kv_bytes / (peaks["hbm_gbs"] * 1e9) * 1e6, "l2": "flushed (256 MiB write) per iteration",
+            "launch": "CUDA graph replay of the C-ABI calls"}
 
 
 def run_decode_like(args, world, rank, local, peaks, peak_src):
@@ -446,11 +462,11 @@ def run_decode_like(args, world, rank, local, peaks, peak_src):
         step = pipeline.DecodeStep(inp["q"], inp["k"], inp["v"], w.bs, w.kb)
         step.pool_cache()
         run = lambda: step.run(with_lse=False)   # noqa: E731
-        launches = 5
+        launches = 4   # score, top-k, split-K attention, combine
     else:
         step = pipeline.GistStep(inp["q"], inp["k"], inp["v"], inp["gk"], inp["gv"], w.bs, w.kb)
         run = lambda: step.run(with_lse=False)   # noqa: E731
-        launches = 5
+        launches = 5   # gist score, top-k, union lists, split-K attention, combine
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
         run()
@@ -460,6 +476,7 @@ def run_decode_like(args, world, rank, local, peaks, peak_src):
         nbytes = acc.decode_kv_bytes(idx, w.bs, w.d, 2)
     else:
         nbytes = acc.gist_kv_bytes(idx, w.G, w.bs, w.N // w.bs, w.d, 2)
+    graph = capture_graph(run)
     stream = torch.cuda.current_stream()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     sampler = ClockSampler(local).start()
@@ -467,7 +484,7 @@ def run_decode_like(args, world, rank, local, peaks, peak_src):
     for s in range(args.steps):
         flush.fill_(s & 0xFF)
         ev[s][0].record(stream)
-        run()
+        graph.replay()
         ev[s][1].record(stream)
     wait_gpu(ev[-1][1])
     t1 = time.time()
@@ -479,7 +496,8 @@ def run_decode_like(args, world, rank, local, peaks, peak_src):
         "warmup": args.warmup, "ms_per_step": us / 1e3, "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "ctx": w.N, "block": w.bs,
-                   "budget": w.kb, "l2": "flushed (256 MiB write) before every step, outside the events"},
+                   "budget": w.kb, "l2": "flushed (256 MiB write) before every step, outside the events",
+                   "launch": "CUDA graph replay of the C-ABI calls"},
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": gbs / peaks["hbm_gbs"], "traffic": None, "peak_source": peak_src,
                      "bytes_per_step": nbytes, "note": "whole step (score + top-k + attention + combine)"},

@@ -275,6 +275,44 @@ def test_decode_split_count_invariance():
     _status_clean()
 
 
+def test_decode_and_gist_graph_replay_match_eager():
+    """The decode and gist steps captured into CUDA graphs (as the benchmark
+    replays them) give the same bytes as the eager C-ABI calls."""
+    pipe = _pipe()
+    w = W.get("decode_bf16").scaled(B=2, Hq=8, Hkv=2, N=8192, kb=24)
+    inp = W.make_inputs(w, "cuda")
+    step = pipe.DecodeStep(inp["q"], inp["k"], inp["v"], w.bs, w.kb)
+    step.pool_cache()
+    step.run()
+    torch.cuda.synchronize()
+    eager = {k: step.bufs[k].clone() for k in ("scores", "idx", "o", "lse")}
+    for k in ("scores", "o", "lse"):
+        step.bufs[k].zero_()
+    step.bufs["idx"].fill_(-7)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="thread_local"):
+        step.run()
+    g.replay()
+    torch.cuda.synchronize()
+    for k, v in eager.items():
+        assert torch.equal(step.bufs[k], v), k
+    wg = W.get("gist_decode_bf16").scaled(B=1, Hq=8, Hkv=2, N=8192, kb=6)
+    ig = W.make_inputs(wg, "cuda")
+    gs = pipe.GistStep(ig["q"], ig["k"], ig["v"], ig["gk"], ig["gv"], wg.bs, wg.kb)
+    gs.run()
+    torch.cuda.synchronize()
+    o_eager = gs.bufs["o"].clone()
+    gs.bufs["o"].zero_()
+    gg = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gg, capture_error_mode="thread_local"):
+        gs.run()
+    gg.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(gs.bufs["o"], o_eager)
+    del g, gg
+    _status_clean()
+
+
 # ----------------------------------------------------------------------------
 # gist selective expansion (SSA)
 # ----------------------------------------------------------------------------

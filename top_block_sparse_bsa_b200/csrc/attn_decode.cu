@@ -695,8 +695,7 @@ __global__ void gist_union_kernel(const int* __restrict__ idx, int Hq, int Hkv, 
 cudaError_t launch_attn_decode_bf16(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
                                     const CUtensorMap* tmGK, const CUtensorMap* tmGV, const DecodeArgs& a,
                                     cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(decode::attn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(decode::kSmemBytes));
+  cudaError_t e = ensure_dynamic_smem<decode::attn_decode_kernel>(decode::kSmemBytes);
   if (e != cudaSuccess) return e;
   decode::Params p;
   p.B = a.B;

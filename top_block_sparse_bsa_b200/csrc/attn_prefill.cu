@@ -616,8 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int BS>
 static cudaError_t launch_bs(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
                              const Params& p, unsigned grid, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(attn_prefill_kernel<BS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kSmemBytes));
+  cudaError_t e = ensure_dynamic_smem<attn_prefill_kernel<BS>>(kSmemBytes);
   if (e != cudaSuccess) return e;
   attn_prefill_kernel<BS><<<grid, kThreads, kSmemBytes, st>>>(*tmQ, *tmK, *tmV, p);
   return cudaGetLastError();

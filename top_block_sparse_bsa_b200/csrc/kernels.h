@@ -5,7 +5,29 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace bsa {
+
+// Opt kernel Fn into `bytes` of dynamic shared memory on the current device.
+// The attribute belongs to the (function, device) pair and persists, so the
+// driver call is made only when a device sees a larger request than before;
+// launches after the first cost no extra driver call.
+template <auto Fn>
+inline cudaError_t ensure_dynamic_smem(size_t bytes) {
+  static std::atomic<uint32_t> granted[32];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 32) return cudaErrorInvalidDevice;
+  if (granted[dev].load(std::memory_order_acquire) >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(Fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  if (e != cudaSuccess) return e;
+  uint32_t cur = granted[dev].load(std::memory_order_relaxed);
+  while (cur < bytes && !granted[dev].compare_exchange_weak(cur, static_cast<uint32_t>(bytes))) {
+  }
+  return cudaSuccess;
+}
 
 // selector.cu
 cudaError_t launch_pool(const void* src, bool bf16, int B, int Hsrc, int Hgroups, int heads_sum, int N,

@@ -221,13 +221,11 @@ cudaError_t launch_pool_prefill(const void* q, const void* k, bool bf16, int B, 
   const unsigned grid = static_cast<unsigned>(units < num_sms ? units : num_sms);
   cudaError_t e;
   if (bf16) {
-    e = cudaFuncSetAttribute(pool_stream_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
+    e = ensure_dynamic_smem<pool_stream_kernel<__nv_bfloat16>>(smem);
     if (e != cudaSuccess) return e;
     pool_stream_kernel<__nv_bfloat16><<<grid, 160, smem, st>>>(jq, jk, B, Hkv, N, d, bs, status);
   } else {
-    e = cudaFuncSetAttribute(pool_stream_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
+    e = ensure_dynamic_smem<pool_stream_kernel<float>>(smem);
     if (e != cudaSuccess) return e;
     pool_stream_kernel<float><<<grid, 160, smem, st>>>(jq, jk, B, Hkv, N, d, bs, status);
   }
@@ -317,8 +315,7 @@ cudaError_t launch_score_prefill(const float* qbar, const float* kbar, int B, in
   dim3 grid((nb + kScoreTile - 1) / kScoreTile, (nb + kScoreTile - 1) / kScoreTile, B * Hkv);
   const size_t smem = 2 * kScoreTile * (d + 4) * sizeof(float);
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(score_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    cudaError_t e = ensure_dynamic_smem<score_prefill_kernel>(smem);
     if (e != cudaSuccess) return e;
   }
   score_prefill_kernel<<<grid, 256, smem, st>>>(qbar, kbar, nb, d, scale, s);
@@ -410,8 +407,7 @@ template <typename T, int D>
 static cudaError_t launch_score_decode_d(dim3 grid, const void* q, const float* kbar, int Hq, int Hkv, int nb,
                                         float scale, float* s, float* qbar_out, cudaStream_t st) {
   constexpr size_t smem = (128 * (D + 4) + D) * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(score_decode_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = ensure_dynamic_smem<score_decode_kernel<T, D>>(smem);
   if (e != cudaSuccess) return e;
   score_decode_kernel<T, D><<<grid, 128, smem, st>>>(static_cast<const T*>(q), kbar, Hq, Hkv, nb, scale, s, qbar_out);
   return cudaGetLastError();
