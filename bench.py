@@ -461,12 +461,17 @@ def run_decode_like(args, world, rank, local, peaks, peak_src):
     if w.kind == "decode":
         step = pipeline.DecodeStep(inp["q"], inp["k"], inp["v"], w.bs, w.kb)
         step.pool_cache()
-        run = lambda: step.run(with_lse=False)   # noqa: E731
-        launches = 4   # score, top-k, split-K attention, combine
+        select = step.select
+        attend = lambda: step.attend(with_lse=False)   # noqa: E731
+        launches = 4   # score, top-k | split-K attention, combine
+        attn_file, attn_kernel = "attn_decode.cu", "attn_decode_kernel (+ combine_kernel)"
     else:
         step = pipeline.GistStep(inp["q"], inp["k"], inp["v"], inp["gk"], inp["gv"], w.bs, w.kb)
-        run = lambda: step.run(with_lse=False)   # noqa: E731
-        launches = 5   # gist score, top-k, union lists, split-K attention, combine
+        select = lambda: step.run(with_lse=False)   # noqa: E731  (full step; its outputs feed the next call)
+        attend = lambda: step.run(idx_in=step.bufs["idx"], with_lse=False)   # noqa: E731
+        launches = 5   # gist score, top-k | union lists, split-K attention, combine
+        attn_file, attn_kernel = "attn_decode.cu", "gist_union_kernel + attn_decode_kernel + combine_kernel"
+    run = lambda: (select(), attend()) if w.kind == "decode" else select()   # noqa: E731
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
         run()
@@ -476,7 +481,10 @@ def run_decode_like(args, world, rank, local, peaks, peak_src):
         nbytes = acc.decode_kv_bytes(idx, w.bs, w.d, 2)
     else:
         nbytes = acc.gist_kv_bytes(idx, w.G, w.bs, w.N // w.bs, w.d, 2)
+    # whole step (timed value) and its attention part alone (roofline of the
+    # dominant kernel), each replayed from a CUDA graph, L2 flushed first
     graph = capture_graph(run)
+    g_att = capture_graph(attend)
     stream = torch.cuda.current_stream()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     sampler = ClockSampler(local).start()
@@ -490,7 +498,19 @@ def run_decode_like(args, world, rank, local, peaks, peak_src):
     t1 = time.time()
     sampler.stop()
     us = statistics.mean(1e3 * a.elapsed_time(b) for a, b in ev)
-    gbs = nbytes / (us / 1e6) / 1e9
+    ea = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for s in range(args.steps):
+        flush.fill_(s & 0xFF)
+        ea[s][0].record(stream)
+        g_att.replay()
+        ea[s][1].record(stream)
+    wait_gpu(ea[-1][1])
+    attn_us = statistics.mean(1e3 * a.elapsed_time(b) for a, b in ea)
+    del graph, g_att
+    gbs = nbytes / (attn_us / 1e6) / 1e9
+    traffic, sha = profile_traffic(attn_file, f"attn_decode_{w.name}.md")
+    if sha is not None and sha != kernel_source_sha(["attn_decode.cu", "common.cuh"]):
+        traffic = None
     line = {
         "metric": "us per decode step", "value": us, "unit": "us", "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": us / 1e3, "higher_is_better": False, "scaling": "weak",
@@ -499,8 +519,9 @@ def run_decode_like(args, world, rank, local, peaks, peak_src):
                    "budget": w.kb, "l2": "flushed (256 MiB write) before every step, outside the events",
                    "launch": "CUDA graph replay of the C-ABI calls"},
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": gbs / peaks["hbm_gbs"], "traffic": None, "peak_source": peak_src,
-                     "bytes_per_step": nbytes, "note": "whole step (score + top-k + attention + combine)"},
+                     "frac": gbs / peaks["hbm_gbs"], "traffic": traffic, "peak_source": peak_src,
+                     "kernel": attn_kernel, "kernel_us": attn_us, "selected_kv_bytes_per_launch": nbytes,
+                     "step_gbs": nbytes / (us / 1e6) / 1e9},
         "clocks": sampler.summary(t0, t1), "gpu_launches": launches * args.steps,
     }
     print(json.dumps(line), flush=True)

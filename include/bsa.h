@@ -190,7 +190,8 @@ bsa_status_t bsa_sparse_attn_decode(const bsa_shape_t* shape, const void* q, con
  * topk: chunks expanded per query head (0 <= topk <= nc).
  * idx_in [B,Hq,topk] int32 (optional): if given, these chunks are expanded
  *   and no scoring/selection runs (the way to inject a known index set).
- * idx_out [B,Hq,topk] int32 (optional): receives the chosen chunks ascending.
+ * idx_out [B,Hq,topk] int32 (optional): receives the chosen chunks ascending
+ *   (with idx_in, a copy of it; idx_out may be idx_in itself).
  * workspace: bsa_workspace_bytes(BSA_OP_GIST_DECODE, shape, topk) bytes.
  * o [B,Hq,d] (dtype); lse [B,Hq] fp32 (optional).
  * Built: BF16, d = 128, block = 64.

@@ -397,7 +397,7 @@ bsa_status_t bsa_gist_expand_decode(const bsa_shape_t* s, const void* q, const v
       e = cudaMemsetAsync(idx_dst, 0xff, static_cast<size_t>(rows) * sizeof(int), cs);
     }
     idx = idx_dst;
-  } else if (idx_out != nullptr && topk > 0) {
+  } else if (idx_out != nullptr && topk > 0 && idx_out != idx_in) {
     e = cudaMemcpyAsync(idx_out, idx_in, static_cast<size_t>(rows) * topk * sizeof(int), cudaMemcpyDeviceToDevice, cs);
   }
   uint32_t* expanded = reinterpret_cast<uint32_t*>(ws + L.expanded);
