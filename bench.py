@@ -421,21 +421,26 @@ def run_decode_secondary(dev, peaks, iters: int = 20):
     torch.cuda.synchronize()
     idx = step.bufs["idx"].cpu().numpy()
     kv_bytes = acc.decode_kv_bytes(idx, w.bs, w.d, 2)
+    # the step as one graph; its attention part timed behind the selection
+    g_step = capture_graph(lambda: (step.select(), step.attend(with_lse=False)))
     g_sel = capture_graph(step.select)
     g_att = capture_graph(lambda: step.attend(with_lse=False))
     stream = torch.cuda.current_stream()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(iters)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(iters)]
     for it in range(iters):
         flush.fill_(it & 0xFF)
         ev[it][0].record(stream)
-        g_sel.replay()
+        g_step.replay()
         ev[it][1].record(stream)
-        g_att.replay()
+        flush.fill_((it + 1) & 0xFF)
+        g_sel.replay()
         ev[it][2].record(stream)
+        g_att.replay()
+        ev[it][3].record(stream)
     torch.cuda.synchronize()
-    del g_sel, g_att
-    step_us = statistics.median(1e3 * e[0].elapsed_time(e[2]) for e in ev)
-    attn_us = statistics.median(1e3 * e[1].elapsed_time(e[2]) for e in ev)
+    del g_step, g_sel, g_att
+    step_us = statistics.median(1e3 * e[0].elapsed_time(e[1]) for e in ev)
+    attn_us = statistics.median(1e3 * e[2].elapsed_time(e[3]) for e in ev)
     gbs = kv_bytes / (attn_us / 1e6) / 1e9
     del inp, step, flush
     torch.cuda.empty_cache()
@@ -467,46 +472,57 @@ def run_decode_like(args, world, rank, local, peaks, peak_src):
         attn_file, attn_kernel = "attn_decode.cu", "attn_decode_kernel (+ combine_kernel)"
     else:
         step = pipeline.GistStep(inp["q"], inp["k"], inp["v"], inp["gk"], inp["gv"], w.bs, w.kb)
-        select = lambda: step.run(with_lse=False)   # noqa: E731  (full step; its outputs feed the next call)
+        select = lambda: step.run(with_lse=False)   # noqa: E731  (the whole step in one call)
         attend = lambda: step.run(idx_in=step.bufs["idx"], with_lse=False)   # noqa: E731
-        launches = 5   # gist score, top-k | union lists, split-K attention, combine
+        launches = 5   # gist score, top-k, union lists, split-K attention, combine
         attn_file, attn_kernel = "attn_decode.cu", "gist_union_kernel + attn_decode_kernel + combine_kernel"
-    run = lambda: (select(), attend()) if w.kind == "decode" else select()   # noqa: E731
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
-        run()
+        select()
+        attend()
     torch.cuda.synchronize()
     idx = step.bufs["idx"].cpu().numpy()
     if w.kind == "decode":
         nbytes = acc.decode_kv_bytes(idx, w.bs, w.d, 2)
     else:
         nbytes = acc.gist_kv_bytes(idx, w.G, w.bs, w.N // w.bs, w.d, 2)
-    # whole step (timed value) and its attention part alone (roofline of the
-    # dominant kernel), each replayed from a CUDA graph, L2 flushed first
-    graph = capture_graph(run)
+    # Each step is replayed from CUDA graphs of the C-ABI calls, L2 flushed
+    # first.  The timed step is one graph holding the whole step.  The
+    # attention part is timed in a second pass: decode replays the selection
+    # graph and then the attention graph, timing the latter (its launch is
+    # queued behind the selection, as inside a step); gist (whose step is one
+    # call) replays the attention-only call (its own indices injected) after
+    # another L2 flush, queued behind that flush.
+    if w.kind == "decode":
+        g_step = capture_graph(lambda: (select(), attend()))
+    else:
+        g_step = capture_graph(select)
+    g_sel = capture_graph(select) if w.kind == "decode" else None
     g_att = capture_graph(attend)
     stream = torch.cuda.current_stream()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     sampler = ClockSampler(local).start()
     t0 = time.time()
     for s in range(args.steps):
         flush.fill_(s & 0xFF)
         ev[s][0].record(stream)
-        graph.replay()
+        g_step.replay()
         ev[s][1].record(stream)
     wait_gpu(ev[-1][1])
     t1 = time.time()
     sampler.stop()
-    us = statistics.mean(1e3 * a.elapsed_time(b) for a, b in ev)
-    ea = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    us = statistics.mean(1e3 * e[0].elapsed_time(e[1]) for e in ev)
+    ea = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     for s in range(args.steps):
         flush.fill_(s & 0xFF)
+        if g_sel is not None:
+            g_sel.replay()
         ea[s][0].record(stream)
         g_att.replay()
         ea[s][1].record(stream)
     wait_gpu(ea[-1][1])
-    attn_us = statistics.mean(1e3 * a.elapsed_time(b) for a, b in ea)
-    del graph, g_att
+    attn_us = statistics.mean(1e3 * e[0].elapsed_time(e[1]) for e in ea)
+    del g_step, g_sel, g_att
     gbs = nbytes / (attn_us / 1e6) / 1e9
     traffic, sha = profile_traffic(attn_file, f"attn_decode_{w.name}.md")
     if sha is not None and sha != kernel_source_sha(["attn_decode.cu", "common.cuh"]):

@@ -360,6 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  griddep_wait();   // kept lists / union lists come from the kernel launched before
   const uint32_t tmem = misc->tmem_base;   // S^T buffers at columns 0 / 16, O^T at 32
 
   if (warp == 6) {
@@ -598,6 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 __global__ void combine_kernel(const float* __restrict__ partial, int rows, int G, int list_len, int64_t total,
                                int num_ctas, int max_slots, int d, int out_bf16, void* __restrict__ o,
                                float* __restrict__ lse) {
+  griddep_wait();
   const int row = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
@@ -639,6 +641,7 @@ __global__ void combine_kernel(const float* __restrict__ partial, int rows, int 
 __global__ void gist_union_kernel(const int* __restrict__ idx, int Hq, int Hkv, int topk, int idx_stride, int nc,
                                   uint32_t* __restrict__ expanded, int* __restrict__ union_list, int union_stride,
                                   uint32_t* __restrict__ status) {
+  griddep_wait();
   extern __shared__ uint32_t sbits[];   // [G+1][nc/32]; row G = union
   const int G = Hq / Hkv;
   const int words = nc / 32;
@@ -716,9 +719,8 @@ cudaError_t launch_attn_decode_bf16(const CUtensorMap* tmQ, const CUtensorMap* t
   p.partial = a.partial;
   p.status = a.status;
   const int grid = a.num_ctas;
-  decode::attn_decode_kernel<<<grid, decode::kThreads, decode::kSmemBytes, st>>>(
-      *tmQ, *tmK, *tmV, tmGK ? *tmGK : *tmK, tmGV ? *tmGV : *tmV, p);
-  return cudaGetLastError();
+  return launch_dependent(decode::attn_decode_kernel, dim3(grid), dim3(decode::kThreads), decode::kSmemBytes, st, *tmQ,
+                          *tmK, *tmV, tmGK ? *tmGK : *tmK, tmGV ? *tmGV : *tmV, p);
 }
 
 cudaError_t launch_decode_combine(const float* partial, const DecodeArgs& a, int d, bool out_bf16, void* o,
@@ -726,9 +728,8 @@ cudaError_t launch_decode_combine(const float* partial, const DecodeArgs& a, int
   const int warps = 8;
   const int rows = a.B * a.Hq;
   const int64_t total = static_cast<int64_t>(a.B) * a.Hkv * a.list_len;
-  decode::combine_kernel<<<(rows + warps - 1) / warps, warps * 32, 0, st>>>(
-      partial, rows, a.Hq / a.Hkv, a.list_len, total, a.num_ctas, a.max_slots, d, out_bf16 ? 1 : 0, o, lse);
-  return cudaGetLastError();
+  return launch_dependent(decode::combine_kernel, dim3((rows + warps - 1) / warps), dim3(warps * 32), 0, st, partial,
+                          rows, a.Hq / a.Hkv, a.list_len, total, a.num_ctas, a.max_slots, d, out_bf16 ? 1 : 0, o, lse);
 }
 
 int decode_slots_for(int rows, int list_len, int num_ctas) {
@@ -748,9 +749,8 @@ cudaError_t launch_gist_union(const int* idx, int B, int Hq, int Hkv, int topk, 
                               cudaStream_t st) {
   const int G = Hq / Hkv;
   const size_t smem = static_cast<size_t>(G + 1) * (nc / 32) * sizeof(uint32_t);
-  decode::gist_union_kernel<<<B * Hkv, 256, smem, st>>>(idx, Hq, Hkv, topk, idx_stride, nc, expanded, union_list,
-                                                        union_stride, status);
-  return cudaGetLastError();
+  return launch_dependent(decode::gist_union_kernel, dim3(B * Hkv), dim3(256), smem, st, idx, Hq, Hkv, topk, idx_stride,
+                          nc, expanded, union_list, union_stride, status);
 }
 
 }  // namespace bsa

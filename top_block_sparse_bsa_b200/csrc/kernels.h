@@ -29,6 +29,26 @@ inline cudaError_t ensure_dynamic_smem(size_t bytes) {
   return cudaSuccess;
 }
 
+// Launch a kernel that may start while the previous kernel on the stream is
+// finishing (programmatic dependent launch): its launch and prologue overlap
+// that kernel's tail, and it calls griddep_wait() before reading that
+// kernel's output.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                   Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // selector.cu
 cudaError_t launch_pool(const void* src, bool bf16, int B, int Hsrc, int Hgroups, int heads_sum, int N,
                         int d, int bs, float* out, cudaStream_t st);

@@ -498,6 +498,7 @@ constexpr int kTopkThreads = 256;
 __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restrict__ scores, int ncols,
                                                             int mode, int kb, int* __restrict__ idx_out,
                                                             int idx_stride, int* __restrict__ count_out) {
+  griddep_wait();   // the scores come from the kernel launched before
   extern __shared__ uint32_t skeys[];
   __shared__ uint32_t hist[256];
   __shared__ uint32_t s_digit;
@@ -616,6 +617,7 @@ template <int KPL>
 __global__ void __launch_bounds__(128) topk_warp_kernel(const float* __restrict__ scores, int rows, int ncols,
                                                         int mode, int kb, int* __restrict__ idx_out, int idx_stride,
                                                         int* __restrict__ count_out) {
+  griddep_wait();   // the scores come from the kernel launched before
   const int lane = threadIdx.x & 31;
   const int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (r >= rows) return;
@@ -706,6 +708,7 @@ template <int KPT>
 __global__ void __launch_bounds__(256) topk_cta_kernel(const float* __restrict__ scores, int ncols, int mode, int kb,
                                                        int* __restrict__ idx_out, int idx_stride,
                                                        int* __restrict__ count_out) {
+  griddep_wait();   // the scores come from the kernel launched before
   __shared__ int hist[256];
   __shared__ uint32_t wsum[8];
   __shared__ int sel_digit, sel_above;
@@ -838,12 +841,15 @@ cudaError_t launch_topk(const float* scores, int rows, int ncols, int mode, int 
   if (ncols <= 32 * 16) {
     const int warps = 4;
     const unsigned grid = static_cast<unsigned>((rows + warps - 1) / warps);
-    topk_warp_kernel<16><<<grid, 32 * warps, 0, st>>>(scores, rows, ncols, mode, kb, idx_out, idx_stride, count_out);
+    return launch_dependent(topk_warp_kernel<16>, dim3(grid), dim3(32 * warps), 0, st, scores, rows, ncols, mode, kb,
+                            idx_out, idx_stride, count_out);
   } else if (ncols <= 256 * 8) {
-    topk_cta_kernel<8><<<rows, 256, 0, st>>>(scores, ncols, mode, kb, idx_out, idx_stride, count_out);
+    return launch_dependent(topk_cta_kernel<8>, dim3(rows), dim3(256), 0, st, scores, ncols, mode, kb, idx_out,
+                            idx_stride, count_out);
   } else {
     const size_t smem = static_cast<size_t>(ncols) * sizeof(uint32_t);
-    topk_kernel<<<rows, kTopkThreads, smem, st>>>(scores, ncols, mode, kb, idx_out, idx_stride, count_out);
+    return launch_dependent(topk_kernel, dim3(rows), dim3(kTopkThreads), smem, st, scores, ncols, mode, kb, idx_out,
+                            idx_stride, count_out);
   }
   return cudaGetLastError();
 }
