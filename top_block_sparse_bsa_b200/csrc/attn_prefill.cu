@@ -108,6 +108,7 @@ struct Params {
   const float* sel;     // gated when non-null
   float scale_log2;
   __nv_bfloat16* o;
+  int o_v8;             // o is 32-byte aligned: 256-bit row stores
   float* lse;
   uint32_t* status;
 };
@@ -595,9 +596,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(BAR_OE + t));   // O may be overwritten by the next item from here on
         if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(p.o + orow_idx * kD);
+          if (p.o_v8) {   // whole 32-byte sectors per store
 #pragma unroll
-          for (int e = 0; e < 16; ++e) dst[e] = make_uint4(ob[4 * e], ob[4 * e + 1], ob[4 * e + 2], ob[4 * e + 3]);
+            for (int e = 0; e < 8; ++e) st_global_v8(p.o + orow_idx * kD + 16 * e, ob + 8 * e);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(p.o + orow_idx * kD);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) dst[e] = make_uint4(ob[4 * e], ob[4 * e + 1], ob[4 * e + 2], ob[4 * e + 3]);
+          }
           if (p.lse) p.lse[orow_idx] = (l_run > 0.0f) ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
         }
       }
@@ -644,6 +650,7 @@ cudaError_t launch_attn_prefill_bf16(const CUtensorMap* tmQ, const CUtensorMap* 
   p.sel = a.sel_scores;
   p.scale_log2 = a.softmax_scale * prefill::kLog2e;
   p.o = static_cast<__nv_bfloat16*>(a.o);
+  p.o_v8 = (reinterpret_cast<uintptr_t>(a.o) & 31u) == 0 ? 1 : 0;
   p.lse = a.lse;
   p.status = a.status;
   const unsigned grid = static_cast<unsigned>(items < a.num_sms ? items : a.num_sms);
