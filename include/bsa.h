@@ -172,7 +172,8 @@ bsa_status_t bsa_gated_attn_fwd(const bsa_shape_t* shape, const void* q, const v
  *   bsa_workspace_bytes(BSA_OP_DECODE, shape, idx_stride) bytes, 256-byte
  *   aligned; its contents on entry do not matter.
  * o [B,Hq,d] (dtype); lse [B,Hq] fp32 (optional).
- * Built: BF16, d = 128, block = 64.
+ * Built: BF16, d = 128, block = 64, at most 16 query heads per KV group
+ * (BSA_ERR_UNSUPPORTED otherwise).
  */
 bsa_status_t bsa_sparse_attn_decode(const bsa_shape_t* shape, const void* q, const void* k_cache,
                                     const void* v_cache, const int* idx, int idx_stride,
@@ -194,7 +195,8 @@ bsa_status_t bsa_sparse_attn_decode(const bsa_shape_t* shape, const void* q, con
  *   (with idx_in, a copy of it; idx_out may be idx_in itself).
  * workspace: bsa_workspace_bytes(BSA_OP_GIST_DECODE, shape, topk) bytes.
  * o [B,Hq,d] (dtype); lse [B,Hq] fp32 (optional).
- * Built: BF16, d = 128, block = 64.
+ * Built: BF16, d = 128, block = 64, at most 16 query heads per KV group
+ * (BSA_ERR_UNSUPPORTED otherwise).
  */
 bsa_status_t bsa_gist_expand_decode(const bsa_shape_t* shape, const void* q, const void* k_cache,
                                     const void* v_cache, const void* gist_k, const void* gist_v,

@@ -67,6 +67,19 @@ def test_host_checks_reject_before_any_launch(bsa):
                                   None, None, None) == 1
 
 
+def test_decode_rejects_groups_wider_than_the_mma_tile(bsa):
+    # the decode kernels hold at most 16 query heads of a group (MMA N = 16):
+    # 17..32 heads per KV group are refused on the host as unsupported
+    lib = bsa.lib
+    p = ctypes.c_void_p(4096)   # aligned stand-in pointers; nothing is dereferenced
+    for hq in (17 * 2, 32 * 2):
+        shape = bsa.make_shape(1, hq, 2, 1, 4096, 128, 64, bsa.BSA_BF16)
+        assert lib.bsa_sparse_attn_decode(ctypes.byref(shape), p, p, p, p, 8, ctypes.c_float(0.1), p,
+                                          ctypes.c_size_t(1 << 30), p, None, None) == 2
+        assert lib.bsa_gist_expand_decode(ctypes.byref(shape), p, p, p, p, p, 4, None, None, ctypes.c_float(0.1),
+                                          p, ctypes.c_size_t(1 << 30), p, None, None) == 2
+
+
 def test_product_path_does_not_import_the_oracle():
     pkg = os.path.join(ROOT, "top_block_sparse_bsa_b200")
     for dirpath, _, files in os.walk(pkg):

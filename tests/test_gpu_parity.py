@@ -254,6 +254,14 @@ def test_decode_bf16_full_size_sampled():
     _decode_case(w, groups=[(0, 0), (5, 3), (15, 7), (9, 1)])
 
 
+@pytest.mark.parametrize("hq,hkv", [(2, 2), (4, 2), (16, 2), (32, 2)])
+def test_decode_group_widths(hq, hkv):
+    # G = 1, 2, 8, 16 query heads per KV group (the softmax is specialised on
+    # the padded group width 4 / 8 / 16)
+    w = W.get("decode_bf16").scaled(B=1, Hq=hq, Hkv=hkv, N=4096, kb=10)
+    _decode_case(w)
+
+
 def test_decode_split_count_invariance():
     bsa = _bsa()
     pipe = _pipe()
@@ -356,6 +364,12 @@ def test_gist_bf16_small():
 def test_gist_bf16_edge_budgets(topk):
     w = W.get("gist_decode_bf16").scaled(B=1, Hq=4, Hkv=1, N=8192, kb=topk)
     _gist_case(w, topk=topk)
+
+
+@pytest.mark.parametrize("hq,hkv", [(2, 2), (16, 2), (32, 2)])
+def test_gist_group_widths(hq, hkv):
+    w = W.get("gist_decode_bf16").scaled(B=1, Hq=hq, Hkv=hkv, N=8192, kb=5)
+    _gist_case(w)
 
 
 def test_gist_bf16_full_size_sampled():

@@ -317,7 +317,7 @@ static bsa_status_t decode_checks(const bsa_shape_t* s, const void* q, const voi
   if (s->Nq != 1 || !q || !kc || !vc || !o) return BSA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(kc) || !aligned16(vc) || !aligned16(o)) return BSA_ERR_INVALID_ARG;
   if (s->dtype != BSA_BF16 || s->d != 128 || s->block != 64) return BSA_ERR_UNSUPPORTED;
-  if (s->Hq / s->Hkv > 32) return BSA_ERR_UNSUPPORTED;
+  if (s->Hq / s->Hkv > 16) return BSA_ERR_UNSUPPORTED;   // the MMA N tile holds a group of at most 16 heads
   return BSA_OK;
 }
 

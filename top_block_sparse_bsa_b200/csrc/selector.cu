@@ -116,18 +116,20 @@ static cudaError_t launch_pool_jobs(const PoolJob& j0, const PoolJob& j1, bool b
 }
 
 // Streamed variant (persistent, one CTA per SM): a producer thread copies each
-// unit's rows (heads_sum runs of bs*d contiguous elements) into one of two
-// shared-memory buffers with bulk copies while 128 threads sum the previous
-// unit, column c by thread c, rows in the fixed order.  Units of the query
-// job come first, then those of the key job.
+// unit's rows (heads_sum runs of bs*d contiguous elements) into one of
+// kPoolStages shared-memory buffers with bulk copies while 128 threads sum an
+// earlier unit, column c by thread c, rows in the fixed order (two units stay
+// in flight per SM).  Units of the query job come first, then those of the
+// key job.
 constexpr int kPoolStreamBytes = 64 * 1024;
+constexpr int kPoolStages = 3;
 
 template <typename T>
 __global__ void __launch_bounds__(160, 1) pool_stream_kernel(PoolJob jq, PoolJob jk, int B, int Hgroups, int N, int d,
                                                              int bs, uint32_t* status) {
   extern __shared__ uint8_t psmem_raw[];
   uint8_t* psmem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(psmem_raw) + 127) & ~uintptr_t(127));
-  __shared__ __align__(8) uint64_t bars[4];   // full[2], empty[2]
+  __shared__ __align__(8) uint64_t bars[2 * kPoolStages];
   __shared__ int abort_flag;
   const uint32_t sb = smem_u32(psmem);
   auto bar = [&](int i) -> uint32_t { return smem_u32(&bars[i]); };
@@ -135,10 +137,10 @@ __global__ void __launch_bounds__(160, 1) pool_stream_kernel(PoolJob jq, PoolJob
   const int64_t units_per_job = static_cast<int64_t>(B) * Hgroups * nb;
   const int64_t units = units_per_job * (jk.src ? 2 : 1);
   if (threadIdx.x == 0) {
-    mbar_init(bar(0), 1);
-    mbar_init(bar(1), 1);
-    mbar_init(bar(2), 128);
-    mbar_init(bar(3), 128);
+    for (int i = 0; i < kPoolStages; ++i) {
+      mbar_init(bar(i), 1);
+      mbar_init(bar(kPoolStages + i), 128);
+    }
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -156,8 +158,8 @@ __global__ void __launch_bounds__(160, 1) pool_stream_kernel(PoolJob jq, PoolJob
         const int64_t b = unit / (static_cast<int64_t>(Hgroups) * nb);
         const int64_t g = (unit / nb) % Hgroups;
         const int64_t j = unit % nb;
-        const int buf = k & 1;
-        if (k >= 2 && !mbar_wait(bar(2 + buf), ((k >> 1) - 1) & 1, ab, status)) break;
+        const int buf = k % kPoolStages, use = k / kPoolStages;
+        if (k >= kPoolStages && !mbar_wait(bar(kPoolStages + buf), (use - 1) & 1, ab, status)) break;
         const uint32_t run = static_cast<uint32_t>(bs) * d * sizeof(T);
         mbar_arrive_expect_tx(bar(buf), run * job.heads_sum);
         const T* src = static_cast<const T*>(job.src);
@@ -168,7 +170,8 @@ __global__ void __launch_bounds__(160, 1) pool_stream_kernel(PoolJob jq, PoolJob
         ++issued;
       }
       if (*ab) {   // let the copies still in flight land before the CTA exits
-        for (int q = issued > 2 ? issued - 2 : 0; q < issued; ++q) mbar_drain(bar(q & 1), (q >> 1) & 1);
+        for (int q = issued > kPoolStages ? issued - kPoolStages : 0; q < issued; ++q)
+          mbar_drain(bar(q % kPoolStages), (q / kPoolStages) & 1);
       }
     }
   } else {
@@ -178,8 +181,8 @@ __global__ void __launch_bounds__(160, 1) pool_stream_kernel(PoolJob jq, PoolJob
       const bool isk = u >= units_per_job;
       const PoolJob& job = isk ? jk : jq;
       const int64_t unit = isk ? u - units_per_job : u;
-      const int buf = k & 1;
-      if (!mbar_wait(bar(buf), (k >> 1) & 1, ab, status)) break;
+      const int buf = k % kPoolStages, use = k / kPoolStages;
+      if (!mbar_wait(bar(buf), use & 1, ab, status)) break;
       const T* sv = reinterpret_cast<const T*>(psmem + buf * kPoolStreamBytes);
       const int rows = job.heads_sum * bs;   // a multiple of 16
       if (c < d) {
@@ -193,7 +196,7 @@ __global__ void __launch_bounds__(160, 1) pool_stream_kernel(PoolJob jq, PoolJob
         }
         job.out[unit * d + c] = __fdiv_rn(acc, static_cast<float>(rows));
       }
-      mbar_arrive(bar(2 + buf));
+      mbar_arrive(bar(kPoolStages + buf));
     }
   }
   __syncthreads();
@@ -216,7 +219,7 @@ cudaError_t launch_pool_prefill(const void* q, const void* k, bool bf16, int B, 
   const size_t unit_bytes = static_cast<size_t>(Hq / Hkv) * bs * d * esize;
   if (unit_bytes > kPoolStreamBytes || d > 128 || bs % 16 != 0 || (static_cast<size_t>(bs) * d * esize) % 16 != 0)
     return launch_pool_jobs(jq, jk, bf16, B, Hkv, N, d, bs, st);
-  const size_t smem = 2 * kPoolStreamBytes + 128;
+  const size_t smem = kPoolStages * kPoolStreamBytes + 128;
   const int64_t units = 2ll * B * Hkv * (N / bs);
   const unsigned grid = static_cast<unsigned>(units < num_sms ? units : num_sms);
   cudaError_t e;
@@ -644,12 +647,14 @@ __global__ void __launch_bounds__(128) topk_warp_kernel(const float* __restrict_
   uint32_t thresh = 0u;
   int remaining = take;     // how many keys equal to thresh are taken
   if (!take_all && take > 0) {
+    // slots past the candidates hold key 0, and every threshold tried has a
+    // bit set, so they never count: the counting loops need no bounds test
     uint32_t prefix = 0u;
     for (int bit = 31; bit >= 0; --bit) {
       const uint32_t cand = prefix | (1u << bit);
       int cnt = 0;
 #pragma unroll
-      for (int e = 0; e < KPL; ++e) cnt += (e * 32 + lane < ncand && key[e] >= cand) ? 1 : 0;
+      for (int e = 0; e < KPL; ++e) cnt += (key[e] >= cand) ? 1 : 0;
       cnt = __reduce_add_sync(0xffffffffu, cnt);
       if (cnt >= take) prefix = cand;
     }
