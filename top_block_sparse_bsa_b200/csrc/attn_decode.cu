@@ -127,19 +127,6 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
   return __all_sync(0xffffffffu, ok);
 }
 
-// Is key `kk` (0..127) of a step allowed for head slot h?  tile_a / tile_b
-// are the step's two tiles (tile_b < INT_MIN marks "no second tile").
-__device__ __forceinline__ bool key_allowed(int kk, int tile_a, int tile_b, bool has_b, const uint32_t* bits) {
-  const bool second = kk >= 64;
-  if (second && !has_b) return false;
-  const int tile = second ? tile_b : tile_a;
-  if (bits == nullptr) return true;                                  // plain decode
-  if (tile >= 0) return (bits[tile >> 5] >> (tile & 31)) & 1u;        // expanded chunk: its tokens
-  const int c = (-(tile + 1)) * 64 + (kk & 63);                      // gist of chunk c
-  return !((bits[c >> 5] >> (c & 31)) & 1u);                          // only if c is not expanded
-}
-
-
 // Softmax role (warps 0-3), specialised on GH >= G query heads per group:
 // only GH columns of S^T and O^T are read, reduced and written.
 template <int GH>
@@ -180,8 +167,22 @@ __device__ __forceinline__ void softmax_role(const Params& p, Misc* misc, uint8_
           l_part[h] = 0.0f;
         }
         const int nsteps = (n + 1) / 2;
+        const int words = p.nc / 32;
         for (int s = 0; s < nsteps; ++s) {
           const int sb = s_read & 1;
+          // this thread's key r lies in one tile of the step; in gist mode
+          // its allowance per head is one bit of that head's expanded-chunk
+          // bitmap, loaded here so the load overlaps the wait for S
+          const int ta = inf->tiles[2 * s];
+          const bool has_b = 2 * s + 1 < n;
+          const int tbv = has_b ? inf->tiles[2 * s + 1] : 0;
+          const bool has_mine = (r < 64) || has_b;
+          const int mytile = (r < 64) ? ta : tbv;
+          const int bitpos = (mytile >= 0) ? mytile : (-(mytile + 1)) * 64 + (r & 63);
+          uint32_t word[GH];
+#pragma unroll
+          for (int h = 0; h < GH; ++h)
+            word[h] = (gist && h < G && has_mine) ? __ldg(bits_base + h * words + (bitpos >> 5)) : 0u;
           if (!(ok = warp_wait(bar(BAR_SF + sb), (s_read >> 1) & 1, abortp, p.status))) break;
           tc_fence_after();
           uint32_t sv[GH];
@@ -189,14 +190,15 @@ __device__ __forceinline__ void softmax_role(const Params& p, Misc* misc, uint8_
           tc_fence_before();
           mbar_arrive(bar(BAR_SE + sb));   // S buffer may be rewritten
           ++s_read;
-          const int ta = inf->tiles[2 * s];
-          const bool has_b = 2 * s + 1 < n;
-          const int tbv = has_b ? inf->tiles[2 * s + 1] : 0;
           float x[GH];
 #pragma unroll
           for (int h = 0; h < GH; ++h) {
-            bool allowed = h < G;
-            if (allowed) allowed = key_allowed(r, ta, tbv, has_b, gist ? bits_base + h * (p.nc / 32) : nullptr);
+            bool allowed = h < G && has_mine;
+            if (allowed && gist) {
+              const bool bit = (word[h] >> (bitpos & 31)) & 1u;
+              // an expanded chunk's tokens, or the gist of a chunk not expanded
+              allowed = (mytile >= 0) ? bit : !bit;
+            }
             x[h] = allowed ? __uint_as_float(sv[h]) * p.scale_log2 : -INFINITY;
           }
           // tile maximum per head across the 128 keys
