@@ -464,10 +464,70 @@ __global__ void score_gist_kernel(const T* __restrict__ q, const T* __restrict__
         __fmul_rn(dot_fixed_order(qs + hh * d, ks + r * pitch, d, 1), scale);
 }
 
+// Gist, bf16, d = 128: grid (tiles of 64 gists, B*Hkv), 64*G threads = (head,
+// gist).  The tile's 64 gist keys are read with 16-byte loads (8 bf16 per
+// load, a warp covering 512 contiguous bytes) and widened into rows padded to
+// 132 floats, so float4 reads of eight consecutive rows fall in distinct
+// banks; each thread then runs the fixed-order dot product of its (head,
+// gist) pair, channels ascending, as the generic kernel does.
+__global__ void score_gist_bf16_d128_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ gk,
+                                            int Hq, int Hkv, int nc, float scale, float* __restrict__ s) {
+  constexpr int D = 128, kPitch = D + 4;
+  extern __shared__ __align__(16) float sm_gist[];
+  const int G = Hq / Hkv;
+  float* ks = sm_gist;                // [64][kPitch]
+  float* qs = sm_gist + 64 * kPitch;  // [G][D]
+  const int64_t bg = blockIdx.y;
+  const int64_t b = bg / Hkv, g = bg % Hkv;
+  const int c0 = blockIdx.x * 64;
+  const int rows = min(64, nc - c0);
+  const uint4* src = reinterpret_cast<const uint4*>(gk + (bg * nc + c0) * D);
+  for (int e = threadIdx.x; e < rows * (D / 8); e += blockDim.x) {
+    const int r = e >> 4, c8 = e & 15;   // row, 8-channel chunk
+    const uint4 v = __ldg(src + e);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+    float4 lo, hi;
+    float2 f;
+    f = __bfloat1622float2(h[0]); lo.x = f.x; lo.y = f.y;
+    f = __bfloat1622float2(h[1]); lo.z = f.x; lo.w = f.y;
+    f = __bfloat1622float2(h[2]); hi.x = f.x; hi.y = f.y;
+    f = __bfloat1622float2(h[3]); hi.z = f.x; hi.w = f.y;
+    float4* dst = reinterpret_cast<float4*>(ks + r * kPitch + 8 * c8);
+    dst[0] = lo;
+    dst[1] = hi;
+  }
+  for (int e = threadIdx.x; e < G * D; e += blockDim.x)
+    qs[e] = __bfloat162float(q[(b * Hq + g * G) * D + e]);
+  __syncthreads();
+  const int hh = threadIdx.x / 64, r = threadIdx.x % 64;
+  if (hh >= G || r >= rows) return;
+  const float4* kr = reinterpret_cast<const float4*>(ks + r * kPitch);
+  const float4* qr = reinterpret_cast<const float4*>(qs + hh * D);
+  float acc = 0.0f;
+#pragma unroll
+  for (int e = 0; e < D / 4; ++e) {
+    const float4 kv = kr[e], qv = qr[e];
+    acc = __fadd_rn(acc, __fmul_rn(qv.x, kv.x));
+    acc = __fadd_rn(acc, __fmul_rn(qv.y, kv.y));
+    acc = __fadd_rn(acc, __fmul_rn(qv.z, kv.z));
+    acc = __fadd_rn(acc, __fmul_rn(qv.w, kv.w));
+  }
+  s[((b * Hq + g * G + hh) * nc) + c0 + r] = __fmul_rn(acc, scale);
+}
+
 cudaError_t launch_score_gist(const void* q, const void* gk, bool bf16, int B, int Hq, int Hkv, int nc,
                               int d, float scale, float* s, cudaStream_t st) {
   const int G = Hq / Hkv;
   dim3 grid((nc + 63) / 64, B * Hkv);
+  if (bf16 && d == 128) {
+    const size_t smem2 = (64 * (128 + 4) + G * 128) * sizeof(float);
+    cudaError_t e = ensure_dynamic_smem<score_gist_bf16_d128_kernel>(smem2);
+    if (e != cudaSuccess) return e;
+    score_gist_bf16_d128_kernel<<<grid, 64 * G, smem2, st>>>(static_cast<const __nv_bfloat16*>(q),
+                                                             static_cast<const __nv_bfloat16*>(gk), Hq, Hkv, nc,
+                                                             scale, s);
+    return cudaGetLastError();
+  }
   const size_t smem = (G * d + 64 * (d + 1)) * sizeof(float);
   if (bf16)
     score_gist_kernel<__nv_bfloat16><<<grid, 64 * G, smem, st>>>(
