@@ -67,6 +67,46 @@ def dist_setup(args):
     return world, rank, local
 
 
+# ----------------------------------------------------------------------------
+# ranks: one process per GPU, each on its own independent problem (the path
+# shards by (batch, KV group) with no exchange step); the process group only
+# carries the barrier and the max-over-ranks timing.
+# ----------------------------------------------------------------------------
+
+def init_ranks(world: int, backend: str = "nccl", timeout_s: float = 120.0):
+    """The process group for world > 1 (None otherwise); a short timeout so
+    that ranks waiting for a rank that died end with an error."""
+    if world <= 1:
+        return None
+    import datetime
+    import torch.distributed as dist
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
+    return dist
+
+
+def rank_workload(base, rank: int):
+    """Rank r's independent problem: the same shapes, its own input seed."""
+    return base.scaled(seed=base.seed + 1000 * rank, name=base.name) if rank else base
+
+
+def reduce_over_ranks(dist, step_time: float, units: float, device=None):
+    """(max step time over ranks, units summed over ranks); identity for one rank."""
+    if dist is None:
+        return step_time, units
+    import torch
+    t = torch.tensor([step_time], dtype=torch.float64, device=device)
+    u = torch.tensor([units], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
+def close_ranks(dist):
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -261,17 +301,13 @@ def run_prefill(args, world, rank, local, peaks, peak_src):
     from top_block_sparse_bsa_b200 import accounting as acc
     from top_block_sparse_bsa_b200 import pipeline
 
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     torch.cuda.set_device(local)
+    dist = init_ranks(world)
     dev = torch.device("cuda", local)
     base = W.get(args.config)
     if args.batch:
         base = base.scaled(B=args.batch, name=base.name)
-    w = base.scaled(seed=base.seed + 1000 * rank, name=base.name) if rank else base
+    w = rank_workload(base, rank)
     inp = W.make_inputs(w, dev)
     q, k, v = inp["q"], inp["k"], inp["v"]
     step = pipeline.PrefillStep(q, k, v, w.bs, w.kb, gated=(w.kind == "gated"))
@@ -309,11 +345,9 @@ def run_prefill(args, world, rank, local, peaks, peak_src):
     sampler.stop()
     step_ms = ev0.elapsed_time(ev1) / args.steps
     attn_ms = statistics.mean(ka[s].elapsed_time(kb_[s]) for s in range(args.steps))
-    if dist:
-        t = torch.tensor([step_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_ms = float(t.item())
-    value = pairs * world / (step_ms / 1e3)
+    # whole job: the slowest rank's step, the pairs of every rank's problem
+    step_ms, job_pairs = reduce_over_ranks(dist, step_ms, pairs, device=dev)
+    value = job_pairs / (step_ms / 1e3)
 
     # roofline of the dominant kernel (sparse attention)
     sustained = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
@@ -362,12 +396,9 @@ def run_prefill(args, world, rank, local, peaks, peak_src):
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-        if dist:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms, _ = reduce_over_ranks(dist, e2e_ms, pairs, device=dev)
         h2d = (hq.numel() + hk.numel() + hv.numel()) * hq.element_size()
-        e2e = {"value": pairs * world / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        e2e = {"value": job_pairs / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": ho.numel() * ho.element_size(), "ms_per_step": e2e_ms}
 
     secondary = None
@@ -384,9 +415,7 @@ def run_prefill(args, world, rank, local, peaks, peak_src):
                                    f"random query rows of that group"),
                         "detail": detail}
 
-    if dist:
-        dist.barrier()
-        dist.destroy_process_group()
+    close_ranks(dist)
     if rank != 0:
         return 0
     line = {
@@ -463,10 +492,12 @@ def run_decode_like(args, world, rank, local, peaks, peak_src):
     from top_block_sparse_bsa_b200 import accounting as acc
     from top_block_sparse_bsa_b200 import pipeline
     torch.cuda.set_device(local)
+    dist = init_ranks(world)
     dev = torch.device("cuda", local)
-    w = W.get(args.config)
+    base = W.get(args.config)
     if args.batch:
-        w = w.scaled(B=args.batch, name=w.name)
+        base = base.scaled(B=args.batch, name=base.name)
+    w = rank_workload(base, rank)
     inp = W.make_inputs(w, dev)
     if w.kind == "decode":
         step = pipeline.DecodeStep(inp["q"], inp["k"], inp["v"], w.bs, w.kb)
@@ -507,6 +538,9 @@ def run_decode_like(args, world, rank, local, peaks, peak_src):
     stream = torch.cuda.current_stream()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     sampler = ClockSampler(local).start()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
     t0 = time.time()
     for s in range(args.steps):
         flush.fill_(s & 0xFF)
@@ -528,16 +562,23 @@ def run_decode_like(args, world, rank, local, peaks, peak_src):
     wait_gpu(ea[-1][1])
     attn_us = statistics.mean(1e3 * e[0].elapsed_time(e[1]) for e in ea)
     del g_step, g_sel, g_att
+    # whole job: every rank runs its own batch; a step takes the slowest rank's time
+    us, _ = reduce_over_ranks(dist, us, 1.0, device=dev)
+    attn_us, _ = reduce_over_ranks(dist, attn_us, 1.0, device=dev)
+    close_ranks(dist)
+    if rank != 0:
+        return 0
     gbs = nbytes / (attn_us / 1e6) / 1e9
     traffic, sha = profile_traffic(attn_file, f"attn_decode_{w.name}.md")
     if sha is not None and sha != kernel_source_sha(["attn_decode.cu", "common.cuh"]):
         traffic = None
     line = {
-        "metric": "us per decode step", "value": us, "unit": "us", "n_gpus": 1, "steps": args.steps,
+        "metric": "us per decode step", "value": us, "unit": "us", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": us / 1e3, "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "ctx": w.N, "block": w.bs,
-                   "budget": w.kb, "l2": "flushed (256 MiB write) before every step, outside the events",
+                   "budget": w.kb, "global_batch": w.B * world, "parallelism": f"independent problems x{world}",
+                   "l2": "flushed (256 MiB write) before every step, outside the events",
                    "launch": "CUDA graph replay of the C-ABI calls"},
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": gbs / peaks["hbm_gbs"], "traffic": traffic, "peak_source": peak_src,
