@@ -96,6 +96,15 @@ def test_tiny_prefill_f32_full_config(gated):
     _prefill_case(W.get("tiny_prefill_f32"), gated)
 
 
+@pytest.mark.parametrize("bs,hq", [(64, 1), (64, 3), (64, 5), (128, 1), (128, 3)])
+def test_prefill_bf16_ragged_tiles(bs, hq):
+    # G*bs stacked rows that do not fill 128-row tiles (64, 192, 320 rows at
+    # bs 64) and units with an odd tile count (single-tile items)
+    w = W.get("prefill_gqa_bf16").scaled(B=1, Hq=hq, Hkv=1, N=2048, bs=bs, kb=3)
+    _prefill_case(w, gated=False)
+    _prefill_case(w, gated=True)
+
+
 @pytest.mark.parametrize("kb", [4, 5])
 def test_prefill_gqa_bf16_small(kb):
     # 32 blocks, kept lists of odd and even length, two 128-row tiles per CTA

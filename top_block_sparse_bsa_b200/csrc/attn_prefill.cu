@@ -23,10 +23,15 @@
 // the previous item's tail and epilogue.
 //
 // Roles (384 threads, three warpgroups):
-//   warp 0      TMA producer: Q tiles per item, K and V of every step into a
-//               two-stage ring, gathered by block index;
+//   warp 0      TMA producer of Q (per item) and K (per step, two-stage
+//               ring, gathered by block index);
+//   warp 3      TMA producer of V (per step, two-stage ring): a separate
+//               thread, because the K ring drains after S and the V ring
+//               after O += P V;
 //   warp 1      TMEM owner + MMA issuer (one thread): S = Q K^T (SS form),
-//               O += P V (TS form, P read from tensor memory);
+//               O += P V (TS form, P read from tensor memory); per step it
+//               issues O += P V of the previous step before S of this one,
+//               tile by tile;
 //   warp 2      item loader: kept-block list and gate biases into a
 //               double-buffered metadata slot;
 //   warps 4-7   softmax + epilogue of tile 0 (thread = query row = TMEM lane);
@@ -42,7 +47,7 @@
 // block (bs = 128); the last step of an odd list holds one 64-token block.
 //
 // Softmax uses the base-2 exponent with the scale and the gate bias folded
-// into one FMA, and a lazy rescale: the running maximum is only moved (and O
+// into one packed (f32x2) FMA per key pair, and a lazy rescale: the running maximum is only moved (and O
 // rescaled in tensor memory) when a row's new maximum exceeds it by more than
 // 8 (a factor 256), which keeps every P <= 256 and is exact after the final
 // division.
