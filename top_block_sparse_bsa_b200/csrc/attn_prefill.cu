@@ -143,35 +143,61 @@ __device__ __forceinline__ void softmax_step(uint32_t t_s, uint32_t t_o, bool fi
                                              float bias1, bool diag0, bool diag1, int tb, float& m_run,
                                              float& l_run) {
   uint32_t v[KEYS];
-  if constexpr (KEYS == 128) {
-    tmem_ld128(t_s, v);
-  } else {
-    tmem_ld64(t_s, reinterpret_cast<uint32_t(&)[64]>(v));
-  }
-  if constexpr (MASK) {
+  constexpr int H0 = (BS == 64 && KEYS == 128) ? 64 : KEYS;
+  auto mask_range = [&](int c0, int c1) {
+    if constexpr (MASK) {
 #pragma unroll
-    for (int c = 0; c < KEYS; ++c) {
-      const bool second = (BS == 64) && (c >= 64);
-      const int koff = (BS == 64) ? (c & 63) : c;
-      if ((second ? diag1 : diag0) && koff > tb) v[c] = 0xFF800000u;   // -inf
+      for (int c = c0; c < c1; ++c) {
+        const bool second = (BS == 64) && (c >= 64);
+        const int koff = (BS == 64) ? (c & 63) : c;
+        if ((second ? diag1 : diag0) && koff > tb) v[c] = 0xFF800000u;   // -inf
+      }
     }
-  }
+  };
   // row maximum of the raw scores per block (the scale is positive and the
   // bias is constant over a block, so the maximum commutes with both);
   // three-input maxima in 8 independent chains
-  constexpr int H0 = (BS == 64 && KEYS == 128) ? 64 : KEYS;
-  auto block_max = [&](int c0, int c1) {
-    float m8[8];
+  float m8[8];
+  auto max_init = [&]() {
 #pragma unroll
     for (int a = 0; a < 8; ++a) m8[a] = -INFINITY;
+  };
+  auto max_acc = [&](int c0, int c1) {
 #pragma unroll
     for (int c = c0; c < c1; c += 2)
       m8[(c >> 1) & 7] = fmax3(m8[(c >> 1) & 7], __uint_as_float(v[c]), __uint_as_float(v[c + 1]));
+  };
+  auto max_fin = [&]() {
     return fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
   };
-  const float mx0 = block_max(0, H0);
+  float mx0, mx1 = -INFINITY;
+  if constexpr (KEYS == 128) {
+    // first 64 columns, then the second 64 in flight while the first are reduced
+    uint32_t(&lo)[64] = *reinterpret_cast<uint32_t(*)[64]>(&v[0]);
+    uint32_t(&hi)[64] = *reinterpret_cast<uint32_t(*)[64]>(&v[64]);
+    tmem_ld64(t_s, lo);
+    tmem_ld64_nowait(t_s + 64, hi);
+    mask_range(0, 64);
+    max_init();
+    max_acc(0, 64);
+    if constexpr (H0 < KEYS) {
+      mx0 = max_fin();
+      max_init();
+    }
+    tmem_wait_ld_tied64(hi);
+    mask_range(64, 128);
+    max_acc(64, 128);
+    if constexpr (H0 < KEYS) mx1 = max_fin();
+    else mx0 = max_fin();
+  } else {
+    tmem_ld64(t_s, reinterpret_cast<uint32_t(&)[64]>(v));
+    mask_range(0, KEYS);
+    max_init();
+    max_acc(0, KEYS);
+    mx0 = max_fin();
+  }
   float mx = fmaf(mx0, scale_log2, bias0);
-  if constexpr (H0 < KEYS) mx = fmaxf(mx, fmaf(block_max(H0, KEYS), scale_log2, bias1));
+  if constexpr (H0 < KEYS) mx = fmaxf(mx, fmaf(mx1, scale_log2, bias1));
   const float m_new = fmaxf(m_run, mx);
   const bool need = m_new > m_run + kRescaleThreshold;
   const float m_use = need ? m_new : m_run;
