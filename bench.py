@@ -217,6 +217,15 @@ def profile_traffic(kernel_file: str, summary_name: str):
     return float(m_t.group(1)), m_h.group(1)
 
 
+def prefill_kernel_of(w):
+    """The bf16 prefill kernel the library runs for this shape: units of an
+    odd number of 128-row tiles (G*bs rows) go to the split-half kernel."""
+    tiles = (w.G * w.bs + 127) // 128
+    if tiles % 2 == 1:
+        return "attn_prefill_split.cu", "attn_prefill_kernel (split halves, one tile per item)"
+    return "attn_prefill.cu", "attn_prefill_kernel (paired tiles)"
+
+
 def kernel_source_sha(files):
     h = hashlib.sha256()
     for f in files:
@@ -356,8 +365,9 @@ def run_prefill(args, world, rank, local, peaks, peak_src):
     hbm = peaks["hbm_gbs"]
     t_flop = flops / (burst * 1e12)
     t_hbm = kv_bytes / (hbm * 1e9)
-    traffic, sha = profile_traffic("attn_prefill.cu", f"attn_prefill_{w.name}.md")
-    if sha is not None and sha != kernel_source_sha(["attn_prefill.cu", "common.cuh"]):
+    kfile, kname = prefill_kernel_of(w)
+    traffic, sha = profile_traffic(kfile, f"{kfile[:-3]}_{w.name}.md")
+    if sha is not None and sha != kernel_source_sha([kfile, "common.cuh", "tmem_wide.cuh"]):
         traffic = None
     # The burst peak is the denominator: the clock samples of the timed region
     # show the SM clock at its maximum with no power-cap reason, i.e. the
@@ -368,7 +378,7 @@ def run_prefill(args, world, rank, local, peaks, peak_src):
         "frac": achieved_tflops / burst, "traffic": traffic,
         "peak_source": f"{peak_src} bf16 burst (cuBLAS GEMM timed alone)",
         "frac_of_sustained_peak": achieved_tflops / sustained,
-        "kernel": "attn_prefill_kernel", "kernel_ms": attn_ms,
+        "kernel": kname, "kernel_ms": attn_ms,
         "algorithmic_flop_per_launch": flops, "selected_kv_bytes_per_launch": kv_bytes,
         "roofline_time_ms": 1e3 * max(t_flop, t_hbm),
         "frac_of_roofline_time": (1e3 * max(t_flop, t_hbm)) / attn_ms,

@@ -16,7 +16,9 @@
 // each are stacked into G*bs rows that all read the same K/V tiles.  An item
 // is two 128-row tiles of one unit ("ping-pong": while one tile's softmax
 // runs on CUDA cores, the tensor core works on the other tile), so each K/V
-// tile is fetched into shared memory once for 256 query rows.  The kernel is
+// tile is fetched into shared memory once for 256 query rows.  Units with an
+// odd number of tiles go to the split-half kernel (attn_prefill_split.cu),
+// which runs one tile per item with two S buffers.  The kernel is
 // persistent: one CTA per SM walks items blockIdx.x, +gridDim.x, ... (heavy
 // items first); the K/V ring, the item metadata and the Q buffer roll over
 // from one item to the next, so the next item's loads and first MMAs overlap
@@ -672,6 +674,8 @@ cudaError_t launch_attn_prefill_bf16(const CUtensorMap* tmQ, const CUtensorMap* 
   p.G = a.Hq / a.Hkv;
   p.rows_per_unit = p.G * a.bs;
   p.tiles_per_unit = (p.rows_per_unit + 127) / 128;
+  // an odd tile count would leave one tile per unit without a partner
+  if (p.tiles_per_unit % 2 == 1) return launch_attn_prefill_split_bf16(tmQ, tmK, tmV, a, st);
   p.ctas_per_unit = (p.tiles_per_unit + 1) / 2;
   const int64_t items = static_cast<int64_t>(a.B) * a.Hkv * p.nb * p.ctas_per_unit;
   if (items <= 0) return cudaSuccess;
