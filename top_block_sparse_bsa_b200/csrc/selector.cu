@@ -116,11 +116,12 @@ static cudaError_t launch_pool_jobs(const PoolJob& j0, const PoolJob& j1, bool b
 }
 
 // Streamed variant (persistent, one CTA per SM): a producer thread copies each
-// unit's rows (heads_sum runs of bs*d contiguous elements) into one of
-// kPoolStages shared-memory buffers with bulk copies while 128 threads sum an
-// earlier unit, column c by thread c, rows in the fixed order (two units stay
-// in flight per SM).  Units of the query job come first, then those of the
-// key job.
+// unit's rows (heads_sum runs of bs*d contiguous elements) into
+// kPoolStages shared-memory buffers with bulk copies, a chunk of whole runs
+// per buffer, while 128 threads sum earlier chunks, column c by thread c,
+// rows in the fixed order (head, then row), the running sum carried from one
+// chunk of a unit to the next.  Units of the query job come first, then those
+// of the key job.
 constexpr int kPoolStreamBytes = 64 * 1024;
 constexpr int kPoolStages = 3;
 
@@ -136,6 +137,8 @@ __global__ void __launch_bounds__(160, 1) pool_stream_kernel(PoolJob jq, PoolJob
   const int nb = N / bs;
   const int64_t units_per_job = static_cast<int64_t>(B) * Hgroups * nb;
   const int64_t units = units_per_job * (jk.src ? 2 : 1);
+  const uint32_t run = static_cast<uint32_t>(bs) * d * sizeof(T);       // one head's rows of a unit
+  const int runs_per_chunk = static_cast<int>(kPoolStreamBytes / run);   // >= 1 (checked by the launcher)
   if (threadIdx.x == 0) {
     for (int i = 0; i < kPoolStages; ++i) {
       mbar_init(bar(i), 1);
@@ -149,54 +152,60 @@ __global__ void __launch_bounds__(160, 1) pool_stream_kernel(PoolJob jq, PoolJob
   const int warp = threadIdx.x >> 5;
   if (warp == 4) {
     if ((threadIdx.x & 31) == 0) {
-      int k = 0;
-      int issued = 0;
-      for (int64_t u = blockIdx.x; u < units; u += gridDim.x, ++k) {
+      int k = 0;   // chunks issued
+      bool ok = true;
+      for (int64_t u = blockIdx.x; ok && u < units; u += gridDim.x) {
         const bool isk = u >= units_per_job;
         const PoolJob& job = isk ? jk : jq;
         const int64_t unit = isk ? u - units_per_job : u;
         const int64_t b = unit / (static_cast<int64_t>(Hgroups) * nb);
         const int64_t g = (unit / nb) % Hgroups;
         const int64_t j = unit % nb;
-        const int buf = k % kPoolStages, use = k / kPoolStages;
-        if (k >= kPoolStages && !mbar_wait(bar(kPoolStages + buf), (use - 1) & 1, ab, status)) break;
-        const uint32_t run = static_cast<uint32_t>(bs) * d * sizeof(T);
-        mbar_arrive_expect_tx(bar(buf), run * job.heads_sum);
         const T* src = static_cast<const T*>(job.src);
-        for (int hh = 0; hh < job.heads_sum; ++hh)
-          bulk_load(sb + buf * kPoolStreamBytes + hh * run,
-                    src + ((b * job.Hsrc + g * job.heads_sum + hh) * static_cast<int64_t>(N) + j * bs) * d, run,
-                    bar(buf));
-        ++issued;
+        for (int h0 = 0; h0 < job.heads_sum; h0 += runs_per_chunk, ++k) {
+          const int nr = min(runs_per_chunk, job.heads_sum - h0);
+          const int buf = k % kPoolStages, use = k / kPoolStages;
+          if (k >= kPoolStages && !(ok = mbar_wait(bar(kPoolStages + buf), (use - 1) & 1, ab, status))) break;
+          mbar_arrive_expect_tx(bar(buf), run * nr);
+          for (int hh = h0; hh < h0 + nr; ++hh)
+            bulk_load(sb + buf * kPoolStreamBytes + (hh - h0) * run,
+                      src + ((b * job.Hsrc + g * job.heads_sum + hh) * static_cast<int64_t>(N) + j * bs) * d, run,
+                      bar(buf));
+        }
       }
       if (*ab) {   // let the copies still in flight land before the CTA exits
-        for (int q = issued > kPoolStages ? issued - kPoolStages : 0; q < issued; ++q)
+        for (int q = k > kPoolStages ? k - kPoolStages : 0; q < k; ++q)
           mbar_drain(bar(q % kPoolStages), (q / kPoolStages) & 1);
       }
     }
   } else {
     const int c = threadIdx.x;   // column
-    int k = 0;
-    for (int64_t u = blockIdx.x; u < units; u += gridDim.x, ++k) {
+    int k = 0;   // chunks consumed
+    bool ok = true;
+    for (int64_t u = blockIdx.x; ok && u < units; u += gridDim.x) {
       const bool isk = u >= units_per_job;
       const PoolJob& job = isk ? jk : jq;
       const int64_t unit = isk ? u - units_per_job : u;
-      const int buf = k % kPoolStages, use = k / kPoolStages;
-      if (!mbar_wait(bar(buf), use & 1, ab, status)) break;
-      const T* sv = reinterpret_cast<const T*>(psmem + buf * kPoolStreamBytes);
-      const int rows = job.heads_sum * bs;   // a multiple of 16
-      if (c < d) {
-        float acc = 0.0f;
-        for (int r = 0; r < rows; r += 16) {
-          float x[16];
+      float acc = 0.0f;
+      for (int h0 = 0; h0 < job.heads_sum; h0 += runs_per_chunk, ++k) {
+        const int nr = min(runs_per_chunk, job.heads_sum - h0);
+        const int buf = k % kPoolStages, use = k / kPoolStages;
+        if (!(ok = mbar_wait(bar(buf), use & 1, ab, status))) break;
+        const T* sv = reinterpret_cast<const T*>(psmem + buf * kPoolStreamBytes);
+        const int rows = nr * bs;   // a multiple of 16
+        if (c < d) {
+          for (int r = 0; r < rows; r += 16) {
+            float x[16];
 #pragma unroll
-          for (int t = 0; t < 16; ++t) x[t] = static_cast<float>(sv[(r + t) * d + c]);
+            for (int t = 0; t < 16; ++t) x[t] = static_cast<float>(sv[(r + t) * d + c]);
 #pragma unroll
-          for (int t = 0; t < 16; ++t) acc = __fadd_rn(acc, x[t]);
+            for (int t = 0; t < 16; ++t) acc = __fadd_rn(acc, x[t]);
+          }
         }
-        job.out[unit * d + c] = __fdiv_rn(acc, static_cast<float>(rows));
+        mbar_arrive(bar(kPoolStages + buf));
       }
-      mbar_arrive(bar(kPoolStages + buf));
+      if (!ok) break;
+      if (c < d) job.out[unit * d + c] = __fdiv_rn(acc, static_cast<float>(job.heads_sum * bs));
     }
   }
   __syncthreads();
@@ -210,14 +219,15 @@ cudaError_t launch_pool(const void* src, bool bf16, int B, int Hsrc, int Hgroups
 }
 
 // Prefill: grouped queries (heads_sum G) and keys (heads_sum 1) in one launch
-// of the streamed kernel when a query unit fits a buffer and d <= 128.
+// of the streamed kernel when one head's rows of a unit fit a buffer and
+// d <= 128.
 cudaError_t launch_pool_prefill(const void* q, const void* k, bool bf16, int B, int Hq, int Hkv, int N, int d,
                                 int bs, float* qbar, float* kbar, int num_sms, uint32_t* status, cudaStream_t st) {
   const PoolJob jq{q, Hq, Hq / Hkv, qbar};
   const PoolJob jk{k, Hkv, 1, kbar};
   const size_t esize = bf16 ? 2 : 4;
-  const size_t unit_bytes = static_cast<size_t>(Hq / Hkv) * bs * d * esize;
-  if (unit_bytes > kPoolStreamBytes || d > 128 || bs % 16 != 0 || (static_cast<size_t>(bs) * d * esize) % 16 != 0)
+  const size_t run_bytes = static_cast<size_t>(bs) * d * esize;
+  if (run_bytes > kPoolStreamBytes || d > 128 || bs % 16 != 0 || run_bytes % 16 != 0)
     return launch_pool_jobs(jq, jk, bf16, B, Hkv, N, d, bs, st);
   const size_t smem = kPoolStages * kPoolStreamBytes + 128;
   const int64_t units = 2ll * B * Hkv * (N / bs);
