@@ -178,6 +178,39 @@ def test_prefill_empty_and_bad_lists():
     _status_clean()
 
 
+@pytest.mark.parametrize("hq,gated", [(10, False), (10, True), (8, False)])
+def test_prefill_empty_lists_between_items(hq, gated):
+    """Empty kept lists on a seeded half of the query blocks, with enough
+    units that every persistent CTA walks several items, so items without
+    keys sit between items with keys (G 5: three 128-row tiles per unit, the
+    one-tile-per-item kernel; G 4: two tiles, the paired kernel).  Both sides
+    get the oracle's index set with the same lists emptied; every output row
+    is compared, the emptied blocks' rows are exactly zero with LSE -inf."""
+    pipe = _pipe()
+    w = W.get("prefill_gqa_bf16").scaled(B=1, Hq=hq, Hkv=2, N=8192, kb=3)
+    inp = W.make_inputs(w, "cuda")
+    q, k, v = inp["q"], inp["k"], inp["v"]
+    step = pipe.PrefillStep(q, k, v, w.bs, w.kb, gated=gated)
+    step.select()
+    qc, kc, vc = q.float().cpu(), k.float().cpu(), v.float().cpu()
+    _, _, s, idx, _ = oracle.prefill_select(qc, kc, w.Hkv, w.bs, w.kb)
+    nb = w.N // w.bs
+    empty = np.random.default_rng(11).random((w.Hkv, nb)) < 0.5
+    idx = idx.copy()
+    idx[0][empty] = -1
+    step.attend(idx=torch.from_numpy(idx).cuda())
+    torch.cuda.synchronize()
+    _status_clean()
+    want, want_lse = oracle.attend_prefill(qc, kc, vc, w.bs, idx, gate_scores=s if gated else None)
+    got = step.bufs["o"].float().reshape(-1, w.d).cpu().numpy()
+    got_lse = step.bufs["lse"].reshape(-1).cpu().numpy().astype(np.float64)
+    _assert_close(got, want, TOL_BF16, "out")
+    fin = np.isfinite(want_lse)
+    assert (~fin).sum() > 0 and np.array_equal(np.isneginf(got_lse), ~fin), "LSE -inf rows differ"
+    _assert_close(got_lse[fin], want_lse[fin], dict(max_abs=2e-3, mean_abs=2e-4), "lse")
+    assert np.all(got[~fin] == 0.0), "rows of emptied blocks are not zero"
+
+
 # ----------------------------------------------------------------------------
 # top-k selection on crafted scores (ties, NaN, budgets)
 # ----------------------------------------------------------------------------
