@@ -218,8 +218,11 @@ def profile_traffic(kernel_file: str, summary_name: str):
 
 
 def prefill_kernel_of(w):
-    """The bf16 prefill kernel the library runs for this shape: units of an
-    odd number of 128-row tiles (G*bs rows) go to the split-half kernel."""
+    """The prefill kernel the library runs for this shape: fp32 inputs run the
+    SIMT kernel; bf16 units of an odd number of 128-row tiles (G*bs rows) go
+    to the split-half kernel, even counts to the paired-tile kernel."""
+    if w.dtype == "f32":
+        return "attn_f32.cu", "attn_prefill_f32_kernel"
     tiles = (w.G * w.bs + 127) // 128
     if tiles % 2 == 1:
         return "attn_prefill_split.cu", "attn_prefill_kernel (split halves, one tile per item)"
