@@ -88,3 +88,24 @@ def test_product_path_does_not_import_the_oracle():
                 src = open(os.path.join(dirpath, f), encoding="utf-8").read()
                 assert "import oracle" not in src and "from oracle" not in src, f
                 assert "bsa_oracle" not in src, f
+
+
+def test_build_compiles_every_kernel_source():
+    """libbsa.so is linked from exactly the .cu files under csrc/ (a source
+    left out would only show as an undefined symbol when the library loads)."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("_bsa_build_under_test",
+                                                  os.path.join(ROOT, "top_block_sparse_bsa_b200", "_build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    on_disk = sorted(f for f in os.listdir(mod.CSRC) if f.endswith(".cu"))
+    assert sorted(mod.SOURCES) == on_disk
+    headers = sorted(f for f in os.listdir(mod.CSRC) if f.endswith((".cuh", ".h")))
+    assert sorted(mod.HEADERS) == headers
+
+
+def test_library_has_no_undefined_bsa_symbols():
+    lib = os.path.join(ROOT, "top_block_sparse_bsa_b200", "libbsa.so")
+    out = subprocess.run(["nm", "-D", "--undefined-only", lib], capture_output=True, text=True, check=True).stdout
+    missing = [line for line in out.splitlines() if "bsa" in line]
+    assert not missing, missing
