@@ -22,7 +22,7 @@ both sides, so that does not matter.
 from __future__ import annotations
 
 import dataclasses
-from typing import Dict, Optional
+from typing import Dict
 
 import torch
 

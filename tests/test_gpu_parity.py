@@ -10,7 +10,6 @@ inputs) of the oracle's fp64 result.
 Small cases span several tiles and odd (ragged) kept lists and are checked on
 every output row; the full workload sizes are checked on sampled rows.
 """
-import math
 import os
 
 import numpy as np
@@ -113,7 +112,7 @@ def test_prefill_gqa_bf16_small(kb):
 
 
 def test_gated_bf16_small_group_of_seven():
-    # G = 7 heads x 128 rows: four CTAs per unit, the last with one tile
+    # G = 7 heads x 128 rows: seven tiles per unit, an odd count (one-tile-per-item kernel)
     w = W.get("gated_prefill_bf16").scaled(B=1, Hq=7, Hkv=1, N=2048, kb=3)
     _prefill_case(w, gated=True)
 
