@@ -52,7 +52,7 @@ def parse_args():
     ap.add_argument("--cpu-rows", type=int, default=65536, help="query rows in the oracle CPU-baseline sample")
     ap.add_argument("--ref-rows", type=int, default=1024, help="query rows per reference-arm step")
     ap.add_argument("--e2e-steps", type=int, default=5)
-    ap.add_argument("--no-secondary", action="store_true", help="skip the decode secondary figures")
+    ap.add_argument("--no-secondary", action="store_true", help="skip the other workloads' figures")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=0, help="override the workload batch (small profiling cases)")
     return ap.parse_args()
@@ -130,7 +130,7 @@ class ClockSampler:
         "hw_power_brake_slowdown": "nvmlClocksEventReasonHwPowerBrakeSlowdown",
     }
 
-    def __init__(self, device_index: int, period: float = 0.02):
+    def __init__(self, device_index: int, period: float = 0.001):
         self.samples = []
         self.period = period
         self._stop = threading.Event()
@@ -148,11 +148,14 @@ class ClockSampler:
 
     def _run(self):
         nv = self.nv
+        power, n = None, 0
         while not self._stop.is_set():
             try:
                 mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
                 reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                power = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                if n % 8 == 0:   # power changes slowly; read it on every eighth sample
+                    power = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                n += 1
                 self.samples.append((time.time(), mhz, reasons, power))
             except Exception:
                 pass
@@ -181,7 +184,8 @@ class ClockSampler:
                     active.add(name)
         return {"sm_mhz": statistics.median([s[1] for s in win]) if win else None,
                 "sm_max_mhz": self.max_mhz, "reasons": sorted(active),
-                "power_w_max": max(s[3] for s in win) if win else None, "samples": len(win)}
+                "power_w_max": max((s[3] for s in win if s[3] is not None), default=None),
+                "samples": len(win)}
 
 
 def wait_gpu(ev):
@@ -274,13 +278,34 @@ def oracle_prefill_sample(w, q, k, v, group: int, rows: int, seed: int):
     return pairs, charged, {"t_select_s": t_sel, "t_attend_s": t_att, "rows": int(len(flat))}
 
 
+def prefill_config(w, world: int) -> dict:
+    """The config object of a prefill line (both arms print the same one)."""
+    in_mib = (w.B * w.Hq * w.N + 2 * w.B * w.Hkv * w.N) * w.d * (2 if w.dtype == "bf16" else 4) / 2**20
+    l2_note = (f"inputs larger than L2 ({in_mib:.0f} MiB > 126 MiB)" if in_mib > 126 else
+               f"inputs fit in L2 ({in_mib:.1f} MiB): L2-warm timing of a small workload")
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "seq_len": w.N, "d": w.d,
+            "block": w.bs, "budget": f"{w.kb}+current", "gated": w.kind == "gated",
+            "global_batch": w.B * world, "parallelism": f"independent problems x{world}", "l2": l2_note,
+            "dense_causal_pairs": w.N * (w.N + 1) // 2 * w.B * w.Hq}
+
+
+def decode_config(w, world: int) -> dict:
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "ctx": w.N, "block": w.bs,
+            "budget": w.kb, "global_batch": w.B * world, "parallelism": f"independent problems x{world}",
+            "l2": "flushed (256 MiB write) before every step, outside the events",
+            "launch": "CUDA graph replay of the C-ABI calls"}
+
+
 def run_reference(args, world, rank):
     import bsa_workloads as W
     import oracle
-    import torch
     if rank != 0:
         return 0
     w = W.get(args.config)
+    if w.kind in ("decode", "gist"):
+        print(json.dumps({"impl": "reference", "unavailable": "the reference arm times the oracle on the "
+                          "prefill workloads only"}), flush=True)
+        return 0
     inp = W.make_inputs(w, "cpu")
     threads = oracle.max_threads()
     pairs_total, secs_total = 0, 0.0
@@ -297,7 +322,7 @@ def run_reference(args, world, rank):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs_total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": w.name},
+        "data": "synthetic", "config": prefill_config(w, args.gpus),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -309,25 +334,20 @@ def run_reference(args, world, rank):
 # our arm
 # ----------------------------------------------------------------------------
 
-def run_prefill(args, world, rank, local, peaks, peak_src):
+def measure_prefill(w, dev, steps: int, warmup: int, peaks, peak_src, dist=None):
+    """Times `steps` prefill steps (pool + score + top-k + sparse attention)
+    of workload w on one stream, the attention launch of each step between
+    its own pair of events.  Returns (figures, step object)."""
     import torch
-    import bsa_workloads as W
     from top_block_sparse_bsa_b200 import accounting as acc
     from top_block_sparse_bsa_b200 import pipeline
 
-    torch.cuda.set_device(local)
-    dist = init_ranks(world)
-    dev = torch.device("cuda", local)
-    base = W.get(args.config)
-    if args.batch:
-        base = base.scaled(B=args.batch, name=base.name)
-    w = rank_workload(base, rank)
+    import bsa_workloads as W
     inp = W.make_inputs(w, dev)
     q, k, v = inp["q"], inp["k"], inp["v"]
     step = pipeline.PrefillStep(q, k, v, w.bs, w.kb, gated=(w.kind == "gated"))
     stream = torch.cuda.current_stream()
-
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         step.run(with_lse=False)
     torch.cuda.synchronize()
     idx = step.bufs["idx"].cpu().numpy()
@@ -336,17 +356,17 @@ def run_prefill(args, world, rank, local, peaks, peak_src):
     kv_bytes = acc.prefill_kv_bytes(idx, w.bs, w.d, 2 if w.dtype == "bf16" else 4)
     full_pairs = acc.dense_pairs(w.N, causal=True) * w.B * w.Hq
 
-    sampler = ClockSampler(local).start()
+    sampler = ClockSampler(dev.index or 0).start()
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
-    ka = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    kb_ = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ka = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    kb_ = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     t_wall0 = time.time()
     ev0.record(stream)
-    for s in range(args.steps):
+    for s in range(steps):
         step.select()
         ka[s].record(stream)
         step.attend(with_lse=False)
@@ -357,13 +377,9 @@ def run_prefill(args, world, rank, local, peaks, peak_src):
     if dist:
         dist.barrier()
     sampler.stop()
-    step_ms = ev0.elapsed_time(ev1) / args.steps
-    attn_ms = statistics.mean(ka[s].elapsed_time(kb_[s]) for s in range(args.steps))
-    # whole job: the slowest rank's step, the pairs of every rank's problem
-    step_ms, job_pairs = reduce_over_ranks(dist, step_ms, pairs, device=dev)
-    value = job_pairs / (step_ms / 1e3)
+    step_ms = ev0.elapsed_time(ev1) / steps
+    attn_ms = statistics.mean(ka[s].elapsed_time(kb_[s]) for s in range(steps))
 
-    # roofline of the dominant kernel (sparse attention)
     sustained = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
     burst = peaks["bf16_tflops"]
     achieved_tflops = flops / (attn_ms / 1e3) / 1e12
@@ -395,7 +411,30 @@ def run_prefill(args, world, rank, local, peaks, peak_src):
         "frac_of_roofline_time": (1e3 * max(t_flop, t_hbm)) / attn_ms,
         "hbm_gbs_on_selected_bytes": kv_bytes / (attn_ms / 1e3) / 1e9,
     }
-    clocks = sampler.summary(t_wall0, t_wall1)
+    fig = {"step_ms": step_ms, "attn_ms": attn_ms, "pairs": pairs, "full_pairs": full_pairs,
+           "roofline": roofline, "clocks": sampler.summary(t_wall0, t_wall1),
+           "sparsity": acc.sparsity(pairs, full_pairs)}
+    return fig, step
+
+
+def run_prefill(args, world, rank, local, peaks, peak_src):
+    import torch
+    import bsa_workloads as W
+
+    torch.cuda.set_device(local)
+    dist = init_ranks(world)
+    dev = torch.device("cuda", local)
+    base = W.get(args.config)
+    if args.batch:
+        base = base.scaled(B=args.batch, name=base.name)
+    w = rank_workload(base, rank)
+    fig, step = measure_prefill(w, dev, args.steps, args.warmup, peaks, peak_src, dist)
+    pairs = fig["pairs"]
+    # whole job: the slowest rank's step, the pairs of every rank's problem
+    step_ms, job_pairs = reduce_over_ranks(dist, fig["step_ms"], pairs, device=dev)
+    value = job_pairs / (step_ms / 1e3)
+    stream = torch.cuda.current_stream()
+    q, k, v = step.q, step.k, step.v
 
     # end to end through the C ABI with host buffers
     e2e = None
@@ -421,14 +460,7 @@ def run_prefill(args, world, rank, local, peaks, peak_src):
         h2d = (hq.numel() + hk.numel() + hv.numel()) * hq.element_size()
         e2e = {"value": job_pairs / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": ho.numel() * ho.element_size(), "ms_per_step": e2e_ms}
-
-    secondary = None
-    if not args.no_secondary and world == 1:
-        secondary = {"decode": run_decode_secondary(dev, peaks)}
-
-    in_mib = (q.numel() + k.numel() + v.numel()) * q.element_size() / 2**20
-    l2_note = (f"inputs larger than L2 ({in_mib:.0f} MiB > 126 MiB)" if in_mib > 126 else
-               f"inputs fit in L2 ({in_mib:.1f} MiB): L2-warm timing of a small parity workload")
+        del hq, hk, hv, ho
 
     cpu_baseline = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -439,6 +471,12 @@ def run_prefill(args, world, rank, local, peaks, peak_src):
                                    f"sequence, charged pro rata, plus fp64 attention for {detail['rows']} "
                                    f"random query rows of that group"),
                         "detail": detail}
+    del step, q, k, v
+    torch.cuda.empty_cache()
+
+    secondary = None
+    if not args.no_secondary and world == 1:
+        secondary = run_secondaries(dev, peaks, peak_src, exclude=w.name)
 
     close_ranks(dist)
     if rank != 0:
@@ -447,15 +485,12 @@ def run_prefill(args, world, rank, local, peaks, peak_src):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "seq_len": w.N, "d": w.d,
-                   "block": w.bs, "budget": f"{w.kb}+current", "global_batch": w.B * world,
-                   "parallelism": f"independent problems x{world}",
-                   "l2": l2_note,
-                   "sparsity": acc.sparsity(pairs, full_pairs)},
-        "roofline": roofline,
+        "config": prefill_config(w, world),
+        "sparsity": fig["sparsity"],
+        "roofline": fig["roofline"],
         "cpu_baseline": cpu_baseline,
         "e2e": e2e,
-        "clocks": clocks,
+        "clocks": fig["clocks"],
         "gpu_launches": 5 * args.steps,
         "secondary": secondary,
     }
@@ -463,66 +498,44 @@ def run_prefill(args, world, rank, local, peaks, peak_src):
     return 0
 
 
-def run_decode_secondary(dev, peaks, iters: int = 20):
-    """µs per decode step and HBM GB/s over the selected bytes for the
-    131072-token decode workload, L2 flushed before every iteration."""
-    import torch
-    import bsa_workloads as W
-    from top_block_sparse_bsa_b200 import accounting as acc
-    from top_block_sparse_bsa_b200 import pipeline
-    w = W.get("decode_bf16")
-    inp = W.make_inputs(w, dev)
-    step = pipeline.DecodeStep(inp["q"], inp["k"], inp["v"], w.bs, w.kb)
-    step.pool_cache()
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    for _ in range(3):
-        step.run(with_lse=False)
-    torch.cuda.synchronize()
-    idx = step.bufs["idx"].cpu().numpy()
-    kv_bytes = acc.decode_kv_bytes(idx, w.bs, w.d, 2)
-    # the step as one graph; its attention part timed behind the selection
-    g_step = capture_graph(lambda: (step.select(), step.attend(with_lse=False)))
-    g_sel = capture_graph(step.select)
-    g_att = capture_graph(lambda: step.attend(with_lse=False))
-    stream = torch.cuda.current_stream()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(iters)]
-    for it in range(iters):
-        flush.fill_(it & 0xFF)
-        ev[it][0].record(stream)
-        g_step.replay()
-        ev[it][1].record(stream)
-        flush.fill_((it + 1) & 0xFF)
-        g_sel.replay()
-        ev[it][2].record(stream)
-        g_att.replay()
-        ev[it][3].record(stream)
-    torch.cuda.synchronize()
-    del g_step, g_sel, g_att
-    step_us = statistics.median(1e3 * e[0].elapsed_time(e[1]) for e in ev)
-    attn_us = statistics.median(1e3 * e[2].elapsed_time(e[3]) for e in ev)
-    gbs = kv_bytes / (attn_us / 1e6) / 1e9
-    del inp, step, flush
-    torch.cuda.empty_cache()
-    return {"workload": w.name, "us_per_step": step_us, "attn_us": attn_us, "selected_kv_bytes": kv_bytes,
-            "hbm_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
-            "roofline_us": kv_bytes / (peaks["hbm_gbs"] * 1e9) * 1e6, "l2": "flushed (256 MiB write) per iteration",
-            "launch": "CUDA graph replay of the C-ABI calls"}
+SECONDARY_STEPS, SECONDARY_WARMUP = 20, 5
 
 
-def run_decode_like(args, world, rank, local, peaks, peak_src):
-    """Decode or gist-decode workload: microseconds per step, HBM GB/s over
-    the bytes the attention must read, L2 flushed before every step."""
+def run_secondaries(dev, peaks, peak_src, exclude: str):
+    """One figure set per other workload, each with its own roofline, step
+    time and clock samples: the other prefill workloads (gated bf16, tiny
+    fp32) through measure_prefill, decode and gist decode through
+    measure_decode_like."""
     import torch
     import bsa_workloads as W
+    out = {}
+    for name in ("gated_prefill_bf16", "tiny_prefill_f32", "decode_bf16", "gist_decode_bf16"):
+        if name == exclude:
+            continue
+        w = W.get(name)
+        if w.kind in ("decode", "gist"):
+            fig = measure_decode_like(w, dev, SECONDARY_STEPS, SECONDARY_WARMUP, peaks, peak_src)
+            out[name] = {"metric": "us per decode step", "us_per_step": fig["us"], "attn_us": fig["attn_us"],
+                         "roofline": fig["roofline"], "clocks": fig["clocks"],
+                         "config": decode_config(w, 1), "gpu_launches_per_step": fig["launches"]}
+        else:
+            fig, step = measure_prefill(w, dev, SECONDARY_STEPS, SECONDARY_WARMUP, peaks, peak_src)
+            del step
+            out[name] = {"metric": METRIC, "value": fig["pairs"] / (fig["step_ms"] / 1e3), "unit": UNIT,
+                         "ms_per_step": fig["step_ms"], "roofline": fig["roofline"], "clocks": fig["clocks"],
+                         "config": prefill_config(w, 1), "sparsity": fig["sparsity"],
+                         "gpu_launches_per_step": 5}
+        torch.cuda.empty_cache()
+    return out
+
+
+def measure_decode_like(w, dev, steps: int, warmup: int, peaks, peak_src, dist=None):
+    """Decode or gist-decode workload: microseconds per step and HBM GB/s
+    over the bytes the attention must read, L2 flushed before every step."""
+    import torch
     from top_block_sparse_bsa_b200 import accounting as acc
     from top_block_sparse_bsa_b200 import pipeline
-    torch.cuda.set_device(local)
-    dist = init_ranks(world)
-    dev = torch.device("cuda", local)
-    base = W.get(args.config)
-    if args.batch:
-        base = base.scaled(B=args.batch, name=base.name)
-    w = rank_workload(base, rank)
+    import bsa_workloads as W
     inp = W.make_inputs(w, dev)
     if w.kind == "decode":
         step = pipeline.DecodeStep(inp["q"], inp["k"], inp["v"], w.bs, w.kb)
@@ -530,15 +543,15 @@ def run_decode_like(args, world, rank, local, peaks, peak_src):
         select = step.select
         attend = lambda: step.attend(with_lse=False)   # noqa: E731
         launches = 4   # score, top-k | split-K attention, combine
-        attn_file, attn_kernel = "attn_decode.cu", "attn_decode_kernel (+ combine_kernel)"
+        attn_kernel = "attn_decode_kernel (+ combine_kernel)"
     else:
         step = pipeline.GistStep(inp["q"], inp["k"], inp["v"], inp["gk"], inp["gv"], w.bs, w.kb)
         select = lambda: step.run(with_lse=False)   # noqa: E731  (the whole step in one call)
         attend = lambda: step.run(idx_in=step.bufs["idx"], with_lse=False)   # noqa: E731
         launches = 5   # gist score, top-k, union lists, split-K attention, combine
-        attn_file, attn_kernel = "attn_decode.cu", "gist_union_kernel + attn_decode_kernel + combine_kernel"
+        attn_kernel = "gist_union_kernel + attn_decode_kernel + combine_kernel"
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         select()
         attend()
     torch.cuda.synchronize()
@@ -561,13 +574,13 @@ def run_decode_like(args, world, rank, local, peaks, peak_src):
     g_sel = capture_graph(select) if w.kind == "decode" else None
     g_att = capture_graph(attend)
     stream = torch.cuda.current_stream()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-    sampler = ClockSampler(local).start()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    sampler = ClockSampler(dev.index or 0).start()
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     t0 = time.time()
-    for s in range(args.steps):
+    for s in range(steps):
         flush.fill_(s & 0xFF)
         ev[s][0].record(stream)
         g_step.replay()
@@ -576,8 +589,8 @@ def run_decode_like(args, world, rank, local, peaks, peak_src):
     t1 = time.time()
     sampler.stop()
     us = statistics.mean(1e3 * e[0].elapsed_time(e[1]) for e in ev)
-    ea = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-    for s in range(args.steps):
+    ea = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    for s in range(steps):
         flush.fill_(s & 0xFF)
         if g_sel is not None:
             g_sel.replay()
@@ -587,29 +600,48 @@ def run_decode_like(args, world, rank, local, peaks, peak_src):
     wait_gpu(ea[-1][1])
     attn_us = statistics.mean(1e3 * e[0].elapsed_time(e[1]) for e in ea)
     del g_step, g_sel, g_att
+    gbs = nbytes / (attn_us / 1e6) / 1e9
+    traffic, sha = profile_traffic("attn_decode.cu", f"attn_decode_{w.name}.md")
+    if sha is not None and sha != kernel_source_sha(["attn_decode.cu", "common.cuh"]):
+        traffic = None
+    roofline = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": gbs / peaks["hbm_gbs"], "traffic": traffic, "peak_source": peak_src,
+                "kernel": attn_kernel, "kernel_us": attn_us, "selected_kv_bytes_per_launch": nbytes,
+                "step_gbs": nbytes / (us / 1e6) / 1e9, "roofline_us": nbytes / (peaks["hbm_gbs"] * 1e9) * 1e6}
+    fig = {"us": us, "attn_us": attn_us, "nbytes": nbytes, "roofline": roofline,
+           "clocks": sampler.summary(t0, t1), "launches": launches}
+    del step, inp, flush
+    return fig
+
+
+def run_decode_like(args, world, rank, local, peaks, peak_src):
+    import torch
+    import bsa_workloads as W
+    torch.cuda.set_device(local)
+    dist = init_ranks(world)
+    dev = torch.device("cuda", local)
+    base = W.get(args.config)
+    if args.batch:
+        base = base.scaled(B=args.batch, name=base.name)
+    w = rank_workload(base, rank)
+    fig = measure_decode_like(w, dev, args.steps, args.warmup, peaks, peak_src, dist)
     # whole job: every rank runs its own batch; a step takes the slowest rank's time
-    us, _ = reduce_over_ranks(dist, us, 1.0, device=dev)
-    attn_us, _ = reduce_over_ranks(dist, attn_us, 1.0, device=dev)
+    us, _ = reduce_over_ranks(dist, fig["us"], 1.0, device=dev)
+    attn_us, _ = reduce_over_ranks(dist, fig["attn_us"], 1.0, device=dev)
     close_ranks(dist)
     if rank != 0:
         return 0
-    gbs = nbytes / (attn_us / 1e6) / 1e9
-    traffic, sha = profile_traffic(attn_file, f"attn_decode_{w.name}.md")
-    if sha is not None and sha != kernel_source_sha(["attn_decode.cu", "common.cuh"]):
-        traffic = None
+    roofline = dict(fig["roofline"])
+    gbs = fig["nbytes"] / (attn_us / 1e6) / 1e9
+    roofline.update(achieved=gbs, frac=gbs / peaks["hbm_gbs"], kernel_us=attn_us,
+                    step_gbs=fig["nbytes"] / (us / 1e6) / 1e9)
     line = {
         "metric": "us per decode step", "value": us, "unit": "us", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": us / 1e3, "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "ctx": w.N, "block": w.bs,
-                   "budget": w.kb, "global_batch": w.B * world, "parallelism": f"independent problems x{world}",
-                   "l2": "flushed (256 MiB write) before every step, outside the events",
-                   "launch": "CUDA graph replay of the C-ABI calls"},
-        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": gbs / peaks["hbm_gbs"], "traffic": traffic, "peak_source": peak_src,
-                     "kernel": attn_kernel, "kernel_us": attn_us, "selected_kv_bytes_per_launch": nbytes,
-                     "step_gbs": nbytes / (us / 1e6) / 1e9},
-        "clocks": sampler.summary(t0, t1), "gpu_launches": launches * args.steps,
+        "config": decode_config(w, world),
+        "roofline": roofline,
+        "clocks": fig["clocks"], "gpu_launches": fig["launches"] * args.steps,
     }
     print(json.dumps(line), flush=True)
     return 0

@@ -35,7 +35,8 @@
  *              kernel records a flag in the device status word, skips the bad
  *              work and returns; read it with bsa_device_status().
  *   Threads    calls are thread-safe; the only global state is the tensor-map
- *              entry point and the device status word.
+ *              entry point, the device status word and the decode split
+ *              override of the testing hooks below.
  */
 #ifndef BSA_H_
 #define BSA_H_
@@ -216,8 +217,9 @@ bsa_status_t bsa_gist_expand_decode(const bsa_shape_t* shape, const void* q, con
  * Arguments, layouts and results are those of bsa_sparse_attn_decode.
  * Returns BSA_ERR_UNSUPPORTED, before launching anything, when the shape
  * needs more than 4 MiB of scratch (bsa_workspace_bytes(BSA_OP_DECODE, ...)).
- * The first call on a device looks up the array's device address; make that
- * first call before any stream capture.  All calls on a device share the
+ * The first call on a device (and the first after a device reset, which
+ * reloads the library's module) looks up the array's device address; make
+ * that first call before any stream capture.  All calls on a device share the
  * array: calls whose work may overlap on the GPU (unordered streams) race.
  * Nothing in the array needs to start zeroed between calls.
  * Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
@@ -240,6 +242,30 @@ bsa_status_t bsa_device_status(unsigned int* flags, int reset);
 
 /* Library ABI version (major*100 + minor). */
 int bsa_version(void);
+
+/*
+ * Testing and tuning hooks (no counterpart on the source pages).
+ *
+ * bsa_decode_split_override -- fixes the number of split-K ranges the decode
+ * calls cut a batch's kept-block lists into (num_splits > 0), or restores the
+ * default of one range per SM (num_splits <= 0).  Process-wide; returns the
+ * previous setting (0 = default).  It changes bsa_workspace_bytes() for the
+ * decode operations too, so set it before sizing a workspace, and do not
+ * change it while a decode call is being enqueued on another thread.  The
+ * result of a decode does not depend on it beyond fp32 rounding order.
+ */
+int bsa_decode_split_override(int num_splits);
+
+/*
+ * bsa_selftest_wait_expiry -- enqueues a one-thread kernel that waits, with
+ * a budget of budget_cycles SM cycles, on a shared-memory barrier nothing
+ * arrives on, through the same bounded-wait helper every kernel uses.  The
+ * wait expires, BSA_DEV_TIMEOUT is raised in the device status word and the
+ * kernel returns; bsa_device_status() then reports BSA_ERR_TIMEOUT.  It
+ * exists to test that expiry path; it faults nothing and leaves the device
+ * usable.  budget_cycles < 0 -> BSA_ERR_INVALID_ARG.
+ */
+bsa_status_t bsa_selftest_wait_expiry(long long budget_cycles, void* stream);
 
 #ifdef __cplusplus
 }

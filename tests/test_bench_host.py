@@ -40,3 +40,14 @@ def test_committed_prefill_summaries_carry_traffic_and_source_hash():
         traffic, sha = b.profile_traffic(kfile, f"{kfile[:-3]}_{name}.md")
         assert traffic is not None and traffic > 0, name
         assert sha is not None and len(sha) == 64, name
+
+
+def test_reference_arm_prints_the_same_config_as_ours():
+    """Both arms describe the workload with the same config object, so the
+    two lines can be matched config for config."""
+    b = _bench()
+    for name in ("prefill_gqa_bf16", "gated_prefill_bf16", "tiny_prefill_f32"):
+        w = W.get(name)
+        c = b.prefill_config(w, 1)
+        assert c["workload"] == name and c["seq_len"] == w.N and c["Hq"] == w.Hq
+        assert c == b.prefill_config(W.get(name), 1)

@@ -10,8 +10,6 @@ inputs) of the oracle's fp64 result.
 Small cases span several tiles and odd (ragged) kept lists and are checked on
 every output row; the full workload sizes are checked on sampled rows.
 """
-import os
-
 import numpy as np
 import pytest
 import torch
@@ -144,6 +142,60 @@ def test_prefill_gqa_bf16_full_size_sampled():
 def test_gated_bf16_full_size_sampled():
     w = W.get("gated_prefill_bf16")
     _prefill_case(w, gated=True, rows_sample=_sample_rows(w, 96, 3))
+
+
+@pytest.mark.parametrize("fp32_d", [128])
+@pytest.mark.parametrize("gated", [False, True])
+def test_tiny_prefill_f32_head_dim_128(fp32_d, gated):
+    # the fp32 path at the other head dimension it is built for
+    w = W.get("tiny_prefill_f32").scaled(d=fp32_d)
+    _prefill_case(w, gated)
+
+
+# Budgets at or above the number of history blocks: every block j <= i is
+# kept, so the sparse result must be dense causal attention (the tutorial's
+# softmax(QK^T/sqrt(d))V with the causal mask, §1).  These runs also reach the
+# longest kept lists the prefill kernels take.
+@pytest.mark.parametrize("hq,gated", [(4, False), (4, True), (5, False), (5, True)])
+def test_prefill_bf16_full_budget_dense_causal(hq, gated):
+    # G 4: 256 stacked rows, two tiles (paired kernel); G 5: 320 rows, three
+    # tiles (one-tile-per-item kernel).  128 blocks, budget 127 + current.
+    w = W.get("prefill_gqa_bf16").scaled(B=1, Hq=hq, Hkv=1, N=8192, kb=127)
+    _prefill_case(w, gated=gated)
+
+
+def test_gated_bf16_block128_full_budget_group_of_seven():
+    # 128-token blocks, G 7 (seven tiles per unit), 64 blocks, budget 63 + current
+    w = W.get("gated_prefill_bf16").scaled(B=1, Hq=7, Hkv=1, N=8192, kb=63)
+    _prefill_case(w, gated=True)
+
+
+def test_prefill_bf16_longest_lists():
+    """256 blocks with budget 255 + current: kept lists of up to 256 entries,
+    the longest the prefill entry points accept (idx_stride <= 256)."""
+    w = W.get("prefill_gqa_bf16").scaled(B=1, Hq=4, Hkv=1, N=16384, kb=255)
+    _prefill_case(w, gated=False)
+
+
+def test_prefill_full_budget_equals_dense_causal_closed_form():
+    """The closed form itself, on the GPU output: at full budget the sparse
+    prefill equals dense causal attention computed as one fp64 softmax over
+    every earlier token (no index list involved)."""
+    w = W.get("prefill_gqa_bf16").scaled(B=1, Hq=4, Hkv=1, N=2048, kb=31)
+    pipe = _pipe()
+    inp = W.make_inputs(w, "cuda")
+    step = pipe.PrefillStep(inp["q"], inp["k"], inp["v"], w.bs, w.kb)
+    step.run()
+    torch.cuda.synchronize()
+    _status_clean()
+    q = inp["q"].double().cpu()[0]
+    k = inp["k"].double().cpu()[0, 0]
+    v = inp["v"].double().cpu()[0, 0]
+    logits = torch.einsum("htd,ud->htu", q, k) / np.sqrt(w.d)
+    causal = torch.ones(w.N, w.N, dtype=torch.bool).tril()
+    logits = logits.masked_fill(~causal, float("-inf"))
+    want = torch.softmax(logits, dim=-1) @ v
+    _assert_close(step.bufs["o"][0].float().cpu().numpy(), want.numpy(), TOL_BF16, "dense causal")
 
 
 def test_prefill_empty_and_bad_lists():
@@ -290,9 +342,39 @@ def test_decode_bf16_small_even_list_and_full_budget():
     _decode_case(w)
 
 
-def test_decode_bf16_full_size_sampled():
+def test_decode_bf16_full_size_every_row():
+    """The full decode workload (16 sequences x 131072 cached tokens): pooled
+    keys, scores and kept indices of all 128 (sequence, group) rows compared
+    bit for bit, and the outputs of all 512 query heads against the oracle,
+    one sequence at a time on the host."""
+    pipe = _pipe()
     w = W.get("decode_bf16")
-    _decode_case(w, groups=[(0, 0), (5, 3), (15, 7), (9, 1)])
+    inp = W.make_inputs(w, "cuda")
+    q, kc, vc = inp["q"], inp["k"], inp["v"]
+    step = pipe.DecodeStep(q, kc, vc, w.bs, w.kb)
+    step.pool_cache()
+    step.select()
+    torch.cuda.synchronize()
+    b_ = step.bufs
+    idx_gpu = b_["idx"].cpu().numpy()
+    oracle_idx = np.empty_like(idx_gpu)
+    for b in range(w.B):
+        kbar = oracle.pool_keys(kc[b:b + 1].float().cpu(), w.bs)
+        assert np.array_equal(b_["kbar"][b:b + 1].cpu().numpy(), kbar), b
+        _, s, idx, _ = oracle.decode_select(q[b:b + 1].float().cpu(), kbar, w.Hkv, w.kb)
+        assert np.array_equal(b_["scores"][b:b + 1].cpu().numpy(), s), b
+        assert np.array_equal(idx_gpu[b:b + 1], idx), b
+        oracle_idx[b] = idx[0]
+    step.attend(idx=torch.from_numpy(oracle_idx).cuda())
+    torch.cuda.synchronize()
+    _status_clean()
+    got = b_["o"].float().cpu().numpy()
+    got_lse = b_["lse"].cpu().numpy()
+    for b in range(w.B):
+        want, want_lse = oracle.attend_decode(q[b:b + 1].float().cpu(), kc[b:b + 1].float().cpu(),
+                                              vc[b:b + 1].float().cpu(), w.bs, oracle_idx[b:b + 1])
+        _assert_close(got[b], want, TOL_BF16, f"decode sequence {b}")
+        _assert_close(got_lse[b], want_lse, dict(max_abs=2e-3, mean_abs=2e-4), f"decode lse {b}")
 
 
 @pytest.mark.parametrize("hq,hkv", [(2, 2), (4, 2), (16, 2), (32, 2)])
@@ -309,8 +391,8 @@ def test_decode_split_count_invariance():
     w = W.get("decode_bf16").scaled(B=2, Hq=8, Hkv=2, N=8192, kb=40)
     inp = W.make_inputs(w, "cuda")
     outs = []
-    for splits in ("1", "3", "7"):
-        os.environ["BSA_DECODE_SPLITS"] = splits
+    for splits in (1, 3, 7, 0):
+        prev = bsa.bsa_decode_split_override(splits)
         try:
             step = pipe.DecodeStep(inp["q"], inp["k"], inp["v"], w.bs, w.kb)
             step.pool_cache()
@@ -318,9 +400,32 @@ def test_decode_split_count_invariance():
             torch.cuda.synchronize()
             outs.append(step.bufs["o"].float().cpu())
         finally:
-            del os.environ["BSA_DECODE_SPLITS"]
+            bsa.bsa_decode_split_override(prev)
     for o in outs[1:]:
         assert (o - outs[0]).abs().max().item() <= 1e-2
+    _status_clean()
+
+
+def test_bounded_wait_expiry_reports_timeout_and_leaves_the_device_usable():
+    """The bounded-wait expiry path: a self-test kernel waits, through the
+    same helper every kernel uses, on a barrier nothing arrives on, with a
+    budget of 1e5 cycles.  It returns, the status word reports a timeout, a
+    reset clears it, and a following real call runs clean."""
+    bsa = _bsa()
+    pipe = _pipe()
+    bsa.bsa_device_status(reset=True)
+    bsa.bsa_selftest_wait_expiry(100_000)
+    code, flags = bsa.bsa_device_status(reset=True)
+    assert code == bsa.BSA_ERR_TIMEOUT and flags & 1, (code, flags)
+    code, flags = bsa.bsa_device_status(reset=False)
+    assert code == 0 and flags == 0
+    w = W.get("decode_bf16").scaled(B=1, Hq=8, Hkv=2, N=4096, kb=6)
+    inp = W.make_inputs(w, "cuda")
+    step = pipe.DecodeStep(inp["q"], inp["k"], inp["v"], w.bs, w.kb)
+    step.pool_cache()
+    step.run()
+    torch.cuda.synchronize()
+    assert torch.isfinite(step.bufs["o"].float()).all()
     _status_clean()
 
 
@@ -413,9 +518,29 @@ def test_gist_group_widths(hq, hkv):
     _gist_case(w)
 
 
-def test_gist_bf16_full_size_sampled():
+def test_gist_bf16_full_size_every_group():
+    """The full gist workload (8 sequences x 131072 tokens, 2048 gists): the
+    chosen chunks of all 256 query heads compared exactly, and the outputs of
+    all 256 heads against the oracle, one sequence at a time on the host."""
+    pipe = _pipe()
     w = W.get("gist_decode_bf16")
-    _gist_case(w, groups=[(0, 0), (3, 5), (7, 7)])
+    inp = W.make_inputs(w, "cuda")
+    step = pipe.GistStep(inp["q"], inp["k"], inp["v"], inp["gk"], inp["gv"], w.bs, w.kb)
+    step.run()
+    torch.cuda.synchronize()
+    _status_clean()
+    got_idx = step.bufs["idx"].cpu().numpy()
+    got = step.bufs["o"].float().cpu().numpy()
+    got_lse = step.bufs["lse"].cpu().numpy()
+    for b in range(w.B):
+        qs = inp["q"][b:b + 1].float().cpu()
+        gks = inp["gk"][b:b + 1].float().cpu()
+        _, idx, _ = oracle.gist_select(qs, gks, w.kb)
+        assert np.array_equal(got_idx[b:b + 1], idx), b
+        want, want_lse = oracle.attend_gist(qs, inp["k"][b:b + 1].float().cpu(), inp["v"][b:b + 1].float().cpu(),
+                                            gks, inp["gv"][b:b + 1].float().cpu(), w.bs, idx)
+        _assert_close(got[b], want, TOL_BF16, f"gist sequence {b}")
+        _assert_close(got_lse[b], want_lse, dict(max_abs=2e-3, mean_abs=2e-4), f"gist lse {b}")
 
 
 def test_gist_injected_index_set():

@@ -53,6 +53,38 @@ def test_noalloc_decode_matches_workspace_decode_twice():
     assert code == 0 and flags == 0
 
 
+def test_noalloc_decode_after_a_call_with_another_split_layout():
+    """Stale partial records: a call with many split ranges (the scratch laid
+    out with more slots per row) runs first, then calls with the default
+    plan read the same array.  Each result must still equal the workspace
+    decode run with the same plan."""
+    import top_block_sparse_bsa_b200 as bsa
+    from top_block_sparse_bsa_b200 import pipeline
+    torch.cuda.set_device(0)
+    w = W.get("decode_bf16").scaled(B=2, Hq=8, Hkv=2, N=8192, kb=40, seed=5)
+    inp = W.make_inputs(w, "cuda")
+    scale = 1.0 / math.sqrt(w.d)
+    for splits in (61, 0, 7):
+        prev = bsa.bsa_decode_split_override(splits)
+        try:
+            step = pipeline.DecodeStep(inp["q"], inp["k"], inp["v"], w.bs, w.kb)
+            step.pool_cache()
+            step.run()
+            torch.cuda.synchronize()
+            idx = step.bufs["idx"]
+            o = torch.full_like(step.bufs["o"], float("nan"))
+            lse = torch.full_like(step.bufs["lse"], float("nan"))
+            bsa.bsa_sparse_attn_decode_noalloc(step.shape, inp["q"], inp["k"], inp["v"], idx, idx.shape[-1],
+                                               scale, o, lse)
+            torch.cuda.synchronize()
+            assert torch.equal(o, step.bufs["o"]), splits
+            assert torch.equal(lse, step.bufs["lse"]), splits
+        finally:
+            bsa.bsa_decode_split_override(prev)
+    code, flags = bsa.bsa_device_status(reset=True)
+    assert code == 0 and flags == 0
+
+
 def test_noalloc_decode_rejects_shapes_beyond_its_scratch():
     import top_block_sparse_bsa_b200 as bsa
     torch.cuda.set_device(0)

@@ -24,7 +24,8 @@ __all__ = [
     "make_shape", "bsa_score_blocks", "bsa_topk_select", "bsa_sparse_attn_prefill",
     "bsa_gated_attn_fwd", "bsa_sparse_attn_decode", "bsa_gist_expand_decode",
     "bsa_workspace_bytes", "bsa_status_string", "bsa_device_status", "bsa_version",
-    "bsa_sparse_attn_decode_noalloc", "EXPORTED_SYMBOLS",
+    "bsa_sparse_attn_decode_noalloc", "bsa_decode_split_override", "bsa_selftest_wait_expiry",
+    "EXPORTED_SYMBOLS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libbsa.so")
@@ -40,6 +41,7 @@ EXPORTED_SYMBOLS = (
     "bsa_score_blocks", "bsa_topk_select", "bsa_sparse_attn_prefill", "bsa_gated_attn_fwd",
     "bsa_sparse_attn_decode", "bsa_gist_expand_decode", "bsa_workspace_bytes",
     "bsa_status_string", "bsa_device_status", "bsa_version", "bsa_sparse_attn_decode_noalloc",
+    "bsa_decode_split_override", "bsa_selftest_wait_expiry",
 )
 
 
@@ -75,6 +77,8 @@ _SIGS = {
     "bsa_status_string": (ctypes.c_char_p, [_i]),
     "bsa_device_status": (_i, [ctypes.POINTER(ctypes.c_uint), _i]),
     "bsa_version": (_i, []),
+    "bsa_decode_split_override": (_i, [_i]),
+    "bsa_selftest_wait_expiry": (_i, [ctypes.c_longlong, _p]),
 }
 
 
@@ -147,6 +151,16 @@ def bsa_device_status(reset: bool = False):
     flags = ctypes.c_uint(0)
     code = lib.bsa_device_status(ctypes.byref(flags), 1 if reset else 0)
     return int(code), int(flags.value)
+
+
+def bsa_decode_split_override(num_splits: int) -> int:
+    """Fix the decode split-K range count (> 0) or restore the default (<= 0); returns the previous setting."""
+    return int(lib.bsa_decode_split_override(int(num_splits)))
+
+
+def bsa_selftest_wait_expiry(budget_cycles: int, stream=None) -> None:
+    """Enqueue the bounded-wait expiry self-test kernel (sets BSA_DEV_TIMEOUT in the status word)."""
+    _check("bsa_selftest_wait_expiry", lib.bsa_selftest_wait_expiry(int(budget_cycles), _stream(stream)))
 
 
 def bsa_workspace_bytes(op: int, shape: BsaShape, budget: int) -> int:

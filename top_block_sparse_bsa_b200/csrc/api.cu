@@ -2,8 +2,8 @@
 // tensor maps, workspace layout and kernel dispatch.  No call here allocates
 // or frees device memory; scratch comes from the caller.
 #include <math.h>
-#include <stdlib.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "../../include/bsa.h"
@@ -20,23 +20,48 @@ namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 uint32_t* g_status_ptr[kMaxDevices] = {};
+uint64_t g_status_ctx[kMaxDevices] = {};
 int g_num_sms[kMaxDevices] = {};
+
+// Split-count override of the decode plan (0: one split range per SM); set
+// only through bsa_decode_split_override().
+std::atomic<int> g_split_override{0};
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn g_encode = nullptr;
 
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+std::atomic<CtxGetCurrentFn> g_ctx_current{nullptr};
+std::atomic<CtxGetIdFn> g_ctx_id{nullptr};
+
+template <typename Fn>
+Fn driver_entry(const char* name) {
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPointByVersion(name, &fn, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<Fn>(fn);
+}
+
 bsa_status_t device_state(uint32_t** status, int* num_sms) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BSA_ERR_CUDA;
+  const uint64_t ctx = current_context_id();
   std::lock_guard<std::mutex> lock(g_mu);
-  if (g_status_ptr[dev] == nullptr) {
+  if (g_status_ptr[dev] == nullptr || ctx == 0 || g_status_ctx[dev] != ctx) {
+    // first use on this device, or a new context since (a device reset
+    // reloads the module, so the status word has a new address); the
+    // runtime calls below make the device's primary context current
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return BSA_ERR_CUDA;
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return BSA_ERR_CUDA;
     g_status_ptr[dev] = static_cast<uint32_t*>(p);
+    g_status_ctx[dev] = current_context_id();
     g_num_sms[dev] = sms;
   }
   if (g_encode == nullptr) {
@@ -97,10 +122,8 @@ DecodePlan decode_plan(int rows, int list_len, int num_sms) {
   P.list_len = list_len;
   const int64_t total = static_cast<int64_t>(rows) * list_len;
   int64_t c = num_sms;
-  if (const char* env = getenv("BSA_DECODE_SPLITS")) {
-    const int v = atoi(env);
-    if (v > 0) c = v;
-  }
+  const int forced = g_split_override.load(std::memory_order_relaxed);
+  if (forced > 0) c = forced;
   const int64_t need = (total + 127) / 128;   // ceil(total / c) <= 128
   if (c < need) c = need;
   if (c > total) c = total > 0 ? total : 1;
@@ -137,7 +160,38 @@ GistLayout gist_layout(const bsa_shape_t* s, int topk, int num_sms) {
   return L;
 }
 
+// Self-test of the bounded-wait expiry path: one thread waits, with a small
+// budget, on a shared-memory barrier that nothing arrives on.  The wait gives
+// up, raises BSA_DEV_TIMEOUT in the status word and the kernel returns.
+__global__ void wait_expiry_selftest_kernel(long long budget, uint32_t* status) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  abort_flag = 0;
+  const uint32_t b = smem_u32(&bar);
+  mbar_init(b, 1);
+  fence_barrier_init();
+  mbar_wait(b, 0, &abort_flag, status, budget);   // phase 0 never completes
+}
+
 }  // namespace
+
+uint64_t current_context_id() {
+  CtxGetCurrentFn cur = g_ctx_current.load(std::memory_order_acquire);
+  CtxGetIdFn id = g_ctx_id.load(std::memory_order_acquire);
+  if (cur == nullptr || id == nullptr) {
+    cur = driver_entry<CtxGetCurrentFn>("cuCtxGetCurrent");
+    id = driver_entry<CtxGetIdFn>("cuCtxGetId");
+    if (cur == nullptr || id == nullptr) return 0;
+    g_ctx_current.store(cur, std::memory_order_release);
+    g_ctx_id.store(id, std::memory_order_release);
+  }
+  CUcontext ctx = nullptr;
+  unsigned long long v = 0;
+  if (cur(&ctx) != CUDA_SUCCESS || ctx == nullptr || id(ctx, &v) != CUDA_SUCCESS) return 0;
+  return static_cast<uint64_t>(v);
+}
+
 }  // namespace bsa
 
 using namespace bsa;
@@ -156,6 +210,19 @@ const char* bsa_status_string(bsa_status_t st) {
     case BSA_ERR_DEVICE: return "BSA_ERR_DEVICE";
   }
   return "BSA_ERR_UNKNOWN";
+}
+
+int bsa_decode_split_override(int num_splits) {
+  return g_split_override.exchange(num_splits > 0 ? num_splits : 0);
+}
+
+bsa_status_t bsa_selftest_wait_expiry(long long budget_cycles, void* stream) {
+  if (budget_cycles < 0) return BSA_ERR_INVALID_ARG;
+  uint32_t* status = nullptr;
+  bsa_status_t st = device_state(&status, nullptr);
+  if (st != BSA_OK) return st;
+  wait_expiry_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(budget_cycles, status);
+  return cuda_status(cudaGetLastError());
 }
 
 bsa_status_t bsa_device_status(unsigned int* flags, int reset) {

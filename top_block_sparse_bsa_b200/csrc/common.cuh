@@ -21,7 +21,8 @@ enum : uint32_t {
   BSA_DEV_BAD_SHAPE = 1u << 2,   // a kernel saw a shape it cannot handle
 };
 
-// ~2^31 SM cycles (about one second) before a wait gives up.
+// Default budget of a bounded wait: ~2^31 SM cycles (about one second at
+// the maximum SM clock) before it gives up.
 constexpr long long kWaitBudgetCycles = 1ll << 31;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -68,17 +69,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase with the given parity to complete.  Returns
-// false (and raises the CTA's abort flag and the device status) on expiry,
-// or as soon as another thread of the CTA has raised the abort flag.
+// false (and raises the CTA's abort flag and the device status) once
+// `budget` SM cycles have passed, or as soon as another thread of the CTA has
+// raised the abort flag.  The kernels use the default budget; a self-test
+// kernel passes a small one to drive the expiry path.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          uint32_t* status) {
+                                          uint32_t* status, long long budget = kWaitBudgetCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63) == 63) {
       if (*abort_flag) return false;
-      if (clock64() - t0 > kWaitBudgetCycles) {
+      if (clock64() - t0 > budget) {
         *abort_flag = 1;
         atomicOr(status, BSA_DEV_TIMEOUT);
         return false;

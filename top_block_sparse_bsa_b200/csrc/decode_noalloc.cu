@@ -20,6 +20,7 @@
 
 #include "../../include/bsa.h"
 #include "common.cuh"
+#include "kernels.h"
 
 namespace bsa {
 namespace {
@@ -31,18 +32,23 @@ static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchB
 
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[kMaxDevices] = {};
+uint64_t g_noalloc_ctx[kMaxDevices] = {};
 
 // Device address of the array on the current device.  In host code the
 // array's name only stands in for the symbol; the address a kernel can use
-// must be asked for once per device, with that device current.
+// must be asked for once per device, with that device current.  The address
+// is looked up again when the device's context has changed (a device reset
+// reloads the library's module, and the array with it).
 bsa_status_t scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BSA_ERR_CUDA;
+  const uint64_t ctx = current_context_id();
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
+  if (g_noalloc_ptr[dev] == nullptr || ctx == 0 || g_noalloc_ctx[dev] != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return BSA_ERR_CUDA;
     g_noalloc_ptr[dev] = p;
+    g_noalloc_ctx[dev] = current_context_id();
   }
   *out = g_noalloc_ptr[dev];
   return BSA_OK;

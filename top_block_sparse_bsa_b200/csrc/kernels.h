@@ -9,22 +9,37 @@
 
 namespace bsa {
 
+// Identifier of the CUDA context current on the calling thread (unique for
+// the life of the process: a context created after a device reset gets a new
+// one); 0 if it cannot be read.  Per-device caches of device addresses and
+// function attributes are keyed on it, because a device reset unloads the
+// module they belong to.
+uint64_t current_context_id();
+
 // Opt kernel Fn into `bytes` of dynamic shared memory on the current device.
-// The attribute belongs to the (function, device) pair and persists, so the
-// driver call is made only when a device sees a larger request than before;
-// launches after the first cost no extra driver call.
+// The attribute belongs to the function in the current context and persists,
+// so the driver call is made only when a context sees a larger request than
+// before; launches after the first cost no extra driver call.
 template <auto Fn>
 inline cudaError_t ensure_dynamic_smem(size_t bytes) {
+  static std::atomic<uint64_t> granted_ctx[32];
   static std::atomic<uint32_t> granted[32];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 32) return cudaErrorInvalidDevice;
-  if (granted[dev].load(std::memory_order_acquire) >= bytes) return cudaSuccess;
+  const uint64_t ctx = current_context_id();
+  if (ctx != 0 && granted_ctx[dev].load(std::memory_order_acquire) == ctx &&
+      granted[dev].load(std::memory_order_acquire) >= bytes)
+    return cudaSuccess;
   e = cudaFuncSetAttribute(Fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
   if (e != cudaSuccess) return e;
-  uint32_t cur = granted[dev].load(std::memory_order_relaxed);
-  while (cur < bytes && !granted[dev].compare_exchange_weak(cur, static_cast<uint32_t>(bytes))) {
+  if (granted_ctx[dev].exchange(ctx, std::memory_order_acq_rel) != ctx) {
+    granted[dev].store(static_cast<uint32_t>(bytes), std::memory_order_release);
+  } else {
+    uint32_t cur = granted[dev].load(std::memory_order_relaxed);
+    while (cur < bytes && !granted[dev].compare_exchange_weak(cur, static_cast<uint32_t>(bytes))) {
+    }
   }
   return cudaSuccess;
 }
