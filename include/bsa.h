@@ -35,8 +35,8 @@
  *              kernel records a flag in the device status word, skips the bad
  *              work and returns; read it with bsa_device_status().
  *   Threads    calls are thread-safe; the only global state is the tensor-map
- *              entry point, the device status word and the decode split
- *              override of the testing hooks below.
+ *              entry point, the device status word and the overrides of
+ *              the testing hooks below.
  */
 #ifndef BSA_H_
 #define BSA_H_
@@ -255,6 +255,16 @@ int bsa_version(void);
  * result of a decode does not depend on it beyond fp32 rounding order.
  */
 int bsa_decode_split_override(int num_splits);
+
+/*
+ * bsa_prefill_kernel_override -- selects which bf16 prefill kernel the
+ * prefill and gated calls run: 0 = chosen by shape (default), 1 = paired
+ * tiles (two 128-row tiles per SM), 2 = one 128-row tile per SM with split
+ * key halves, 3 = SM pair (two SMs per 256 rows, MMAs of M = 256).
+ * Process-wide; returns the previous setting.  All kernels compute the same
+ * result up to fp32 rounding order; the hook exists to test and time each.
+ */
+int bsa_prefill_kernel_override(int kernel);
 
 /*
  * bsa_selftest_wait_expiry -- enqueues a one-thread kernel that waits, with

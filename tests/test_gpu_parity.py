@@ -125,6 +125,33 @@ def test_prefill_bf16_block128_ungated():
     _prefill_case(w, gated=False)
 
 
+@pytest.mark.parametrize("kernel", [1, 2, 3])
+@pytest.mark.parametrize("hq,bs,gated", [(4, 64, False), (5, 64, True), (7, 128, True), (3, 64, False)])
+def test_prefill_every_kernel_matches_the_oracle(kernel, hq, bs, gated):
+    """Each bf16 prefill kernel, forced through the testing hook (1 paired
+    tiles, 2 one tile per SM, 3 SM pair with MMAs of M = 256), on even and
+    odd tile counts per unit, ungated and gated, with odd and even kept lists."""
+    bsa = _bsa()
+    w = W.get("prefill_gqa_bf16").scaled(B=1, Hq=hq, Hkv=1, N=4096, bs=bs, kb=5)
+    prev = bsa.bsa_prefill_kernel_override(kernel)
+    try:
+        _prefill_case(w, gated=gated)
+    finally:
+        bsa.bsa_prefill_kernel_override(prev)
+
+
+def test_sm_pair_prefill_full_budget_and_empty_lists():
+    """The SM-pair kernel on the longest lists (dense causal at full budget)
+    and with emptied lists between items."""
+    bsa = _bsa()
+    prev = bsa.bsa_prefill_kernel_override(3)
+    try:
+        _prefill_case(W.get("prefill_gqa_bf16").scaled(B=1, Hq=4, Hkv=1, N=8192, kb=127), gated=True)
+        _prefill_case(W.get("gated_prefill_bf16").scaled(B=2, Hq=14, Hkv=2, N=4096, kb=8), gated=True)
+    finally:
+        bsa.bsa_prefill_kernel_override(prev)
+
+
 def _sample_rows(w: W.Workload, n: int, seed: int):
     r = np.random.default_rng(seed)
     b = r.integers(0, w.B, n)

@@ -25,7 +25,7 @@ __all__ = [
     "bsa_gated_attn_fwd", "bsa_sparse_attn_decode", "bsa_gist_expand_decode",
     "bsa_workspace_bytes", "bsa_status_string", "bsa_device_status", "bsa_version",
     "bsa_sparse_attn_decode_noalloc", "bsa_decode_split_override", "bsa_selftest_wait_expiry",
-    "EXPORTED_SYMBOLS",
+    "bsa_prefill_kernel_override", "EXPORTED_SYMBOLS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libbsa.so")
@@ -41,7 +41,7 @@ EXPORTED_SYMBOLS = (
     "bsa_score_blocks", "bsa_topk_select", "bsa_sparse_attn_prefill", "bsa_gated_attn_fwd",
     "bsa_sparse_attn_decode", "bsa_gist_expand_decode", "bsa_workspace_bytes",
     "bsa_status_string", "bsa_device_status", "bsa_version", "bsa_sparse_attn_decode_noalloc",
-    "bsa_decode_split_override", "bsa_selftest_wait_expiry",
+    "bsa_decode_split_override", "bsa_selftest_wait_expiry", "bsa_prefill_kernel_override",
 )
 
 
@@ -78,6 +78,7 @@ _SIGS = {
     "bsa_device_status": (_i, [ctypes.POINTER(ctypes.c_uint), _i]),
     "bsa_version": (_i, []),
     "bsa_decode_split_override": (_i, [_i]),
+    "bsa_prefill_kernel_override": (_i, [_i]),
     "bsa_selftest_wait_expiry": (_i, [ctypes.c_longlong, _p]),
 }
 
@@ -156,6 +157,12 @@ def bsa_device_status(reset: bool = False):
 def bsa_decode_split_override(num_splits: int) -> int:
     """Fix the decode split-K range count (> 0) or restore the default (<= 0); returns the previous setting."""
     return int(lib.bsa_decode_split_override(int(num_splits)))
+
+
+def bsa_prefill_kernel_override(kernel: int) -> int:
+    """Force a bf16 prefill kernel (1 paired tiles, 2 one tile per SM, 3 SM pair) or 0 for the
+    shape's default; returns the previous setting."""
+    return int(lib.bsa_prefill_kernel_override(int(kernel)))
 
 
 def bsa_selftest_wait_expiry(budget_cycles: int, stream=None) -> None:

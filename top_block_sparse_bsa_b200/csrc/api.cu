@@ -26,6 +26,9 @@ int g_num_sms[kMaxDevices] = {};
 // Split-count override of the decode plan (0: one split range per SM); set
 // only through bsa_decode_split_override().
 std::atomic<int> g_split_override{0};
+// Prefill kernel override (0: chosen by shape); set only through
+// bsa_prefill_kernel_override().
+std::atomic<int> g_prefill_kernel{0};
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -212,6 +215,10 @@ const char* bsa_status_string(bsa_status_t st) {
   return "BSA_ERR_UNKNOWN";
 }
 
+int bsa_prefill_kernel_override(int kernel) {
+  return g_prefill_kernel.exchange(kernel >= 1 && kernel <= 3 ? kernel : 0);
+}
+
 int bsa_decode_split_override(int num_splits) {
   return g_split_override.exchange(num_splits > 0 ? num_splits : 0);
 }
@@ -350,6 +357,7 @@ static bsa_status_t prefill_common(const bsa_shape_t* s, const void* q, const vo
   a.o = o;
   a.lse = lse;
   a.status = status;
+  a.kernel = g_prefill_kernel.load(std::memory_order_relaxed);
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   if (s->dtype == BSA_BF16) {
     if (s->d != 128) return BSA_ERR_UNSUPPORTED;

@@ -674,8 +674,10 @@ cudaError_t launch_attn_prefill_bf16(const CUtensorMap* tmQ, const CUtensorMap* 
   p.G = a.Hq / a.Hkv;
   p.rows_per_unit = p.G * a.bs;
   p.tiles_per_unit = (p.rows_per_unit + 127) / 128;
+  if (a.kernel == 3) return launch_attn_prefill_pair_bf16(tmQ, tmK, tmV, a, st);
   // an odd tile count would leave one tile per unit without a partner
-  if (p.tiles_per_unit % 2 == 1) return launch_attn_prefill_split_bf16(tmQ, tmK, tmV, a, st);
+  if (a.kernel == 2 || (a.kernel == 0 && p.tiles_per_unit % 2 == 1))
+    return launch_attn_prefill_split_bf16(tmQ, tmK, tmV, a, st);
   p.ctas_per_unit = (p.tiles_per_unit + 1) / 2;
   const int64_t items = static_cast<int64_t>(a.B) * a.Hkv * p.nb * p.ctas_per_unit;
   if (items <= 0) return cudaSuccess;

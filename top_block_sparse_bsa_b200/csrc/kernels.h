@@ -89,12 +89,17 @@ struct PrefillArgs {
   float* lse;
   uint32_t* status;
   int num_sms;
+  int kernel;                // 0: chosen by shape; 1 paired tiles; 2 one tile per item; 3 SM pair
 };
 cudaError_t launch_attn_prefill_bf16(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
                                      const PrefillArgs& a, cudaStream_t st);
 // attn_prefill_split.cu (one tile per item; called for odd tile counts per unit)
 cudaError_t launch_attn_prefill_split_bf16(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
                                            const PrefillArgs& a, cudaStream_t st);
+
+// attn_prefill_pair.cu (two SMs per item, MMAs of M = 256)
+cudaError_t launch_attn_prefill_pair_bf16(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
+                                          const PrefillArgs& a, cudaStream_t st);
 
 // attn_f32.cu (fp32 SIMT path)
 cudaError_t launch_attn_prefill_f32(const float* q, const float* k, const float* v, const PrefillArgs& a,
