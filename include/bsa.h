@@ -124,6 +124,26 @@ bsa_status_t bsa_topk_select(const float* scores, int rows, int ncols, int mode,
                              int* idx_out, int idx_stride, int* count_out, void* stream);
 
 /*
+ * bsa_decode_select -- the decode selector in one call: the group query
+ * mean, its scores against the pooled-key summary kept next to the cache,
+ * and the top-kb history blocks with the last block kept.
+ * Cite: 稀疏注意力 tutorial §4.6 (coarse block scoring) and §5 (decode: one
+ * new query against the history); SAS page, 推理 paragraph (the k best units
+ * kept) and 核心模块 3 (the current block always kept).
+ * Results equal bsa_score_blocks(BSA_SCORE_DECODE, pooled_k_in = pooled_k)
+ * followed by bsa_topk_select(BSA_TOPK_LAST_BLOCK) bit for bit; with d = 128
+ * and at most 2048 blocks they come from one kernel that keeps the scores
+ * on chip between the two steps.
+ * q [B,Hq,d] (dtype); pooled_k [B,Hkv,nb,d] fp32 with nb = Nk/block; Nq = 1.
+ * scores [B,Hkv,nb] fp32 (required, written); idx_out [B,Hkv,idx_stride]
+ * int32, idx_stride >= kb + 1; count_out [B,Hkv] int32 and pooled_q_out
+ * [B,Hkv,d] fp32 are optional.  Limits: nb <= 8192.
+ */
+bsa_status_t bsa_decode_select(const bsa_shape_t* shape, const void* q, const float* pooled_k, int kb,
+                               float* pooled_q_out, float* scores, int* idx_out, int idx_stride,
+                               int* count_out, void* stream);
+
+/*
  * bsa_sparse_attn_prefill -- block-sparse causal attention (prefill).
  * Cite: 稀疏注意力 tutorial §1 (softmax(QK^T/sqrt(d))V), §2 (additive mask
  * M in {0,-inf}; skip the masked region instead of computing it), §4.5

@@ -359,6 +359,48 @@ def _decode_case(w: W.Workload, groups=None):
                       dict(max_abs=2e-3, mean_abs=2e-4), "decode lse")
 
 
+@pytest.mark.parametrize("nb,kb,d,dtype", [(128, 12, 128, "bf16"), (200, 17, 128, "bf16"), (2048, 96, 128, "bf16"),
+                                          (1, 3, 128, "bf16"), (129, 0, 128, "bf16"), (300, 400, 128, "bf16"),
+                                          (256, 20, 128, "f32"), (96, 7, 64, "bf16"), (2500, 30, 128, "bf16")])
+def test_decode_select_one_call_equals_score_then_topk(nb, kb, d, dtype):
+    """bsa_decode_select (one kernel for d 128 and up to 2048 blocks, the two
+    kernels otherwise) gives the bits of bsa_score_blocks(DECODE) followed by
+    bsa_topk_select(LAST_BLOCK), and the oracle's scores and kept blocks:
+    ragged last chunks (200, 129, 300 blocks), one block, budget 0 and a
+    budget above the candidates, fp32 queries, d 64 and 2500 blocks (the two
+    kernel path)."""
+    bsa = _bsa()
+    B, Hq, Hkv, bs = 2, 8, 2, 64
+    g = torch.Generator(device="cuda").manual_seed(nb * 7 + kb)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    q = torch.randn((B, Hq, d), generator=g, device="cuda").to(tdt)
+    kbar = torch.randn((B, Hkv, nb, d), generator=g, device="cuda")
+    shape = bsa.make_shape(B, Hq, Hkv, 1, nb * bs, d, bs, tdt)
+    stride = kb + 3
+    outs = []
+    for fused in (True, False):
+        sc = torch.full((B, Hkv, nb), float("nan"), device="cuda")
+        qb = torch.full((B, Hkv, d), float("nan"), device="cuda")
+        idx = torch.full((B, Hkv, stride), -7, dtype=torch.int32, device="cuda")
+        cnt = torch.full((B, Hkv), -7, dtype=torch.int32, device="cuda")
+        if fused:
+            bsa.bsa_decode_select(shape, q, kbar, kb, sc, idx, stride, pooled_q_out=qb, count_out=cnt)
+        else:
+            bsa.bsa_score_blocks(shape, bsa.BSA_SCORE_DECODE, q, None, kbar, qb, None, sc)
+            bsa.bsa_topk_select(sc, B * Hkv, nb, bsa.BSA_TOPK_LAST_BLOCK, kb, idx, stride, cnt)
+        torch.cuda.synchronize()
+        outs.append((sc.cpu().numpy(), qb.cpu().numpy(), idx.cpu().numpy(), cnt.cpu().numpy()))
+    for a, b in zip(outs[0], outs[1]):
+        assert np.array_equal(a, b)
+    qbar, s, want_idx, want_cnt = oracle.decode_select(q.float().cpu(), kbar.cpu(), Hkv, kb)
+    assert np.array_equal(outs[0][0], s)
+    assert np.array_equal(outs[0][1], qbar)
+    assert np.array_equal(outs[0][2][..., :want_idx.shape[-1]], want_idx)
+    assert np.all(outs[0][2][..., want_idx.shape[-1]:] == -1)
+    assert np.array_equal(outs[0][3], want_cnt)
+    _status_clean()
+
+
 def test_decode_bf16_small():
     w = W.get("decode_bf16").scaled(B=2, Hq=8, Hkv=2, N=8192, kb=12)
     _decode_case(w)

@@ -25,7 +25,7 @@ __all__ = [
     "bsa_gated_attn_fwd", "bsa_sparse_attn_decode", "bsa_gist_expand_decode",
     "bsa_workspace_bytes", "bsa_status_string", "bsa_device_status", "bsa_version",
     "bsa_sparse_attn_decode_noalloc", "bsa_decode_split_override", "bsa_selftest_wait_expiry",
-    "bsa_prefill_kernel_override", "EXPORTED_SYMBOLS",
+    "bsa_prefill_kernel_override", "bsa_decode_select", "EXPORTED_SYMBOLS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libbsa.so")
@@ -42,6 +42,7 @@ EXPORTED_SYMBOLS = (
     "bsa_sparse_attn_decode", "bsa_gist_expand_decode", "bsa_workspace_bytes",
     "bsa_status_string", "bsa_device_status", "bsa_version", "bsa_sparse_attn_decode_noalloc",
     "bsa_decode_split_override", "bsa_selftest_wait_expiry", "bsa_prefill_kernel_override",
+    "bsa_decode_select",
 )
 
 
@@ -65,6 +66,7 @@ _i = ctypes.c_int
 _SIGS = {
     "bsa_score_blocks": (_i, [ctypes.POINTER(BsaShape), _i, _p, _p, _p, _p, _p, _p, _p]),
     "bsa_topk_select": (_i, [_p, _i, _i, _i, _i, _p, _i, _p, _p]),
+    "bsa_decode_select": (_i, [ctypes.POINTER(BsaShape), _p, _p, _i, _p, _p, _p, _i, _p, _p]),
     "bsa_sparse_attn_prefill": (_i, [ctypes.POINTER(BsaShape), _p, _p, _p, _p, _i, ctypes.c_float, _p, _p, _p]),
     "bsa_gated_attn_fwd": (_i, [ctypes.POINTER(BsaShape), _p, _p, _p, _p, _i, _p, ctypes.c_float, _p, _p, _p]),
     "bsa_sparse_attn_decode": (_i, [ctypes.POINTER(BsaShape), _p, _p, _p, _p, _i, ctypes.c_float, _p,
@@ -186,6 +188,13 @@ def bsa_topk_select(scores, rows: int, ncols: int, mode: int, kb: int, idx_out, 
     _check("bsa_topk_select", lib.bsa_topk_select(
         _ptr(scores), int(rows), int(ncols), int(mode), int(kb), _ptr(idx_out), int(idx_stride),
         _ptr(count_out), _stream(stream)))
+
+
+def bsa_decode_select(shape: BsaShape, q, pooled_k, kb: int, scores, idx_out, idx_stride: int,
+                      pooled_q_out=None, count_out=None, stream=None) -> None:
+    _check("bsa_decode_select", lib.bsa_decode_select(
+        ctypes.byref(shape), _ptr(q), _ptr(pooled_k), int(kb), _ptr(pooled_q_out), _ptr(scores), _ptr(idx_out),
+        int(idx_stride), _ptr(count_out), _stream(stream)))
 
 
 def bsa_sparse_attn_prefill(shape: BsaShape, q, k, v, idx, idx_stride: int, softmax_scale: float, o,

@@ -93,6 +93,18 @@ bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D fp32 view [rows, 128] with a box of 32 columns (128 bytes) x 128 rows
+// and the 128-byte swizzle (the decode selector's pooled-key chunks).
+bool make_map_f32_rows128(CUtensorMap* m, const void* base, uint64_t rows) {
+  const cuuint64_t dims[2] = {128, rows};
+  const cuuint64_t strides[1] = {128 * 4};
+  const cuuint32_t box[2] = {32, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bsa_status_t check_shape(const bsa_shape_t* s) {
@@ -329,6 +341,36 @@ bsa_status_t bsa_topk_select(const float* scores, int rows, int ncols, int mode,
                                  static_cast<cudaStream_t>(stream)));
 }
 
+bsa_status_t bsa_decode_select(const bsa_shape_t* s, const void* q, const float* pooled_k, int kb,
+                               float* pooled_q_out, float* scores, int* idx_out, int idx_stride, int* count_out,
+                               void* stream) {
+  bsa_status_t st = check_shape(s);
+  if (st != BSA_OK) return st;
+  if (s->Nq != 1 || !q || !pooled_k || !scores || !idx_out || kb < 0) return BSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(pooled_k) || !aligned16(scores)) return BSA_ERR_INVALID_ARG;
+  if (idx_stride < kb + 1) return BSA_ERR_INVALID_ARG;
+  if (s->d % 8 != 0 || s->d > 1024) return BSA_ERR_UNSUPPORTED;
+  const int nb = s->Nk / s->block;
+  if (nb > 8192) return BSA_ERR_UNSUPPORTED;
+  uint32_t* status = nullptr;
+  if ((st = device_state(&status, nullptr)) != BSA_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const bool bf16 = s->dtype == BSA_BF16;
+  const float scale = score_scale(s->d);
+  if (decode_select_fused_ok(s->d, nb)) {
+    CUtensorMap mk;
+    if (!make_map_f32_rows128(&mk, pooled_k, static_cast<uint64_t>(s->B) * s->Hkv * nb)) return BSA_ERR_CUDA;
+    return cuda_status(launch_decode_select(&mk, q, bf16, s->B, s->Hq, s->Hkv, nb, scale, kb, scores, pooled_q_out,
+                                            idx_out, idx_stride, count_out, status, cs));
+  }
+  // other head dimensions or longer rows: the scoring and selection kernels
+  cudaError_t e =
+      launch_score_decode(q, bf16, pooled_k, s->B, s->Hq, s->Hkv, nb, s->d, scale, scores, pooled_q_out, cs);
+  if (e == cudaSuccess)
+    e = launch_topk(scores, s->B * s->Hkv, nb, BSA_TOPK_LAST_BLOCK, kb, idx_out, idx_stride, count_out, cs);
+  return cuda_status(e);
+}
+
 static bsa_status_t prefill_common(const bsa_shape_t* s, const void* q, const void* k, const void* v,
                                    const int* idx, int idx_stride, const float* sel, float scale, void* o,
                                    float* lse, void* stream) {
@@ -462,6 +504,16 @@ bsa_status_t bsa_gist_expand_decode(const bsa_shape_t* s, const void* q, const v
   const int* idx = idx_in;
   const int idx_stride = topk > 0 ? topk : 1;
   cudaError_t e = cudaSuccess;
+  uint32_t* expanded = reinterpret_cast<uint32_t*>(ws + L.expanded);
+  int* ulist = reinterpret_cast<int*>(ws + L.union_list);
+  // every tensor map first, so that nothing is enqueued when one fails
+  CUtensorMap mq, mk, mv, mgk, mgv;
+  if (!make_map_bf16(&mq, q, static_cast<uint64_t>(rows), static_cast<uint32_t>(G)) ||
+      !make_map_bf16(&mk, k_cache, static_cast<uint64_t>(s->B) * s->Hkv * s->Nk, 64) ||
+      !make_map_bf16(&mv, v_cache, static_cast<uint64_t>(s->B) * s->Hkv * s->Nk, 64) ||
+      !make_map_bf16(&mgk, gist_k, static_cast<uint64_t>(s->B) * s->Hkv * nc, 64) ||
+      !make_map_bf16(&mgv, gist_v, static_cast<uint64_t>(s->B) * s->Hkv * nc, 64))
+    return BSA_ERR_CUDA;
   if (idx == nullptr) {
     int* idx_dst = (idx_out && topk > 0) ? idx_out : reinterpret_cast<int*>(ws + L.idx);
     if (topk > 0) {
@@ -475,17 +527,8 @@ bsa_status_t bsa_gist_expand_decode(const bsa_shape_t* s, const void* q, const v
   } else if (idx_out != nullptr && topk > 0 && idx_out != idx_in) {
     e = cudaMemcpyAsync(idx_out, idx_in, static_cast<size_t>(rows) * topk * sizeof(int), cudaMemcpyDeviceToDevice, cs);
   }
-  uint32_t* expanded = reinterpret_cast<uint32_t*>(ws + L.expanded);
-  int* ulist = reinterpret_cast<int*>(ws + L.union_list);
   if (e == cudaSuccess)
     e = launch_gist_union(idx, s->B, s->Hq, s->Hkv, topk, idx_stride, nc, expanded, ulist, L.union_stride, status, cs);
-  CUtensorMap mq, mk, mv, mgk, mgv;
-  if (!make_map_bf16(&mq, q, static_cast<uint64_t>(rows), static_cast<uint32_t>(G)) ||
-      !make_map_bf16(&mk, k_cache, static_cast<uint64_t>(s->B) * s->Hkv * s->Nk, 64) ||
-      !make_map_bf16(&mv, v_cache, static_cast<uint64_t>(s->B) * s->Hkv * s->Nk, 64) ||
-      !make_map_bf16(&mgk, gist_k, static_cast<uint64_t>(s->B) * s->Hkv * nc, 64) ||
-      !make_map_bf16(&mgv, gist_v, static_cast<uint64_t>(s->B) * s->Hkv * nc, 64))
-    return BSA_ERR_CUDA;
   DecodeArgs a;
   a.B = s->B;
   a.Hq = s->Hq;

@@ -77,6 +77,11 @@ cudaError_t launch_score_gist(const void* q, const void* gk, bool bf16, int B, i
                               int d, float scale, float* s, cudaStream_t st);
 cudaError_t launch_topk(const float* scores, int rows, int ncols, int mode, int kb, int* idx_out,
                         int idx_stride, int* count_out, cudaStream_t st);
+// decode scores + top-k in one kernel (tmKbar: fp32 [rows, 128], box 32 x 128, 128-byte swizzle)
+bool decode_select_fused_ok(int d, int nb);
+cudaError_t launch_decode_select(const CUtensorMap* tmKbar, const void* q, bool bf16, int B, int Hq, int Hkv,
+                                 int nb, float scale, int kb, float* scores, float* qbar_out, int* idx_out,
+                                 int idx_stride, int* count_out, uint32_t* status, cudaStream_t st);
 
 // attn_prefill.cu (bf16, d = 128, tcgen05)
 struct PrefillArgs {

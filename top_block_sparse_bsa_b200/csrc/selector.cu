@@ -17,6 +17,7 @@
 // so the sequential order costs nothing that matters.
 #include "common.cuh"
 #include "kernels.h"
+#include "topk.cuh"
 
 namespace bsa {
 
@@ -551,14 +552,6 @@ cudaError_t launch_score_gist(const void* q, const void* gk, bool bf16, int B, i
 }
 
 // ------------------------------------------------------------------ top-k
-// Monotone unsigned key of an fp32 score: a larger score gives a larger key,
-// -0 and +0 share one key, and every NaN gets key 0 (below -inf).
-__device__ __forceinline__ uint32_t order_key(float f) {
-  if (f != f) return 0u;
-  uint32_t u = __float_as_uint(f);
-  if (f == 0.0f) u = 0u;
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
 
 // One CTA per row.  Radix select (4 passes of 8 bits, most significant
 // first) finds the key T of the k-th best candidate and how many candidates
@@ -784,10 +777,7 @@ __global__ void __launch_bounds__(256) topk_cta_kernel(const float* __restrict__
                                                        int* __restrict__ idx_out, int idx_stride,
                                                        int* __restrict__ count_out) {
   griddep_wait();   // the scores come from the kernel launched before
-  __shared__ int hist[256];
-  __shared__ uint32_t wsum[8];
-  __shared__ int sel_digit, sel_above;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   const int64_t r = blockIdx.x;
   int ncand, forced;
   if (mode == 0) {
@@ -805,110 +795,146 @@ __global__ void __launch_bounds__(256) topk_cta_kernel(const float* __restrict__
   uint32_t key[KPT];
 #pragma unroll
   for (int e = 0; e < KPT; ++e) key[e] = (j0 + e < ncand) ? order_key(__ldg(srow + j0 + e)) : 0u;
-  const int take = min(kb, ncand);
-  const bool take_all = (take == ncand);
-  uint32_t thresh = 0u;
-  int remaining = take;   // ties (== thresh) to keep
-  if (!take_all && take > 0) {
-    uint32_t prefix = 0u, pmask = 0u;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      hist[tid] = 0;
-      __syncthreads();
-#pragma unroll
-      for (int e = 0; e < KPT; ++e)
-        if (j0 + e < ncand && (key[e] & pmask) == prefix) atomicAdd(&hist[(key[e] >> shift) & 255u], 1);
-      __syncthreads();
-      if (warp == 0) {
-        // lane l owns bins 255-8l .. 248-8l (descending); suffix counts
-        int c[8];
-        int run = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          run += hist[255 - 8 * lane - i];
-          c[i] = run;
-        }
-        int incl = run;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int v = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += v;
-        }
-        const int excl = incl - run;   // keys in higher bins than this lane's
-        // the digit is the first bin (from the top) whose suffix count reaches remaining
-        int found = -1, above = 0;
-#pragma unroll
-        for (int i = 7; i >= 0; --i) {
-          const int ge = excl + c[i];
-          const int gt = excl + (i ? c[i - 1] : 0);
-          if (ge >= remaining && gt < remaining) {
-            found = 255 - 8 * lane - i;
-            above = gt;
-          }
-        }
-        const unsigned who = __ballot_sync(0xffffffffu, found >= 0);
-        const int src = __ffs(who) - 1;
-        const int d = __shfl_sync(0xffffffffu, found, src);
-        const int ab = __shfl_sync(0xffffffffu, above, src);
-        if (lane == 0) {
-          sel_digit = d;
-          sel_above = ab;
-        }
-      }
-      __syncthreads();
-      prefix |= static_cast<uint32_t>(sel_digit) << shift;
-      pmask |= 255u << shift;
-      remaining -= sel_above;
-      __syncthreads();   // hist and sel_* are rewritten by the next pass
-    }
-    thresh = prefix;
+  cta_topk_select<KPT>(key, ncand, kb, forced, idx_out + r * idx_stride, idx_stride,
+                       count_out ? count_out + r : nullptr);
+}
+
+// ------------------------------------------------------- decode selector
+// The decode selector in one kernel (d = 128, at most 2048 blocks): one CTA
+// per (batch, KV group) row forms the group query mean, streams the row's
+// pooled-key summary through shared memory and scores every block, then
+// keeps the top-kb history blocks and the last block -- the work of
+// score_decode_kernel followed by topk_cta_kernel<8>, with the scores held in
+// shared memory between the two (tutorial §5: decode reads the history for
+// one new query; SAS page, 推理: the k best units are kept, the last block
+// always).  Same arithmetic, same order, so the same bits.
+//
+// The summary rows arrive by TMA in chunks of 128 rows: four boxes of 32
+// channels (128 bytes) x 128 rows with the 128-byte swizzle, so the float4
+// reads of eight consecutive rows at one channel offset fall in distinct
+// banks.  Three chunks are in flight while threads 0..127 score the oldest
+// (thread = row, channels ascending).
+constexpr int kDsThreads = 256;
+constexpr int kDsRows = 128;
+constexpr int kDsStages = 3;
+constexpr uint32_t kDsBox = 128u * 128u;             // 128 rows x 128 bytes
+constexpr uint32_t kDsChunk = 4u * kDsBox;           // 128 rows x 128 floats
+constexpr int kDsMaxBlocks = 256 * 8;                // the CTA select holds 8 keys per thread
+constexpr uint32_t kDsScores = kDsStages * kDsChunk;                    // float[kDsMaxBlocks]
+constexpr uint32_t kDsQm = kDsScores + kDsMaxBlocks * 4;                // float[128]
+constexpr uint32_t kDsBar = kDsQm + 128 * 4;                            // kDsStages mbarriers
+constexpr uint32_t kDsSmem = kDsBar + kDsStages * 8 + 1024;             // + alignment slack
+
+template <typename T>
+__global__ void __launch_bounds__(kDsThreads, 1)
+    decode_select_kernel(const __grid_constant__ CUtensorMap tmKbar, const T* __restrict__ q, int Hq, int Hkv,
+                         int nb, float scale, int kb, float* __restrict__ scores, float* __restrict__ qbar_out,
+                         int* __restrict__ idx_out, int idx_stride, int* __restrict__ count_out,
+                         uint32_t* __restrict__ status) {
+  extern __shared__ uint8_t ds_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ds_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(sm);
+  float* sc = reinterpret_cast<float*>(sm + kDsScores);
+  float* qm = reinterpret_cast<float*>(sm + kDsQm);
+  __shared__ int abort_flag;
+  const int tid = threadIdx.x;
+  const int64_t bg = blockIdx.x;
+  const int64_t b = bg / Hkv, g = bg % Hkv;
+  const int G = Hq / Hkv;
+  const int nchunks = (nb + kDsRows - 1) / kDsRows;
+  auto bar = [&](int st) -> uint32_t { return sbase + kDsBar + 8u * st; };
+  auto issue = [&](int c) {
+    const int st = c % kDsStages;
+    mbar_arrive_expect_tx(bar(st), kDsChunk);
+    const int y = static_cast<int>(bg * nb) + c * kDsRows;   // rows past the tensor read the zero fill
+    for (int k = 0; k < 4; ++k) tma_load_2d(sbase + st * kDsChunk + k * kDsBox, &tmKbar, bar(st), 32 * k, y);
+  };
+  if (tid == 0) {
+    abort_flag = 0;
+    for (int st = 0; st < kDsStages; ++st) mbar_init(bar(st), 1);
+    fence_barrier_init();
+    prefetch_tmap(&tmKbar);
   }
-  // this thread's kept candidates: every key > thresh, ties counted separately
-  int ngt = 0, ntie = 0;
-#pragma unroll
-  for (int e = 0; e < KPT; ++e) {
-    const bool valid = j0 + e < ncand;
-    if (take_all) {
-      ngt += valid ? 1 : 0;
-    } else if (take > 0) {
-      ngt += (valid && key[e] > thresh) ? 1 : 0;
-      ntie += (valid && key[e] == thresh) ? 1 : 0;
-    }
-  }
-  // block exclusive scan of the packed (gt, tie) counts (each < 2^16)
-  const uint32_t mine = static_cast<uint32_t>(ngt) | (static_cast<uint32_t>(ntie) << 16);
-  uint32_t incl = mine;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  if (lane == 31) wsum[warp] = incl;
   __syncthreads();
-  uint32_t base = 0u, total = 0u;
+  griddep_wait();   // the query may come from the kernel launched before
+  int issued = 0;   // chunks whose copies thread 0 has started
+  if (tid == 0)
+    for (; issued < min(kDsStages, nchunks); ++issued) issue(issued);
+  if (tid < 128) {
+    // group query mean, heads ascending, one division (as score_decode_kernel)
+    float acc = 0.0f;
+    for (int hh = 0; hh < G; ++hh) acc = __fadd_rn(acc, static_cast<float>(q[(b * Hq + g * G + hh) * 128 + tid]));
+    const float m = __fdiv_rn(acc, static_cast<float>(G));
+    qm[tid] = m;
+    if (qbar_out) qbar_out[bg * 128 + tid] = m;
+  }
+  __syncthreads();
+  bool ok = true;
+  for (int c = 0; c < nchunks; ++c) {
+    const int st = c % kDsStages;
+    ok = mbar_wait(bar(st), (c / kDsStages) & 1, &abort_flag, status);
+    if (ok && tid < kDsRows) {
+      const int r = tid, row = c * kDsRows + r;
+      if (row < nb) {
+        const uint32_t rbase = sbase + st * kDsChunk + r * 128u;
+        float acc = 0.0f;
 #pragma unroll
-  for (int w = 0; w < 8; ++w) {
-    if (w < warp) base += wsum[w];
-    total += wsum[w];
+        for (int e = 0; e < 32; ++e) {
+          // channels 4e..4e+3: box e/8, 16-byte chunk (e%8) XOR (row%8)
+          const uint32_t a = rbase + (e >> 3) * kDsBox + ((((e & 7) ^ (r & 7)) & 7) << 4);
+          float4 v;
+          asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+                       : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                       : "r"(a));
+          acc = __fadd_rn(acc, __fmul_rn(qm[4 * e + 0], v.x));
+          acc = __fadd_rn(acc, __fmul_rn(qm[4 * e + 1], v.y));
+          acc = __fadd_rn(acc, __fmul_rn(qm[4 * e + 2], v.z));
+          acc = __fadd_rn(acc, __fmul_rn(qm[4 * e + 3], v.w));
+        }
+        const float sv = __fmul_rn(acc, scale);
+        sc[row] = sv;
+        scores[bg * nb + row] = sv;
+      }
+    }
+    // every thread has passed the wait of chunk c (or given up) before its
+    // stage is refilled
+    if (!__syncthreads_and(ok)) break;
+    if (tid == 0 && c + kDsStages < nchunks) issue(issued++);
   }
-  const uint32_t excl = base + incl - mine;
-  int gt_before = static_cast<int>(excl & 0xFFFFu), tie_before = static_cast<int>(excl >> 16);
-  int* out = idx_out + r * idx_stride;
+  if (abort_flag) {
+    // an expired wait was recorded in the status word; let the copies in
+    // flight land before the CTA exits
+    if (tid == 0)
+      for (int c = max(0, issued - kDsStages); c < issued; ++c) mbar_drain(bar(c % kDsStages), (c / kDsStages) & 1);
+    return;
+  }
+  // top-k of blocks 0..nb-2, block nb-1 kept (the decode candidate rule)
+  const int ncand = nb - 1;
+  uint32_t key[8];
 #pragma unroll
-  for (int e = 0; e < KPT; ++e) {
-    const bool valid = j0 + e < ncand;
-    const bool gt = take_all ? valid : (take > 0 && valid && key[e] > thresh);
-    const bool tie = !take_all && take > 0 && valid && key[e] == thresh;
-    if (gt || (tie && tie_before < remaining)) out[gt_before + min(tie_before, remaining)] = j0 + e;
-    gt_before += gt ? 1 : 0;
-    tie_before += tie ? 1 : 0;
+  for (int e = 0; e < 8; ++e) key[e] = (tid * 8 + e < ncand) ? order_key(sc[tid * 8 + e]) : 0u;
+  cta_topk_select<8>(key, ncand, kb, nb - 1, idx_out + bg * idx_stride, idx_stride,
+                     count_out ? count_out + bg : nullptr);
+}
+
+bool decode_select_fused_ok(int d, int nb) { return d == 128 && nb >= 1 && nb <= kDsMaxBlocks; }
+
+cudaError_t launch_decode_select(const CUtensorMap* tmKbar, const void* q, bool bf16, int B, int Hq, int Hkv,
+                                 int nb, float scale, int kb, float* scores, float* qbar_out, int* idx_out,
+                                 int idx_stride, int* count_out, uint32_t* status, cudaStream_t st) {
+  const dim3 grid(B * Hkv);
+  if (bf16) {
+    cudaError_t e = ensure_dynamic_smem<decode_select_kernel<__nv_bfloat16>>(kDsSmem);
+    if (e != cudaSuccess) return e;
+    return launch_dependent(decode_select_kernel<__nv_bfloat16>, grid, dim3(kDsThreads), kDsSmem, st, *tmKbar,
+                            static_cast<const __nv_bfloat16*>(q), Hq, Hkv, nb, scale, kb, scores, qbar_out, idx_out,
+                            idx_stride, count_out, status);
   }
-  int n = static_cast<int>(total & 0xFFFFu) + min(static_cast<int>(total >> 16), remaining);
-  if (forced >= 0) {
-    if (tid == 0) out[n] = forced;
-    ++n;
-  }
-  for (int t = n + tid; t < idx_stride; t += 256) out[t] = -1;
-  if (count_out && tid == 0) count_out[r] = n;
+  cudaError_t e = ensure_dynamic_smem<decode_select_kernel<float>>(kDsSmem);
+  if (e != cudaSuccess) return e;
+  return launch_dependent(decode_select_kernel<float>, grid, dim3(kDsThreads), kDsSmem, st, *tmKbar,
+                          static_cast<const float*>(q), Hq, Hkv, nb, scale, kb, scores, qbar_out, idx_out, idx_stride,
+                          count_out, status);
 }
 
 cudaError_t launch_topk(const float* scores, int rows, int ncols, int mode, int kb, int* idx_out,

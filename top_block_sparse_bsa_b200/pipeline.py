@@ -15,7 +15,7 @@ from typing import Dict, Optional
 import torch
 
 from . import (BSA_OP_DECODE, BSA_OP_GIST_DECODE, BSA_SCORE_DECODE, BSA_SCORE_PREFILL,
-               BSA_TOPK_CAUSAL_BLOCK, BSA_TOPK_LAST_BLOCK, bsa_gated_attn_fwd, bsa_gist_expand_decode,
+               BSA_TOPK_CAUSAL_BLOCK, bsa_decode_select, bsa_gated_attn_fwd, bsa_gist_expand_decode,
                bsa_score_blocks, bsa_sparse_attn_decode, bsa_sparse_attn_prefill, bsa_topk_select,
                bsa_workspace_bytes, make_shape)
 
@@ -126,11 +126,8 @@ class DecodeStep:
 
     def select(self, stream=None):
         b = self.bufs
-        bsa_score_blocks(self.shape, BSA_SCORE_DECODE, self.q, None, b["kbar"], b["qbar"], None, b["scores"],
-                         stream=stream)
-        rows = self.shape.B * self.shape.Hkv
-        bsa_topk_select(b["scores"], rows, self.nb, BSA_TOPK_LAST_BLOCK, self.kb, b["idx"], self.idx_stride,
-                        b["count"], stream=stream)
+        bsa_decode_select(self.shape, self.q, b["kbar"], self.kb, b["scores"], b["idx"], self.idx_stride,
+                          pooled_q_out=b["qbar"], count_out=b["count"], stream=stream)
 
     def attend(self, idx: Optional[torch.Tensor] = None, stream=None, with_lse: bool = True):
         b = self.bufs
