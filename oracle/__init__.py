@@ -75,6 +75,11 @@ def _declare(L):
                                       ctypes.c_double, _p, _i64, _p, _p],
         "oracle_attend_gist_rows": [_p, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _i64, _i64, _p,
                                     _i64, ctypes.c_double, _p, _i64, _p, _p],
+        "oracle_topk_pattern": [_p, _i64, _i64, _i64, _i64, _i64, _p, _i64, _p],
+        "oracle_topk_joint_heads": [_p, _i64, _i64, _i64, _i64, _p, _i64, _p],
+        "oracle_attend_decode_heads_rows": [_p, _p, _p, _i64, _i64, _i64, _i64, _i64, _i64, _p, _i64,
+                                            ctypes.c_double, _p, _i64, _p, _p],
+        "oracle_paged_gather": [_p, _p, _i64, _i64, _i64, _i64, _i64, _i64, _p],
         "oracle_max_threads": [],
         "oracle_set_threads": [ctypes.c_int],
     }
@@ -303,3 +308,67 @@ def gist_select(q, gk, kb: int):
     s = scores_gist(q, gk)
     idx, cnt = topk(s, TOPK_PLAIN, kb)
     return s, idx, cnt
+
+
+# ----------------------------------------------------------------------------
+# 7-9. fixed pattern + dynamic blocks, shared head budget, paged cache
+# ----------------------------------------------------------------------------
+
+def topk_pattern(scores, sink: int, local: int, kb: int, idx_stride: Optional[int] = None
+                 ) -> Tuple[np.ndarray, np.ndarray]:
+    """scores [..., nb, nb] (row = query block i) -> kept blocks: the first
+    `sink` blocks, the `local` most recent (current included) and the kb best
+    of the others (MInference block-sparse, Sparse Frontier review §2.2.3)."""
+    s = _f32(scores)
+    ncols = s.shape[-1]
+    lead = s.shape[:-1]
+    rows = int(np.prod(lead)) if lead else 1
+    if idx_stride is None:
+        idx_stride = sink + local + kb
+    idx = np.empty(lead + (idx_stride,), np.int32)
+    cnt = np.empty(lead, np.int32)
+    lib().oracle_topk_pattern(_ptr(s), rows, ncols, sink, local, kb, _ptr(idx), idx_stride, _ptr(cnt))
+    return idx, cnt
+
+
+def topk_joint_heads(scores, kb_total: int, idx_stride: Optional[int] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """scores [B, Hkv, G, nb] per-head decode scores -> per-head kept blocks
+    [B, Hkv, G, idx_stride] under one budget of kb_total (head, block) pairs per
+    group, the last block kept by every head (Ada-KV, review §2.3.2)."""
+    s = _f32(scores)
+    B, Hkv, G, nb = s.shape
+    if idx_stride is None:
+        idx_stride = min(kb_total, nb - 1) + 1
+    idx = np.empty((B, Hkv, G, idx_stride), np.int32)
+    cnt = np.empty((B, Hkv, G), np.int32)
+    lib().oracle_topk_joint_heads(_ptr(s), B * Hkv, G, nb, kb_total, _ptr(idx), idx_stride, _ptr(cnt))
+    return idx, cnt
+
+
+def attend_decode_heads(q, k, v, bs: int, idx, scale: Optional[float] = None, rows=None
+                        ) -> Tuple[np.ndarray, np.ndarray]:
+    """Decode attention (fp64) with each query head's own kept blocks.
+    q [B,Hq,d], k/v [B,Hkv,Nk,d], idx [B,Hq,stride]."""
+    q, k, v, idx = _f32(q), _f32(k), _f32(v), _i32(idx)
+    B, Hq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    r = _rows_arg(rows, B * Hq)
+    out = np.empty((len(r), d), np.float64)
+    lse = np.empty((len(r),), np.float64)
+    lib().oracle_attend_decode_heads_rows(_ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, Nk, d, bs,
+                                          _ptr(idx), idx.shape[-1], float(scale),
+                                          _ptr(r), len(r), _ptr(out), _ptr(lse))
+    return out, lse
+
+
+def paged_gather(pool, table, nb: int) -> np.ndarray:
+    """pool [P, Hkv, bs, d], table [B, max_blocks] -> the logical cache
+    [B, Hkv, nb*bs, d] of the first nb blocks (PagedAttention, tutorial §7)."""
+    pool, table = _f32(pool), _i32(table)
+    P, Hkv, bs, d = pool.shape
+    B, max_blocks = table.shape
+    out = np.empty((B, Hkv, nb * bs, d), np.float32)
+    lib().oracle_paged_gather(_ptr(pool), _ptr(table), B, Hkv, nb, bs, d, max_blocks, _ptr(out))
+    return out

@@ -469,6 +469,142 @@ void oracle_attend_gist_rows(const float* q, const float* k, const float* v,
 }
 
 /* Threads the OpenMP runtime will use (for reporting the CPU baseline). */
+/* ------------------------------------------------------------------------ */
+/* 7. Fixed pattern + dynamic blocks (MInference block-sparse)              */
+/* ------------------------------------------------------------------------ */
+
+/* The Sparse Frontier review (§2.2.3, and its §3.2 method table: "局部 +
+ * 首块 + 动态选择块") describes block-sparse prefill as a local window, the
+ * first block(s) of the sequence (the attention sinks of StreamingLLM,
+ * §2.2.3) and a set of dynamically selected blocks per query block.
+ * Row r is query block i = r % ncols.  Forced: the first `sink` blocks
+ * (j < sink, j <= i) and the `local` most recent blocks (i-local < j <= i,
+ * the current block included).  Candidates: every other block j < i; the
+ * min(kb, #candidates) best of them by the step-3 order are kept.  Output:
+ * kept blocks ascending, then -1; count = their number. */
+void oracle_topk_pattern(const float* s, int64_t rows, int64_t ncols, int64_t sink, int64_t local,
+                         int64_t kb, int32_t* idx, int64_t idx_stride, int32_t* count)
+{
+#pragma omp parallel for schedule(dynamic, 16)
+    for (int64_t r = 0; r < rows; ++r) {
+        const int64_t i = r % ncols;
+        unsigned char* forced = (unsigned char*)calloc((size_t)(i + 1), 1);
+        cand_t* c = (cand_t*)malloc(sizeof(cand_t) * (size_t)(i + 1));
+        for (int64_t j = 0; j <= i; ++j)
+            if (j < sink || j > i - local) forced[j] = 1;
+        int64_t ncand = 0;
+        for (int64_t j = 0; j < i; ++j)
+            if (!forced[j]) { c[ncand].s = s[r * ncols + j]; c[ncand].j = (int32_t)j; ++ncand; }
+        qsort(c, (size_t)ncand, sizeof(cand_t), cand_cmp);
+        const int64_t take = (kb < ncand) ? kb : ncand;
+        int32_t* out = idx + r * idx_stride;
+        int64_t n = 0;
+        for (int64_t t = 0; t < take; ++t) out[n++] = c[t].j;
+        for (int64_t j = 0; j <= i; ++j) if (forced[j]) out[n++] = (int32_t)j;
+        qsort(out, (size_t)n, sizeof(int32_t), int_cmp);
+        for (int64_t t = n; t < idx_stride; ++t) out[t] = -1;
+        if (count) count[r] = (int32_t)n;
+        free(c); free(forced);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* 8. One budget shared by the heads of a group (Ada-KV)                    */
+/* ------------------------------------------------------------------------ */
+
+/* Ada-KV (Sparse Frontier review §2.3.2) keeps the top (k x h) units over
+ * all h heads together, so that important heads keep more keys and others
+ * fewer.  s [rows][G][ncols]: each query head's decode scores of one
+ * (batch, KV group) row.  The candidates are the pairs (h, j), j < ncols-1
+ * (decode: the last block is kept by every head); the min(kb_total,
+ * G*(ncols-1)) best by score are kept, equal scores going to the lower flat
+ * index h*(ncols-1) + j, NaN below every number.  idx [rows][G][idx_stride]:
+ * each head's kept blocks ascending, the last block included, then -1;
+ * count [rows][G]. */
+void oracle_topk_joint_heads(const float* s, int64_t rows, int64_t G, int64_t ncols, int64_t kb_total,
+                             int32_t* idx, int64_t idx_stride, int32_t* count)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < rows; ++r) {
+        const int64_t per = ncols - 1, ncand = G * per;
+        cand_t* c = (cand_t*)malloc(sizeof(cand_t) * (size_t)(ncand > 0 ? ncand : 1));
+        for (int64_t h = 0; h < G; ++h)
+            for (int64_t j = 0; j < per; ++j) {
+                c[h * per + j].s = s[(r * G + h) * ncols + j];
+                c[h * per + j].j = (int32_t)(h * per + j);
+            }
+        qsort(c, (size_t)ncand, sizeof(cand_t), cand_cmp);
+        const int64_t take = (kb_total < ncand) ? kb_total : ncand;
+        for (int64_t h = 0; h < G; ++h) {
+            int32_t* out = idx + (r * G + h) * idx_stride;
+            int64_t n = 0;
+            for (int64_t t = 0; t < take; ++t)
+                if (c[t].j / per == h) out[n++] = (int32_t)(c[t].j % per);
+            out[n++] = (int32_t)(ncols - 1);
+            qsort(out, (size_t)n, sizeof(int32_t), int_cmp);
+            for (int64_t t = n; t < idx_stride; ++t) out[t] = -1;
+            if (count) count[r * G + h] = (int32_t)n;
+        }
+        free(c);
+    }
+}
+
+/* Decode rows where every query head has its own kept blocks: as step 6's
+ * decode, with idx [B,Hq,idx_stride] read per head.  rows[n] = b*Hq + h. */
+void oracle_attend_decode_heads_rows(const float* q, const float* k, const float* v,
+                                     int64_t B, int64_t Hq, int64_t Hkv, int64_t Nk, int64_t d,
+                                     int64_t bs, const int32_t* idx, int64_t idx_stride, double scale,
+                                     const int64_t* rows, int64_t nrows, double* out, double* lse)
+{
+    const int64_t nb = Nk / bs, G = Hq / Hkv;
+    (void)B;
+#pragma omp parallel
+    {
+        unsigned char* sel = (unsigned char*)malloc((size_t)nb);
+        double* logits = (double*)malloc(sizeof(double) * (size_t)Nk);
+        const float** vals = (const float**)malloc(sizeof(float*) * (size_t)Nk);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t n = 0; n < nrows; ++n) {
+            const int64_t r = rows[n];
+            const int64_t b = r / Hq, h = r % Hq, g = h / G;
+            mark_blocks(idx + r * idx_stride, idx_stride, nb, sel);
+            const float* kb = k + (b * Hkv + g) * Nk * d;
+            const float* vb = v + (b * Hkv + g) * Nk * d;
+            int64_t m = 0;
+            for (int64_t u = 0; u < Nk; ++u) {
+                if (!sel[u / bs]) continue;
+                logits[m] = dot64(q + r * d, kb + u * d, d) * scale;
+                vals[m] = vb + u * d;
+                ++m;
+            }
+            softmax_rows(logits, vals, m, d, out + n * d, lse + n);
+        }
+        free(sel); free(logits); free(vals);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* 9. Paged KV cache                                                        */
+/* ------------------------------------------------------------------------ */
+
+/* PagedAttention (稀疏注意力 tutorial §7): the logically contiguous KV cache
+ * of a sequence is mapped onto physical blocks that need not be contiguous.
+ * pool [P][Hkv][bs][d] holds physical blocks; table [B][max_blocks] maps
+ * sequence b's logical block j to physical block table[b][j].  Writes the
+ * logical view out [B][Hkv][nb*bs][d] of the first nb blocks. */
+void oracle_paged_gather(const float* pool, const int32_t* table, int64_t B, int64_t Hkv, int64_t nb,
+                         int64_t bs, int64_t d, int64_t max_blocks, float* out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t bg = 0; bg < B * Hkv; ++bg) {
+        const int64_t b = bg / Hkv, g = bg % Hkv;
+        for (int64_t j = 0; j < nb; ++j) {
+            const int64_t p = table[b * max_blocks + j];
+            memcpy(out + ((bg * nb + j) * bs) * d, pool + ((p * Hkv + g) * bs) * d, sizeof(float) * (size_t)(bs * d));
+        }
+    }
+}
+
 int oracle_max_threads(void)
 {
 #ifdef _OPENMP

@@ -476,3 +476,148 @@ def test_gist_mixture_matches_library_on_explicit_key_set():
             V = np.concatenate(vals)[None, None]
             ref = _sdpa64(q[b, h][None, None, None, :], K, V)
             assert np.allclose(out[b * Hq + h], ref[0, 0, 0], atol=1e-10, rtol=0)
+
+
+# ----------------------------------------------------------------------------
+# fixed pattern + dynamic blocks (MInference block-sparse): brute force, the
+# tutorial's sliding window, and the plain causal top-k it reduces to
+# ----------------------------------------------------------------------------
+
+def test_topk_pattern_matches_bruteforce():
+    r = _rng(70)
+    for trial in range(60):
+        nb = int(r.integers(1, 10))
+        sink = int(r.integers(0, 3))
+        local = int(r.integers(1, 4))
+        kb = int(r.integers(0, nb + 1))
+        s = r.integers(-3, 4, size=(nb, nb)).astype(np.float32)   # many ties
+        idx, cnt = oracle.topk_pattern(s, sink, local, kb)
+        for i in range(nb):
+            forced = [j for j in range(i + 1) if j < sink or j > i - local]
+            cand = [j for j in range(i) if j not in forced]
+            want = sorted(_brute_topk(s[i].tolist(), cand, kb) + forced)
+            got = [int(x) for x in idx[i] if x >= 0]
+            assert got == want, (trial, i, sink, local, kb)
+            assert cnt[i] == len(want) and np.all(idx[i][len(want):] == -1)
+
+
+def test_topk_pattern_without_sink_and_window_is_the_causal_topk():
+    r = _rng(71)
+    s = r.standard_normal((2, 3, 40, 40)).astype(np.float32)
+    for kb in (0, 3, 17, 40):
+        got, gcnt = oracle.topk_pattern(s, 0, 1, kb, idx_stride=kb + 1)
+        want, wcnt = oracle.topk(s, oracle.TOPK_CAUSAL_BLOCK, kb)
+        assert np.array_equal(got, want) and np.array_equal(gcnt, wcnt)
+
+
+def test_topk_pattern_window_only_is_the_tutorial_w3_window():
+    """No sink, a local window of 3 blocks of one token, no dynamic blocks:
+    the tutorial's 6-token, w = 3 causal sliding window (§3)."""
+    golden = _read_golden_sets("sliding_window_w3.txt")
+    N = 6
+    s = _rng(72).standard_normal((N, N)).astype(np.float32)   # scores play no part
+    idx, _ = oracle.topk_pattern(s, 0, 3, 0)
+    mask = oracle.prefill_mask(N, 1, idx)
+    for t in range(N):
+        assert [u + 1 for u in range(N) if mask[t, u]] == golden[t + 1]
+
+
+def test_topk_pattern_streaming_sink_plus_window_closed_form():
+    """One sink block, a window of w blocks, no dynamic blocks: the
+    StreamingLLM-style set {0} u {i-w+1, ..., i} (review §2.2.3)."""
+    nb, w = 20, 4
+    s = _rng(73).standard_normal((nb, nb)).astype(np.float32)
+    idx, cnt = oracle.topk_pattern(s, 1, w, 0)
+    for i in range(nb):
+        want = sorted(set([0]) | set(range(max(0, i - w + 1), i + 1)))
+        assert [int(x) for x in idx[i] if x >= 0] == want and cnt[i] == len(want)
+
+
+# ----------------------------------------------------------------------------
+# one budget shared by a group's heads (Ada-KV)
+# ----------------------------------------------------------------------------
+
+def test_topk_joint_heads_matches_bruteforce():
+    r = _rng(74)
+    for trial in range(40):
+        G = int(r.integers(1, 4))
+        nb = int(r.integers(1, 6))
+        kb_total = int(r.integers(0, G * nb + 1))
+        s = r.integers(-2, 3, size=(1, 1, G, nb)).astype(np.float32)
+        idx, cnt = oracle.topk_joint_heads(s, kb_total, idx_stride=G * nb + 1)
+        flat = [float(s[0, 0, h, j]) for h in range(G) for j in range(nb - 1)]
+        chosen = _brute_topk(flat, list(range(len(flat))), kb_total)
+        for h in range(G):
+            want = sorted([c % (nb - 1) for c in chosen if c // (nb - 1) == h] + [nb - 1]) if nb > 1 else [0]
+            got = [int(x) for x in idx[0, 0, h] if x >= 0]
+            assert got == want, (trial, G, nb, kb_total, h)
+            assert cnt[0, 0, h] == len(want)
+        assert sum(int(c) for c in cnt[0, 0]) == min(kb_total, G * (nb - 1)) + G
+
+
+def test_topk_joint_heads_single_head_is_the_decode_topk():
+    r = _rng(75)
+    s = r.standard_normal((3, 2, 1, 300)).astype(np.float32)
+    for kb in (0, 5, 96, 400):
+        got, gcnt = oracle.topk_joint_heads(s, kb, idx_stride=min(kb, 299) + 1)
+        want, wcnt = oracle.topk(s[:, :, 0], oracle.TOPK_LAST_BLOCK, kb, idx_stride=min(kb, 299) + 1)
+        assert np.array_equal(got[:, :, 0], want) and np.array_equal(gcnt[:, :, 0], wcnt)
+
+
+def test_decode_heads_with_shared_lists_is_the_group_decode():
+    q, k, v = _small_decode(76)
+    bs, kb = 32, 4
+    Hkv = k.shape[1]
+    G = q.shape[1] // Hkv
+    kbar = oracle.pool_keys(k, bs)
+    _, _, idx, _ = oracle.decode_select(q, kbar, Hkv, kb)
+    per_head = np.repeat(idx, G, axis=1)   # every head of a group keeps the group's blocks
+    a, la = oracle.attend_decode(q, k, v, bs, idx)
+    b, lb = oracle.attend_decode_heads(q, k, v, bs, per_head)
+    assert np.array_equal(a, b) and np.array_equal(la, lb)
+
+
+def test_decode_heads_matches_library_with_per_head_masks():
+    q, k, v = _small_decode(77)
+    bs = 32
+    B, Hq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    G = Hq // Hkv
+    nb = Nk // bs
+    r = _rng(78)
+    idx = np.full((B, Hq, 6), -1, np.int32)
+    mask = np.zeros((B, Hq, 1, Nk), bool)
+    for b in range(B):
+        for h in range(Hq):
+            sel = sorted(r.choice(nb, size=int(r.integers(1, 6)), replace=False).tolist())
+            idx[b, h, :len(sel)] = sel
+            for j in sel:
+                mask[b, h, 0, j * bs:(j + 1) * bs] = True
+    out, _ = oracle.attend_decode_heads(q, k, v, bs, idx)
+    ref = _sdpa64(q[:, :, None, :], np.repeat(k, G, 1), np.repeat(v, G, 1), mask=mask)
+    assert np.allclose(out.reshape(B, Hq, d), ref[:, :, 0], atol=1e-10, rtol=0)
+
+
+# ----------------------------------------------------------------------------
+# paged KV cache
+# ----------------------------------------------------------------------------
+
+def test_paged_gather_identity_table_is_the_contiguous_cache():
+    B, Hkv, nb, bs, d = 2, 3, 5, 4, 8
+    k = _rng(79).standard_normal((B, Hkv, nb * bs, d)).astype(np.float32)
+    # pool laid out [P][Hkv][bs][d] with P = B*nb and the identity mapping
+    pool = k.reshape(B, Hkv, nb, bs, d).transpose(0, 2, 1, 3, 4).reshape(B * nb, Hkv, bs, d)
+    table = np.arange(B * nb, dtype=np.int32).reshape(B, nb)
+    assert np.array_equal(oracle.paged_gather(pool, table, nb), k)
+
+
+def test_paged_gather_permuted_pages():
+    r = _rng(80)
+    B, Hkv, nb, bs, d, P = 2, 2, 4, 3, 5, 11
+    pool = r.standard_normal((P, Hkv, bs, d)).astype(np.float32)
+    table = np.stack([r.permutation(P)[:nb] for _ in range(B)]).astype(np.int32)
+    out = oracle.paged_gather(pool, table, nb)
+    for b in range(B):
+        for j in range(nb):
+            for g in range(Hkv):
+                assert np.array_equal(out[b, g, j * bs:(j + 1) * bs], pool[table[b, j], g])
