@@ -67,11 +67,11 @@ typedef struct {
 } bsa_shape_t;
 
 /* selector modes for bsa_score_blocks */
-enum { BSA_SCORE_PREFILL = 0, BSA_SCORE_DECODE = 1, BSA_SCORE_GIST = 2 };
+enum { BSA_SCORE_PREFILL = 0, BSA_SCORE_DECODE = 1, BSA_SCORE_GIST = 2, BSA_SCORE_DECODE_HEADS = 3 };
 /* candidate rules for bsa_topk_select */
 enum { BSA_TOPK_CAUSAL_BLOCK = 0, BSA_TOPK_LAST_BLOCK = 1, BSA_TOPK_PLAIN = 2 };
 /* operations for bsa_workspace_bytes */
-enum { BSA_OP_DECODE = 0, BSA_OP_GIST_DECODE = 1 };
+enum { BSA_OP_DECODE = 0, BSA_OP_GIST_DECODE = 1, BSA_OP_DECODE_HEADS = 2 };
 
 /*
  * bsa_score_blocks -- the cheap selector (block pooling + scoring).
@@ -98,6 +98,11 @@ enum { BSA_OP_DECODE = 0, BSA_OP_GIST_DECODE = 1 };
  * mode BSA_SCORE_GIST     (SSA: per query head, no pooling)
  *   q [B,Hq,d]; k = gist keys [B,Hkv,nc,d] with nc = Nk/block;
  *   scores [B,Hq,nc] fp32.  pooled_* must be NULL.
+ * mode BSA_SCORE_DECODE_HEADS  (one score row per query head, for a budget
+ *   shared across the heads: Sparse Frontier review §2.3.2, Ada-KV)
+ *   q [B,Hq,d] (d in {64,128}); pooled_k_in [B,Hkv,nb,d] fp32 (required);
+ *   scores [B,Hq,nb] fp32: q_h . pooled_k_j / sqrt(d) in the same fixed
+ *   order.  k, pooled_q_out and pooled_k_out must be NULL.
  */
 bsa_status_t bsa_score_blocks(const bsa_shape_t* shape, int mode, const void* q, const void* k,
                               const float* pooled_k_in, float* pooled_q_out, float* pooled_k_out,
@@ -122,6 +127,43 @@ bsa_status_t bsa_score_blocks(const bsa_shape_t* shape, int mode, const void* q,
  */
 bsa_status_t bsa_topk_select(const float* scores, int rows, int ncols, int mode, int kb,
                              int* idx_out, int idx_stride, int* count_out, void* stream);
+
+/*
+ * bsa_topk_select_pattern -- prefill selection with a fixed part and a
+ * dynamic part.
+ * Cite: Sparse Frontier review §2.2.3 (MInference block-sparse: each query
+ * block keeps the local blocks, the first block and a set of dynamically
+ * selected blocks; StreamingLLM's attention sinks: the first tokens) and its
+ * §3.2 method table (局部 + 首块 + 动态选择块).
+ * scores [rows, ncols] as for BSA_TOPK_CAUSAL_BLOCK (row r is query block
+ * i = r % ncols).  Kept for row r: blocks j < sink (j <= i), the `local` most
+ * recent blocks i-local < j <= i (current included), and the kb best of the
+ * blocks in between by the order of bsa_topk_select.  sink >= 0, local >= 1,
+ * kb >= 0.  idx_out [rows, idx_stride], idx_stride >= sink + local + kb:
+ * kept blocks ascending, then -1; count_out [rows] (optional).
+ * Limits: ncols <= 8192.  With sink = 0 and local = 1 it is
+ * bsa_topk_select(BSA_TOPK_CAUSAL_BLOCK).
+ */
+bsa_status_t bsa_topk_select_pattern(const float* scores, int rows, int ncols, int sink, int local, int kb,
+                                     int* idx_out, int idx_stride, int* count_out, void* stream);
+
+/*
+ * bsa_topk_select_joint_heads -- decode selection under one budget shared by
+ * the query heads of a KV group.
+ * Cite: Sparse Frontier review §2.3.2 (Ada-KV: the top (k x h) units over
+ * all h heads, so important heads keep more keys and others fewer).
+ * scores [rows, heads, ncols] fp32: per-head decode scores of one (batch, KV
+ * group) row each (bsa_score_blocks mode BSA_SCORE_DECODE_HEADS).  Candidates:
+ * the pairs (h, j), j < ncols-1; the kb_total best are kept (equal scores:
+ * the lower h*(ncols-1)+j first; NaN below every number); the last block
+ * ncols-1 is kept by every head.  idx_out [rows, heads, idx_stride]: each
+ * head's kept blocks ascending, then -1, idx_stride >= min(kb_total,
+ * ncols-1) + 1; count_out [rows, heads] (optional).
+ * Limits: heads <= 16, heads*(ncols-1) <= 8192.  With one head it is
+ * bsa_topk_select(BSA_TOPK_LAST_BLOCK).
+ */
+bsa_status_t bsa_topk_select_joint_heads(const float* scores, int rows, int heads, int ncols, int kb_total,
+                                         int* idx_out, int idx_stride, int* count_out, void* stream);
 
 /*
  * bsa_decode_select -- the decode selector in one call: the group query
@@ -226,6 +268,69 @@ bsa_status_t bsa_gist_expand_decode(const bsa_shape_t* shape, const void* q, con
                                     void* o, float* lse, void* stream);
 
 /*
+ * bsa_sparse_attn_decode_heads -- decode where every query head has its own
+ * kept blocks (e.g. from bsa_topk_select_joint_heads).
+ * Cite: 稀疏注意力 tutorial §5 (decode over the history); Sparse Frontier
+ * review §2.3.2 (Ada-KV: per-head budgets) and §2.4.2 (full cache retained,
+ * selective loading).
+ * As bsa_sparse_attn_decode, but idx [B,Hq,idx_stride] holds one ascending,
+ * -1 ended list per query head.  The union of a group's lists is gathered
+ * once and each head masks the blocks it did not keep.
+ * workspace: bsa_workspace_bytes(BSA_OP_DECODE_HEADS, shape, idx_stride).
+ * Built: BF16, d = 128, block = 64, nb = Nk/64 a multiple of 32 and at most
+ * 8192, at most 16 query heads per KV group.
+ */
+bsa_status_t bsa_sparse_attn_decode_heads(const bsa_shape_t* shape, const void* q, const void* k_cache,
+                                          const void* v_cache, const int* idx, int idx_stride,
+                                          float softmax_scale, void* workspace, size_t workspace_bytes,
+                                          void* o, float* lse, void* stream);
+
+/*
+ * bsa_sparse_attn_decode_paged -- bsa_sparse_attn_decode over a paged KV
+ * cache.
+ * Cite: 稀疏注意力 tutorial §7 (PagedAttention: the logically contiguous KV
+ * cache is mapped onto physical blocks that need not be contiguous) and §5
+ * (decode); Sparse Frontier review §2.4.2 (full cache retained, selective
+ * loading).
+ * k_pool/v_pool [num_pages, Hkv, 64, d] bf16: physical blocks of 64 tokens.
+ * block_table [B, table_stride] int32: sequence b's logical block j is
+ * physical block block_table[b*table_stride + j] (the same for every KV
+ * head); table_stride >= nb = Nk/64, shape->Nk = the logical cache length.
+ * idx [B,Hkv,idx_stride] holds LOGICAL block ids (as the selector gives them
+ * from the logical pooled summary); a logical id out of range or a table
+ * entry outside [0, num_pages) is skipped and flagged (BSA_DEV_BAD_INDEX).
+ * Otherwise as bsa_sparse_attn_decode (workspace: bsa_workspace_bytes(
+ * BSA_OP_DECODE, shape, idx_stride)); with the identity table the result is
+ * that of bsa_sparse_attn_decode on the contiguous cache, bit for bit.
+ */
+bsa_status_t bsa_sparse_attn_decode_paged(const bsa_shape_t* shape, const void* q, const void* k_pool,
+                                          const void* v_pool, int num_pages, const int* block_table,
+                                          int table_stride, const int* idx, int idx_stride, float softmax_scale,
+                                          void* workspace, size_t workspace_bytes, void* o, float* lse,
+                                          void* stream);
+
+/*
+ * bsa_paged_append -- append shape->Nq new tokens to every sequence of a
+ * paged cache and keep the decode selector's block-mean summary current.
+ * Cite: 稀疏注意力 tutorial §7 (PagedAttention) and §4.6 (one pooled key per
+ * block for coarse scoring); Sparse Frontier review §2.4.2 (the retained
+ * cache grows as decoding proceeds).
+ * k_new/v_new [B, Hkv, Nq, d] bf16; seq_lens [B] int32: the tokens each
+ * sequence holds before the append (left unchanged: the caller advances
+ * them); token t goes to logical position seq_lens[b] + t, i.e. logical block
+ * (seq_lens[b]+t)/64 through block_table [B, table_stride].  pooled_k
+ * [B, Hkv, table_stride, d] fp32 (optional): every block that this append
+ * completes gets its mean key (tokens ascending, fp32, one division --
+ * the arithmetic of bsa_score_blocks' pooling, so equal to pooling the
+ * whole logical cache).  Incomplete blocks are not pooled.  Built: BF16,
+ * block 64.  A position past the table or a table entry outside
+ * [0, num_pages) is skipped and flagged (BSA_DEV_BAD_INDEX).
+ */
+bsa_status_t bsa_paged_append(const bsa_shape_t* shape, const void* k_new, const void* v_new, const int* seq_lens,
+                              const int* block_table, int table_stride, int num_pages, void* k_pool,
+                              void* v_pool, float* pooled_k, void* stream);
+
+/*
  * bsa_sparse_attn_decode_noalloc -- bsa_sparse_attn_decode for callers that
  * cannot allocate device memory (no counterpart on the source pages; it is a
  * deployment convenience).  Some callers have no way to provide the decode
@@ -249,7 +354,8 @@ bsa_status_t bsa_sparse_attn_decode_noalloc(const bsa_shape_t* shape, const void
                                             float softmax_scale, void* o, float* lse, void* stream);
 
 /* Scratch bytes a decode call needs (op = BSA_OP_*; budget = idx_stride for
- * BSA_OP_DECODE, topk for BSA_OP_GIST_DECODE).  0 on a bad shape. */
+ * BSA_OP_DECODE and BSA_OP_DECODE_HEADS, topk for BSA_OP_GIST_DECODE).  0 on
+ * a bad shape. */
 size_t bsa_workspace_bytes(int op, const bsa_shape_t* shape, int budget);
 
 /* Human-readable name of a status code (static string). */

@@ -18,23 +18,25 @@ import torch
 __all__ = [
     "BsaError", "BsaShape", "lib", "LIB_PATH",
     "BSA_F32", "BSA_BF16",
-    "BSA_SCORE_PREFILL", "BSA_SCORE_DECODE", "BSA_SCORE_GIST",
+    "BSA_SCORE_PREFILL", "BSA_SCORE_DECODE", "BSA_SCORE_GIST", "BSA_SCORE_DECODE_HEADS",
     "BSA_TOPK_CAUSAL_BLOCK", "BSA_TOPK_LAST_BLOCK", "BSA_TOPK_PLAIN",
-    "BSA_OP_DECODE", "BSA_OP_GIST_DECODE",
+    "BSA_OP_DECODE", "BSA_OP_GIST_DECODE", "BSA_OP_DECODE_HEADS",
     "make_shape", "bsa_score_blocks", "bsa_topk_select", "bsa_sparse_attn_prefill",
     "bsa_gated_attn_fwd", "bsa_sparse_attn_decode", "bsa_gist_expand_decode",
     "bsa_workspace_bytes", "bsa_status_string", "bsa_device_status", "bsa_version",
     "bsa_sparse_attn_decode_noalloc", "bsa_decode_split_override", "bsa_selftest_wait_expiry",
-    "bsa_prefill_kernel_override", "bsa_decode_select", "EXPORTED_SYMBOLS",
+    "bsa_prefill_kernel_override", "bsa_decode_select", "bsa_topk_select_pattern",
+    "bsa_topk_select_joint_heads", "bsa_sparse_attn_decode_heads", "bsa_sparse_attn_decode_paged",
+    "bsa_paged_append", "EXPORTED_SYMBOLS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libbsa.so")
 
 BSA_OK, BSA_ERR_INVALID_ARG, BSA_ERR_UNSUPPORTED, BSA_ERR_CUDA, BSA_ERR_TIMEOUT, BSA_ERR_DEVICE = range(6)
 BSA_F32, BSA_BF16 = 0, 1
-BSA_SCORE_PREFILL, BSA_SCORE_DECODE, BSA_SCORE_GIST = 0, 1, 2
+BSA_SCORE_PREFILL, BSA_SCORE_DECODE, BSA_SCORE_GIST, BSA_SCORE_DECODE_HEADS = 0, 1, 2, 3
 BSA_TOPK_CAUSAL_BLOCK, BSA_TOPK_LAST_BLOCK, BSA_TOPK_PLAIN = 0, 1, 2
-BSA_OP_DECODE, BSA_OP_GIST_DECODE = 0, 1
+BSA_OP_DECODE, BSA_OP_GIST_DECODE, BSA_OP_DECODE_HEADS = 0, 1, 2
 
 # Every symbol the C header declares.
 EXPORTED_SYMBOLS = (
@@ -42,7 +44,8 @@ EXPORTED_SYMBOLS = (
     "bsa_sparse_attn_decode", "bsa_gist_expand_decode", "bsa_workspace_bytes",
     "bsa_status_string", "bsa_device_status", "bsa_version", "bsa_sparse_attn_decode_noalloc",
     "bsa_decode_split_override", "bsa_selftest_wait_expiry", "bsa_prefill_kernel_override",
-    "bsa_decode_select",
+    "bsa_decode_select", "bsa_topk_select_pattern", "bsa_topk_select_joint_heads", "bsa_sparse_attn_decode_heads",
+    "bsa_sparse_attn_decode_paged", "bsa_paged_append",
 )
 
 
@@ -67,6 +70,13 @@ _SIGS = {
     "bsa_score_blocks": (_i, [ctypes.POINTER(BsaShape), _i, _p, _p, _p, _p, _p, _p, _p]),
     "bsa_topk_select": (_i, [_p, _i, _i, _i, _i, _p, _i, _p, _p]),
     "bsa_decode_select": (_i, [ctypes.POINTER(BsaShape), _p, _p, _i, _p, _p, _p, _i, _p, _p]),
+    "bsa_topk_select_pattern": (_i, [_p, _i, _i, _i, _i, _i, _p, _i, _p, _p]),
+    "bsa_sparse_attn_decode_paged": (_i, [ctypes.POINTER(BsaShape), _p, _p, _p, _i, _p, _i, _p, _i, ctypes.c_float,
+                                          _p, ctypes.c_size_t, _p, _p, _p]),
+    "bsa_paged_append": (_i, [ctypes.POINTER(BsaShape), _p, _p, _p, _p, _i, _i, _p, _p, _p, _p]),
+    "bsa_topk_select_joint_heads": (_i, [_p, _i, _i, _i, _i, _p, _i, _p, _p]),
+    "bsa_sparse_attn_decode_heads": (_i, [ctypes.POINTER(BsaShape), _p, _p, _p, _p, _i, ctypes.c_float, _p,
+                                          ctypes.c_size_t, _p, _p, _p]),
     "bsa_sparse_attn_prefill": (_i, [ctypes.POINTER(BsaShape), _p, _p, _p, _p, _i, ctypes.c_float, _p, _p, _p]),
     "bsa_gated_attn_fwd": (_i, [ctypes.POINTER(BsaShape), _p, _p, _p, _p, _i, _p, ctypes.c_float, _p, _p, _p]),
     "bsa_sparse_attn_decode": (_i, [ctypes.POINTER(BsaShape), _p, _p, _p, _p, _i, ctypes.c_float, _p,
@@ -188,6 +198,45 @@ def bsa_topk_select(scores, rows: int, ncols: int, mode: int, kb: int, idx_out, 
     _check("bsa_topk_select", lib.bsa_topk_select(
         _ptr(scores), int(rows), int(ncols), int(mode), int(kb), _ptr(idx_out), int(idx_stride),
         _ptr(count_out), _stream(stream)))
+
+
+def bsa_topk_select_pattern(scores, rows: int, ncols: int, sink: int, local: int, kb: int, idx_out,
+                            idx_stride: int, count_out=None, stream=None) -> None:
+    _check("bsa_topk_select_pattern", lib.bsa_topk_select_pattern(
+        _ptr(scores), int(rows), int(ncols), int(sink), int(local), int(kb), _ptr(idx_out), int(idx_stride),
+        _ptr(count_out), _stream(stream)))
+
+
+def bsa_topk_select_joint_heads(scores, rows: int, heads: int, ncols: int, kb_total: int, idx_out,
+                                idx_stride: int, count_out=None, stream=None) -> None:
+    _check("bsa_topk_select_joint_heads", lib.bsa_topk_select_joint_heads(
+        _ptr(scores), int(rows), int(heads), int(ncols), int(kb_total), _ptr(idx_out), int(idx_stride),
+        _ptr(count_out), _stream(stream)))
+
+
+def bsa_sparse_attn_decode_heads(shape: BsaShape, q, k_cache, v_cache, idx, idx_stride: int, softmax_scale: float,
+                                 workspace, o, lse=None, stream=None) -> None:
+    _check("bsa_sparse_attn_decode_heads", lib.bsa_sparse_attn_decode_heads(
+        ctypes.byref(shape), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(idx), int(idx_stride),
+        ctypes.c_float(softmax_scale), _ptr(workspace), ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+        _ptr(o), _ptr(lse), _stream(stream)))
+
+
+def bsa_sparse_attn_decode_paged(shape: BsaShape, q, k_pool, v_pool, block_table, idx, idx_stride: int,
+                                 softmax_scale: float, workspace, o, lse=None, stream=None) -> None:
+    """Decode over a paged cache: pools [P,Hkv,64,d], block_table [B, table_stride]."""
+    _check("bsa_sparse_attn_decode_paged", lib.bsa_sparse_attn_decode_paged(
+        ctypes.byref(shape), _ptr(q), _ptr(k_pool), _ptr(v_pool), int(k_pool.shape[0]), _ptr(block_table),
+        int(block_table.shape[-1]), _ptr(idx), int(idx_stride), ctypes.c_float(softmax_scale), _ptr(workspace),
+        ctypes.c_size_t(workspace.numel() * workspace.element_size()), _ptr(o), _ptr(lse), _stream(stream)))
+
+
+def bsa_paged_append(shape: BsaShape, k_new, v_new, seq_lens, block_table, k_pool, v_pool, pooled_k=None,
+                     stream=None) -> None:
+    """Write k_new/v_new [B,Hkv,T,d] at positions seq_lens[b]+t of the paged cache; pool completed blocks."""
+    _check("bsa_paged_append", lib.bsa_paged_append(
+        ctypes.byref(shape), _ptr(k_new), _ptr(v_new), _ptr(seq_lens), _ptr(block_table), int(block_table.shape[-1]),
+        int(k_pool.shape[0]), _ptr(k_pool), _ptr(v_pool), _ptr(pooled_k), _stream(stream)))
 
 
 def bsa_decode_select(shape: BsaShape, q, pooled_k, kb: int, scores, idx_out, idx_stride: int,

@@ -3,6 +3,7 @@
 // or frees device memory; scratch comes from the caller.
 #include <math.h>
 
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 
@@ -175,6 +176,32 @@ GistLayout gist_layout(const bsa_shape_t* s, int topk, int num_sms) {
   return L;
 }
 
+// Workspace of the per-head decode: each head's kept-block bitmap, the
+// group's union list (count first), the split partials.
+struct HeadsLayout {
+  size_t expanded, union_list, partial, total;
+  int union_stride;
+  DecodePlan plan;
+};
+
+HeadsLayout heads_layout(const bsa_shape_t* s, int idx_stride, int num_sms) {
+  HeadsLayout L{};
+  const int nb = s->Nk / s->block;
+  const int G = s->Hq / s->Hkv;
+  const int64_t rows = static_cast<int64_t>(s->B) * s->Hq;
+  L.union_stride = 1 + std::min(nb, G * idx_stride);
+  L.plan = decode_plan(s->B * s->Hkv, L.union_stride - 1, num_sms);
+  size_t off = 0;
+  L.expanded = off;
+  off = align256(off + rows * (nb / 32) * sizeof(uint32_t));
+  L.union_list = off;
+  off = align256(off + static_cast<size_t>(s->B) * s->Hkv * L.union_stride * sizeof(int));
+  L.partial = off;
+  off = align256(off + rows * L.plan.max_slots * (s->d + 4) * sizeof(float));
+  L.total = off;
+  return L;
+}
+
 // Self-test of the bounded-wait expiry path: one thread waits, with a small
 // budget, on a shared-memory barrier that nothing arrives on.  The wait gives
 // up, raises BSA_DEV_TIMEOUT in the status word and the kernel returns.
@@ -271,6 +298,10 @@ size_t bsa_workspace_bytes(int op, const bsa_shape_t* s, int budget) {
     return align256(static_cast<size_t>(s->B) * s->Hq * P.max_slots * (s->d + 4) * sizeof(float));
   }
   if (op == BSA_OP_GIST_DECODE) return gist_layout(s, budget, sms).total;
+  if (op == BSA_OP_DECODE_HEADS) {
+    if (budget < 1) return 0;
+    return heads_layout(s, budget, sms).total;
+  }
   return 0;
 }
 
@@ -316,6 +347,13 @@ bsa_status_t bsa_score_blocks(const bsa_shape_t* s, int mode, const void* q, con
     if (e == cudaSuccess)
       e = launch_score_decode(q, bf16, kbar, s->B, s->Hq, s->Hkv, nb, s->d, scale, scores, pooled_q_out, cs);
     return cuda_status(e);
+  }
+  if (mode == BSA_SCORE_DECODE_HEADS) {
+    if (s->Nq != 1 || pooled_k_in == nullptr || !aligned16(pooled_k_in) || k || pooled_q_out || pooled_k_out)
+      return BSA_ERR_INVALID_ARG;
+    if (s->d != 64 && s->d != 128) return BSA_ERR_UNSUPPORTED;
+    if (G > 16) return BSA_ERR_UNSUPPORTED;
+    return cuda_status(launch_score_heads(q, bf16, pooled_k_in, s->B, s->Hq, s->Hkv, nb, s->d, scale, scores, cs));
   }
   if (mode == BSA_SCORE_GIST) {
     if (s->Nq != 1 || k == nullptr || !aligned16(k) || pooled_k_in || pooled_q_out || pooled_k_out)
@@ -369,6 +407,32 @@ bsa_status_t bsa_decode_select(const bsa_shape_t* s, const void* q, const float*
   if (e == cudaSuccess)
     e = launch_topk(scores, s->B * s->Hkv, nb, BSA_TOPK_LAST_BLOCK, kb, idx_out, idx_stride, count_out, cs);
   return cuda_status(e);
+}
+
+bsa_status_t bsa_topk_select_pattern(const float* scores, int rows, int ncols, int sink, int local, int kb,
+                                     int* idx_out, int idx_stride, int* count_out, void* stream) {
+  if (scores == nullptr || idx_out == nullptr || rows < 0 || ncols < 1 || kb < 0 || sink < 0 || local < 1)
+    return BSA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(idx_stride) < static_cast<int64_t>(sink) + local + kb) return BSA_ERR_INVALID_ARG;
+  if (ncols > 8192) return BSA_ERR_UNSUPPORTED;
+  if (rows == 0) return BSA_OK;
+  bsa_status_t st = device_state(nullptr, nullptr);
+  if (st != BSA_OK) return st;
+  return cuda_status(launch_topk_pattern(scores, rows, ncols, sink, local, kb, idx_out, idx_stride, count_out,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+bsa_status_t bsa_topk_select_joint_heads(const float* scores, int rows, int heads, int ncols, int kb_total,
+                                         int* idx_out, int idx_stride, int* count_out, void* stream) {
+  if (scores == nullptr || idx_out == nullptr || rows < 0 || heads < 1 || ncols < 1 || kb_total < 0)
+    return BSA_ERR_INVALID_ARG;
+  if (idx_stride < std::min(kb_total, ncols - 1) + 1) return BSA_ERR_INVALID_ARG;
+  if (heads > 16 || static_cast<int64_t>(heads) * (ncols - 1) > 8192) return BSA_ERR_UNSUPPORTED;
+  if (rows == 0) return BSA_OK;
+  bsa_status_t st = device_state(nullptr, nullptr);
+  if (st != BSA_OK) return st;
+  return cuda_status(launch_topk_joint(scores, rows, heads, ncols, kb_total, idx_out, idx_stride, count_out,
+                                       static_cast<cudaStream_t>(stream)));
 }
 
 static bsa_status_t prefill_common(const bsa_shape_t* s, const void* q, const void* k, const void* v,
@@ -528,7 +592,8 @@ bsa_status_t bsa_gist_expand_decode(const bsa_shape_t* s, const void* q, const v
     e = cudaMemcpyAsync(idx_out, idx_in, static_cast<size_t>(rows) * topk * sizeof(int), cudaMemcpyDeviceToDevice, cs);
   }
   if (e == cudaSuccess)
-    e = launch_gist_union(idx, s->B, s->Hq, s->Hkv, topk, idx_stride, nc, expanded, ulist, L.union_stride, status, cs);
+    e = launch_gist_union(idx, s->B, s->Hq, s->Hkv, topk, idx_stride, nc, expanded, ulist, L.union_stride, true,
+                          status, cs);
   DecodeArgs a;
   a.B = s->B;
   a.Hq = s->Hq;
@@ -549,6 +614,124 @@ bsa_status_t bsa_gist_expand_decode(const bsa_shape_t* s, const void* q, const v
   if (e == cudaSuccess) e = launch_attn_decode_bf16(&mq, &mk, &mv, &mgk, &mgv, a, cs);
   if (e == cudaSuccess) e = launch_decode_combine(a.partial, a, s->d, true, o, lse, cs);
   return cuda_status(e);
+}
+
+bsa_status_t bsa_sparse_attn_decode_heads(const bsa_shape_t* s, const void* q, const void* k_cache,
+                                          const void* v_cache, const int* idx, int idx_stride, float softmax_scale,
+                                          void* workspace, size_t workspace_bytes, void* o, float* lse,
+                                          void* stream) {
+  bsa_status_t st = decode_checks(s, q, k_cache, v_cache, o);
+  if (st != BSA_OK) return st;
+  const int nb = s->Nk / s->block;
+  if (!idx || idx_stride < 1 || !(softmax_scale > 0.0f) || !workspace) return BSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return BSA_ERR_INVALID_ARG;
+  if (nb % 32 != 0 || nb > 8192) return BSA_ERR_UNSUPPORTED;
+  uint32_t* status = nullptr;
+  int sms = 0;
+  if ((st = device_state(&status, &sms)) != BSA_OK) return st;
+  const HeadsLayout L = heads_layout(s, idx_stride, sms);
+  if (workspace_bytes < L.total) return BSA_ERR_INVALID_ARG;
+  char* ws = static_cast<char*>(workspace);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const int G = s->Hq / s->Hkv;
+  const int rows = s->B * s->Hq;
+  uint32_t* expanded = reinterpret_cast<uint32_t*>(ws + L.expanded);
+  int* ulist = reinterpret_cast<int*>(ws + L.union_list);
+  CUtensorMap mq, mk, mv;
+  if (!make_map_bf16(&mq, q, static_cast<uint64_t>(rows), static_cast<uint32_t>(G)) ||
+      !make_map_bf16(&mk, k_cache, static_cast<uint64_t>(s->B) * s->Hkv * s->Nk, 64) ||
+      !make_map_bf16(&mv, v_cache, static_cast<uint64_t>(s->B) * s->Hkv * s->Nk, 64))
+    return BSA_ERR_CUDA;
+  // the union of the heads' kept blocks, each head's bitmap; no gists
+  cudaError_t e = launch_gist_union(idx, s->B, s->Hq, s->Hkv, idx_stride, idx_stride, nb, expanded, ulist,
+                                    L.union_stride, false, status, cs);
+  DecodeArgs a;
+  a.B = s->B;
+  a.Hq = s->Hq;
+  a.Hkv = s->Hkv;
+  a.Nk = s->Nk;
+  a.bs = s->block;
+  a.list = ulist;
+  a.list_stride = L.union_stride;
+  a.list_has_count = 1;
+  a.expanded = expanded;
+  a.nc = nb;
+  a.list_len = L.plan.list_len;
+  a.num_ctas = L.plan.num_ctas;
+  a.max_slots = L.plan.max_slots;
+  a.softmax_scale = softmax_scale;
+  a.partial = reinterpret_cast<float*>(ws + L.partial);
+  a.status = status;
+  if (e == cudaSuccess) e = launch_attn_decode_bf16(&mq, &mk, &mv, &mk, &mv, a, cs);
+  if (e == cudaSuccess) e = launch_decode_combine(a.partial, a, s->d, true, o, lse, cs);
+  return cuda_status(e);
+}
+
+bsa_status_t bsa_sparse_attn_decode_paged(const bsa_shape_t* s, const void* q, const void* k_pool, const void* v_pool,
+                                          int num_pages, const int* block_table, int table_stride, const int* idx,
+                                          int idx_stride, float softmax_scale, void* workspace,
+                                          size_t workspace_bytes, void* o, float* lse, void* stream) {
+  bsa_status_t st = decode_checks(s, q, k_pool, v_pool, o);
+  if (st != BSA_OK) return st;
+  const int nb = s->Nk / s->block;
+  if (!block_table || num_pages < 1 || table_stride < nb) return BSA_ERR_INVALID_ARG;
+  if (!idx || idx_stride < 1 || !(softmax_scale > 0.0f) || !workspace) return BSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return BSA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(num_pages) * s->Hkv * s->block >= (1ll << 31)) return BSA_ERR_UNSUPPORTED;
+  uint32_t* status = nullptr;
+  int sms = 0;
+  if ((st = device_state(&status, &sms)) != BSA_OK) return st;
+  const int G = s->Hq / s->Hkv;
+  const DecodePlan P = decode_plan(s->B * s->Hkv, idx_stride, sms);
+  const size_t need = align256(static_cast<size_t>(s->B) * s->Hq * P.max_slots * (s->d + 4) * sizeof(float));
+  if (workspace_bytes < need) return BSA_ERR_INVALID_ARG;
+  const uint64_t pool_rows = static_cast<uint64_t>(num_pages) * s->Hkv * s->block;
+  CUtensorMap mq, mk, mv;
+  if (!make_map_bf16(&mq, q, static_cast<uint64_t>(s->B) * s->Hq, static_cast<uint32_t>(G)) ||
+      !make_map_bf16(&mk, k_pool, pool_rows, 64) || !make_map_bf16(&mv, v_pool, pool_rows, 64))
+    return BSA_ERR_CUDA;
+  DecodeArgs a;
+  a.B = s->B;
+  a.Hq = s->Hq;
+  a.Hkv = s->Hkv;
+  a.Nk = s->Nk;
+  a.bs = s->block;
+  a.list = idx;
+  a.list_stride = idx_stride;
+  a.list_has_count = 0;
+  a.expanded = nullptr;
+  a.nc = 0;
+  a.list_len = P.list_len;
+  a.num_ctas = P.num_ctas;
+  a.max_slots = P.max_slots;
+  a.softmax_scale = softmax_scale;
+  a.partial = static_cast<float*>(workspace);
+  a.status = status;
+  a.table = block_table;
+  a.table_stride = table_stride;
+  a.num_pages = num_pages;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_attn_decode_bf16(&mq, &mk, &mv, nullptr, nullptr, a, cs);
+  if (e == cudaSuccess) e = launch_decode_combine(a.partial, a, s->d, true, o, lse, cs);
+  return cuda_status(e);
+}
+
+bsa_status_t bsa_paged_append(const bsa_shape_t* s, const void* k_new, const void* v_new, const int* seq_lens,
+                              const int* block_table, int table_stride, int num_pages, void* k_pool, void* v_pool,
+                              float* pooled_k, void* stream) {
+  bsa_status_t st = check_shape(s);
+  if (st != BSA_OK) return st;
+  if (!k_new || !v_new || !seq_lens || !block_table || !k_pool || !v_pool) return BSA_ERR_INVALID_ARG;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_pool) || !aligned16(v_pool)) return BSA_ERR_INVALID_ARG;
+  if (pooled_k && !aligned16(pooled_k)) return BSA_ERR_INVALID_ARG;
+  if (table_stride < 1 || num_pages < 1) return BSA_ERR_INVALID_ARG;
+  if (s->dtype != BSA_BF16 || s->block != 64 || s->d % 8 != 0 || s->d > 1024) return BSA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(num_pages) * s->Hkv * s->block * s->d >= (1ll << 40)) return BSA_ERR_UNSUPPORTED;
+  uint32_t* status = nullptr;
+  if ((st = device_state(&status, nullptr)) != BSA_OK) return st;
+  return cuda_status(launch_paged_append(k_new, v_new, s->B, s->Hkv, s->Nq, s->d, seq_lens, block_table,
+                                         table_stride, num_pages, k_pool, v_pool, pooled_k, status,
+                                         static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -105,6 +105,10 @@ struct Params {
   float scale_log2;
   float* partial;
   uint32_t* status;
+  // paged cache (plain decode only): logical block j of sequence b lives in
+  // physical block table[b * table_stride + j] of the pools [P][Hkv][64][d]
+  const int* table;
+  int table_stride, num_pages;
 };
 
 // The split space is every group row's list positions laid end to end; CTA c
@@ -403,11 +407,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int base = a; base < stop; base += 32) {
         const int t = base + lane;
         const int v = (t < stop) ? src[t] : 0;
-        const bool bad = (t < stop) && (gist ? (v >= nb_cache || v < -ngist) : (v < 0 || v >= nb_cache));
+        bool bad = (t < stop) && (gist ? (v >= nb_cache || v < -ngist) : (v < 0 || v >= nb_cache));
+        int tile = v;
+        if (p.table != nullptr && t < stop && !bad) {
+          // paged cache: the kept logical block's physical block
+          tile = __ldg(p.table + static_cast<int64_t>(bg / p.Hkv) * p.table_stride + v);
+          bad = tile < 0 || tile >= p.num_pages;
+        }
         if (bad) atomicOr(p.status, BSA_DEV_BAD_INDEX);
         const bool keep = (t < stop) && !bad && (w + (t - base) < kMaxItemTiles);
         const unsigned km = __ballot_sync(0xffffffffu, keep);
-        if (keep) inf->tiles[w + __popc(km & lt)] = v;
+        if (keep) inf->tiles[w + __popc(km & lt)] = tile;
         w += __popc(km);
       }
       if (lane == 0) {
@@ -457,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int y;
                 if (tile >= 0) {
                   map = kv ? &tmV : &tmK;
-                  y = inf->bg * p.Nk + tile * 64;
+                  y = (p.table != nullptr) ? (tile * p.Hkv + inf->g) * 64 : inf->bg * p.Nk + tile * 64;
                 } else {
                   map = kv ? &tmGV : &tmGK;
                   y = inf->bg * p.nc + (-(tile + 1)) * 64;
@@ -639,10 +649,12 @@ __global__ void combine_kernel(const float* __restrict__ partial, int rows, int 
 }
 
 // Gist: per (b, g) build each head's expanded-chunk bitmap and the ascending
-// union of expanded chunks followed by every gist block (-(gb+1)).
+// union of expanded chunks followed by every gist block (-(gb+1)) when
+// with_gists is set.  Without gists (per-head decode, where chunk = block)
+// the union lists only the heads' kept blocks.
 __global__ void gist_union_kernel(const int* __restrict__ idx, int Hq, int Hkv, int topk, int idx_stride, int nc,
                                   uint32_t* __restrict__ expanded, int* __restrict__ union_list, int union_stride,
-                                  uint32_t* __restrict__ status) {
+                                  int with_gists, uint32_t* __restrict__ status) {
   griddep_wait();
   extern __shared__ uint32_t sbits[];   // [G+1][nc/32]; row G = union
   const int G = Hq / Hkv;
@@ -689,7 +701,7 @@ __global__ void gist_union_kernel(const int* __restrict__ idx, int Hq, int Hkv, 
       }
       run += __shfl_sync(0xffffffffu, incl, 31);
     }
-    const int ngb = nc / 64;
+    const int ngb = with_gists ? nc / 64 : 0;
     for (int t = lane; t < ngb; t += 32) out[1 + run + t] = -(t + 1);
     if (lane == 0) out[0] = run + ngb;
   }
@@ -720,6 +732,9 @@ cudaError_t launch_attn_decode_bf16(const CUtensorMap* tmQ, const CUtensorMap* t
   p.scale_log2 = a.softmax_scale * decode::kLog2e;
   p.partial = a.partial;
   p.status = a.status;
+  p.table = a.table;
+  p.table_stride = a.table_stride;
+  p.num_pages = a.num_pages;
   const int grid = a.num_ctas;
   return launch_dependent(decode::attn_decode_kernel, dim3(grid), dim3(decode::kThreads), decode::kSmemBytes, st, *tmQ,
                           *tmK, *tmV, tmGK ? *tmGK : *tmK, tmGV ? *tmGV : *tmV, p);
@@ -747,12 +762,12 @@ int decode_slots_for(int rows, int list_len, int num_ctas) {
 }
 
 cudaError_t launch_gist_union(const int* idx, int B, int Hq, int Hkv, int topk, int idx_stride, int nc,
-                              uint32_t* expanded, int* union_list, int union_stride, uint32_t* status,
-                              cudaStream_t st) {
+                              uint32_t* expanded, int* union_list, int union_stride, bool with_gists,
+                              uint32_t* status, cudaStream_t st) {
   const int G = Hq / Hkv;
   const size_t smem = static_cast<size_t>(G + 1) * (nc / 32) * sizeof(uint32_t);
   return launch_dependent(decode::gist_union_kernel, dim3(B * Hkv), dim3(256), smem, st, idx, Hq, Hkv, topk, idx_stride,
-                          nc, expanded, union_list, union_stride, status);
+                          nc, expanded, union_list, union_stride, with_gists ? 1 : 0, status);
 }
 
 }  // namespace bsa

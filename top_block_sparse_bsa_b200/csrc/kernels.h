@@ -77,6 +77,12 @@ cudaError_t launch_score_gist(const void* q, const void* gk, bool bf16, int B, i
                               int d, float scale, float* s, cudaStream_t st);
 cudaError_t launch_topk(const float* scores, int rows, int ncols, int mode, int kb, int* idx_out,
                         int idx_stride, int* count_out, cudaStream_t st);
+cudaError_t launch_topk_pattern(const float* scores, int rows, int ncols, int sink, int local, int kb, int* idx_out,
+                                int idx_stride, int* count_out, cudaStream_t st);
+cudaError_t launch_score_heads(const void* q, bool bf16, const float* kbar, int B, int Hq, int Hkv, int nb, int d,
+                               float scale, float* s, cudaStream_t st);
+cudaError_t launch_topk_joint(const float* scores, int rows, int G, int nb, int kb_total, int* idx_out,
+                              int idx_stride, int* count_out, cudaStream_t st);
 // decode scores + top-k in one kernel (tmKbar: fp32 [rows, 128], box 32 x 128, 128-byte swizzle)
 bool decode_select_fused_ok(int d, int nb);
 cudaError_t launch_decode_select(const CUtensorMap* tmKbar, const void* q, bool bf16, int B, int Hq, int Hkv,
@@ -106,6 +112,11 @@ cudaError_t launch_attn_prefill_split_bf16(const CUtensorMap* tmQ, const CUtenso
 cudaError_t launch_attn_prefill_pair_bf16(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
                                           const PrefillArgs& a, cudaStream_t st);
 
+// paged.cu (paged cache upkeep)
+cudaError_t launch_paged_append(const void* k_new, const void* v_new, int B, int Hkv, int T, int d,
+                                const int* seq_lens, const int* table, int table_stride, int num_pages, void* k_pool,
+                                void* v_pool, float* pooled_k, uint32_t* status, cudaStream_t st);
+
 // attn_f32.cu (fp32 SIMT path)
 cudaError_t launch_attn_prefill_f32(const float* q, const float* k, const float* v, const PrefillArgs& a,
                                     int d, cudaStream_t st);
@@ -126,6 +137,10 @@ struct DecodeArgs {
   float softmax_scale;
   float* partial;            // [B*Hq][max_slots][d+4]
   uint32_t* status;
+  // paged cache (plain decode): logical block j of sequence b is physical block
+  // table[b*table_stride + j] of pools [num_pages][Hkv][64][d]; null: contiguous
+  const int* table = nullptr;
+  int table_stride = 0, num_pages = 0;
 };
 cudaError_t launch_attn_decode_bf16(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
                                     const CUtensorMap* tmGK, const CUtensorMap* tmGV, const DecodeArgs& a,
@@ -134,7 +149,7 @@ cudaError_t launch_decode_combine(const float* partial, const DecodeArgs& a, int
                                   float* lse, cudaStream_t st);
 int decode_slots_for(int rows, int list_len, int num_ctas);
 cudaError_t launch_gist_union(const int* idx, int B, int Hq, int Hkv, int topk, int idx_stride, int nc,
-                              uint32_t* expanded, int* union_list, int union_stride, uint32_t* status,
-                              cudaStream_t st);
+                              uint32_t* expanded, int* union_list, int union_stride, bool with_gists,
+                              uint32_t* status, cudaStream_t st);
 
 }  // namespace bsa

@@ -937,6 +937,184 @@ cudaError_t launch_decode_select(const CUtensorMap* tmKbar, const void* q, bool 
                           count_out, status);
 }
 
+// ------------------------------------------- fixed pattern + dynamic blocks
+// Prefill selection with a fixed part (Sparse Frontier review §2.2.3,
+// MInference block-sparse: the first blocks of the sequence, the local window,
+// and a set of dynamically selected blocks per query block).  Row r is query
+// block i = r % ncols.  Kept: the first `sink` blocks, the `local` most recent
+// blocks (i included) and the kb best of the blocks between them.  The three
+// sets are disjoint ranges in block order, [0, P) | candidates [P, S) | [S, i],
+// so the list is written already ascending.  One CTA per row.
+template <int KPT>
+__global__ void __launch_bounds__(256) topk_pattern_kernel(const float* __restrict__ scores, int ncols, int sink,
+                                                           int local, int kb, int* __restrict__ idx_out,
+                                                           int idx_stride, int* __restrict__ count_out) {
+  griddep_wait();   // the scores come from the kernel launched before
+  __shared__ int s_nsel;
+  const int tid = threadIdx.x;
+  const int64_t r = blockIdx.x;
+  const int i = static_cast<int>(r % ncols);
+  const int P = min(sink, i + 1);
+  const int S = max(P, i - local + 1);
+  const int ncand = S - P;
+  int* out = idx_out + r * idx_stride;
+  const float* srow = scores + r * ncols + P;
+  uint32_t key[KPT];
+#pragma unroll
+  for (int e = 0; e < KPT; ++e) key[e] = (tid * KPT + e < ncand) ? order_key(__ldg(srow + tid * KPT + e)) : 0u;
+  for (int t = tid; t < P; t += 256) out[t] = t;
+  cta_topk_select<KPT>(key, ncand, kb, -1, out + P, idx_stride - P, &s_nsel, P);
+  __syncthreads();
+  const int n0 = P + s_nsel;
+  for (int t = tid; t <= i - S; t += 256) out[n0 + t] = S + t;
+  if (tid == 0 && count_out) count_out[r] = n0 + (i + 1 - S);
+}
+
+cudaError_t launch_topk_pattern(const float* scores, int rows, int ncols, int sink, int local, int kb, int* idx_out,
+                                int idx_stride, int* count_out, cudaStream_t st) {
+  if (ncols <= 256 * 8)
+    return launch_dependent(topk_pattern_kernel<8>, dim3(rows), dim3(256), 0, st, scores, ncols, sink, local, kb,
+                            idx_out, idx_stride, count_out);
+  return launch_dependent(topk_pattern_kernel<32>, dim3(rows), dim3(256), 0, st, scores, ncols, sink, local, kb,
+                          idx_out, idx_stride, count_out);
+}
+
+// --------------------------------------------- per-head decode scores
+// Each query head's decode scores against the pooled-key summary,
+// s[b][h][j] = q_h . kbar_{g,j} / sqrt(d) in the fixed order (channels
+// ascending, products and sums rounded separately) -- the per-head scores
+// that a budget shared across the heads (Ada-KV) ranks.  Grid (tiles of 128
+// blocks, B*Hkv); thread = block row; the CTA's pooled rows are staged as in
+// score_decode_kernel, the G query rows as floats.
+template <typename T, int D>
+__global__ void __launch_bounds__(128) score_heads_kernel(const T* __restrict__ q, const float* __restrict__ kbar,
+                                                          int Hq, int Hkv, int nb, float scale,
+                                                          float* __restrict__ s) {
+  constexpr int kPitch = D + 4;
+  constexpr int kChunks = D / 4;
+  extern __shared__ __align__(16) float sm_heads[];
+  float* ks = sm_heads;                  // [128][kPitch]
+  float* qs = sm_heads + 128 * kPitch;   // [G][D]
+  const int64_t bg = blockIdx.y;
+  const int64_t b = bg / Hkv, g = bg % Hkv;
+  const int G = Hq / Hkv;
+  const int j0 = blockIdx.x * 128;
+  const int rows = min(128, nb - j0);
+  const float* src = kbar + (bg * nb + j0) * D;
+  for (int e = threadIdx.x; e < rows * kChunks; e += 128) {
+    const int r = e / kChunks, c = e % kChunks;
+    cp_async16(smem_u32(ks + r * kPitch + 4 * c), src + static_cast<int64_t>(r) * D + 4 * c);
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  for (int e = threadIdx.x; e < G * D; e += 128) qs[e] = static_cast<float>(q[(b * Hq + g * G) * D + e]);
+  cp_async_wait_all();
+  __syncthreads();
+  const int r = threadIdx.x;
+  if (r >= rows) return;
+  const float4* row = reinterpret_cast<const float4*>(ks + r * kPitch);
+  for (int hh = 0; hh < G; ++hh) {
+    const float* qr = qs + hh * D;
+    float acc = 0.0f;
+#pragma unroll
+    for (int e = 0; e < kChunks; ++e) {
+      const float4 kv = row[e];
+      acc = __fadd_rn(acc, __fmul_rn(qr[4 * e + 0], kv.x));
+      acc = __fadd_rn(acc, __fmul_rn(qr[4 * e + 1], kv.y));
+      acc = __fadd_rn(acc, __fmul_rn(qr[4 * e + 2], kv.z));
+      acc = __fadd_rn(acc, __fmul_rn(qr[4 * e + 3], kv.w));
+    }
+    s[((b * Hq + g * G + hh) * nb) + j0 + r] = __fmul_rn(acc, scale);
+  }
+}
+
+template <typename T, int D>
+static cudaError_t launch_score_heads_d(dim3 grid, int G, const void* q, const float* kbar, int Hq, int Hkv, int nb,
+                                        float scale, float* s, cudaStream_t st) {
+  const size_t smem = (128 * (D + 4) + G * D) * sizeof(float);
+  cudaError_t e = ensure_dynamic_smem<score_heads_kernel<T, D>>(smem);
+  if (e != cudaSuccess) return e;
+  score_heads_kernel<T, D><<<grid, 128, smem, st>>>(static_cast<const T*>(q), kbar, Hq, Hkv, nb, scale, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_score_heads(const void* q, bool bf16, const float* kbar, int B, int Hq, int Hkv, int nb, int d,
+                               float scale, float* s, cudaStream_t st) {
+  const dim3 grid((nb + 127) / 128, B * Hkv);
+  const int G = Hq / Hkv;
+  if (d == 128)
+    return bf16 ? launch_score_heads_d<__nv_bfloat16, 128>(grid, G, q, kbar, Hq, Hkv, nb, scale, s, st)
+                : launch_score_heads_d<float, 128>(grid, G, q, kbar, Hq, Hkv, nb, scale, s, st);
+  if (d == 64)
+    return bf16 ? launch_score_heads_d<__nv_bfloat16, 64>(grid, G, q, kbar, Hq, Hkv, nb, scale, s, st)
+                : launch_score_heads_d<float, 64>(grid, G, q, kbar, Hq, Hkv, nb, scale, s, st);
+  return cudaErrorInvalidValue;
+}
+
+// ------------------------------------------ one budget across a group's heads
+// Ada-KV (Sparse Frontier review §2.3.2): the group's G heads share one
+// budget of kb_total (head, block) pairs, so an important head keeps more
+// blocks and others fewer.  One CTA per (batch, KV group) row; candidate
+// c = h*(nb-1) + j (j < nb-1: the last block is kept by every head) has the
+// score s[b][g*G+h][j].  The CTA select takes the best kb_total candidates
+// (equal scores: lower c first) and writes them ascending in c into shared
+// memory, i.e. head by head with blocks ascending; each head's run then
+// becomes its kept list, the last block appended.
+template <int KPT>
+__global__ void __launch_bounds__(256) topk_joint_kernel(const float* __restrict__ scores, int G, int nb,
+                                                         int kb_total, int* __restrict__ idx_out, int idx_stride,
+                                                         int* __restrict__ count_out) {
+  griddep_wait();
+  extern __shared__ int sl_joint[];   // [min(kb_total, G*(nb-1))]
+  __shared__ int s_n;
+  __shared__ int s_cnt[16], s_start[16];
+  const int tid = threadIdx.x;
+  const int64_t bg = blockIdx.x;
+  const int per = nb - 1, ncand = G * per;
+  const float* sbase = scores + bg * G * nb;
+  uint32_t key[KPT];
+#pragma unroll
+  for (int e = 0; e < KPT; ++e) {
+    const int c = tid * KPT + e;
+    key[e] = (c < ncand) ? order_key(__ldg(sbase + (c / per) * nb + c % per)) : 0u;
+  }
+  if (tid < 16) s_cnt[tid] = 0;
+  const int cap = min(kb_total, ncand);
+  cta_topk_select<KPT>(key, ncand, kb_total, -1, sl_joint, cap, &s_n);
+  __syncthreads();
+  const int n = s_n;
+  for (int t = tid; t < n; t += 256) atomicAdd(&s_cnt[sl_joint[t] / per], 1);
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int h = 0; h < G; ++h) {
+      s_start[h] = run;
+      run += s_cnt[h];
+    }
+  }
+  __syncthreads();
+  for (int t = tid; t < n; t += 256) {
+    const int c = sl_joint[t], h = c / per;
+    idx_out[(bg * G + h) * idx_stride + (t - s_start[h])] = c % per;
+  }
+  for (int e = tid; e < G * idx_stride; e += 256) {
+    const int h = e / idx_stride, t = e % idx_stride;
+    if (t == s_cnt[h]) idx_out[(bg * G + h) * idx_stride + t] = nb - 1;
+    else if (t > s_cnt[h]) idx_out[(bg * G + h) * idx_stride + t] = -1;
+  }
+  if (count_out && tid < G) count_out[bg * G + tid] = s_cnt[tid] + 1;
+}
+
+cudaError_t launch_topk_joint(const float* scores, int rows, int G, int nb, int kb_total, int* idx_out,
+                              int idx_stride, int* count_out, cudaStream_t st) {
+  const int ncand = G * (nb - 1);
+  const size_t smem = static_cast<size_t>(max(1, min(kb_total, ncand))) * sizeof(int);
+  if (ncand <= 256 * 8)
+    return launch_dependent(topk_joint_kernel<8>, dim3(rows), dim3(256), smem, st, scores, G, nb, kb_total, idx_out,
+                            idx_stride, count_out);
+  return launch_dependent(topk_joint_kernel<32>, dim3(rows), dim3(256), smem, st, scores, G, nb, kb_total, idx_out,
+                          idx_stride, count_out);
+}
+
 cudaError_t launch_topk(const float* scores, int rows, int ncols, int mode, int kb, int* idx_out,
                         int idx_stride, int* count_out, cudaStream_t st) {
   if (ncols <= 32 * 16) {

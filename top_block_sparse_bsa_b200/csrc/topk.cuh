@@ -20,10 +20,12 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 // topk_cta_kernel in selector.cu):
 // thread t holds the keys of candidates t*KPT .. t*KPT+KPT-1 (key 0 past
 // ncand); writes the kept list (ascending, forced block last, -1 after it)
-// to out and its length to *count_out (optional).
+// to out and its length to *count_out (optional).  Candidate t is written as
+// index_base + t.
 template <int KPT>
 __device__ __forceinline__ void cta_topk_select(const uint32_t (&key)[KPT], int ncand, int kb, int forced,
-                                                int* __restrict__ out, int idx_stride, int* __restrict__ count_out) {
+                                                int* __restrict__ out, int idx_stride, int* __restrict__ count_out,
+                                                int index_base = 0) {
   __shared__ int hist[256];
   __shared__ uint32_t wsum[8];
   __shared__ int sel_digit, sel_above;
@@ -121,7 +123,7 @@ __device__ __forceinline__ void cta_topk_select(const uint32_t (&key)[KPT], int 
     const bool valid = j0 + e < ncand;
     const bool gt = take_all ? valid : (take > 0 && valid && key[e] > thresh);
     const bool tie = !take_all && take > 0 && valid && key[e] == thresh;
-    if (gt || (tie && tie_before < remaining)) out[gt_before + min(tie_before, remaining)] = j0 + e;
+    if (gt || (tie && tie_before < remaining)) out[gt_before + min(tie_before, remaining)] = index_base + j0 + e;
     gt_before += gt ? 1 : 0;
     tie_before += tie ? 1 : 0;
   }
