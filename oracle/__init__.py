@@ -80,6 +80,9 @@ def _declare(L):
         "oracle_attend_decode_heads_rows": [_p, _p, _p, _i64, _i64, _i64, _i64, _i64, _i64, _p, _i64,
                                             ctypes.c_double, _p, _i64, _p, _p],
         "oracle_paged_gather": [_p, _p, _i64, _i64, _i64, _i64, _i64, _i64, _p],
+        "oracle_hssa_select": [_p, _p, _p, _i64, _i64, _i64, _i64, _i64, _i64, _i64, _i64, _p, _i64, _p, _i64],
+        "oracle_attend_hssa_rows": [_p, _p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _i64, _i64, _i64, _p, _i64,
+                                    _p, _i64, ctypes.c_double, _p, _i64, _p, _p],
         "oracle_max_threads": [],
         "oracle_set_threads": [ctypes.c_int],
     }
@@ -372,3 +375,41 @@ def paged_gather(pool, table, nb: int) -> np.ndarray:
     out = np.empty((B, Hkv, nb * bs, d), np.float32)
     lib().oracle_paged_gather(_ptr(pool), _ptr(table), B, Hkv, nb, bs, d, max_blocks, _ptr(out))
     return out
+
+
+# ----------------------------------------------------------------------------
+# 10. two-level gist routing (H-SSA)
+# ----------------------------------------------------------------------------
+
+def hssa_select(q, gk, mk, M: int, km: int, k: int):
+    """Meta-gist then gist selection per query head (SSA page, H-SSA).
+    q [B,Hq,d], gk [B,Hkv,nc,d], mk [B,Hkv,nc/M,d] -> (meta_idx [B,Hq,km],
+    chunk_idx [B,Hq,k]), ascending, -1 padded."""
+    q, gk, mk = _f32(q), _f32(gk), _f32(mk)
+    B, Hq, d = q.shape
+    Hkv, nc = gk.shape[1], gk.shape[2]
+    meta = np.empty((B, Hq, max(km, 1)), np.int32)
+    chunks = np.empty((B, Hq, max(k, 1)), np.int32)
+    lib().oracle_hssa_select(_ptr(q), _ptr(gk), _ptr(mk), B, Hq, Hkv, nc, M, d, km, k,
+                             _ptr(meta), meta.shape[-1], _ptr(chunks), chunks.shape[-1])
+    return meta, chunks
+
+
+def attend_hssa(q, k, v, gk, gv, mk, mv, chunk: int, M: int, meta_idx, chunk_idx,
+                scale: Optional[float] = None, rows=None) -> Tuple[np.ndarray, np.ndarray]:
+    """H-SSA decode attention (fp64): expanded chunks' tokens, gists of the
+    other chunks of kept groups, meta-gists of groups not kept."""
+    q, k, v, gk, gv, mk, mv = (_f32(x) for x in (q, k, v, gk, gv, mk, mv))
+    meta_idx, chunk_idx = _i32(meta_idx), _i32(chunk_idx)
+    B, Hq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    r = _rows_arg(rows, B * Hq)
+    out = np.empty((len(r), d), np.float64)
+    lse = np.empty((len(r),), np.float64)
+    lib().oracle_attend_hssa_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(gk), _ptr(gv), _ptr(mk), _ptr(mv),
+                                  B, Hq, Hkv, Nk, d, chunk, M, _ptr(meta_idx), meta_idx.shape[-1],
+                                  _ptr(chunk_idx), chunk_idx.shape[-1], float(scale), _ptr(r), len(r),
+                                  _ptr(out), _ptr(lse))
+    return out, lse

@@ -605,6 +605,112 @@ void oracle_paged_gather(const float* pool, const int32_t* table, int64_t B, int
     }
 }
 
+/* ------------------------------------------------------------------------ */
+/* 10. Two-level gist routing (H-SSA)                                       */
+/* ------------------------------------------------------------------------ */
+
+/* SSA page, 层级扩展 H-SSA: meta-gist tokens ("gist-of-gist", one per group of
+ * M consecutive chunks) make a coarse selection first; then, inside the
+ * selected groups, the ordinary gists score the chunks finely and the best
+ * are expanded.  Per query head h of row b:
+ *   meta  -- score q_h against the nm = nc/M meta-gist keys (step 2's fixed
+ *            order), keep the km best groups (step 3's order, nothing forced);
+ *   fine  -- score q_h against the gists of the chunks in the kept groups,
+ *            keep the k best of those chunks.
+ * mk [B,Hkv,nm,d], gk [B,Hkv,nc,d].  meta_idx [B,Hq,km_stride] and chunk_idx
+ * [B,Hq,k_stride]: ascending, -1 padded. */
+void oracle_hssa_select(const float* q, const float* gk, const float* mk, int64_t B, int64_t Hq, int64_t Hkv,
+                        int64_t nc, int64_t M, int64_t d, int64_t km, int64_t k, int32_t* meta_idx,
+                        int64_t km_stride, int32_t* chunk_idx, int64_t k_stride)
+{
+    const int64_t nm = nc / M, G = Hq / Hkv;
+    const float scale = score_scale(d);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < B * Hq; ++r) {
+        const int64_t b = r / Hq, h = r % Hq, g = h / G;
+        const float* qr = q + r * d;
+        cand_t* c = (cand_t*)malloc(sizeof(cand_t) * (size_t)(nc > nm ? nc : nm));
+        for (int64_t m = 0; m < nm; ++m) {
+            c[m].s = score_dot(qr, mk + ((b * Hkv + g) * nm + m) * d, d, scale);
+            c[m].j = (int32_t)m;
+        }
+        qsort(c, (size_t)nm, sizeof(cand_t), cand_cmp);
+        const int64_t tm = (km < nm) ? km : nm;
+        int32_t* mo = meta_idx + r * km_stride;
+        for (int64_t t = 0; t < tm; ++t) mo[t] = c[t].j;
+        qsort(mo, (size_t)tm, sizeof(int32_t), int_cmp);
+        for (int64_t t = tm; t < km_stride; ++t) mo[t] = -1;
+        int64_t n = 0;
+        for (int64_t t = 0; t < tm; ++t)
+            for (int64_t x = 0; x < M; ++x) {
+                const int64_t ch = (int64_t)mo[t] * M + x;
+                c[n].s = score_dot(qr, gk + ((b * Hkv + g) * nc + ch) * d, d, scale);
+                c[n].j = (int32_t)ch;
+                ++n;
+            }
+        qsort(c, (size_t)n, sizeof(cand_t), cand_cmp);
+        const int64_t tk = (k < n) ? k : n;
+        int32_t* co = chunk_idx + r * k_stride;
+        for (int64_t t = 0; t < tk; ++t) co[t] = c[t].j;
+        qsort(co, (size_t)tk, sizeof(int32_t), int_cmp);
+        for (int64_t t = tk; t < k_stride; ++t) co[t] = -1;
+        free(c);
+    }
+}
+
+/* H-SSA rows.  Keys of query head h (the reading of the page's coarse-to-
+ * fine routing, as SSA's mixed attention one level up): every token of an
+ * expanded chunk; the gist of every other chunk inside a kept group; the
+ * meta-gist of every group not kept.  rows[n] = b*Hq + h. */
+void oracle_attend_hssa_rows(const float* q, const float* k, const float* v, const float* gk, const float* gv,
+                             const float* mk, const float* mv, int64_t B, int64_t Hq, int64_t Hkv, int64_t Nk,
+                             int64_t d, int64_t chunk, int64_t M, const int32_t* meta_idx, int64_t km_stride,
+                             const int32_t* chunk_idx, int64_t k_stride, double scale, const int64_t* rows,
+                             int64_t nrows, double* out, double* lse)
+{
+    const int64_t nc = Nk / chunk, nm = nc / M, G = Hq / Hkv;
+    (void)B;
+#pragma omp parallel
+    {
+        unsigned char* kept = (unsigned char*)malloc((size_t)nm);
+        unsigned char* exp_ = (unsigned char*)malloc((size_t)nc);
+        double* logits = (double*)malloc(sizeof(double) * (size_t)(Nk + nc + nm));
+        const float** vals = (const float**)malloc(sizeof(float*) * (size_t)(Nk + nc + nm));
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t n = 0; n < nrows; ++n) {
+            const int64_t r = rows[n];
+            const int64_t b = r / Hq, g = (r % Hq) / G;
+            mark_blocks(meta_idx + r * km_stride, km_stride, nm, kept);
+            mark_blocks(chunk_idx + r * k_stride, k_stride, nc, exp_);
+            const int64_t bg = b * Hkv + g;
+            int64_t m = 0;
+            for (int64_t gr = 0; gr < nm; ++gr) {
+                if (!kept[gr]) {
+                    logits[m] = dot64(q + r * d, mk + (bg * nm + gr) * d, d) * scale;
+                    vals[m] = mv + (bg * nm + gr) * d;
+                    ++m;
+                    continue;
+                }
+                for (int64_t c = gr * M; c < (gr + 1) * M; ++c) {
+                    if (exp_[c]) {
+                        for (int64_t u = c * chunk; u < (c + 1) * chunk; ++u) {
+                            logits[m] = dot64(q + r * d, k + (bg * Nk + u) * d, d) * scale;
+                            vals[m] = v + (bg * Nk + u) * d;
+                            ++m;
+                        }
+                    } else {
+                        logits[m] = dot64(q + r * d, gk + (bg * nc + c) * d, d) * scale;
+                        vals[m] = gv + (bg * nc + c) * d;
+                        ++m;
+                    }
+                }
+            }
+            softmax_rows(logits, vals, m, d, out + n * d, lse + n);
+        }
+        free(kept); free(exp_); free(logits); free(vals);
+    }
+}
+
 int oracle_max_threads(void)
 {
 #ifdef _OPENMP

@@ -621,3 +621,108 @@ def test_paged_gather_permuted_pages():
         for j in range(nb):
             for g in range(Hkv):
                 assert np.array_equal(out[b, g, j * bs:(j + 1) * bs], pool[table[b, j], g])
+
+
+# ----------------------------------------------------------------------------
+# two-level gist routing (H-SSA)
+# ----------------------------------------------------------------------------
+
+def _small_hssa(seed, B=2, Hq=4, Hkv=2, Nk=512, d=16, chunk=16, M=4):
+    r = _rng(seed)
+    nc = Nk // chunk
+    q = r.standard_normal((B, Hq, d)).astype(np.float32)
+    k = r.standard_normal((B, Hkv, Nk, d)).astype(np.float32)
+    v = r.standard_normal((B, Hkv, Nk, d)).astype(np.float32)
+    gk = r.standard_normal((B, Hkv, nc, d)).astype(np.float32)
+    gv = r.standard_normal((B, Hkv, nc, d)).astype(np.float32)
+    mk = r.standard_normal((B, Hkv, nc // M, d)).astype(np.float32)
+    mv = r.standard_normal((B, Hkv, nc // M, d)).astype(np.float32)
+    return q, k, v, gk, gv, mk, mv
+
+
+def test_hssa_with_every_group_kept_is_ssa():
+    """Keeping every group, the fine step scores every gist: H-SSA's choice
+    and attention are SSA's (SSA page, 推理时的关键模块)."""
+    q, k, v, gk, gv, mk, mv = _small_hssa(90)
+    chunk, M, kk = 16, 4, 5
+    nm = gk.shape[2] // M
+    meta, chunks = oracle.hssa_select(q, gk, mk, M, nm, kk)
+    assert np.array_equal(meta, np.broadcast_to(np.arange(nm, dtype=np.int32), meta.shape))
+    _, idx, _ = oracle.gist_select(q, gk, kk)
+    assert np.array_equal(chunks, idx)
+    a, la = oracle.attend_hssa(q, k, v, gk, gv, mk, mv, chunk, M, meta, chunks)
+    b, lb = oracle.attend_gist(q, k, v, gk, gv, chunk, idx)
+    assert np.allclose(a, b, atol=1e-12, rtol=0) and np.allclose(la, lb, atol=1e-12, rtol=0)
+
+
+def test_hssa_with_nothing_kept_attends_the_meta_gists():
+    q, k, v, gk, gv, mk, mv = _small_hssa(91)
+    B, Hq, d = q.shape
+    G = Hq // k.shape[1]
+    meta, chunks = oracle.hssa_select(q, gk, mk, 4, 0, 0)
+    assert np.all(meta == -1) and np.all(chunks == -1)
+    out, _ = oracle.attend_hssa(q, k, v, gk, gv, mk, mv, 16, 4, meta, chunks)
+    ref = _sdpa64(q[:, :, None, :], np.repeat(mk, G, 1), np.repeat(mv, G, 1))
+    assert np.allclose(out.reshape(B, Hq, d), ref[:, :, 0], atol=1e-10, rtol=0)
+
+
+def test_hssa_one_chunk_groups_expanding_every_kept_group():
+    """Groups of one chunk, every kept group expanded: the keys are the kept
+    chunks' tokens and the meta-gists of the rest, i.e. SSA with the
+    meta-gists as the gists and the meta selection as the expanded set."""
+    q, k, v, gk, gv, mk, mv = _small_hssa(92, M=1)
+    chunk, km = 16, 6
+    meta, chunks = oracle.hssa_select(q, gk, mk, 1, km, km)
+    assert np.array_equal(meta, chunks)
+    a, _ = oracle.attend_hssa(q, k, v, gk, gv, mk, mv, chunk, 1, meta, chunks)
+    b, _ = oracle.attend_gist(q, k, v, mk, mv, chunk, meta)
+    assert np.allclose(a, b, atol=1e-12, rtol=0)
+
+
+def test_hssa_selection_matches_bruteforce():
+    """Integer-valued queries and keys make every score exact, with many
+    ties: the two-level choice equals brute force over subsets."""
+    r = _rng(93)
+    for trial in range(20):
+        B, Hq, Hkv, d, M = 1, 2, 1, 4, 3
+        nc = 3 * M
+        km = int(r.integers(0, 4))
+        kk = int(r.integers(0, km * M + 2))
+        q = r.integers(-2, 3, (B, Hq, d)).astype(np.float32)
+        gk = r.integers(-2, 3, (B, Hkv, nc, d)).astype(np.float32)
+        mk = r.integers(-2, 3, (B, Hkv, nc // M, d)).astype(np.float32)
+        meta, chunks = oracle.hssa_select(q, gk, mk, M, km, kk)
+        for h in range(Hq):
+            ms = [float(np.dot(q[0, h], mk[0, 0, m])) for m in range(nc // M)]
+            want_m = sorted(_brute_topk(ms, list(range(nc // M)), km))
+            assert [int(x) for x in meta[0, h] if x >= 0] == want_m
+            cand = [c for m in want_m for c in range(m * M, (m + 1) * M)]
+            cs = {c: float(np.dot(q[0, h], gk[0, 0, c])) for c in cand}
+            want_c = sorted(_brute_topk([cs.get(c, 0.0) for c in range(nc)], cand, kk))
+            assert [int(x) for x in chunks[0, h] if x >= 0] == want_c, (trial, h)
+
+
+def test_hssa_attention_matches_library_on_explicit_key_set():
+    q, k, v, gk, gv, mk, mv = _small_hssa(94)
+    chunk, M, km, kk = 16, 4, 3, 4
+    B, Hq, d = q.shape
+    G = Hq // k.shape[1]
+    nc, nm = gk.shape[2], mk.shape[2]
+    meta, chunks = oracle.hssa_select(q, gk, mk, M, km, kk)
+    out, _ = oracle.attend_hssa(q, k, v, gk, gv, mk, mv, chunk, M, meta, chunks)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // G
+            keys, vals = [], []
+            kept = set(int(x) for x in meta[b, h] if x >= 0)
+            exp = set(int(x) for x in chunks[b, h] if x >= 0)
+            for m in range(nm):
+                if m not in kept:
+                    keys.append(mk[b, g, m]); vals.append(mv[b, g, m]); continue
+                for c in range(m * M, (m + 1) * M):
+                    if c in exp:
+                        keys.extend(k[b, g, c * chunk:(c + 1) * chunk]); vals.extend(v[b, g, c * chunk:(c + 1) * chunk])
+                    else:
+                        keys.append(gk[b, g, c]); vals.append(gv[b, g, c])
+            ref = _sdpa64(q[b, h][None, None], np.array(keys)[None], np.array(vals)[None])
+            assert np.allclose(out[b * Hq + h], ref[0, 0], atol=1e-10, rtol=0)
