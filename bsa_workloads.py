@@ -30,7 +30,7 @@ import torch
 @dataclasses.dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str            # "prefill", "gated", "decode", "gist"
+    kind: str            # "prefill", "gated", "decode", "gist", "hssa"
     B: int
     Hq: int
     Hkv: int
@@ -85,6 +85,15 @@ WORKLOADS: Dict[str, Workload] = {
         bs=64, kb=32, dtype="bf16", seed=4),
 }
 
+# Workloads of the widened path (not among the five above): the gist workload
+# with one meta-gist per 64 chunks, 4 groups kept per head, 32 chunks expanded.
+EXTRA_WORKLOADS: Dict[str, Workload] = {
+    "hssa_decode_bf16": Workload(
+        name="hssa_decode_bf16", kind="hssa", B=8, Hq=32, Hkv=8, N=131072, d=128,
+        bs=64, kb=32, dtype="bf16", seed=5),
+}
+HSSA_GROUPS_KEPT = 4
+
 
 def _randn(shape, gen: torch.Generator, device, dtype) -> torch.Tensor:
     return torch.randn(shape, generator=gen, device=device, dtype=torch.float32).to(dtype)
@@ -106,6 +115,7 @@ def make_inputs(w: Workload, device="cpu") -> Dict[str, torch.Tensor]:
     prefill / gated: q [B,Hq,N,d], k [B,Hkv,N,d], v [B,Hkv,N,d]
     decode:          q [B,Hq,d],   k [B,Hkv,N,d], v [B,Hkv,N,d]
     gist:            q [B,Hq,d],   k, v [B,Hkv,N,d], gk, gv [B,Hkv,N/bs,d]
+    hssa:            as gist, plus mk, mv [B,Hkv,N/bs/64,d]
     """
     device = torch.device(device)
     gen = torch.Generator(device=device)
@@ -144,17 +154,21 @@ def make_inputs(w: Workload, device="cpu") -> Dict[str, torch.Tensor]:
                     kb = k[b, g, blocks].to(torch.float32) + shift
                     k[b, g, blocks] = kb.to(dt)
         out["q"] = out["q"].to(dt)
-    elif w.kind == "gist":
+    elif w.kind in ("gist", "hssa"):
         nc = w.N // w.bs
         out["q"] = _randn((w.B, w.Hq, w.d), gen, device, dt)
         out["k"] = _randn_big((w.B, w.Hkv, w.N, w.d), gen, device, dt)
         out["v"] = _randn_big((w.B, w.Hkv, w.N, w.d), gen, device, dt)
         out["gk"] = _randn((w.B, w.Hkv, nc, w.d), gen, device, dt)
         out["gv"] = _randn((w.B, w.Hkv, nc, w.d), gen, device, dt)
+        if w.kind == "hssa":
+            # one meta-gist key/value per group of 64 chunks ("gist-of-gist")
+            out["mk"] = _randn((w.B, w.Hkv, nc // 64, w.d), gen, device, dt)
+            out["mv"] = _randn((w.B, w.Hkv, nc // 64, w.d), gen, device, dt)
     else:
         raise ValueError(f"unknown workload kind {w.kind!r}")
     return out
 
 
 def get(name: str) -> Workload:
-    return WORKLOADS[name]
+    return WORKLOADS[name] if name in WORKLOADS else EXTRA_WORKLOADS[name]

@@ -331,6 +331,35 @@ bsa_status_t bsa_paged_append(const bsa_shape_t* shape, const void* k_new, const
                               void* v_pool, float* pooled_k, void* stream);
 
 /*
+ * bsa_hssa_decode -- two-level gist routing (H-SSA) decode.
+ * Cite: SSA page, 层级扩展：H-SSA (meta-gist tokens, "gist-of-gist", make a
+ * coarse selection; inside the selected groups the ordinary gists score the
+ * chunks finely and the best are expanded) and 推理时的关键模块 1-3 (per-head
+ * selection under GQA; mixed attention over tokens and summaries).
+ * Groups are 64 consecutive chunks; meta_k/meta_v [B,Hkv,nm,d] hold one
+ * meta-gist per group, nm = nc/64 (nc = Nk/block chunks, gist_k/gist_v
+ * [B,Hkv,nc,d]).  Per query head: score the nm meta-gists, keep the km best
+ * groups; score the gists of the kept groups' chunks, expand the topk best
+ * chunks.  Keys of the head (a reading: SSA's mixed attention one level
+ * up): the tokens of its expanded chunks, the gists of the other chunks of
+ * its kept groups, the meta-gists of the groups it did not keep.
+ * Scores and order as bsa_score_blocks / bsa_topk_select (fixed-order fp32;
+ * larger first, ties to the lower index, nothing forced).
+ * meta_out [B,Hq,km] and idx_out [B,Hq,topk] int32 (optional): the kept
+ * groups and expanded chunks, ascending.  workspace:
+ * bsa_workspace_bytes_hssa(shape, km, topk) bytes, 256-byte aligned.
+ * Built: BF16, d = 128, block = 64, nc a multiple of 64 and at most 4096,
+ * 1 <= km <= nm, 0 <= topk <= 64*km, at most 16 query heads per KV group.
+ */
+bsa_status_t bsa_hssa_decode(const bsa_shape_t* shape, const void* q, const void* k_cache, const void* v_cache,
+                             const void* gist_k, const void* gist_v, const void* meta_k, const void* meta_v,
+                             int km, int topk, int* meta_out, int* idx_out, float softmax_scale,
+                             void* workspace, size_t workspace_bytes, void* o, float* lse, void* stream);
+
+/* Scratch bytes of bsa_hssa_decode; 0 on a bad shape. */
+size_t bsa_workspace_bytes_hssa(const bsa_shape_t* shape, int km, int topk);
+
+/*
  * bsa_sparse_attn_decode_noalloc -- bsa_sparse_attn_decode for callers that
  * cannot allocate device memory (no counterpart on the source pages; it is a
  * deployment convenience).  Some callers have no way to provide the decode

@@ -83,6 +83,8 @@ def _declare(L):
         "oracle_hssa_select": [_p, _p, _p, _i64, _i64, _i64, _i64, _i64, _i64, _i64, _i64, _p, _i64, _p, _i64],
         "oracle_attend_hssa_rows": [_p, _p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _i64, _i64, _i64, _p, _i64,
                                     _p, _i64, ctypes.c_double, _p, _i64, _p, _p],
+        "oracle_attend_prefill_bwd": [_p, _p, _p, _p, _i64, _i64, _i64, _i64, _i64, _i64, _p, _i64, _p,
+                                      ctypes.c_double, _p, _p, _p, _p],
         "oracle_max_threads": [],
         "oracle_set_threads": [ctypes.c_int],
     }
@@ -413,3 +415,27 @@ def attend_hssa(q, k, v, gk, gv, mk, mv, chunk: int, M: int, meta_idx, chunk_idx
                                   _ptr(chunk_idx), chunk_idx.shape[-1], float(scale), _ptr(r), len(r),
                                   _ptr(out), _ptr(lse))
     return out, lse
+
+
+# ----------------------------------------------------------------------------
+# 11. backward of the (gated) sparse prefill attention
+# ----------------------------------------------------------------------------
+
+def attend_prefill_bwd(q, k, v, dO, bs: int, idx, gate_scores=None, scale: Optional[float] = None):
+    """Gradients (fp64) of sum(dO * O) for O = attend_prefill(q, k, v, bs, idx,
+    gate_scores): (dq [B,Hq,N,d], dk, dv [B,Hkv,N,d], ds [B,Hkv,nb,nb] or None)."""
+    q, k, v, dO, idx = _f32(q), _f32(k), _f32(v), _f32(dO), _i32(idx)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    nb = N // bs
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = np.empty((B, Hq, N, d), np.float64)
+    dk = np.empty((B, Hkv, N, d), np.float64)
+    dv = np.empty((B, Hkv, N, d), np.float64)
+    gs = _f32(gate_scores) if gate_scores is not None else None
+    ds = np.empty((B, Hkv, nb, nb), np.float64) if gs is not None else None
+    lib().oracle_attend_prefill_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), B, Hq, Hkv, N, d, bs, _ptr(idx),
+                                    idx.shape[-1], _ptr(gs) if gs is not None else None, float(scale),
+                                    _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ds) if ds is not None else None)
+    return dq, dk, dv, ds

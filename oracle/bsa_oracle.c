@@ -711,6 +711,113 @@ void oracle_attend_hssa_rows(const float* q, const float* k, const float* v, con
     }
 }
 
+/* ------------------------------------------------------------------------ */
+/* 11. Backward of the (gated) sparse prefill attention                      */
+/* ------------------------------------------------------------------------ */
+
+/* SAS page, 核心洞察 and 核心模块 2: because the selector's continuous score
+ * enters the softmax logits in log form, the language-modelling loss reaches
+ * the selector by ordinary back-propagation.  Given the upstream gradient dO
+ * of the output of step 4/5 (prefill rows, the mask of step 4, the gate of
+ * step 5), this computes by the definition, in fp64:
+ *   P_{t,u} = softmax_u(l_{t,u}),  l_{t,u} = scale q_t.k_u + log g_{j(u)}
+ *   dV_u  += sum_t P_{t,u} dO_t
+ *   dl_{t,u} = P_{t,u} (dO_t.v_u - sum_w P_{t,w} dO_t.v_w)
+ *   dQ_t   = scale sum_u dl_{t,u} k_u,   dK_u += scale sum_t dl_{t,u} q_t
+ *   for the unit (b, g, i) of row t and its kept block l:
+ *   ds_{b,g,i,l} = sum_j dlogg_j (delta_{jl} - g_l), dlogg_j = sum over the
+ *   unit's rows t and block j's keys u of dl_{t,u}   (d log g_j / d s_l).
+ * q/dq [B,Hq,N,d], k/v/dk/dv [B,Hkv,N,d], dO [B,Hq,N,d]; gate_scores NULL:
+ * ungated (ds untouched); ds [B,Hkv,nb,nb] (zero where no block is kept).
+ * Every output is written whole (zero where nothing contributes). */
+void oracle_attend_prefill_bwd(const float* q, const float* k, const float* v, const float* dO, int64_t B,
+                               int64_t Hq, int64_t Hkv, int64_t N, int64_t d, int64_t bs, const int32_t* idx,
+                               int64_t idx_stride, const float* gate_scores, double scale, double* dq, double* dk,
+                               double* dv, double* ds)
+{
+    const int64_t nb = N / bs, G = Hq / Hkv;
+    memset(dq, 0, sizeof(double) * (size_t)(B * Hq * N * d));
+    memset(dk, 0, sizeof(double) * (size_t)(B * Hkv * N * d));
+    memset(dv, 0, sizeof(double) * (size_t)(B * Hkv * N * d));
+    if (gate_scores) memset(ds, 0, sizeof(double) * (size_t)(B * Hkv * nb * nb));
+    /* one (batch, group) at a time: its dk, dv and ds are written by it alone */
+#pragma omp parallel
+    {
+        unsigned char* sel = (unsigned char*)malloc((size_t)nb);
+        double* logg = (double*)malloc(sizeof(double) * (size_t)nb);
+        double* dlogg = (double*)malloc(sizeof(double) * (size_t)nb);
+        double* p = (double*)malloc(sizeof(double) * (size_t)N);
+        double* dp = (double*)malloc(sizeof(double) * (size_t)N);
+        int64_t* keys = (int64_t*)malloc(sizeof(int64_t) * (size_t)N);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t bg = 0; bg < B * Hkv; ++bg) {
+            const int64_t b = bg / Hkv, g = bg % Hkv;
+            const float* kb = k + bg * N * d;
+            const float* vb = v + bg * N * d;
+            for (int64_t i = 0; i < nb; ++i) {
+                const int32_t* list = idx + (bg * nb + i) * idx_stride;
+                mark_blocks(list, idx_stride, nb, sel);
+                if (gate_scores) gate_log_weights(gate_scores + (bg * nb + i) * nb, list, idx_stride, nb, logg);
+                for (int64_t j = 0; j < nb; ++j) dlogg[j] = 0.0;
+                for (int64_t hh = 0; hh < G; ++hh) {
+                    const int64_t h = g * G + hh;
+                    for (int64_t t = i * bs; t < (i + 1) * bs; ++t) {
+                        const int64_t r = (b * Hq + h) * N + t;
+                        const float* qr = q + r * d;
+                        const float* dor = dO + r * d;
+                        int64_t m = 0;
+                        double mx = -INFINITY;
+                        for (int64_t u = 0; u < N; ++u) {
+                            if (!key_allowed(sel, bs, t, u)) continue;
+                            double l = dot64(qr, kb + u * d, d) * scale;
+                            if (gate_scores) {
+                                if (logg[u / bs] == -INFINITY) continue;
+                                l += logg[u / bs];
+                            }
+                            keys[m] = u;
+                            p[m] = l;
+                            if (l > mx) mx = l;
+                            ++m;
+                        }
+                        if (m == 0) continue;
+                        double z = 0.0;
+                        for (int64_t a = 0; a < m; ++a) { p[a] = exp(p[a] - mx); z += p[a]; }
+                        double dsum = 0.0;
+                        for (int64_t a = 0; a < m; ++a) {
+                            p[a] /= z;
+                            dp[a] = dot64(dor, vb + keys[a] * d, d);
+                            dsum += p[a] * dp[a];
+                        }
+                        double* dqr = dq + r * d;
+                        for (int64_t a = 0; a < m; ++a) {
+                            const int64_t u = keys[a];
+                            const double dl = p[a] * (dp[a] - dsum);
+                            double* dkr = dk + (bg * N + u) * d;
+                            double* dvr = dv + (bg * N + u) * d;
+                            const float* kr = kb + u * d;
+                            for (int64_t c = 0; c < d; ++c) {
+                                dqr[c] += scale * dl * (double)kr[c];
+                                dkr[c] += scale * dl * (double)qr[c];
+                                dvr[c] += p[a] * (double)dor[c];
+                            }
+                            dlogg[u / bs] += dl;
+                        }
+                    }
+                }
+                if (gate_scores) {
+                    /* chain through log g_j = s_j - log sum_l exp(s_l) over the kept blocks */
+                    double tot = 0.0;
+                    for (int64_t j = 0; j < nb; ++j) if (logg[j] != -INFINITY) tot += dlogg[j];
+                    double* dsr = ds + (bg * nb + i) * nb;
+                    for (int64_t l = 0; l < nb; ++l)
+                        if (logg[l] != -INFINITY) dsr[l] = dlogg[l] - exp(logg[l]) * tot;
+                }
+            }
+        }
+        free(sel); free(logg); free(dlogg); free(p); free(dp); free(keys);
+    }
+}
+
 int oracle_max_threads(void)
 {
 #ifdef _OPENMP

@@ -268,3 +268,54 @@ def test_paged_decode_full_size_permuted_pages_sampled():
         want, _ = oracle.attend_decode(qs, inp["k"][b:b + 1, g:g + 1].float().cpu(),
                                        inp["v"][b:b + 1, g:g + 1].float().cpu(), w.bs, want_idx)
         _assert_close(step.bufs["o"][b, g * w.G:(g + 1) * w.G].float().cpu().numpy(), want, TOL_BF16, f"({b},{g})")
+
+
+# ----------------------------------------------------------------------------
+# two-level gist routing (H-SSA)
+# ----------------------------------------------------------------------------
+
+def _hssa_case(w, km, topk, rows_per_batch=None):
+    pipe = _pipe()
+    inp = W.make_inputs(w, "cuda")
+    step = pipe.HssaStep(inp["q"], inp["k"], inp["v"], inp["gk"], inp["gv"], inp["mk"], inp["mv"], w.bs, km, topk)
+    step.run()
+    torch.cuda.synchronize()
+    _status_clean()
+    got_meta = step.bufs["meta_idx"].cpu().numpy()
+    got_idx = step.bufs["idx"].cpu().numpy()
+    for b in range(w.B):
+        sl = slice(b, b + 1)
+        q = inp["q"][sl].float().cpu()
+        gk, gv = inp["gk"][sl].float().cpu(), inp["gv"][sl].float().cpu()
+        mk, mv = inp["mk"][sl].float().cpu(), inp["mv"][sl].float().cpu()
+        meta, chunks = oracle.hssa_select(q, gk, mk, 64, km, topk)
+        assert np.array_equal(got_meta[sl], meta), b
+        if topk > 0:
+            assert np.array_equal(got_idx[sl], chunks), b
+        rows = None if rows_per_batch is None else np.arange(rows_per_batch)
+        want, want_lse = oracle.attend_hssa(q, inp["k"][sl].float().cpu(), inp["v"][sl].float().cpu(), gk, gv, mk, mv,
+                                            w.bs, 64, meta, chunks, rows=rows)
+        got = step.bufs["o"][b].float().cpu().numpy()
+        got_lse = step.bufs["lse"][b].cpu().numpy()
+        if rows is not None:
+            got, got_lse = got[rows], got_lse[rows]
+        _assert_close(got, want, TOL_BF16, f"hssa b={b}")
+        _assert_close(got_lse, want_lse, TOL_LSE, "hssa lse")
+
+
+@pytest.mark.parametrize("hq,hkv,km,topk", [(8, 2, 2, 8), (4, 1, 1, 0), (4, 1, 4, 256), (16, 2, 3, 5), (2, 2, 1, 64)])
+def test_hssa_small(hq, hkv, km, topk):
+    """16384 tokens = 256 chunks = 4 groups of 64 chunks: one group kept (all
+    its chunks expanded at topk 64), no chunk expanded (gists and meta-gists
+    only), every group kept with every chunk expanded (dense over tokens)."""
+    w = W.get("hssa_decode_bf16").scaled(B=2, Hq=hq, Hkv=hkv, N=16384, kb=topk)
+    _hssa_case(w, km, topk)
+
+
+def test_hssa_full_size():
+    """The gist workload's shape with meta-gists: 8 sequences x 131072 tokens,
+    2048 chunks in 32 groups, 4 groups kept and 32 chunks expanded per head;
+    every head's choice compared, outputs of every head of the first two
+    sequences."""
+    w = W.get("hssa_decode_bf16")
+    _hssa_case(w.scaled(B=2, name=w.name), W.HSSA_GROUPS_KEPT, w.kb)

@@ -726,3 +726,121 @@ def test_hssa_attention_matches_library_on_explicit_key_set():
                         keys.append(gk[b, g, c]); vals.append(gv[b, g, c])
             ref = _sdpa64(q[b, h][None, None], np.array(keys)[None], np.array(vals)[None])
             assert np.allclose(out[b * Hq + h], ref[0, 0], atol=1e-10, rtol=0)
+
+
+# ----------------------------------------------------------------------------
+# backward of the (gated) sparse prefill attention
+# ----------------------------------------------------------------------------
+
+def _bwd_case(seed, B=1, Hq=4, Hkv=2, N=96, d=8, bs=16, kb=2):
+    r = _rng(seed)
+    q = r.standard_normal((B, Hq, N, d)).astype(np.float32)
+    k = r.standard_normal((B, Hkv, N, d)).astype(np.float32)
+    v = r.standard_normal((B, Hkv, N, d)).astype(np.float32)
+    dO = r.standard_normal((B, Hq, N, d)).astype(np.float32)
+    _, _, s, idx, _ = oracle.prefill_select(q, k, Hkv, bs, kb)
+    return q, k, v, dO, s, idx
+
+
+def _autograd_reference(q, k, v, dO, s, idx, bs, gated):
+    """torch autograd (fp64) of sum(dO * SDPA(q, k, v, bias)) where bias is the
+    sparse causal mask (-inf off the kept blocks) plus, gated, log_softmax of
+    the kept blocks' scores broadcast over each block's keys."""
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    G, nb = Hq // Hkv, N // bs
+    tq = torch.tensor(q, dtype=torch.float64, requires_grad=True)
+    tk = torch.tensor(k, dtype=torch.float64, requires_grad=True)
+    tv = torch.tensor(v, dtype=torch.float64, requires_grad=True)
+    ts = torch.tensor(s, dtype=torch.float64, requires_grad=True)
+    kept = torch.zeros((B, Hkv, nb, nb), dtype=torch.bool)
+    for b in range(B):
+        for g in range(Hkv):
+            for i in range(nb):
+                for j in idx[b, g, i]:
+                    if j >= 0:
+                        kept[b, g, i, j] = True
+    bias_blk = torch.where(kept, torch.zeros((), dtype=torch.float64), torch.tensor(float("-inf"), dtype=torch.float64))
+    if gated:
+        logits = ts.masked_fill(~kept, float("-inf"))
+        bias_blk = bias_blk + torch.log_softmax(logits, dim=-1).masked_fill(~kept, 0.0)
+    bias = bias_blk.repeat_interleave(bs, dim=2).repeat_interleave(bs, dim=3)          # [B,Hkv,N,N]
+    causal = torch.ones(N, N, dtype=torch.bool).tril()
+    bias = bias.masked_fill(~causal, float("-inf")).repeat_interleave(G, dim=1)       # [B,Hq,N,N]
+    o = F.scaled_dot_product_attention(tq, tk.repeat_interleave(G, 1), tv.repeat_interleave(G, 1), attn_mask=bias)
+    (o * torch.tensor(dO, dtype=torch.float64)).sum().backward()
+    return tq.grad.numpy(), tk.grad.numpy(), tv.grad.numpy(), (ts.grad.numpy() if gated else None)
+
+
+@pytest.mark.parametrize("gated", [False, True])
+def test_backward_matches_library_autograd(gated):
+    q, k, v, dO, s, idx = _bwd_case(100 + gated)
+    dq, dk, dv, ds = oracle.attend_prefill_bwd(q, k, v, dO, 16, idx, gate_scores=s if gated else None)
+    rq, rk, rv, rs = _autograd_reference(q, k, v, dO, s, idx, 16, gated)
+    for got, want in ((dq, rq), (dk, rk), (dv, rv)):
+        assert np.allclose(got, want, atol=1e-10, rtol=1e-9)
+    if gated:
+        assert np.allclose(ds, rs, atol=1e-10, rtol=1e-9)
+
+
+def test_backward_central_differences():
+    """d/dx of sum(dO * O) by central differences of the oracle's own forward,
+    at sampled coordinates of q, k, v and the selector scores."""
+    q, k, v, dO, s, idx = _bwd_case(102, N=48, d=4, bs=8, kb=2)
+    dq, dk, dv, ds = oracle.attend_prefill_bwd(q, k, v, dO, 8, idx, gate_scores=s)
+
+    def loss(q_, k_, v_, s_):
+        o, _ = oracle.attend_prefill(q_, k_, v_, 8, idx, gate_scores=s_)
+        return float((o.reshape(dO.shape) * dO.astype(np.float64)).sum())
+
+    r = _rng(103)
+    eps = 1e-2
+    for name, arr, grad in (("q", q, dq), ("k", k, dk), ("v", v, dv), ("s", s, ds)):
+        for _ in range(6):
+            pos = tuple(int(r.integers(0, n)) for n in arr.shape)
+            if name == "s" and not np.isfinite(arr[pos]):
+                continue
+            hi, lo = arr.copy(), arr.copy()
+            hi[pos] += eps
+            lo[pos] -= eps
+            args = {"q": q, "k": k, "v": v, "s": s}
+            args_hi = dict(args, **{name: hi})
+            args_lo = dict(args, **{name: lo})
+            fd = (loss(args_hi["q"], args_hi["k"], args_hi["v"], args_hi["s"]) -
+                  loss(args_lo["q"], args_lo["k"], args_lo["v"], args_lo["s"])) / (float(hi[pos]) - float(lo[pos]))
+            assert abs(fd - grad[pos]) <= 1e-4 * max(1.0, abs(grad[pos])), (name, pos, fd, grad[pos])
+
+
+def test_backward_score_gradient_sums_to_zero_per_unit():
+    """log g_j = s_j - log sum exp(s_kept): adding a constant to a unit's
+    scores changes nothing, so the unit's score gradients sum to zero."""
+    q, k, v, dO, s, idx = _bwd_case(104)
+    _, _, _, ds = oracle.attend_prefill_bwd(q, k, v, dO, 16, idx, gate_scores=s)
+    assert np.abs(ds.sum(axis=-1)).max() < 1e-12
+    assert np.abs(ds).max() > 1e-3
+
+
+def test_backward_uniform_gate_equals_ungated():
+    q, k, v, dO, s, idx = _bwd_case(105)
+    flat = np.zeros_like(s)
+    a = oracle.attend_prefill_bwd(q, k, v, dO, 16, idx, gate_scores=flat)
+    b = oracle.attend_prefill_bwd(q, k, v, dO, 16, idx)
+    for x, y in zip(a[:3], b[:3]):
+        assert np.allclose(x, y, atol=1e-12, rtol=0)
+
+
+def test_backward_full_budget_is_dense_causal():
+    q, k, v, dO, _, _ = _bwd_case(106)
+    N, bs = q.shape[2], 16
+    nb = N // bs
+    _, _, s, idx, _ = oracle.prefill_select(q, k, k.shape[1], bs, nb)
+    dq, dk, dv, _ = oracle.attend_prefill_bwd(q, k, v, dO, bs, idx)
+    G = q.shape[1] // k.shape[1]
+    tq = torch.tensor(q, dtype=torch.float64, requires_grad=True)
+    tk = torch.tensor(k, dtype=torch.float64, requires_grad=True)
+    tv = torch.tensor(v, dtype=torch.float64, requires_grad=True)
+    o = F.scaled_dot_product_attention(tq, tk.repeat_interleave(G, 1), tv.repeat_interleave(G, 1), is_causal=True)
+    (o * torch.tensor(dO, dtype=torch.float64)).sum().backward()
+    assert np.allclose(dq, tq.grad.numpy(), atol=1e-10, rtol=1e-9)
+    assert np.allclose(dk, tk.grad.numpy(), atol=1e-10, rtol=1e-9)
+    assert np.allclose(dv, tv.grad.numpy(), atol=1e-10, rtol=1e-9)

@@ -27,7 +27,7 @@ __all__ = [
     "bsa_sparse_attn_decode_noalloc", "bsa_decode_split_override", "bsa_selftest_wait_expiry",
     "bsa_prefill_kernel_override", "bsa_decode_select", "bsa_topk_select_pattern",
     "bsa_topk_select_joint_heads", "bsa_sparse_attn_decode_heads", "bsa_sparse_attn_decode_paged",
-    "bsa_paged_append", "EXPORTED_SYMBOLS",
+    "bsa_paged_append", "bsa_hssa_decode", "bsa_workspace_bytes_hssa", "EXPORTED_SYMBOLS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libbsa.so")
@@ -45,7 +45,7 @@ EXPORTED_SYMBOLS = (
     "bsa_status_string", "bsa_device_status", "bsa_version", "bsa_sparse_attn_decode_noalloc",
     "bsa_decode_split_override", "bsa_selftest_wait_expiry", "bsa_prefill_kernel_override",
     "bsa_decode_select", "bsa_topk_select_pattern", "bsa_topk_select_joint_heads", "bsa_sparse_attn_decode_heads",
-    "bsa_sparse_attn_decode_paged", "bsa_paged_append",
+    "bsa_sparse_attn_decode_paged", "bsa_paged_append", "bsa_hssa_decode", "bsa_workspace_bytes_hssa",
 )
 
 
@@ -74,6 +74,9 @@ _SIGS = {
     "bsa_sparse_attn_decode_paged": (_i, [ctypes.POINTER(BsaShape), _p, _p, _p, _i, _p, _i, _p, _i, ctypes.c_float,
                                           _p, ctypes.c_size_t, _p, _p, _p]),
     "bsa_paged_append": (_i, [ctypes.POINTER(BsaShape), _p, _p, _p, _p, _i, _i, _p, _p, _p, _p]),
+    "bsa_hssa_decode": (_i, [ctypes.POINTER(BsaShape), _p, _p, _p, _p, _p, _p, _p, _i, _i, _p, _p, ctypes.c_float,
+                             _p, ctypes.c_size_t, _p, _p, _p]),
+    "bsa_workspace_bytes_hssa": (ctypes.c_size_t, [ctypes.POINTER(BsaShape), _i, _i]),
     "bsa_topk_select_joint_heads": (_i, [_p, _i, _i, _i, _i, _p, _i, _p, _p]),
     "bsa_sparse_attn_decode_heads": (_i, [ctypes.POINTER(BsaShape), _p, _p, _p, _p, _i, ctypes.c_float, _p,
                                           ctypes.c_size_t, _p, _p, _p]),
@@ -237,6 +240,20 @@ def bsa_paged_append(shape: BsaShape, k_new, v_new, seq_lens, block_table, k_poo
     _check("bsa_paged_append", lib.bsa_paged_append(
         ctypes.byref(shape), _ptr(k_new), _ptr(v_new), _ptr(seq_lens), _ptr(block_table), int(block_table.shape[-1]),
         int(k_pool.shape[0]), _ptr(k_pool), _ptr(v_pool), _ptr(pooled_k), _stream(stream)))
+
+
+def bsa_hssa_decode(shape: BsaShape, q, k_cache, v_cache, gist_k, gist_v, meta_k, meta_v, km: int, topk: int,
+                    meta_out=None, idx_out=None, softmax_scale: float = 0.0, workspace=None, o=None, lse=None,
+                    stream=None) -> None:
+    _check("bsa_hssa_decode", lib.bsa_hssa_decode(
+        ctypes.byref(shape), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(gist_k), _ptr(gist_v), _ptr(meta_k),
+        _ptr(meta_v), int(km), int(topk), _ptr(meta_out), _ptr(idx_out), ctypes.c_float(softmax_scale),
+        _ptr(workspace), ctypes.c_size_t(workspace.numel() * workspace.element_size() if workspace is not None else 0),
+        _ptr(o), _ptr(lse), _stream(stream)))
+
+
+def bsa_workspace_bytes_hssa(shape: BsaShape, km: int, topk: int) -> int:
+    return int(lib.bsa_workspace_bytes_hssa(ctypes.byref(shape), int(km), int(topk)))
 
 
 def bsa_decode_select(shape: BsaShape, q, pooled_k, kb: int, scores, idx_out, idx_stride: int,

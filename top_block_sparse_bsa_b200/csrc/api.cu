@@ -202,6 +202,44 @@ HeadsLayout heads_layout(const bsa_shape_t* s, int idx_stride, int num_sms) {
   return L;
 }
 
+// Workspace of the two-level gist decode.
+struct HssaLayout {
+  size_t meta_scores, meta_idx, fine, pos, chunks, expanded, allow, union_list, partial, total;
+  int union_stride, k_stride;
+  DecodePlan plan;
+};
+
+HssaLayout hssa_layout(const bsa_shape_t* s, int km, int topk, int num_sms) {
+  HssaLayout L{};
+  const int nc = s->Nk / s->block, nm = nc / 64;
+  const int G = s->Hq / s->Hkv;
+  const int64_t rows = static_cast<int64_t>(s->B) * s->Hq;
+  L.k_stride = topk > 0 ? topk : 1;
+  L.union_stride = 1 + std::min(nc, G * topk) + nm + 1;
+  L.plan = decode_plan(s->B * s->Hkv, L.union_stride - 1, num_sms);
+  size_t off = 0;
+  L.meta_scores = off;
+  off = align256(off + rows * nm * sizeof(float));
+  L.meta_idx = off;
+  off = align256(off + rows * km * sizeof(int));
+  L.fine = off;
+  off = align256(off + rows * km * 64 * sizeof(float));
+  L.pos = off;
+  off = align256(off + rows * L.k_stride * sizeof(int));
+  L.chunks = off;
+  off = align256(off + rows * L.k_stride * sizeof(int));
+  L.expanded = off;
+  off = align256(off + rows * (nc / 32) * sizeof(uint32_t));
+  L.allow = off;
+  off = align256(off + rows * ((nc + 64) / 32) * sizeof(uint32_t));
+  L.union_list = off;
+  off = align256(off + static_cast<size_t>(s->B) * s->Hkv * L.union_stride * sizeof(int));
+  L.partial = off;
+  off = align256(off + rows * L.plan.max_slots * (s->d + 4) * sizeof(float));
+  L.total = off;
+  return L;
+}
+
 // Self-test of the bounded-wait expiry path: one thread waits, with a small
 // budget, on a shared-memory barrier that nothing arrives on.  The wait gives
 // up, raises BSA_DEV_TIMEOUT in the status word and the kernel returns.
@@ -303,6 +341,13 @@ size_t bsa_workspace_bytes(int op, const bsa_shape_t* s, int budget) {
     return heads_layout(s, budget, sms).total;
   }
   return 0;
+}
+
+size_t bsa_workspace_bytes_hssa(const bsa_shape_t* s, int km, int topk) {
+  if (check_shape(s) != BSA_OK || km < 1 || topk < 0) return 0;
+  int sms = 0;
+  if (device_state(nullptr, &sms) != BSA_OK) return 0;
+  return hssa_layout(s, km, topk, sms).total;
 }
 
 bsa_status_t bsa_score_blocks(const bsa_shape_t* s, int mode, const void* q, const void* k,
@@ -732,6 +777,79 @@ bsa_status_t bsa_paged_append(const bsa_shape_t* s, const void* k_new, const voi
   return cuda_status(launch_paged_append(k_new, v_new, s->B, s->Hkv, s->Nq, s->d, seq_lens, block_table,
                                          table_stride, num_pages, k_pool, v_pool, pooled_k, status,
                                          static_cast<cudaStream_t>(stream)));
+}
+
+bsa_status_t bsa_hssa_decode(const bsa_shape_t* s, const void* q, const void* k_cache, const void* v_cache,
+                             const void* gist_k, const void* gist_v, const void* meta_k, const void* meta_v, int km,
+                             int topk, int* meta_out, int* idx_out, float softmax_scale, void* workspace,
+                             size_t workspace_bytes, void* o, float* lse, void* stream) {
+  bsa_status_t st = decode_checks(s, q, k_cache, v_cache, o);
+  if (st != BSA_OK) return st;
+  const int nc = s->Nk / s->block;
+  if (!gist_k || !gist_v || !meta_k || !meta_v) return BSA_ERR_INVALID_ARG;
+  if (!aligned16(gist_k) || !aligned16(gist_v) || !aligned16(meta_k) || !aligned16(meta_v)) return BSA_ERR_INVALID_ARG;
+  if (nc % 64 != 0 || nc / 64 > 64) return BSA_ERR_UNSUPPORTED;   // groups of 64 chunks, at most 64 groups
+  const int nm = nc / 64;
+  if (km < 1 || km > nm || topk < 0 || topk > km * 64 || !(softmax_scale > 0.0f) || !workspace)
+    return BSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return BSA_ERR_INVALID_ARG;
+  uint32_t* status = nullptr;
+  int sms = 0;
+  if ((st = device_state(&status, &sms)) != BSA_OK) return st;
+  const HssaLayout L = hssa_layout(s, km, topk, sms);
+  if (workspace_bytes < L.total) return BSA_ERR_INVALID_ARG;
+  char* ws = static_cast<char*>(workspace);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const int G = s->Hq / s->Hkv;
+  const int rows = s->B * s->Hq;
+  const uint64_t bgs = static_cast<uint64_t>(s->B) * s->Hkv;
+  CUtensorMap mq, mk, mv, mgk, mgv, mmk, mmv;
+  if (!make_map_bf16(&mq, q, static_cast<uint64_t>(rows), static_cast<uint32_t>(G)) ||
+      !make_map_bf16(&mk, k_cache, bgs * s->Nk, 64) || !make_map_bf16(&mv, v_cache, bgs * s->Nk, 64) ||
+      !make_map_bf16(&mgk, gist_k, bgs * nc, 64) || !make_map_bf16(&mgv, gist_v, bgs * nc, 64) ||
+      !make_map_bf16(&mmk, meta_k, bgs * nm, 64) || !make_map_bf16(&mmv, meta_v, bgs * nm, 64))
+    return BSA_ERR_CUDA;
+  const float scale = score_scale(s->d);
+  float* meta_scores = reinterpret_cast<float*>(ws + L.meta_scores);
+  int* meta_idx = meta_out ? meta_out : reinterpret_cast<int*>(ws + L.meta_idx);
+  float* fine = reinterpret_cast<float*>(ws + L.fine);
+  int* pos = reinterpret_cast<int*>(ws + L.pos);
+  int* chunks = (idx_out && topk > 0) ? idx_out : reinterpret_cast<int*>(ws + L.chunks);
+  uint32_t* expanded = reinterpret_cast<uint32_t*>(ws + L.expanded);
+  uint32_t* allow = reinterpret_cast<uint32_t*>(ws + L.allow);
+  int* ulist = reinterpret_cast<int*>(ws + L.union_list);
+  // coarse: meta-gist scores and the km best groups per head
+  cudaError_t e = launch_score_gist(q, meta_k, true, s->B, s->Hq, s->Hkv, nm, s->d, scale, meta_scores, cs);
+  if (e == cudaSuccess) e = launch_topk(meta_scores, rows, nm, BSA_TOPK_PLAIN, km, meta_idx, km, nullptr, cs);
+  // fine: the gists of the kept groups' chunks and the topk best per head
+  if (e == cudaSuccess) e = launch_score_gist_groups(q, gist_k, meta_idx, km, s->B, s->Hq, s->Hkv, nc, scale, fine, cs);
+  if (e == cudaSuccess)
+    e = launch_topk(fine, rows, km * 64, BSA_TOPK_PLAIN, topk, pos, L.k_stride, nullptr, cs);
+  if (e == cudaSuccess)
+    e = launch_hssa_union(meta_idx, km, pos, L.k_stride, s->B, s->Hq, s->Hkv, nc, nm, chunks, expanded, allow, ulist,
+                          L.union_stride, status, cs);
+  DecodeArgs a;
+  a.B = s->B;
+  a.Hq = s->Hq;
+  a.Hkv = s->Hkv;
+  a.Nk = s->Nk;
+  a.bs = s->block;
+  a.list = ulist;
+  a.list_stride = L.union_stride;
+  a.list_has_count = 1;
+  a.expanded = expanded;
+  a.nc = nc;
+  a.list_len = L.plan.list_len;
+  a.num_ctas = L.plan.num_ctas;
+  a.max_slots = L.plan.max_slots;
+  a.softmax_scale = softmax_scale;
+  a.partial = reinterpret_cast<float*>(ws + L.partial);
+  a.status = status;
+  a.gist_allow = allow;
+  a.meta_rows = nm;
+  if (e == cudaSuccess) e = launch_attn_decode_bf16(&mq, &mk, &mv, &mgk, &mgv, a, cs, &mmk, &mmv);
+  if (e == cudaSuccess) e = launch_decode_combine(a.partial, a, s->d, true, o, lse, cs);
+  return cuda_status(e);
 }
 
 }  // extern "C"

@@ -109,6 +109,12 @@ struct Params {
   // physical block table[b * table_stride + j] of the pools [P][Hkv][64][d]
   const int* table;
   int table_stride, num_pages;
+  // two-level gists (H-SSA): gist tiles at or past nc/64 are meta-gist tiles
+  // (rows bg*meta_rows + ..., of the meta maps); gist_allow [B*Hq][(nc+64)/32]
+  // says per head which gist / meta-gist rows it attends (null: SSA's rule,
+  // the gist of every chunk the head did not expand)
+  const uint32_t* gist_allow;
+  int meta_rows;
 };
 
 // The split space is every group row's list positions laid end to end; CTA c
@@ -164,6 +170,10 @@ __device__ __forceinline__ void softmax_role(const Params& p, Misc* misc, uint8_
       } else {
         const uint32_t* bits_base =
             gist ? p.expanded + (static_cast<int64_t>(b) * p.Hq + g * G) * (p.nc / 32) : nullptr;
+        const bool two_level = p.gist_allow != nullptr;
+        const int words_g = (p.nc + 64) / 32;
+        const uint32_t* allow_base =
+            two_level ? p.gist_allow + (static_cast<int64_t>(b) * p.Hq + g * G) * words_g : nullptr;
         float m_run[GH], l_part[GH];
 #pragma unroll
         for (int h = 0; h < GH; ++h) {
@@ -186,7 +196,10 @@ __device__ __forceinline__ void softmax_role(const Params& p, Misc* misc, uint8_
           uint32_t word[GH];
 #pragma unroll
           for (int h = 0; h < GH; ++h)
-            word[h] = (gist && h < G && has_mine) ? __ldg(bits_base + h * words + (bitpos >> 5)) : 0u;
+            word[h] = (gist && h < G && has_mine)
+                          ? ((two_level && mytile < 0) ? __ldg(allow_base + h * words_g + (bitpos >> 5))
+                                                       : __ldg(bits_base + h * words + (bitpos >> 5)))
+                          : 0u;
           if (!(ok = warp_wait(bar(BAR_SF + sb), (s_read >> 1) & 1, abortp, p.status))) break;
           tc_fence_after();
           uint32_t sv[GH];
@@ -200,8 +213,9 @@ __device__ __forceinline__ void softmax_role(const Params& p, Misc* misc, uint8_
             bool allowed = h < G && has_mine;
             if (allowed && gist) {
               const bool bit = (word[h] >> (bitpos & 31)) & 1u;
-              // an expanded chunk's tokens, or the gist of a chunk not expanded
-              allowed = (mytile >= 0) ? bit : !bit;
+              // an expanded chunk's tokens, or the gist of a chunk not expanded;
+              // with two-level gists, a gist or meta-gist row the head attends
+              allowed = (mytile >= 0 || two_level) ? bit : !bit;
             }
             x[h] = allowed ? __uint_as_float(sv[h]) * p.scale_log2 : -INFINITY;
           }
@@ -314,7 +328,8 @@ __device__ __forceinline__ void softmax_role(const Params& p, Misc* misc, uint8_
 __global__ void __launch_bounds__(kThreads, 1)
     attn_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmGK,
-                       const __grid_constant__ CUtensorMap tmGV, const Params p) {
+                       const __grid_constant__ CUtensorMap tmGV, const __grid_constant__ CUtensorMap tmMK,
+                       const __grid_constant__ CUtensorMap tmMV, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -357,6 +372,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (gist) {
       prefetch_tmap(&tmGK);
       prefetch_tmap(&tmGV);
+      if (p.meta_rows > 0) {
+        prefetch_tmap(&tmMK);
+        prefetch_tmap(&tmMV);
+      }
     }
   }
   if (warp == 5) {
@@ -371,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 6) {
     // ------------------------------------------------ item loader
-    const int nb_cache = p.Nk / 64, ngist = p.nc / 64;
+    const int nb_cache = p.Nk / 64, ngist = p.nc / 64 + (p.meta_rows > 0 ? 1 : 0);
     int r0 = 0;
     const int nitems = cta_items(p, blockIdx.x, &r0);
     const int64_t lo = static_cast<int64_t>(blockIdx.x) * p.total / p.num_ctas;
@@ -468,9 +487,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (tile >= 0) {
                   map = kv ? &tmV : &tmK;
                   y = (p.table != nullptr) ? (tile * p.Hkv + inf->g) * 64 : inf->bg * p.Nk + tile * 64;
-                } else {
+                } else if (-(tile + 1) < p.nc / 64) {
                   map = kv ? &tmGV : &tmGK;
                   y = inf->bg * p.nc + (-(tile + 1)) * 64;
+                } else {   // the meta-gist tile (two-level gists)
+                  map = kv ? &tmMV : &tmMK;
+                  y = inf->bg * p.meta_rows + (-(tile + 1) - p.nc / 64) * 64;
                 }
                 for (int hf = 0; hf < 2; ++hf)
                   tma_load_2d(dst0 + hf * kHalfBytes + tt * 8192u, map, bar(full + slot), hf * 64, y);
@@ -707,11 +729,117 @@ __global__ void gist_union_kernel(const int* __restrict__ idx, int Hq, int Hkv, 
   }
 }
 
+// Two-level gists (H-SSA): per (b, g) from each head's kept groups (meta_idx
+// [B*Hq][km], ascending) and chosen positions among its kept groups' chunks
+// (pos_idx [B*Hq][k]: position t*64 + x = chunk x of its t-th kept group,
+// ascending): each head's chunk list (chunk_out), its expanded-chunk bitmap,
+// its gist-allowed bitmap over the rows [gists 0..nc) | [meta-gists nm..)
+// (a gist of a kept group not expanded; a meta-gist of a group not kept),
+// and the group's tile list: expanded chunks ascending, the gist tiles of the
+// groups any head kept, then the meta-gist tile.  Groups are 64 chunks, so a
+// kept group's gists are one gist tile.
+__global__ void hssa_union_kernel(const int* __restrict__ meta_idx, int km, const int* __restrict__ pos_idx, int k,
+                                  int Hq, int Hkv, int nc, int nm, int* __restrict__ chunk_out,
+                                  uint32_t* __restrict__ expanded, uint32_t* __restrict__ gist_allow,
+                                  int* __restrict__ union_list, int union_stride, uint32_t* __restrict__ status) {
+  griddep_wait();
+  extern __shared__ uint32_t sb[];
+  const int G = Hq / Hkv;
+  const int words = nc / 32, words_g = (nc + 64) / 32;
+  uint32_t* ex = sb;                       // [G+1][words]: heads' expanded chunks, then the union
+  uint32_t* al = sb + (G + 1) * words;     // [G][words_g]: heads' allowed gist / meta rows
+  uint32_t* kg = al + G * words_g;         // [G+1][2]: heads' kept groups (nm <= 64), then the union
+  const int bg = blockIdx.x;
+  const int b = bg / Hkv, g = bg % Hkv;
+  const int total = (G + 1) * words + G * words_g + (G + 1) * 2;
+  for (int e = threadIdx.x; e < total; e += blockDim.x) sb[e] = 0u;
+  __syncthreads();
+  const int64_t row0 = static_cast<int64_t>(b) * Hq + g * G;
+  for (int e = threadIdx.x; e < G * km; e += blockDim.x) {
+    const int hh = e / km, t = e % km;
+    const int m = meta_idx[(row0 + hh) * km + t];
+    if (m < 0) continue;
+    if (m >= nm) {
+      atomicOr(status, BSA_DEV_BAD_INDEX);
+      continue;
+    }
+    atomicOr(&kg[hh * 2 + (m >> 5)], 1u << (m & 31));
+    atomicOr(&kg[G * 2 + (m >> 5)], 1u << (m & 31));
+  }
+  for (int e = threadIdx.x; e < G * k; e += blockDim.x) {
+    const int hh = e / k, t = e % k;
+    const int pos = pos_idx[(row0 + hh) * k + t];
+    int c = -1;
+    if (pos >= 0) {
+      const int grp = pos >> 6;
+      const int m = (grp < km) ? meta_idx[(row0 + hh) * km + grp] : -1;
+      c = (m >= 0 && m < nm) ? m * 64 + (pos & 63) : -1;
+      if (c < 0 || c >= nc) {
+        atomicOr(status, BSA_DEV_BAD_INDEX);
+        c = -1;
+      }
+    }
+    chunk_out[(row0 + hh) * k + t] = c;
+    if (c < 0) continue;
+    atomicOr(&ex[hh * words + (c >> 5)], 1u << (c & 31));
+    atomicOr(&ex[G * words + (c >> 5)], 1u << (c & 31));
+  }
+  __syncthreads();
+  // allowed rows: gist c of a kept group not expanded; meta-gist m of a group not kept
+  for (int e = threadIdx.x; e < G * words_g; e += blockDim.x) {
+    const int hh = e / words_g, w = e % words_g;
+    uint32_t bits = 0u;
+    if (w < words) {
+      const int m = (w * 32) >> 6;   // 32 consecutive chunks lie in one group of 64
+      if ((kg[hh * 2 + (m >> 5)] >> (m & 31)) & 1u) bits = ~ex[hh * words + w];
+    } else {
+      for (int x = 0; x < 32; ++x) {
+        const int m = (w - words) * 32 + x;
+        if (m < nm && !((kg[hh * 2 + (m >> 5)] >> (m & 31)) & 1u)) bits |= 1u << x;
+      }
+    }
+    al[e] = bits;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < G * words; e += blockDim.x) expanded[row0 * words + e] = ex[e];
+  for (int e = threadIdx.x; e < G * words_g; e += blockDim.x) gist_allow[row0 * words_g + e] = al[e];
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    int* out = union_list + static_cast<int64_t>(bg) * union_stride;
+    int run = 0;
+    for (int base = 0; base < words; base += 32) {
+      const int w = base + lane;
+      const uint32_t bitsw = (w < words) ? ex[G * words + w] : 0u;
+      const int cnt = __popc(bitsw);
+      int incl = cnt;
+      for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+      }
+      int pos = run + incl - cnt;
+      uint32_t mm = bitsw;
+      while (mm) {
+        const int bit = __ffs(mm) - 1;
+        mm &= mm - 1;
+        out[1 + pos++] = w * 32 + bit;
+      }
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    // the gist tiles of kept groups (tile -(m+1) holds the 64 gists of group m), then the meta tile
+    if (lane == 0) {
+      for (int m = 0; m < nm; ++m)
+        if ((kg[G * 2 + (m >> 5)] >> (m & 31)) & 1u) out[1 + run++] = -(m + 1);
+      out[1 + run++] = -(nc / 64 + 1);
+      out[0] = run;
+    }
+  }
+}
+
 }  // namespace decode
 
 cudaError_t launch_attn_decode_bf16(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
                                     const CUtensorMap* tmGK, const CUtensorMap* tmGV, const DecodeArgs& a,
-                                    cudaStream_t st) {
+                                    cudaStream_t st, const CUtensorMap* tmMK, const CUtensorMap* tmMV) {
   cudaError_t e = ensure_dynamic_smem<decode::attn_decode_kernel>(decode::kSmemBytes);
   if (e != cudaSuccess) return e;
   decode::Params p;
@@ -735,9 +863,12 @@ cudaError_t launch_attn_decode_bf16(const CUtensorMap* tmQ, const CUtensorMap* t
   p.table = a.table;
   p.table_stride = a.table_stride;
   p.num_pages = a.num_pages;
+  p.gist_allow = a.gist_allow;
+  p.meta_rows = (tmMK != nullptr) ? a.meta_rows : 0;
   const int grid = a.num_ctas;
   return launch_dependent(decode::attn_decode_kernel, dim3(grid), dim3(decode::kThreads), decode::kSmemBytes, st, *tmQ,
-                          *tmK, *tmV, tmGK ? *tmGK : *tmK, tmGV ? *tmGV : *tmV, p);
+                          *tmK, *tmV, tmGK ? *tmGK : *tmK, tmGV ? *tmGV : *tmV, tmMK ? *tmMK : *tmK,
+                          tmMV ? *tmMV : *tmV, p);
 }
 
 cudaError_t launch_decode_combine(const float* partial, const DecodeArgs& a, int d, bool out_bf16, void* o,
@@ -768,6 +899,17 @@ cudaError_t launch_gist_union(const int* idx, int B, int Hq, int Hkv, int topk, 
   const size_t smem = static_cast<size_t>(G + 1) * (nc / 32) * sizeof(uint32_t);
   return launch_dependent(decode::gist_union_kernel, dim3(B * Hkv), dim3(256), smem, st, idx, Hq, Hkv, topk, idx_stride,
                           nc, expanded, union_list, union_stride, with_gists ? 1 : 0, status);
+}
+
+cudaError_t launch_hssa_union(const int* meta_idx, int km, const int* pos_idx, int k, int B, int Hq, int Hkv, int nc,
+                              int nm, int* chunk_out, uint32_t* expanded, uint32_t* gist_allow, int* union_list,
+                              int union_stride, uint32_t* status, cudaStream_t st) {
+  const int G = Hq / Hkv;
+  const size_t smem = (static_cast<size_t>(G + 1) * (nc / 32) + static_cast<size_t>(G) * ((nc + 64) / 32) +
+                       static_cast<size_t>(G + 1) * 2) *
+                      sizeof(uint32_t);
+  return launch_dependent(decode::hssa_union_kernel, dim3(B * Hkv), dim3(256), smem, st, meta_idx, km, pos_idx, k, Hq,
+                          Hkv, nc, nm, chunk_out, expanded, gist_allow, union_list, union_stride, status);
 }
 
 }  // namespace bsa

@@ -83,6 +83,8 @@ cudaError_t launch_score_heads(const void* q, bool bf16, const float* kbar, int 
                                float scale, float* s, cudaStream_t st);
 cudaError_t launch_topk_joint(const float* scores, int rows, int G, int nb, int kb_total, int* idx_out,
                               int idx_stride, int* count_out, cudaStream_t st);
+cudaError_t launch_score_gist_groups(const void* q, const void* gk, const int* meta_idx, int km, int B, int Hq,
+                                     int Hkv, int nc, float scale, float* fine, cudaStream_t st);
 // decode scores + top-k in one kernel (tmKbar: fp32 [rows, 128], box 32 x 128, 128-byte swizzle)
 bool decode_select_fused_ok(int d, int nb);
 cudaError_t launch_decode_select(const CUtensorMap* tmKbar, const void* q, bool bf16, int B, int Hq, int Hkv,
@@ -141,10 +143,17 @@ struct DecodeArgs {
   // table[b*table_stride + j] of pools [num_pages][Hkv][64][d]; null: contiguous
   const int* table = nullptr;
   int table_stride = 0, num_pages = 0;
+  // two-level gists: per-head allowed gist / meta-gist rows; meta rows per (b, g)
+  const uint32_t* gist_allow = nullptr;
+  int meta_rows = 0;
 };
 cudaError_t launch_attn_decode_bf16(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
                                     const CUtensorMap* tmGK, const CUtensorMap* tmGV, const DecodeArgs& a,
-                                    cudaStream_t st);
+                                    cudaStream_t st, const CUtensorMap* tmMK = nullptr,
+                                    const CUtensorMap* tmMV = nullptr);
+cudaError_t launch_hssa_union(const int* meta_idx, int km, const int* pos_idx, int k, int B, int Hq, int Hkv, int nc,
+                              int nm, int* chunk_out, uint32_t* expanded, uint32_t* gist_allow, int* union_list,
+                              int union_stride, uint32_t* status, cudaStream_t st);
 cudaError_t launch_decode_combine(const float* partial, const DecodeArgs& a, int d, bool out_bf16, void* o,
                                   float* lse, cudaStream_t st);
 int decode_slots_for(int rows, int list_len, int num_ctas);

@@ -1115,6 +1115,68 @@ cudaError_t launch_topk_joint(const float* scores, int rows, int G, int nb, int 
                           idx_stride, count_out);
 }
 
+// ------------------------------------------------- two-level gists: fine scores
+// H-SSA's fine step (SSA page, 层级扩展): query head (b, h) scores the gists of
+// the chunks inside its t-th kept group (64 chunks per group).  Grid (km,
+// B*Hq), 64 threads = the group's chunks; the group's 64 gist rows are read
+// with 16-byte loads into padded float rows, then each thread runs the
+// fixed-order dot product of its chunk's gist (as score_gist_bf16_d128_kernel).
+// fine [B*Hq][km*64]: position t*64 + x.  A group slot past the kept ones
+// gets NaN (never ranked above a number).
+__global__ void __launch_bounds__(64) score_gist_groups_kernel(const __nv_bfloat16* __restrict__ q,
+                                                               const __nv_bfloat16* __restrict__ gk,
+                                                               const int* __restrict__ meta_idx, int km, int Hq,
+                                                               int Hkv, int nc, float scale,
+                                                               float* __restrict__ fine) {
+  griddep_wait();   // the kept groups come from the kernel launched before
+  constexpr int D = 128, kPitch = D + 4;
+  __shared__ __align__(16) float ks[64 * kPitch];
+  __shared__ __align__(16) float qs[D];
+  const int t = blockIdx.x;
+  const int64_t row = blockIdx.y;   // b * Hq + h
+  const int64_t b = row / Hq;
+  const int g = static_cast<int>(row % Hq) / (Hq / Hkv);
+  const int m = meta_idx[row * km + t];
+  float* out = fine + row * (static_cast<int64_t>(km) * 64) + t * 64;
+  if (m < 0 || m >= nc / 64) {
+    out[threadIdx.x] = __int_as_float(0x7fc00000);   // NaN
+    return;
+  }
+  const uint4* src = reinterpret_cast<const uint4*>(gk + ((b * Hkv + g) * static_cast<int64_t>(nc) + m * 64) * D);
+  for (int e = threadIdx.x; e < 64 * (D / 8); e += 64) {
+    const int r = e >> 4, c8 = e & 15;
+    const uint4 v = __ldg(src + e);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float* dst = ks + r * kPitch + 8 * c8;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      dst[2 * i] = __uint_as_float(w[i] << 16);
+      dst[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+  for (int e = threadIdx.x; e < D; e += 64) qs[e] = __bfloat162float(q[row * D + e]);
+  __syncthreads();
+  const float4* kr = reinterpret_cast<const float4*>(ks + threadIdx.x * kPitch);
+  const float4* qr = reinterpret_cast<const float4*>(qs);
+  float acc = 0.0f;
+#pragma unroll
+  for (int e = 0; e < D / 4; ++e) {
+    const float4 kv = kr[e], qv = qr[e];
+    acc = __fadd_rn(acc, __fmul_rn(qv.x, kv.x));
+    acc = __fadd_rn(acc, __fmul_rn(qv.y, kv.y));
+    acc = __fadd_rn(acc, __fmul_rn(qv.z, kv.z));
+    acc = __fadd_rn(acc, __fmul_rn(qv.w, kv.w));
+  }
+  out[threadIdx.x] = __fmul_rn(acc, scale);
+}
+
+cudaError_t launch_score_gist_groups(const void* q, const void* gk, const int* meta_idx, int km, int B, int Hq,
+                                     int Hkv, int nc, float scale, float* fine, cudaStream_t st) {
+  return launch_dependent(score_gist_groups_kernel, dim3(km, B * Hq), dim3(64), 0, st,
+                          static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(gk), meta_idx, km,
+                          Hq, Hkv, nc, scale, fine);
+}
+
 cudaError_t launch_topk(const float* scores, int rows, int ncols, int mode, int kb, int* idx_out,
                         int idx_stride, int* count_out, cudaStream_t st) {
   if (ncols <= 32 * 16) {

@@ -17,7 +17,7 @@ import torch
 from . import (BSA_OP_DECODE, BSA_OP_DECODE_HEADS, BSA_OP_GIST_DECODE, BSA_SCORE_DECODE,
                BSA_SCORE_DECODE_HEADS, BSA_SCORE_PREFILL, BSA_TOPK_CAUSAL_BLOCK, bsa_decode_select,
                bsa_gated_attn_fwd, bsa_gist_expand_decode, bsa_score_blocks, bsa_sparse_attn_decode,
-               bsa_paged_append, bsa_sparse_attn_decode_heads, bsa_sparse_attn_decode_paged, bsa_sparse_attn_prefill,
+               bsa_hssa_decode, bsa_paged_append, bsa_sparse_attn_decode_heads, bsa_workspace_bytes_hssa, bsa_sparse_attn_decode_paged, bsa_sparse_attn_prefill,
                bsa_topk_select, bsa_topk_select_joint_heads, bsa_topk_select_pattern, bsa_workspace_bytes,
                make_shape)
 
@@ -314,3 +314,45 @@ class PagedDecodeStep:
         self.select(stream)
         self.attend(stream=stream, with_lse=with_lse)
         return self.bufs
+
+
+@dataclass
+class HssaStep:
+    """Two-level gist routing decode (H-SSA): meta-gist scores -> km groups
+    per head -> gist scores inside them -> topk chunks per head -> attention
+    over expanded tokens, gists of kept groups, meta-gists of the rest (one C
+    call).  Groups are 64 chunks; meta_k/meta_v [B,Hkv,nc/64,d]."""
+    q: torch.Tensor
+    k_cache: torch.Tensor
+    v_cache: torch.Tensor
+    gist_k: torch.Tensor
+    gist_v: torch.Tensor
+    meta_k: torch.Tensor
+    meta_v: torch.Tensor
+    chunk: int
+    km: int
+    topk: int
+    softmax_scale: Optional[float] = None
+    bufs: Dict[str, torch.Tensor] = field(default_factory=dict)
+
+    def __post_init__(self):
+        B, Hq, d = self.q.shape
+        Hkv, Nk = self.k_cache.shape[1], self.k_cache.shape[2]
+        self.shape = make_shape(B, Hq, Hkv, 1, Nk, d, self.chunk, self.q.dtype)
+        if self.softmax_scale is None:
+            self.softmax_scale = 1.0 / math.sqrt(d)
+        dev = _dev(self.q)
+        b = self.bufs
+        ws = bsa_workspace_bytes_hssa(self.shape, self.km, self.topk)
+        b.setdefault("workspace", torch.empty((max(ws, 256),), dtype=torch.uint8, device=dev))
+        b.setdefault("meta_idx", torch.empty((B, Hq, self.km), dtype=torch.int32, device=dev))
+        b.setdefault("idx", torch.empty((B, Hq, max(self.topk, 1)), dtype=torch.int32, device=dev))
+        b.setdefault("o", torch.empty_like(self.q))
+        b.setdefault("lse", torch.empty((B, Hq), dtype=torch.float32, device=dev))
+
+    def run(self, stream=None, with_lse: bool = True):
+        b = self.bufs
+        bsa_hssa_decode(self.shape, self.q, self.k_cache, self.v_cache, self.gist_k, self.gist_v, self.meta_k,
+                        self.meta_v, self.km, self.topk, b["meta_idx"], b["idx"] if self.topk > 0 else None,
+                        self.softmax_scale, b["workspace"], b["o"], b["lse"] if with_lse else None, stream=stream)
+        return b
