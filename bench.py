@@ -334,7 +334,7 @@ def run_reference(args, world, rank):
 # our arm
 # ----------------------------------------------------------------------------
 
-def measure_prefill(w, dev, steps: int, warmup: int, peaks, peak_src, dist=None):
+def measure_prefill(w, dev, steps: int, warmup: int, peaks, peak_src, dist=None, pattern=None):
     """Times `steps` prefill steps (pool + score + top-k + sparse attention)
     of workload w on one stream, the attention launch of each step between
     its own pair of events.  Returns (figures, step object)."""
@@ -345,7 +345,7 @@ def measure_prefill(w, dev, steps: int, warmup: int, peaks, peak_src, dist=None)
     import bsa_workloads as W
     inp = W.make_inputs(w, dev)
     q, k, v = inp["q"], inp["k"], inp["v"]
-    step = pipeline.PrefillStep(q, k, v, w.bs, w.kb, gated=(w.kind == "gated"))
+    step = pipeline.PrefillStep(q, k, v, w.bs, w.kb, gated=(w.kind == "gated"), pattern=pattern)
     stream = torch.cuda.current_stream()
     for _ in range(warmup):
         step.run(with_lse=False)
@@ -505,7 +505,10 @@ def run_secondaries(dev, peaks, peak_src, exclude: str):
     """One figure set per other workload, each with its own roofline, step
     time and clock samples: the other prefill workloads (gated bf16, tiny
     fp32) through measure_prefill, decode and gist decode through
-    measure_decode_like."""
+    measure_decode_like; then the widened path on the same shapes -- the
+    prefill with a sink + local + top-k pattern, decode with one budget per
+    head group, decode over a paged cache, the two-level gist decode, and the
+    backward of the gated prefill."""
     import torch
     import bsa_workloads as W
     out = {}
@@ -514,22 +517,89 @@ def run_secondaries(dev, peaks, peak_src, exclude: str):
             continue
         w = W.get(name)
         if w.kind in ("decode", "gist"):
-            fig = measure_decode_like(w, dev, SECONDARY_STEPS, SECONDARY_WARMUP, peaks, peak_src)
-            out[name] = {"metric": "us per decode step", "us_per_step": fig["us"], "attn_us": fig["attn_us"],
-                         "roofline": fig["roofline"], "clocks": fig["clocks"],
-                         "config": decode_config(w, 1), "gpu_launches_per_step": fig["launches"]}
+            out[name] = _decode_entry(w, dev, peaks, peak_src)
         else:
-            fig, step = measure_prefill(w, dev, SECONDARY_STEPS, SECONDARY_WARMUP, peaks, peak_src)
-            del step
-            out[name] = {"metric": METRIC, "value": fig["pairs"] / (fig["step_ms"] / 1e3), "unit": UNIT,
-                         "ms_per_step": fig["step_ms"], "roofline": fig["roofline"], "clocks": fig["clocks"],
-                         "config": prefill_config(w, 1), "sparsity": fig["sparsity"],
-                         "gpu_launches_per_step": 5}
+            out[name] = _prefill_entry(w, dev, peaks, peak_src)
         torch.cuda.empty_cache()
+    c2 = W.get("prefill_gqa_bf16")
+    out["prefill_gqa_bf16 pattern(sink 1, local 2, top 14)"] = _prefill_entry(c2.scaled(kb=14, name=c2.name), dev,
+                                                                               peaks, peak_src, pattern=(1, 2))
+    torch.cuda.empty_cache()
+    dec = W.get("decode_bf16")
+    out["decode_bf16 one budget per head group (96 x G)"] = _decode_entry(dec, dev, peaks, peak_src, "heads")
+    torch.cuda.empty_cache()
+    out["decode_bf16 paged (permuted pages)"] = _decode_entry(dec, dev, peaks, peak_src, "paged")
+    torch.cuda.empty_cache()
+    out["hssa_decode_bf16"] = _decode_entry(W.get("hssa_decode_bf16"), dev, peaks, peak_src)
+    torch.cuda.empty_cache()
+    out["gated_prefill_bf16 backward"] = measure_backward(W.get("gated_prefill_bf16"), dev, SECONDARY_STEPS,
+                                                          SECONDARY_WARMUP)
+    torch.cuda.empty_cache()
     return out
 
 
-def measure_decode_like(w, dev, steps: int, warmup: int, peaks, peak_src, dist=None):
+def _decode_entry(w, dev, peaks, peak_src, variant: str = ""):
+    fig = measure_decode_like(w, dev, SECONDARY_STEPS, SECONDARY_WARMUP, peaks, peak_src, variant=variant)
+    return {"metric": "us per decode step", "us_per_step": fig["us"], "attn_us": fig["attn_us"],
+            "roofline": fig["roofline"], "clocks": fig["clocks"], "config": decode_config(w, 1),
+            "gpu_launches_per_step": fig["launches"]}
+
+
+def _prefill_entry(w, dev, peaks, peak_src, pattern=None):
+    fig, step = measure_prefill(w, dev, SECONDARY_STEPS, SECONDARY_WARMUP, peaks, peak_src, pattern=pattern)
+    del step
+    config = prefill_config(w, 1)
+    if pattern is not None:
+        config["pattern"] = {"sink": pattern[0], "local": pattern[1], "top": w.kb}
+    return {"metric": METRIC, "value": fig["pairs"] / (fig["step_ms"] / 1e3), "unit": UNIT,
+            "ms_per_step": fig["step_ms"], "roofline": fig["roofline"], "clocks": fig["clocks"],
+            "config": config, "sparsity": fig["sparsity"], "gpu_launches_per_step": 5}
+
+
+def measure_backward(w, dev, steps: int, warmup: int):
+    """The backward of the gated prefill on workload w: one forward (with its
+    LSE) on the selected blocks, then `steps` timed backward calls.  FLOPs per
+    call: 10 d per causal pair (recomputed Q K^T, dO V^T, dV, dQ, dK); the
+    kernels run fp32 arithmetic on the CUDA cores, so the bound is the fp32
+    FMA rate."""
+    import torch
+    import bsa_workloads as W
+    from top_block_sparse_bsa_b200 import accounting as acc
+    from top_block_sparse_bsa_b200 import pipeline
+    inp = W.make_inputs(w, dev)
+    step = pipeline.PrefillStep(inp["q"], inp["k"], inp["v"], w.bs, w.kb, gated=(w.kind == "gated"))
+    step.run()
+    g = torch.Generator(device=dev).manual_seed(3)
+    d_o = torch.randn(inp["q"].shape, generator=g, device=dev).to(torch.bfloat16)
+    for _ in range(warmup):
+        step.backward(d_o)
+    torch.cuda.synchronize()
+    pairs = acc.prefill_pairs(step.bufs["idx"].cpu().numpy(), w.bs, w.G)
+    flops = 10.0 * w.d * pairs
+    sampler = ClockSampler(dev.index or 0).start()
+    stream = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    t0 = time.time()
+    e0.record(stream)
+    for _ in range(steps):
+        step.backward(d_o)
+    e1.record(stream)
+    wait_gpu(e1)
+    t1 = time.time()
+    sampler.stop()
+    ms = e0.elapsed_time(e1) / steps
+    achieved = flops / (ms / 1e3) / 1e12
+    del step, inp, d_o
+    return {"metric": "ms per backward call", "ms_per_call": ms, "config": prefill_config(w, 1),
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": F32_FMA_PEAK_TFLOPS, "unit": "TFLOP/s",
+                         "frac": achieved / F32_FMA_PEAK_TFLOPS, "traffic": None,
+                         "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1.965 GHz",
+                         "algorithmic_flop_per_call": flops, "kernel": "bsa_gated_attn_bwd (6 launches, fp32 SIMT)"},
+            "clocks": sampler.summary(t0, t1), "gpu_launches_per_step": 6}
+
+
+def measure_decode_like(w, dev, steps: int, warmup: int, peaks, peak_src, dist=None, variant: str = ""):
     """Decode or gist-decode workload: microseconds per step and HBM GB/s
     over the bytes the attention must read, L2 flushed before every step."""
     import torch
@@ -537,13 +607,52 @@ def measure_decode_like(w, dev, steps: int, warmup: int, peaks, peak_src, dist=N
     from top_block_sparse_bsa_b200 import pipeline
     import bsa_workloads as W
     inp = W.make_inputs(w, dev)
-    if w.kind == "decode":
+    if w.kind == "decode" and variant == "heads":
+        step = pipeline.HeadBudgetDecodeStep(inp["q"], inp["k"], inp["v"], w.bs, w.kb * w.G)
+        step.pool_cache()
+        select = step.select
+        attend = lambda: step.attend(with_lse=False)   # noqa: E731
+        launches = 5   # per-head scores, joint top-k | union lists, split-K attention, combine
+        attn_kernel = "gist_union_kernel (no gists) + attn_decode_kernel + combine_kernel"
+    elif w.kind == "decode" and variant == "paged":
+        ref = pipeline.DecodeStep(inp["q"], inp["k"], inp["v"], w.bs, w.kb)
+        ref.pool_cache()
+        nb = w.N // w.bs
+        perm = torch.from_numpy(np.random.default_rng(7).permutation(w.B * nb).astype(np.int32)).to(dev)
+        table = perm.view(w.B, nb)
+        pools = []
+        for name in ("k", "v"):
+            blocks = inp[name].view(w.B, w.Hkv, nb, w.bs, w.d).permute(0, 2, 1, 3, 4).reshape(w.B * nb, w.Hkv,
+                                                                                                w.bs, w.d)
+            pool = torch.empty_like(blocks)
+            pool[perm.long()] = blocks
+            pools.append(pool)
+            del blocks
+        kbar = ref.bufs["kbar"]
+        del ref
+        inp = {"q": inp["q"]}
+        torch.cuda.empty_cache()
+        step = pipeline.PagedDecodeStep(inp["q"], pools[0], pools[1], table, w.bs, w.kb)
+        step.bufs["kbar"].copy_(kbar)
+        del kbar
+        select = step.select
+        attend = lambda: step.attend(with_lse=False)   # noqa: E731
+        launches = 3   # fused select | split-K attention over the block table, combine
+        attn_kernel = "attn_decode_kernel (paged) + combine_kernel"
+    elif w.kind == "decode":
         step = pipeline.DecodeStep(inp["q"], inp["k"], inp["v"], w.bs, w.kb)
         step.pool_cache()
         select = step.select
         attend = lambda: step.attend(with_lse=False)   # noqa: E731
-        launches = 4   # score, top-k | split-K attention, combine
+        launches = 3   # fused score + top-k | split-K attention, combine
         attn_kernel = "attn_decode_kernel (+ combine_kernel)"
+    elif w.kind == "hssa":
+        step = pipeline.HssaStep(inp["q"], inp["k"], inp["v"], inp["gk"], inp["gv"], inp["mk"], inp["mv"], w.bs,
+                                 W.HSSA_GROUPS_KEPT, w.kb)
+        select = lambda: step.run(with_lse=False)   # noqa: E731  (the whole step in one call)
+        attend = None
+        launches = 7   # meta scores, top-km, group gist scores, top-k, union, attention, combine
+        attn_kernel = "whole two-level gist step (one call)"
     else:
         step = pipeline.GistStep(inp["q"], inp["k"], inp["v"], inp["gk"], inp["gv"], w.bs, w.kb)
         select = lambda: step.run(with_lse=False)   # noqa: E731  (the whole step in one call)
@@ -553,11 +662,16 @@ def measure_decode_like(w, dev, steps: int, warmup: int, peaks, peak_src, dist=N
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     for _ in range(warmup):
         select()
-        attend()
+        if attend is not None:
+            attend()
     torch.cuda.synchronize()
     idx = step.bufs["idx"].cpu().numpy()
-    if w.kind == "decode":
+    if w.kind == "decode" and variant == "heads":
+        nbytes = acc.heads_kv_bytes(idx, w.G, w.bs, w.d, 2)
+    elif w.kind == "decode":
         nbytes = acc.decode_kv_bytes(idx, w.bs, w.d, 2)
+    elif w.kind == "hssa":
+        nbytes = acc.hssa_kv_bytes(idx, step.bufs["meta_idx"].cpu().numpy(), w.G, w.bs, w.d, 2)
     else:
         nbytes = acc.gist_kv_bytes(idx, w.G, w.bs, w.N // w.bs, w.d, 2)
     # Each step is replayed from CUDA graphs of the C-ABI calls, L2 flushed
@@ -572,7 +686,7 @@ def measure_decode_like(w, dev, steps: int, warmup: int, peaks, peak_src, dist=N
     else:
         g_step = capture_graph(select)
     g_sel = capture_graph(select) if w.kind == "decode" else None
-    g_att = capture_graph(attend)
+    g_att = capture_graph(attend) if attend is not None else g_step
     stream = torch.cuda.current_stream()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
     sampler = ClockSampler(dev.index or 0).start()
@@ -604,6 +718,8 @@ def measure_decode_like(w, dev, steps: int, warmup: int, peaks, peak_src, dist=N
     traffic, sha = profile_traffic("attn_decode.cu", f"attn_decode_{w.name}.md")
     if sha is not None and sha != kernel_source_sha(["attn_decode.cu", "common.cuh"]):
         traffic = None
+    if variant or w.kind == "hssa":
+        traffic = None   # no committed counter summary for these variants
     roofline = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": gbs / peaks["hbm_gbs"], "traffic": traffic, "peak_source": peak_src,
                 "kernel": attn_kernel, "kernel_us": attn_us, "selected_kv_bytes_per_launch": nbytes,

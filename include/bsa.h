@@ -222,6 +222,33 @@ bsa_status_t bsa_gated_attn_fwd(const bsa_shape_t* shape, const void* q, const v
                                 void* stream);
 
 /*
+ * bsa_gated_attn_bwd -- backward of bsa_sparse_attn_prefill (sel_scores =
+ * NULL) or bsa_gated_attn_fwd: the gradients of sum(dO * O) with respect to
+ * q, k, v and, gated, the selector scores.
+ * Cite: SAS page, 核心洞察 (the continuous score injected into the attention
+ * logits lets the language-modelling loss update the context ranking by
+ * standard back-propagation) and 核心模块 2-3 (the log-form gate inside the
+ * softmax, normalised over the kept blocks and the current block).
+ * Inputs: the forward's q, k, v, idx, idx_stride, sel_scores, softmax_scale;
+ * its output o [B,Hq,N,d] (dtype) and natural-log row LSE lse [B,Hq,N] fp32
+ * (required); the upstream gradient d_o [B,Hq,N,d] (dtype).
+ * Outputs (fp32, written whole): dq [B,Hq,N,d], dk and dv [B,Hkv,N,d]; dsel
+ * [B,Hkv,nb,nb] (optional, gated only): for query block i of group g and its
+ * kept block l, d/ds[i][l] through log g_l = s_l - log sum_{kept} exp(s),
+ * zero elsewhere.  The selection itself (the hard top-k) passes no gradient.
+ * workspace: bsa_workspace_bytes_bwd(shape, idx_stride) bytes, 256-byte
+ * aligned.  Built: BF16, d = 128, block in {64, 128} (fp32 arithmetic on
+ * the CUDA cores).
+ */
+bsa_status_t bsa_gated_attn_bwd(const bsa_shape_t* shape, const void* q, const void* k, const void* v,
+                                const void* o, const float* lse, const void* d_o, const int* idx, int idx_stride,
+                                const float* sel_scores, float softmax_scale, float* dq, float* dk, float* dv,
+                                float* dsel, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Scratch bytes of bsa_gated_attn_bwd; 0 on a bad shape. */
+size_t bsa_workspace_bytes_bwd(const bsa_shape_t* shape, int idx_stride);
+
+/*
  * bsa_sparse_attn_decode -- one query token per sequence over a retained KV
  * cache, reading only the kept blocks.
  * Cite: 稀疏注意力 tutorial §5 (decode: one new query against the history);

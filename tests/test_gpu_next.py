@@ -1,7 +1,10 @@
 """GPU parity of the widened path against the CPU oracle: the fixed pattern +
 dynamic blocks selection (MInference block-sparse), one budget shared by a
 group's heads with per-head decode attention (Ada-KV), decode over a paged
-KV cache with the pooled summary kept up by appends (PagedAttention).
+KV cache with the pooled summary kept up by appends (PagedAttention),
+two-level gist routing (H-SSA), and the backward of the sparse / gated
+prefill attention (SAS: gradients reach the selector scores through the
+inner log-gate).
 
 Selections are compared bit for bit (both sides use the same fixed-order fp32
 scores); attention runs on the oracle's index sets and must be within
@@ -319,3 +322,59 @@ def test_hssa_full_size():
     sequences."""
     w = W.get("hssa_decode_bf16")
     _hssa_case(w.scaled(B=2, name=w.name), W.HSSA_GROUPS_KEPT, w.kb)
+
+
+# ----------------------------------------------------------------------------
+# backward of the sparse / gated prefill attention
+# ----------------------------------------------------------------------------
+
+def _bwd_case(w, gated, empty_frac=0.0):
+    pipe = _pipe()
+    inp = W.make_inputs(w, "cuda")
+    q, k, v = inp["q"], inp["k"], inp["v"]
+    step = pipe.PrefillStep(q, k, v, w.bs, w.kb, gated=gated)
+    step.select()
+    torch.cuda.synchronize()
+    qc, kc, vc = q.float().cpu(), k.float().cpu(), v.float().cpu()
+    _, _, s, idx, _ = oracle.prefill_select(qc, kc, w.Hkv, w.bs, w.kb)
+    if empty_frac > 0:
+        empty = np.random.default_rng(12).random(idx.shape[:3]) < empty_frac
+        idx = idx.copy()
+        idx[empty] = -1
+    idx_dev = torch.from_numpy(idx).cuda()
+    step.attend(idx=idx_dev)
+    g = torch.Generator(device="cuda").manual_seed(77)
+    d_o = torch.randn(q.shape, generator=g, device="cuda").to(torch.bfloat16)
+    step.backward(d_o, idx=idx_dev)
+    torch.cuda.synchronize()
+    _status_clean()
+    dq, dk, dv, ds = oracle.attend_prefill_bwd(qc, kc, vc, d_o.float().cpu(), w.bs, idx,
+                                               gate_scores=s if gated else None)
+    b = step.bufs
+    _assert_close(b["dq"].cpu().numpy(), dq, TOL_BF16, "dq")
+    _assert_close(b["dk"].cpu().numpy(), dk, TOL_BF16, "dk")
+    _assert_close(b["dv"].cpu().numpy(), dv, TOL_BF16, "dv")
+    if gated:
+        _assert_close(b["dsel"].cpu().numpy(), ds, TOL_BF16, "dsel")
+        kept = ds != 0
+        assert np.all(b["dsel"].cpu().numpy()[~kept] == 0.0)
+
+
+@pytest.mark.parametrize("gated", [False, True])
+@pytest.mark.parametrize("hq,hkv,bs,kb", [(4, 2, 64, 3), (5, 1, 64, 4), (7, 1, 128, 3)])
+def test_backward_small(gated, hq, hkv, bs, kb):
+    w = W.get("prefill_gqa_bf16").scaled(B=1, Hq=hq, Hkv=hkv, N=2048, bs=bs, kb=kb)
+    _bwd_case(w, gated)
+
+
+def test_backward_full_budget_and_empty_lists():
+    base = W.get("prefill_gqa_bf16")
+    _bwd_case(base.scaled(B=1, Hq=4, Hkv=1, N=2048, kb=31), gated=True)
+    _bwd_case(base.scaled(B=2, Hq=4, Hkv=2, N=2048, kb=4), gated=True, empty_frac=0.4)
+
+
+def test_backward_gated_workload_shape_sampled():
+    """The gated workload's head layout (28 query / 4 KV heads, 128-token
+    blocks, budget 8 + current) at 4096 tokens, checked element by element."""
+    w = W.get("gated_prefill_bf16").scaled(B=1, N=4096)
+    _bwd_case(w, gated=True)

@@ -14,7 +14,7 @@ BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libbsa.so")
 
 SOURCES = ["api.cu", "selector.cu", "attn_prefill.cu", "attn_prefill_split.cu", "attn_prefill_pair.cu",
-           "attn_decode.cu", "attn_f32.cu", "decode_noalloc.cu", "paged.cu"]
+           "attn_decode.cu", "attn_f32.cu", "decode_noalloc.cu", "paged.cu", "attn_bwd.cu"]
 HEADERS = ["common.cuh", "kernels.h", "tmem_wide.cuh", "topk.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

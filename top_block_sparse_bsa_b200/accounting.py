@@ -85,3 +85,31 @@ def gist_pairs(idx: np.ndarray, chunk: int, nc: int) -> int:
     idx = np.asarray(idx)
     k = (idx >= 0).sum(axis=-1)
     return int((k * chunk + (nc - k)).sum())
+
+
+def heads_kv_bytes(idx: np.ndarray, G: int, bs: int, d: int, elem: int) -> int:
+    """idx [B,Hq,stride] per-head kept blocks -> bytes of the union of each
+    (b, group)'s blocks (each gathered once for the group's heads), K and V."""
+    idx = np.asarray(idx)
+    B, Hq, _ = idx.shape
+    total = 0
+    for b in range(B):
+        for g in range(Hq // G):
+            sel = idx[b, g * G:(g + 1) * G].ravel()
+            total += len(np.unique(sel[sel >= 0]))
+    return total * bs * d * elem * 2
+
+
+def hssa_kv_bytes(chunks: np.ndarray, groups: np.ndarray, G: int, chunk: int, d: int, elem: int) -> int:
+    """Two-level gist decode: per (b, group) the union of the heads' expanded
+    chunks (chunk tokens each), the gists of the union of their kept groups
+    (64 per group) and the 64-row meta-gist tile, K and V."""
+    chunks, groups = np.asarray(chunks), np.asarray(groups)
+    B, Hq, _ = chunks.shape
+    rows = 0
+    for b in range(B):
+        for g in range(Hq // G):
+            c = chunks[b, g * G:(g + 1) * G].ravel()
+            m = groups[b, g * G:(g + 1) * G].ravel()
+            rows += len(np.unique(c[c >= 0])) * chunk + len(np.unique(m[m >= 0])) * 64 + 64
+    return rows * d * elem * 2

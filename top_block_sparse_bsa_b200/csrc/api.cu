@@ -852,4 +852,33 @@ bsa_status_t bsa_hssa_decode(const bsa_shape_t* s, const void* q, const void* k_
   return cuda_status(e);
 }
 
+size_t bsa_workspace_bytes_bwd(const bsa_shape_t* s, int idx_stride) {
+  if (check_shape(s) != BSA_OK || idx_stride < 1 || s->Nq != s->Nk) return 0;
+  return attn_bwd_workspace(s->B, s->Hq, s->Hkv, s->Nk, s->block, idx_stride);
+}
+
+bsa_status_t bsa_gated_attn_bwd(const bsa_shape_t* s, const void* q, const void* k, const void* v, const void* o,
+                                const float* lse, const void* d_o, const int* idx, int idx_stride,
+                                const float* sel_scores, float softmax_scale, float* dq, float* dk, float* dv,
+                                float* dsel, void* workspace, size_t workspace_bytes, void* stream) {
+  bsa_status_t st = check_shape(s);
+  if (st != BSA_OK) return st;
+  if (s->Nq != s->Nk) return BSA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !o || !lse || !d_o || !idx || !dq || !dk || !dv || !workspace) return BSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(d_o) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv))
+    return BSA_ERR_INVALID_ARG;
+  if (dsel && !sel_scores) return BSA_ERR_INVALID_ARG;
+  if (idx_stride < 1 || !(softmax_scale > 0.0f) || !isfinite(softmax_scale)) return BSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return BSA_ERR_INVALID_ARG;
+  if (s->dtype != BSA_BF16 || s->d != 128 || (s->block != 64 && s->block != 128)) return BSA_ERR_UNSUPPORTED;
+  if (workspace_bytes < attn_bwd_workspace(s->B, s->Hq, s->Hkv, s->Nk, s->block, idx_stride))
+    return BSA_ERR_INVALID_ARG;
+  uint32_t* status = nullptr;
+  if ((st = device_state(&status, nullptr)) != BSA_OK) return st;
+  return cuda_status(launch_attn_bwd(q, k, v, o, lse, d_o, idx, idx_stride, sel_scores, softmax_scale, s->B, s->Hq,
+                                     s->Hkv, s->Nk, s->block, dq, dk, dv, dsel, workspace, status,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -14,7 +14,7 @@ from typing import Dict, Optional, Tuple
 
 import torch
 
-from . import (BSA_OP_DECODE, BSA_OP_DECODE_HEADS, BSA_OP_GIST_DECODE, BSA_SCORE_DECODE,
+from . import (bsa_gated_attn_bwd, bsa_workspace_bytes_bwd, BSA_OP_DECODE, BSA_OP_DECODE_HEADS, BSA_OP_GIST_DECODE, BSA_SCORE_DECODE,
                BSA_SCORE_DECODE_HEADS, BSA_SCORE_PREFILL, BSA_TOPK_CAUSAL_BLOCK, bsa_decode_select,
                bsa_gated_attn_fwd, bsa_gist_expand_decode, bsa_score_blocks, bsa_sparse_attn_decode,
                bsa_hssa_decode, bsa_paged_append, bsa_sparse_attn_decode_heads, bsa_workspace_bytes_hssa, bsa_sparse_attn_decode_paged, bsa_sparse_attn_prefill,
@@ -91,6 +91,26 @@ class PrefillStep:
         self.select(stream)
         self.attend(stream=stream, with_lse=with_lse)
         return self.bufs
+
+    def backward(self, d_o: torch.Tensor, idx: Optional[torch.Tensor] = None, stream=None):
+        """Gradients of sum(d_o * O) for the last attend() (run with its LSE):
+        fp32 dq, dk, dv and, gated, dsel (the selector scores' gradient)."""
+        b = self.bufs
+        idx = b["idx"] if idx is None else idx
+        dev = _dev(self.q)
+        f32 = torch.float32
+        b.setdefault("dq", torch.empty(self.q.shape, dtype=f32, device=dev))
+        b.setdefault("dk", torch.empty(self.k.shape, dtype=f32, device=dev))
+        b.setdefault("dv", torch.empty(self.v.shape, dtype=f32, device=dev))
+        if self.gated:
+            b.setdefault("dsel", torch.empty(b["scores"].shape, dtype=f32, device=dev))
+        ws = bsa_workspace_bytes_bwd(self.shape, idx.shape[-1])
+        if "bwd_workspace" not in b or b["bwd_workspace"].numel() < ws:
+            b["bwd_workspace"] = torch.empty((max(ws, 256),), dtype=torch.uint8, device=dev)
+        bsa_gated_attn_bwd(self.shape, self.q, self.k, self.v, b["o"], b["lse"], d_o, idx, idx.shape[-1],
+                           b["scores"] if self.gated else None, self.softmax_scale, b["dq"], b["dk"], b["dv"],
+                           b["dsel"] if self.gated else None, b["bwd_workspace"], stream=stream)
+        return b
 
 
 @dataclass
