@@ -55,6 +55,10 @@ def parse_args():
     ap.add_argument("--no-secondary", action="store_true", help="skip the other workloads' figures")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=0, help="override the workload batch (small profiling cases)")
+    ap.add_argument("--variant", default="", choices=["", "pattern", "backward", "heads", "paged"],
+                    help="a widened-path variant of the workload: prefill with the sink + local + top-k pattern, "
+                         "the backward of the gated prefill, decode with one budget per head group, decode over "
+                         "a paged cache")
     return ap.parse_args()
 
 
@@ -428,7 +432,18 @@ def run_prefill(args, world, rank, local, peaks, peak_src):
     if args.batch:
         base = base.scaled(B=args.batch, name=base.name)
     w = rank_workload(base, rank)
-    fig, step = measure_prefill(w, dev, args.steps, args.warmup, peaks, peak_src, dist)
+    if args.variant == "backward":
+        fig = measure_backward(w, dev, args.steps, args.warmup)
+        close_ranks(dist)
+        if rank == 0:
+            print(json.dumps(dict(fig, variant="backward", n_gpus=world, steps=args.steps, warmup=args.warmup,
+                                  higher_is_better=False, data="synthetic")), flush=True)
+        return 0
+    pattern = None
+    if args.variant == "pattern":
+        w = w.scaled(kb=w.kb - 2, name=w.name)
+        pattern = (1, 2)
+    fig, step = measure_prefill(w, dev, args.steps, args.warmup, peaks, peak_src, dist, pattern=pattern)
     pairs = fig["pairs"]
     # whole job: the slowest rank's step, the pairs of every rank's problem
     step_ms, job_pairs = reduce_over_ranks(dist, fig["step_ms"], pairs, device=dev)
@@ -740,7 +755,7 @@ def run_decode_like(args, world, rank, local, peaks, peak_src):
     if args.batch:
         base = base.scaled(B=args.batch, name=base.name)
     w = rank_workload(base, rank)
-    fig = measure_decode_like(w, dev, args.steps, args.warmup, peaks, peak_src, dist)
+    fig = measure_decode_like(w, dev, args.steps, args.warmup, peaks, peak_src, dist, variant=args.variant)
     # whole job: every rank runs its own batch; a step takes the slowest rank's time
     us, _ = reduce_over_ranks(dist, fig["us"], 1.0, device=dev)
     attn_us, _ = reduce_over_ranks(dist, fig["attn_us"], 1.0, device=dev)
@@ -770,7 +785,7 @@ def main():
         return run_reference(args, world, rank)
     peaks, src = load_peaks()
     import bsa_workloads as W
-    if W.get(args.config).kind in ("decode", "gist"):
+    if W.get(args.config).kind in ("decode", "gist", "hssa"):
         return run_decode_like(args, world, rank, local, peaks, src)
     return run_prefill(args, world, rank, local, peaks, src)
 
