@@ -433,7 +433,7 @@ def run_prefill(args, world, rank, local, peaks, peak_src):
         base = base.scaled(B=args.batch, name=base.name)
     w = rank_workload(base, rank)
     if args.variant == "backward":
-        fig = measure_backward(w, dev, args.steps, args.warmup)
+        fig = measure_backward(w, dev, args.steps, args.warmup, peaks, peak_src)
         close_ranks(dist)
         if rank == 0:
             print(json.dumps(dict(fig, variant="backward", n_gpus=world, steps=args.steps, warmup=args.warmup,
@@ -548,7 +548,7 @@ def run_secondaries(dev, peaks, peak_src, exclude: str):
     out["hssa_decode_bf16"] = _decode_entry(W.get("hssa_decode_bf16"), dev, peaks, peak_src)
     torch.cuda.empty_cache()
     out["gated_prefill_bf16 backward"] = measure_backward(W.get("gated_prefill_bf16"), dev, SECONDARY_STEPS,
-                                                          SECONDARY_WARMUP)
+                                                          SECONDARY_WARMUP, peaks, peak_src)
     torch.cuda.empty_cache()
     return out
 
@@ -571,12 +571,14 @@ def _prefill_entry(w, dev, peaks, peak_src, pattern=None):
             "config": config, "sparsity": fig["sparsity"], "gpu_launches_per_step": 5}
 
 
-def measure_backward(w, dev, steps: int, warmup: int):
+def measure_backward(w, dev, steps: int, warmup: int, peaks, peak_src):
     """The backward of the gated prefill on workload w: one forward (with its
     LSE) on the selected blocks, then `steps` timed backward calls.  FLOPs per
-    call: 10 d per causal pair (recomputed Q K^T, dO V^T, dV, dQ, dK); the
-    kernels run fp32 arithmetic on the CUDA cores, so the bound is the fp32
-    FMA rate."""
+    call: 10 d per causal pair (Q K^T, dO V^T, dV, dQ, dK; the recomputation
+    of Q K^T and dO V^T in the second pass and the query-major pass's extra
+    sweep that forms D are not counted); the products run on the bf16 tensor
+    cores, so the bound is the measured bf16 GEMM rate (burst: the call is
+    timed alone)."""
     import torch
     import bsa_workloads as W
     from top_block_sparse_bsa_b200 import accounting as acc
@@ -605,13 +607,14 @@ def measure_backward(w, dev, steps: int, warmup: int):
     sampler.stop()
     ms = e0.elapsed_time(e1) / steps
     achieved = flops / (ms / 1e3) / 1e12
+    peak = peaks["bf16_tflops"]
     del step, inp, d_o
     return {"metric": "ms per backward call", "ms_per_call": ms, "config": prefill_config(w, 1),
-            "roofline": {"bound": "alu", "achieved": achieved, "peak": F32_FMA_PEAK_TFLOPS, "unit": "TFLOP/s",
-                         "frac": achieved / F32_FMA_PEAK_TFLOPS, "traffic": None,
-                         "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1.965 GHz",
-                         "algorithmic_flop_per_call": flops, "kernel": "bsa_gated_attn_bwd (6 launches, fp32 SIMT)"},
-            "clocks": sampler.summary(t0, t1), "gpu_launches_per_step": 6}
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": None, "peak_source": peak_src,
+                         "algorithmic_flop_per_call": flops,
+                         "kernel": "bsa_gated_attn_bwd (5 launches: gate, transpose, dq_tc, dkv_tc, dsel)"},
+            "clocks": sampler.summary(t0, t1), "gpu_launches_per_step": 5}
 
 
 def measure_decode_like(w, dev, steps: int, warmup: int, peaks, peak_src, dist=None, variant: str = ""):

@@ -230,18 +230,23 @@ bsa_status_t bsa_gated_attn_fwd(const bsa_shape_t* shape, const void* q, const v
  * standard back-propagation) and 核心模块 2-3 (the log-form gate inside the
  * softmax, normalised over the kept blocks and the current block).
  * Inputs: the forward's q, k, v, idx, idx_stride, sel_scores, softmax_scale;
- * its output o [B,Hq,N,d] (dtype) and natural-log row LSE lse [B,Hq,N] fp32
- * (required); the upstream gradient d_o [B,Hq,N,d] (dtype).
+ * its natural-log row LSE lse [B,Hq,N] fp32 (required); the upstream
+ * gradient d_o [B,Hq,N,d] (dtype).  The forward's output O is not an input:
+ * the row term D_t = dO_t . O_t is formed as sum_u P_{t,u} (dO_t . v_u) from
+ * the recomputed probabilities, so the bf16 rounding of the stored O does not
+ * enter the gradients.
  * Outputs (fp32, written whole): dq [B,Hq,N,d], dk and dv [B,Hkv,N,d]; dsel
  * [B,Hkv,nb,nb] (optional, gated only): for query block i of group g and its
  * kept block l, d/ds[i][l] through log g_l = s_l - log sum_{kept} exp(s),
  * zero elsewhere.  The selection itself (the hard top-k) passes no gradient.
  * workspace: bsa_workspace_bytes_bwd(shape, idx_stride) bytes, 256-byte
- * aligned.  Built: BF16, d = 128, block in {64, 128} (fp32 arithmetic on
- * the CUDA cores).
+ * aligned.  Built: BF16, d = 128, block in {64, 128}, idx_stride <= 256
+ * (BSA_ERR_UNSUPPORTED otherwise); tcgen05 MMAs with fp32 accumulation, P and
+ * dS rounded to bf16 as MMA operands, D and the selector-score gradient
+ * summed in fp32 from the unrounded values.
  */
 bsa_status_t bsa_gated_attn_bwd(const bsa_shape_t* shape, const void* q, const void* k, const void* v,
-                                const void* o, const float* lse, const void* d_o, const int* idx, int idx_stride,
+                                const float* lse, const void* d_o, const int* idx, int idx_stride,
                                 const float* sel_scores, float softmax_scale, float* dq, float* dk, float* dv,
                                 float* dsel, void* workspace, size_t workspace_bytes, void* stream);
 

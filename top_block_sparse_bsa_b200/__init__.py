@@ -79,7 +79,7 @@ _SIGS = {
     "bsa_hssa_decode": (_i, [ctypes.POINTER(BsaShape), _p, _p, _p, _p, _p, _p, _p, _i, _i, _p, _p, ctypes.c_float,
                              _p, ctypes.c_size_t, _p, _p, _p]),
     "bsa_workspace_bytes_hssa": (ctypes.c_size_t, [ctypes.POINTER(BsaShape), _i, _i]),
-    "bsa_gated_attn_bwd": (_i, [ctypes.POINTER(BsaShape), _p, _p, _p, _p, _p, _p, _p, _i, _p, ctypes.c_float, _p, _p,
+    "bsa_gated_attn_bwd": (_i, [ctypes.POINTER(BsaShape), _p, _p, _p, _p, _p, _p, _i, _p, ctypes.c_float, _p, _p,
                                 _p, _p, _p, ctypes.c_size_t, _p]),
     "bsa_workspace_bytes_bwd": (ctypes.c_size_t, [ctypes.POINTER(BsaShape), _i]),
     "bsa_topk_select_joint_heads": (_i, [_p, _i, _i, _i, _i, _p, _i, _p, _p]),
@@ -261,11 +261,11 @@ def bsa_workspace_bytes_hssa(shape: BsaShape, km: int, topk: int) -> int:
     return int(lib.bsa_workspace_bytes_hssa(ctypes.byref(shape), int(km), int(topk)))
 
 
-def bsa_gated_attn_bwd(shape: BsaShape, q, k, v, o, lse, d_o, idx, idx_stride: int, sel_scores, softmax_scale: float,
+def bsa_gated_attn_bwd(shape: BsaShape, q, k, v, lse, d_o, idx, idx_stride: int, sel_scores, softmax_scale: float,
                        dq, dk, dv, dsel=None, workspace=None, stream=None) -> None:
     """Backward of the sparse (sel_scores None) or gated prefill attention: fp32 dq, dk, dv (and dsel)."""
     _check("bsa_gated_attn_bwd", lib.bsa_gated_attn_bwd(
-        ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(d_o), _ptr(idx), int(idx_stride),
+        ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(lse), _ptr(d_o), _ptr(idx), int(idx_stride),
         _ptr(sel_scores), ctypes.c_float(softmax_scale), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dsel), _ptr(workspace),
         ctypes.c_size_t(workspace.numel() * workspace.element_size() if workspace is not None else 0),
         _stream(stream)))

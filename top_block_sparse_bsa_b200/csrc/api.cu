@@ -857,27 +857,34 @@ size_t bsa_workspace_bytes_bwd(const bsa_shape_t* s, int idx_stride) {
   return attn_bwd_workspace(s->B, s->Hq, s->Hkv, s->Nk, s->block, idx_stride);
 }
 
-bsa_status_t bsa_gated_attn_bwd(const bsa_shape_t* s, const void* q, const void* k, const void* v, const void* o,
+bsa_status_t bsa_gated_attn_bwd(const bsa_shape_t* s, const void* q, const void* k, const void* v,
                                 const float* lse, const void* d_o, const int* idx, int idx_stride,
                                 const float* sel_scores, float softmax_scale, float* dq, float* dk, float* dv,
                                 float* dsel, void* workspace, size_t workspace_bytes, void* stream) {
   bsa_status_t st = check_shape(s);
   if (st != BSA_OK) return st;
   if (s->Nq != s->Nk) return BSA_ERR_INVALID_ARG;
-  if (!q || !k || !v || !o || !lse || !d_o || !idx || !dq || !dk || !dv || !workspace) return BSA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(d_o) || !aligned16(dq) ||
+  if (!q || !k || !v || !lse || !d_o || !idx || !dq || !dk || !dv || !workspace) return BSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(d_o) || !aligned16(dq) ||
       !aligned16(dk) || !aligned16(dv))
     return BSA_ERR_INVALID_ARG;
   if (dsel && !sel_scores) return BSA_ERR_INVALID_ARG;
   if (idx_stride < 1 || !(softmax_scale > 0.0f) || !isfinite(softmax_scale)) return BSA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return BSA_ERR_INVALID_ARG;
   if (s->dtype != BSA_BF16 || s->d != 128 || (s->block != 64 && s->block != 128)) return BSA_ERR_UNSUPPORTED;
+  if (idx_stride > 256) return BSA_ERR_UNSUPPORTED;   // the dQ pass keeps per-slot sums for 256 slots
   if (workspace_bytes < attn_bwd_workspace(s->B, s->Hq, s->Hkv, s->Nk, s->block, idx_stride))
     return BSA_ERR_INVALID_ARG;
   uint32_t* status = nullptr;
-  if ((st = device_state(&status, nullptr)) != BSA_OK) return st;
-  return cuda_status(launch_attn_bwd(q, k, v, o, lse, d_o, idx, idx_stride, sel_scores, softmax_scale, s->B, s->Hq,
-                                     s->Hkv, s->Nk, s->block, dq, dk, dv, dsel, workspace, status,
+  int sms = 0;
+  if ((st = device_state(&status, &sms)) != BSA_OK) return st;
+  CUtensorMap mq, mdo, mk, mv;
+  const uint64_t qrows = static_cast<uint64_t>(s->B) * s->Hq * s->Nk, kvrows = static_cast<uint64_t>(s->B) * s->Hkv * s->Nk;
+  if (!make_map_bf16(&mq, q, qrows, 64) || !make_map_bf16(&mdo, d_o, qrows, 64) ||
+      !make_map_bf16(&mk, k, kvrows, 64) || !make_map_bf16(&mv, v, kvrows, 64))
+    return BSA_ERR_CUDA;
+  return cuda_status(launch_attn_bwd(&mq, &mdo, &mk, &mv, lse, idx, idx_stride, sel_scores, softmax_scale, s->B,
+                                     s->Hq, s->Hkv, s->Nk, s->block, dq, dk, dv, dsel, workspace, status, sms,
                                      static_cast<cudaStream_t>(stream)));
 }
 

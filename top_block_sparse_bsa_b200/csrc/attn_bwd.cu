@@ -1,5 +1,6 @@
 // attn_bwd.cu -- backward of the block-sparse (and SAS gated) prefill
-// attention, bf16 inputs, d = 128, fp32 arithmetic on the CUDA cores.
+// attention, bf16 inputs, d = 128, on sm_100a tensor cores (tcgen05 MMA into
+// tensor memory, TMA tile loads).
 //
 // What it computes (SAS page, 核心洞察 and 核心模块 2: the selector's
 // continuous score sits inside the softmax logits in log form, so the
@@ -7,21 +8,35 @@
 // forward's P_{t,u} = exp(scale q_t.k_u + log g_{j(u)} - LSE_t) over the kept,
 // causal keys of row t (LSE_t: the forward's natural-log row LSE) and the
 // upstream gradient dO:
-//   D_t      = dO_t . O_t
-//   dl_{t,u} = P_{t,u} (dO_t . v_u - D_t)
-//   dQ_t     = scale sum_u dl_{t,u} k_u           (query-block-major pass)
-//   dK_u     = scale sum_t dl_{t,u} q_t,  dV_u = sum_t P_{t,u} dO_t
-//                                                 (key-block-major pass)
+//   D_t      = sum_u P_{t,u} (dO_t . v_u)        (= dO_t . O_t in exact arithmetic;
+//              formed from P and V rather than from the stored bf16 O, whose
+//              rounding would otherwise enter every gradient through D)
+//   dS_{t,u} = P_{t,u} (dO_t . v_u - D_t)
+//   dQ_t     = scale sum_u dS_{t,u} k_u
+//   dK_u     = scale sum_t dS_{t,u} q_t,  dV_u = sum_t P_{t,u} dO_t
 //   for a unit (b, g, i) and its kept block l:
 //   dsel_l   = dlogg_l - g_l sum_j dlogg_j,  dlogg_j = sum over the unit's
-//              rows t and block j's keys u of dl_{t,u}.
-// Both passes recompute P from Q, K and the saved LSE (no n x n storage);
-// the key-block-major pass walks, for each key block, the query blocks that
-// kept it (a transposed index built first), so no output is accumulated by
-// atomics and every sum runs in a fixed order.
+//              rows t and block j's keys u of dS_{t,u}.
+// P is recomputed from Q, K and the saved LSE (no n x n storage).  Two
+// passes, neither accumulating by atomics, every sum in a fixed order:
+//   query-major (dq_tc_kernel): per 128-row tile of a unit (the unit's G
+//     heads' rows stacked, as in the forward), two sweeps over its kept
+//     blocks: S = Q K^T and dP = dO V^T on the tensor core, the first sweep
+//     sums D_t, the second writes dS (bf16) over S in tensor memory and
+//     accumulates dQ += dS K there, plus the rows' share of dlogg;
+//   key-major (dkv_tc_kernel): per key block j, every (query block i that
+//     kept j, 128 of its rows): S^T = K Q^T and dP^T = V dO^T, then P^T and
+//     dS^T (bf16) over them, dV += P^T dO and dK += dS^T Q accumulated in
+//     tensor memory over all of them (a transposed index, built first, lists
+//     the query blocks of each key block).
+// P and dS enter the dQ/dK/dV products rounded to bf16, as the forward's P
+// enters O += P V; D and dlogg are summed in fp32 from the unrounded values.
 //
-// Threads: four per row (dQ pass) or per key (dK/dV pass), each holding 32
-// of the 128 channels; dot products are finished with two shuffles.
+// Roles of both kernels (192 threads): warps 0-3 one TMEM lane each (a row
+// in the query-major pass, a key in the key-major one), warp 4 one thread
+// issuing the MMAs, warp 5 one thread issuing the TMA loads.  Waits are
+// bounded (mbarrier try-wait with a clock budget); a wait that gives up
+// raises the CTA's abort flag and the device status word.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -29,45 +44,16 @@ namespace bsa {
 namespace bwd {
 
 constexpr int kD = 128;
-constexpr int kRows = 64;          // rows (dQ pass) or keys (dK/dV pass) per CTA
-constexpr int kThreads = 4 * kRows;
+constexpr int kMaxList = 256;
+constexpr int kThreadsTC = 192;
+constexpr uint32_t kHalf = 128u * 128u;   // 128 rows x 64 bf16 (one swizzle span)
+constexpr uint32_t kTile = 2u * kHalf;    // 128 rows x 128 bf16
+constexpr float kLog2e = 1.44269504088896340736f;
 
-__device__ __forceinline__ float quad_sum(float x) {
-  x += __shfl_xor_sync(0xffffffffu, x, 1);
-  x += __shfl_xor_sync(0xffffffffu, x, 2);
-  return x;
-}
-
-__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&x)[32]) {
-  const uint4* p = reinterpret_cast<const uint4*>(src);
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const uint4 w = __ldg(p + e);
-    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      x[8 * e + 2 * i] = __uint_as_float(ws[i] << 16);
-      x[8 * e + 2 * i + 1] = __uint_as_float(ws[i] & 0xFFFF0000u);
-    }
-  }
-}
-
-// D_t = dO_t . O_t, one warp per row.
-__global__ void rowdot_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ d_o,
-                              int64_t rows, float* __restrict__ D) {
-  const int64_t r = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (r >= rows) return;
-  const __nv_bfloat162 a0 = reinterpret_cast<const __nv_bfloat162*>(o + r * kD)[lane * 2];
-  const __nv_bfloat162 a1 = reinterpret_cast<const __nv_bfloat162*>(o + r * kD)[lane * 2 + 1];
-  const __nv_bfloat162 b0 = reinterpret_cast<const __nv_bfloat162*>(d_o + r * kD)[lane * 2];
-  const __nv_bfloat162 b1 = reinterpret_cast<const __nv_bfloat162*>(d_o + r * kD)[lane * 2 + 1];
-  const float2 fa0 = __bfloat1622float2(a0), fa1 = __bfloat1622float2(a1);
-  const float2 fb0 = __bfloat1622float2(b0), fb1 = __bfloat1622float2(b1);
-  float acc = fa0.x * fb0.x + fa0.y * fb0.y + fa1.x * fb1.x + fa1.y * fb1.y;
-#pragma unroll
-  for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (lane == 0) D[r] = acc;
+// A wait by a whole warp: every lane polls, all agree on the outcome.
+__device__ __forceinline__ bool warp_wait_all(uint32_t bar, uint32_t parity, volatile int* ab, uint32_t* st) {
+  bool ok = mbar_wait(bar, parity, ab, st);
+  return __all_sync(0xffffffffu, ok);
 }
 
 // Per unit (b, g, i): its kept list (validated as the forward does) and, per
@@ -143,200 +129,639 @@ __global__ void transpose_kernel(const int* __restrict__ lists, const int* __res
 }
 
 struct Params {
-  const __nv_bfloat16 *q, *k, *v, *d_o;
-  const float *lse, *D, *logg;
+  const float *lse, *logg;
   const int *lists, *counts, *toff;
   const int2* tlist;
-  int B, Hq, Hkv, N, nb, G, bs, idx_stride, chunks;   // chunks: 64-row chunks per unit
+  float* D;                 // written by the query-major pass, read by the key-major pass
+  float* dlogg_part;        // [units][idx_stride][tiles]
+  int B, Hq, Hkv, N, nb, G, idx_stride, tiles;   // tiles: 128-row tiles per unit
   float scale;
-  float *dq, *dk, *dv, *dlogg_part;                    // dlogg_part [units][idx_stride][chunks]
+  float *dq, *dk, *dv;
+  uint32_t* status;
 };
 
-// dQ pass.  CTA = (unit, chunk of 64 of its G*bs stacked rows); thread
-// (row, quarter).  Every kept block of the unit in list order; its keys are
-// staged in shared memory as fp32, 64 at a time.
-constexpr size_t kTileSmem = 2 * static_cast<size_t>(kRows) * (kD + 4) * sizeof(float);
+// ------------------------------------------------------------------ query-major
+namespace qm {
+constexpr uint32_t SM_Q = 0, SM_DO = kTile, SM_K = 2 * kTile, SM_V = 4 * kTile;   // K, V: two stages each
+constexpr uint32_t SM_RED = 6 * kTile;                                            // float [4][kMaxList]
+constexpr uint32_t SM_BAR = SM_RED + 4 * kMaxList * 4;
+enum { QF = 0, QE, KF, KE = KF + 2, SF = KE + 2, PF, OF, OE, RS, NBAR };   // RS: dlogg sums written
+constexpr uint32_t SM_MISC = SM_BAR + NBAR * 8;   // tmem base, abort flag
+constexpr uint32_t kSmem = SM_MISC + 16 + 1024;
+}  // namespace qm
 
-__global__ void __launch_bounds__(kThreads) dq_kernel(const Params p) {
-  extern __shared__ __align__(16) float dq_sm[];
-  float (*ks)[kD + 4] = reinterpret_cast<float (*)[kD + 4]>(dq_sm);
-  float (*vs)[kD + 4] = reinterpret_cast<float (*)[kD + 4]>(dq_sm + kRows * (kD + 4));
-  __shared__ float red[kThreads / 32];
-  const int64_t unit = blockIdx.x / p.chunks;
-  const int chunk = static_cast<int>(blockIdx.x % p.chunks);
-  const int64_t bg = unit / p.nb;
-  const int i = static_cast<int>(unit % p.nb);
-  const int b = static_cast<int>(bg / p.Hkv), g = static_cast<int>(bg % p.Hkv);
-  const int rl = threadIdx.x >> 2, qt = threadIdx.x & 3;
-  const int R = chunk * kRows + rl;
-  const bool valid = R < p.G * p.bs;
-  const int h = g * p.G + (valid ? R / p.bs : 0);
-  const int t = i * p.bs + R % p.bs;
-  const int64_t row = (static_cast<int64_t>(b) * p.Hq + h) * p.N + t;
-  float qv[32], dov[32], dq[32];
-  if (valid) {
-    load_bf16x32(p.q + row * kD + qt * 32, qv);
-    load_bf16x32(p.d_o + row * kD + qt * 32, dov);
+template <int BS>
+__global__ void __launch_bounds__(kThreadsTC, 1)
+    dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
+                 const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const Params p) {
+  using namespace qm;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  auto bar = [&](int b) -> uint32_t { return sb + SM_BAR + 8u * b; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM_MISC);
+  volatile int* abortp = reinterpret_cast<volatile int*>(smem + SM_MISC + 4);
+  float* red = reinterpret_cast<float*>(smem + SM_RED);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rows_per_unit = p.G * BS;
+  const int64_t units = static_cast<int64_t>(p.B) * p.Hkv * p.nb;
+  const int64_t items = units * p.tiles;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(QF), 1);
+    mbar_init(bar(QE), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(KF + s), 1);
+      mbar_init(bar(KE + s), 1);
+    }
+    mbar_init(bar(SF), 1);
+    mbar_init(bar(PF), 4);
+    mbar_init(bar(OF), 1);
+    mbar_init(bar(OE), 4);
+    mbar_init(bar(RS), 128);
+    *abortp = 0;
+    fence_barrier_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;   // S | dP | dQ
+  auto item_unit = [&](int64_t item, int& tile, int64_t& bg, int& i) {
+    const int64_t unit = item / p.tiles;
+    tile = static_cast<int>(item % p.tiles);
+    bg = unit / p.nb;
+    i = p.nb - 1 - static_cast<int>(unit % p.nb);   // heavy (late) query blocks first
+    return bg * p.nb + i;
+  };
+
+  if (warp == 5) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      int gs = 0, qc = 0;
+      bool ok = true;
+      for (int64_t item = blockIdx.x; ok && item < items; item += gridDim.x) {
+        int tile, i;
+        int64_t bg;
+        const int64_t unit = item_unit(item, tile, bg, i);
+        const int n = p.counts[unit];
+        if (n == 0) continue;
+        const int b = static_cast<int>(bg / p.Hkv), g = static_cast<int>(bg % p.Hkv);
+        if (qc > 0 && !(ok = mbar_wait(bar(QE), (qc - 1) & 1, abortp, p.status))) break;
+        uint32_t bytes = 0;
+        for (int pc = 0; pc < 2; ++pc)
+          if (tile * 128 + pc * 64 < rows_per_unit) bytes += 4 * 8192;
+        mbar_arrive_expect_tx(bar(QF), bytes);
+        for (int pc = 0; pc < 2; ++pc) {
+          const int R0 = tile * 128 + pc * 64;
+          if (R0 >= rows_per_unit) continue;
+          const int h = g * p.G + R0 / BS;
+          const int y = (b * p.Hq + h) * p.N + i * BS + R0 % BS;
+          for (int hf = 0; hf < 2; ++hf) {
+            tma_load_2d(sb + SM_Q + hf * kHalf + pc * 8192, &tmQ, bar(QF), hf * 64, y);
+            tma_load_2d(sb + SM_DO + hf * kHalf + pc * 8192, &tmDO, bar(QF), hf * 64, y);
+          }
+        }
+        ++qc;
+        const int* list = p.lists + unit * p.idx_stride;
+        const int kvrow0 = static_cast<int>(bg) * p.N;
+        const int nsteps = (BS == 64) ? (n + 1) / 2 : n;
+        for (int sw = 0; ok && sw < 2; ++sw)
+          for (int s = 0; s < nsteps; ++s, ++gs) {
+            const int st = gs & 1, use = gs >> 1;
+            int jb[2] = {list[(BS == 64) ? 2 * s : s], 0};
+            const int nblk = (BS == 64 && 2 * s + 1 < n) ? 2 : 1;
+            if (nblk == 2) jb[1] = list[2 * s + 1];
+            if (gs >= 2 && !(ok = mbar_wait(bar(KE + st), (use - 1) & 1, abortp, p.status))) break;
+            mbar_arrive_expect_tx(bar(KF + st), static_cast<uint32_t>(nblk * BS) * 512u);
+            for (int bl = 0; bl < nblk; ++bl)
+              for (int r = 0; r < BS / 64; ++r) {
+                const uint32_t rowoff = static_cast<uint32_t>(bl * BS + r * 64) * 128u;
+                const int y = kvrow0 + jb[bl] * BS + r * 64;
+                for (int hf = 0; hf < 2; ++hf) {
+                  tma_load_2d(sb + SM_K + st * kTile + hf * kHalf + rowoff, &tmK, bar(KF + st), hf * 64, y);
+                  tma_load_2d(sb + SM_V + st * kTile + hf * kHalf + rowoff, &tmV, bar(KF + st), hf * 64, y);
+                }
+              }
+          }
+      }
+      if (*abortp) {
+        if (qc > 0) mbar_drain(bar(QF), (qc - 1) & 1);
+        for (int s = max(0, gs - 2); s < gs; ++s) mbar_drain(bar(KF + (s & 1)), (s >> 1) & 1);
+      }
+    }
+  } else if (warp == 4) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      const uint32_t id128 = idesc_bf16_f32(128, 128, 0, 0);
+      const uint32_t id64 = idesc_bf16_f32(128, 64, 0, 0);
+      const uint32_t id_mn = idesc_bf16_f32(128, 128, 0, 1);
+      const uint64_t qd = smem_desc_sw128(sb + SM_Q, 16, 1024);
+      const uint64_t dod = smem_desc_sw128(sb + SM_DO, 16, 1024);
+      const uint64_t kd0 = smem_desc_sw128(sb + SM_K, 16, 1024);
+      const uint64_t vd0 = smem_desc_sw128(sb + SM_V, 16, 1024);
+      const uint64_t kmn0 = smem_desc_sw128(sb + SM_K, kHalf, 1024);
+      const uint32_t tS = tmem, tP = tmem + 128, tQ = tmem + 256;
+      int gs = 0, qc = 0, sf = 0, done = 0;
+      bool ok = true, pf_pending = false;
+      for (int64_t item = blockIdx.x; ok && item < items; item += gridDim.x) {
+        int tile, i;
+        int64_t bg;
+        const int64_t unit = item_unit(item, tile, bg, i);
+        const int n = p.counts[unit];
+        if (n == 0) continue;
+        const int nsteps = (BS == 64) ? (n + 1) / 2 : n;
+        if (!(ok = mbar_wait(bar(QF), qc & 1, abortp, p.status))) break;
+        ++qc;
+        tc_fence_after();
+        for (int sw = 0; ok && sw < 2; ++sw)
+          for (int s = 0; s < nsteps; ++s, ++gs) {
+            const int st = gs & 1, use = gs >> 1;
+            const int keys = (BS == 64 && 2 * s + 1 >= n) ? 64 : 128;
+            // S and dP are overwritten: the lanes must be done with the previous ones
+            if (pf_pending && !(ok = mbar_wait(bar(PF), (sf - 1) & 1, abortp, p.status))) break;
+            pf_pending = false;
+            if (!(ok = mbar_wait(bar(KF + st), use & 1, abortp, p.status))) break;
+            tc_fence_after();
+            const uint64_t kd = kd0 + ((st * kTile) >> 4), vd = vd0 + ((st * kTile) >> 4);
+            const uint32_t id = (keys == 128) ? id128 : id64;
+#pragma unroll
+            for (int kk = 0; kk < kD / 16; ++kk) {
+              const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
+              mma_ss(tS, qd + off, kd + off, id, kk > 0 ? 1u : 0u);
+            }
+#pragma unroll
+            for (int kk = 0; kk < kD / 16; ++kk) {
+              const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
+              mma_ss(tP, dod + off, vd + off, id, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(bar(SF));
+            ++sf;
+            if (sw == 0) {
+              tc_commit(bar(KE + st));
+              pf_pending = true;
+              continue;
+            }
+            // second sweep: dQ += dS K once the lanes have written dS over S
+            if (!(ok = mbar_wait(bar(PF), (sf - 1) & 1, abortp, p.status))) break;
+            if (s == 0 && done > 0 && !(ok = mbar_wait(bar(OE), (done - 1) & 1, abortp, p.status))) break;
+            tc_fence_after();
+            const uint64_t kmn = kmn0 + ((st * kTile) >> 4);
+            for (int kk = 0; kk < keys / 16; ++kk)
+              mma_ts(tQ, tS + kk * 8, kmn + ((kk * 2048) >> 4), id_mn, (s > 0 || kk > 0) ? 1u : 0u);
+            tc_commit(bar(KE + st));
+          }
+        if (!ok) break;
+        tc_commit(bar(OF));
+        tc_commit(bar(QE));
+        ++done;
+      }
+      if (!ok) {
+        // every MMA issued so far must finish before tensor memory is freed
+        tc_commit(bar(OF));
+        mbar_drain(bar(OF), done & 1);
+      }
+    }
   } else {
+    // ------------------------------------------------ lanes (one row each)
+    const int r = warp * 32 + lane;
+    const uint32_t la = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t tS = la, tP = la + 128, tQ = la + 256;
+    const float scale2 = p.scale * kLog2e;
+    int sf = 0, done = 0, rs = 0;
+    bool ok = true;
+    for (int64_t item = blockIdx.x; ok && item < items; item += gridDim.x) {
+      int tile, i;
+      int64_t bg;
+      const int64_t unit = item_unit(item, tile, bg, i);
+      const int n = p.counts[unit];
+      const int b = static_cast<int>(bg / p.Hkv), g = static_cast<int>(bg % p.Hkv);
+      const int R = tile * 128 + r;
+      const bool valid = R < rows_per_unit;
+      const int h = g * p.G + (valid ? R / BS : 0);
+      const int tb = R % BS;
+      const int64_t row = (static_cast<int64_t>(b) * p.Hq + h) * p.N + static_cast<int64_t>(i) * BS + tb;
+      if (n == 0) {
+        if (valid) {
+          float4* dst = reinterpret_cast<float4*>(p.dq + row * kD);
+          for (int c = 0; c < kD / 4; ++c) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+          p.D[row] = 0.0f;
+        }
+        continue;
+      }
+      const float lse = valid ? p.lse[row] : -INFINITY;
+      const bool live = valid && lse > -INFINITY;
+      const float lse2 = live ? lse * kLog2e : 0.0f;
+      const int* list = p.lists + unit * p.idx_stride;
+      const float* lg = p.logg + unit * p.idx_stride;
+      const int nsteps = (BS == 64) ? (n + 1) / 2 : n;
+      float Dt = 0.0f;
+      for (int sw = 0; ok && sw < 2; ++sw) {
+        for (int s = 0; s < nsteps; ++s) {
+          const int s0 = (BS == 64) ? 2 * s : s;
+          const int nblk = (BS == 64 && s0 + 1 < n) ? 2 : 1;
+          const int keys = nblk * BS > 128 ? 128 : nblk * BS;
+          const int j0 = list[s0], j1 = (nblk == 2) ? list[s0 + 1] : -1;
+          const float off0 = lg[s0] * kLog2e - lse2;
+          const float off1 = (nblk == 2) ? lg[s0 + 1] * kLog2e - lse2 : 0.0f;
+          if (!(ok = warp_wait_all(bar(SF), sf & 1, abortp, p.status))) break;
+          ++sf;
+          tc_fence_after();
+          float dl0 = 0.0f, dl1 = 0.0f;
+          for (int part = 0; part < keys / 32; ++part) {
+            uint32_t sv[32], dv[32];
+            tmem_ld32(tS + part * 32, sv);
+            tmem_ld32(tP + part * 32, dv);
+            const int kk0 = part * 32;
+            const bool second = (BS == 64) && kk0 >= 64;
+            const int jj = second ? j1 : j0;
+            const float off = second ? off1 : off0;
+            const int kbase = (BS == 64) ? (kk0 & 63) : kk0;   // key offset inside its block
+            const bool diag = (jj == i);
+            uint32_t pk[16];
 #pragma unroll
-    for (int c = 0; c < 32; ++c) qv[c] = dov[c] = 0.0f;
-  }
+            for (int e = 0; e < 32; e += 2) {
+              float pe[2], de[2];
 #pragma unroll
-  for (int c = 0; c < 32; ++c) dq[c] = 0.0f;
-  const float lse = valid ? p.lse[row] : -INFINITY;
-  const float Dt = valid ? p.D[row] : 0.0f;
-  const bool live = valid && lse > -INFINITY;
-  const int count = p.counts[unit];
-  const int* list = p.lists + unit * p.idx_stride;
-  const float* lg = p.logg + unit * p.idx_stride;
-  const int64_t kvbase = bg * static_cast<int64_t>(p.N);
-  for (int s = 0; s < count; ++s) {
-    const int j = list[s];
-    const float bias = lg[s];
-    float dlsum = 0.0f;
-    for (int k0 = 0; k0 < p.bs; k0 += kRows) {
-      __syncthreads();
-      for (int e = threadIdx.x; e < kRows * (kD / 8); e += kThreads) {
-        const int kr = e >> 4, c8 = e & 15;
-        const int64_t src = (kvbase + j * p.bs + k0 + kr) * kD + c8 * 8;
-        const uint4 wk = __ldg(reinterpret_cast<const uint4*>(p.k + src));
-        const uint4 wv = __ldg(reinterpret_cast<const uint4*>(p.v + src));
-        const uint32_t kk[4] = {wk.x, wk.y, wk.z, wk.w}, vv[4] = {wv.x, wv.y, wv.z, wv.w};
+              for (int x = 0; x < 2; ++x) {
+                const bool on = live && !(diag && kbase + e + x > tb);
+                const float pv = on ? fast_exp2(fmaf(__uint_as_float(sv[e + x]), scale2, off)) : 0.0f;
+                const float dp = __uint_as_float(dv[e + x]);
+                if (sw == 0) {
+                  Dt = fmaf(pv, dp, Dt);
+                  de[x] = 0.0f;
+                } else {
+                  de[x] = on ? pv * (dp - Dt) : 0.0f;
+                }
+                pe[x] = pv;
+              }
+              if (sw == 1) {
+                pk[e >> 1] = pack_bf16x2(de[0], de[1]);
+                if (second) dl1 += de[0] + de[1];
+                else dl0 += de[0] + de[1];
+              }
+            }
+            if (sw == 1) tmem_st16(tS + part * 16, pk);
+          }
+          if (sw == 1) {
+            tmem_wait_st();
+            // the rows' share of dlogg for this step's blocks, per warp
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          ks[kr][c8 * 8 + 2 * x] = __uint_as_float(kk[x] << 16);
-          ks[kr][c8 * 8 + 2 * x + 1] = __uint_as_float(kk[x] & 0xFFFF0000u);
-          vs[kr][c8 * 8 + 2 * x] = __uint_as_float(vv[x] << 16);
-          vs[kr][c8 * 8 + 2 * x + 1] = __uint_as_float(vv[x] & 0xFFFF0000u);
+            for (int o = 16; o; o >>= 1) {
+              dl0 += __shfl_xor_sync(0xffffffffu, dl0, o);
+              dl1 += __shfl_xor_sync(0xffffffffu, dl1, o);
+            }
+            if (lane == 0) {
+              red[warp * kMaxList + s0] = dl0;
+              if (nblk == 2) red[warp * kMaxList + s0 + 1] = dl1;
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(PF));
+        }
+        if (sw == 0 && valid) p.D[row] = Dt;
+      }
+      if (!ok) break;
+      if (!(ok = warp_wait_all(bar(OF), done & 1, abortp, p.status))) break;
+      ++done;
+      tc_fence_after();
+      float* dst = p.dq + row * kD;
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t v[32];
+        tmem_ld32(tQ + ch * 32, v);
+        if (valid) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 4)
+            *reinterpret_cast<float4*>(dst + ch * 32 + c) =
+                make_float4(__uint_as_float(v[c]) * p.scale, __uint_as_float(v[c + 1]) * p.scale,
+                            __uint_as_float(v[c + 2]) * p.scale, __uint_as_float(v[c + 3]) * p.scale);
         }
       }
-      __syncthreads();
-      const int kend = (j == i) ? min(kRows, t - (j * p.bs + k0) + 1) : kRows;   // causal inside block i
-      for (int u = 0; u < kRows; ++u) {
-        const float* kr = &ks[u][qt * 32];
-        const float* vr = &vs[u][qt * 32];
-        float sdot = 0.0f, pdot = 0.0f;
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          sdot = fmaf(qv[c], kr[c], sdot);
-          pdot = fmaf(dov[c], vr[c], pdot);
-        }
-        sdot = quad_sum(sdot);
-        pdot = quad_sum(pdot);
-        const bool on = live && u < kend;
-        const float P = on ? __expf(fmaf(sdot, p.scale, bias) - lse) : 0.0f;
-        const float dl = P * (pdot - Dt);
-        dlsum += dl;
-        const float f = dl * p.scale;
-#pragma unroll
-        for (int c = 0; c < 32; ++c) dq[c] = fmaf(f, kr[c], dq[c]);
-      }
-    }
-    // the chunk's rows' share of dlogg for this slot (quarter 0 of each row counts it)
-    float x = (qt == 0) ? dlsum : 0.0f;
-#pragma unroll
-    for (int off = 16; off; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = x;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float tot = 0.0f;
-      for (int w = 0; w < kThreads / 32; ++w) tot += red[w];
-      p.dlogg_part[(unit * p.idx_stride + s) * p.chunks + chunk] = tot;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(OE));
+      // this tile's dlogg partial per kept slot: the four warps' sums in
+      // order.  (A warp writes the next item's sums only after every warp has
+      // passed this point: its S waits on all four warps' earlier P arrivals.)
+      mbar_arrive(bar(RS));
+      if (!(ok = warp_wait_all(bar(RS), rs & 1, abortp, p.status))) break;
+      ++rs;
+      for (int x = r; x < n; x += 128)
+        p.dlogg_part[(unit * p.idx_stride + x) * p.tiles + tile] =
+            ((red[x] + red[kMaxList + x]) + red[2 * kMaxList + x]) + red[3 * kMaxList + x];
     }
   }
-  if (valid) {
-    float* dst = p.dq + row * kD + qt * 32;
-#pragma unroll
-    for (int c = 0; c < 32; c += 4) *reinterpret_cast<float4*>(dst + c) = make_float4(dq[c], dq[c + 1], dq[c + 2], dq[c + 3]);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
   }
 }
 
-// dK / dV pass.  CTA = (b, g, key block j, chunk of 64 of its keys); thread
-// (key, quarter).  Every query block i that kept j (ascending), every head of
-// the group, its rows staged 64 at a time.
-__global__ void __launch_bounds__(kThreads) dkv_kernel(const Params p) {
-  extern __shared__ __align__(16) float dkv_sm[];
-  float (*qs)[kD + 4] = reinterpret_cast<float (*)[kD + 4]>(dkv_sm);
-  float (*dos)[kD + 4] = reinterpret_cast<float (*)[kD + 4]>(dkv_sm + kRows * (kD + 4));
-  __shared__ float ls[kRows], dsh[kRows];
-  const int kchunks = p.bs / kRows;
-  const int64_t blk = blockIdx.x / kchunks;           // (bg, j)
-  const int k0 = static_cast<int>(blockIdx.x % kchunks) * kRows;
-  const int64_t bg = blk / p.nb;
-  const int j = static_cast<int>(blk % p.nb);
-  const int b = static_cast<int>(bg / p.Hkv), g = static_cast<int>(bg % p.Hkv);
-  const int kl = threadIdx.x >> 2, qt = threadIdx.x & 3;
-  const int u = j * p.bs + k0 + kl;                    // this thread's key position
-  const int64_t krow = bg * static_cast<int64_t>(p.N) + u;
-  float kv[32], vv[32], dk[32], dv[32];
-  load_bf16x32(p.k + krow * kD + qt * 32, kv);
-  load_bf16x32(p.v + krow * kD + qt * 32, vv);
-#pragma unroll
-  for (int c = 0; c < 32; ++c) dk[c] = dv[c] = 0.0f;
-  const int* off = p.toff + bg * (p.nb + 1);
-  const int2* tl = p.tlist + bg * static_cast<int64_t>(p.nb) * p.idx_stride;
-  for (int e = off[j]; e < off[j + 1]; ++e) {
-    const int i = tl[e].x, s = tl[e].y;
-    const float bias = p.logg[(bg * p.nb + i) * p.idx_stride + s];
-    for (int hh = 0; hh < p.G; ++hh) {
-      const int h = g * p.G + hh;
-      for (int r0 = 0; r0 < p.bs; r0 += kRows) {
-        const int64_t rbase = (static_cast<int64_t>(b) * p.Hq + h) * p.N + i * p.bs + r0;
-        __syncthreads();
-        for (int x = threadIdx.x; x < kRows * (kD / 8); x += kThreads) {
-          const int rr = x >> 4, c8 = x & 15;
-          const int64_t src = (rbase + rr) * kD + c8 * 8;
-          const uint4 wq = __ldg(reinterpret_cast<const uint4*>(p.q + src));
-          const uint4 wd = __ldg(reinterpret_cast<const uint4*>(p.d_o + src));
-          const uint32_t a[4] = {wq.x, wq.y, wq.z, wq.w}, d2[4] = {wd.x, wd.y, wd.z, wd.w};
-#pragma unroll
-          for (int y = 0; y < 4; ++y) {
-            qs[rr][c8 * 8 + 2 * y] = __uint_as_float(a[y] << 16);
-            qs[rr][c8 * 8 + 2 * y + 1] = __uint_as_float(a[y] & 0xFFFF0000u);
-            dos[rr][c8 * 8 + 2 * y] = __uint_as_float(d2[y] << 16);
-            dos[rr][c8 * 8 + 2 * y + 1] = __uint_as_float(d2[y] & 0xFFFF0000u);
+// ------------------------------------------------------------------ key-major
+namespace km {
+constexpr uint32_t SM_K = 0, SM_V = kTile, SM_Q = 2 * kTile, SM_DO = 4 * kTile;   // Q, dO: two stages each
+constexpr uint32_t SM_ROW = 6 * kTile;                                            // float [2][2][128]
+constexpr uint32_t SM_BAR = SM_ROW + 2 * 2 * 128 * 4;
+enum { KVF = 0, KVE, CF, CE = CF + 2, SF = CE + 2, PF, OF, OE, RS, NBAR };   // RS: chunk row data written
+constexpr uint32_t SM_MISC = SM_BAR + NBAR * 8;
+constexpr uint32_t kSmem = SM_MISC + 16 + 1024;
+}  // namespace km
+
+template <int BS>
+__global__ void __launch_bounds__(kThreadsTC, 1)
+    dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
+                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const Params p) {
+  using namespace km;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  auto bar = [&](int b) -> uint32_t { return sb + SM_BAR + 8u * b; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM_MISC);
+  volatile int* abortp = reinterpret_cast<volatile int*>(smem + SM_MISC + 4);
+  float* rowc = reinterpret_cast<float*>(smem + SM_ROW);   // [2][128] log2 offsets (logg - lse) * log2e
+  float* rowd = rowc + 2 * 128;                            // [2][128] D
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int cpe = (BS == 128) ? p.G : (p.G + 1) / 2;   // 128-row chunks per (query block, key block)
+  const int64_t items = static_cast<int64_t>(p.B) * p.Hkv * p.nb;
+
+  // never-loaded rows of the operand buffers (the upper 64 keys of a 64-token
+  // block, a missing second head of a chunk) must hold finite values: zero
+  // them once, before the first copy lands
+  if (warp < 4) {
+    uint4* z = reinterpret_cast<uint4*>(smem);
+    for (uint32_t x = threadIdx.x; x < 6 * kTile / 16; x += 128) z[x] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+  }
+  if (threadIdx.x == 0) {
+    mbar_init(bar(KVF), 1);
+    mbar_init(bar(KVE), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(CF + s), 1);
+      mbar_init(bar(CE + s), 1);
+    }
+    mbar_init(bar(SF), 1);
+    mbar_init(bar(PF), 4);
+    mbar_init(bar(OF), 1);
+    mbar_init(bar(OE), 4);
+    mbar_init(bar(RS), 128);
+    *abortp = 0;
+    fence_barrier_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;   // S^T | dP^T | dV | dK
+
+  if (warp == 5) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      int gc = 0, kvc = 0;
+      bool ok = true;
+      for (int64_t item = blockIdx.x; ok && item < items; item += gridDim.x) {
+        const int64_t bg = item / p.nb;
+        const int j = static_cast<int>(item % p.nb);
+        const int* off = p.toff + bg * (p.nb + 1);
+        const int e0 = off[j], ne = off[j + 1] - e0;
+        if (ne == 0) continue;
+        const int b = static_cast<int>(bg / p.Hkv), g = static_cast<int>(bg % p.Hkv);
+        const int2* tl = p.tlist + bg * static_cast<int64_t>(p.nb) * p.idx_stride + e0;
+        if (kvc > 0 && !(ok = mbar_wait(bar(KVE), (kvc - 1) & 1, abortp, p.status))) break;
+        mbar_arrive_expect_tx(bar(KVF), static_cast<uint32_t>(BS) * 512u);
+        for (int r = 0; r < BS / 64; ++r) {
+          const int y = static_cast<int>(bg) * p.N + j * BS + r * 64;
+          for (int hf = 0; hf < 2; ++hf) {
+            tma_load_2d(sb + SM_K + hf * kHalf + r * 8192, &tmK, bar(KVF), hf * 64, y);
+            tma_load_2d(sb + SM_V + hf * kHalf + r * 8192, &tmV, bar(KVF), hf * 64, y);
           }
         }
-        if (threadIdx.x < kRows) {
-          ls[threadIdx.x] = p.lse[rbase + threadIdx.x];
-          dsh[threadIdx.x] = p.D[rbase + threadIdx.x];
-        }
-        __syncthreads();
-        for (int rr = 0; rr < kRows; ++rr) {
-          const float* qr = &qs[rr][qt * 32];
-          const float* dr = &dos[rr][qt * 32];
-          float sdot = 0.0f, pdot = 0.0f;
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            sdot = fmaf(qr[c], kv[c], sdot);
-            pdot = fmaf(dr[c], vv[c], pdot);
+        ++kvc;
+        for (int c = 0; ok && c < ne * cpe; ++c, ++gc) {
+          const int st = gc & 1, use = gc >> 1;
+          const int i = tl[c / cpe].x, hc = c % cpe;
+          if (gc >= 2 && !(ok = mbar_wait(bar(CE + st), (use - 1) & 1, abortp, p.status))) break;
+          int heads[2], rows0[2], npc = 0;
+          if (BS == 128) {
+            heads[0] = heads[1] = hc;
+            rows0[0] = i * 128;
+            rows0[1] = i * 128 + 64;
+            npc = 2;
+          } else {
+            heads[0] = 2 * hc;
+            heads[1] = 2 * hc + 1;
+            rows0[0] = rows0[1] = i * 64;
+            npc = (2 * hc + 1 < p.G) ? 2 : 1;
           }
-          sdot = quad_sum(sdot);
-          pdot = quad_sum(pdot);
-          const int t = i * p.bs + r0 + rr;
-          const float lse = ls[rr];
-          const bool on = lse > -INFINITY && (i != j || u <= t);
-          const float P = on ? __expf(fmaf(sdot, p.scale, bias) - lse) : 0.0f;
-          const float f = P * (pdot - dsh[rr]) * p.scale;
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            dv[c] = fmaf(P, dr[c], dv[c]);
-            dk[c] = fmaf(f, qr[c], dk[c]);
+          mbar_arrive_expect_tx(bar(CF + st), static_cast<uint32_t>(npc) * 4u * 8192u);
+          for (int pc = 0; pc < npc; ++pc) {
+            const int y = (b * p.Hq + g * p.G + heads[pc]) * p.N + rows0[pc];
+            for (int hf = 0; hf < 2; ++hf) {
+              tma_load_2d(sb + SM_Q + st * kTile + hf * kHalf + pc * 8192, &tmQ, bar(CF + st), hf * 64, y);
+              tma_load_2d(sb + SM_DO + st * kTile + hf * kHalf + pc * 8192, &tmDO, bar(CF + st), hf * 64, y);
+            }
           }
         }
       }
+      if (*abortp) {
+        if (kvc > 0) mbar_drain(bar(KVF), (kvc - 1) & 1);
+        for (int s = max(0, gc - 2); s < gc; ++s) mbar_drain(bar(CF + (s & 1)), (s >> 1) & 1);
+      }
+    }
+  } else if (warp == 4) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      const uint32_t id_k = idesc_bf16_f32(128, 128, 0, 0);
+      const uint32_t id_mn = idesc_bf16_f32(128, 128, 0, 1);
+      const uint64_t kd = smem_desc_sw128(sb + SM_K, 16, 1024);
+      const uint64_t vd = smem_desc_sw128(sb + SM_V, 16, 1024);
+      const uint64_t qd0 = smem_desc_sw128(sb + SM_Q, 16, 1024);
+      const uint64_t dod0 = smem_desc_sw128(sb + SM_DO, 16, 1024);
+      const uint64_t qmn0 = smem_desc_sw128(sb + SM_Q, kHalf, 1024);
+      const uint64_t domn0 = smem_desc_sw128(sb + SM_DO, kHalf, 1024);
+      const uint32_t tS = tmem, tP = tmem + 128, tV = tmem + 256, tK = tmem + 384;
+      int gc = 0, kvc = 0, sf = 0, done = 0;
+      bool ok = true;
+      for (int64_t item = blockIdx.x; ok && item < items; item += gridDim.x) {
+        const int64_t bg = item / p.nb;
+        const int j = static_cast<int>(item % p.nb);
+        const int* off = p.toff + bg * (p.nb + 1);
+        const int ne = off[j + 1] - off[j];
+        if (ne == 0) continue;
+        if (!(ok = mbar_wait(bar(KVF), kvc & 1, abortp, p.status))) break;
+        ++kvc;
+        for (int c = 0; c < ne * cpe; ++c, ++gc) {
+          const int st = gc & 1, use = gc >> 1;
+          if (!(ok = mbar_wait(bar(CF + st), use & 1, abortp, p.status))) break;
+          tc_fence_after();
+          const uint64_t qd = qd0 + ((st * kTile) >> 4), dod = dod0 + ((st * kTile) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk) {
+            const uint32_t o = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
+            mma_ss(tS, kd + o, qd + o, id_k, kk > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk) {
+            const uint32_t o = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
+            mma_ss(tP, vd + o, dod + o, id_k, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(bar(SF));
+          ++sf;
+          if (!(ok = mbar_wait(bar(PF), (sf - 1) & 1, abortp, p.status))) break;
+          if (c == 0 && done > 0 && !(ok = mbar_wait(bar(OE), (done - 1) & 1, abortp, p.status))) break;
+          tc_fence_after();
+          const uint64_t qmn = qmn0 + ((st * kTile) >> 4), domn = domn0 + ((st * kTile) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tV, tS + kk * 8, domn + ((kk * 2048) >> 4), id_mn, (c > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tK, tP + kk * 8, qmn + ((kk * 2048) >> 4), id_mn, (c > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(bar(CE + st));
+        }
+        if (!ok) break;
+        tc_commit(bar(OF));
+        tc_commit(bar(KVE));
+        ++done;
+      }
+      if (!ok) {
+        tc_commit(bar(OF));
+        mbar_drain(bar(OF), done & 1);
+      }
+    }
+  } else {
+    // ------------------------------------------------ lanes (one key each)
+    const int u = warp * 32 + lane;
+    const uint32_t la = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t tS = la, tP = la + 128, tV = la + 256, tK = la + 384;
+    const float scale2 = p.scale * kLog2e;
+    const bool kvalid = (BS == 128) || u < 64;
+    int gc = 0, sf = 0, done = 0;
+    bool ok = true;
+    for (int64_t item = blockIdx.x; ok && item < items; item += gridDim.x) {
+      const int64_t bg = item / p.nb;
+      const int j = static_cast<int>(item % p.nb);
+      const int b = static_cast<int>(bg / p.Hkv), g = static_cast<int>(bg % p.Hkv);
+      const int* off = p.toff + bg * (p.nb + 1);
+      const int e0 = off[j], ne = off[j + 1] - e0;
+      const int64_t krow = bg * static_cast<int64_t>(p.N) + static_cast<int64_t>(j) * BS + u;
+      if (ne == 0) {
+        if (kvalid) {
+          float4* dk = reinterpret_cast<float4*>(p.dk + krow * kD);
+          float4* dv = reinterpret_cast<float4*>(p.dv + krow * kD);
+          for (int c = 0; c < kD / 4; ++c) dk[c] = dv[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        continue;
+      }
+      const int2* tl = p.tlist + bg * static_cast<int64_t>(p.nb) * p.idx_stride + e0;
+      for (int c = 0; c < ne * cpe; ++c, ++gc) {
+        const int2 ent = tl[c / cpe];
+        const int i = ent.x, hc = c % cpe;
+        const float lgv = p.logg[(bg * p.nb + i) * p.idx_stride + ent.y];
+        // this chunk's 128 rows: log2 offset (logg - LSE) * log2e, or -inf
+        // for a row that does not exist or attends to nothing; and D
+        {
+          const int x = u;   // chunk row handled by this thread
+          const int hh = (BS == 128) ? hc : 2 * hc + (x >> 6);
+          const int tb = (BS == 128) ? x : (x & 63);
+          float cv = -INFINITY, dvv = 0.0f;
+          if (hh < p.G) {
+            const int64_t row = (static_cast<int64_t>(b) * p.Hq + g * p.G + hh) * p.N + static_cast<int64_t>(i) * BS + tb;
+            const float lse = p.lse[row];
+            if (lse > -INFINITY) {
+              cv = (lgv - lse) * kLog2e;
+              dvv = p.D[row];
+            }
+          }
+          rowc[(gc & 1) * 128 + x] = cv;
+          rowd[(gc & 1) * 128 + x] = dvv;
+        }
+        // (the other slot may still be read for the previous chunk: a thread
+        // writes it again only after every thread has arrived for that chunk)
+        mbar_arrive(bar(RS));
+        if (!(ok = warp_wait_all(bar(RS), gc & 1, abortp, p.status))) break;
+        if (!(ok = warp_wait_all(bar(SF), sf & 1, abortp, p.status))) break;
+        ++sf;
+        tc_fence_after();
+        const float* rc = rowc + (gc & 1) * 128;
+        const float* rd = rowd + (gc & 1) * 128;
+        const bool diag = (i == j);
+#pragma unroll 1
+        for (int part = 0; part < 4; ++part) {
+          uint32_t sv[32], dv[32];
+          tmem_ld32(tS + part * 32, sv);
+          tmem_ld32(tP + part * 32, dv);
+          uint32_t pk[16], dk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            float pe[2], de[2];
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+              const int t = part * 32 + e + x;
+              const int tb = (BS == 128) ? t : (t & 63);
+              const float cv = rc[t];
+              const bool on = kvalid && cv > -INFINITY && !(diag && u > tb);
+              const float pv = on ? fast_exp2(fmaf(__uint_as_float(sv[e + x]), scale2, cv)) : 0.0f;
+              pe[x] = pv;
+              de[x] = on ? pv * (__uint_as_float(dv[e + x]) - rd[t]) : 0.0f;
+            }
+            pk[e >> 1] = pack_bf16x2(pe[0], pe[1]);
+            dk[e >> 1] = pack_bf16x2(de[0], de[1]);
+          }
+          tmem_st16(tS + part * 16, pk);
+          tmem_st16(tP + part * 16, dk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(PF));
+      }
+      if (!ok) break;
+      if (!(ok = warp_wait_all(bar(OF), done & 1, abortp, p.status))) break;
+      ++done;
+      tc_fence_after();
+      float* dkd = p.dk + krow * kD;
+      float* dvd = p.dv + krow * kD;
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t a[32], v[32];
+        tmem_ld32(tK + ch * 32, a);
+        tmem_ld32(tV + ch * 32, v);
+        if (kvalid) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 4) {
+            *reinterpret_cast<float4*>(dkd + ch * 32 + c) =
+                make_float4(__uint_as_float(a[c]) * p.scale, __uint_as_float(a[c + 1]) * p.scale,
+                            __uint_as_float(a[c + 2]) * p.scale, __uint_as_float(a[c + 3]) * p.scale);
+            *reinterpret_cast<float4*>(dvd + ch * 32 + c) =
+                make_float4(__uint_as_float(v[c]), __uint_as_float(v[c + 1]), __uint_as_float(v[c + 2]),
+                            __uint_as_float(v[c + 3]));
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(OE));
     }
   }
-  float* dkd = p.dk + krow * kD + qt * 32;
-  float* dvd = p.dv + krow * kD + qt * 32;
-#pragma unroll
-  for (int c = 0; c < 32; c += 4) {
-    *reinterpret_cast<float4*>(dkd + c) = make_float4(dk[c], dk[c + 1], dk[c + 2], dk[c + 3]);
-    *reinterpret_cast<float4*>(dvd + c) = make_float4(dv[c], dv[c + 1], dv[c + 2], dv[c + 3]);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
   }
 }
 
-// dsel per unit: dlogg_l (the chunks' partials summed in order) minus
+// dsel per unit: dlogg_l (the row tiles' partials summed in order) minus
 // g_l * (sum over the kept blocks of dlogg_j); zero off the kept blocks.
 // One warp per unit.
 __global__ void dsel_kernel(const Params p, int64_t units, float* __restrict__ dsel) {
@@ -351,13 +776,13 @@ __global__ void dsel_kernel(const Params p, int64_t units, float* __restrict__ d
   float tot = 0.0f;
   for (int s = lane; s < count; s += 32) {
     float x = 0.0f;
-    for (int c = 0; c < p.chunks; ++c) x += p.dlogg_part[(unit * p.idx_stride + s) * p.chunks + c];
+    for (int c = 0; c < p.tiles; ++c) x += p.dlogg_part[(unit * p.idx_stride + s) * p.tiles + c];
     tot += x;
   }
   for (int off = 16; off; off >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, off);
   for (int s = lane; s < count; s += 32) {
     float x = 0.0f;
-    for (int c = 0; c < p.chunks; ++c) x += p.dlogg_part[(unit * p.idx_stride + s) * p.chunks + c];
+    for (int c = 0; c < p.tiles; ++c) x += p.dlogg_part[(unit * p.idx_stride + s) * p.tiles + c];
     row[list[s]] = x - __expf(p.logg[unit * p.idx_stride + s]) * tot;
   }
 }
@@ -368,31 +793,28 @@ size_t attn_bwd_workspace(int B, int Hq, int Hkv, int N, int bs, int idx_stride)
   auto a256 = [](size_t x) { return (x + 255) & ~size_t(255); };
   const int nb = N / bs;
   const int64_t units = static_cast<int64_t>(B) * Hkv * nb;
-  const int chunks = (Hq / Hkv * bs + bwd::kRows - 1) / bwd::kRows;
+  const int tiles = (Hq / Hkv * bs + 127) / 128;
   size_t off = 0;
-  off = a256(off + static_cast<size_t>(B) * Hq * N * sizeof(float));            // D
+  off = a256(off + static_cast<size_t>(B) * Hq * N * sizeof(float));            // D (written by the dQ pass)
   off = a256(off + units * idx_stride * sizeof(float));                          // logg
   off = a256(off + units * idx_stride * sizeof(int));                            // lists
   off = a256(off + units * sizeof(int));                                         // counts
   off = a256(off + static_cast<size_t>(B) * Hkv * (nb + 1) * sizeof(int));       // toff
   off = a256(off + units * idx_stride * sizeof(int2));                           // tlist
-  off = a256(off + units * idx_stride * chunks * sizeof(float));                 // dlogg partials
+  off = a256(off + units * idx_stride * tiles * sizeof(float));                  // dlogg partials
   return off;
 }
 
-cudaError_t launch_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
-                            const void* d_o, const int* idx, int idx_stride, const float* sel, float scale, int B,
-                            int Hq, int Hkv, int N, int bs, float* dq, float* dk, float* dv, float* dsel,
-                            void* workspace, uint32_t* status, cudaStream_t st) {
+cudaError_t launch_attn_bwd(const CUtensorMap* tmQ, const CUtensorMap* tmDO, const CUtensorMap* tmK,
+                            const CUtensorMap* tmV, const float* lse, const int* idx, int idx_stride,
+                            const float* sel, float scale, int B, int Hq, int Hkv, int N, int bs, float* dq,
+                            float* dk, float* dv, float* dsel, void* workspace, uint32_t* status, int num_sms,
+                            cudaStream_t st) {
   auto a256 = [](size_t x) { return (x + 255) & ~size_t(255); };
   const int nb = N / bs;
   const int64_t units = static_cast<int64_t>(B) * Hkv * nb;
   const int64_t rows = static_cast<int64_t>(B) * Hq * N;
   bwd::Params p;
-  p.q = static_cast<const __nv_bfloat16*>(q);
-  p.k = static_cast<const __nv_bfloat16*>(k);
-  p.v = static_cast<const __nv_bfloat16*>(v);
-  p.d_o = static_cast<const __nv_bfloat16*>(d_o);
   p.lse = lse;
   p.B = B;
   p.Hq = Hq;
@@ -400,16 +822,16 @@ cudaError_t launch_attn_bwd(const void* q, const void* k, const void* v, const v
   p.N = N;
   p.nb = nb;
   p.G = Hq / Hkv;
-  p.bs = bs;
   p.idx_stride = idx_stride;
-  p.chunks = (p.G * bs + bwd::kRows - 1) / bwd::kRows;
+  p.tiles = (p.G * bs + 127) / 128;
   p.scale = scale;
   p.dq = dq;
   p.dk = dk;
   p.dv = dv;
+  p.status = status;
   char* ws = static_cast<char*>(workspace);
   size_t off = 0;
-  float* D = reinterpret_cast<float*>(ws + off);
+  p.D = reinterpret_cast<float*>(ws + off);
   off = a256(off + rows * sizeof(float));
   float* logg = reinterpret_cast<float*>(ws + off);
   off = a256(off + units * idx_stride * sizeof(float));
@@ -422,24 +844,32 @@ cudaError_t launch_attn_bwd(const void* q, const void* k, const void* v, const v
   int2* tlist = reinterpret_cast<int2*>(ws + off);
   off = a256(off + units * idx_stride * sizeof(int2));
   p.dlogg_part = reinterpret_cast<float*>(ws + off);
-  p.D = D;
   p.logg = logg;
   p.lists = lists;
   p.counts = counts;
   p.toff = toff;
   p.tlist = tlist;
-  bwd::rowdot_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(o),
-                                                                             p.d_o, rows, D);
   bwd::gate_kernel<<<static_cast<unsigned>((units + 7) / 8), 256, 0, st>>>(idx, idx_stride, sel, nb, units, lists,
                                                                            counts, logg, status);
   const int bgs = B * Hkv;
   bwd::transpose_kernel<<<(bgs + 63) / 64, 64, 0, st>>>(lists, counts, idx_stride, nb, bgs, toff, tlist);
-  cudaError_t e = ensure_dynamic_smem<bwd::dq_kernel>(bwd::kTileSmem);
-  if (e == cudaSuccess) e = ensure_dynamic_smem<bwd::dkv_kernel>(bwd::kTileSmem);
-  if (e != cudaSuccess) return e;
-  bwd::dq_kernel<<<static_cast<unsigned>(units * p.chunks), bwd::kThreads, bwd::kTileSmem, st>>>(p);
-  bwd::dkv_kernel<<<static_cast<unsigned>(static_cast<int64_t>(bgs) * nb * (bs / bwd::kRows)), bwd::kThreads,
-                    bwd::kTileSmem, st>>>(p);
+  const int64_t items_q = units * p.tiles, items_k = static_cast<int64_t>(bgs) * nb;
+  const unsigned grid_q = static_cast<unsigned>(items_q < num_sms ? items_q : num_sms);
+  const unsigned grid_k = static_cast<unsigned>(items_k < num_sms ? items_k : num_sms);
+  cudaError_t e = cudaSuccess;
+  if (bs == 64) {
+    e = ensure_dynamic_smem<bwd::dq_tc_kernel<64>>(bwd::qm::kSmem);
+    if (e == cudaSuccess) e = ensure_dynamic_smem<bwd::dkv_tc_kernel<64>>(bwd::km::kSmem);
+    if (e != cudaSuccess) return e;
+    if (grid_q > 0) bwd::dq_tc_kernel<64><<<grid_q, bwd::kThreadsTC, bwd::qm::kSmem, st>>>(*tmQ, *tmDO, *tmK, *tmV, p);
+    if (grid_k > 0) bwd::dkv_tc_kernel<64><<<grid_k, bwd::kThreadsTC, bwd::km::kSmem, st>>>(*tmQ, *tmDO, *tmK, *tmV, p);
+  } else {
+    e = ensure_dynamic_smem<bwd::dq_tc_kernel<128>>(bwd::qm::kSmem);
+    if (e == cudaSuccess) e = ensure_dynamic_smem<bwd::dkv_tc_kernel<128>>(bwd::km::kSmem);
+    if (e != cudaSuccess) return e;
+    if (grid_q > 0) bwd::dq_tc_kernel<128><<<grid_q, bwd::kThreadsTC, bwd::qm::kSmem, st>>>(*tmQ, *tmDO, *tmK, *tmV, p);
+    if (grid_k > 0) bwd::dkv_tc_kernel<128><<<grid_k, bwd::kThreadsTC, bwd::km::kSmem, st>>>(*tmQ, *tmDO, *tmK, *tmV, p);
+  }
   if (dsel != nullptr)
     bwd::dsel_kernel<<<static_cast<unsigned>((units + 7) / 8), 256, 0, st>>>(p, units, dsel);
   return cudaGetLastError();

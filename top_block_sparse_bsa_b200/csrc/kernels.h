@@ -116,10 +116,11 @@ cudaError_t launch_attn_prefill_pair_bf16(const CUtensorMap* tmQ, const CUtensor
 
 // attn_bwd.cu (backward of the sparse / gated prefill attention)
 size_t attn_bwd_workspace(int B, int Hq, int Hkv, int N, int bs, int idx_stride);
-cudaError_t launch_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
-                            const void* d_o, const int* idx, int idx_stride, const float* sel, float scale, int B,
-                            int Hq, int Hkv, int N, int bs, float* dq, float* dk, float* dv, float* dsel,
-                            void* workspace, uint32_t* status, cudaStream_t st);
+cudaError_t launch_attn_bwd(const CUtensorMap* tmQ, const CUtensorMap* tmDO, const CUtensorMap* tmK,
+                            const CUtensorMap* tmV, const float* lse, const int* idx, int idx_stride,
+                            const float* sel, float scale, int B, int Hq, int Hkv, int N, int bs, float* dq,
+                            float* dk, float* dv, float* dsel, void* workspace, uint32_t* status, int num_sms,
+                            cudaStream_t st);
 
 // paged.cu (paged cache upkeep)
 cudaError_t launch_paged_append(const void* k_new, const void* v_new, int B, int Hkv, int T, int d,

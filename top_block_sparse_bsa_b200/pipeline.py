@@ -107,7 +107,7 @@ class PrefillStep:
         ws = bsa_workspace_bytes_bwd(self.shape, idx.shape[-1])
         if "bwd_workspace" not in b or b["bwd_workspace"].numel() < ws:
             b["bwd_workspace"] = torch.empty((max(ws, 256),), dtype=torch.uint8, device=dev)
-        bsa_gated_attn_bwd(self.shape, self.q, self.k, self.v, b["o"], b["lse"], d_o, idx, idx.shape[-1],
+        bsa_gated_attn_bwd(self.shape, self.q, self.k, self.v, b["lse"], d_o, idx, idx.shape[-1],
                            b["scores"] if self.gated else None, self.softmax_scale, b["dq"], b["dk"], b["dv"],
                            b["dsel"] if self.gated else None, b["bwd_workspace"], stream=stream)
         return b
