@@ -104,28 +104,85 @@ __global__ void gate_kernel(const int* __restrict__ idx, int idx_stride, const f
 }
 
 // For each (b, g): the query blocks i (ascending) that kept each key block j,
-// with the slot of j in i's list.  One thread per (b, g), sequential, so the
-// lists come out in a fixed order.
-__global__ void transpose_kernel(const int* __restrict__ lists, const int* __restrict__ counts, int idx_stride,
-                                 int nb, int bgs, int* __restrict__ toff, int2* __restrict__ tlist) {
-  const int bg = blockIdx.x * blockDim.x + threadIdx.x;
-  if (bg >= bgs) return;
-  int* off = toff + static_cast<int64_t>(bg) * (nb + 1);
+// with the slot of j in i's list.  One CTA per (b, g): counts per key block
+// by shared-memory atomics, an exclusive scan, then the fill, which walks the
+// query blocks in ascending order (a list's entries are distinct, so its
+// entries take their cursors without conflict), so every transposed list
+// comes out in a fixed order.  Lists are staged in shared memory kTrChunk at
+// a time.  Dynamic shared memory: transpose_smem_bytes(nb, idx_stride).
+constexpr int kTrThreads = 256;
+constexpr int kTrChunk = 32;
+inline size_t transpose_smem_bytes(int nb, int idx_stride) {
+  return static_cast<size_t>(nb) * sizeof(int) + static_cast<size_t>(kTrChunk) * (idx_stride + 1) * sizeof(int) +
+         kTrThreads * sizeof(int);
+}
+
+__global__ void __launch_bounds__(kTrThreads) transpose_kernel(const int* __restrict__ lists,
+                                                               const int* __restrict__ counts, int idx_stride,
+                                                               int nb, int* __restrict__ toff,
+                                                               int2* __restrict__ tlist) {
+  extern __shared__ int tr_sm[];
+  int* cur = tr_sm;                            // [nb] counts, then cursors
+  int* lbuf = cur + nb;                        // [kTrChunk][idx_stride] staged lists
+  int* lcnt = lbuf + kTrChunk * idx_stride;    // [kTrChunk] their counts
+  int* part = lcnt + kTrChunk;                 // [kTrThreads] scan partials
+  const int bg = blockIdx.x, tid = threadIdx.x;
   const int64_t ubase = static_cast<int64_t>(bg) * nb;
-  for (int j = 0; j <= nb; ++j) off[j] = 0;
-  for (int i = 0; i < nb; ++i) {
-    const int* l = lists + (ubase + i) * idx_stride;
-    for (int s = 0; s < counts[ubase + i]; ++s) ++off[l[s] + 1];
-  }
-  for (int j = 0; j < nb; ++j) off[j + 1] += off[j];
-  // fill, then restore the starts (each count was used as a cursor)
+  int* off = toff + static_cast<int64_t>(bg) * (nb + 1);
   int2* tl = tlist + ubase * idx_stride;
-  for (int i = 0; i < nb; ++i) {
-    const int* l = lists + (ubase + i) * idx_stride;
-    for (int s = 0; s < counts[ubase + i]; ++s) tl[off[l[s]]++] = make_int2(i, s);
+  for (int j = tid; j < nb; j += kTrThreads) cur[j] = 0;
+  auto stage = [&](int i0) {
+    __syncthreads();
+    const int nl = min(kTrChunk, nb - i0);
+    for (int x = tid; x < nl * idx_stride; x += kTrThreads)
+      lbuf[x] = lists[(ubase + i0) * idx_stride + x];
+    for (int x = tid; x < nl; x += kTrThreads) lcnt[x] = counts[ubase + i0 + x];
+    __syncthreads();
+    return nl;
+  };
+  // counts
+  for (int i0 = 0; i0 < nb; i0 += kTrChunk) {
+    const int nl = stage(i0);
+    for (int x = tid; x < nl * idx_stride; x += kTrThreads)
+      if (x % idx_stride < lcnt[x / idx_stride]) atomicAdd(&cur[lbuf[x]], 1);
   }
-  for (int j = nb; j > 0; --j) off[j] = off[j - 1];
-  off[0] = 0;
+  __syncthreads();
+  // exclusive scan: each thread a contiguous segment
+  const int seg = (nb + kTrThreads - 1) / kTrThreads;
+  const int j0 = min(nb, tid * seg), j1 = min(nb, j0 + seg);
+  int sum = 0;
+  for (int j = j0; j < j1; ++j) sum += cur[j];
+  part[tid] = sum;
+  __syncthreads();
+  if (tid == 0) {
+    int acc = 0;
+    for (int t = 0; t < kTrThreads; ++t) {
+      const int v = part[t];
+      part[t] = acc;
+      acc += v;
+    }
+    off[nb] = acc;
+  }
+  __syncthreads();
+  int acc = part[tid];
+  for (int j = j0; j < j1; ++j) {
+    const int v = cur[j];
+    cur[j] = acc;
+    off[j] = acc;
+    acc += v;
+  }
+  // fill: query blocks in ascending order, one list at a time
+  for (int i0 = 0; i0 < nb; i0 += kTrChunk) {
+    const int nl = stage(i0);
+    for (int x = 0; x < nl; ++x) {
+      const int c = lcnt[x];
+      for (int s = tid; s < c; s += kTrThreads) {
+        const int j = lbuf[x * idx_stride + s];
+        tl[cur[j]++] = make_int2(i0 + x, s);
+      }
+      __syncthreads();
+    }
+  }
 }
 
 struct Params {
@@ -141,11 +198,17 @@ struct Params {
 };
 
 // ------------------------------------------------------------------ query-major
+// Steps of 64 keys; two S | dP buffers in tensor memory, so the MMAs of step
+// s+1 run while the lanes work on step s.
 namespace qm {
-constexpr uint32_t SM_Q = 0, SM_DO = kTile, SM_K = 2 * kTile, SM_V = 4 * kTile;   // K, V: two stages each
-constexpr uint32_t SM_RED = 6 * kTile;                                            // float [4][kMaxList]
+constexpr int kStagesK = 4;                                    // K/V stages of 64 keys
+constexpr uint32_t kKV = 64u * 128u * 2u;                      // 64 keys x 128 bf16
+constexpr uint32_t kKVHalf = kKV / 2;
+constexpr uint32_t SM_Q = 0, SM_DO = kTile;
+constexpr uint32_t SM_K = 2 * kTile, SM_V = SM_K + kStagesK * kKV;
+constexpr uint32_t SM_RED = SM_V + kStagesK * kKV;              // float [4][kMaxList]
 constexpr uint32_t SM_BAR = SM_RED + 4 * kMaxList * 4;
-enum { QF = 0, QE, KF, KE = KF + 2, SF = KE + 2, PF, OF, OE, RS, NBAR };   // RS: dlogg sums written
+enum { QF = 0, QE, KF, KE = KF + kStagesK, SF = KE + kStagesK, PF = SF + 2, OF = PF + 2, OE, RS, NBAR };
 constexpr uint32_t SM_MISC = SM_BAR + NBAR * 8;   // tmem base, abort flag
 constexpr uint32_t kSmem = SM_MISC + 16 + 1024;
 }  // namespace qm
@@ -155,6 +218,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const Params p) {
   using namespace qm;
+  constexpr int kHalves = BS / 64;   // 64-key steps per block
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
@@ -170,12 +234,14 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   if (threadIdx.x == 0) {
     mbar_init(bar(QF), 1);
     mbar_init(bar(QE), 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kStagesK; ++s) {
       mbar_init(bar(KF + s), 1);
       mbar_init(bar(KE + s), 1);
     }
-    mbar_init(bar(SF), 1);
-    mbar_init(bar(PF), 4);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(SF + b), 1);
+      mbar_init(bar(PF + b), 4);
+    }
     mbar_init(bar(OF), 1);
     mbar_init(bar(OE), 4);
     mbar_init(bar(RS), 128);
@@ -189,7 +255,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;   // S | dP | dQ
+  const uint32_t tmem = *tmem_slot;   // [S | dP] x 2 buffers (64 + 64 columns each) | dQ
   auto item_unit = [&](int64_t item, int& tile, int64_t& bg, int& i) {
     const int64_t unit = item / p.tiles;
     tile = static_cast<int>(item % p.tiles);
@@ -228,92 +294,91 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         ++qc;
         const int* list = p.lists + unit * p.idx_stride;
         const int kvrow0 = static_cast<int>(bg) * p.N;
-        const int nsteps = (BS == 64) ? (n + 1) / 2 : n;
+        const int nst = n * kHalves;
         for (int sw = 0; ok && sw < 2; ++sw)
-          for (int s = 0; s < nsteps; ++s, ++gs) {
-            const int st = gs & 1, use = gs >> 1;
-            int jb[2] = {list[(BS == 64) ? 2 * s : s], 0};
-            const int nblk = (BS == 64 && 2 * s + 1 < n) ? 2 : 1;
-            if (nblk == 2) jb[1] = list[2 * s + 1];
-            if (gs >= 2 && !(ok = mbar_wait(bar(KE + st), (use - 1) & 1, abortp, p.status))) break;
-            mbar_arrive_expect_tx(bar(KF + st), static_cast<uint32_t>(nblk * BS) * 512u);
-            for (int bl = 0; bl < nblk; ++bl)
-              for (int r = 0; r < BS / 64; ++r) {
-                const uint32_t rowoff = static_cast<uint32_t>(bl * BS + r * 64) * 128u;
-                const int y = kvrow0 + jb[bl] * BS + r * 64;
-                for (int hf = 0; hf < 2; ++hf) {
-                  tma_load_2d(sb + SM_K + st * kTile + hf * kHalf + rowoff, &tmK, bar(KF + st), hf * 64, y);
-                  tma_load_2d(sb + SM_V + st * kTile + hf * kHalf + rowoff, &tmV, bar(KF + st), hf * 64, y);
-                }
-              }
+          for (int s = 0; s < nst; ++s, ++gs) {
+            const int st = gs % kStagesK, use = gs / kStagesK;
+            if (gs >= kStagesK && !(ok = mbar_wait(bar(KE + st), (use - 1) & 1, abortp, p.status))) break;
+            mbar_arrive_expect_tx(bar(KF + st), 4u * 8192u);
+            const int y = kvrow0 + list[s / kHalves] * BS + (s % kHalves) * 64;
+            for (int hf = 0; hf < 2; ++hf) {
+              tma_load_2d(sb + SM_K + st * kKV + hf * kKVHalf, &tmK, bar(KF + st), hf * 64, y);
+              tma_load_2d(sb + SM_V + st * kKV + hf * kKVHalf, &tmV, bar(KF + st), hf * 64, y);
+            }
           }
       }
       if (*abortp) {
         if (qc > 0) mbar_drain(bar(QF), (qc - 1) & 1);
-        for (int s = max(0, gs - 2); s < gs; ++s) mbar_drain(bar(KF + (s & 1)), (s >> 1) & 1);
+        for (int s = max(0, gs - kStagesK); s < gs; ++s) mbar_drain(bar(KF + s % kStagesK), (s / kStagesK) & 1);
       }
     }
   } else if (warp == 4) {
     if (lane == 0) {
       // ------------------------------------------------ MMA issuer
-      const uint32_t id128 = idesc_bf16_f32(128, 128, 0, 0);
-      const uint32_t id64 = idesc_bf16_f32(128, 64, 0, 0);
-      const uint32_t id_mn = idesc_bf16_f32(128, 128, 0, 1);
+      const uint32_t id_s = idesc_bf16_f32(128, 64, 0, 0);     // S, dP: 128 rows x 64 keys
+      const uint32_t id_mn = idesc_bf16_f32(128, 128, 0, 1);   // dQ: 128 rows x 128 channels
       const uint64_t qd = smem_desc_sw128(sb + SM_Q, 16, 1024);
       const uint64_t dod = smem_desc_sw128(sb + SM_DO, 16, 1024);
       const uint64_t kd0 = smem_desc_sw128(sb + SM_K, 16, 1024);
       const uint64_t vd0 = smem_desc_sw128(sb + SM_V, 16, 1024);
-      const uint64_t kmn0 = smem_desc_sw128(sb + SM_K, kHalf, 1024);
-      const uint32_t tS = tmem, tP = tmem + 128, tQ = tmem + 256;
-      int gs = 0, qc = 0, sf = 0, done = 0;
-      bool ok = true, pf_pending = false;
+      const uint64_t kmn0 = smem_desc_sw128(sb + SM_K, kKVHalf, 1024);
+      const uint32_t tQ = tmem + 256;
+      int gs = 0, qc = 0, done = 0;
+      int pfu[2] = {0, 0};
+      bool ok = true;
+      // S = Q K^T and dP = dO V^T of global step `g` into buffer g & 1; in the
+      // first sweep the K/V stage is free once they complete
+      auto issue_sdp = [&](int g, bool release) -> bool {
+        const int st = g % kStagesK, buf = g & 1;
+        if (!mbar_wait(bar(KF + st), (g / kStagesK) & 1, abortp, p.status)) return false;
+        tc_fence_after();
+        const uint64_t kd = kd0 + ((st * kKV) >> 4), vd = vd0 + ((st * kKV) >> 4);
+        const uint32_t tS = tmem + buf * 128, tP = tS + 64;
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t oa = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
+          const uint32_t ob = ((kk >> 2) * kKVHalf + (kk & 3) * 32) >> 4;
+          mma_ss(tS, qd + oa, kd + ob, id_s, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t oa = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
+          const uint32_t ob = ((kk >> 2) * kKVHalf + (kk & 3) * 32) >> 4;
+          mma_ss(tP, dod + oa, vd + ob, id_s, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(SF + buf));
+        if (release) tc_commit(bar(KE + st));
+        return true;
+      };
       for (int64_t item = blockIdx.x; ok && item < items; item += gridDim.x) {
         int tile, i;
         int64_t bg;
         const int64_t unit = item_unit(item, tile, bg, i);
         const int n = p.counts[unit];
         if (n == 0) continue;
-        const int nsteps = (BS == 64) ? (n + 1) / 2 : n;
+        const int nst = n * kHalves;
         if (!(ok = mbar_wait(bar(QF), qc & 1, abortp, p.status))) break;
         ++qc;
         tc_fence_after();
-        for (int sw = 0; ok && sw < 2; ++sw)
-          for (int s = 0; s < nsteps; ++s, ++gs) {
-            const int st = gs & 1, use = gs >> 1;
-            const int keys = (BS == 64 && 2 * s + 1 >= n) ? 64 : 128;
-            // S and dP are overwritten: the lanes must be done with the previous ones
-            if (pf_pending && !(ok = mbar_wait(bar(PF), (sf - 1) & 1, abortp, p.status))) break;
-            pf_pending = false;
-            if (!(ok = mbar_wait(bar(KF + st), use & 1, abortp, p.status))) break;
-            tc_fence_after();
-            const uint64_t kd = kd0 + ((st * kTile) >> 4), vd = vd0 + ((st * kTile) >> 4);
-            const uint32_t id = (keys == 128) ? id128 : id64;
+        if (!(ok = issue_sdp(gs, true))) break;
+        for (int x = 0; x < 2 * nst; ++x, ++gs) {
+          const int sw = x / nst, s = x % nst;
+          const int st = gs % kStagesK, buf = gs & 1;
+          // the next step's products go out before this step's lanes are done
+          if (x + 1 < 2 * nst && !(ok = issue_sdp(gs + 1, x + 1 < nst))) break;
+          if (!(ok = mbar_wait(bar(PF + buf), pfu[buf] & 1, abortp, p.status))) break;
+          ++pfu[buf];
+          if (sw == 0) continue;
+          // second sweep: dQ += dS K once the lanes have written dS over S
+          if (s == 0 && done > 0 && !(ok = mbar_wait(bar(OE), (done - 1) & 1, abortp, p.status))) break;
+          tc_fence_after();
+          const uint64_t kmn = kmn0 + ((st * kKV) >> 4);
+          const uint32_t tS = tmem + buf * 128;
 #pragma unroll
-            for (int kk = 0; kk < kD / 16; ++kk) {
-              const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
-              mma_ss(tS, qd + off, kd + off, id, kk > 0 ? 1u : 0u);
-            }
-#pragma unroll
-            for (int kk = 0; kk < kD / 16; ++kk) {
-              const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
-              mma_ss(tP, dod + off, vd + off, id, kk > 0 ? 1u : 0u);
-            }
-            tc_commit(bar(SF));
-            ++sf;
-            if (sw == 0) {
-              tc_commit(bar(KE + st));
-              pf_pending = true;
-              continue;
-            }
-            // second sweep: dQ += dS K once the lanes have written dS over S
-            if (!(ok = mbar_wait(bar(PF), (sf - 1) & 1, abortp, p.status))) break;
-            if (s == 0 && done > 0 && !(ok = mbar_wait(bar(OE), (done - 1) & 1, abortp, p.status))) break;
-            tc_fence_after();
-            const uint64_t kmn = kmn0 + ((st * kTile) >> 4);
-            for (int kk = 0; kk < keys / 16; ++kk)
-              mma_ts(tQ, tS + kk * 8, kmn + ((kk * 2048) >> 4), id_mn, (s > 0 || kk > 0) ? 1u : 0u);
-            tc_commit(bar(KE + st));
-          }
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ts(tQ, tS + kk * 8, kmn + ((kk * 2048) >> 4), id_mn, (s > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(bar(KE + st));
+        }
         if (!ok) break;
         tc_commit(bar(OF));
         tc_commit(bar(QE));
@@ -329,9 +394,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     // ------------------------------------------------ lanes (one row each)
     const int r = warp * 32 + lane;
     const uint32_t la = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    const uint32_t tS = la, tP = la + 128, tQ = la + 256;
+    const uint32_t tQ = la + 256;
     const float scale2 = p.scale * kLog2e;
-    int sf = 0, done = 0, rs = 0;
+    int gs = 0, done = 0, rs = 0;
+    int sfu[2] = {0, 0};
     bool ok = true;
     for (int64_t item = blockIdx.x; ok && item < items; item += gridDim.x) {
       int tile, i;
@@ -357,73 +423,62 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       const float lse2 = live ? lse * kLog2e : 0.0f;
       const int* list = p.lists + unit * p.idx_stride;
       const float* lg = p.logg + unit * p.idx_stride;
-      const int nsteps = (BS == 64) ? (n + 1) / 2 : n;
-      float Dt = 0.0f;
-      for (int sw = 0; ok && sw < 2; ++sw) {
-        for (int s = 0; s < nsteps; ++s) {
-          const int s0 = (BS == 64) ? 2 * s : s;
-          const int nblk = (BS == 64 && s0 + 1 < n) ? 2 : 1;
-          const int keys = nblk * BS > 128 ? 128 : nblk * BS;
-          const int j0 = list[s0], j1 = (nblk == 2) ? list[s0 + 1] : -1;
-          const float off0 = lg[s0] * kLog2e - lse2;
-          const float off1 = (nblk == 2) ? lg[s0 + 1] * kLog2e - lse2 : 0.0f;
-          if (!(ok = warp_wait_all(bar(SF), sf & 1, abortp, p.status))) break;
-          ++sf;
-          tc_fence_after();
-          float dl0 = 0.0f, dl1 = 0.0f;
-          for (int part = 0; part < keys / 32; ++part) {
-            uint32_t sv[32], dv[32];
-            tmem_ld32(tS + part * 32, sv);
-            tmem_ld32(tP + part * 32, dv);
-            const int kk0 = part * 32;
-            const bool second = (BS == 64) && kk0 >= 64;
-            const int jj = second ? j1 : j0;
-            const float off = second ? off1 : off0;
-            const int kbase = (BS == 64) ? (kk0 & 63) : kk0;   // key offset inside its block
-            const bool diag = (jj == i);
-            uint32_t pk[16];
+      const int nst = n * kHalves;
+      float Dt = 0.0f, dl = 0.0f;
+      for (int x = 0; ok && x < 2 * nst; ++x, ++gs) {
+        const int sw = x / nst, s = x % nst;
+        const int slot = s / kHalves, half = s % kHalves;
+        const int jj = list[slot];
+        const float off = lg[slot] * kLog2e - lse2;
+        const int buf = gs & 1;
+        if (!(ok = warp_wait_all(bar(SF + buf), sfu[buf] & 1, abortp, p.status))) break;
+        ++sfu[buf];
+        tc_fence_after();
+        const uint32_t tS = la + buf * 128, tP = tS + 64;
+        const bool diag = (jj == i);
+#pragma unroll 1
+        for (int part = 0; part < 2; ++part) {
+          uint32_t sv[32], dv[32];
+          tmem_ld32(tS + part * 32, sv);
+          tmem_ld32(tP + part * 32, dv);
+          const int kbase = half * 64 + part * 32;   // key offset inside block jj
+          uint32_t pk[16];
 #pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              float pe[2], de[2];
+          for (int e = 0; e < 32; e += 2) {
+            float de[2];
 #pragma unroll
-              for (int x = 0; x < 2; ++x) {
-                const bool on = live && !(diag && kbase + e + x > tb);
-                const float pv = on ? fast_exp2(fmaf(__uint_as_float(sv[e + x]), scale2, off)) : 0.0f;
-                const float dp = __uint_as_float(dv[e + x]);
-                if (sw == 0) {
-                  Dt = fmaf(pv, dp, Dt);
-                  de[x] = 0.0f;
-                } else {
-                  de[x] = on ? pv * (dp - Dt) : 0.0f;
-                }
-                pe[x] = pv;
-              }
-              if (sw == 1) {
-                pk[e >> 1] = pack_bf16x2(de[0], de[1]);
-                if (second) dl1 += de[0] + de[1];
-                else dl0 += de[0] + de[1];
+            for (int y = 0; y < 2; ++y) {
+              const bool on = live && !(diag && kbase + e + y > tb);
+              const float pv = on ? fast_exp2(fmaf(__uint_as_float(sv[e + y]), scale2, off)) : 0.0f;
+              const float dp = __uint_as_float(dv[e + y]);
+              if (sw == 0) {
+                Dt = fmaf(pv, dp, Dt);
+                de[y] = 0.0f;
+              } else {
+                de[y] = on ? pv * (dp - Dt) : 0.0f;
               }
             }
-            if (sw == 1) tmem_st16(tS + part * 16, pk);
-          }
-          if (sw == 1) {
-            tmem_wait_st();
-            // the rows' share of dlogg for this step's blocks, per warp
-#pragma unroll
-            for (int o = 16; o; o >>= 1) {
-              dl0 += __shfl_xor_sync(0xffffffffu, dl0, o);
-              dl1 += __shfl_xor_sync(0xffffffffu, dl1, o);
-            }
-            if (lane == 0) {
-              red[warp * kMaxList + s0] = dl0;
-              if (nblk == 2) red[warp * kMaxList + s0 + 1] = dl1;
+            if (sw == 1) {
+              pk[e >> 1] = pack_bf16x2(de[0], de[1]);
+              dl += de[0] + de[1];
             }
           }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(PF));
+          if (sw == 1) tmem_st16(tS + part * 16, pk);
         }
-        if (sw == 0 && valid) p.D[row] = Dt;
+        if (sw == 1) {
+          tmem_wait_st();
+          if (half == kHalves - 1) {
+            // the rows' share of dlogg for this block, per warp
+#pragma unroll
+            for (int o = 16; o; o >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, o);
+            if (lane == 0) red[warp * kMaxList + slot] = dl;
+            dl = 0.0f;
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(PF + buf));
+        if (sw == 0 && s == nst - 1 && valid) p.D[row] = Dt;
       }
       if (!ok) break;
       if (!(ok = warp_wait_all(bar(OF), done & 1, abortp, p.status))) break;
@@ -465,11 +520,17 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 }
 
 // ------------------------------------------------------------------ key-major
+// Chunks of 64 query rows; two S^T | dP^T buffers in tensor memory, so the
+// MMAs of chunk c+1 run while the lanes turn chunk c into P^T and dS^T.
 namespace km {
-constexpr uint32_t SM_K = 0, SM_V = kTile, SM_Q = 2 * kTile, SM_DO = 4 * kTile;   // Q, dO: two stages each
-constexpr uint32_t SM_ROW = 6 * kTile;                                            // float [2][2][128]
-constexpr uint32_t SM_BAR = SM_ROW + 2 * 2 * 128 * 4;
-enum { KVF = 0, KVE, CF, CE = CF + 2, SF = CE + 2, PF, OF, OE, RS, NBAR };   // RS: chunk row data written
+constexpr int kStagesC = 4;                                   // Q/dO chunk stages
+constexpr uint32_t kChunk = 64u * 128u * 2u;                  // 64 rows x 128 bf16
+constexpr uint32_t kChunkHalf = kChunk / 2;                   // 64 rows x 64 bf16
+constexpr uint32_t SM_K = 0, SM_V = kTile;
+constexpr uint32_t SM_Q = 2 * kTile, SM_DO = SM_Q + kStagesC * kChunk;
+constexpr uint32_t SM_ROW = SM_DO + kStagesC * kChunk;        // float [2 slots][2 arrays][64]
+constexpr uint32_t SM_BAR = SM_ROW + 2 * 2 * 64 * 4;
+enum { KVF = 0, KVE, CF, CE = CF + kStagesC, SF = CE + kStagesC, PF = SF + 2, OF = PF + 2, OE, RS, NBAR };
 constexpr uint32_t SM_MISC = SM_BAR + NBAR * 8;
 constexpr uint32_t kSmem = SM_MISC + 16 + 1024;
 }  // namespace km
@@ -485,29 +546,32 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   auto bar = [&](int b) -> uint32_t { return sb + SM_BAR + 8u * b; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM_MISC);
   volatile int* abortp = reinterpret_cast<volatile int*>(smem + SM_MISC + 4);
-  float* rowc = reinterpret_cast<float*>(smem + SM_ROW);   // [2][128] log2 offsets (logg - lse) * log2e
-  float* rowd = rowc + 2 * 128;                            // [2][128] D
+  float* rowc = reinterpret_cast<float*>(smem + SM_ROW);   // [2][64] log2 offsets (logg - lse) * log2e
+  float* rowd = rowc + 2 * 64;                             // [2][64] D
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int cpe = (BS == 128) ? p.G : (p.G + 1) / 2;   // 128-row chunks per (query block, key block)
+  // 64-row chunks per (query block, key block): one head each (bs 64), or
+  // the two halves of each head's 128 rows (bs 128)
+  const int cpe = (BS == 128) ? 2 * p.G : p.G;
   const int64_t items = static_cast<int64_t>(p.B) * p.Hkv * p.nb;
 
-  // never-loaded rows of the operand buffers (the upper 64 keys of a 64-token
-  // block, a missing second head of a chunk) must hold finite values: zero
-  // them once, before the first copy lands
+  // the upper 64 keys of a 64-token block are never loaded: zero them (and
+  // the rest of the K/V tiles) once, before the first copy lands
   if (warp < 4) {
     uint4* z = reinterpret_cast<uint4*>(smem);
-    for (uint32_t x = threadIdx.x; x < 6 * kTile / 16; x += 128) z[x] = make_uint4(0, 0, 0, 0);
+    for (uint32_t x = threadIdx.x; x < 2 * kTile / 16; x += 128) z[x] = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
   }
   if (threadIdx.x == 0) {
     mbar_init(bar(KVF), 1);
     mbar_init(bar(KVE), 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kStagesC; ++s) {
       mbar_init(bar(CF + s), 1);
       mbar_init(bar(CE + s), 1);
     }
-    mbar_init(bar(SF), 1);
-    mbar_init(bar(PF), 4);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(SF + b), 1);
+      mbar_init(bar(PF + b), 4);
+    }
     mbar_init(bar(OF), 1);
     mbar_init(bar(OE), 4);
     mbar_init(bar(RS), 128);
@@ -521,7 +585,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;   // S^T | dP^T | dV | dK
+  const uint32_t tmem = *tmem_slot;   // [S^T | dP^T] x 2 buffers (64 + 64 columns each) | dV | dK
 
   if (warp == 5) {
     if (lane == 0) {
@@ -547,84 +611,85 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         }
         ++kvc;
         for (int c = 0; ok && c < ne * cpe; ++c, ++gc) {
-          const int st = gc & 1, use = gc >> 1;
+          const int st = gc % kStagesC, use = gc / kStagesC;
           const int i = tl[c / cpe].x, hc = c % cpe;
-          if (gc >= 2 && !(ok = mbar_wait(bar(CE + st), (use - 1) & 1, abortp, p.status))) break;
-          int heads[2], rows0[2], npc = 0;
-          if (BS == 128) {
-            heads[0] = heads[1] = hc;
-            rows0[0] = i * 128;
-            rows0[1] = i * 128 + 64;
-            npc = 2;
-          } else {
-            heads[0] = 2 * hc;
-            heads[1] = 2 * hc + 1;
-            rows0[0] = rows0[1] = i * 64;
-            npc = (2 * hc + 1 < p.G) ? 2 : 1;
-          }
-          mbar_arrive_expect_tx(bar(CF + st), static_cast<uint32_t>(npc) * 4u * 8192u);
-          for (int pc = 0; pc < npc; ++pc) {
-            const int y = (b * p.Hq + g * p.G + heads[pc]) * p.N + rows0[pc];
-            for (int hf = 0; hf < 2; ++hf) {
-              tma_load_2d(sb + SM_Q + st * kTile + hf * kHalf + pc * 8192, &tmQ, bar(CF + st), hf * 64, y);
-              tma_load_2d(sb + SM_DO + st * kTile + hf * kHalf + pc * 8192, &tmDO, bar(CF + st), hf * 64, y);
-            }
+          const int hh = (BS == 128) ? hc >> 1 : hc;
+          const int r0 = (BS == 128) ? (hc & 1) * 64 : 0;
+          if (gc >= kStagesC && !(ok = mbar_wait(bar(CE + st), (use - 1) & 1, abortp, p.status))) break;
+          mbar_arrive_expect_tx(bar(CF + st), 4u * 8192u);
+          const int y = (b * p.Hq + g * p.G + hh) * p.N + i * BS + r0;
+          for (int hf = 0; hf < 2; ++hf) {
+            tma_load_2d(sb + SM_Q + st * kChunk + hf * kChunkHalf, &tmQ, bar(CF + st), hf * 64, y);
+            tma_load_2d(sb + SM_DO + st * kChunk + hf * kChunkHalf, &tmDO, bar(CF + st), hf * 64, y);
           }
         }
       }
       if (*abortp) {
         if (kvc > 0) mbar_drain(bar(KVF), (kvc - 1) & 1);
-        for (int s = max(0, gc - 2); s < gc; ++s) mbar_drain(bar(CF + (s & 1)), (s >> 1) & 1);
+        for (int s = max(0, gc - kStagesC); s < gc; ++s) mbar_drain(bar(CF + s % kStagesC), (s / kStagesC) & 1);
       }
     }
   } else if (warp == 4) {
     if (lane == 0) {
       // ------------------------------------------------ MMA issuer
-      const uint32_t id_k = idesc_bf16_f32(128, 128, 0, 0);
-      const uint32_t id_mn = idesc_bf16_f32(128, 128, 0, 1);
+      const uint32_t id_s = idesc_bf16_f32(128, 64, 0, 0);     // S^T, dP^T: 128 keys x 64 rows
+      const uint32_t id_mn = idesc_bf16_f32(128, 128, 0, 1);   // dV, dK: 128 keys x 128 channels
       const uint64_t kd = smem_desc_sw128(sb + SM_K, 16, 1024);
       const uint64_t vd = smem_desc_sw128(sb + SM_V, 16, 1024);
       const uint64_t qd0 = smem_desc_sw128(sb + SM_Q, 16, 1024);
       const uint64_t dod0 = smem_desc_sw128(sb + SM_DO, 16, 1024);
-      const uint64_t qmn0 = smem_desc_sw128(sb + SM_Q, kHalf, 1024);
-      const uint64_t domn0 = smem_desc_sw128(sb + SM_DO, kHalf, 1024);
-      const uint32_t tS = tmem, tP = tmem + 128, tV = tmem + 256, tK = tmem + 384;
-      int gc = 0, kvc = 0, sf = 0, done = 0;
+      const uint64_t qmn0 = smem_desc_sw128(sb + SM_Q, kChunkHalf, 1024);
+      const uint64_t domn0 = smem_desc_sw128(sb + SM_DO, kChunkHalf, 1024);
+      const uint32_t tV = tmem + 256, tK = tmem + 384;
+      int gc = 0, kvc = 0, done = 0;
+      int pfu[2] = {0, 0};   // P-ready phases consumed per buffer
       bool ok = true;
+      // S^T = K Q^T and dP^T = V dO^T of chunk number `cg` into buffer cg & 1
+      auto issue_sdp = [&](int cg) -> bool {
+        const int st = cg % kStagesC, buf = cg & 1;
+        if (!mbar_wait(bar(CF + st), (cg / kStagesC) & 1, abortp, p.status)) return false;
+        tc_fence_after();
+        const uint64_t qd = qd0 + ((st * kChunk) >> 4), dod = dod0 + ((st * kChunk) >> 4);
+        const uint32_t tS = tmem + buf * 128, tP = tS + 64;
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t oa = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
+          const uint32_t ob = ((kk >> 2) * kChunkHalf + (kk & 3) * 32) >> 4;
+          mma_ss(tS, kd + oa, qd + ob, id_s, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t oa = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
+          const uint32_t ob = ((kk >> 2) * kChunkHalf + (kk & 3) * 32) >> 4;
+          mma_ss(tP, vd + oa, dod + ob, id_s, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(SF + buf));
+        return true;
+      };
       for (int64_t item = blockIdx.x; ok && item < items; item += gridDim.x) {
         const int64_t bg = item / p.nb;
         const int j = static_cast<int>(item % p.nb);
         const int* off = p.toff + bg * (p.nb + 1);
-        const int ne = off[j + 1] - off[j];
-        if (ne == 0) continue;
+        const int nch = (off[j + 1] - off[j]) * cpe;
+        if (nch == 0) continue;
         if (!(ok = mbar_wait(bar(KVF), kvc & 1, abortp, p.status))) break;
         ++kvc;
-        for (int c = 0; c < ne * cpe; ++c, ++gc) {
-          const int st = gc & 1, use = gc >> 1;
-          if (!(ok = mbar_wait(bar(CF + st), use & 1, abortp, p.status))) break;
-          tc_fence_after();
-          const uint64_t qd = qd0 + ((st * kTile) >> 4), dod = dod0 + ((st * kTile) >> 4);
-#pragma unroll
-          for (int kk = 0; kk < kD / 16; ++kk) {
-            const uint32_t o = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
-            mma_ss(tS, kd + o, qd + o, id_k, kk > 0 ? 1u : 0u);
-          }
-#pragma unroll
-          for (int kk = 0; kk < kD / 16; ++kk) {
-            const uint32_t o = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
-            mma_ss(tP, vd + o, dod + o, id_k, kk > 0 ? 1u : 0u);
-          }
-          tc_commit(bar(SF));
-          ++sf;
-          if (!(ok = mbar_wait(bar(PF), (sf - 1) & 1, abortp, p.status))) break;
+        if (!(ok = issue_sdp(gc))) break;
+        for (int c = 0; c < nch; ++c, ++gc) {
+          const int st = gc % kStagesC, buf = gc & 1;
+          // the next chunk's products go out before this chunk's lanes are done
+          if (c + 1 < nch && !(ok = issue_sdp(gc + 1))) break;
+          if (!(ok = mbar_wait(bar(PF + buf), pfu[buf] & 1, abortp, p.status))) break;
+          ++pfu[buf];
           if (c == 0 && done > 0 && !(ok = mbar_wait(bar(OE), (done - 1) & 1, abortp, p.status))) break;
           tc_fence_after();
-          const uint64_t qmn = qmn0 + ((st * kTile) >> 4), domn = domn0 + ((st * kTile) >> 4);
+          const uint32_t tS = tmem + buf * 128, tP = tS + 64;
+          const uint64_t qmn = qmn0 + ((st * kChunk) >> 4), domn = domn0 + ((st * kChunk) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
+          for (int kk = 0; kk < 4; ++kk)
             mma_ts(tV, tS + kk * 8, domn + ((kk * 2048) >> 4), id_mn, (c > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
+          for (int kk = 0; kk < 4; ++kk)
             mma_ts(tK, tP + kk * 8, qmn + ((kk * 2048) >> 4), id_mn, (c > 0 || kk > 0) ? 1u : 0u);
           tc_commit(bar(CE + st));
         }
@@ -642,10 +707,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     // ------------------------------------------------ lanes (one key each)
     const int u = warp * 32 + lane;
     const uint32_t la = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    const uint32_t tS = la, tP = la + 128, tV = la + 256, tK = la + 384;
+    const uint32_t tV = la + 256, tK = la + 384;
     const float scale2 = p.scale * kLog2e;
     const bool kvalid = (BS == 128) || u < 64;
-    int gc = 0, sf = 0, done = 0;
+    int gc = 0, done = 0;
+    int sfu[2] = {0, 0};
     bool ok = true;
     for (int64_t item = blockIdx.x; ok && item < items; item += gridDim.x) {
       const int64_t bg = item / p.nb;
@@ -666,37 +732,35 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       for (int c = 0; c < ne * cpe; ++c, ++gc) {
         const int2 ent = tl[c / cpe];
         const int i = ent.x, hc = c % cpe;
-        const float lgv = p.logg[(bg * p.nb + i) * p.idx_stride + ent.y];
-        // this chunk's 128 rows: log2 offset (logg - LSE) * log2e, or -inf
-        // for a row that does not exist or attends to nothing; and D
-        {
-          const int x = u;   // chunk row handled by this thread
-          const int hh = (BS == 128) ? hc : 2 * hc + (x >> 6);
-          const int tb = (BS == 128) ? x : (x & 63);
+        const int hh = (BS == 128) ? hc >> 1 : hc;
+        const int r0 = (BS == 128) ? (hc & 1) * 64 : 0;   // first row of the chunk inside query block i
+        // this chunk's 64 rows: log2 offset (logg - LSE) * log2e, or -inf for
+        // a row that attends to nothing; and D
+        if (u < 64) {
+          const int64_t row = (static_cast<int64_t>(b) * p.Hq + g * p.G + hh) * p.N + static_cast<int64_t>(i) * BS + r0 + u;
+          const float lse = p.lse[row];
           float cv = -INFINITY, dvv = 0.0f;
-          if (hh < p.G) {
-            const int64_t row = (static_cast<int64_t>(b) * p.Hq + g * p.G + hh) * p.N + static_cast<int64_t>(i) * BS + tb;
-            const float lse = p.lse[row];
-            if (lse > -INFINITY) {
-              cv = (lgv - lse) * kLog2e;
-              dvv = p.D[row];
-            }
+          if (lse > -INFINITY) {
+            cv = (p.logg[(bg * p.nb + i) * p.idx_stride + ent.y] - lse) * kLog2e;
+            dvv = p.D[row];
           }
-          rowc[(gc & 1) * 128 + x] = cv;
-          rowd[(gc & 1) * 128 + x] = dvv;
+          rowc[(gc & 1) * 64 + u] = cv;
+          rowd[(gc & 1) * 64 + u] = dvv;
         }
         // (the other slot may still be read for the previous chunk: a thread
         // writes it again only after every thread has arrived for that chunk)
         mbar_arrive(bar(RS));
         if (!(ok = warp_wait_all(bar(RS), gc & 1, abortp, p.status))) break;
-        if (!(ok = warp_wait_all(bar(SF), sf & 1, abortp, p.status))) break;
-        ++sf;
+        const int buf = gc & 1;
+        if (!(ok = warp_wait_all(bar(SF + buf), sfu[buf] & 1, abortp, p.status))) break;
+        ++sfu[buf];
         tc_fence_after();
-        const float* rc = rowc + (gc & 1) * 128;
-        const float* rd = rowd + (gc & 1) * 128;
+        const float* rc = rowc + (gc & 1) * 64;
+        const float* rd = rowd + (gc & 1) * 64;
         const bool diag = (i == j);
+        const uint32_t tS = la + buf * 128, tP = tS + 64;
 #pragma unroll 1
-        for (int part = 0; part < 4; ++part) {
+        for (int part = 0; part < 2; ++part) {
           uint32_t sv[32], dv[32];
           tmem_ld32(tS + part * 32, sv);
           tmem_ld32(tP + part * 32, dv);
@@ -707,9 +771,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 #pragma unroll
             for (int x = 0; x < 2; ++x) {
               const int t = part * 32 + e + x;
-              const int tb = (BS == 128) ? t : (t & 63);
               const float cv = rc[t];
-              const bool on = kvalid && cv > -INFINITY && !(diag && u > tb);
+              const bool on = kvalid && cv > -INFINITY && !(diag && u > r0 + t);
               const float pv = on ? fast_exp2(fmaf(__uint_as_float(sv[e + x]), scale2, cv)) : 0.0f;
               pe[x] = pv;
               de[x] = on ? pv * (__uint_as_float(dv[e + x]) - rd[t]) : 0.0f;
@@ -723,7 +786,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(PF));
+        if (lane == 0) mbar_arrive(bar(PF + buf));
       }
       if (!ok) break;
       if (!(ok = warp_wait_all(bar(OF), done & 1, abortp, p.status))) break;
@@ -852,11 +915,13 @@ cudaError_t launch_attn_bwd(const CUtensorMap* tmQ, const CUtensorMap* tmDO, con
   bwd::gate_kernel<<<static_cast<unsigned>((units + 7) / 8), 256, 0, st>>>(idx, idx_stride, sel, nb, units, lists,
                                                                            counts, logg, status);
   const int bgs = B * Hkv;
-  bwd::transpose_kernel<<<(bgs + 63) / 64, 64, 0, st>>>(lists, counts, idx_stride, nb, bgs, toff, tlist);
+  const size_t tr_smem = bwd::transpose_smem_bytes(nb, idx_stride);
+  cudaError_t e = ensure_dynamic_smem<bwd::transpose_kernel>(tr_smem);
+  if (e != cudaSuccess) return e;
+  bwd::transpose_kernel<<<bgs, bwd::kTrThreads, tr_smem, st>>>(lists, counts, idx_stride, nb, toff, tlist);
   const int64_t items_q = units * p.tiles, items_k = static_cast<int64_t>(bgs) * nb;
   const unsigned grid_q = static_cast<unsigned>(items_q < num_sms ? items_q : num_sms);
   const unsigned grid_k = static_cast<unsigned>(items_k < num_sms ? items_k : num_sms);
-  cudaError_t e = cudaSuccess;
   if (bs == 64) {
     e = ensure_dynamic_smem<bwd::dq_tc_kernel<64>>(bwd::qm::kSmem);
     if (e == cudaSuccess) e = ensure_dynamic_smem<bwd::dkv_tc_kernel<64>>(bwd::km::kSmem);
