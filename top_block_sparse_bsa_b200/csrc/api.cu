@@ -404,7 +404,14 @@ bsa_status_t bsa_score_blocks(const bsa_shape_t* s, int mode, const void* q, con
     if (s->Nq != 1 || k == nullptr || !aligned16(k) || pooled_k_in || pooled_q_out || pooled_k_out)
       return BSA_ERR_INVALID_ARG;
     if (G > 16) return BSA_ERR_UNSUPPORTED;
-    return cuda_status(launch_score_gist(q, k, bf16, s->B, s->Hq, s->Hkv, nb, s->d, scale, scores, cs));
+    uint32_t* status = nullptr;
+    int sms = 0;
+    if ((st = device_state(&status, &sms)) != BSA_OK) return st;
+    CUtensorMap mg;
+    const bool tma = bf16 && s->d == 128;
+    if (tma && !make_map_bf16(&mg, k, static_cast<uint64_t>(s->B) * s->Hkv * nb, 64)) return BSA_ERR_CUDA;
+    return cuda_status(launch_score_gist(tma ? &mg : nullptr, q, k, bf16, s->B, s->Hq, s->Hkv, nb, s->d, scale,
+                                         scores, status, sms, cs));
   }
   return BSA_ERR_INVALID_ARG;
 }
@@ -627,7 +634,8 @@ bsa_status_t bsa_gist_expand_decode(const bsa_shape_t* s, const void* q, const v
     int* idx_dst = (idx_out && topk > 0) ? idx_out : reinterpret_cast<int*>(ws + L.idx);
     if (topk > 0) {
       float* sc = reinterpret_cast<float*>(ws + L.scores);
-      e = launch_score_gist(q, gist_k, true, s->B, s->Hq, s->Hkv, nc, s->d, score_scale(s->d), sc, cs);
+      e = launch_score_gist(&mgk, q, gist_k, true, s->B, s->Hq, s->Hkv, nc, s->d, score_scale(s->d), sc, status,
+                            sms, cs);
       if (e == cudaSuccess) e = launch_topk(sc, rows, nc, BSA_TOPK_PLAIN, topk, idx_dst, idx_stride, nullptr, cs);
     } else {
       e = cudaMemsetAsync(idx_dst, 0xff, static_cast<size_t>(rows) * sizeof(int), cs);
@@ -819,7 +827,8 @@ bsa_status_t bsa_hssa_decode(const bsa_shape_t* s, const void* q, const void* k_
   uint32_t* allow = reinterpret_cast<uint32_t*>(ws + L.allow);
   int* ulist = reinterpret_cast<int*>(ws + L.union_list);
   // coarse: meta-gist scores and the km best groups per head
-  cudaError_t e = launch_score_gist(q, meta_k, true, s->B, s->Hq, s->Hkv, nm, s->d, scale, meta_scores, cs);
+  cudaError_t e = launch_score_gist(&mmk, q, meta_k, true, s->B, s->Hq, s->Hkv, nm, s->d, scale, meta_scores, status,
+                                    sms, cs);
   if (e == cudaSuccess) e = launch_topk(meta_scores, rows, nm, BSA_TOPK_PLAIN, km, meta_idx, km, nullptr, cs);
   // fine: the gists of the kept groups' chunks and the topk best per head
   if (e == cudaSuccess) e = launch_score_gist_groups(q, gist_k, meta_idx, km, s->B, s->Hq, s->Hkv, nc, scale, fine, cs);

@@ -435,35 +435,45 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         ++sfu[buf];
         tc_fence_after();
         const uint32_t tS = la + buf * 128, tP = tS + 64;
-        const bool diag = (jj == i);
+        // keys of this step this row may see: all 64, or (the diagonal block)
+        // those not after the row, or none (a row that attends to nothing)
+        const int lim_step = !live ? 0 : (jj == i ? min(64, max(0, tb - half * 64 + 1)) : 64);
 #pragma unroll 1
         for (int part = 0; part < 2; ++part) {
           uint32_t sv[32], dv[32];
           tmem_ld32(tS + part * 32, sv);
           tmem_ld32(tP + part * 32, dv);
-          const int kbase = half * 64 + part * 32;   // key offset inside block jj
-          uint32_t pk[16];
+          const int lim = min(32, max(0, lim_step - part * 32));
+          if (sw == 0) {
+            // D_t += sum of P dP over the part, four independent partial sums
+            float a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            if (lim == 32) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            float de[2];
+              for (int e = 0; e < 32; ++e)
+                a[e & 3] = fmaf(fast_exp2(fmaf(__uint_as_float(sv[e]), scale2, off)), __uint_as_float(dv[e]), a[e & 3]);
+            } else {
 #pragma unroll
-            for (int y = 0; y < 2; ++y) {
-              const bool on = live && !(diag && kbase + e + y > tb);
-              const float pv = on ? fast_exp2(fmaf(__uint_as_float(sv[e + y]), scale2, off)) : 0.0f;
-              const float dp = __uint_as_float(dv[e + y]);
-              if (sw == 0) {
-                Dt = fmaf(pv, dp, Dt);
-                de[y] = 0.0f;
-              } else {
-                de[y] = on ? pv * (dp - Dt) : 0.0f;
+              for (int e = 0; e < 32; ++e) {
+                const float pv = (e < lim) ? fast_exp2(fmaf(__uint_as_float(sv[e]), scale2, off)) : 0.0f;
+                a[e & 3] = fmaf(pv, __uint_as_float(dv[e]), a[e & 3]);
               }
             }
-            if (sw == 1) {
+            Dt += (a[0] + a[1]) + (a[2] + a[3]);
+          } else {
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              float de[2];
+#pragma unroll
+              for (int y = 0; y < 2; ++y) {
+                const float pv = fast_exp2(fmaf(__uint_as_float(sv[e + y]), scale2, off));
+                de[y] = (e + y < lim) ? pv * (__uint_as_float(dv[e + y]) - Dt) : 0.0f;
+              }
               pk[e >> 1] = pack_bf16x2(de[0], de[1]);
               dl += de[0] + de[1];
             }
+            tmem_st16(tS + part * 16, pk);
           }
-          if (sw == 1) tmem_st16(tS + part * 16, pk);
         }
         if (sw == 1) {
           tmem_wait_st();
@@ -729,56 +739,72 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         continue;
       }
       const int2* tl = p.tlist + bg * static_cast<int64_t>(p.nb) * p.idx_stride + e0;
-      for (int c = 0; c < ne * cpe; ++c, ++gc) {
+      // a chunk's 64 rows: log2 offset (logg - LSE) * log2e, or -inf for a
+      // row that attends to nothing (its P is then exactly 0); and D.  Lane
+      // u < 64 reads row u of the next chunk while this one is processed.
+      auto row_data = [&](int c, float& cv, float& dvv) {
+        cv = -INFINITY;
+        dvv = 0.0f;
+        if (u >= 64 || c >= ne * cpe) return;
         const int2 ent = tl[c / cpe];
-        const int i = ent.x, hc = c % cpe;
+        const int hc = c % cpe;
         const int hh = (BS == 128) ? hc >> 1 : hc;
+        const int r0 = (BS == 128) ? (hc & 1) * 64 : 0;
+        const int64_t row =
+            (static_cast<int64_t>(b) * p.Hq + g * p.G + hh) * p.N + static_cast<int64_t>(ent.x) * BS + r0 + u;
+        const float lse = p.lse[row];
+        if (lse > -INFINITY) {
+          cv = (p.logg[(bg * p.nb + ent.x) * p.idx_stride + ent.y] - lse) * kLog2e;
+          dvv = p.D[row];
+        }
+      };
+      float cv_next, dv_next;
+      row_data(0, cv_next, dv_next);
+      for (int c = 0; c < ne * cpe; ++c, ++gc) {
+        const int i = tl[c / cpe].x, hc = c % cpe;
         const int r0 = (BS == 128) ? (hc & 1) * 64 : 0;   // first row of the chunk inside query block i
-        // this chunk's 64 rows: log2 offset (logg - LSE) * log2e, or -inf for
-        // a row that attends to nothing; and D
         if (u < 64) {
-          const int64_t row = (static_cast<int64_t>(b) * p.Hq + g * p.G + hh) * p.N + static_cast<int64_t>(i) * BS + r0 + u;
-          const float lse = p.lse[row];
-          float cv = -INFINITY, dvv = 0.0f;
-          if (lse > -INFINITY) {
-            cv = (p.logg[(bg * p.nb + i) * p.idx_stride + ent.y] - lse) * kLog2e;
-            dvv = p.D[row];
-          }
-          rowc[(gc & 1) * 64 + u] = cv;
-          rowd[(gc & 1) * 64 + u] = dvv;
+          rowc[(gc & 1) * 64 + u] = cv_next;
+          rowd[(gc & 1) * 64 + u] = dv_next;
         }
         // (the other slot may still be read for the previous chunk: a thread
         // writes it again only after every thread has arrived for that chunk)
         mbar_arrive(bar(RS));
+        row_data(c + 1, cv_next, dv_next);
         if (!(ok = warp_wait_all(bar(RS), gc & 1, abortp, p.status))) break;
         const int buf = gc & 1;
         if (!(ok = warp_wait_all(bar(SF + buf), sfu[buf] & 1, abortp, p.status))) break;
         ++sfu[buf];
         tc_fence_after();
-        const float* rc = rowc + (gc & 1) * 64;
-        const float* rd = rowd + (gc & 1) * 64;
-        const bool diag = (i == j);
+        const float4* rc4 = reinterpret_cast<const float4*>(rowc + (gc & 1) * 64);
+        const float4* rd4 = reinterpret_cast<const float4*>(rowd + (gc & 1) * 64);
+        // columns (rows of the chunk) this key may not see: all when the key
+        // does not exist, those before the key's position on the diagonal
+        const int tmin = !kvalid ? 64 : (i == j ? min(64, max(0, u - r0)) : 0);
         const uint32_t tS = la + buf * 128, tP = tS + 64;
 #pragma unroll 1
         for (int part = 0; part < 2; ++part) {
           uint32_t sv[32], dv[32];
           tmem_ld32(tS + part * 32, sv);
           tmem_ld32(tP + part * 32, dv);
+          const int m = min(32, max(0, tmin - part * 32));
           uint32_t pk[16], dk[16];
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            float pe[2], de[2];
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 c4 = rc4[part * 8 + e4], d4 = rd4[part * 8 + e4];
+            const float cc[4] = {c4.x, c4.y, c4.z, c4.w}, dd[4] = {d4.x, d4.y, d4.z, d4.w};
+            float pe[4], de[4];
 #pragma unroll
-            for (int x = 0; x < 2; ++x) {
-              const int t = part * 32 + e + x;
-              const float cv = rc[t];
-              const bool on = kvalid && cv > -INFINITY && !(diag && u > r0 + t);
-              const float pv = on ? fast_exp2(fmaf(__uint_as_float(sv[e + x]), scale2, cv)) : 0.0f;
-              pe[x] = pv;
-              de[x] = on ? pv * (__uint_as_float(dv[e + x]) - rd[t]) : 0.0f;
+            for (int y = 0; y < 4; ++y) {
+              const int e = e4 * 4 + y;
+              const float pv = (e >= m) ? fast_exp2(fmaf(__uint_as_float(sv[e]), scale2, cc[y])) : 0.0f;
+              pe[y] = pv;
+              de[y] = pv * (__uint_as_float(dv[e]) - dd[y]);
             }
-            pk[e >> 1] = pack_bf16x2(pe[0], pe[1]);
-            dk[e >> 1] = pack_bf16x2(de[0], de[1]);
+            pk[e4 * 2] = pack_bf16x2(pe[0], pe[1]);
+            pk[e4 * 2 + 1] = pack_bf16x2(pe[2], pe[3]);
+            dk[e4 * 2] = pack_bf16x2(de[0], de[1]);
+            dk[e4 * 2 + 1] = pack_bf16x2(de[2], de[3]);
           }
           tmem_st16(tS + part * 16, pk);
           tmem_st16(tP + part * 16, dk);

@@ -73,8 +73,11 @@ cudaError_t launch_score_prefill(const float* qbar, const float* kbar, int B, in
                                  float scale, float* s, cudaStream_t st);
 cudaError_t launch_score_decode(const void* q, bool bf16, const float* kbar, int B, int Hq, int Hkv,
                                 int nb, int d, float scale, float* s, float* qbar_out, cudaStream_t st);
-cudaError_t launch_score_gist(const void* q, const void* gk, bool bf16, int B, int Hq, int Hkv, int nc,
-                              int d, float scale, float* s, cudaStream_t st);
+// tmG: the gist keys as make_map_bf16 (rows B*Hkv*nc, box 64 rows), or null
+// (then the generic kernel runs; bf16 with d = 128 uses the TMA kernel).
+cudaError_t launch_score_gist(const CUtensorMap* tmG, const void* q, const void* gk, bool bf16, int B, int Hq,
+                              int Hkv, int nc, int d, float scale, float* s, uint32_t* status, int num_sms,
+                              cudaStream_t st);
 cudaError_t launch_topk(const float* scores, int rows, int ncols, int mode, int kb, int* idx_out,
                         int idx_stride, int* count_out, cudaStream_t st);
 cudaError_t launch_topk_pattern(const float* scores, int rows, int ncols, int sink, int local, int kb, int* idx_out,

@@ -475,68 +475,110 @@ __global__ void score_gist_kernel(const T* __restrict__ q, const T* __restrict__
         __fmul_rn(dot_fixed_order(qs + hh * d, ks + r * pitch, d, 1), scale);
 }
 
-// Gist, bf16, d = 128: grid (tiles of 64 gists, B*Hkv), 64*G threads = (head,
-// gist).  The tile's 64 gist keys are read with 16-byte loads (8 bf16 per
-// load, a warp covering 512 contiguous bytes) and widened into rows padded to
-// 132 floats, so float4 reads of eight consecutive rows fall in distinct
-// banks; each thread then runs the fixed-order dot product of its (head,
-// gist) pair, channels ascending, as the generic kernel does.
-__global__ void score_gist_bf16_d128_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ gk,
-                                            int Hq, int Hkv, int nc, float scale, float* __restrict__ s) {
-  constexpr int D = 128, kPitch = D + 4;
-  extern __shared__ __align__(16) float sm_gist[];
+// Gist, bf16, d = 128: persistent, 64*G threads = (head, gist of the tile).
+// A tile is 64 consecutive gist keys of one (b, g), brought into shared
+// memory by TMA (two 64-channel halves, 128-byte swizzle) kGistStages tiles
+// ahead, so the HBM stream does not stall on each tile's dot products.  The
+// swizzle puts the same 16-byte chunk of eight consecutive rows in distinct
+// banks, so each thread reads its gist row chunk by chunk, channels
+// ascending, and runs the fixed-order dot product of its (head, gist) pair,
+// as the generic kernel does.
+constexpr int kGistStages = 4;
+constexpr int kGistTileBytes = 64 * 128 * 2;
+
+__global__ void score_gist_bf16_d128_kernel(const __grid_constant__ CUtensorMap tmG, const __nv_bfloat16* __restrict__ q,
+                                            int Hq, int Hkv, int nc, int64_t tiles, float scale,
+                                            float* __restrict__ s, uint32_t* __restrict__ status) {
+  constexpr int D = 128;
+  extern __shared__ uint8_t sm_raw[];
+  uint8_t* sm_gist = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t full[kGistStages];
+  __shared__ float qs[16 * D];
+  __shared__ int abort_flag;
   const int G = Hq / Hkv;
-  float* ks = sm_gist;                // [64][kPitch]
-  float* qs = sm_gist + 64 * kPitch;  // [G][D]
-  const int64_t bg = blockIdx.y;
-  const int64_t b = bg / Hkv, g = bg % Hkv;
-  const int c0 = blockIdx.x * 64;
-  const int rows = min(64, nc - c0);
-  const uint4* src = reinterpret_cast<const uint4*>(gk + (bg * nc + c0) * D);
-  for (int e = threadIdx.x; e < rows * (D / 8); e += blockDim.x) {
-    const int r = e >> 4, c8 = e & 15;   // row, 8-channel chunk
-    const uint4 v = __ldg(src + e);
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
-    float4 lo, hi;
-    float2 f;
-    f = __bfloat1622float2(h[0]); lo.x = f.x; lo.y = f.y;
-    f = __bfloat1622float2(h[1]); lo.z = f.x; lo.w = f.y;
-    f = __bfloat1622float2(h[2]); hi.x = f.x; hi.y = f.y;
-    f = __bfloat1622float2(h[3]); hi.z = f.x; hi.w = f.y;
-    float4* dst = reinterpret_cast<float4*>(ks + r * kPitch + 8 * c8);
-    dst[0] = lo;
-    dst[1] = hi;
+  const int tpb = (nc + 63) / 64;   // tiles per (b, g)
+  const uint32_t sbase = smem_u32(sm_gist);
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tmG);
+    for (int i = 0; i < kGistStages; ++i) mbar_init(smem_u32(&full[i]), 1);
+    abort_flag = 0;
+    fence_barrier_init();
   }
-  for (int e = threadIdx.x; e < G * D; e += blockDim.x)
-    qs[e] = __bfloat162float(q[(b * Hq + g * G) * D + e]);
   __syncthreads();
+  auto issue = [&](int64_t tile, int stage) {
+    const int64_t bg = tile / tpb;
+    const int c0 = static_cast<int>(tile % tpb) * 64;
+    const uint32_t bar = smem_u32(&full[stage]);
+    mbar_arrive_expect_tx(bar, kGistTileBytes);   // rows past the last gist are zero-filled
+    const int y = static_cast<int>(bg * nc + c0);
+    tma_load_2d(sbase + stage * kGistTileBytes, &tmG, bar, 0, y);
+    tma_load_2d(sbase + stage * kGistTileBytes + kGistTileBytes / 2, &tmG, bar, 64, y);
+  };
+  if (threadIdx.x == 0)
+    for (int i = 0; i < kGistStages; ++i) {
+      const int64_t tile = blockIdx.x + static_cast<int64_t>(i) * gridDim.x;
+      if (tile < tiles) issue(tile, i);
+    }
   const int hh = threadIdx.x / 64, r = threadIdx.x % 64;
-  if (hh >= G || r >= rows) return;
-  const float4* kr = reinterpret_cast<const float4*>(ks + r * kPitch);
-  const float4* qr = reinterpret_cast<const float4*>(qs + hh * D);
-  float acc = 0.0f;
+  int k = 0;
+  for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++k) {
+    const int stage = k % kGistStages;
+    const int64_t bg = tile / tpb;
+    const int64_t b = bg / Hkv, g = bg % Hkv;
+    const int c0 = static_cast<int>(tile % tpb) * 64;
+    const int rows = min(64, nc - c0);
+    for (int e = threadIdx.x; e < G * D; e += blockDim.x) qs[e] = __bfloat162float(q[(b * Hq + g * G) * D + e]);
+    const bool ok = mbar_wait(smem_u32(&full[stage]), (k / kGistStages) & 1, &abort_flag, status);
+    __syncthreads();
+    if (ok && hh < G && r < rows) {
+      const uint8_t* tb = sm_gist + stage * kGistTileBytes + r * 128;
+      const float* qr = qs + hh * D;
+      float acc = 0.0f;
 #pragma unroll
-  for (int e = 0; e < D / 4; ++e) {
-    const float4 kv = kr[e], qv = qr[e];
-    acc = __fadd_rn(acc, __fmul_rn(qv.x, kv.x));
-    acc = __fadd_rn(acc, __fmul_rn(qv.y, kv.y));
-    acc = __fadd_rn(acc, __fmul_rn(qv.z, kv.z));
-    acc = __fadd_rn(acc, __fmul_rn(qv.w, kv.w));
+      for (int x = 0; x < 16; ++x) {
+        // chunk x (channels 8x .. 8x+7): half x / 8, 16-byte slot (x % 8) ^ (r % 8)
+        const uint4 w = *reinterpret_cast<const uint4*>(tb + (x >> 3) * (kGistTileBytes / 2) + (((x & 7) ^ (r & 7)) << 4));
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+          acc = __fadd_rn(acc, __fmul_rn(qr[8 * x + 2 * y], __uint_as_float(ws[y] << 16)));
+          acc = __fadd_rn(acc, __fmul_rn(qr[8 * x + 2 * y + 1], __uint_as_float(ws[y] & 0xFFFF0000u)));
+        }
+      }
+      s[((b * Hq + g * G + hh) * nc) + c0 + r] = __fmul_rn(acc, scale);
+    }
+    __syncthreads();   // the stage and the query rows are free again
+    if (!ok) break;
+    if (threadIdx.x == 0) {
+      const int64_t next = tile + static_cast<int64_t>(kGistStages) * gridDim.x;
+      if (next < tiles) issue(next, stage);
+    }
   }
-  s[((b * Hq + g * G + hh) * nc) + c0 + r] = __fmul_rn(acc, scale);
+  if (threadIdx.x == 0 && abort_flag) {
+    // let the copies in flight land before the CTA exits
+    for (int i = 0; i < kGistStages; ++i) {
+      const int kk = k + i;
+      const int64_t tile = blockIdx.x + static_cast<int64_t>(kk) * gridDim.x;
+      if (tile < tiles) mbar_drain(smem_u32(&full[kk % kGistStages]), (kk / kGistStages) & 1);
+    }
+  }
 }
 
-cudaError_t launch_score_gist(const void* q, const void* gk, bool bf16, int B, int Hq, int Hkv, int nc,
-                              int d, float scale, float* s, cudaStream_t st) {
+cudaError_t launch_score_gist(const CUtensorMap* tmG, const void* q, const void* gk, bool bf16, int B, int Hq,
+                              int Hkv, int nc, int d, float scale, float* s, uint32_t* status, int num_sms,
+                              cudaStream_t st) {
   const int G = Hq / Hkv;
   dim3 grid((nc + 63) / 64, B * Hkv);
-  if (bf16 && d == 128) {
-    const size_t smem2 = (64 * (128 + 4) + G * 128) * sizeof(float);
+  if (tmG != nullptr && bf16 && d == 128 && G <= 16) {
+    const size_t smem2 = static_cast<size_t>(kGistStages) * kGistTileBytes + 1024;   // + alignment slack
     cudaError_t e = ensure_dynamic_smem<score_gist_bf16_d128_kernel>(smem2);
     if (e != cudaSuccess) return e;
-    score_gist_bf16_d128_kernel<<<grid, 64 * G, smem2, st>>>(static_cast<const __nv_bfloat16*>(q),
-                                                             static_cast<const __nv_bfloat16*>(gk), Hq, Hkv, nc,
-                                                             scale, s);
+    const int64_t tiles = static_cast<int64_t>(B) * Hkv * ((nc + 63) / 64);
+    const int64_t want = static_cast<int64_t>(num_sms) * 2;
+    const unsigned ctas = static_cast<unsigned>(tiles < want ? tiles : want);
+    if (ctas == 0) return cudaSuccess;
+    score_gist_bf16_d128_kernel<<<ctas, 64 * G, smem2, st>>>(*tmG, static_cast<const __nv_bfloat16*>(q), Hq, Hkv,
+                                                             nc, tiles, scale, s, status);
     return cudaGetLastError();
   }
   const size_t smem = (G * d + 64 * (d + 1)) * sizeof(float);
