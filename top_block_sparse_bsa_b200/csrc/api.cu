@@ -831,7 +831,7 @@ bsa_status_t bsa_hssa_decode(const bsa_shape_t* s, const void* q, const void* k_
                                     sms, cs);
   if (e == cudaSuccess) e = launch_topk(meta_scores, rows, nm, BSA_TOPK_PLAIN, km, meta_idx, km, nullptr, cs);
   // fine: the gists of the kept groups' chunks and the topk best per head
-  if (e == cudaSuccess) e = launch_score_gist_groups(q, gist_k, meta_idx, km, s->B, s->Hq, s->Hkv, nc, scale, fine, cs);
+  if (e == cudaSuccess) e = launch_score_gist_groups(&mgk, q, meta_idx, km, s->B, s->Hq, s->Hkv, nc, scale, fine, status, cs);
   if (e == cudaSuccess)
     e = launch_topk(fine, rows, km * 64, BSA_TOPK_PLAIN, topk, pos, L.k_stride, nullptr, cs);
   if (e == cudaSuccess)

@@ -425,11 +425,19 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       const float* lg = p.logg + unit * p.idx_stride;
       const int nst = n * kHalves;
       float Dt = 0.0f, dl = 0.0f;
+      // the next step's block and gate weight are read one step ahead
+      int jj_next = list[0];
+      float lg_next = lg[0];
       for (int x = 0; ok && x < 2 * nst; ++x, ++gs) {
         const int sw = x / nst, s = x % nst;
         const int slot = s / kHalves, half = s % kHalves;
-        const int jj = list[slot];
-        const float off = lg[slot] * kLog2e - lse2;
+        const int jj = jj_next;
+        const float off = lg_next * kLog2e - lse2;
+        if (x + 1 < 2 * nst) {
+          const int slot1 = ((x + 1) % nst) / kHalves;
+          jj_next = list[slot1];
+          lg_next = lg[slot1];
+        }
         const int buf = gs & 1;
         if (!(ok = warp_wait_all(bar(SF + buf), sfu[buf] & 1, abortp, p.status))) break;
         ++sfu[buf];
@@ -742,11 +750,12 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       // a chunk's 64 rows: log2 offset (logg - LSE) * log2e, or -inf for a
       // row that attends to nothing (its P is then exactly 0); and D.  Lane
       // u < 64 reads row u of the next chunk while this one is processed.
-      auto row_data = [&](int c, float& cv, float& dvv) {
+      auto row_data = [&](int c, float& cv, float& dvv, int2& ent) {
         cv = -INFINITY;
         dvv = 0.0f;
-        if (u >= 64 || c >= ne * cpe) return;
-        const int2 ent = tl[c / cpe];
+        if (c >= ne * cpe) return;
+        ent = tl[c / cpe];
+        if (u >= 64) return;
         const int hc = c % cpe;
         const int hh = (BS == 128) ? hc >> 1 : hc;
         const int r0 = (BS == 128) ? (hc & 1) * 64 : 0;
@@ -759,9 +768,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         }
       };
       float cv_next, dv_next;
-      row_data(0, cv_next, dv_next);
+      int2 ent_next = make_int2(0, 0);
+      row_data(0, cv_next, dv_next, ent_next);
       for (int c = 0; c < ne * cpe; ++c, ++gc) {
-        const int i = tl[c / cpe].x, hc = c % cpe;
+        const int i = ent_next.x, hc = c % cpe;
         const int r0 = (BS == 128) ? (hc & 1) * 64 : 0;   // first row of the chunk inside query block i
         if (u < 64) {
           rowc[(gc & 1) * 64 + u] = cv_next;
@@ -770,7 +780,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         // (the other slot may still be read for the previous chunk: a thread
         // writes it again only after every thread has arrived for that chunk)
         mbar_arrive(bar(RS));
-        row_data(c + 1, cv_next, dv_next);
+        row_data(c + 1, cv_next, dv_next, ent_next);
         if (!(ok = warp_wait_all(bar(RS), gc & 1, abortp, p.status))) break;
         const int buf = gc & 1;
         if (!(ok = warp_wait_all(bar(SF + buf), sfu[buf] & 1, abortp, p.status))) break;

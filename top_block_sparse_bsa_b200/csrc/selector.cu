@@ -476,9 +476,11 @@ __global__ void score_gist_kernel(const T* __restrict__ q, const T* __restrict__
 }
 
 // Gist, bf16, d = 128: persistent, 64*G threads = (head, gist of the tile).
-// A tile is 64 consecutive gist keys of one (b, g), brought into shared
-// memory by TMA (two 64-channel halves, 128-byte swizzle) kGistStages tiles
-// ahead, so the HBM stream does not stall on each tile's dot products.  The
+// A tile is 64 consecutive gist keys of one (b, g); each CTA takes a
+// contiguous range of tiles (so the group's query rows are staged once per
+// (b, g), not per tile), brought into shared memory by TMA (two 64-channel
+// halves, 128-byte swizzle) kGistStages tiles ahead, so the HBM stream does
+// not stall on each tile's dot products.  The
 // swizzle puts the same 16-byte chunk of eight consecutive rows in distinct
 // banks, so each thread reads its gist row chunk by chunk, channels
 // ascending, and runs the fixed-order dot product of its (head, gist) pair,
@@ -486,7 +488,9 @@ __global__ void score_gist_kernel(const T* __restrict__ q, const T* __restrict__
 constexpr int kGistStages = 4;
 constexpr int kGistTileBytes = 64 * 128 * 2;
 
-__global__ void score_gist_bf16_d128_kernel(const __grid_constant__ CUtensorMap tmG, const __nv_bfloat16* __restrict__ q,
+// 64 * G threads, up to 1024 (G <= 16): registers capped so every group width launches.
+__global__ void __launch_bounds__(1024) score_gist_bf16_d128_kernel(const __grid_constant__ CUtensorMap tmG,
+                                                                   const __nv_bfloat16* __restrict__ q,
                                             int Hq, int Hkv, int nc, int64_t tiles, float scale,
                                             float* __restrict__ s, uint32_t* __restrict__ status) {
   constexpr int D = 128;
@@ -505,6 +509,9 @@ __global__ void score_gist_bf16_d128_kernel(const __grid_constant__ CUtensorMap 
     fence_barrier_init();
   }
   __syncthreads();
+  // this CTA's tiles: [t0, t1)
+  const int64_t per = (tiles + gridDim.x - 1) / gridDim.x;
+  const int64_t t0 = min(tiles, static_cast<int64_t>(blockIdx.x) * per), t1 = min(tiles, t0 + per);
   auto issue = [&](int64_t tile, int stage) {
     const int64_t bg = tile / tpb;
     const int c0 = static_cast<int>(tile % tpb) * 64;
@@ -515,19 +522,20 @@ __global__ void score_gist_bf16_d128_kernel(const __grid_constant__ CUtensorMap 
     tma_load_2d(sbase + stage * kGistTileBytes + kGistTileBytes / 2, &tmG, bar, 64, y);
   };
   if (threadIdx.x == 0)
-    for (int i = 0; i < kGistStages; ++i) {
-      const int64_t tile = blockIdx.x + static_cast<int64_t>(i) * gridDim.x;
-      if (tile < tiles) issue(tile, i);
-    }
+    for (int i = 0; i < kGistStages && t0 + i < t1; ++i) issue(t0 + i, i);
   const int hh = threadIdx.x / 64, r = threadIdx.x % 64;
   int k = 0;
-  for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++k) {
+  int64_t qbg = -1;   // (b, g) whose query rows are in qs
+  for (int64_t tile = t0; tile < t1; ++tile, ++k) {
     const int stage = k % kGistStages;
     const int64_t bg = tile / tpb;
     const int64_t b = bg / Hkv, g = bg % Hkv;
     const int c0 = static_cast<int>(tile % tpb) * 64;
     const int rows = min(64, nc - c0);
-    for (int e = threadIdx.x; e < G * D; e += blockDim.x) qs[e] = __bfloat162float(q[(b * Hq + g * G) * D + e]);
+    if (bg != qbg) {
+      for (int e = threadIdx.x; e < G * D; e += blockDim.x) qs[e] = __bfloat162float(q[(b * Hq + g * G) * D + e]);
+      qbg = bg;
+    }
     const bool ok = mbar_wait(smem_u32(&full[stage]), (k / kGistStages) & 1, &abort_flag, status);
     __syncthreads();
     if (ok && hh < G && r < rows) {
@@ -547,19 +555,17 @@ __global__ void score_gist_bf16_d128_kernel(const __grid_constant__ CUtensorMap 
       }
       s[((b * Hq + g * G + hh) * nc) + c0 + r] = __fmul_rn(acc, scale);
     }
-    __syncthreads();   // the stage and the query rows are free again
+    // the stage is free again; so are the query rows if the next tile
+    // belongs to another (b, g)
+    __syncthreads();
     if (!ok) break;
-    if (threadIdx.x == 0) {
-      const int64_t next = tile + static_cast<int64_t>(kGistStages) * gridDim.x;
-      if (next < tiles) issue(next, stage);
-    }
+    if (threadIdx.x == 0 && tile + kGistStages < t1) issue(tile + kGistStages, stage);
   }
   if (threadIdx.x == 0 && abort_flag) {
     // let the copies in flight land before the CTA exits
     for (int i = 0; i < kGistStages; ++i) {
       const int kk = k + i;
-      const int64_t tile = blockIdx.x + static_cast<int64_t>(kk) * gridDim.x;
-      if (tile < tiles) mbar_drain(smem_u32(&full[kk % kGistStages]), (kk / kGistStages) & 1);
+      if (t0 + kk < t1) mbar_drain(smem_u32(&full[kk % kGistStages]), (kk / kGistStages) & 1);
     }
   }
 }
@@ -1157,66 +1163,111 @@ cudaError_t launch_topk_joint(const float* scores, int rows, int G, int nb, int 
                           idx_stride, count_out);
 }
 
-// ------------------------------------------------- two-level gists: fine scores
-// H-SSA's fine step (SSA page, 层级扩展): query head (b, h) scores the gists of
-// the chunks inside its t-th kept group (64 chunks per group).  Grid (km,
-// B*Hq), 64 threads = the group's chunks; the group's 64 gist rows are read
-// with 16-byte loads into padded float rows, then each thread runs the
-// fixed-order dot product of its chunk's gist (as score_gist_bf16_d128_kernel).
-// fine [B*Hq][km*64]: position t*64 + x.  A group slot past the kept ones
-// gets NaN (never ranked above a number).
-__global__ void __launch_bounds__(64) score_gist_groups_kernel(const __nv_bfloat16* __restrict__ q,
-                                                               const __nv_bfloat16* __restrict__ gk,
-                                                               const int* __restrict__ meta_idx, int km, int Hq,
-                                                               int Hkv, int nc, float scale,
-                                                               float* __restrict__ fine) {
-  griddep_wait();   // the kept groups come from the kernel launched before
-  constexpr int D = 128, kPitch = D + 4;
-  __shared__ __align__(16) float ks[64 * kPitch];
-  __shared__ __align__(16) float qs[D];
-  const int t = blockIdx.x;
-  const int64_t row = blockIdx.y;   // b * Hq + h
+// Two-level gists, fine stage: for row (b, h) and each of its km kept groups
+// t (meta_idx), the scores of the group's 64 chunk gists.  One CTA per row,
+// 256 threads = four groups at a time x 64 gists; the group tiles arrive by
+// TMA (two 64-channel halves, 128-byte swizzle) in a four-stage ring, the
+// next round's tiles loading while this round's dot products run.  Each
+// thread runs the fixed-order dot product of its gist, channels ascending
+// (as score_gist_bf16_d128_kernel).  fine [B*Hq][km*64]: position t*64 + x.
+// A group slot past the kept ones gets NaN (never ranked above a number).
+constexpr int kGroupStages = 4;
+
+__global__ void __launch_bounds__(256) score_gist_groups_kernel(const __grid_constant__ CUtensorMap tmG,
+                                                                const __nv_bfloat16* __restrict__ q,
+                                                                const int* __restrict__ meta_idx, int km, int Hq,
+                                                                int Hkv, int nc, float scale,
+                                                                float* __restrict__ fine,
+                                                                uint32_t* __restrict__ status) {
+  constexpr int D = 128;
+  extern __shared__ uint8_t sm_raw[];
+  uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t full[kGroupStages];
+  __shared__ float qs[D];
+  __shared__ int abort_flag;
+  const int64_t row = blockIdx.x;   // b * Hq + h
   const int64_t b = row / Hq;
   const int g = static_cast<int>(row % Hq) / (Hq / Hkv);
-  const int m = meta_idx[row * km + t];
-  float* out = fine + row * (static_cast<int64_t>(km) * 64) + t * 64;
-  if (m < 0 || m >= nc / 64) {
-    out[threadIdx.x] = __int_as_float(0x7fc00000);   // NaN
-    return;
+  const int grp = threadIdx.x >> 6, r = threadIdx.x & 63;
+  const uint32_t sbase = smem_u32(tiles);
+  const int nm = nc / 64;
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tmG);
+    for (int i = 0; i < kGroupStages; ++i) mbar_init(smem_u32(&full[i]), 1);
+    abort_flag = 0;
+    fence_barrier_init();
   }
-  const uint4* src = reinterpret_cast<const uint4*>(gk + ((b * Hkv + g) * static_cast<int64_t>(nc) + m * 64) * D);
-  for (int e = threadIdx.x; e < 64 * (D / 8); e += 64) {
-    const int r = e >> 4, c8 = e & 15;
-    const uint4 v = __ldg(src + e);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    float* dst = ks + r * kPitch + 8 * c8;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      dst[2 * i] = __uint_as_float(w[i] << 16);
-      dst[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-  }
-  for (int e = threadIdx.x; e < D; e += 64) qs[e] = __bfloat162float(q[row * D + e]);
   __syncthreads();
-  const float4* kr = reinterpret_cast<const float4*>(ks + threadIdx.x * kPitch);
-  const float4* qr = reinterpret_cast<const float4*>(qs);
-  float acc = 0.0f;
+  griddep_wait();   // the kept groups come from the kernel launched before
+  const int* mrow = meta_idx + row * km;
+  // tile t into stage t % kGroupStages; a slot without a valid group still
+  // completes its phase (an arrive without bytes), so the parities stay aligned
+  auto issue = [&](int t) {
+    const uint32_t bar = smem_u32(&full[t % kGroupStages]);
+    const int m = mrow[t];
+    if (m < 0 || m >= nm) {
+      mbar_arrive(bar);
+      return;
+    }
+    mbar_arrive_expect_tx(bar, 64 * D * 2);
+    const int y = static_cast<int>((b * Hkv + g) * static_cast<int64_t>(nc) + m * 64);
+    const uint32_t dst = sbase + (t % kGroupStages) * (64 * D * 2);
+    tma_load_2d(dst, &tmG, bar, 0, y);
+    tma_load_2d(dst + 64 * 128, &tmG, bar, 64, y);
+  };
+  int issued = 0;   // thread 0: tiles issued so far
+  if (threadIdx.x == 0)
+    for (; issued < km && issued < kGroupStages; ++issued) issue(issued);
+  if (threadIdx.x < D) qs[threadIdx.x] = __bfloat162float(q[row * D + threadIdx.x]);
+  __syncthreads();
+  float* out = fine + row * (static_cast<int64_t>(km) * 64);
+  bool ok = true;
+  for (int base = 0; base < km; base += kGroupStages) {
+    const int t = base + grp;
+    if (t < km) {
+      const int m = mrow[t];
+      const bool valid = m >= 0 && m < nm;
+      const bool got = mbar_wait(smem_u32(&full[t % kGroupStages]), (t / kGroupStages) & 1, &abort_flag, status);
+      ok = ok && got;
+      if (!valid) {
+        out[t * 64 + r] = __int_as_float(0x7fc00000);   // NaN
+      } else if (got) {
+        const uint8_t* tb = tiles + (t % kGroupStages) * (64 * D * 2) + r * 128;
+        float acc = 0.0f;
 #pragma unroll
-  for (int e = 0; e < D / 4; ++e) {
-    const float4 kv = kr[e], qv = qr[e];
-    acc = __fadd_rn(acc, __fmul_rn(qv.x, kv.x));
-    acc = __fadd_rn(acc, __fmul_rn(qv.y, kv.y));
-    acc = __fadd_rn(acc, __fmul_rn(qv.z, kv.z));
-    acc = __fadd_rn(acc, __fmul_rn(qv.w, kv.w));
+        for (int x = 0; x < 16; ++x) {
+          // chunk x (channels 8x .. 8x+7): half x / 8, 16-byte slot (x % 8) ^ (r % 8)
+          const uint4 w = *reinterpret_cast<const uint4*>(tb + (x >> 3) * (64 * 128) + (((x & 7) ^ (r & 7)) << 4));
+          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int y = 0; y < 4; ++y) {
+            acc = __fadd_rn(acc, __fmul_rn(qs[8 * x + 2 * y], __uint_as_float(ws[y] << 16)));
+            acc = __fadd_rn(acc, __fmul_rn(qs[8 * x + 2 * y + 1], __uint_as_float(ws[y] & 0xFFFF0000u)));
+          }
+        }
+        out[t * 64 + r] = __fmul_rn(acc, scale);
+      }
+    }
+    __syncthreads();   // this round's stages are free again
+    if (abort_flag) break;
+    if (threadIdx.x == 0)
+      for (; issued < km && issued < base + 2 * kGroupStages; ++issued) issue(issued);
   }
-  out[threadIdx.x] = __fmul_rn(acc, scale);
+  if (threadIdx.x == 0 && abort_flag) {
+    // let the copies in flight land before the CTA exits
+    for (int t = max(0, issued - kGroupStages); t < issued; ++t)
+      mbar_drain(smem_u32(&full[t % kGroupStages]), (t / kGroupStages) & 1);
+  }
 }
 
-cudaError_t launch_score_gist_groups(const void* q, const void* gk, const int* meta_idx, int km, int B, int Hq,
-                                     int Hkv, int nc, float scale, float* fine, cudaStream_t st) {
-  return launch_dependent(score_gist_groups_kernel, dim3(km, B * Hq), dim3(64), 0, st,
-                          static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(gk), meta_idx, km,
-                          Hq, Hkv, nc, scale, fine);
+cudaError_t launch_score_gist_groups(const CUtensorMap* tmG, const void* q, const int* meta_idx, int km, int B,
+                                     int Hq, int Hkv, int nc, float scale, float* fine, uint32_t* status,
+                                     cudaStream_t st) {
+  const size_t smem = static_cast<size_t>(kGroupStages) * 64 * 128 * 2 + 1024;   // + alignment slack
+  cudaError_t e = ensure_dynamic_smem<score_gist_groups_kernel>(smem);
+  if (e != cudaSuccess) return e;
+  return launch_dependent(score_gist_groups_kernel, dim3(B * Hq), dim3(256), smem, st, *tmG,
+                          static_cast<const __nv_bfloat16*>(q), meta_idx, km, Hq, Hkv, nc, scale, fine, status);
 }
 
 cudaError_t launch_topk(const float* scores, int rows, int ncols, int mode, int kb, int* idx_out,
