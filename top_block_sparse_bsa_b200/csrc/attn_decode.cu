@@ -629,7 +629,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Merge the partial records of one output row (b, h) (one warp per row):
-// the row's group was cut into nseg segments, one record each.
+// the row's group was cut into nseg segments, one record each.  Up to four
+// records are read in one round (every load issued before any is used), so
+// a row costs one memory round trip rather than one per segment.
 __global__ void combine_kernel(const float* __restrict__ partial, int rows, int G, int list_len, int64_t total,
                                int num_ctas, int max_slots, int d, int out_bf16, void* __restrict__ o,
                                float* __restrict__ lse) {
@@ -644,18 +646,40 @@ __global__ void combine_kernel(const float* __restrict__ partial, int rows, int 
   const int rec = d + 4;
   const float* pr = partial + static_cast<int64_t>(row) * max_slots * rec;
   float M = -INFINITY;
-  for (int s = 0; s < nseg; ++s) M = fmaxf(M, pr[s * rec]);
   float L = 0.0f;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int s = 0; s < nseg; ++s) {
-    const float ms = pr[s * rec];
-    if (ms == -INFINITY) continue;
-    const float w = exp2f(ms - M);
-    L += w * pr[s * rec + 1];
-    for (int e = 0; e < 4; ++e) {
-      const int c = lane + 32 * e;
-      if (c < d) acc[e] += w * pr[s * rec + 4 + c];
+  for (int s0 = 0; s0 < nseg; s0 += 4) {
+    float ms[4], ls[4], ov[4][4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const bool in = s0 + k < nseg;
+      const float* r = pr + (s0 + k) * rec;
+      ms[k] = in ? r[0] : -INFINITY;
+      ls[k] = in ? r[1] : 0.0f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int c = lane + 32 * e;
+        ov[k][e] = (in && c < d) ? r[4 + c] : 0.0f;
+      }
     }
+    // fold this round into the running (M, L, acc), segments in order
+    float Mn = M;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) Mn = fmaxf(Mn, ms[k]);
+    if (Mn == -INFINITY) continue;
+    const float a = (M == -INFINITY) ? 0.0f : exp2f(M - Mn);
+    L *= a;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[e] *= a;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if (ms[k] == -INFINITY) continue;
+      const float w = exp2f(ms[k] - Mn);
+      L += w * ls[k];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[e] += w * ov[k][e];
+    }
+    M = Mn;
   }
   const float inv = (L > 0.0f) ? 1.0f / L : 0.0f;
   for (int e = 0; e < 4; ++e) {
