@@ -8,9 +8,11 @@
 // §1-2, §4.5), optionally with the SAS log-gate log g_j on every key of kept
 // block j (SAS page, 核心模块 2-3).
 //
-// One CTA per (query block i, query head h, batch b); one thread per query
-// row.  Each kept K/V block is staged in shared memory and every thread runs
-// an online softmax over its keys.
+// One CTA per (query block i, query head h, batch b); four threads per query
+// row, each holding a quarter of the channels (dot products finished with two
+// shuffles).  Each kept K/V block is staged in shared memory; a row first
+// scores all of the block's keys (independent dot products), then moves its
+// running maximum once per block and accumulates the block's keys.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -76,12 +78,14 @@ __global__ void attn_prefill_f32_kernel(const float* __restrict__ q, const float
     if (lane == 0) s_n = count;
   }
   __syncthreads();
+  constexpr int DQ = D / 4;           // channels per thread
   const int n = s_n;
-  const int tpos = i * bs + t;
-  const float* qrow = q + ((static_cast<int64_t>(b) * Hq + h) * N + tpos) * D;
-  float qr[D], acc[D];
+  const int r = t >> 2, qt = t & 3;   // query row inside the block, channel quarter
+  const int tpos = i * bs + r;
+  const float* qrow = q + ((static_cast<int64_t>(b) * Hq + h) * N + tpos) * D + qt * DQ;
+  float qr[DQ], acc[DQ];
 #pragma unroll
-  for (int c = 0; c < D; ++c) {
+  for (int c = 0; c < DQ; ++c) {
     qr[c] = qrow[c];
     acc[c] = 0.0f;
   }
@@ -90,37 +94,56 @@ __global__ void attn_prefill_f32_kernel(const float* __restrict__ q, const float
     const int j = s_list[e];
     const float bias = s_bias[e];
     __syncthreads();
-    const float* kb = k + (bg * N + static_cast<int64_t>(j) * bs) * D;
-    const float* vb = v + (bg * N + static_cast<int64_t>(j) * bs) * D;
-    for (int x = threadIdx.x; x < bs * D; x += blockDim.x) {
-      ks[x] = kb[x];
-      vs[x] = vb[x];
+    const float4* kb = reinterpret_cast<const float4*>(k + (bg * N + static_cast<int64_t>(j) * bs) * D);
+    const float4* vb = reinterpret_cast<const float4*>(v + (bg * N + static_cast<int64_t>(j) * bs) * D);
+    for (int x = threadIdx.x; x < bs * D / 4; x += blockDim.x) {
+      reinterpret_cast<float4*>(ks)[x] = kb[x];
+      reinterpret_cast<float4*>(vs)[x] = vb[x];
     }
     __syncthreads();
-    const int umax = (j == i) ? t : bs - 1;   // causal inside the current block
-    for (int u = 0; u <= umax; ++u) {
-      float dot = 0.0f;
+    const int umax = (j == i) ? r : bs - 1;   // causal inside the current block
+    // the key loop runs to the warp's last row (r | 7: a warp holds 8 rows),
+    // so every lane takes part in the shuffles; keys past umax are masked
+    const int uend = (j == i) ? (r | 7) : bs - 1;
+    // scores of the block's keys in chunks of 16, the chunk's maximum first
+    for (int u0 = 0; u0 <= uend; u0 += 16) {
+      float sc[16];
 #pragma unroll
-      for (int c = 0; c < D; ++c) dot = fmaf(qr[c], ks[u * D + c], dot);
-      const float s = dot * scale + bias;
-      if (s > m) {
-        const float r = expf(m - s);   // m = -inf -> 0
-        l *= r;
+      for (int x = 0; x < 16; ++x) {
+        const float* kr = ks + (u0 + x) * D + qt * DQ;
+        float dot = 0.0f;
 #pragma unroll
-        for (int c = 0; c < D; ++c) acc[c] *= r;
-        m = s;
+        for (int c = 0; c < DQ; ++c) dot = fmaf(qr[c], kr[c], dot);
+        dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+        dot += __shfl_xor_sync(0xffffffffu, dot, 2);
+        sc[x] = (u0 + x <= umax) ? dot * scale + bias : -INFINITY;
       }
-      const float pw = expf(s - m);
-      l += pw;
+      float mb = sc[0];
 #pragma unroll
-      for (int c = 0; c < D; ++c) acc[c] = fmaf(pw, vs[u * D + c], acc[c]);
+      for (int x = 1; x < 16; ++x) mb = fmaxf(mb, sc[x]);
+      if (mb > m) {
+        const float rs = expf(m - mb);   // m = -inf -> 0
+        l *= rs;
+#pragma unroll
+        for (int c = 0; c < DQ; ++c) acc[c] *= rs;
+        m = mb;
+      }
+      if (m == -INFINITY) continue;   // every score so far is -inf (a -inf gate weight)
+#pragma unroll
+      for (int x = 0; x < 16; ++x) {
+        const float pw = expf(sc[x] - m);
+        l += pw;
+        const float* vr = vs + (u0 + x) * D + qt * DQ;
+#pragma unroll
+        for (int c = 0; c < DQ; ++c) acc[c] = fmaf(pw, vr[c], acc[c]);
+      }
     }
   }
-  float* orow = o + ((static_cast<int64_t>(b) * Hq + h) * N + tpos) * D;
+  float* orow = o + ((static_cast<int64_t>(b) * Hq + h) * N + tpos) * D + qt * DQ;
   const float inv = (l > 0.0f) ? 1.0f / l : 0.0f;
 #pragma unroll
-  for (int c = 0; c < D; ++c) orow[c] = acc[c] * inv;
-  if (lse) lse[(static_cast<int64_t>(b) * Hq + h) * N + tpos] = (l > 0.0f) ? m + logf(l) : -INFINITY;
+  for (int c = 0; c < DQ; ++c) orow[c] = acc[c] * inv;
+  if (lse && qt == 0) lse[(static_cast<int64_t>(b) * Hq + h) * N + tpos] = (l > 0.0f) ? m + logf(l) : -INFINITY;
 }
 
 }  // namespace f32path
@@ -134,14 +157,14 @@ cudaError_t launch_attn_prefill_f32(const float* q, const float* k, const float*
     cudaError_t e = cudaFuncSetAttribute(f32path::attn_prefill_f32_kernel<64>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    f32path::attn_prefill_f32_kernel<64><<<grid, a.bs, smem, st>>>(q, k, v, a.Hq, a.Hkv, a.N, a.bs, a.idx,
+    f32path::attn_prefill_f32_kernel<64><<<grid, 4 * a.bs, smem, st>>>(q, k, v, a.Hq, a.Hkv, a.N, a.bs, a.idx,
                                                                    a.idx_stride, a.sel_scores, a.softmax_scale,
                                                                    static_cast<float*>(a.o), a.lse, a.status);
   } else {
     cudaError_t e = cudaFuncSetAttribute(f32path::attn_prefill_f32_kernel<128>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    f32path::attn_prefill_f32_kernel<128><<<grid, a.bs, smem, st>>>(q, k, v, a.Hq, a.Hkv, a.N, a.bs, a.idx,
+    f32path::attn_prefill_f32_kernel<128><<<grid, 4 * a.bs, smem, st>>>(q, k, v, a.Hq, a.Hkv, a.N, a.bs, a.idx,
                                                                     a.idx_stride, a.sel_scores, a.softmax_scale,
                                                                     static_cast<float*>(a.o), a.lse, a.status);
   }

@@ -475,44 +475,46 @@ __global__ void score_gist_kernel(const T* __restrict__ q, const T* __restrict__
         __fmul_rn(dot_fixed_order(qs + hh * d, ks + r * pitch, d, 1), scale);
 }
 
-// Gist, bf16, d = 128: persistent, 64*G threads = (head, gist of the tile).
-// A tile is 64 consecutive gist keys of one (b, g); each CTA takes a
-// contiguous range of tiles (so the group's query rows are staged once per
-// (b, g), not per tile), brought into shared memory by TMA (two 64-channel
-// halves, 128-byte swizzle) kGistStages tiles ahead, so the HBM stream does
-// not stall on each tile's dot products.  The
-// swizzle puts the same 16-byte chunk of eight consecutive rows in distinct
-// banks, so each thread reads its gist row chunk by chunk, channels
-// ascending, and runs the fixed-order dot product of its (head, gist) pair,
-// as the generic kernel does.
-constexpr int kGistStages = 4;
+// Gist, bf16, d = 128: persistent; a thread owns one gist row of a tile and
+// a pair of the group's heads, so the two heads' fixed-order dot products
+// advance together in packed f32x2 products and sums (each lane rounded as
+// the scalar mul.rn / add.rn; channels ascending, as the generic kernel).  A
+// tile is 64 consecutive gist keys of one (b, g); each CTA takes a contiguous
+// range of tiles, R tiles at a time (R = threads / (64 x head pairs)), the
+// tiles brought in by TMA (two 64-channel halves, 128-byte swizzle, so the
+// same 16-byte chunk of eight consecutive rows sits in eight distinct bank
+// groups) two rounds ahead; the group's query rows are staged, as head-pair
+// interleaved floats, only when a slot's (b, g) changes.
 constexpr int kGistTileBytes = 64 * 128 * 2;
+constexpr int kGistMaxStages = 8;
 
-// 64 * G threads, up to 1024 (G <= 16): registers capped so every group width launches.
-__global__ void __launch_bounds__(1024) score_gist_bf16_d128_kernel(const __grid_constant__ CUtensorMap tmG,
-                                                                   const __nv_bfloat16* __restrict__ q,
-                                            int Hq, int Hkv, int nc, int64_t tiles, float scale,
-                                            float* __restrict__ s, uint32_t* __restrict__ status) {
+__global__ void __launch_bounds__(512) score_gist_bf16_d128_kernel(const __grid_constant__ CUtensorMap tmG,
+                                                                  const __nv_bfloat16* __restrict__ q, int Hq,
+                                                                  int Hkv, int nc, int64_t tiles, float scale,
+                                                                  float* __restrict__ s, uint32_t* __restrict__ status) {
   constexpr int D = 128;
   extern __shared__ uint8_t sm_raw[];
   uint8_t* sm_gist = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t full[kGistStages];
-  __shared__ float qs[16 * D];
+  __shared__ __align__(8) uint64_t full[kGistMaxStages];
+  __shared__ __align__(16) float qs[16 * D];   // per round slot: head pairs x channels x 2
   __shared__ int abort_flag;
-  const int G = Hq / Hkv;
-  const int tpb = (nc + 63) / 64;   // tiles per (b, g)
+  const int G = Hq / Hkv, HP = (G + 1) / 2;
+  const int tpt = 64 * HP;                     // threads per tile
+  const int R = blockDim.x / tpt;              // tiles per round
+  const int S = 2 * R;                         // stages: two rounds in flight
+  const int tpb = (nc + 63) / 64;              // tiles per (b, g)
   const uint32_t sbase = smem_u32(sm_gist);
   if (threadIdx.x == 0) {
     prefetch_tmap(&tmG);
-    for (int i = 0; i < kGistStages; ++i) mbar_init(smem_u32(&full[i]), 1);
+    for (int i = 0; i < S; ++i) mbar_init(smem_u32(&full[i]), 1);
     abort_flag = 0;
     fence_barrier_init();
   }
   __syncthreads();
-  // this CTA's tiles: [t0, t1)
   const int64_t per = (tiles + gridDim.x - 1) / gridDim.x;
   const int64_t t0 = min(tiles, static_cast<int64_t>(blockIdx.x) * per), t1 = min(tiles, t0 + per);
-  auto issue = [&](int64_t tile, int stage) {
+  auto issue = [&](int64_t tile) {
+    const int k = static_cast<int>(tile - t0), stage = k % S;
     const int64_t bg = tile / tpb;
     const int c0 = static_cast<int>(tile % tpb) * 64;
     const uint32_t bar = smem_u32(&full[stage]);
@@ -522,50 +524,71 @@ __global__ void __launch_bounds__(1024) score_gist_bf16_d128_kernel(const __grid
     tma_load_2d(sbase + stage * kGistTileBytes + kGistTileBytes / 2, &tmG, bar, 64, y);
   };
   if (threadIdx.x == 0)
-    for (int i = 0; i < kGistStages && t0 + i < t1; ++i) issue(t0 + i, i);
-  const int hh = threadIdx.x / 64, r = threadIdx.x % 64;
-  int k = 0;
-  int64_t qbg = -1;   // (b, g) whose query rows are in qs
-  for (int64_t tile = t0; tile < t1; ++tile, ++k) {
-    const int stage = k % kGistStages;
-    const int64_t bg = tile / tpb;
+    for (int64_t t = t0; t < t1 && t < t0 + S; ++t) issue(t);
+  const int slot = threadIdx.x / tpt, within = threadIdx.x % tpt;
+  const int pr = within / 64, r = within % 64;   // head pair, gist row
+  const bool active = slot < R;
+  float* qslot = qs + slot * (HP * 2 * D);
+  int64_t qbg = -1, cur = t0;
+  bool ok = true;
+  for (int64_t base = t0; base < t1; base += R) {
+    cur = base;
+    const int64_t tile = base + slot;
+    const bool mine = active && tile < t1;
+    const int64_t bg = mine ? tile / tpb : -1;
     const int64_t b = bg / Hkv, g = bg % Hkv;
-    const int c0 = static_cast<int>(tile % tpb) * 64;
-    const int rows = min(64, nc - c0);
-    if (bg != qbg) {
-      for (int e = threadIdx.x; e < G * D; e += blockDim.x) qs[e] = __bfloat162float(q[(b * Hq + g * G) * D + e]);
+    // the slot's query rows, head pair interleaved: [pair][channel][2]
+    if (mine && bg != qbg) {
+      for (int e = within; e < HP * D; e += tpt) {
+        const int p2 = e / D, c = e % D;
+        const int h0 = 2 * p2, h1 = 2 * p2 + 1;
+        qslot[(p2 * D + c) * 2] = __bfloat162float(q[(b * Hq + g * G + h0) * D + c]);
+        qslot[(p2 * D + c) * 2 + 1] = (h1 < G) ? __bfloat162float(q[(b * Hq + g * G + h1) * D + c]) : 0.0f;
+      }
       qbg = bg;
     }
-    const bool ok = mbar_wait(smem_u32(&full[stage]), (k / kGistStages) & 1, &abort_flag, status);
+    const int k = static_cast<int>(tile - t0), stage = k % S;
+    if (mine) ok = mbar_wait(smem_u32(&full[stage]), (k / S) & 1, &abort_flag, status) && ok;
     __syncthreads();
-    if (ok && hh < G && r < rows) {
-      const uint8_t* tb = sm_gist + stage * kGistTileBytes + r * 128;
-      const float* qr = qs + hh * D;
-      float acc = 0.0f;
+    if (mine && ok) {
+      const int c0 = static_cast<int>(tile % tpb) * 64;
+      if (r < min(64, nc - c0)) {
+        const uint8_t* tb = sm_gist + stage * kGistTileBytes + r * 128;
+        const float4* q4 = reinterpret_cast<const float4*>(qslot + pr * 2 * D);
+        uint64_t acc = f2_pack(0.0f, 0.0f);
 #pragma unroll
-      for (int x = 0; x < 16; ++x) {
-        // chunk x (channels 8x .. 8x+7): half x / 8, 16-byte slot (x % 8) ^ (r % 8)
-        const uint4 w = *reinterpret_cast<const uint4*>(tb + (x >> 3) * (kGistTileBytes / 2) + (((x & 7) ^ (r & 7)) << 4));
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+        for (int x = 0; x < 16; ++x) {
+          // chunk x (channels 8x .. 8x+7): half x / 8, 16-byte slot (x % 8) ^ (r % 8)
+          const uint4 w = *reinterpret_cast<const uint4*>(tb + (x >> 3) * (kGistTileBytes / 2) + (((x & 7) ^ (r & 7)) << 4));
+          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-        for (int y = 0; y < 4; ++y) {
-          acc = __fadd_rn(acc, __fmul_rn(qr[8 * x + 2 * y], __uint_as_float(ws[y] << 16)));
-          acc = __fadd_rn(acc, __fmul_rn(qr[8 * x + 2 * y + 1], __uint_as_float(ws[y] & 0xFFFF0000u)));
+          for (int y = 0; y < 4; ++y) {
+            const float4 qq = q4[4 * x + y];   // channels 8x+2y, 8x+2y+1, both heads
+            const float k0 = __uint_as_float(ws[y] << 16), k1 = __uint_as_float(ws[y] & 0xFFFF0000u);
+            acc = f2_add(acc, f2_mul(f2_pack(qq.x, qq.y), f2_pack(k0, k0)));
+            acc = f2_add(acc, f2_mul(f2_pack(qq.z, qq.w), f2_pack(k1, k1)));
+          }
         }
+        float a0, a1;
+        f2_unpack(acc, a0, a1);
+        const int h0 = 2 * pr, h1 = 2 * pr + 1;
+        s[((b * Hq + g * G + h0) * nc) + c0 + r] = __fmul_rn(a0, scale);
+        if (h1 < G) s[((b * Hq + g * G + h1) * nc) + c0 + r] = __fmul_rn(a1, scale);
       }
-      s[((b * Hq + g * G + hh) * nc) + c0 + r] = __fmul_rn(acc, scale);
     }
-    // the stage is free again; so are the query rows if the next tile
-    // belongs to another (b, g)
+    // the round's stages are free again; so are the query rows of a slot
+    // whose next tile belongs to another (b, g)
     __syncthreads();
-    if (!ok) break;
-    if (threadIdx.x == 0 && tile + kGistStages < t1) issue(tile + kGistStages, stage);
+    if (abort_flag) break;
+    if (threadIdx.x == 0)
+      for (int64_t t = base + S; t < t1 && t < base + S + R; ++t) issue(t);
   }
   if (threadIdx.x == 0 && abort_flag) {
-    // let the copies in flight land before the CTA exits
-    for (int i = 0; i < kGistStages; ++i) {
-      const int kk = k + i;
-      if (t0 + kk < t1) mbar_drain(smem_u32(&full[kk % kGistStages]), (kk / kGistStages) & 1);
+    // let the copies in flight land before the CTA exits: the tiles of the
+    // round that gave up and of the one issued ahead of it
+    for (int64_t t = cur; t < t1 && t < cur + S; ++t) {
+      const int k = static_cast<int>(t - t0);
+      mbar_drain(smem_u32(&full[k % S]), (k / S) & 1);
     }
   }
 }
@@ -576,15 +599,20 @@ cudaError_t launch_score_gist(const CUtensorMap* tmG, const void* q, const void*
   const int G = Hq / Hkv;
   dim3 grid((nc + 63) / 64, B * Hkv);
   if (tmG != nullptr && bf16 && d == 128 && G <= 16) {
-    const size_t smem2 = static_cast<size_t>(kGistStages) * kGistTileBytes + 1024;   // + alignment slack
+    const int HP = (G + 1) / 2;
+    const int threads = max(256, 64 * HP);
+    const int R = threads / (64 * HP);
+    const size_t smem2 = static_cast<size_t>(2 * R) * kGistTileBytes + 1024;   // + alignment slack
     cudaError_t e = ensure_dynamic_smem<score_gist_bf16_d128_kernel>(smem2);
     if (e != cudaSuccess) return e;
     const int64_t tiles = static_cast<int64_t>(B) * Hkv * ((nc + 63) / 64);
-    const int64_t want = static_cast<int64_t>(num_sms) * 2;
-    const unsigned ctas = static_cast<unsigned>(tiles < want ? tiles : want);
+    // as many CTAs as fit (one round of R tiles each at least)
+    const int64_t want = static_cast<int64_t>(num_sms) * (R >= 4 ? 1 : 2);
+    const int64_t need = (tiles + R - 1) / R;
+    const unsigned ctas = static_cast<unsigned>(need < want ? need : want);
     if (ctas == 0) return cudaSuccess;
-    score_gist_bf16_d128_kernel<<<ctas, 64 * G, smem2, st>>>(*tmG, static_cast<const __nv_bfloat16*>(q), Hq, Hkv,
-                                                             nc, tiles, scale, s, status);
+    score_gist_bf16_d128_kernel<<<ctas, threads, smem2, st>>>(*tmG, static_cast<const __nv_bfloat16*>(q), Hq, Hkv,
+                                                              nc, tiles, scale, s, status);
     return cudaGetLastError();
   }
   const size_t smem = (G * d + 64 * (d + 1)) * sizeof(float);
