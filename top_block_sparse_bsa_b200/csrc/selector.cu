@@ -116,15 +116,13 @@ static cudaError_t launch_pool_jobs(const PoolJob& j0, const PoolJob& j1, bool b
   return cudaGetLastError();
 }
 
-// Streamed variant (persistent, one CTA per SM): the work is the sequence of
-// runs (one head's bs*d contiguous elements of a unit), units of the query
-// job first, then those of the key job; each CTA takes a contiguous range of
-// units.  A producer thread copies consecutive runs -- several units' worth
-// when a unit has fewer heads than a buffer holds -- into kPoolStages
-// shared-memory buffers with bulk copies, while 128 threads sum earlier
-// buffers, column c by thread c, rows in the fixed order (head, then row), the
-// running sum carried across the runs (and buffers) of a unit and written out
-// with its last run.
+// Streamed variant (persistent, one CTA per SM): a producer thread copies each
+// unit's rows (heads_sum runs of bs*d contiguous elements) into
+// kPoolStages shared-memory buffers with bulk copies, a chunk of whole runs
+// per buffer, while 128 threads sum earlier chunks, column c by thread c,
+// rows in the fixed order (head, then row), the running sum carried from one
+// chunk of a unit to the next.  Units of the query job come first, then those
+// of the key job.
 constexpr int kPoolStreamBytes = 64 * 1024;
 constexpr int kPoolStages = 3;
 
@@ -142,34 +140,6 @@ __global__ void __launch_bounds__(160, 1) pool_stream_kernel(PoolJob jq, PoolJob
   const int64_t units = units_per_job * (jk.src ? 2 : 1);
   const uint32_t run = static_cast<uint32_t>(bs) * d * sizeof(T);       // one head's rows of a unit
   const int runs_per_chunk = static_cast<int>(kPoolStreamBytes / run);   // >= 1 (checked by the launcher)
-  // this CTA's units [u0, u1) and their runs [r0, r1): query units have
-  // jq.heads_sum runs each, key units jk.heads_sum; the split balances runs
-  // (bytes), each unit whole inside one CTA
-  auto run_start = [&](int64_t u) -> int64_t {   // global index of unit u's first run
-    return u <= units_per_job ? u * jq.heads_sum
-                              : units_per_job * jq.heads_sum + (u - units_per_job) * jk.heads_sum;
-  };
-  auto first_unit_at = [&](int64_t rr) -> int64_t {   // the first unit whose first run is >= rr
-    const int64_t qruns = units_per_job * jq.heads_sum;
-    if (rr <= qruns) return (rr + jq.heads_sum - 1) / jq.heads_sum;
-    return min(units, units_per_job + (rr - qruns + jk.heads_sum - 1) / jk.heads_sum);
-  };
-  const int64_t total_runs = run_start(units);
-  const int64_t rper = (total_runs + gridDim.x - 1) / gridDim.x;
-  const int64_t u0 = first_unit_at(min(total_runs, static_cast<int64_t>(blockIdx.x) * rper));
-  const int64_t u1 = first_unit_at(min(total_runs, static_cast<int64_t>(blockIdx.x + 1) * rper));
-  auto run_unit = [&](int64_t rr, int64_t& unit, int& head, bool& isk) {   // the unit and head of run rr
-    const int64_t qruns = units_per_job * jq.heads_sum;
-    isk = rr >= qruns;
-    if (!isk) {
-      unit = rr / jq.heads_sum;
-      head = static_cast<int>(rr % jq.heads_sum);
-    } else {
-      unit = (rr - qruns) / jk.heads_sum;
-      head = static_cast<int>((rr - qruns) % jk.heads_sum);
-    }
-  };
-  const int64_t r0 = run_start(u0), r1 = run_start(u1);
   if (threadIdx.x == 0) {
     for (int i = 0; i < kPoolStages; ++i) {
       mbar_init(bar(i), 1);
@@ -185,24 +155,23 @@ __global__ void __launch_bounds__(160, 1) pool_stream_kernel(PoolJob jq, PoolJob
     if ((threadIdx.x & 31) == 0) {
       int k = 0;   // chunks issued
       bool ok = true;
-      for (int64_t rc = r0; ok && rc < r1; rc += runs_per_chunk, ++k) {
-        const int nr = static_cast<int>(min(static_cast<int64_t>(runs_per_chunk), r1 - rc));
-        const int buf = k % kPoolStages, use = k / kPoolStages;
-        if (k >= kPoolStages && !(ok = mbar_wait(bar(kPoolStages + buf), (use - 1) & 1, ab, status))) break;
-        mbar_arrive_expect_tx(bar(buf), run * nr);
-        for (int x = 0; x < nr; ++x) {
-          int64_t unit;
-          int head;
-          bool isk;
-          run_unit(rc + x, unit, head, isk);
-          const PoolJob& job = isk ? jk : jq;
-          const int64_t b = unit / (static_cast<int64_t>(Hgroups) * nb);
-          const int64_t g = (unit / nb) % Hgroups;
-          const int64_t j = unit % nb;
-          const T* src = static_cast<const T*>(job.src);
-          bulk_load(sb + buf * kPoolStreamBytes + x * run,
-                    src + ((b * job.Hsrc + g * job.heads_sum + head) * static_cast<int64_t>(N) + j * bs) * d, run,
-                    bar(buf));
+      for (int64_t u = blockIdx.x; ok && u < units; u += gridDim.x) {
+        const bool isk = u >= units_per_job;
+        const PoolJob& job = isk ? jk : jq;
+        const int64_t unit = isk ? u - units_per_job : u;
+        const int64_t b = unit / (static_cast<int64_t>(Hgroups) * nb);
+        const int64_t g = (unit / nb) % Hgroups;
+        const int64_t j = unit % nb;
+        const T* src = static_cast<const T*>(job.src);
+        for (int h0 = 0; h0 < job.heads_sum; h0 += runs_per_chunk, ++k) {
+          const int nr = min(runs_per_chunk, job.heads_sum - h0);
+          const int buf = k % kPoolStages, use = k / kPoolStages;
+          if (k >= kPoolStages && !(ok = mbar_wait(bar(kPoolStages + buf), (use - 1) & 1, ab, status))) break;
+          mbar_arrive_expect_tx(bar(buf), run * nr);
+          for (int hh = h0; hh < h0 + nr; ++hh)
+            bulk_load(sb + buf * kPoolStreamBytes + (hh - h0) * run,
+                      src + ((b * job.Hsrc + g * job.heads_sum + hh) * static_cast<int64_t>(N) + j * bs) * d, run,
+                      bar(buf));
         }
       }
       if (*ab) {   // let the copies still in flight land before the CTA exits
@@ -214,31 +183,30 @@ __global__ void __launch_bounds__(160, 1) pool_stream_kernel(PoolJob jq, PoolJob
     const int c = threadIdx.x;   // column
     int k = 0;   // chunks consumed
     bool ok = true;
-    float acc = 0.0f;
-    for (int64_t rc = r0; ok && rc < r1; rc += runs_per_chunk, ++k) {
-      const int nr = static_cast<int>(min(static_cast<int64_t>(runs_per_chunk), r1 - rc));
-      const int buf = k % kPoolStages, use = k / kPoolStages;
-      if (!(ok = mbar_wait(bar(buf), use & 1, ab, status))) break;
-      for (int x = 0; x < nr; ++x) {
-        int64_t unit;
-        int head;
-        bool isk;
-        run_unit(rc + x, unit, head, isk);
-        const PoolJob& job = isk ? jk : jq;
-        if (head == 0) acc = 0.0f;
-        const T* sv = reinterpret_cast<const T*>(psmem + buf * kPoolStreamBytes + x * run);
+    for (int64_t u = blockIdx.x; ok && u < units; u += gridDim.x) {
+      const bool isk = u >= units_per_job;
+      const PoolJob& job = isk ? jk : jq;
+      const int64_t unit = isk ? u - units_per_job : u;
+      float acc = 0.0f;
+      for (int h0 = 0; h0 < job.heads_sum; h0 += runs_per_chunk, ++k) {
+        const int nr = min(runs_per_chunk, job.heads_sum - h0);
+        const int buf = k % kPoolStages, use = k / kPoolStages;
+        if (!(ok = mbar_wait(bar(buf), use & 1, ab, status))) break;
+        const T* sv = reinterpret_cast<const T*>(psmem + buf * kPoolStreamBytes);
+        const int rows = nr * bs;   // a multiple of 16
         if (c < d) {
-          for (int r = 0; r < bs; r += 16) {   // bs is a multiple of 16
-            float xv[16];
+          for (int r = 0; r < rows; r += 16) {
+            float x[16];
 #pragma unroll
-            for (int t = 0; t < 16; ++t) xv[t] = static_cast<float>(sv[(r + t) * d + c]);
+            for (int t = 0; t < 16; ++t) x[t] = static_cast<float>(sv[(r + t) * d + c]);
 #pragma unroll
-            for (int t = 0; t < 16; ++t) acc = __fadd_rn(acc, xv[t]);
+            for (int t = 0; t < 16; ++t) acc = __fadd_rn(acc, x[t]);
           }
-          if (head == job.heads_sum - 1) job.out[unit * d + c] = __fdiv_rn(acc, static_cast<float>(job.heads_sum * bs));
         }
+        mbar_arrive(bar(kPoolStages + buf));
       }
-      mbar_arrive(bar(kPoolStages + buf));
+      if (!ok) break;
+      if (c < d) job.out[unit * d + c] = __fdiv_rn(acc, static_cast<float>(job.heads_sum * bs));
     }
   }
   __syncthreads();
@@ -326,31 +294,47 @@ __global__ void __launch_bounds__(256) score_prefill_kernel(const float* __restr
     cp_async_wait_all();
   }
   __syncthreads();
-  float acc[4][4];
+  // acc2[a][p] holds the pair of sums (a, 2p) and (a, 2p+1), advanced by one
+  // packed f32x2 product and one packed sum per channel (each lane rounded as
+  // the scalar mul.rn / add.rn), channels ascending, four channels per
+  // shared-memory read
+  uint64_t acc2[4][2];
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
+  for (int a = 0; a < 4; ++a) acc2[a][0] = acc2[a][1] = f2_pack(0.0f, 0.0f);
+  for (int c = 0; c < d; c += 4) {
+    float4 qv[4], kv[4];
 #pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
-  for (int c = 0; c < d; ++c) {
-    float qv[4], kv[4];
+    for (int a = 0; a < 4; ++a) qv[a] = *reinterpret_cast<const float4*>(qs + (ty + 16 * a) * pitch + c);
 #pragma unroll
-    for (int a = 0; a < 4; ++a) qv[a] = qs[(ty + 16 * a) * pitch + c];
+    for (int b = 0; b < 4; ++b) kv[b] = *reinterpret_cast<const float4*>(ks + (tx + 16 * b) * pitch + c);
 #pragma unroll
-    for (int b = 0; b < 4; ++b) kv[b] = ks[(tx + 16 * b) * pitch + c];
+    for (int cc = 0; cc < 4; ++cc) {
+      float qa[4], kb[4];
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
+      for (int a = 0; a < 4; ++a) qa[a] = (cc == 0) ? qv[a].x : (cc == 1) ? qv[a].y : (cc == 2) ? qv[a].z : qv[a].w;
 #pragma unroll
-      for (int b = 0; b < 4; ++b) acc[a][b] = __fadd_rn(acc[a][b], __fmul_rn(qv[a], kv[b]));
+      for (int b = 0; b < 4; ++b) kb[b] = (cc == 0) ? kv[b].x : (cc == 1) ? kv[b].y : (cc == 2) ? kv[b].z : kv[b].w;
+      const uint64_t k01 = f2_pack(kb[0], kb[1]), k23 = f2_pack(kb[2], kb[3]);
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        const uint64_t q2 = f2_pack(qa[a], qa[a]);
+        acc2[a][0] = f2_add(acc2[a][0], f2_mul(q2, k01));
+        acc2[a][1] = f2_add(acc2[a][1], f2_mul(q2, k23));
+      }
+    }
   }
 #pragma unroll
   for (int a = 0; a < 4; ++a) {
     const int i = i0 + ty + 16 * a;
     if (i >= nb) continue;
+    float accv[4];
+    f2_unpack(acc2[a][0], accv[0], accv[1]);
+    f2_unpack(acc2[a][1], accv[2], accv[3]);
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
       const int j = j0 + tx + 16 * b;
       if (j >= nb) continue;
-      srow[static_cast<int64_t>(i) * nb + j] = (j <= i) ? __fmul_rn(acc[a][b], scale) : -INFINITY;
+      srow[static_cast<int64_t>(i) * nb + j] = (j <= i) ? __fmul_rn(accv[b], scale) : -INFINITY;
     }
   }
 }
