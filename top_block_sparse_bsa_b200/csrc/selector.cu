@@ -294,47 +294,31 @@ __global__ void __launch_bounds__(256) score_prefill_kernel(const float* __restr
     cp_async_wait_all();
   }
   __syncthreads();
-  // acc2[a][p] holds the pair of sums (a, 2p) and (a, 2p+1), advanced by one
-  // packed f32x2 product and one packed sum per channel (each lane rounded as
-  // the scalar mul.rn / add.rn), channels ascending, four channels per
-  // shared-memory read
-  uint64_t acc2[4][2];
+  float acc[4][4];
 #pragma unroll
-  for (int a = 0; a < 4; ++a) acc2[a][0] = acc2[a][1] = f2_pack(0.0f, 0.0f);
-  for (int c = 0; c < d; c += 4) {
-    float4 qv[4], kv[4];
+  for (int a = 0; a < 4; ++a)
 #pragma unroll
-    for (int a = 0; a < 4; ++a) qv[a] = *reinterpret_cast<const float4*>(qs + (ty + 16 * a) * pitch + c);
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
+  for (int c = 0; c < d; ++c) {
+    float qv[4], kv[4];
 #pragma unroll
-    for (int b = 0; b < 4; ++b) kv[b] = *reinterpret_cast<const float4*>(ks + (tx + 16 * b) * pitch + c);
+    for (int a = 0; a < 4; ++a) qv[a] = qs[(ty + 16 * a) * pitch + c];
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-      float qa[4], kb[4];
+    for (int b = 0; b < 4; ++b) kv[b] = ks[(tx + 16 * b) * pitch + c];
 #pragma unroll
-      for (int a = 0; a < 4; ++a) qa[a] = (cc == 0) ? qv[a].x : (cc == 1) ? qv[a].y : (cc == 2) ? qv[a].z : qv[a].w;
+    for (int a = 0; a < 4; ++a)
 #pragma unroll
-      for (int b = 0; b < 4; ++b) kb[b] = (cc == 0) ? kv[b].x : (cc == 1) ? kv[b].y : (cc == 2) ? kv[b].z : kv[b].w;
-      const uint64_t k01 = f2_pack(kb[0], kb[1]), k23 = f2_pack(kb[2], kb[3]);
-#pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        const uint64_t q2 = f2_pack(qa[a], qa[a]);
-        acc2[a][0] = f2_add(acc2[a][0], f2_mul(q2, k01));
-        acc2[a][1] = f2_add(acc2[a][1], f2_mul(q2, k23));
-      }
-    }
+      for (int b = 0; b < 4; ++b) acc[a][b] = __fadd_rn(acc[a][b], __fmul_rn(qv[a], kv[b]));
   }
 #pragma unroll
   for (int a = 0; a < 4; ++a) {
     const int i = i0 + ty + 16 * a;
     if (i >= nb) continue;
-    float accv[4];
-    f2_unpack(acc2[a][0], accv[0], accv[1]);
-    f2_unpack(acc2[a][1], accv[2], accv[3]);
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
       const int j = j0 + tx + 16 * b;
       if (j >= nb) continue;
-      srow[static_cast<int64_t>(i) * nb + j] = (j <= i) ? __fmul_rn(accv[b], scale) : -INFINITY;
+      srow[static_cast<int64_t>(i) * nb + j] = (j <= i) ? __fmul_rn(acc[a][b], scale) : -INFINITY;
     }
   }
 }
@@ -492,9 +476,9 @@ __global__ void score_gist_kernel(const T* __restrict__ q, const T* __restrict__
 }
 
 // Gist, bf16, d = 128: persistent; a thread owns one gist row of a tile and
-// a pair of the group's heads, so the two heads' fixed-order dot products
-// advance together in packed f32x2 products and sums (each lane rounded as
-// the scalar mul.rn / add.rn; channels ascending, as the generic kernel).  A
+// a pair of the group's heads, so each widened gist value serves both heads'
+// fixed-order dot products (channels ascending, each product and sum rounded
+// on its own, as the generic kernel).  A
 // tile is 64 consecutive gist keys of one (b, g); each CTA takes a contiguous
 // range of tiles, R tiles at a time (R = threads / (64 x head pairs)), the
 // tiles brought in by TMA (two 64-channel halves, 128-byte swizzle, so the
@@ -571,7 +555,7 @@ __global__ void __launch_bounds__(512) score_gist_bf16_d128_kernel(const __grid_
       if (r < min(64, nc - c0)) {
         const uint8_t* tb = sm_gist + stage * kGistTileBytes + r * 128;
         const float4* q4 = reinterpret_cast<const float4*>(qslot + pr * 2 * D);
-        uint64_t acc = f2_pack(0.0f, 0.0f);
+        float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
         for (int x = 0; x < 16; ++x) {
           // chunk x (channels 8x .. 8x+7): half x / 8, 16-byte slot (x % 8) ^ (r % 8)
@@ -581,12 +565,12 @@ __global__ void __launch_bounds__(512) score_gist_bf16_d128_kernel(const __grid_
           for (int y = 0; y < 4; ++y) {
             const float4 qq = q4[4 * x + y];   // channels 8x+2y, 8x+2y+1, both heads
             const float k0 = __uint_as_float(ws[y] << 16), k1 = __uint_as_float(ws[y] & 0xFFFF0000u);
-            acc = f2_add(acc, f2_mul(f2_pack(qq.x, qq.y), f2_pack(k0, k0)));
-            acc = f2_add(acc, f2_mul(f2_pack(qq.z, qq.w), f2_pack(k1, k1)));
+            a0 = __fadd_rn(a0, __fmul_rn(qq.x, k0));
+            a1 = __fadd_rn(a1, __fmul_rn(qq.y, k0));
+            a0 = __fadd_rn(a0, __fmul_rn(qq.z, k1));
+            a1 = __fadd_rn(a1, __fmul_rn(qq.w, k1));
           }
         }
-        float a0, a1;
-        f2_unpack(acc, a0, a1);
         const int h0 = 2 * pr, h1 = 2 * pr + 1;
         s[((b * Hq + g * G + h0) * nc) + c0 + r] = __fmul_rn(a0, scale);
         if (h1 < G) s[((b * Hq + g * G + h1) * nc) + c0 + r] = __fmul_rn(a1, scale);
