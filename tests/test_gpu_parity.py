@@ -581,7 +581,27 @@ def test_gist_bf16_edge_budgets(topk):
     _gist_case(w, topk=topk)
 
 
-@pytest.mark.parametrize("hq,hkv", [(2, 2), (16, 2), (32, 2)])
+@pytest.mark.parametrize("hq,hkv,nc", [(8, 2, 2048), (6, 2, 128), (7, 1, 96), (2, 2, 64), (32, 2, 256)])
+def test_gist_scores_bit_exact(hq, hkv, nc):
+    """The gist scores themselves (SSA page, 推理时的关键模块 1: the query
+    against every chunk's gist key), fixed-order fp32, bit for bit against the
+    oracle for several group widths (odd ones leave one head of a pair empty)
+    and gist counts (a partial last tile of 64)."""
+    bsa = _bsa()
+    g = torch.Generator(device="cuda").manual_seed(31)
+    B, d = 2, 128
+    q = torch.randn((B, hq, d), generator=g, device="cuda").to(torch.bfloat16)
+    gk = torch.randn((B, hkv, nc, d), generator=g, device="cuda").to(torch.bfloat16)
+    scores = torch.empty((B, hq, nc), dtype=torch.float32, device="cuda")
+    shape = bsa.make_shape(B, hq, hkv, 1, nc * 64, d, 64, torch.bfloat16)
+    bsa.bsa_score_blocks(shape, bsa.BSA_SCORE_GIST, q, gk, None, None, None, scores)
+    torch.cuda.synchronize()
+    _status_clean()
+    want = oracle.scores_gist(q.float().cpu(), gk.float().cpu())
+    assert np.array_equal(scores.cpu().numpy(), want)
+
+
+@pytest.mark.parametrize("hq,hkv", [(2, 2), (6, 2), (7, 1), (16, 2), (32, 2)])
 def test_gist_group_widths(hq, hkv):
     w = W.get("gist_decode_bf16").scaled(B=1, Hq=hq, Hkv=hkv, N=8192, kb=5)
     _gist_case(w)
