@@ -451,31 +451,58 @@ def run_prefill(args, world, rank, local, peaks, peak_src):
     stream = torch.cuda.current_stream()
     q, k, v = step.q, step.k, step.v
 
-    # end to end through the C ABI with host buffers
+    # end to end through the C ABI with host buffers: every step copies its
+    # inputs from pinned host memory, runs the step and copies its output
+    # back.  Two device buffer sets and three streams (copy in, compute, copy
+    # out), as a serving loop would run it: step s's inputs go up while step
+    # s-1 computes and step s-2's output comes down (the link is full
+    # duplex); a set is refilled only after its previous output has left.
     e2e = None
     if args.e2e_steps > 0:
+        from top_block_sparse_bsa_b200 import pipeline
         hq = q.cpu().pin_memory()
         hk = k.cpu().pin_memory()
         hv = v.cpu().pin_memory()
-        ho = torch.empty_like(hq).pin_memory()
+        ho = [torch.empty_like(hq).pin_memory() for _ in range(2)]
+        other = pipeline.PrefillStep(torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), w.bs, w.kb,
+                                     gated=(w.kind == "gated"), pattern=pattern)
+        sets = [step, other]
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
-        for it in range(args.e2e_steps + 1):
-            if it == 1:
-                e0.record(stream)
-            q.copy_(hq, non_blocking=True)
-            k.copy_(hk, non_blocking=True)
-            v.copy_(hv, non_blocking=True)
-            step.run(with_lse=False)
-            ho.copy_(step.bufs["o"], non_blocking=True)
-        e1.record(stream)
+        torch.cuda.synchronize()
+        n_it = args.e2e_steps + 2   # two untimed steps fill the pipeline
+        for it in range(n_it):
+            x = it % 2
+            st = sets[x]
+            if it == 2:
+                e0.record(s_in)   # the timed region starts at step 2's copy-in, the pipeline running
+            with torch.cuda.stream(s_in):
+                if it >= 2:
+                    s_in.wait_event(ev_out[x])
+                st.q.copy_(hq, non_blocking=True)
+                st.k.copy_(hk, non_blocking=True)
+                st.v.copy_(hv, non_blocking=True)
+                ev_in[x].record(s_in)
+            stream.wait_event(ev_in[x])
+            st.run(stream=stream, with_lse=False)
+            ev_done[x].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_done[x])
+                ho[x].copy_(st.bufs["o"], non_blocking=True)
+                ev_out[x].record(s_out)
+        e1.record(s_out)
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
         e2e_ms, _ = reduce_over_ranks(dist, e2e_ms, pairs, device=dev)
         h2d = (hq.numel() + hk.numel() + hv.numel()) * hq.element_size()
         e2e = {"value": job_pairs / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": ho.numel() * ho.element_size(), "ms_per_step": e2e_ms}
-        del hq, hk, hv, ho
+               "d2h_bytes_per_step": ho[0].numel() * ho[0].element_size(), "ms_per_step": e2e_ms,
+               "pipelined": "two buffer sets; copy-in, compute and copy-out streams"}
+        del hq, hk, hv, ho, other, sets
 
     cpu_baseline = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -483,15 +483,16 @@ __global__ void score_gist_kernel(const T* __restrict__ q, const T* __restrict__
 // range of tiles, R tiles at a time (R = threads / (64 x head pairs)), the
 // tiles brought in by TMA (two 64-channel halves, 128-byte swizzle, so the
 // same 16-byte chunk of eight consecutive rows sits in eight distinct bank
-// groups) two rounds ahead; the group's query rows are staged, as head-pair
-// interleaved floats, only when a slot's (b, g) changes.
+// groups) `stages` tiles ahead; the group's query rows are staged, as
+// head-pair interleaved floats, only when a slot's (b, g) changes.
 constexpr int kGistTileBytes = 64 * 128 * 2;
 constexpr int kGistMaxStages = 8;
 
 __global__ void __launch_bounds__(512) score_gist_bf16_d128_kernel(const __grid_constant__ CUtensorMap tmG,
                                                                   const __nv_bfloat16* __restrict__ q, int Hq,
-                                                                  int Hkv, int nc, int64_t tiles, float scale,
-                                                                  float* __restrict__ s, uint32_t* __restrict__ status) {
+                                                                  int Hkv, int nc, int64_t tiles, int stages,
+                                                                  float scale, float* __restrict__ s,
+                                                                  uint32_t* __restrict__ status) {
   constexpr int D = 128;
   extern __shared__ uint8_t sm_raw[];
   uint8_t* sm_gist = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
@@ -501,7 +502,7 @@ __global__ void __launch_bounds__(512) score_gist_bf16_d128_kernel(const __grid_
   const int G = Hq / Hkv, HP = (G + 1) / 2;
   const int tpt = 64 * HP;                     // threads per tile
   const int R = blockDim.x / tpt;              // tiles per round
-  const int S = 2 * R;                         // stages: two rounds in flight
+  const int S = stages;                        // tile buffers (a multiple of R, at most kGistMaxStages)
   const int tpb = (nc + 63) / 64;              // tiles per (b, g)
   const uint32_t sbase = smem_u32(sm_gist);
   if (threadIdx.x == 0) {
@@ -602,17 +603,20 @@ cudaError_t launch_score_gist(const CUtensorMap* tmG, const void* q, const void*
     const int HP = (G + 1) / 2;
     const int threads = max(256, 64 * HP);
     const int R = threads / (64 * HP);
-    const size_t smem2 = static_cast<size_t>(2 * R) * kGistTileBytes + 1024;   // + alignment slack
+    const int64_t tiles = static_cast<int64_t>(B) * Hkv * ((nc + 63) / 64);
+    // one round of R tiles per CTA while that keeps a few waves of small CTAs
+    // (every tile's copy in flight at once); beyond that, persistent CTAs
+    // with two rounds of buffers
+    const int64_t need = (tiles + R - 1) / R;
+    const int64_t cap = static_cast<int64_t>(num_sms) * 16;
+    const unsigned ctas = static_cast<unsigned>(need < cap ? need : cap);
+    const int stages = (need <= cap) ? R : 2 * R;
+    if (ctas == 0) return cudaSuccess;
+    const size_t smem2 = static_cast<size_t>(stages) * kGistTileBytes + 1024;   // + alignment slack
     cudaError_t e = ensure_dynamic_smem<score_gist_bf16_d128_kernel>(smem2);
     if (e != cudaSuccess) return e;
-    const int64_t tiles = static_cast<int64_t>(B) * Hkv * ((nc + 63) / 64);
-    // as many CTAs as fit (one round of R tiles each at least)
-    const int64_t want = static_cast<int64_t>(num_sms) * (R >= 4 ? 1 : 2);
-    const int64_t need = (tiles + R - 1) / R;
-    const unsigned ctas = static_cast<unsigned>(need < want ? need : want);
-    if (ctas == 0) return cudaSuccess;
     score_gist_bf16_d128_kernel<<<ctas, threads, smem2, st>>>(*tmG, static_cast<const __nv_bfloat16*>(q), Hq, Hkv,
-                                                              nc, tiles, scale, s, status);
+                                                              nc, tiles, stages, scale, s, status);
     return cudaGetLastError();
   }
   const size_t smem = (G * d + 64 * (d + 1)) * sizeof(float);
