@@ -121,8 +121,8 @@ static cudaError_t launch_pool_jobs(const PoolJob& j0, const PoolJob& j1, bool b
 // kPoolStages shared-memory buffers with bulk copies, a chunk of whole runs
 // per buffer, while 128 threads sum earlier chunks, column c by thread c,
 // rows in the fixed order (head, then row), the running sum carried from one
-// chunk of a unit to the next.  Units of the query and the key job alternate
-// (both jobs have the same number of units).
+// chunk of a unit to the next.  Units of the query job come first, then those
+// of the key job.
 constexpr int kPoolStreamBytes = 64 * 1024;
 constexpr int kPoolStages = 3;
 
@@ -156,11 +156,9 @@ __global__ void __launch_bounds__(160, 1) pool_stream_kernel(PoolJob jq, PoolJob
       int k = 0;   // chunks issued
       bool ok = true;
       for (int64_t u = blockIdx.x; ok && u < units; u += gridDim.x) {
-        // query and key units alternate, so a key unit's small copy always
-        // sits next to a query unit's large one in the ring
-        const bool isk = jk.src != nullptr && (u & 1);
+        const bool isk = u >= units_per_job;
         const PoolJob& job = isk ? jk : jq;
-        const int64_t unit = jk.src != nullptr ? (u >> 1) : u;
+        const int64_t unit = isk ? u - units_per_job : u;
         const int64_t b = unit / (static_cast<int64_t>(Hgroups) * nb);
         const int64_t g = (unit / nb) % Hgroups;
         const int64_t j = unit % nb;
@@ -186,9 +184,9 @@ __global__ void __launch_bounds__(160, 1) pool_stream_kernel(PoolJob jq, PoolJob
     int k = 0;   // chunks consumed
     bool ok = true;
     for (int64_t u = blockIdx.x; ok && u < units; u += gridDim.x) {
-      const bool isk = jk.src != nullptr && (u & 1);
+      const bool isk = u >= units_per_job;
       const PoolJob& job = isk ? jk : jq;
-      const int64_t unit = jk.src != nullptr ? (u >> 1) : u;
+      const int64_t unit = isk ? u - units_per_job : u;
       float acc = 0.0f;
       for (int h0 = 0; h0 < job.heads_sum; h0 += runs_per_chunk, ++k) {
         const int nr = min(runs_per_chunk, job.heads_sum - h0);
