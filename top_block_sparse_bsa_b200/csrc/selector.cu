@@ -122,7 +122,8 @@ static cudaError_t launch_pool_jobs(const PoolJob& j0, const PoolJob& j1, bool b
 // per buffer, while 128 threads sum earlier chunks, column c by thread c,
 // rows in the fixed order (head, then row), the running sum carried from one
 // chunk of a unit to the next.  Units of the query job come first, then those
-// of the key job.
+// of the key job; a key unit is a single run and consecutive key units are
+// contiguous in memory, so a buffer takes several of them in one copy.
 constexpr int kPoolStreamBytes = 64 * 1024;
 constexpr int kPoolStages = 3;
 
@@ -137,9 +138,13 @@ __global__ void __launch_bounds__(160, 1) pool_stream_kernel(PoolJob jq, PoolJob
   auto bar = [&](int i) -> uint32_t { return smem_u32(&bars[i]); };
   const int nb = N / bs;
   const int64_t units_per_job = static_cast<int64_t>(B) * Hgroups * nb;
-  const int64_t units = units_per_job * (jk.src ? 2 : 1);
   const uint32_t run = static_cast<uint32_t>(bs) * d * sizeof(T);       // one head's rows of a unit
   const int runs_per_chunk = static_cast<int>(kPoolStreamBytes / run);   // >= 1 (checked by the launcher)
+  // key items: kgrp consecutive key units each (single-run units stored back
+  // to back: unit u's rows start at u * bs * d)
+  const int kgrp = (jk.src != nullptr && jk.heads_sum == 1 && jk.Hsrc == Hgroups) ? runs_per_chunk : 1;
+  const int64_t kitems = jk.src ? (units_per_job + kgrp - 1) / kgrp : 0;
+  const int64_t units = units_per_job + kitems;   // work items
   if (threadIdx.x == 0) {
     for (int i = 0; i < kPoolStages; ++i) {
       mbar_init(bar(i), 1);
@@ -157,6 +162,16 @@ __global__ void __launch_bounds__(160, 1) pool_stream_kernel(PoolJob jq, PoolJob
       bool ok = true;
       for (int64_t u = blockIdx.x; ok && u < units; u += gridDim.x) {
         const bool isk = u >= units_per_job;
+        if (isk && kgrp > 1) {
+          const int64_t u0 = (u - units_per_job) * kgrp;
+          const int nr = static_cast<int>(min(static_cast<int64_t>(kgrp), units_per_job - u0));
+          const int buf = k % kPoolStages, use = k / kPoolStages;
+          if (k >= kPoolStages && !(ok = mbar_wait(bar(kPoolStages + buf), (use - 1) & 1, ab, status))) break;
+          mbar_arrive_expect_tx(bar(buf), run * nr);
+          bulk_load(sb + buf * kPoolStreamBytes, static_cast<const T*>(jk.src) + u0 * bs * d, run * nr, bar(buf));
+          ++k;
+          continue;
+        }
         const PoolJob& job = isk ? jk : jq;
         const int64_t unit = isk ? u - units_per_job : u;
         const int64_t b = unit / (static_cast<int64_t>(Hgroups) * nb);
@@ -185,6 +200,29 @@ __global__ void __launch_bounds__(160, 1) pool_stream_kernel(PoolJob jq, PoolJob
     bool ok = true;
     for (int64_t u = blockIdx.x; ok && u < units; u += gridDim.x) {
       const bool isk = u >= units_per_job;
+      if (isk && kgrp > 1) {
+        const int64_t u0 = (u - units_per_job) * kgrp;
+        const int nr = static_cast<int>(min(static_cast<int64_t>(kgrp), units_per_job - u0));
+        const int buf = k % kPoolStages, use = k / kPoolStages;
+        if (!(ok = mbar_wait(bar(buf), use & 1, ab, status))) break;
+        const T* sv = reinterpret_cast<const T*>(psmem + buf * kPoolStreamBytes);
+        for (int x = 0; x < nr; ++x) {
+          float acc = 0.0f;
+          if (c < d) {
+            for (int r = x * bs; r < (x + 1) * bs; r += 16) {   // bs is a multiple of 16
+              float xv[16];
+#pragma unroll
+              for (int t = 0; t < 16; ++t) xv[t] = static_cast<float>(sv[(r + t) * d + c]);
+#pragma unroll
+              for (int t = 0; t < 16; ++t) acc = __fadd_rn(acc, xv[t]);
+            }
+            jk.out[(u0 + x) * d + c] = __fdiv_rn(acc, static_cast<float>(bs));
+          }
+        }
+        mbar_arrive(bar(kPoolStages + buf));
+        ++k;
+        continue;
+      }
       const PoolJob& job = isk ? jk : jq;
       const int64_t unit = isk ? u - units_per_job : u;
       float acc = 0.0f;
