@@ -8,13 +8,11 @@
 // §1-2, §4.5), optionally with the SAS log-gate log g_j on every key of kept
 // block j (SAS page, 核心模块 2-3).
 //
-// One CTA per (query block i, query head h, batch b), 512 threads: 8 (bs 64)
-// or 4 (bs 128) per query row = KG key groups x four channel quarters.
-// Each kept K/V block is staged in shared memory; a thread scores its key
-// group's keys of the block 16 at a time against its quarter of the row (dot
-// products finished with two shuffles) and keeps its own running maximum,
-// sum and output quarter; the KG partial states of a row are merged at the
-// end (the same rescale-and-add as the decode combine).
+// One CTA per (query block i, query head h, batch b); four threads per query
+// row, each holding a quarter of the channels (dot products finished with two
+// shuffles).  Each kept K/V block is staged in shared memory; a row first
+// scores all of the block's keys (independent dot products), then moves its
+// running maximum once per block and accumulates the block's keys.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -23,8 +21,8 @@ namespace f32path {
 
 constexpr int kMaxList = 256;
 
-template <int D, int KG>
-__global__ void __launch_bounds__(512) attn_prefill_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
+template <int D>
+__global__ void attn_prefill_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
                                         const float* __restrict__ v, int Hq, int Hkv, int N, int bs,
                                         const int* __restrict__ idx, int idx_stride, const float* __restrict__ sel,
                                         float scale, float* __restrict__ o, float* __restrict__ lse,
@@ -80,10 +78,9 @@ __global__ void __launch_bounds__(512) attn_prefill_f32_kernel(const float* __re
     if (lane == 0) s_n = count;
   }
   __syncthreads();
-  constexpr int DQ = D / 4;                 // channels per thread
+  constexpr int DQ = D / 4;           // channels per thread
   const int n = s_n;
-  const int qt = t & 3, kg = (t >> 2) % KG, r = t / (4 * KG);   // channel quarter, key group, row
-  const int kper = bs / KG;                 // keys of a block per key group (a multiple of 16)
+  const int r = t >> 2, qt = t & 3;   // query row inside the block, channel quarter
   const int tpos = i * bs + r;
   const float* qrow = q + ((static_cast<int64_t>(b) * Hq + h) * N + tpos) * D + qt * DQ;
   float qr[DQ], acc[DQ];
@@ -105,9 +102,11 @@ __global__ void __launch_bounds__(512) attn_prefill_f32_kernel(const float* __re
     }
     __syncthreads();
     const int umax = (j == i) ? r : bs - 1;   // causal inside the current block
-    // every lane runs the same number of chunks (the shuffles need the whole
-    // warp); keys past umax are masked
-    for (int u0 = kg * kper; u0 < (kg + 1) * kper; u0 += 16) {
+    // the key loop runs to the warp's last row (r | 7: a warp holds 8 rows),
+    // so every lane takes part in the shuffles; keys past umax are masked
+    const int uend = (j == i) ? (r | 7) : bs - 1;
+    // scores of the block's keys in chunks of 16, the chunk's maximum first
+    for (int u0 = 0; u0 <= uend; u0 += 16) {
       float sc[16];
 #pragma unroll
       for (int x = 0; x < 16; ++x) {
@@ -140,53 +139,36 @@ __global__ void __launch_bounds__(512) attn_prefill_f32_kernel(const float* __re
       }
     }
   }
-  // merge the row's KG partial states (lanes that differ in the key-group bits)
+  float* orow = o + ((static_cast<int64_t>(b) * Hq + h) * N + tpos) * D + qt * DQ;
+  const float inv = (l > 0.0f) ? 1.0f / l : 0.0f;
 #pragma unroll
-  for (int off = 4; off < 4 * KG; off <<= 1) {
-    const float mo = __shfl_xor_sync(0xffffffffu, m, off);
-    const float lo = __shfl_xor_sync(0xffffffffu, l, off);
-    const float mn = fmaxf(m, mo);
-    const float a = (m == -INFINITY) ? 0.0f : expf(m - mn);
-    const float bo = (mo == -INFINITY) ? 0.0f : expf(mo - mn);
-    l = l * a + lo * bo;
-#pragma unroll
-    for (int c = 0; c < DQ; ++c) {
-      const float ao = __shfl_xor_sync(0xffffffffu, acc[c], off);
-      acc[c] = acc[c] * a + ao * bo;
-    }
-    m = mn;
-  }
-  if (kg == 0) {
-    float* orow = o + ((static_cast<int64_t>(b) * Hq + h) * N + tpos) * D + qt * DQ;
-    const float inv = (l > 0.0f) ? 1.0f / l : 0.0f;
-#pragma unroll
-    for (int c = 0; c < DQ; ++c) orow[c] = acc[c] * inv;
-    if (lse && qt == 0) lse[(static_cast<int64_t>(b) * Hq + h) * N + tpos] = (l > 0.0f) ? m + logf(l) : -INFINITY;
-  }
+  for (int c = 0; c < DQ; ++c) orow[c] = acc[c] * inv;
+  if (lse && qt == 0) lse[(static_cast<int64_t>(b) * Hq + h) * N + tpos] = (l > 0.0f) ? m + logf(l) : -INFINITY;
 }
 
 }  // namespace f32path
-
-template <int D, int KG>
-static cudaError_t launch_f32(const float* q, const float* k, const float* v, const PrefillArgs& a, dim3 grid,
-                              size_t smem, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(f32path::attn_prefill_f32_kernel<D, KG>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  f32path::attn_prefill_f32_kernel<D, KG><<<grid, 4 * KG * a.bs, smem, st>>>(
-      q, k, v, a.Hq, a.Hkv, a.N, a.bs, a.idx, a.idx_stride, a.sel_scores, a.softmax_scale, static_cast<float*>(a.o),
-      a.lse, a.status);
-  return cudaGetLastError();
-}
 
 cudaError_t launch_attn_prefill_f32(const float* q, const float* k, const float* v, const PrefillArgs& a, int d,
                                     cudaStream_t st) {
   const int nb = a.N / a.bs;
   dim3 grid(nb, a.Hq, a.B);
   const size_t smem = 2ull * a.bs * d * sizeof(float);
-  // 512 threads: two key groups of a 64-token block, one of a 128-token one
-  if (a.bs == 64) return d == 64 ? launch_f32<64, 2>(q, k, v, a, grid, smem, st) : launch_f32<128, 2>(q, k, v, a, grid, smem, st);
-  return d == 64 ? launch_f32<64, 1>(q, k, v, a, grid, smem, st) : launch_f32<128, 1>(q, k, v, a, grid, smem, st);
+  if (d == 64) {
+    cudaError_t e = cudaFuncSetAttribute(f32path::attn_prefill_f32_kernel<64>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    f32path::attn_prefill_f32_kernel<64><<<grid, 4 * a.bs, smem, st>>>(q, k, v, a.Hq, a.Hkv, a.N, a.bs, a.idx,
+                                                                   a.idx_stride, a.sel_scores, a.softmax_scale,
+                                                                   static_cast<float*>(a.o), a.lse, a.status);
+  } else {
+    cudaError_t e = cudaFuncSetAttribute(f32path::attn_prefill_f32_kernel<128>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    f32path::attn_prefill_f32_kernel<128><<<grid, 4 * a.bs, smem, st>>>(q, k, v, a.Hq, a.Hkv, a.N, a.bs, a.idx,
+                                                                    a.idx_stride, a.sel_scores, a.softmax_scale,
+                                                                    static_cast<float*>(a.o), a.lse, a.status);
+  }
+  return cudaGetLastError();
 }
 
 }  // namespace bsa
