@@ -119,22 +119,17 @@ static cudaError_t launch_pool_jobs(const PoolJob& j0, const PoolJob& j1, bool b
 // Streamed variant (persistent, one CTA per SM): a producer thread copies each
 // unit's rows (heads_sum runs of bs*d contiguous elements) into
 // kPoolStages shared-memory buffers with bulk copies, a chunk of whole runs
-// per buffer, while kPoolGroups groups of 128 threads sum earlier chunks --
-// group g the CTA's work items g, g + kPoolGroups, ... -- column c by thread
-// c, rows in the fixed order (head, then row), the running sum carried from
-// one chunk of a unit to the next.  (A column's sum is one dependent chain,
-// so the groups are what keeps the SM busy.)  Units of the query job come
-// first, then those of the key job; a key unit is a single run and
-// consecutive key units are contiguous in memory, so a buffer takes several
-// of them in one copy.
+// per buffer, while 128 threads sum earlier chunks, column c by thread c,
+// rows in the fixed order (head, then row), the running sum carried from one
+// chunk of a unit to the next.  Units of the query job come first, then those
+// of the key job; a key unit is a single run and consecutive key units are
+// contiguous in memory, so a buffer takes several of them in one copy.
 constexpr int kPoolStreamBytes = 64 * 1024;
 constexpr int kPoolStages = 3;
-constexpr int kPoolGroups = 3;
-constexpr int kPoolThreads = 32 + 128 * kPoolGroups;
 
 template <typename T>
-__global__ void __launch_bounds__(kPoolThreads, 1) pool_stream_kernel(PoolJob jq, PoolJob jk, int B, int Hgroups,
-                                                                      int N, int d, int bs, uint32_t* status) {
+__global__ void __launch_bounds__(160, 1) pool_stream_kernel(PoolJob jq, PoolJob jk, int B, int Hgroups, int N, int d,
+                                                             int bs, uint32_t* status) {
   extern __shared__ uint8_t psmem_raw[];
   uint8_t* psmem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(psmem_raw) + 127) & ~uintptr_t(127));
   __shared__ __align__(8) uint64_t bars[2 * kPoolStages];
@@ -150,12 +145,6 @@ __global__ void __launch_bounds__(kPoolThreads, 1) pool_stream_kernel(PoolJob jq
   const int kgrp = (jk.src != nullptr && jk.heads_sum == 1 && jk.Hsrc == Hgroups) ? runs_per_chunk : 1;
   const int64_t kitems = jk.src ? (units_per_job + kgrp - 1) / kgrp : 0;
   const int64_t units = units_per_job + kitems;   // work items
-  // chunks of work item u
-  auto chunks_of = [&](int64_t u) -> int {
-    if (u >= units_per_job && kgrp > 1) return 1;
-    const int hs = (u >= units_per_job) ? jk.heads_sum : jq.heads_sum;
-    return (hs + runs_per_chunk - 1) / runs_per_chunk;
-  };
   if (threadIdx.x == 0) {
     for (int i = 0; i < kPoolStages; ++i) {
       mbar_init(bar(i), 1);
@@ -167,7 +156,7 @@ __global__ void __launch_bounds__(kPoolThreads, 1) pool_stream_kernel(PoolJob jq
   __syncthreads();
   volatile int* ab = &abort_flag;
   const int warp = threadIdx.x >> 5;
-  if (warp == 0) {
+  if (warp == 4) {
     if ((threadIdx.x & 31) == 0) {
       int k = 0;   // chunks issued
       bool ok = true;
@@ -206,17 +195,10 @@ __global__ void __launch_bounds__(kPoolThreads, 1) pool_stream_kernel(PoolJob jq
       }
     }
   } else {
-    const int grp = (warp - 1) / 4;   // consumer group
-    const int c = (threadIdx.x - 32) & 127;   // column
-    int k = 0;   // chunks of the items before the current one
+    const int c = threadIdx.x;   // column
+    int k = 0;   // chunks consumed
     bool ok = true;
-    int q = 0;   // item sequence number inside this CTA
-    for (int64_t u = blockIdx.x; ok && u < units; u += gridDim.x, ++q) {
-      const int nch = chunks_of(u);
-      if (q % kPoolGroups != grp) {   // another group's item: skip its chunks
-        k += nch;
-        continue;
-      }
+    for (int64_t u = blockIdx.x; ok && u < units; u += gridDim.x) {
       const bool isk = u >= units_per_job;
       if (isk && kgrp > 1) {
         const int64_t u0 = (u - units_per_job) * kgrp;
@@ -293,11 +275,11 @@ cudaError_t launch_pool_prefill(const void* q, const void* k, bool bf16, int B, 
   if (bf16) {
     e = ensure_dynamic_smem<pool_stream_kernel<__nv_bfloat16>>(smem);
     if (e != cudaSuccess) return e;
-    pool_stream_kernel<__nv_bfloat16><<<grid, kPoolThreads, smem, st>>>(jq, jk, B, Hkv, N, d, bs, status);
+    pool_stream_kernel<__nv_bfloat16><<<grid, 160, smem, st>>>(jq, jk, B, Hkv, N, d, bs, status);
   } else {
     e = ensure_dynamic_smem<pool_stream_kernel<float>>(smem);
     if (e != cudaSuccess) return e;
-    pool_stream_kernel<float><<<grid, kPoolThreads, smem, st>>>(jq, jk, B, Hkv, N, d, bs, status);
+    pool_stream_kernel<float><<<grid, 160, smem, st>>>(jq, jk, B, Hkv, N, d, bs, status);
   }
   return cudaGetLastError();
 }
