@@ -607,6 +607,32 @@ def test_gist_group_widths(hq, hkv):
     _gist_case(w)
 
 
+def test_gist_union_kernel_above_2048_chunks():
+    """Above 2048 chunks per row the union of the heads' expanded chunks is
+    built by its own kernel instead of inside the attention kernel: 4096
+    chunks, two groups of widths 3."""
+    w = W.get("gist_decode_bf16").scaled(B=1, Hq=6, Hkv=2, N=4096 * 64, kb=9)
+    _gist_case(w)
+
+
+def test_gist_injected_lists_with_padding_and_repeats():
+    """Injected per-head lists with -1 padding, a chunk kept by every head and
+    a head that expands nothing: the union and the per-head masks built in the
+    attention kernel."""
+    pipe = _pipe()
+    w = W.get("gist_decode_bf16").scaled(B=1, Hq=4, Hkv=1, N=8192, kb=4)
+    inp = W.make_inputs(w, "cuda")
+    idx = torch.tensor([[[3, 40, 127, -1], [3, 4, -1, -1], [-1, -1, -1, -1], [0, 3, 64, 126]]],
+                       dtype=torch.int32, device="cuda")
+    step = pipe.GistStep(inp["q"], inp["k"], inp["v"], inp["gk"], inp["gv"], w.bs, 4)
+    step.run(idx_in=idx)
+    torch.cuda.synchronize()
+    want, _ = oracle.attend_gist(inp["q"].float().cpu(), inp["k"].float().cpu(), inp["v"].float().cpu(),
+                                 inp["gk"].float().cpu(), inp["gv"].float().cpu(), w.bs, idx.cpu().numpy())
+    _assert_close(step.bufs["o"][0].float().cpu().numpy(), want, TOL_BF16, "gist padded lists")
+    _status_clean()
+
+
 def test_gist_bf16_full_size_every_group():
     """The full gist workload (8 sequences x 131072 tokens, 2048 gists): the
     chosen chunks of all 256 query heads compared exactly, and the outputs of

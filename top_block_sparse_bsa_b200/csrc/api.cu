@@ -644,7 +644,9 @@ bsa_status_t bsa_gist_expand_decode(const bsa_shape_t* s, const void* q, const v
   } else if (idx_out != nullptr && topk > 0 && idx_out != idx_in) {
     e = cudaMemcpyAsync(idx_out, idx_in, static_cast<size_t>(rows) * topk * sizeof(int), cudaMemcpyDeviceToDevice, cs);
   }
-  if (e == cudaSuccess)
+  // up to 2048 chunks the attention kernel builds the group's union itself
+  const bool fused_union = nc <= 2048;
+  if (e == cudaSuccess && !fused_union)
     e = launch_gist_union(idx, s->B, s->Hq, s->Hkv, topk, idx_stride, nc, expanded, ulist, L.union_stride, true,
                           status, cs);
   DecodeArgs a;
@@ -664,6 +666,13 @@ bsa_status_t bsa_gist_expand_decode(const bsa_shape_t* s, const void* q, const v
   a.softmax_scale = softmax_scale;
   a.partial = reinterpret_cast<float*>(ws + L.partial);
   a.status = status;
+  if (fused_union) {
+    a.list = nullptr;
+    a.expanded = nullptr;
+    a.heads_idx = idx;
+    a.heads_topk = topk;
+    a.heads_stride = idx_stride;
+  }
   if (e == cudaSuccess) e = launch_attn_decode_bf16(&mq, &mk, &mv, &mgk, &mgv, a, cs);
   if (e == cudaSuccess) e = launch_decode_combine(a.partial, a, s->d, true, o, lse, cs);
   return cuda_status(e);

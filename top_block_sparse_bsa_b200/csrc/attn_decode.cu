@@ -71,9 +71,11 @@ enum {
 };
 constexpr uint32_t kListConsumers = 2 + 4;   // producer, MMA, one lane per softmax warp
 
+constexpr int kUnionWords = 64;         // fused gist union: up to 2048 chunks per row
 struct ItemInfo {
   int n, b, g, bg, slot, pad0, pad1, pad2;
   int tiles[kMaxItemTiles];
+  uint32_t bits[kNH + 1][kUnionWords];   // fused gist union: heads' expanded chunks, then the union
 };
 
 struct Misc {
@@ -86,6 +88,7 @@ struct Misc {
 };
 constexpr uint32_t kSmemMisc = kSmemBar + NUM_BARS * 8;
 constexpr uint32_t kSmemBytes = kSmemMisc + sizeof(Misc) + 1024;
+static_assert(kSmemBytes <= 232448, "dynamic shared memory above the sm_100 per-CTA limit");
 
 constexpr float kLog2e = 1.44269504088896340736f;
 constexpr float kRescaleThreshold = 8.0f;
@@ -109,6 +112,11 @@ struct Params {
   // physical block table[b * table_stride + j] of the pools [P][Hkv][64][d]
   const int* table;
   int table_stride, num_pages;
+  // gist decode with the union built in the kernel (nc <= 2048): the heads'
+  // kept chunk lists [B*Hq][heads_stride] (heads_topk entries, -1 = none);
+  // null: list/expanded hold a union built by gist_union_kernel
+  const int* heads_idx;
+  int heads_topk, heads_stride;
   // two-level gists (H-SSA): gist tiles at or past nc/64 are meta-gist tiles
   // (rows bg*meta_rows + ..., of the meta maps); gist_allow [B*Hq][(nc+64)/32]
   // says per head which gist / meta-gist rows it attends (null: SSA's rule,
@@ -168,8 +176,10 @@ __device__ __forceinline__ void softmax_role(const Params& p, Misc* misc, uint8_
           part[4 + r] = 0.0f;
         }
       } else {
+        const bool fused = p.heads_idx != nullptr;
         const uint32_t* bits_base =
-            gist ? p.expanded + (static_cast<int64_t>(b) * p.Hq + g * G) * (p.nc / 32) : nullptr;
+            fused ? &inf->bits[0][0]
+                  : (gist ? p.expanded + (static_cast<int64_t>(b) * p.Hq + g * G) * (p.nc / 32) : nullptr);
         const bool two_level = p.gist_allow != nullptr;
         const int words_g = (p.nc + 64) / 32;
         const uint32_t* allow_base =
@@ -197,8 +207,10 @@ __device__ __forceinline__ void softmax_role(const Params& p, Misc* misc, uint8_
 #pragma unroll
           for (int h = 0; h < GH; ++h)
             word[h] = (gist && h < G && has_mine)
-                          ? ((two_level && mytile < 0) ? __ldg(allow_base + h * words_g + (bitpos >> 5))
-                                                       : __ldg(bits_base + h * words + (bitpos >> 5)))
+                          ? ((two_level && mytile < 0)
+                                 ? __ldg(allow_base + h * words_g + (bitpos >> 5))
+                                 : (fused ? bits_base[h * kUnionWords + (bitpos >> 5)]
+                                          : __ldg(bits_base + h * words + (bitpos >> 5))))
                           : 0u;
           if (!(ok = warp_wait(bar(BAR_SF + sb), (s_read >> 1) & 1, abortp, p.status))) break;
           tc_fence_after();
@@ -337,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar = [&](int b) -> uint32_t { return sbase + kSmemBar + 8u * b; };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abortp = &misc->abort_flag;
-  const bool gist = p.expanded != nullptr;
+  const bool gist = p.expanded != nullptr || p.heads_idx != nullptr;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -404,40 +416,89 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t row0 = static_cast<int64_t>(bg) * p.list_len;
       const int a = static_cast<int>(max(lo, row0) - row0);
       const int e = static_cast<int>(min(hi, row0 + p.list_len) - row0);
-      const int* src = p.list + static_cast<int64_t>(bg) * p.list_stride;
-      int count;
-      if (p.list_has_count) {
-        count = min(src[0], p.list_len);
-        src += 1;
-      } else {
-        count = e;   // the first negative entry ends the list
-        for (int base = 0; base < e; base += 32) {
-          const int t = base + lane;
-          const int v = (t < e) ? src[t] : 0;
-          const unsigned neg = __ballot_sync(0xffffffffu, v < 0);
-          if (neg) {
-            count = base + __ffs(neg) - 1;
-            break;
+      int stop, w = 0;
+      if (p.heads_idx != nullptr) {
+        // gist decode, union built here: each head's expanded chunks and
+        // their union as bitmaps in the item slot, then the row's list =
+        // union chunks ascending followed by every gist tile -(t+1)
+        const int G = p.G, words = p.nc / 32, topk = p.heads_topk;
+        uint32_t* ub = &inf->bits[0][0];
+        for (int t = lane; t < (G + 1) * kUnionWords; t += 32) ub[t] = 0u;
+        __syncwarp();
+        const int* hsrc = p.heads_idx + (static_cast<int64_t>(bg / p.Hkv) * p.Hq + (bg % p.Hkv) * G) *
+                                            static_cast<int64_t>(p.heads_stride);
+        for (int t = lane; t < G * topk; t += 32) {
+          const int hh = t / topk;
+          const int c = __ldg(hsrc + static_cast<int64_t>(hh) * p.heads_stride + (t - hh * topk));
+          if (c < 0) continue;
+          if (c >= p.nc) {
+            atomicOr(p.status, BSA_DEV_BAD_INDEX);
+            continue;
+          }
+          atomicOr(&ub[hh * kUnionWords + (c >> 5)], 1u << (c & 31));
+          atomicOr(&ub[G * kUnionWords + (c >> 5)], 1u << (c & 31));
+        }
+        __syncwarp();
+        const uint32_t w0 = (2 * lane < words) ? ub[G * kUnionWords + 2 * lane] : 0u;
+        const uint32_t w1 = (2 * lane + 1 < words) ? ub[G * kUnionWords + 2 * lane + 1] : 0u;
+        const int cnt = __popc(w0) + __popc(w1);
+        int incl = cnt;
+        for (int off = 1; off < 32; off <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += v;
+        }
+        const int U = __shfl_sync(0xffffffffu, incl, 31);
+        stop = min(e, min(U + ngist, p.list_len));
+        const int lim = min(stop, a + kMaxItemTiles);
+        int pos = incl - cnt;
+        for (int hw = 0; hw < 2; ++hw) {
+          uint32_t m = hw ? w1 : w0;
+          while (m) {
+            const int bit = __ffs(m) - 1;
+            m &= m - 1;
+            if (pos >= a && pos < lim) inf->tiles[pos - a] = (2 * lane + hw) * 32 + bit;
+            ++pos;
           }
         }
-      }
-      const int stop = min(e, count);
-      int w = 0;
-      for (int base = a; base < stop; base += 32) {
-        const int t = base + lane;
-        const int v = (t < stop) ? src[t] : 0;
-        bool bad = (t < stop) && (gist ? (v >= nb_cache || v < -ngist) : (v < 0 || v >= nb_cache));
-        int tile = v;
-        if (p.table != nullptr && t < stop && !bad) {
-          // paged cache: the kept logical block's physical block
-          tile = __ldg(p.table + static_cast<int64_t>(bg / p.Hkv) * p.table_stride + v);
-          bad = tile < 0 || tile >= p.num_pages;
+        for (int t = lane; t < ngist; t += 32)
+          if (U + t >= a && U + t < lim) inf->tiles[U + t - a] = -(t + 1);
+        w = max(0, lim - a);
+        __syncwarp();
+      } else {
+        const int* src = p.list + static_cast<int64_t>(bg) * p.list_stride;
+        int count;
+        if (p.list_has_count) {
+          count = min(src[0], p.list_len);
+          src += 1;
+        } else {
+          count = e;   // the first negative entry ends the list
+          for (int base = 0; base < e; base += 32) {
+            const int t = base + lane;
+            const int v = (t < e) ? src[t] : 0;
+            const unsigned neg = __ballot_sync(0xffffffffu, v < 0);
+            if (neg) {
+              count = base + __ffs(neg) - 1;
+              break;
+            }
+          }
         }
-        if (bad) atomicOr(p.status, BSA_DEV_BAD_INDEX);
-        const bool keep = (t < stop) && !bad && (w + (t - base) < kMaxItemTiles);
-        const unsigned km = __ballot_sync(0xffffffffu, keep);
-        if (keep) inf->tiles[w + __popc(km & lt)] = tile;
-        w += __popc(km);
+        stop = min(e, count);
+        for (int base = a; base < stop; base += 32) {
+          const int t = base + lane;
+          const int v = (t < stop) ? src[t] : 0;
+          bool bad = (t < stop) && (gist ? (v >= nb_cache || v < -ngist) : (v < 0 || v >= nb_cache));
+          int tile = v;
+          if (p.table != nullptr && t < stop && !bad) {
+            // paged cache: the kept logical block's physical block
+            tile = __ldg(p.table + static_cast<int64_t>(bg / p.Hkv) * p.table_stride + v);
+            bad = tile < 0 || tile >= p.num_pages;
+          }
+          if (bad) atomicOr(p.status, BSA_DEV_BAD_INDEX);
+          const bool keep = (t < stop) && !bad && (w + (t - base) < kMaxItemTiles);
+          const unsigned km = __ballot_sync(0xffffffffu, keep);
+          if (keep) inf->tiles[w + __popc(km & lt)] = tile;
+          w += __popc(km);
+        }
       }
       if (lane == 0) {
         if (stop - a > kMaxItemTiles) atomicOr(p.status, BSA_DEV_BAD_SHAPE);
@@ -889,6 +950,11 @@ cudaError_t launch_attn_decode_bf16(const CUtensorMap* tmQ, const CUtensorMap* t
   p.num_pages = a.num_pages;
   p.gist_allow = a.gist_allow;
   p.meta_rows = (tmMK != nullptr) ? a.meta_rows : 0;
+  p.heads_idx = a.heads_idx;
+  p.heads_topk = a.heads_topk;
+  p.heads_stride = a.heads_stride;
+  if (p.heads_idx != nullptr && (p.nc > 32 * decode::kUnionWords || p.G > decode::kNH || p.gist_allow != nullptr))
+    return cudaErrorInvalidValue;
   const int grid = a.num_ctas;
   return launch_dependent(decode::attn_decode_kernel, dim3(grid), dim3(decode::kThreads), decode::kSmemBytes, st, *tmQ,
                           *tmK, *tmV, tmGK ? *tmGK : *tmK, tmGV ? *tmGV : *tmV, tmMK ? *tmMK : *tmK,

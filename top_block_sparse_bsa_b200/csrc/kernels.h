@@ -158,6 +158,10 @@ struct DecodeArgs {
   // two-level gists: per-head allowed gist / meta-gist rows; meta rows per (b, g)
   const uint32_t* gist_allow = nullptr;
   int meta_rows = 0;
+  // gist decode with the union built inside the attention kernel (nc <= 2048,
+  // G <= 16): the heads' kept chunk lists replace list / expanded
+  const int* heads_idx = nullptr;
+  int heads_topk = 0, heads_stride = 0;
 };
 cudaError_t launch_attn_decode_bf16(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
                                     const CUtensorMap* tmGK, const CUtensorMap* tmGV, const DecodeArgs& a,
