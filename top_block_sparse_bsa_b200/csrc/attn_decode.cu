@@ -427,16 +427,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         const int* hsrc = p.heads_idx + (static_cast<int64_t>(bg / p.Hkv) * p.Hq + (bg % p.Hkv) * G) *
                                             static_cast<int64_t>(p.heads_stride);
-        for (int t = lane; t < G * topk; t += 32) {
-          const int hh = t / topk;
-          const int c = __ldg(hsrc + static_cast<int64_t>(hh) * p.heads_stride + (t - hh * topk));
-          if (c < 0) continue;
-          if (c >= p.nc) {
-            atomicOr(p.status, BSA_DEV_BAD_INDEX);
-            continue;
+        // the entries in rounds of 8 per lane, each round's loads issued together
+        for (int t0 = 0; t0 < G * topk; t0 += 32 * 8) {
+          int cv[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int t = t0 + 32 * u + lane;
+            const int hh = t / topk;
+            cv[u] = (t < G * topk) ? __ldg(hsrc + static_cast<int64_t>(hh) * p.heads_stride + (t - hh * topk)) : -1;
           }
-          atomicOr(&ub[hh * kUnionWords + (c >> 5)], 1u << (c & 31));
-          atomicOr(&ub[G * kUnionWords + (c >> 5)], 1u << (c & 31));
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int c = cv[u];
+            if (c < 0) continue;
+            if (c >= p.nc) {
+              atomicOr(p.status, BSA_DEV_BAD_INDEX);
+              continue;
+            }
+            const int hh = (t0 + 32 * u + lane) / topk;
+            atomicOr(&ub[hh * kUnionWords + (c >> 5)], 1u << (c & 31));
+            atomicOr(&ub[G * kUnionWords + (c >> 5)], 1u << (c & 31));
+          }
         }
         __syncwarp();
         const uint32_t w0 = (2 * lane < words) ? ub[G * kUnionWords + 2 * lane] : 0u;
