@@ -703,8 +703,8 @@ def measure_decode_like(w, dev, steps: int, warmup: int, peaks, peak_src, dist=N
         step = pipeline.GistStep(inp["q"], inp["k"], inp["v"], inp["gk"], inp["gv"], w.bs, w.kb)
         select = lambda: step.run(with_lse=False)   # noqa: E731  (the whole step in one call)
         attend = lambda: step.run(idx_in=step.bufs["idx"], with_lse=False)   # noqa: E731
-        launches = 5   # gist score, top-k, union lists, split-K attention, combine
-        attn_kernel = "gist_union_kernel + attn_decode_kernel + combine_kernel"
+        launches = 4   # gist score, top-k, split-K attention (union built inside), combine
+        attn_kernel = "attn_decode_kernel (the group's union built in the kernel) + combine_kernel"
     # L2 flush between steps: a 256 MiB write evicts every input line, and a
     # 256 MiB read of a second buffer then evicts the write's dirty lines, so
     # the timed step neither finds its inputs in L2 nor pays for writing back

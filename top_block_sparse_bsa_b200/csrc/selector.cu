@@ -116,20 +116,26 @@ static cudaError_t launch_pool_jobs(const PoolJob& j0, const PoolJob& j1, bool b
   return cudaGetLastError();
 }
 
-// Streamed variant (persistent, one CTA per SM): a producer thread copies each
-// unit's rows (heads_sum runs of bs*d contiguous elements) into
-// kPoolStages shared-memory buffers with bulk copies, a chunk of whole runs
-// per buffer, while 128 threads sum earlier chunks, column c by thread c,
-// rows in the fixed order (head, then row), the running sum carried from one
-// chunk of a unit to the next.  Units of the query job come first, then those
-// of the key job; a key unit is a single run and consecutive key units are
-// contiguous in memory, so a buffer takes several of them in one copy.
-constexpr int kPoolStreamBytes = 64 * 1024;
+// Streamed variant (persistent): a producer thread copies each unit's rows
+// (heads_sum runs of bs*d contiguous elements) into kPoolStages shared-memory
+// buffers with bulk copies, a chunk of whole runs per buffer, while 128
+// threads sum earlier chunks, column c by thread c, rows in the fixed order
+// (head, then row), the running sum carried from one chunk of a unit to the
+// next.  Units of the query job come first, then those of the key job; a key
+// unit is a single run and consecutive key units are contiguous in memory, so
+// a buffer takes several of them in one copy, and their column sums (separate
+// chains) advance together.  A column's sum over a unit is one dependent chain
+// of additions, so the kernel runs two CTAs per SM with 32 KB chunks when a
+// run fits (two summing warps per SM sub-partition), one with 64 KB chunks
+// otherwise.
+constexpr int kPoolStreamBytes = 64 * 1024;   // largest chunk
+constexpr int kPoolSmallChunk = 32 * 1024;
 constexpr int kPoolStages = 3;
+constexpr int kPoolMaxGroup = 4;              // key units per chunk: 64 KB / 16 KB runs
 
 template <typename T>
-__global__ void __launch_bounds__(160, 1) pool_stream_kernel(PoolJob jq, PoolJob jk, int B, int Hgroups, int N, int d,
-                                                             int bs, uint32_t* status) {
+__global__ void __launch_bounds__(160, 2) pool_stream_kernel(PoolJob jq, PoolJob jk, int B, int Hgroups, int N, int d,
+                                                             int bs, int chunk_bytes, uint32_t* status) {
   extern __shared__ uint8_t psmem_raw[];
   uint8_t* psmem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(psmem_raw) + 127) & ~uintptr_t(127));
   __shared__ __align__(8) uint64_t bars[2 * kPoolStages];
@@ -139,7 +145,7 @@ __global__ void __launch_bounds__(160, 1) pool_stream_kernel(PoolJob jq, PoolJob
   const int nb = N / bs;
   const int64_t units_per_job = static_cast<int64_t>(B) * Hgroups * nb;
   const uint32_t run = static_cast<uint32_t>(bs) * d * sizeof(T);       // one head's rows of a unit
-  const int runs_per_chunk = static_cast<int>(kPoolStreamBytes / run);   // >= 1 (checked by the launcher)
+  const int runs_per_chunk = static_cast<int>(chunk_bytes / run);   // 1 .. kPoolMaxGroup (checked by the launcher)
   // key items: kgrp consecutive key units each (single-run units stored back
   // to back: unit u's rows start at u * bs * d)
   const int kgrp = (jk.src != nullptr && jk.heads_sum == 1 && jk.Hsrc == Hgroups) ? runs_per_chunk : 1;
@@ -168,7 +174,7 @@ __global__ void __launch_bounds__(160, 1) pool_stream_kernel(PoolJob jq, PoolJob
           const int buf = k % kPoolStages, use = k / kPoolStages;
           if (k >= kPoolStages && !(ok = mbar_wait(bar(kPoolStages + buf), (use - 1) & 1, ab, status))) break;
           mbar_arrive_expect_tx(bar(buf), run * nr);
-          bulk_load(sb + buf * kPoolStreamBytes, static_cast<const T*>(jk.src) + u0 * bs * d, run * nr, bar(buf));
+          bulk_load(sb + buf * chunk_bytes, static_cast<const T*>(jk.src) + u0 * bs * d, run * nr, bar(buf));
           ++k;
           continue;
         }
@@ -184,7 +190,7 @@ __global__ void __launch_bounds__(160, 1) pool_stream_kernel(PoolJob jq, PoolJob
           if (k >= kPoolStages && !(ok = mbar_wait(bar(kPoolStages + buf), (use - 1) & 1, ab, status))) break;
           mbar_arrive_expect_tx(bar(buf), run * nr);
           for (int hh = h0; hh < h0 + nr; ++hh)
-            bulk_load(sb + buf * kPoolStreamBytes + (hh - h0) * run,
+            bulk_load(sb + buf * chunk_bytes + (hh - h0) * run,
                       src + ((b * job.Hsrc + g * job.heads_sum + hh) * static_cast<int64_t>(N) + j * bs) * d, run,
                       bar(buf));
         }
@@ -205,19 +211,26 @@ __global__ void __launch_bounds__(160, 1) pool_stream_kernel(PoolJob jq, PoolJob
         const int nr = static_cast<int>(min(static_cast<int64_t>(kgrp), units_per_job - u0));
         const int buf = k % kPoolStages, use = k / kPoolStages;
         if (!(ok = mbar_wait(bar(buf), use & 1, ab, status))) break;
-        const T* sv = reinterpret_cast<const T*>(psmem + buf * kPoolStreamBytes);
-        for (int x = 0; x < nr; ++x) {
-          float acc = 0.0f;
-          if (c < d) {
-            for (int r = x * bs; r < (x + 1) * bs; r += 16) {   // bs is a multiple of 16
-              float xv[16];
+        const T* sv = reinterpret_cast<const T*>(psmem + buf * chunk_bytes);
+        if (c < d) {
+          // the nr units' column sums advance together (independent chains),
+          // each over its own rows in ascending order
+          float acc[kPoolMaxGroup] = {0.0f, 0.0f, 0.0f, 0.0f};
+          for (int r = 0; r < bs; r += 16) {   // bs is a multiple of 16
 #pragma unroll
-              for (int t = 0; t < 16; ++t) xv[t] = static_cast<float>(sv[(r + t) * d + c]);
+            for (int x = 0; x < kPoolMaxGroup; ++x) {
+              if (x < nr) {
+                float xv[16];
 #pragma unroll
-              for (int t = 0; t < 16; ++t) acc = __fadd_rn(acc, xv[t]);
+                for (int t = 0; t < 16; ++t) xv[t] = static_cast<float>(sv[(x * bs + r + t) * d + c]);
+#pragma unroll
+                for (int t = 0; t < 16; ++t) acc[x] = __fadd_rn(acc[x], xv[t]);
+              }
             }
-            jk.out[(u0 + x) * d + c] = __fdiv_rn(acc, static_cast<float>(bs));
           }
+#pragma unroll
+          for (int x = 0; x < kPoolMaxGroup; ++x)
+            if (x < nr) jk.out[(u0 + x) * d + c] = __fdiv_rn(acc[x], static_cast<float>(bs));
         }
         mbar_arrive(bar(kPoolStages + buf));
         ++k;
@@ -230,7 +243,7 @@ __global__ void __launch_bounds__(160, 1) pool_stream_kernel(PoolJob jq, PoolJob
         const int nr = min(runs_per_chunk, job.heads_sum - h0);
         const int buf = k % kPoolStages, use = k / kPoolStages;
         if (!(ok = mbar_wait(bar(buf), use & 1, ab, status))) break;
-        const T* sv = reinterpret_cast<const T*>(psmem + buf * kPoolStreamBytes);
+        const T* sv = reinterpret_cast<const T*>(psmem + buf * chunk_bytes);
         const int rows = nr * bs;   // a multiple of 16
         if (c < d) {
           for (int r = 0; r < rows; r += 16) {
@@ -268,18 +281,25 @@ cudaError_t launch_pool_prefill(const void* q, const void* k, bool bf16, int B, 
   const size_t run_bytes = static_cast<size_t>(bs) * d * esize;
   if (run_bytes > kPoolStreamBytes || d > 128 || bs % 16 != 0 || run_bytes % 16 != 0)
     return launch_pool_jobs(jq, jk, bf16, B, Hkv, N, d, bs, st);
-  const size_t smem = kPoolStages * kPoolStreamBytes + 128;
+  // two CTAs per SM with 32 KB chunks when a run fits, else one with 64 KB
+  // (a chunk holds at most kPoolMaxGroup runs either way: runs are >= 16 KB
+  // for bs*d >= 8192 bf16 values; smaller runs keep one CTA per SM)
+  const bool small = run_bytes <= kPoolSmallChunk && kPoolSmallChunk / run_bytes <= kPoolMaxGroup;
+  const int chunk = small ? kPoolSmallChunk : kPoolStreamBytes;
+  if (static_cast<size_t>(chunk) / run_bytes > kPoolMaxGroup) return launch_pool_jobs(jq, jk, bf16, B, Hkv, N, d, bs, st);
+  const size_t smem = static_cast<size_t>(kPoolStages) * chunk + 128;
   const int64_t units = 2ll * B * Hkv * (N / bs);
-  const unsigned grid = static_cast<unsigned>(units < num_sms ? units : num_sms);
+  const int64_t ctas = static_cast<int64_t>(num_sms) * (small ? 2 : 1);
+  const unsigned grid = static_cast<unsigned>(units < ctas ? units : ctas);
   cudaError_t e;
   if (bf16) {
     e = ensure_dynamic_smem<pool_stream_kernel<__nv_bfloat16>>(smem);
     if (e != cudaSuccess) return e;
-    pool_stream_kernel<__nv_bfloat16><<<grid, 160, smem, st>>>(jq, jk, B, Hkv, N, d, bs, status);
+    pool_stream_kernel<__nv_bfloat16><<<grid, 160, smem, st>>>(jq, jk, B, Hkv, N, d, bs, chunk, status);
   } else {
     e = ensure_dynamic_smem<pool_stream_kernel<float>>(smem);
     if (e != cudaSuccess) return e;
-    pool_stream_kernel<float><<<grid, 160, smem, st>>>(jq, jk, B, Hkv, N, d, bs, status);
+    pool_stream_kernel<float><<<grid, 160, smem, st>>>(jq, jk, B, Hkv, N, d, bs, chunk, status);
   }
   return cudaGetLastError();
 }
