@@ -697,7 +697,7 @@ def measure_decode_like(w, dev, steps: int, warmup: int, peaks, peak_src, dist=N
                                  W.HSSA_GROUPS_KEPT, w.kb)
         select = lambda: step.run(with_lse=False)   # noqa: E731  (the whole step in one call)
         attend = None
-        launches = 7   # meta scores, top-km, group gist scores, top-k, union, attention, combine
+        launches = 6   # meta scores, top-km, group gist scores + top-k, union, attention, combine
         attn_kernel = "whole two-level gist step (one call)"
     else:
         step = pipeline.GistStep(inp["q"], inp["k"], inp["v"], inp["gk"], inp["gv"], w.bs, w.kb)

@@ -315,6 +315,15 @@ def test_hssa_small(hq, hkv, km, topk):
     _hssa_case(w, km, topk)
 
 
+@pytest.mark.parametrize("km,ngroups,topk", [(6, 8, 40), (12, 16, 100), (20, 24, 33)])
+def test_hssa_many_kept_groups(km, ngroups, topk):
+    """More kept groups per head (6, 12, 20 of 8, 16, 24 groups of 64 chunks):
+    the fine top-k then runs over 384, 768 or 1280 positions (two, four or
+    eight keys per thread in the select that shares the scoring launch)."""
+    w = W.get("hssa_decode_bf16").scaled(B=1, Hq=4, Hkv=1, N=ngroups * 64 * 64, kb=topk)
+    _hssa_case(w, km, topk)
+
+
 def test_hssa_full_size():
     """The gist workload's shape with meta-gists: 8 sequences x 131072 tokens,
     2048 chunks in 32 groups, 4 groups kept and 32 chunks expanded per head;

@@ -840,8 +840,12 @@ bsa_status_t bsa_hssa_decode(const bsa_shape_t* s, const void* q, const void* k_
                                     sms, cs);
   if (e == cudaSuccess) e = launch_topk(meta_scores, rows, nm, BSA_TOPK_PLAIN, km, meta_idx, km, nullptr, cs);
   // fine: the gists of the kept groups' chunks and the topk best per head
-  if (e == cudaSuccess) e = launch_score_gist_groups(&mgk, q, meta_idx, km, s->B, s->Hq, s->Hkv, nc, scale, fine, status, cs);
+  // (with up to 32 kept groups the row's top-k runs in the scoring launch)
+  const bool fuse_fine = gist_groups_select_fused_ok(km);
   if (e == cudaSuccess)
+    e = launch_score_gist_groups(&mgk, q, meta_idx, km, s->B, s->Hq, s->Hkv, nc, scale, fine, topk,
+                                 fuse_fine ? pos : nullptr, L.k_stride, status, cs);
+  if (e == cudaSuccess && !fuse_fine)
     e = launch_topk(fine, rows, km * 64, BSA_TOPK_PLAIN, topk, pos, L.k_stride, nullptr, cs);
   if (e == cudaSuccess)
     e = launch_hssa_union(meta_idx, km, pos, L.k_stride, s->B, s->Hq, s->Hkv, nc, nm, chunks, expanded, allow, ulist,

@@ -86,9 +86,12 @@ cudaError_t launch_score_heads(const void* q, bool bf16, const float* kbar, int 
                                float scale, float* s, cudaStream_t st);
 cudaError_t launch_topk_joint(const float* scores, int rows, int G, int nb, int kb_total, int* idx_out,
                               int idx_stride, int* count_out, cudaStream_t st);
+// pos_out non-null: the row's top-k positions (topk of km*64, pos_stride apart) are
+// selected in the same launch and the fine scores are not written (km*64 <= 2048)
+bool gist_groups_select_fused_ok(int km);
 cudaError_t launch_score_gist_groups(const CUtensorMap* tmG, const void* q, const int* meta_idx, int km, int B,
-                                     int Hq, int Hkv, int nc, float scale, float* fine, uint32_t* status,
-                                     cudaStream_t st);
+                                     int Hq, int Hkv, int nc, float scale, float* fine, int topk, int* pos_out,
+                                     int pos_stride, uint32_t* status, cudaStream_t st);
 // decode scores + top-k in one kernel (tmKbar: fp32 [rows, 128], box 32 x 128, 128-byte swizzle)
 bool decode_select_fused_ok(int d, int nb);
 cudaError_t launch_decode_select(const CUtensorMap* tmKbar, const void* q, bool bf16, int B, int Hq, int Hkv,

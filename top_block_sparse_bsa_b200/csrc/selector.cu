@@ -1263,18 +1263,39 @@ cudaError_t launch_topk_joint(const float* scores, int rows, int G, int nb, int 
 // A group slot past the kept ones gets NaN (never ranked above a number).
 constexpr int kGroupStages = 4;
 
+// The row's top-k over its km*64 fine scores held in shared memory (plain
+// rule: every position a candidate, none forced; NaN scores of missing groups
+// rank lowest), written as positions ascending.
+constexpr int kGroupFuseMax = 256 * 8;   // positions the fused select holds (8 keys per thread)
+
+template <int KPT>
+__device__ __forceinline__ void group_row_select(const float* fsc, int ncand, int k, int* out, int stride) {
+  uint32_t key[KPT];
+#pragma unroll
+  for (int e = 0; e < KPT; ++e) {
+    const int j = static_cast<int>(threadIdx.x) * KPT + e;
+    key[e] = (j < ncand) ? order_key(fsc[j]) : 0u;
+  }
+  cta_topk_select<KPT>(key, ncand, k, -1, out, stride, nullptr);
+}
+
+// pos_out != null: the row's fine scores stay in shared memory and the
+// kernel also runs the row's top-k (the separate top-k launch is skipped).
 __global__ void __launch_bounds__(256) score_gist_groups_kernel(const __grid_constant__ CUtensorMap tmG,
                                                                 const __nv_bfloat16* __restrict__ q,
                                                                 const int* __restrict__ meta_idx, int km, int Hq,
                                                                 int Hkv, int nc, float scale,
-                                                                float* __restrict__ fine,
+                                                                float* __restrict__ fine, int topk,
+                                                                int* __restrict__ pos_out, int pos_stride,
                                                                 uint32_t* __restrict__ status) {
   constexpr int D = 128;
   extern __shared__ uint8_t sm_raw[];
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
   __shared__ __align__(8) uint64_t full[kGroupStages];
   __shared__ float qs[D];
+  __shared__ float fsc[kGroupFuseMax];
   __shared__ int abort_flag;
+  const bool fused = pos_out != nullptr;
   const int64_t row = blockIdx.x;   // b * Hq + h
   const int64_t b = row / Hq;
   const int g = static_cast<int>(row % Hq) / (Hq / Hkv);
@@ -1320,7 +1341,8 @@ __global__ void __launch_bounds__(256) score_gist_groups_kernel(const __grid_con
       const bool got = mbar_wait(smem_u32(&full[t % kGroupStages]), (t / kGroupStages) & 1, &abort_flag, status);
       ok = ok && got;
       if (!valid) {
-        out[t * 64 + r] = __int_as_float(0x7fc00000);   // NaN
+        if (fused) fsc[t * 64 + r] = __int_as_float(0x7fc00000);   // NaN
+        else out[t * 64 + r] = __int_as_float(0x7fc00000);
       } else if (got) {
         const uint8_t* tb = tiles + (t % kGroupStages) * (64 * D * 2) + r * 128;
         float acc = 0.0f;
@@ -1335,7 +1357,8 @@ __global__ void __launch_bounds__(256) score_gist_groups_kernel(const __grid_con
             acc = __fadd_rn(acc, __fmul_rn(qs[8 * x + 2 * y + 1], __uint_as_float(ws[y] & 0xFFFF0000u)));
           }
         }
-        out[t * 64 + r] = __fmul_rn(acc, scale);
+        if (fused) fsc[t * 64 + r] = __fmul_rn(acc, scale);
+        else out[t * 64 + r] = __fmul_rn(acc, scale);
       }
     }
     __syncthreads();   // this round's stages are free again
@@ -1348,16 +1371,31 @@ __global__ void __launch_bounds__(256) score_gist_groups_kernel(const __grid_con
     for (int t = max(0, issued - kGroupStages); t < issued; ++t)
       mbar_drain(smem_u32(&full[t % kGroupStages]), (t / kGroupStages) & 1);
   }
+  if (!fused || __syncthreads_or(abort_flag)) return;
+  const int ncand = km * 64;
+  int* prow = pos_out + row * pos_stride;
+  if (ncand <= 256)
+    group_row_select<1>(fsc, ncand, topk, prow, pos_stride);
+  else if (ncand <= 512)
+    group_row_select<2>(fsc, ncand, topk, prow, pos_stride);
+  else if (ncand <= 1024)
+    group_row_select<4>(fsc, ncand, topk, prow, pos_stride);
+  else
+    group_row_select<8>(fsc, ncand, topk, prow, pos_stride);
 }
 
+bool gist_groups_select_fused_ok(int km) { return km >= 1 && km * 64 <= kGroupFuseMax; }
+
 cudaError_t launch_score_gist_groups(const CUtensorMap* tmG, const void* q, const int* meta_idx, int km, int B,
-                                     int Hq, int Hkv, int nc, float scale, float* fine, uint32_t* status,
-                                     cudaStream_t st) {
+                                     int Hq, int Hkv, int nc, float scale, float* fine, int topk, int* pos_out,
+                                     int pos_stride, uint32_t* status, cudaStream_t st) {
+  if (pos_out != nullptr && !gist_groups_select_fused_ok(km)) return cudaErrorInvalidValue;
   const size_t smem = static_cast<size_t>(kGroupStages) * 64 * 128 * 2 + 1024;   // + alignment slack
   cudaError_t e = ensure_dynamic_smem<score_gist_groups_kernel>(smem);
   if (e != cudaSuccess) return e;
   return launch_dependent(score_gist_groups_kernel, dim3(B * Hq), dim3(256), smem, st, *tmG,
-                          static_cast<const __nv_bfloat16*>(q), meta_idx, km, Hq, Hkv, nc, scale, fine, status);
+                          static_cast<const __nv_bfloat16*>(q), meta_idx, km, Hq, Hkv, nc, scale, fine, topk, pos_out,
+                          pos_stride, status);
 }
 
 cudaError_t launch_topk(const float* scores, int rows, int ncols, int mode, int kb, int* idx_out,
