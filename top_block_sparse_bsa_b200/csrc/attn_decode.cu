@@ -26,11 +26,7 @@
 // owner + MMA issuer, warp 6 slice loader.  Tensor memory: two S^T buffers
 // (16 columns each) and O^T (16 columns).  The four softmax warps exchange
 // per-head maxima through shared memory with mbarrier hand-offs (bounded
-// waits, never bar.sync, so an abort cannot strand a warp).  In gist mode
-// with up to 2048 chunks the slice loader builds the group's union itself
-// from the heads' kept lists (per-head and union bitmaps in the item slot in
-// shared memory, list positions by a warp scan of the union's bit counts);
-// above that a separate kernel builds it in global memory.
+// waits, never bar.sync, so an abort cannot strand a warp).
 #include "common.cuh"
 #include "kernels.h"
 
