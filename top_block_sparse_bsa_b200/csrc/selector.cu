@@ -281,9 +281,9 @@ cudaError_t launch_pool_prefill(const void* q, const void* k, bool bf16, int B, 
   const size_t run_bytes = static_cast<size_t>(bs) * d * esize;
   if (run_bytes > kPoolStreamBytes || d > 128 || bs % 16 != 0 || run_bytes % 16 != 0)
     return launch_pool_jobs(jq, jk, bf16, B, Hkv, N, d, bs, st);
-  // two CTAs per SM with 32 KB chunks when a run fits, else one with 64 KB
-  // (a chunk holds at most kPoolMaxGroup runs either way: runs are >= 16 KB
-  // for bs*d >= 8192 bf16 values; smaller runs keep one CTA per SM)
+  // a chunk holds 1 .. kPoolMaxGroup runs: runs of 8 KB to 32 KB take two
+  // CTAs per SM with 32 KB chunks, runs above 32 KB one CTA per SM with 64 KB
+  // chunks, and runs below 8 KB go to pool_kernel
   const bool small = run_bytes <= kPoolSmallChunk && kPoolSmallChunk / run_bytes <= kPoolMaxGroup;
   const int chunk = small ? kPoolSmallChunk : kPoolStreamBytes;
   if (static_cast<size_t>(chunk) / run_bytes > kPoolMaxGroup) return launch_pool_jobs(jq, jk, bf16, B, Hkv, N, d, bs, st);
